@@ -1,0 +1,503 @@
+"""CPU oracle for the ZeRO optimizer step over N logical data-parallel ranks.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()``
+and ``bench.py``'s CPU-baseline / reference leg may import this package.  The
+product library never calls it, and it imports nothing from the product: it
+shares no code, header, table or helper with the CUDA path.  The only thing
+both sides share is the seeded input generator in ``synth``.
+
+What it computes, and where each piece comes from (three web pages on ZeRO):
+  [T]  "ZERO训练技术" (wqh011128.github.io)
+  [M]  "ZeRO：从优化器状态到残差状态的显存优化" (xuesongtap.github.io)
+  [Q]  mstx.cn post 475, a ZeRO interview write-up
+
+* ``plan``            -- the N-way contiguous ownership partition ([T] section
+                         "ZeRO-1", part "optimizer state 怎么切分") and the
+                         fixed-size bucket schedule ([M] section 3.3 "CB").
+* ``all_reduce`` / ``reduce_scatter`` / ``all_gather`` -- the three
+                         collectives as literal copies between per-rank arrays
+                         ([T] sections "ZeRO-1" and "ZeRO-2"; [Q] sections 三, 四).
+* ``run``             -- plain DP and the ZeRO-1/2/3 step flows ([T] sections
+                         "先立一个基线", "ZeRO-1", "ZeRO-2", "ZeRO-3").
+* ``state_bytes`` / ``mem_model`` -- per-rank model-state bytes ([Q] section
+                         六 table; [M] section 5 worked example).
+* ``comm_elems``      -- logical communication volume per rank ([M] section 2;
+                         [Q] sections 三.3, 五.4).
+
+The per-element arithmetic (bf16 rounding, the rank-order reduction, Adam)
+lives in ``zero_oracle.c``; its readings of the pages are stated there.
+
+Pinned by ``tests/test_oracle_*.py``: exhaustive bf16 rounding against
+torch's CPU conversion, reduction against exact sums and error bounds, Adam
+against ``torch.optim.AdamW``, stage equivalence with plain DP, bucket
+invariance, brute force on tiny sizes, and the pages' closed forms and worked
+numbers.  ``grad_norm`` has no exact external pin beyond an fp64 error bound
+against ``math.fsum`` and is compared to the CUDA path within a tolerance.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass, field
+from typing import Callable, List, Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+STAGE_DP, STAGE_Z1, STAGE_Z2, STAGE_Z3 = 0, 1, 2, 3
+GRANULE = 8  # every tensor starts on an 8-element boundary (a stated layout choice)
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = os.path.join(_HERE, "libzero_oracle.so")
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: run __graft_entry__.build() first")
+        lib = ctypes.CDLL(path)
+        vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+        lib.zo_bf16_rne.restype = ctypes.c_uint16
+        lib.zo_bf16_rne.argtypes = [f32]
+        lib.zo_bf16_to_f32.restype = f32
+        lib.zo_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.zo_bf16_rne_array.restype = None
+        lib.zo_bf16_rne_array.argtypes = [i64, vp, vp]
+        lib.zo_bf16_to_f32_array.restype = None
+        lib.zo_bf16_to_f32_array.argtypes = [i64, vp, vp]
+        lib.zo_reduce_mean.restype = None
+        lib.zo_reduce_mean.argtypes = [i32, i64, vp, vp]
+        lib.zo_rank_sum_f32.restype = None
+        lib.zo_rank_sum_f32.argtypes = [i32, i64, vp, vp]
+        lib.zo_adam_scalars.restype = None
+        f64 = ctypes.c_double
+        lib.zo_adam_scalars.argtypes = [f64, f64, f64, f64, f64, i64, vp]
+        lib.zo_adam.restype = None
+        lib.zo_adam.argtypes = [i64, vp, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
+        lib.zo_sumsq.restype = ctypes.c_double
+        lib.zo_sumsq.argtypes = [i64, vp]
+        lib.zo_count_nonfinite.restype = i64
+        lib.zo_count_nonfinite.argtypes = [i64, vp]
+        _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------ elementwise ----
+
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns (uint16), round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    if x.size:
+        _load().zo_bf16_rne_array(x.size, x.ctypes.data, out.ctypes.data)
+    return out
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float32)
+    if h.size:
+        _load().zo_bf16_to_f32_array(h.size, h.ctypes.data, out.ctypes.data)
+    return out
+
+
+def _ptr_array(arrays: Sequence[np.ndarray]):
+    ptrs = (ctypes.c_void_p * len(arrays))()
+    for r, a in enumerate(arrays):
+        ptrs[r] = a.ctypes.data
+    return ptrs
+
+
+def reduce_mean(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
+    """Averaged bf16 gradient of N equal-length rank slices (uint16 arrays)."""
+    rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
+    n = rank_slices[0].size
+    assert all(a.size == n for a in rank_slices)
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().zo_reduce_mean(len(rank_slices), n, _ptr_array(rank_slices), out.ctypes.data)
+    return out
+
+
+def rank_sum_f32(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
+    rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
+    n = rank_slices[0].size
+    out = np.empty(n, dtype=np.float32)
+    if n:
+        _load().zo_rank_sum_f32(len(rank_slices), n, _ptr_array(rank_slices), out.ctypes.data)
+    return out
+
+
+@dataclass(frozen=True)
+class AdamHP:
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.0
+
+
+def adam_scalars(hp: AdamHP, t: int) -> np.ndarray:
+    """float32[9]: beta1, beta2, 1-beta1, 1-beta2, bc1, bc2, decay, lr, eps."""
+    out = np.empty(9, dtype=np.float32)
+    _load().zo_adam_scalars(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t,
+                            out.ctypes.data)
+    return out
+
+
+def adam(g: np.ndarray, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: AdamHP,
+         t: int) -> np.ndarray:
+    """In-place Adam on fp32 master/m/v from the bf16 grad g; returns the bf16 params."""
+    assert master.dtype == np.float32 and m.dtype == np.float32 and v.dtype == np.float32
+    assert master.flags.c_contiguous and m.flags.c_contiguous and v.flags.c_contiguous
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    n = g.size
+    assert master.size == n and m.size == n and v.size == n
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().zo_adam(n, g.ctypes.data, master.ctypes.data, m.ctypes.data, v.ctypes.data,
+                        out.ctypes.data, hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t)
+    return out
+
+
+def sumsq(g: np.ndarray) -> float:
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    return float(_load().zo_sumsq(g.size, g.ctypes.data)) if g.size else 0.0
+
+
+def count_nonfinite(g: np.ndarray) -> int:
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    return int(_load().zo_count_nonfinite(g.size, g.ctypes.data)) if g.size else 0
+
+
+# ------------------------------------------------------------------- plan ----
+
+def _roundup(x: int, m: int) -> int:
+    return (x + m - 1) // m * m
+
+
+@dataclass
+class Plan:
+    """Flat layout of a parameter list cut into N owned segments.
+
+    Reading of "cut the parameter vector into N parts" ([T] section "ZeRO-1",
+    part "optimizer state 怎么切分"): tensors are laid end to end in list
+    order, each starting on an 8-element boundary; the flat length is padded
+    up to a multiple of 8N so the N segments are equal and contiguous; rank r
+    owns [r*S, (r+1)*S).  Pad elements hold 0 everywhere.
+    """
+
+    numel: List[int]
+    layer_id: List[int]
+    n_ranks: int
+    bucket_elems: int
+    offset: List[int] = field(default_factory=list)   # start of each tensor
+    slot_end: List[int] = field(default_factory=list)  # end of each tensor's padded slot
+    psi: int = 0          # real parameter count
+    psi_pad: int = 0      # padded flat length
+    shard: int = 0        # S = psi_pad / N
+    layers: List[tuple] = field(default_factory=list)   # (layer id, lo, hi), list order
+    buckets: List[tuple] = field(default_factory=list)  # (lo, hi), in schedule order
+
+    def owner(self, i: int) -> int:
+        return i // self.shard
+
+    def owned(self, r: int) -> tuple:
+        return (r * self.shard, (r + 1) * self.shard)
+
+    def real_mask(self) -> np.ndarray:
+        mask = np.zeros(self.psi_pad, dtype=bool)
+        for off, n in zip(self.offset, self.numel):
+            mask[off:off + n] = True
+        return mask
+
+
+def plan(numel: Sequence[int], layer_id: Sequence[int], n_ranks: int, bucket_elems: int) -> Plan:
+    assert n_ranks >= 1 and bucket_elems > 0 and bucket_elems % GRANULE == 0
+    assert len(numel) == len(layer_id) and len(numel) >= 1
+    assert all(n >= 0 for n in numel)
+    assert all(a <= b for a, b in zip(layer_id, layer_id[1:]))
+    p = Plan(list(numel), list(layer_id), n_ranks, bucket_elems)
+    cursor = 0
+    for n in numel:
+        p.offset.append(cursor)
+        cursor = _roundup(cursor + n, GRANULE)
+    flat = cursor
+    p.psi = int(sum(numel))
+    p.psi_pad = _roundup(max(flat, 1), GRANULE * n_ranks)
+    p.shard = p.psi_pad // n_ranks
+    # each tensor's padded slot runs to the next tensor's start; the last one
+    # also takes the tail padding up to psi_pad
+    p.slot_end = p.offset[1:] + [p.psi_pad]
+    # layers: maximal runs of equal layer id (contiguous in the flat space)
+    k = 0
+    while k < len(numel):
+        j = k
+        while j + 1 < len(numel) and layer_id[j + 1] == layer_id[k]:
+            j += 1
+        p.layers.append((layer_id[k], p.offset[k], p.slot_end[j]))
+        k = j + 1
+    p.buckets = bucket_schedule(p)
+    return p
+
+
+def bucket_schedule(p: Plan) -> List[tuple]:
+    """Fixed-size buffer schedule ([M] section 3.3 "CB"; [T] section "ZeRO-2",
+    part "2. 反向"): gradients become ready layer by layer from the last layer
+    back, so tensors are walked in reverse list order and packed into the
+    current interval while it stays within ``bucket_elems``; when the next
+    tensor does not fit, the interval is flushed.  A tensor slot larger than
+    the buffer is cut into buffer-sized chunks from its end, each its own
+    interval (the last, lowest chunk may be shorter).
+    """
+    out: List[tuple] = []
+    cur: Optional[list] = None  # [lo, hi]
+    B = p.bucket_elems
+    for k in reversed(range(len(p.numel))):
+        a, b = p.offset[k], p.slot_end[k]
+        size = b - a
+        if size == 0:
+            continue
+        if size > B:
+            if cur is not None:
+                out.append(tuple(cur))
+                cur = None
+            e = b
+            while e - a > B:
+                out.append((e - B, e))
+                e -= B
+            out.append((a, e))
+        elif cur is not None and (cur[1] - cur[0]) + size <= B:
+            cur[0] = a
+        else:
+            if cur is not None:
+                out.append(tuple(cur))
+            cur = [a, b]
+    if cur is not None:
+        out.append(tuple(cur))
+    return out
+
+
+# ------------------------------------------------------------ collectives ----
+
+def all_reduce(rank_grads: Sequence[np.ndarray], lo: int, hi: int) -> None:
+    """All-reduce of [lo, hi) in place ([T] section "ZeRO-1", part "2. 反向"):
+    every rank's replica receives the same averaged gradient."""
+    g = reduce_mean([a[lo:hi] for a in rank_grads])
+    for a in rank_grads:
+        a[lo:hi] = g
+
+
+def reduce_scatter(rank_grads: Sequence[np.ndarray], plan_: Plan, lo: int, hi: int,
+                   grad_shards: List[np.ndarray]) -> None:
+    """Reduce-scatter of [lo, hi) ([T] section "ZeRO-2", part "reduce-scatter
+    是什么"): rank r receives only the reduced values of the elements it owns,
+    written into its shard array (indexed from r*S)."""
+    for r in range(plan_.n_ranks):
+        olo, ohi = plan_.owned(r)
+        a, b = max(lo, olo), min(hi, ohi)
+        if a >= b:
+            continue
+        grad_shards[r][a - olo:b - olo] = reduce_mean([g[a:b] for g in rank_grads])
+
+
+def all_gather(param_shards: Sequence[np.ndarray], plan_: Plan, lo: int, hi: int,
+               rank_out: Sequence[np.ndarray], out_base: int = 0) -> None:
+    """All-gather of [lo, hi) ([T] section "ZeRO-1", part "all-gather 是什么"):
+    each rank contributes the part of its owned shard inside [lo, hi) and
+    every destination receives the concatenation.  ``rank_out[q]`` is indexed
+    from flat position ``out_base``."""
+    for r in range(plan_.n_ranks):
+        olo, ohi = plan_.owned(r)
+        a, b = max(lo, olo), min(hi, ohi)
+        if a >= b:
+            continue
+        piece = param_shards[r][a - olo:b - olo]
+        for q in range(len(rank_out)):
+            rank_out[q][a - out_base:b - out_base] = piece
+
+
+# ----------------------------------------------------------- step flows ----
+
+GradFn = Callable[[int, int], np.ndarray]  # (step, rank) -> uint16[psi_pad], pads 0
+
+
+@dataclass
+class RankState:
+    params: Optional[np.ndarray] = None   # bf16 full replica (DP/Z1/Z2) or shard (Z3)
+    grads: Optional[np.ndarray] = None    # bf16 full (DP/Z1) or owned shard (Z2/Z3)
+    master: Optional[np.ndarray] = None   # fp32, full (DP) or owned shard
+    m: Optional[np.ndarray] = None
+    v: Optional[np.ndarray] = None
+
+
+@dataclass
+class StepReport:
+    grad_norm: float
+    nonfinite: int
+    gathered: Optional[List[List[np.ndarray]]] = None  # Z3: per layer (schedule order), per rank
+
+
+def init_states(plan_: Plan, stage: int, master0: np.ndarray) -> List[RankState]:
+    """Every rank starts from the same fp32 master (pads 0), m = v = 0 and the
+    16-bit parameter copy equal to bf16(master)."""
+    assert master0.dtype == np.float32 and master0.size == plan_.psi_pad
+    p16 = bf16_rne(master0)
+    ranks = []
+    for r in range(plan_.n_ranks):
+        lo, hi = plan_.owned(r)
+        st = RankState()
+        if stage == STAGE_DP:
+            st.master = master0.copy()
+        else:
+            st.master = master0[lo:hi].copy()
+        st.m = np.zeros_like(st.master)
+        st.v = np.zeros_like(st.master)
+        st.params = p16[lo:hi].copy() if stage == STAGE_Z3 else p16.copy()
+        ranks.append(st)
+    return ranks
+
+
+def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
+         hp: AdamHP) -> StepReport:
+    """One optimizer step, t >= 1, following the pages' flow for ``stage``."""
+    N, S = plan_.n_ranks, plan_.shard
+    local = [grads(t, r).astype(np.uint16, copy=True) for r in range(N)]
+    assert all(a.size == plan_.psi_pad for a in local)
+    if stage in (STAGE_DP, STAGE_Z1):
+        # backward ends with a full all-reduce; every rank keeps the full grad
+        for lo, hi in plan_.buckets:
+            all_reduce(local, lo, hi)
+        for r in range(N):
+            ranks[r].grads = local[r]
+        g_full = local[0]
+        if stage == STAGE_DP:
+            # every rank runs the identical update on its full replica
+            for r in range(N):
+                ranks[r].params = adam(local[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t)
+        else:
+            # each rank updates only its owned shard, then all-gather
+            new_shards = []
+            for r in range(N):
+                lo, hi = plan_.owned(r)
+                new_shards.append(adam(local[r][lo:hi], ranks[r].master, ranks[r].m, ranks[r].v, hp, t))
+            all_gather(new_shards, plan_, 0, plan_.psi_pad, [ranks[r].params for r in range(N)])
+        return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full))
+    shards = [np.zeros(S, dtype=np.uint16) for _ in range(N)]
+    if stage == STAGE_Z2:
+        # layer-by-layer reduce-scatter through the fixed-size buffer
+        for lo, hi in plan_.buckets:
+            reduce_scatter(local, plan_, lo, hi, shards)
+        new_shards = []
+        for r in range(N):
+            ranks[r].grads = shards[r]
+            new_shards.append(adam(shards[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t))
+        all_gather(new_shards, plan_, 0, plan_.psi_pad, [ranks[r].params for r in range(N)])
+        g_full = np.concatenate(shards)
+        return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full))
+    assert stage == STAGE_Z3
+    # per layer, last to first: reduce-scatter the layer's gradient
+    for _, lo, hi in reversed(plan_.layers):
+        reduce_scatter(local, plan_, lo, hi, shards)
+    for r in range(N):
+        ranks[r].grads = shards[r]
+        ranks[r].params = adam(shards[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t)
+    # per layer, the all-gather of the updated shards into a temporary
+    # full-layer buffer on every rank, released after use
+    gathered = []
+    for _, lo, hi in reversed(plan_.layers):
+        tmp = [np.zeros(hi - lo, dtype=np.uint16) for _ in range(N)]
+        all_gather([ranks[r].params for r in range(N)], plan_, lo, hi, tmp, out_base=lo)
+        gathered.append(tmp)
+    g_full = np.concatenate(shards)
+    return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full),
+                      gathered=gathered)
+
+
+def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int, hp: AdamHP):
+    ranks = init_states(plan_, stage, master0)
+    reports = [step(plan_, stage, ranks, grads, t, hp) for t in range(1, steps + 1)]
+    return ranks, reports
+
+
+def full_view(plan_: Plan, stage: int, ranks: List[RankState]) -> dict:
+    """Assemble the flat master/m/v/params/grad (psi_pad each) from the ranks:
+    owned shards concatenated in rank order (rank 0's copy for DP)."""
+    if stage == STAGE_DP:
+        r0 = ranks[0]
+        return dict(master=r0.master, m=r0.m, v=r0.v, params=r0.params, grad=r0.grads)
+    cat = lambda name: np.concatenate([getattr(r, name) for r in ranks])
+    out = dict(master=cat("master"), m=cat("m"), v=cat("v"))
+    out["params"] = cat("params") if stage == STAGE_Z3 else ranks[0].params
+    if stage == STAGE_Z1:
+        out["grad"] = ranks[0].grads
+    else:
+        out["grad"] = cat("grads")
+    return out
+
+
+# ---------------------------------------------------- sampled trajectories ----
+
+def trajectory_at(master0: np.ndarray, rank_grads_per_step: Sequence[np.ndarray], hp: AdamHP,
+                  t0: int = 1) -> dict:
+    """Plain-DP result for a sample of elements, which every ZeRO stage must
+    reproduce ([T] sections "ZeRO-1"/"ZeRO-2"/"ZeRO-3": sharding the state
+    does not change the update).  ``rank_grads_per_step[s]`` is uint16[N, k]
+    for step t0 + s; ``master0`` is float32[k].  Returns the final master, m,
+    v, bf16 params and the last step's averaged bf16 grad."""
+    master = np.ascontiguousarray(master0, dtype=np.float32).copy()
+    m = np.zeros_like(master)
+    v = np.zeros_like(master)
+    params = bf16_rne(master)
+    g = np.zeros(master.size, dtype=np.uint16)
+    for s, rg in enumerate(rank_grads_per_step):
+        g = reduce_mean([rg[r] for r in range(rg.shape[0])])
+        params = adam(g, master, m, v, hp, t0 + s)
+    return dict(master=master, m=m, v=v, params=params, grad=g)
+
+
+# ------------------------------------------------- memory and communication ----
+
+def state_bytes(plan_: Plan, stage: int) -> tuple:
+    """Per-rank long-lived model-state bytes (params, grads, optimizer states)
+    for a mixed-precision Adam run ([Q] sections 二, 三.2, 四.2, 五.2; [M]
+    section 1): 16-bit params and grads at 2 B, fp32 master/m/v at 12 B; each
+    stage shards one more of the three ([T] section "一张总对比表")."""
+    P, S = plan_.psi_pad, plan_.shard
+    return {
+        STAGE_DP: (2 * P, 2 * P, 12 * P),
+        STAGE_Z1: (2 * P, 2 * P, 12 * S),
+        STAGE_Z2: (2 * P, 2 * S, 12 * S),
+        STAGE_Z3: (2 * S, 2 * S, 12 * S),
+    }[stage]
+
+
+def mem_model(psi: float, n_ranks: int) -> dict:
+    """The pages' per-card model-state totals in bytes, written out term by
+    term (16-bit params 2, 16-bit grads 2, fp32 master/m/v 12 per param, each
+    sharded over N where the stage shards it)."""
+    return {
+        STAGE_DP: 2 * psi + 2 * psi + 12 * psi,
+        STAGE_Z1: 2 * psi + 2 * psi + 12 * psi / n_ranks,
+        STAGE_Z2: 2 * psi + 2 * psi / n_ranks + 12 * psi / n_ranks,
+        STAGE_Z3: 2 * psi / n_ranks + 2 * psi / n_ranks + 12 * psi / n_ranks,
+    }
+
+
+def comm_elems(plan_: Plan, stage: int) -> dict:
+    """Logical elements each rank sends per step, ring convention: a
+    reduce-scatter or an all-gather of P elements over N ranks sends
+    P(N-1)/N, an all-reduce twice that.  DP: one all-reduce.  ZeRO-1: an
+    all-reduce and the parameter all-gather ([T] section "ZeRO-1"; [Q] section
+    三.3).  ZeRO-2: reduce-scatter plus the all-gather.  ZeRO-3: a parameter
+    all-gather in the forward, another in the backward, and the gradient
+    reduce-scatter ([Q] section 五.4, 七)."""
+    P, N = plan_.psi_pad, plan_.n_ranks
+    one = P * (N - 1) // N
+    return {
+        STAGE_DP: dict(all_reduce=2 * one, reduce_scatter=0, all_gather=0),
+        STAGE_Z1: dict(all_reduce=2 * one, reduce_scatter=0, all_gather=one),
+        STAGE_Z2: dict(all_reduce=0, reduce_scatter=one, all_gather=one),
+        STAGE_Z3: dict(all_reduce=0, reduce_scatter=one, all_gather=2 * one),
+    }[stage]
