@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Throughput of the fused ZeRO optimizer step on B200.
+
+Default workload: 24 transformer layers of hidden 2048 (1,208,598,528
+params), N = 8 logical data-parallel ranks in one GPU's HBM, ZeRO-2 with the
+fixed 200,000,000-element bucket schedule.  One step = one reduce-scatter +
+Adam + all-gather pass over every parameter (7 fused kernel launches), the
+8 gradient replicas already resident in HBM.
+
+Prints one JSON line (rank 0): params/s for the whole job, the fused
+kernel's achieved HBM bandwidth against the measured copy peak, the same
+metric end to end through the C ABI with gradients copied from pinned host
+memory, and the CPU oracle timed on a bounded sample of the same workload.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 (launched by torch.distributed.run, one process per GPU)
+every GPU runs its own full job (independent replicas of the workload; the
+step has no inter-GPU exchange): weak scaling, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fused ZeRO step params/sec (1 B200); achieved HBM GB/s vs ~8 TB/s roofline"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc", "kernels.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle leg")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--blocks-per-sm", type=int, default=0)
+    ap.add_argument("--replica-pad", type=int, default=0)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
+                    help="gpt-1.2b: the benchmark workload; flat-32m: a 33.5M-param flat buffer, "
+                         "N = 8, one bucket (2 GB on the device; for profiler captures)")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------ environment ----
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Largest value over all ranks (every rank calls this the same number of times)."""
+    if dist is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_for_current_kernel(stage: int, n_ranks: int, elems_per_launch: float):
+    """Per-launch DRAM bytes from the committed ncu summary, scaled to this
+    launch size, or None when the kernel source changed since the capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        with open(KERNEL_SOURCE, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if d.get("kernels_cu_sha256") != digest:
+            return None
+        key = f"stage{stage}_N{n_ranks}"
+        per_elem = d["dram_bytes_per_elem"][key]
+        return per_elem * elems_per_launch
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- workload ----
+
+def _gpt_1p2b():
+    from synth import workloads as W
+
+    return W.gpt_1p2b_n8()
+
+
+def _flat_32m():
+    from synth import workloads as W
+
+    w = W.flat_sweep(1 << 25, 8)
+    w.bucket_elems = 1 << 25
+    return w
+
+
+WORKLOADS = {"gpt-1.2b": _gpt_1p2b, "flat-32m": _flat_32m}
+_ARGS = None
+
+
+def workload():
+    return WORKLOADS[_ARGS.workload if _ARGS is not None else "gpt-1.2b"]()
+
+
+def cpu_baseline(w, steps: int = 2) -> dict:
+    """The oracle, as it stands (single-threaded), on a bounded sample of the
+    workload: the first transformer layer's tensors (50,358,272 params), the
+    same N, one fixed-size bucket, ``steps`` literal ZeRO-2 steps."""
+    import numpy as np
+
+    import oracle
+    from synth import workloads as W
+
+    k = w.layer_id.count(0)
+    numel, layer = w.numel[:k], w.layer_id[:k]
+    p = oracle.plan(numel, layer, w.n_ranks, w.bucket_elems)
+    m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+    grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
+             for r in range(w.n_ranks)]
+    ranks = oracle.init_states(p, oracle.STAGE_Z2, m0)
+    hp = oracle.AdamHP(**w.hyper.__dict__)
+    t0 = time.perf_counter()
+    for t in range(1, steps + 1):
+        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+    dt = time.perf_counter() - t0
+    return {"value": p.psi * steps / dt, "unit": "params/s", "cores": 1, "kind": "oracle",
+            "sample": f"first layer of the workload ({p.psi} params, N={w.n_ranks}), {steps} literal "
+                      f"ZeRO-2 steps, single-threaded C+numpy oracle, input generation untimed",
+            "seconds": dt}
+
+
+# -------------------------------------------------------------------- ours ----
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import synth
+    import zero_sharded_optimizer_sm_b200 as z
+    from synth import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = workload()
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, z.ZERO_STAGE_2, bucket_elems=w.bucket_elems,
+                          hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
+                          replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm, device=dev)
+    offsets = opt.offsets()
+    mv = opt.view(z.ZERO_VIEW_MASTER)
+    b = W.master_base(w)
+    for off, n in zip(offsets, w.numel):
+        synth.dev_f32(b, off, n, W.MASTER_DIST, mv.data_ptr() + 4 * off, s)
+    opt.load_master(None)
+    # the step's inputs: N full gradient replicas resident in HBM (19.3 GB)
+    reps = torch.empty((w.n_ranks, opt.psi_pad), dtype=torch.int16, device=dev)
+    for r in range(w.n_ranks):
+        gb = W.grad_base(w, 1, r)
+        for off, n in zip(offsets, w.numel):
+            synth.dev_bf16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
+    rep_list = list(reps)
+    torch.cuda.synchronize(dev)
+    for _ in range(args.warmup):
+        opt.step_resident(rep_list)
+    torch.cuda.synchronize(dev)
+    opt.set_timing(True)
+    opt.kernel_timing()  # empty the record
+    sampler = ClockSampler(local)
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        opt.step_resident(rep_list)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist)
+    clocks = sampler.stop()
+    kt = opt.kernel_timing()
+    opt.set_timing(False)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, dist, dev)
+    stats = opt.read_stats()
+    value = world * w.psi * args.steps / (ms / 1e3)
+    launches = kt["launches"]
+    kernel_ms = kt["ms"] / max(1, launches)
+    achieved = kt["model_bytes"] / max(1, launches) / (kernel_ms / 1e3) / 1e9 if launches else None
+    peak, peak_kind = measured_peaks()
+    elems_per_launch = w.psi / max(1, len(opt.buckets()))
+    traffic = traffic_for_current_kernel(2, w.n_ranks, elems_per_launch)
+
+    # end to end through the C ABI: every bucket's N gradient slices copied
+    # from pinned host memory into the fixed-size buffer, then the fused
+    # launch; the step's statistics read back to the host.
+    e2e = None
+    if not args.no_e2e:
+        max_bucket = max(hi - lo for lo, hi in opt.buckets())
+        host = torch.empty((w.n_ranks, max_bucket), dtype=torch.int16, pin_memory=True)
+        host.copy_(reps[:, :max_bucket])
+        h2d = 0
+
+        def grad_fn(t, lo, hi, bufs, stream_):
+            nonlocal h2d
+            for r, ptr in enumerate(bufs):
+                dst = opt._tensor_at(ptr, hi - lo, torch.int16)
+                dst.copy_(host[r, : hi - lo], non_blocking=True)
+                h2d += 2 * (hi - lo)
+            return 0
+
+        del reps, rep_list
+        torch.cuda.empty_cache()
+        opt.step(grad_fn, stats=True)  # warm-up of the host path
+        h2d = 0
+        barrier(dist)
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            opt.step(grad_fn, stats=True)
+        e2e_s = time.perf_counter() - t0
+        barrier(dist)
+        e2e_s = max_over_ranks(e2e_s, dist, dev)
+        e2e = {"value": world * w.psi * args.e2e_steps / e2e_s, "unit": "params/s",
+               "h2d_bytes_per_step": h2d // args.e2e_steps, "d2h_bytes_per_step": 16,
+               "steps": args.e2e_steps,
+               "how": "zero_step through the C ABI; grad_fn copies each bucket's N gradient slices "
+                      "from pinned host memory into the 200M-element buffer; stats (grad norm, "
+                      "non-finite count) read back every step"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "params/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp32",
+        "data": "synthetic (seeded counter-hash gradients and weights, no dataset)",
+        "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks, "stage": 2,
+                   "bucket_elems": w.bucket_elems, "buckets": len(opt.buckets()),
+                   "storage": "bf16 grads/params, fp32 master/m/v",
+                   "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
+                         f"per step vs 126 MB L2",
+                   "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy peak", "kernel": "fused_step_kernel",
+                     "kernel_ms_per_launch": kernel_ms, "launches": launches,
+                     "model_bytes_per_launch": kt["model_bytes"] / max(1, launches),
+                     "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "grad_norm_last_step": stats["grad_norm"],
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    opt.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------- reference ----
+
+def reference_sample(w, steps_total: int):
+    """A contiguous leading slice of the workload's first layer, sized so that
+    ``steps_total`` oracle steps take about a minute (the oracle does ~9M
+    params/s at N = 8 on one core), at least 8192*N elements."""
+    k = w.layer_id.count(0)
+    numel = list(w.numel[:k])
+    budget = max(8192 * w.n_ranks, int(5e8 / max(1, steps_total)))
+    out, total = [], 0
+    for n in numel:
+        if total >= budget:
+            break
+        take = min(n, budget - total)
+        out.append(take)
+        total += take
+    return out, [0] * len(out)
+
+
+def run_reference(args, world, rank, local):
+    """The CPU oracle timed on the machine's host cores, same metric and unit."""
+    if rank != 0:
+        return
+    from synth import workloads as W
+
+    import oracle
+
+    w = workload()
+    numel, layer = reference_sample(w, args.steps + args.warmup)
+    p = oracle.plan(numel, layer, w.n_ranks, w.bucket_elems)
+    m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+    grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
+             for r in range(w.n_ranks)]
+    ranks = oracle.init_states(p, oracle.STAGE_Z2, m0)
+    hp = oracle.AdamHP(**w.hyper.__dict__)
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        t += 1
+        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+    dt = time.perf_counter() - t0
+    value = p.psi * args.steps / dt
+    sample = (f"leading {p.psi} params of the first layer of {w.name} (N={w.n_ranks}) per step, "
+              f"literal ZeRO-2 step of the single-threaded oracle, input generation untimed")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+        "data": "synthetic", "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks,
+                                        "stage": 2, "bucket_elems": w.bucket_elems},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    global _ARGS
+    args = parse_args(argv)
+    _ARGS = args
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        print(f"--gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,359 @@
+/*
+ * zero_sm.h -- C ABI of the B200 (sm_100a) ZeRO optimizer-step library.
+ *
+ * The library runs the data-parallel optimizer step of ZeRO (Zero Redundancy
+ * Optimizer) over N logical data-parallel ranks whose buffers all live in one
+ * GPU's HBM: it reduces the N ranks' bf16 gradient replicas (fp32 sum in rank
+ * order 0..N-1, then the 1/N mean), runs mixed-precision Adam on each rank's
+ * owned shard (fp32 master weight, m and v, bias-corrected, decoupled weight
+ * decay) and all-gathers the updated bf16 parameters back to the ranks.
+ *
+ * Sources (three web pages on ZeRO; cited by title and section):
+ *   [T] "ZERO训练技术" (wqh011128.github.io)
+ *   [M] "ZeRO：从优化器状态到残差状态的显存优化" (xuesongtap.github.io)
+ *   [Q] mstx.cn post 475, a ZeRO interview write-up
+ *
+ * Conventions for every entry point
+ *   - Returns a zero_status; ZERO_OK (0) on success.  No exception, signal,
+ *     device trap or assert crosses this boundary.  On failure the context
+ *     (when there is one) keeps a message readable through zero_last_error().
+ *   - The library never allocates device memory.  The caller sizes the arenas
+ *     with zero_buffer_sizes(), allocates them (any allocator; 256-byte
+ *     aligned) and lends them with zero_bind() until zero_destroy().  This is
+ *     the pre-allocated contiguous pool of [M] section 3.4 ("MD"): buffer
+ *     lifetimes are managed inside caller-owned memory, never by the system
+ *     allocator during a step.
+ *   - "stream" is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  All device work of a call is enqueued on it, asynchronously.
+ *     Launch errors are reported as ZERO_ECUDA by the call that launched;
+ *     asynchronous device faults surface as ZERO_ECUDA from the next call that
+ *     synchronises (zero_read_stats, or zero_step with a stats pointer).
+ *   - Element indices refer to the padded flat parameter space [0, psi_pad):
+ *     tensors laid end to end in list order, each starting on a multiple of
+ *     8 elements, the total padded to a multiple of 8*N.  Rank r owns the
+ *     contiguous shard [r*S, (r+1)*S), S = psi_pad / N ([T] section "ZeRO-1",
+ *     part on how optimizer states are split).  Interval bounds lo, hi passed
+ *     to the library must be multiples of 8 with 0 <= lo <= hi <= psi_pad.
+ *   - bf16 data travels as raw 16-bit patterns (uint16_t); pad elements of
+ *     every gradient input must be 0.
+ *   - The calls that take a context are not thread-safe on the same context.
+ */
+#ifndef ZERO_SM_H
+#define ZERO_SM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZERO_SM_VERSION 1
+#define ZERO_MAX_RANKS 128
+
+typedef enum zero_status {
+  ZERO_OK = 0,
+  ZERO_EINVAL = 1,   /* a bad argument: null, misaligned, out of range, wrong stage */
+  ZERO_ENOMEM = 2,   /* an arena the caller sized is too small for this context */
+  ZERO_ECUDA = 3,    /* a CUDA runtime error (launch or asynchronous fault) */
+  ZERO_ESTATE = 4,   /* call out of order: arenas not bound, hyper-parameters unset */
+  ZERO_ENOTIMPL = 5  /* a combination this build does not provide */
+} zero_status;
+
+/* ZeRO stages ([T] section "一张总对比表"; [Q] section 一). */
+enum {
+  ZERO_STAGE_DP = 0, /* plain data parallel: every rank holds everything */
+  ZERO_STAGE_1 = 1,  /* optimizer states sharded */
+  ZERO_STAGE_2 = 2,  /* + gradients sharded (bucketed reduce-scatter) */
+  ZERO_STAGE_3 = 3   /* + parameters sharded (per-layer gather into a temporary) */
+};
+
+/* The parameter list: n_tensors sizes in flat order, each tagged with a layer
+ * id; layer ids must be non-decreasing (a layer is a contiguous run). */
+typedef struct zero_layout {
+  int32_t n_tensors;
+  const int64_t* numel;     /* host array, n_tensors entries, each >= 0 */
+  const int32_t* layer_id;  /* host array, n_tensors entries, non-decreasing */
+} zero_layout;
+
+/* Adam hyper-parameters as the user writes them (binary64).  Each scalar the
+ * device uses (beta1, beta2, 1-beta1, 1-beta2, 1-beta^t, 1-lr*wd, lr, eps) is
+ * derived in binary64 and rounded once to binary32. */
+typedef struct zero_adam_hparams {
+  double lr, beta1, beta2, eps, weight_decay;
+} zero_adam_hparams;
+
+/* Arenas the caller allocates and lends (zero_bind).  Unused arenas have
+ * size 0 and may be NULL. */
+enum {
+  ZERO_ARENA_STATES = 0,      /* fp32 master, m, v: 3 x psi_pad x 4 B */
+  ZERO_ARENA_PARAMS = 1,      /* bf16 params: N replicas of psi_pad (stage 1, 2) or the
+                                 psi_pad owned shards, rank order (stage 3) */
+  ZERO_ARENA_GRADS = 2,       /* bf16 gradient inputs: N full replicas (stage 1), N buckets
+                                 of bucket_elems (stage 2, the fixed buffer "CB" of [M]
+                                 section 3.3), N slots of the largest layer (stage 3) */
+  ZERO_ARENA_GRAD_SHARDS = 3, /* bf16 reduced gradient shards, psi_pad (stage 2, 3, unless
+                                 ZERO_OPT_KEEP_GRAD_SHARDS is 0) */
+  ZERO_ARENA_GATHER = 4,      /* stage 3: N temporary full-layer buffers (largest layer) */
+  ZERO_ARENA_SCRATCH = 5,     /* norm partials, counters and stats (small) */
+  ZERO_NUM_ARENAS = 6
+};
+
+typedef struct zero_sizes {
+  int64_t psi;            /* real parameter count */
+  int64_t psi_pad;        /* padded flat length */
+  int64_t shard;          /* S = psi_pad / N */
+  int64_t max_layer;      /* largest layer span (elements, padded) */
+  int64_t replica_pitch;  /* bytes between consecutive rank buffers in PARAMS/GRADS/GATHER */
+  int32_t n_buckets;      /* intervals of the bucket schedule */
+  int32_t n_layers;
+  int64_t arena_bytes[ZERO_NUM_ARENAS];
+} zero_sizes;
+
+typedef struct zero_step_stats {
+  double grad_norm;        /* sqrt(sum of squares of the averaged bf16 gradient), fp64 */
+  int64_t nonfinite;       /* averaged gradient elements that are Inf or NaN */
+  int64_t step;            /* Adam step number t the statistics belong to */
+  int64_t comm_elems[3];   /* logical elements each rank sends per step: all-reduce,
+                              reduce-scatter, all-gather (ring convention) */
+} zero_step_stats;
+
+/* Options (zero_set_option, before zero_bind). */
+enum {
+  ZERO_OPT_KEEP_GRAD_SHARDS = 1, /* stage 2/3: 1 (default) keeps the reduced bf16 gradient
+                                    shards (GRAD_SHARDS arena; the fused step stores them and
+                                    the unfused reduce-scatter/Adam calls use them); 0 drops
+                                    that arena: the fused step keeps the reduced gradient in
+                                    registers only and zero_reduce_scatter/zero_adam_shard
+                                    return ZERO_ESTATE */
+  ZERO_OPT_REPLICA_PAD = 2,      /* extra bytes (multiple of 256, < 1 MiB) between consecutive
+                                    rank buffers; default 0 */
+  ZERO_OPT_BLOCKS_PER_SM = 3,    /* fused-kernel CTAs per SM (0 = occupancy maximum) */
+  ZERO_OPT_TIMING = 4            /* 1: record a CUDA event pair on the launching stream around
+                                    every fused-step kernel launch (read with
+                                    zero_kernel_timing); may be set at any time; default 0 */
+};
+
+/* Views (zero_view). */
+enum {
+  ZERO_VIEW_MASTER = 0,      /* fp32 [psi_pad] */
+  ZERO_VIEW_EXP_AVG = 1,     /* fp32 [psi_pad] (m) */
+  ZERO_VIEW_EXP_AVG_SQ = 2,  /* fp32 [psi_pad] (v) */
+  ZERO_VIEW_PARAM = 3,       /* bf16: rank r's replica [psi_pad] (stage 1, 2) or the
+                                shards [psi_pad] (stage 3, rank ignored) */
+  ZERO_VIEW_GRAD_SHARD = 4,  /* bf16 [psi_pad] (stage 2, 3) */
+  ZERO_VIEW_GRAD_BUF = 5,    /* bf16: rank r's gradient input buffer */
+  ZERO_VIEW_GATHER = 6       /* bf16: rank r's temporary full-layer buffer (stage 3) */
+};
+
+typedef struct zero_ctx zero_ctx;
+
+/*
+ * Gradient producer: the stand-in for the backward pass ([T] section
+ * "ZeRO-2", part "2. 反向": a layer's gradients exist as soon as its backward
+ * finishes).  Called once per interval of the schedule, in schedule order,
+ * before that interval is reduced.  It must fill, for every rank r, the
+ * hi - lo bf16 values of flat elements [lo, hi) at rank_bufs[r] (device
+ * pointers into the GRADS arena) with work enqueued on `stream`.  Returns 0
+ * on success; any other value aborts the step with ZERO_EINVAL.
+ */
+typedef int (*zero_grad_fn)(void* user, int64_t step, int64_t lo, int64_t hi,
+                            void* const* rank_bufs, void* stream);
+
+/*
+ * Consumer of a stage-3 temporary gathered layer ([T] section "ZeRO-3",
+ * parts "1. 前向" and "2. 反向"): called after the layer [lo, hi) has been
+ * gathered into every rank's temporary buffer rank_bufs[r] (hi - lo bf16
+ * values) and before the buffer is reused for the next layer.  Work must be
+ * enqueued on `stream`.  Returns 0 on success.
+ */
+typedef int (*zero_gather_fn)(void* user, int32_t layer, int64_t lo, int64_t hi,
+                              void* const* rank_bufs, void* stream);
+
+/* ------------------------------------------------------------------ setup -- */
+
+/* Library ABI version (ZERO_SM_VERSION). */
+int32_t zero_version(void);
+
+/*
+ * Plan a context for `layout` over n_ranks logical ranks (1..ZERO_MAX_RANKS)
+ * at `stage` (ZERO_STAGE_1..3; ZERO_STAGE_DP returns ZERO_ENOTIMPL), with the
+ * fixed communication buffer of bucket_elems elements per rank ([M] section
+ * 3.3 "CB"; > 0, multiple of 8).  Host only, no device work.  *out receives
+ * a context owned by the caller (free with zero_destroy).
+ * Errors: ZERO_EINVAL for null pointers, bad sizes or decreasing layer ids.
+ */
+zero_status zero_init(const zero_layout* layout, int32_t n_ranks, int32_t stage,
+                      int64_t bucket_elems, zero_ctx** out);
+
+/* Set an option (ZERO_OPT_*) before zero_bind.  ZERO_ESTATE after binding. */
+zero_status zero_set_option(zero_ctx* ctx, int32_t key, int64_t value);
+
+/* Sizes of the plan and of each arena (bytes).  Host only. */
+zero_status zero_buffer_sizes(const zero_ctx* ctx, zero_sizes* out);
+
+/* Flat start of every tensor (host array of n_tensors). */
+zero_status zero_tensor_offsets(const zero_ctx* ctx, int64_t* out, int32_t cap);
+
+/* The bucket schedule ([M] section 3.3; [T] section "ZeRO-2"): tensors
+ * walked from the last to the first, packed into intervals of at most
+ * bucket_elems; a larger tensor is cut into bucket-sized chunks from its end.
+ * Writes min(cap, n) (lo, hi) pairs to lo_hi and returns n through *n_out. */
+zero_status zero_buckets(const zero_ctx* ctx, int64_t* lo_hi, int32_t cap, int32_t* n_out);
+
+/* Layer spans in layer order: (layer id, lo, hi) triples as int64. */
+zero_status zero_layers(const zero_ctx* ctx, int64_t* id_lo_hi, int32_t cap, int32_t* n_out);
+
+/*
+ * Lend the arenas: arenas[k] is a device pointer to at least arena_bytes[k]
+ * bytes (zero_buffer_sizes), 256-byte aligned, or NULL when that size is 0.
+ * Reads the device's SM count and the kernels' occupancy once (the current
+ * CUDA device must be the one the arenas live on).  The memory stays the
+ * caller's; the library uses it until zero_destroy.
+ * Errors: ZERO_EINVAL (null or misaligned), ZERO_ESTATE (already bound),
+ * ZERO_ECUDA (device query failed).
+ */
+zero_status zero_bind(zero_ctx* ctx, void* const* arenas);
+
+/* Adam hyper-parameters (required before any update). */
+zero_status zero_set_hparams(zero_ctx* ctx, const zero_adam_hparams* hp);
+
+/*
+ * Initialise the optimizer state from fp32 master weights: master_dev is a
+ * device array of psi_pad floats (pads 0, 16-byte aligned), or NULL when the
+ * caller has already written the master weights into ZERO_VIEW_MASTER (which
+ * saves a second psi_pad-sized buffer).  Copies them into the master shards,
+ * zeroes m, v and the reduced-gradient shards, writes bf16(master) (round to
+ * nearest even) to every rank's parameter replica (stage 1, 2) or to the
+ * parameter shards (stage 3), and resets the step counter to 0.
+ */
+zero_status zero_load_master(zero_ctx* ctx, const float* master_dev, void* stream);
+
+/* Step counter: the t of the last update (0 after zero_load_master). */
+zero_status zero_get_step(const zero_ctx* ctx, int64_t* t);
+zero_status zero_set_step(zero_ctx* ctx, int64_t t);
+
+/* Device pointer and element count of a view (ZERO_VIEW_*) for rank r. */
+zero_status zero_view(const zero_ctx* ctx, int32_t what, int32_t rank, void** ptr,
+                      int64_t* n_elems);
+
+/* Per-rank long-lived model-state bytes {params, grads, optimizer states}
+ * ([Q] sections 二, 三.2, 四.2, 五.2; [M] section 1): 2 B per 16-bit param or
+ * grad, 12 B per fp32 master+m+v, each sharded 1/N where the stage shards it.
+ * Temporary buffers (the bucket and the gather slots) are not included. */
+zero_status zero_state_bytes(const zero_ctx* ctx, int32_t rank, int64_t out[3]);
+
+/* Logical elements each rank sends per step {all-reduce, reduce-scatter,
+ * all-gather}, ring convention: a reduce-scatter or an all-gather of P
+ * elements sends P(N-1)/N, an all-reduce twice that.  Stage 1: all-reduce +
+ * all-gather ([T] section "ZeRO-1"); stage 2: reduce-scatter + all-gather;
+ * stage 3: reduce-scatter + two all-gathers, forward and backward ([Q]
+ * section 五.4) -- 1.5 times the all-reduce volume ([M] section 2). */
+zero_status zero_comm_elems(const zero_ctx* ctx, int64_t out[3]);
+
+/* ------------------------------------------------ the step and its parts -- */
+
+/*
+ * Reduce-scatter of [lo, hi) ([T] section "ZeRO-2", part on reduce-scatter;
+ * [Q] section 四.3): for every element i, g_i = bf16(fp32 sum over ranks
+ * 0..N-1 of rank_grads[r][i - lo], times fp32(1/N)), written to the owner's
+ * reduced-gradient shard (GRAD_SHARDS arena, flat index i).  rank_grads is a
+ * host array of N device pointers, each at flat element lo of that rank's
+ * gradient (16-byte aligned); NULL means the bound GRADS arena buffers
+ * (bucket/slot start at lo).  Stage 2 and 3 only.  Also accumulates the
+ * gradient norm and non-finite count of the current step.
+ */
+zero_status zero_reduce_scatter(zero_ctx* ctx, int64_t lo, int64_t hi,
+                                const void* const* rank_grads, void* stream);
+
+/*
+ * All-reduce of [lo, hi) in place ([T] section "ZeRO-1", part "2. 反向"):
+ * every rank's gradient buffer receives the same g_i as above.  rank_grads
+ * as for zero_reduce_scatter (NULL = the bound full replicas).  Stage 1.
+ */
+zero_status zero_all_reduce(zero_ctx* ctx, int64_t lo, int64_t hi, void* const* rank_grads,
+                            void* stream);
+
+/*
+ * Adam on rank `rank`'s owned shard (-1 = every rank's shard in one launch)
+ * for step t >= 1 ([T] section "ZeRO-1", part "3. 更新"): per element, in
+ * binary32 with each operation rounded to nearest even, in this order:
+ *   p = p*(1-lr*wd);  m = b1*m + (1-b1)*g;  v = b2*v + (1-b2)*(g*g);
+ *   p = p - lr*((m/(1-b1^t)) / (sqrt(v/(1-b2^t)) + eps));  out = bf16(p).
+ * g is the reduced bf16 gradient (stage 2/3: GRAD_SHARDS; stage 1: the
+ * owner's full replica in GRADS).  out goes to the owner's own parameter
+ * replica (stage 1/2) or to the parameter shards (stage 3).  Does not change
+ * the context's step counter (zero_set_step does).
+ */
+zero_status zero_adam_shard(zero_ctx* ctx, int32_t rank, int64_t t, void* stream);
+
+/*
+ * All-gather of [lo, hi) ([T] section "ZeRO-1", part on all-gather): the
+ * owners' updated bf16 parameters are copied to every rank's destination.
+ * Source: stage 1/2 the owner's own replica, stage 3 the parameter shards.
+ * rank_out: host array of N device pointers, each at flat element lo of the
+ * destination; NULL = the bound destinations (stage 1/2: the N parameter
+ * replicas; stage 3: the N temporary layer buffers, [lo, hi) inside one
+ * layer, placed at offset lo - layer start).
+ */
+zero_status zero_all_gather(zero_ctx* ctx, int64_t lo, int64_t hi, void* const* rank_out,
+                            void* stream);
+
+/*
+ * One full optimizer step t = (step counter) + 1, fused: per interval of the
+ * stage's schedule -- stage 1 and 2 the bucket schedule, stage 3 the layers
+ * from last to first -- grad_fn fills the ranks' gradient buffers, then one
+ * kernel reads the N replicas of each owned element once, reduces them,
+ * runs Adam in registers, writes master/m/v once and writes the bf16 result
+ * to all N destinations ([T] sections "ZeRO-1", "ZeRO-2", "ZeRO-3").
+ * Stage 1 also writes the averaged gradient back to the N replicas (the
+ * all-reduce result); stage 3 also writes the parameter shard and then calls
+ * gather_fn (may be NULL) with the layer's temporary buffers.
+ * grad_fn may be NULL for stage 1 only (the replicas are already filled).
+ * stats (may be NULL): when given, the call synchronises `stream` and fills
+ * it; otherwise nothing synchronises (zero_read_stats reads it later).
+ */
+zero_status zero_step(zero_ctx* ctx, zero_grad_fn grad_fn, void* grad_user,
+                      zero_gather_fn gather_fn, void* gather_user, void* stream,
+                      zero_step_stats* stats);
+
+/*
+ * The same step reading the gradients from caller-held full replicas:
+ * rank_grads is a host array of N device pointers to psi_pad bf16 values
+ * each (16-byte aligned).  The schedule, kernels and results are those of
+ * zero_step; the intervals index straight into the replicas instead of
+ * passing through the fixed-size buffer.  Stage 1 writes the all-reduced
+ * gradient back into these replicas.
+ */
+zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
+                               zero_gather_fn gather_fn, void* gather_user, void* stream,
+                               zero_step_stats* stats);
+
+/*
+ * Fused-kernel timing (ZERO_OPT_TIMING = 1): waits for the last recorded
+ * launch, then returns the summed device time of the launches recorded since
+ * the previous call (*ms), their number (*launches) and the bytes those
+ * launches must move by the byte model of the fused step (*model_bytes):
+ * per element, stage 1: 6N+24 (N gradient reads, N all-reduce write-backs,
+ * 12 B of state read and written, N parameter writes), stage 2: 4N+24,
+ * stage 3: 4N+26 (plus the parameter shard), each +2 when the reduced
+ * gradient shard is kept.  Resets the record.  At most 4096 launches are
+ * recorded between two calls; later ones are not timed.
+ */
+zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, double* model_bytes);
+
+/* Synchronise `stream` and read the last step's statistics. */
+zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
+
+/* Message of the last failure on ctx (never NULL; "" when none).  With
+ * ctx == NULL: the reason the calling thread's last zero_init failed. */
+const char* zero_last_error(const zero_ctx* ctx);
+
+/* Release a context (the arenas stay the caller's). NULL is a no-op. */
+void zero_destroy(zero_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_SM_H */

@@ -1,0 +1,181 @@
+"""CPU tests of the C-ABI library: it loads, exports every function the
+header declares, and its host-side planning and validation agree with the
+oracle's independently written plan.  No call here needs a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from synth import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zero_sm.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[a-z_][\w\s\*]*?\b(zero_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if not n.endswith("_fn")))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    import zero_sharded_optimizer_sm_b200 as z
+
+    declared = _declared_functions()
+    assert len(declared) >= 20, declared
+    lib = ctypes.CDLL(z.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in zero_sm.h but not exported"
+    assert z.zero_version() == 1
+    # and the binding exposes the same names
+    for name in declared:
+        assert callable(getattr(z, name)), name
+
+
+def test_exported_symbols_are_exactly_the_header():
+    import zero_sharded_optimizer_sm_b200 as z
+
+    out = subprocess.run(["nm", "-D", "--defined-only", z.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted(set(re.findall(r"\bT (zero_\w+)$", out, flags=re.M)))
+    assert exported == _declared_functions()
+
+
+def _init(numel, layer, n_ranks, stage, bucket):
+    import zero_sharded_optimizer_sm_b200 as z
+
+    n = len(numel)
+    lay = z.zero_layout(n, (ctypes.c_int64 * n)(*numel), (ctypes.c_int32 * n)(*layer))
+    ctx = ctypes.c_void_p()
+    st = z.zero_init(ctypes.byref(lay), n_ranks, stage, bucket, ctypes.byref(ctx))
+    return st, ctx
+
+
+def _plan_of(ctx):
+    import zero_sharded_optimizer_sm_b200 as z
+
+    sizes = z.zero_sizes()
+    assert z.zero_buffer_sizes(ctx, ctypes.byref(sizes)) == 0
+    n = ctypes.c_int32()
+    z.zero_buckets(ctx, None, 0, ctypes.byref(n))
+    bk = (ctypes.c_int64 * (2 * n.value))()
+    assert z.zero_buckets(ctx, bk, n.value, ctypes.byref(n)) == 0
+    z.zero_layers(ctx, None, 0, ctypes.byref(n))
+    ly = (ctypes.c_int64 * (3 * n.value))()
+    assert z.zero_layers(ctx, ly, n.value, ctypes.byref(n)) == 0
+    return sizes, [(bk[2 * k], bk[2 * k + 1]) for k in range(len(bk) // 2)], \
+        [(int(ly[3 * k]), ly[3 * k + 1], ly[3 * k + 2]) for k in range(len(ly) // 3)]
+
+
+LAYOUTS = [
+    ([1], [0]),
+    ([5, 3], [0, 1]),
+    ([33, 1, 2, 17], [0, 1, 1, 2]),
+    ([7, 0, 11, 13, 2], [0, 0, 1, 2, 2]),
+    W.transformer_layers(3, 24, 96),
+    ([100], [0]),
+]
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("n_ranks", [1, 2, 3, 4, 8, 9, 64, 128])
+@pytest.mark.parametrize("bucket", [8, 16, 24, 200, 1 << 20])
+def test_planner_matches_oracle_plan(layout, n_ranks, bucket):
+    import zero_sharded_optimizer_sm_b200 as z
+
+    numel, layer = layout
+    for stage in (1, 2, 3):
+        st, ctx = _init(numel, layer, n_ranks, stage, bucket)
+        assert st == 0
+        try:
+            sizes, buckets, layers = _plan_of(ctx)
+            p = oracle.plan(numel, layer, n_ranks, bucket)
+            assert (sizes.psi, sizes.psi_pad, sizes.shard) == (p.psi, p.psi_pad, p.shard)
+            assert buckets == p.buckets
+            assert layers == p.layers
+            offs = (ctypes.c_int64 * len(numel))()
+            assert z.zero_tensor_offsets(ctx, offs, len(numel)) == 0
+            assert list(offs) == p.offset
+            for r in (0, n_ranks - 1):
+                got = (ctypes.c_int64 * 3)()
+                assert z.zero_state_bytes(ctx, r, got) == 0
+                assert tuple(got) == oracle.state_bytes(p, stage)
+            ce = (ctypes.c_int64 * 3)()
+            assert z.zero_comm_elems(ctx, ce) == 0
+            want = oracle.comm_elems(p, stage)
+            assert tuple(ce) == (want["all_reduce"], want["reduce_scatter"], want["all_gather"])
+            # arena sizes cover what each stage keeps
+            ab = list(sizes.arena_bytes)
+            assert ab[z.ZERO_ARENA_STATES] >= 12 * p.psi_pad
+            assert ab[z.ZERO_ARENA_SCRATCH] > 0
+            if stage in (1, 2):
+                assert ab[z.ZERO_ARENA_PARAMS] >= 2 * p.psi_pad * n_ranks
+            else:
+                assert ab[z.ZERO_ARENA_PARAMS] >= 2 * p.psi_pad
+                assert ab[z.ZERO_ARENA_GATHER] >= 2 * n_ranks * max(hi - lo for _, lo, hi in p.layers)
+            if stage == 2:
+                assert ab[z.ZERO_ARENA_GRADS] >= 2 * n_ranks * max(hi - lo for lo, hi in p.buckets)
+            if all(a % 256 == 0 for a in ab):
+                pass
+        finally:
+            z.zero_destroy(ctx)
+
+
+def test_init_rejects_bad_arguments():
+    import zero_sharded_optimizer_sm_b200 as z
+
+    assert _init([8], [0], 0, 2, 8)[0] == z.ZERO_EINVAL            # no ranks
+    assert _init([8], [0], 129, 2, 8)[0] == z.ZERO_EINVAL          # beyond the rank limit
+    assert _init([8], [0], 2, 4, 8)[0] == z.ZERO_EINVAL            # no such stage
+    assert _init([8], [0], 2, 0, 8)[0] == z.ZERO_ENOTIMPL          # plain DP is oracle-only
+    assert _init([8], [0], 2, 2, 12)[0] == z.ZERO_EINVAL           # bucket not a multiple of 8
+    assert _init([8], [0], 2, 2, 0)[0] == z.ZERO_EINVAL
+    assert _init([8, 8], [1, 0], 2, 2, 8)[0] == z.ZERO_EINVAL      # decreasing layer ids
+    assert b"non-decreasing" in z.zero_last_error(None)
+    assert _init([8, -1], [0, 0], 2, 2, 8)[0] == z.ZERO_EINVAL     # negative size
+    assert b"negative" in z.zero_last_error(None)
+    ctx = ctypes.c_void_p()
+    assert z.zero_init(None, 2, 2, 8, ctypes.byref(ctx)) == z.ZERO_EINVAL
+    assert z.zero_init(None, 2, 2, 8, None) == z.ZERO_EINVAL
+
+
+def test_calls_out_of_order_and_bad_pointers_fail_cleanly():
+    import zero_sharded_optimizer_sm_b200 as z
+
+    st, ctx = _init([64, 64], [0, 1], 4, 2, 64)
+    assert st == 0
+    try:
+        # nothing bound: every device call refuses with ZERO_ESTATE
+        assert z.zero_reduce_scatter(ctx, 0, 64, None, None) == z.ZERO_ESTATE
+        assert z.zero_adam_shard(ctx, -1, 1, None) == z.ZERO_ESTATE
+        assert z.zero_all_gather(ctx, 0, 64, None, None) == z.ZERO_ESTATE
+        assert z.zero_step(ctx, z.zero_grad_fn(), None, z.zero_gather_fn(), None, None, None) == z.ZERO_ESTATE
+        assert z.zero_load_master(ctx, None, None) == z.ZERO_ESTATE
+        assert b"not bound" in z.zero_last_error(ctx)
+        # options are validated
+        assert z.zero_set_option(ctx, z.ZERO_OPT_REPLICA_PAD, 100) == z.ZERO_EINVAL
+        assert z.zero_set_option(ctx, 99, 1) == z.ZERO_EINVAL
+        assert z.zero_set_option(ctx, z.ZERO_OPT_REPLICA_PAD, 512) == 0
+        # bind validates the pointers before touching the device
+        arenas = (ctypes.c_void_p * z.ZERO_NUM_ARENAS)(*([0x1000] * z.ZERO_NUM_ARENAS))
+        arenas[z.ZERO_ARENA_STATES] = 0x1010  # not 256-byte aligned
+        assert z.zero_bind(ctx, arenas) == z.ZERO_EINVAL
+        arenas[z.ZERO_ARENA_STATES] = None
+        assert z.zero_bind(ctx, arenas) == z.ZERO_EINVAL
+        assert z.zero_bind(ctx, None) == z.ZERO_EINVAL
+        hp = z.zero_adam_hparams(1e-3, 1.0, 0.999, 1e-8, 0.0)  # beta1 = 1 is out of range
+        assert z.zero_set_hparams(ctx, ctypes.byref(hp)) == z.ZERO_EINVAL
+        hp = z.zero_adam_hparams(1e-3, 0.9, 0.999, 1e-8, 0.0)
+        assert z.zero_set_hparams(ctx, ctypes.byref(hp)) == 0
+        v = ctypes.c_void_p()
+        n = ctypes.c_int64()
+        assert z.zero_view(ctx, z.ZERO_VIEW_MASTER, 0, ctypes.byref(v), ctypes.byref(n)) == z.ZERO_ESTATE
+        assert z.zero_state_bytes(ctx, 4, (ctypes.c_int64 * 3)()) == z.ZERO_EINVAL
+    finally:
+        z.zero_destroy(ctx)
+    z.zero_destroy(None)

@@ -1,0 +1,492 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs.
+
+Tolerances (stated for the method): reduced gradients and all indexing
+bit-exact; fp32 master/m/v within 2 ulp (relative 2.4e-7); bf16 parameters
+within 1 bf16 ulp.  The design computes the same IEEE operations in the same
+order as the oracle, so most checks below also assert bit equality.
+"""
+import gc
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle  # noqa: E402
+import synth  # noqa: E402
+from synth import workloads as W  # noqa: E402
+
+from harness import (DeviceFill, assert_bf16_close, assert_bits_equal, assert_f32_close,  # noqa: E402
+                     oracle_sampled, sample_indices, to_np)
+
+pytestmark = pytest.mark.gpu
+
+STAGE_OF = {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2, 3: oracle.STAGE_Z3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def _z():
+    import zero_sharded_optimizer_sm_b200 as z
+    return z
+
+
+def _hp(w):
+    z = _z()
+    return z.AdamHParams(**w.hyper.__dict__)
+
+
+def make_opt(w, stage, bucket=None, keep=True, **kw):
+    z = _z()
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=bucket, hparams=_hp(w),
+                          keep_grad_shards=keep, **kw)
+    fill = DeviceFill(w, opt.offsets(), opt.psi_pad)
+    stream = torch.cuda.current_stream().cuda_stream
+    mv = opt.view(z.ZERO_VIEW_MASTER)
+    fill.master_into(mv.data_ptr(), mv, stream)
+    opt.load_master(None)
+    return opt, fill
+
+
+def grad_fn_for(opt, fill):
+    def fn(t, lo, hi, bufs, stream):
+        for r, p in enumerate(bufs):
+            fill.grads_into(t, r, lo, hi, p, opt._tensor_at(p, hi - lo, torch.int16), stream)
+        return 0
+    return fn
+
+
+def norm_tol(n):
+    # both sides sum n exactly-squared terms in binary64 in different orders
+    return 2 * n * 2.0**-53 + 1e-15
+
+
+# -------------------------------------------------------------- generator ----
+
+def test_device_generator_matches_host_bitwise():
+    s = torch.cuda.current_stream().cuda_stream
+    for dist in (synth.Dist(synth.NORMAL, 1e-2, zero_mod=100), synth.Dist(synth.UNIFORM, 1e-2),
+                 synth.Dist(synth.NORMAL, 0.02)):
+        b = synth.base(0x5EED0002, synth.STREAM_GRAD, 3, 5)
+        n, idx0 = 1_000_003, 987_654_321
+        dev = torch.empty(n, dtype=torch.int16, device="cuda")
+        synth.dev_bf16(b, idx0, n, dist, dev.data_ptr(), s)
+        assert np.array_equal(to_np(dev), synth.host_bf16(b, idx0, n, dist))
+        devf = torch.empty(n, dtype=torch.float32, device="cuda")
+        synth.dev_f32(b, idx0, n, dist, devf.data_ptr(), s)
+        assert np.array_equal(to_np(devf).view(np.uint32), synth.host_f32(b, idx0, n, dist).view(np.uint32))
+
+
+# ------------------------------------------------------ oracle literal runs ----
+
+def _oracle_run(w, stage, bucket):
+    p = oracle.plan(w.numel, w.layer_id, w.n_ranks, bucket)
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def g(t, r):
+        return W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), w.grad_dist)
+
+    ranks, reps = oracle.run(p, stage, m0, g, w.steps, oracle.AdamHP(**w.hyper.__dict__))
+    return p, ranks, reps
+
+
+def _check_against_oracle(w, stage, bucket, exact=True):
+    z = _z()
+    p, ranks, reps = _oracle_run(w, STAGE_OF[stage], bucket)
+    ref = oracle.full_view(p, STAGE_OF[stage], ranks)
+    opt, fill = make_opt(w, stage, bucket=bucket, keep=True)
+    assert opt.offsets() == p.offset and opt.buckets() == p.buckets
+    gathered = []
+
+    def gather(layer, lo, hi, bufs, stream):
+        gathered.append((layer, lo, hi, [to_np(opt._tensor_at(b, hi - lo, torch.int16)) for b in bufs]))
+        return 0
+
+    gfn = grad_fn_for(opt, fill)
+    for t in range(1, w.steps + 1):
+        gathered.clear()
+        st = opt.step(gfn, gather if stage == 3 else None, stats=True)
+        assert st["step"] == t
+        rep = reps[t - 1]
+        assert st["nonfinite"] == rep.nonfinite
+        assert math.isclose(st["grad_norm"], rep.grad_norm, rel_tol=norm_tol(p.psi_pad))
+    got = dict(master=to_np(opt.view(z.ZERO_VIEW_MASTER)), m=to_np(opt.view(z.ZERO_VIEW_EXP_AVG)),
+               v=to_np(opt.view(z.ZERO_VIEW_EXP_AVG_SQ)))
+    for k in ("master", "m", "v"):
+        assert_f32_close(got[k], ref[k], f"stage {stage} {k}")
+        if exact:
+            assert_bits_equal(got[k], ref[k], f"stage {stage} {k}")
+    if stage in (1, 2):
+        for r in range(w.n_ranks):
+            pr = to_np(opt.view(z.ZERO_VIEW_PARAM, r))
+            assert_bf16_close(pr, ref["params"], f"stage {stage} params replica {r}")
+            if exact:
+                assert_bits_equal(pr, ref["params"], f"stage {stage} params replica {r}")
+    else:
+        ps = to_np(opt.view(z.ZERO_VIEW_PARAM))
+        assert_bf16_close(ps, ref["params"], "stage 3 param shards")
+        if exact:
+            assert_bits_equal(ps, ref["params"], "stage 3 param shards")
+        want = reps[-1].gathered
+        assert len(gathered) == len(want) == len(p.layers)
+        for (layer, lo, hi, bufs), (lid, llo, lhi), tmp in zip(gathered, reversed(p.layers), want):
+            assert (layer, lo, hi) == (lid, llo, lhi)
+            for r in range(w.n_ranks):
+                assert_bits_equal(bufs[r], tmp[r], f"stage 3 gathered layer {layer} rank {r}")
+    if stage == 1:
+        for r in range(w.n_ranks):
+            assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GRAD_BUF, r)), ranks[r].grads,
+                              f"stage 1 all-reduced grads rank {r}")
+    else:
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GRAD_SHARD)), ref["grad"], f"stage {stage} grad shards")
+    opt.close()
+
+
+def test_flat_1m_n4_zero2_every_element():
+    """1,048,576 params (4 x 512x512), N = 4, ZeRO-2, one bucket, 3 steps."""
+    w = W.flat_1m_n4()
+    _check_against_oracle(w, 2, None)
+
+
+TINY = [([1], [0]), ([5, 3], [0, 1]), ([8, 16, 9], [0, 0, 1]), ([33, 1, 2, 17], [0, 1, 1, 2]),
+        ([7, 0, 11, 13, 2], [0, 0, 1, 2, 2]), ([3000, 1, 4100], [0, 1, 2])]
+
+
+@pytest.mark.parametrize("layout", TINY)
+def test_tiny_layouts_all_ranks_buckets_stages(layout):
+    """Brute force: N = 1..9 and 16, bucket sizes 8/16/24/all, stages 1-3, 3
+    steps each, every element against the oracle's literal per-rank run."""
+    numel, layer = layout
+    for n_ranks in list(range(1, 10)) + [16]:
+        p0 = oracle.plan(numel, layer, n_ranks, 8)
+        for bucket in sorted({8, 16, 24, p0.psi_pad}):
+            for stage in (1, 2, 3):
+                w = W.Workload("tiny", numel, layer, n_ranks, (stage,), bucket,
+                               synth.Dist(synth.NORMAL, 1e-2, zero_mod=7), W.MASTER_DIST, 3,
+                               W.Hyper(lr=1e-2, weight_decay=0.1), 0xA0 + n_ranks)
+                _check_against_oracle(w, stage, bucket)
+
+
+def test_max_ranks_128():
+    numel, layer = [1000, 24], [0, 1]
+    w = W.Workload("tiny-N128", numel, layer, 128, (2,), 512, synth.Dist(synth.NORMAL, 1e-2),
+                   W.MASTER_DIST, 2, W.Hyper(), 0xC0)
+    for stage in (1, 2, 3):
+        _check_against_oracle(w, stage, 512)
+
+
+def test_two_layer_h768_n8_all_stages_every_element():
+    """Reduced transformer list (2 layers, hidden 768, 14.2M params), N = 8,
+    1% zero grads, AdamW wd 0.01, 5 steps: every element of every stage."""
+    numel, layer = W.transformer_layers(2, 768, 3072)
+    w = W.Workload("transformer-2L-h768-N8", numel, layer, 8, (1, 2, 3), 3_000_000,
+                   synth.Dist(synth.NORMAL, 1e-2, zero_mod=100), W.MASTER_DIST, 5,
+                   W.Hyper(weight_decay=0.01), W.SEED0 + 2)
+    for stage in (1, 2, 3):
+        _check_against_oracle(w, stage, 3_000_000)
+
+
+# ------------------------------------------------------------ unfused path ----
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_unfused_calls_equal_fused_step(stage):
+    """reduce-scatter (or all-reduce) per interval, Adam on every shard,
+    all-gather: the same bits as the fused step."""
+    z = _z()
+    numel, layer = W.transformer_layers(3, 64, 256)
+    w = W.Workload("unfused", numel, layer, 6, (stage,), 4096, synth.Dist(synth.NORMAL, 1e-2, zero_mod=9),
+                   W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01), 0xD0 + stage)
+    fused, ff = make_opt(w, stage, bucket=w.bucket_elems)
+    split, sf = make_opt(w, stage, bucket=w.bucket_elems)
+    gf = grad_fn_for(fused, ff)
+    gs = grad_fn_for(split, sf)
+    intervals = split.buckets() if stage != 3 else [(lo, hi) for _, lo, hi in reversed(split.layers())]
+    for t in range(1, w.steps + 1):
+        sf_ = fused.step(gf, stats=True)
+        for lo, hi in intervals:
+            if stage == 1:
+                bufs = [split.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() + 2 * lo for r in range(w.n_ranks)]
+                gs(t, lo, hi, bufs, torch.cuda.current_stream().cuda_stream)
+                split.all_reduce(lo, hi)
+            else:
+                bufs = [split.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() for r in range(w.n_ranks)]
+                gs(t, lo, hi, bufs, torch.cuda.current_stream().cuda_stream)
+                split.reduce_scatter(lo, hi)
+        split.adam_shard(-1, t)
+        for lo, hi in intervals:
+            split.all_gather(lo, hi)
+        split.t = t
+        ss = split.read_stats()
+        assert ss["grad_norm"] == sf_["grad_norm"] or math.isclose(ss["grad_norm"], sf_["grad_norm"], rel_tol=1e-12)
+        assert ss["nonfinite"] == sf_["nonfinite"]
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(fused.view(what), split.view(what))
+    for r in range(w.n_ranks if stage != 3 else 1):
+        assert torch.equal(fused.view(z.ZERO_VIEW_PARAM, r), split.view(z.ZERO_VIEW_PARAM, r))
+    if stage == 3:
+        # the last all-gather left the first layer in the temporary buffers
+        lo, hi = intervals[-1]
+        for r in range(w.n_ranks):
+            assert torch.equal(fused.view(z.ZERO_VIEW_GATHER, r)[: hi - lo], split.view(z.ZERO_VIEW_GATHER, r)[: hi - lo])
+    fused.close()
+    split.close()
+
+
+def test_adam_shard_per_rank_equals_all_ranks():
+    z = _z()
+    numel, layer = [4096, 2048], [0, 1]
+    w = W.Workload("per-rank", numel, layer, 4, (2,), 8192, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST,
+                   1, W.Hyper(), 0xE0)
+    a, fa = make_opt(w, 2, bucket=8192)
+    b, fb = make_opt(w, 2, bucket=8192)
+    for o, f in ((a, fa), (b, fb)):
+        bufs = [o.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() for r in range(4)]
+        grad_fn_for(o, f)(1, 0, o.psi_pad, bufs, torch.cuda.current_stream().cuda_stream)
+        o.reduce_scatter(0, o.psi_pad)
+    a.adam_shard(-1, 1)
+    for r in range(4):
+        b.adam_shard(r, 1)
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(a.view(what), b.view(what))
+    for r in range(4):
+        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+    a.close()
+    b.close()
+
+
+# ------------------------------------------------------------- edge cases ----
+
+def test_nonfinite_gradients_are_counted_and_propagate_like_the_oracle():
+    z = _z()
+    numel, layer = [4096, 1024], [0, 1]
+    w = W.Workload("nonfinite", numel, layer, 4, (2,), 8192, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST,
+                   1, W.Hyper(), 0xF0)
+    opt, fill = make_opt(w, 2, bucket=8192)
+    p = oracle.plan(numel, layer, 4, 8192)
+    host = [W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist) for r in range(4)]
+    host[1][[5, 77, 4100]] = [0x7F80, 0xFFC0, 0xFF80]  # +inf, NaN, -inf in rank 1
+    host[3][77] = 0x7F80
+    dev = [torch.from_numpy(h.view(np.int16)).cuda() for h in host]
+    st = opt.step_resident(dev, stats=True)
+    ranks = oracle.init_states(p, oracle.STAGE_Z2, W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w),
+                                                                 W.MASTER_DIST, as_f32=True))
+    rep = oracle.step(p, oracle.STAGE_Z2, ranks, lambda t, r: host[r], 1, oracle.AdamHP())
+    assert st["nonfinite"] == rep.nonfinite == 3
+    assert math.isnan(st["grad_norm"]) and math.isnan(rep.grad_norm)
+    ref = oracle.full_view(p, oracle.STAGE_Z2, ranks)
+    got = to_np(opt.view(z.ZERO_VIEW_MASTER))
+    assert np.array_equal(np.isnan(got), np.isnan(ref["master"]))
+    assert_f32_close(got, ref["master"], "master with nonfinite grads")
+    opt.close()
+
+
+def test_grad_fn_failure_aborts_the_step_with_einval():
+    z = _z()
+    w = W.Workload("abort", [1024], [0], 2, (2,), 1024, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 1,
+                   W.Hyper(), 1)
+    opt, _ = make_opt(w, 2)
+    with pytest.raises(z.ZeroError) as ei:
+        opt.step(lambda t, lo, hi, bufs, s: 7)
+    assert ei.value.status == z.ZERO_EINVAL
+    assert opt.t == 0
+    with pytest.raises(z.ZeroError):
+        opt.reduce_scatter(0, 12)  # not a multiple of 8
+    with pytest.raises(z.ZeroError):
+        opt.all_gather(0, opt.psi_pad + 8)
+    opt.close()
+
+
+# ------------------------------------------- full-size workloads, sampled ----
+
+def _sampled_check(opt, w, steps, stage, idx, ref):
+    z = _z()
+    it = torch.from_numpy(idx).cuda()
+    for name, what in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        got = to_np(opt.view(what)[it])
+        assert_f32_close(got, ref[name], f"{w.name} stage {stage} {name}")
+        assert_bits_equal(got, ref[name], f"{w.name} stage {stage} {name}")
+    if stage == 3:
+        got = to_np(opt.view(z.ZERO_VIEW_PARAM)[it])
+        assert_bits_equal(got, ref["params"], f"{w.name} param shards")
+    else:
+        for r in sorted({0, w.n_ranks // 2, w.n_ranks - 1}):
+            got = to_np(opt.view(z.ZERO_VIEW_PARAM, r)[it])
+            assert_bf16_close(got, ref["params"], f"{w.name} params replica {r}")
+            assert_bits_equal(got, ref["params"], f"{w.name} params replica {r}")
+    if stage in (2, 3):
+        got = to_np(opt.view(z.ZERO_VIEW_GRAD_SHARD)[it])
+        assert_bits_equal(got, ref["grad"], f"{w.name} grad shards")
+
+
+def test_transformer_85m_n8_stages_agree_and_match_dp():
+    """12 layers, hidden 768 (85,054,464 params), N = 8, ZeRO-1/2/3 from the
+    same seed, 5 steps: the three stages agree bit for bit on the device, and
+    sampled elements match the oracle's plain-DP result."""
+    z = _z()
+    w = W.gpt_85m_n8()
+    opts = {}
+    for stage in (1, 2, 3):
+        opt, fill = make_opt(w, stage, bucket=20_000_000)
+        gathered_ok = []
+
+        def gather(layer, lo, hi, bufs, stream, opt=opt):
+            shard = opt.view(z.ZERO_VIEW_PARAM)[lo:hi]
+            gathered_ok.append(all(torch.equal(opt._tensor_at(b, hi - lo, torch.int16), shard) for b in bufs))
+            return 0
+
+        gfn = grad_fn_for(opt, fill)
+        for t in range(1, w.steps + 1):
+            opt.step(gfn, gather if stage == 3 else None)
+        if stage == 3:
+            assert len(gathered_ok) == 12 * w.steps and all(gathered_ok)
+        else:
+            for r in range(1, w.n_ranks):
+                assert torch.equal(opt.view(z.ZERO_VIEW_PARAM, 0), opt.view(z.ZERO_VIEW_PARAM, r))
+        opts[stage] = opt
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(opts[1].view(what), opts[2].view(what))
+        assert torch.equal(opts[1].view(what), opts[3].view(what))
+    assert torch.equal(opts[1].view(z.ZERO_VIEW_PARAM, 0), opts[3].view(z.ZERO_VIEW_PARAM))
+    assert torch.equal(opts[2].view(z.ZERO_VIEW_GRAD_SHARD), opts[3].view(z.ZERO_VIEW_GRAD_SHARD))
+    o = opts[2]
+    idx = sample_indices(o.offsets(), w.numel, o.psi_pad, o.shard, w.n_ranks, 60_000, intervals=o.buckets())
+    ref = oracle_sampled(w, idx, w.steps)
+    for stage in (1, 2, 3):
+        _sampled_check(opts[stage], w, w.steps, stage, idx, ref)
+    # stage 1 keeps the all-reduced gradient in every replica
+    it = torch.from_numpy(idx).cuda()
+    for r in (0, 7):
+        assert_bits_equal(to_np(opts[1].view(z.ZERO_VIEW_GRAD_BUF, r)[it]), ref["grad"], "stage 1 grads")
+    for o in opts.values():
+        o.close()
+
+
+def test_transformer_1p2b_n8_zero2_bucket200m():
+    """24 layers, hidden 2048 (1,208,598,528 params), N = 8, ZeRO-2 through
+    the fixed 200M-element buffer, 3 steps: sampled elements against the
+    oracle, and the resident-replica step (the bench's launch configuration)
+    equal bit for bit on the device."""
+    z = _z()
+    w = W.gpt_1p2b_n8()
+    opt, fill = make_opt(w, 2, bucket=w.bucket_elems)
+    assert len(opt.buckets()) == 7
+    gfn = grad_fn_for(opt, fill)
+    norms = []
+    for t in range(1, w.steps + 1):
+        norms.append(opt.step(gfn, stats=True))
+    idx = sample_indices(opt.offsets(), w.numel, opt.psi_pad, opt.shard, w.n_ranks, 40_000,
+                         intervals=opt.buckets())
+    ref = oracle_sampled(w, idx, w.steps)
+    _sampled_check(opt, w, w.steps, 2, idx, ref)
+    keep = {what: opt.view(what).clone() for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ)}
+    keep["p0"] = opt.view(z.ZERO_VIEW_PARAM, 0).clone()
+    opt.close()
+    del opt
+    gc.collect()
+    torch.cuda.empty_cache()
+    # resident replicas, no keep of the grad shard: the bench configuration
+    res, rfill = make_opt(w, 2, bucket=w.bucket_elems, keep=False)
+    reps = torch.empty((w.n_ranks, res.psi_pad), dtype=torch.int16, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    for t in range(1, w.steps + 1):
+        for r in range(w.n_ranks):
+            rfill.grads_into(t, r, 0, res.psi_pad, reps[r].data_ptr(), reps[r], s)
+        st = res.step_resident(list(reps), stats=True)
+        assert st["grad_norm"] == norms[t - 1]["grad_norm"] or math.isclose(
+            st["grad_norm"], norms[t - 1]["grad_norm"], rel_tol=1e-12)
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(res.view(what), keep[what])
+    for r in range(w.n_ranks):
+        assert torch.equal(res.view(z.ZERO_VIEW_PARAM, r), keep["p0"])
+    res.close()
+    del reps, keep
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def test_transformer_6p4b_n64_zero3_one_layer_live():
+    """32 layers, hidden 4096 (6,444,154,880 params), N = 64, ZeRO-3 with one
+    layer's 64 gradient replicas and 64 temporary gathered layers live, 2
+    steps: every gathered layer equals the updated shards on every rank, and
+    sampled elements match the oracle."""
+    z = _z()
+    w = W.gpt_6p4b_n64()
+    free, _ = torch.cuda.mem_get_info()
+    opt_need = 12 * 6_444_154_880 + 2 * 6_444_154_880 + 4 * 64 * 201_379_840
+    if free < opt_need + (4 << 30):
+        pytest.skip(f"needs {opt_need / 1e9:.0f} GB free, have {free / 1e9:.0f} GB")
+    opt, fill = make_opt(w, 3, keep=False)
+    assert opt.sizes.max_layer == 201_379_840
+    ok = []
+
+    def gather(layer, lo, hi, bufs, stream):
+        shard = opt.view(z.ZERO_VIEW_PARAM)[lo:hi]
+        ok.append(all(torch.equal(opt._tensor_at(b, hi - lo, torch.int16), shard) for b in bufs))
+        return 0
+
+    gfn = grad_fn_for(opt, fill)
+    for t in range(1, w.steps + 1):
+        opt.step(gfn, gather)
+    assert len(ok) == 32 * w.steps and all(ok)
+    idx = sample_indices(opt.offsets(), w.numel, opt.psi_pad, opt.shard, w.n_ranks, 20_000,
+                         intervals=[(lo, hi) for _, lo, hi in opt.layers()])
+    ref = oracle_sampled(w, idx, w.steps)
+    it = torch.from_numpy(idx).cuda()
+    for name, what in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(opt.view(what)[it]), ref[name], f"6.4B {name}")
+    assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM)[it]), ref["params"], "6.4B param shards")
+    opt.close()
+    del opt
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+SWEEP_SMALL = [(e, n) for e in (1024, 16384, 262144) for n in W.SWEEP_RANKS]
+
+
+@pytest.mark.parametrize("elems,n_ranks", SWEEP_SMALL)
+def test_flat_sweep_cells_every_element(elems, n_ranks):
+    """Flat-buffer sweep cells (U(-1e-2, 1e-2) grads, one bucket), every element."""
+    w = W.flat_sweep(elems, n_ranks)
+    _check_against_oracle(w, 2, None)
+
+
+@pytest.mark.parametrize("elems,n_ranks", [(1 << 30, 2), (1 << 28, 16), (1 << 26, 64), (1 << 24, 8)])
+def test_flat_sweep_large_cells_fused_equals_unfused_and_oracle_samples(elems, n_ranks):
+    z = _z()
+    w = W.flat_sweep(elems, n_ranks)
+    fused, ff = make_opt(w, 2, keep=False)
+    s = torch.cuda.current_stream().cuda_stream
+    reps = torch.empty((n_ranks, fused.psi_pad), dtype=torch.int16, device="cuda")
+    for r in range(n_ranks):
+        ff.grads_into(1, r, 0, fused.psi_pad, reps[r].data_ptr(), reps[r], s)
+    fused.step_resident(list(reps))
+    idx = sample_indices(fused.offsets(), w.numel, fused.psi_pad, fused.shard, n_ranks, 20_000)
+    ref = oracle_sampled(w, idx, 1)
+    it = torch.from_numpy(idx).cuda()
+    assert_bits_equal(to_np(fused.view(z.ZERO_VIEW_MASTER)[it]), ref["master"], "sweep master")
+    assert_bits_equal(to_np(fused.view(z.ZERO_VIEW_PARAM, n_ranks - 1)[it]), ref["params"], "sweep params")
+    keep = fused.view(z.ZERO_VIEW_MASTER).clone()
+    p_last = fused.view(z.ZERO_VIEW_PARAM, n_ranks - 1).clone()
+    fused.close()
+    del fused
+    split, sf = make_opt(w, 2, keep=True)
+    split.reduce_scatter(0, split.psi_pad, [reps[r].data_ptr() for r in range(n_ranks)])
+    split.adam_shard(-1, 1)
+    split.all_gather(0, split.psi_pad)
+    assert torch.equal(split.view(z.ZERO_VIEW_MASTER), keep)
+    assert torch.equal(split.view(z.ZERO_VIEW_PARAM, n_ranks - 1), p_last)
+    split.close()
+    del split, reps, keep, p_last
+    gc.collect()
+    torch.cuda.empty_cache()

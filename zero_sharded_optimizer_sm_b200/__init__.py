@@ -1,0 +1,393 @@
+"""B200 (sm_100a) ZeRO optimizer step over N logical data-parallel ranks.
+
+The compute lives in ``libzero_sm.so`` (hand-written CUDA behind a C ABI,
+declared in ``include/zero_sm.h``).  This module only marshals arguments:
+
+* the raw C functions, under their C names (``zero_init``, ``zero_step``, ...),
+  loaded with ctypes;
+* ``ZeroOptimizer``, which sizes and allocates the arenas with torch (device
+  memory is torch's; the library never allocates), binds them, and exposes
+  the entry points with tensors and Python callables.
+
+Importing raises if the native library is missing: there is no CPU or
+PyTorch fallback for any step of the path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Callable, List, Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzero_sm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                      "(the ZeRO step has no fallback implementation)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+# ------------------------------------------------------------------ C ABI ----
+
+ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ENOTIMPL = range(6)
+STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_EINVAL", 2: "ZERO_ENOMEM", 3: "ZERO_ECUDA", 4: "ZERO_ESTATE",
+                5: "ZERO_ENOTIMPL"}
+ZERO_STAGE_DP, ZERO_STAGE_1, ZERO_STAGE_2, ZERO_STAGE_3 = 0, 1, 2, 3
+ZERO_MAX_RANKS = 128
+(ZERO_ARENA_STATES, ZERO_ARENA_PARAMS, ZERO_ARENA_GRADS, ZERO_ARENA_GRAD_SHARDS, ZERO_ARENA_GATHER,
+ ZERO_ARENA_SCRATCH, ZERO_NUM_ARENAS) = range(7)
+ZERO_OPT_KEEP_GRAD_SHARDS, ZERO_OPT_REPLICA_PAD, ZERO_OPT_BLOCKS_PER_SM, ZERO_OPT_TIMING = 1, 2, 3, 4
+(ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
+ ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
+
+
+class zero_layout(ctypes.Structure):
+    _fields_ = [("n_tensors", ctypes.c_int32), ("numel", ctypes.POINTER(ctypes.c_int64)),
+                ("layer_id", ctypes.POINTER(ctypes.c_int32))]
+
+
+class zero_adam_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double)]
+
+
+class zero_sizes(ctypes.Structure):
+    _fields_ = [("psi", ctypes.c_int64), ("psi_pad", ctypes.c_int64), ("shard", ctypes.c_int64),
+                ("max_layer", ctypes.c_int64), ("replica_pitch", ctypes.c_int64),
+                ("n_buckets", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("arena_bytes", ctypes.c_int64 * ZERO_NUM_ARENAS)]
+
+
+class zero_step_stats(ctypes.Structure):
+    _fields_ = [("grad_norm", ctypes.c_double), ("nonfinite", ctypes.c_int64), ("step", ctypes.c_int64),
+                ("comm_elems", ctypes.c_int64 * 3)]
+
+
+zero_grad_fn = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                ctypes.c_int64, ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p)
+zero_gather_fn = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64,
+                                  ctypes.c_int64, ctypes.POINTER(ctypes.c_void_p), ctypes.c_void_p)
+
+_vp, _i32, _i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+_PTRS = ctypes.POINTER(ctypes.c_void_p)
+_SIGS = {
+    "zero_version": (_i32, []),
+    "zero_init": (_i32, [ctypes.POINTER(zero_layout), _i32, _i32, _i64, ctypes.POINTER(_vp)]),
+    "zero_set_option": (_i32, [_vp, _i32, _i64]),
+    "zero_buffer_sizes": (_i32, [_vp, ctypes.POINTER(zero_sizes)]),
+    "zero_tensor_offsets": (_i32, [_vp, ctypes.POINTER(_i64), _i32]),
+    "zero_buckets": (_i32, [_vp, ctypes.POINTER(_i64), _i32, ctypes.POINTER(_i32)]),
+    "zero_layers": (_i32, [_vp, ctypes.POINTER(_i64), _i32, ctypes.POINTER(_i32)]),
+    "zero_bind": (_i32, [_vp, _PTRS]),
+    "zero_set_hparams": (_i32, [_vp, ctypes.POINTER(zero_adam_hparams)]),
+    "zero_load_master": (_i32, [_vp, _vp, _vp]),
+    "zero_get_step": (_i32, [_vp, ctypes.POINTER(_i64)]),
+    "zero_set_step": (_i32, [_vp, _i64]),
+    "zero_view": (_i32, [_vp, _i32, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
+    "zero_state_bytes": (_i32, [_vp, _i32, ctypes.POINTER(_i64)]),
+    "zero_comm_elems": (_i32, [_vp, ctypes.POINTER(_i64)]),
+    "zero_reduce_scatter": (_i32, [_vp, _i64, _i64, _PTRS, _vp]),
+    "zero_all_reduce": (_i32, [_vp, _i64, _i64, _PTRS, _vp]),
+    "zero_adam_shard": (_i32, [_vp, _i32, _i64, _vp]),
+    "zero_all_gather": (_i32, [_vp, _i64, _i64, _PTRS, _vp]),
+    "zero_step": (_i32, [_vp, zero_grad_fn, _vp, zero_gather_fn, _vp, _vp,
+                         ctypes.POINTER(zero_step_stats)]),
+    "zero_step_resident": (_i32, [_vp, _PTRS, zero_gather_fn, _vp, _vp,
+                                  ctypes.POINTER(zero_step_stats)]),
+    "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
+                                  ctypes.POINTER(ctypes.c_double)]),
+    "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
+    "zero_last_error": (ctypes.c_char_p, [_vp]),
+    "zero_destroy": (None, [_vp]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+    globals()[_name] = _fn
+
+__all__ = list(_SIGS) + ["ZeroOptimizer", "AdamHParams", "ZeroError", "lib", "LIB_PATH"]
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _ptr_array(ptrs: Sequence[int]):
+    arr = (ctypes.c_void_p * len(ptrs))()
+    for i, p in enumerate(ptrs):
+        arr[i] = int(p)
+    return arr
+
+
+# ------------------------------------------------------------ Python API ----
+
+@dataclass(frozen=True)
+class AdamHParams:
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.999
+    eps: float = 1e-8
+    weight_decay: float = 0.0
+
+
+class ZeroOptimizer:
+    """One ZeRO context over ``n_ranks`` logical ranks on the current CUDA device.
+
+    ``numel``/``layer_id``: the parameter list (flat order, non-decreasing
+    layer ids).  ``bucket_elems`` defaults to one bucket spanning everything.
+    Arenas are torch uint8 tensors owned by this object.
+    """
+
+    def __init__(self, numel: Sequence[int], layer_id: Sequence[int], n_ranks: int, stage: int,
+                 bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
+                 keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
+                 device=None):
+        import torch
+
+        self._torch = torch
+        self.n_ranks, self.stage = int(n_ranks), int(stage)
+        n = len(numel)
+        self._numel = (ctypes.c_int64 * n)(*[int(x) for x in numel])
+        self._layer = (ctypes.c_int32 * n)(*[int(x) for x in layer_id])
+        lay = zero_layout(n, self._numel, self._layer)
+        if bucket_elems is None:
+            total = 0
+            for x in numel:
+                total = (total + int(x) + 7) // 8 * 8
+            bucket_elems = max(8, (total + 8 * n_ranks - 1) // (8 * n_ranks) * 8 * n_ranks)
+        self.bucket_elems = int(bucket_elems)
+        ctx = ctypes.c_void_p()
+        st = zero_init(ctypes.byref(lay), self.n_ranks, self.stage, self.bucket_elems, ctypes.byref(ctx))
+        if st != ZERO_OK:
+            raise ZeroError(st, "zero_init", zero_last_error(None).decode())
+        self.ctx = ctx
+        if not keep_grad_shards:
+            self._check(zero_set_option(ctx, ZERO_OPT_KEEP_GRAD_SHARDS, 0), "zero_set_option")
+        if replica_pad:
+            self._check(zero_set_option(ctx, ZERO_OPT_REPLICA_PAD, int(replica_pad)), "zero_set_option")
+        if blocks_per_sm:
+            self._check(zero_set_option(ctx, ZERO_OPT_BLOCKS_PER_SM, int(blocks_per_sm)), "zero_set_option")
+        self.sizes = zero_sizes()
+        self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.device = dev
+        self.arenas = []
+        ptrs = (ctypes.c_void_p * ZERO_NUM_ARENAS)()
+        for k in range(ZERO_NUM_ARENAS):
+            nb = int(self.sizes.arena_bytes[k])
+            t = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+            self.arenas.append(t)
+            ptrs[k] = t.data_ptr() if t is not None else None
+        with torch.cuda.device(dev):
+            self._check(zero_bind(ctx, ptrs), "zero_bind")
+        self.set_hparams(hparams)
+        self._keep = []  # callbacks alive during a call
+
+    # -- plumbing --
+    def _check(self, st: int, where: str):
+        if st != ZERO_OK:
+            raise ZeroError(st, where, zero_last_error(self.ctx).decode())
+
+    def _stream(self, stream=None) -> int:
+        if stream is None:
+            return self._torch.cuda.current_stream(self.device).cuda_stream
+        return int(getattr(stream, "cuda_stream", stream))
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            zero_destroy(self.ctx)
+            self.ctx = None
+            self.arenas = []
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- plan --
+    @property
+    def psi(self) -> int:
+        return int(self.sizes.psi)
+
+    @property
+    def psi_pad(self) -> int:
+        return int(self.sizes.psi_pad)
+
+    @property
+    def shard(self) -> int:
+        return int(self.sizes.shard)
+
+    def offsets(self) -> List[int]:
+        n = len(self._numel)
+        out = (ctypes.c_int64 * n)()
+        self._check(zero_tensor_offsets(self.ctx, out, n), "zero_tensor_offsets")
+        return list(out)
+
+    def buckets(self) -> List[tuple]:
+        n = ctypes.c_int32()
+        self._check(zero_buckets(self.ctx, None, 0, ctypes.byref(n)), "zero_buckets")
+        out = (ctypes.c_int64 * (2 * n.value))()
+        self._check(zero_buckets(self.ctx, out, n.value, ctypes.byref(n)), "zero_buckets")
+        return [(out[2 * k], out[2 * k + 1]) for k in range(n.value)]
+
+    def layers(self) -> List[tuple]:
+        n = ctypes.c_int32()
+        self._check(zero_layers(self.ctx, None, 0, ctypes.byref(n)), "zero_layers")
+        out = (ctypes.c_int64 * (3 * n.value))()
+        self._check(zero_layers(self.ctx, out, n.value, ctypes.byref(n)), "zero_layers")
+        return [(int(out[3 * k]), out[3 * k + 1], out[3 * k + 2]) for k in range(n.value)]
+
+    def state_bytes(self, rank: int) -> tuple:
+        out = (ctypes.c_int64 * 3)()
+        self._check(zero_state_bytes(self.ctx, rank, out), "zero_state_bytes")
+        return tuple(out)
+
+    def comm_elems(self) -> tuple:
+        out = (ctypes.c_int64 * 3)()
+        self._check(zero_comm_elems(self.ctx, out), "zero_comm_elems")
+        return tuple(out)
+
+    # -- views --
+    def _tensor_at(self, ptr: int, n: int, dtype):
+        torch = self._torch
+        esize = torch.empty((), dtype=dtype).element_size()
+        for a in self.arenas:
+            if a is None:
+                continue
+            base = a.data_ptr()
+            if base <= ptr and ptr + n * esize <= base + a.numel():
+                off = ptr - base
+                return a[off:off + n * esize].view(dtype)
+        raise ValueError("pointer outside the bound arenas")
+
+    def view(self, what: int, rank: int = 0):
+        """torch view (uint16 for bf16 patterns, float32 for states) of a buffer."""
+        torch = self._torch
+        p = ctypes.c_void_p()
+        n = ctypes.c_int64()
+        self._check(zero_view(self.ctx, what, rank, ctypes.byref(p), ctypes.byref(n)), "zero_view")
+        dtype = torch.float32 if what in (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ) else torch.int16
+        return self._tensor_at(p.value, n.value, dtype)
+
+    # -- state --
+    def set_hparams(self, hp: AdamHParams):
+        h = zero_adam_hparams(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay)
+        self._check(zero_set_hparams(self.ctx, ctypes.byref(h)), "zero_set_hparams")
+        self.hparams = hp
+
+    def load_master(self, master=None, stream=None):
+        """master: float32 CUDA tensor of psi_pad values, or None when the
+        master view has been written in place."""
+        ptr = None if master is None else master.data_ptr()
+        if master is not None:
+            assert master.dtype == self._torch.float32 and master.is_cuda and master.numel() == self.psi_pad
+        self._check(zero_load_master(self.ctx, ptr, self._stream(stream)), "zero_load_master")
+
+    @property
+    def t(self) -> int:
+        v = ctypes.c_int64()
+        self._check(zero_get_step(self.ctx, ctypes.byref(v)), "zero_get_step")
+        return v.value
+
+    @t.setter
+    def t(self, value: int):
+        self._check(zero_set_step(self.ctx, int(value)), "zero_set_step")
+
+    # -- the step --
+    @staticmethod
+    def _stats_dict(s: zero_step_stats) -> dict:
+        return dict(grad_norm=s.grad_norm, nonfinite=int(s.nonfinite), step=int(s.step),
+                    comm_elems=tuple(s.comm_elems))
+
+    def _wrap_gather(self, gather_fn):
+        if gather_fn is None:
+            return zero_gather_fn()
+
+        def cb(user, layer, lo, hi, bufs, stream):
+            try:
+                r = gather_fn(int(layer), int(lo), int(hi), [bufs[i] for i in range(self.n_ranks)], stream)
+                return int(r or 0)
+            except Exception as exc:  # a Python error must not unwind through C
+                self._cb_error = exc
+                return 1
+
+        return zero_gather_fn(cb)
+
+    def step(self, grad_fn: Optional[Callable] = None, gather_fn: Optional[Callable] = None,
+             stats: bool = False, stream=None):
+        """grad_fn(step, lo, hi, rank_buf_ptrs, stream) fills the ranks' buffers;
+        gather_fn(layer, lo, hi, rank_buf_ptrs, stream) consumes a stage-3
+        gathered layer.  Returns the statistics dict when ``stats``."""
+        self._cb_error = None
+        if grad_fn is None:
+            gcb = zero_grad_fn()
+        else:
+            def g(user, t, lo, hi, bufs, stream_):
+                try:
+                    r = grad_fn(int(t), int(lo), int(hi), [bufs[i] for i in range(self.n_ranks)], stream_)
+                    return int(r or 0)
+                except Exception as exc:
+                    self._cb_error = exc
+                    return 1
+            gcb = zero_grad_fn(g)
+        acb = self._wrap_gather(gather_fn)
+        out = zero_step_stats()
+        st = zero_step(self.ctx, gcb, None, acb, None, self._stream(stream),
+                       ctypes.byref(out) if stats else None)
+        if self._cb_error is not None:
+            raise self._cb_error
+        self._check(st, "zero_step")
+        return self._stats_dict(out) if stats else None
+
+    def step_resident(self, rank_grads, gather_fn: Optional[Callable] = None, stats: bool = False,
+                      stream=None):
+        """rank_grads: N CUDA tensors (or one [N, psi_pad] tensor) of bf16 patterns."""
+        ptrs = _ptr_array([g.data_ptr() for g in rank_grads])
+        self._cb_error = None
+        acb = self._wrap_gather(gather_fn)
+        out = zero_step_stats()
+        st = zero_step_resident(self.ctx, ptrs, acb, None, self._stream(stream),
+                                ctypes.byref(out) if stats else None)
+        if self._cb_error is not None:
+            raise self._cb_error
+        self._check(st, "zero_step_resident")
+        return self._stats_dict(out) if stats else None
+
+    def set_timing(self, on: bool):
+        self._check(zero_set_option(self.ctx, ZERO_OPT_TIMING, 1 if on else 0), "zero_set_option")
+
+    def kernel_timing(self) -> dict:
+        """Fused-kernel launches recorded since the last call: device ms,
+        launch count, modelled bytes."""
+        ms = ctypes.c_double()
+        n = ctypes.c_int64()
+        b = ctypes.c_double()
+        self._check(zero_kernel_timing(self.ctx, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(b)),
+                    "zero_kernel_timing")
+        return dict(ms=ms.value, launches=n.value, model_bytes=b.value)
+
+    def read_stats(self, stream=None) -> dict:
+        out = zero_step_stats()
+        self._check(zero_read_stats(self.ctx, self._stream(stream), ctypes.byref(out)), "zero_read_stats")
+        return self._stats_dict(out)
+
+    # -- unfused parts --
+    def reduce_scatter(self, lo: int, hi: int, rank_grads: Optional[Sequence[int]] = None, stream=None):
+        ptrs = None if rank_grads is None else _ptr_array(rank_grads)
+        self._check(zero_reduce_scatter(self.ctx, lo, hi, ptrs, self._stream(stream)), "zero_reduce_scatter")
+
+    def all_reduce(self, lo: int, hi: int, rank_grads: Optional[Sequence[int]] = None, stream=None):
+        ptrs = None if rank_grads is None else _ptr_array(rank_grads)
+        self._check(zero_all_reduce(self.ctx, lo, hi, ptrs, self._stream(stream)), "zero_all_reduce")
+
+    def adam_shard(self, rank: int, t: int, stream=None):
+        self._check(zero_adam_shard(self.ctx, rank, t, self._stream(stream)), "zero_adam_shard")
+
+    def all_gather(self, lo: int, hi: int, rank_out: Optional[Sequence[int]] = None, stream=None):
+        ptrs = None if rank_out is None else _ptr_array(rank_out)
+        self._check(zero_all_gather(self.ctx, lo, hi, ptrs, self._stream(stream)), "zero_all_gather")

@@ -1,0 +1,103 @@
+// Device kernels of the ZeRO optimizer step and their launch arguments.
+//
+// All kernels are memory-bound streams over 16-byte vectors of 8 bf16 (or two
+// float4 of fp32) elements: one lane owns 8 consecutive flat elements per
+// iteration of a grid-stride loop sized to the SM count.  Nothing here is a
+// contraction, so no tensor core is involved.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace zsm {
+
+constexpr int kMaxRanks = 128;   // mirrors ZERO_MAX_RANKS
+constexpr int kVec = 8;          // bf16 elements per 16-byte vector
+constexpr int kThreads = 256;    // threads per CTA for every kernel
+constexpr int kMaxGrid = 4096;   // upper bound on CTAs of a norm-reducing launch
+
+// Binary32 scalars of one Adam step, each rounded once from binary64 on the host.
+struct AdamScalars {
+  float b1, b2, omb1, omb2, bc1, bc2, decay, lr, eps;
+};
+
+// Gradient-norm / non-finite accumulation in the scratch arena.
+struct NormScratch {
+  double* partial_sq;              // [kMaxGrid] per-CTA partial sums of g^2
+  unsigned long long* partial_nf;  // [kMaxGrid] per-CTA non-finite counts
+  unsigned int* done;              // CTAs of the current launch that finished
+  double* step_sq;                 // sum over the launches of the current step
+  unsigned long long* step_nf;
+};
+
+// Fused reduce + Adam + broadcast over one interval [lo, hi) of the flat space.
+// Every pointer is already offset to flat element lo of its buffer.
+struct FusedArgs {
+  const uint16_t* grad[kMaxRanks];  // rank r's bf16 gradient (stage 1: written back)
+  uint16_t* out[kMaxRanks];         // rank r's bf16 parameter destination
+  float* master;
+  float* m;
+  float* v;
+  uint16_t* grad_shard;             // reduced bf16 gradient, or nullptr
+  uint16_t* param_shard;            // stage 3 bf16 parameter shard, or nullptr
+  int64_t n_vec;                    // (hi - lo) / 8
+  int n_ranks;
+  int accumulate;                   // 0: first launch of the step (norm overwrites)
+  float inv_n;                      // binary32 1/N
+  AdamScalars sc;
+  NormScratch ns;
+};
+
+// Reduce only (reduce-scatter to a shard, or all-reduce written back).
+struct ReduceArgs {
+  const uint16_t* grad[kMaxRanks];
+  uint16_t* shard_out;              // reduce-scatter destination, or nullptr
+  int64_t n_vec;
+  int n_ranks;
+  int accumulate;
+  int write_back;                   // all-reduce: write the mean to every grad[r]
+  float inv_n;
+  NormScratch ns;
+};
+
+struct AdamArgs {
+  const uint16_t* grad;
+  float* master;
+  float* m;
+  float* v;
+  uint16_t* out;
+  int64_t n_vec;
+  AdamScalars sc;
+};
+
+struct GatherArgs {
+  const uint16_t* src;
+  uint16_t* out[kMaxRanks];
+  int64_t n_vec;
+  int n_out;
+};
+
+struct InitArgs {
+  const float* master_src;
+  float* master;
+  float* m;
+  float* v;
+  uint16_t* out[kMaxRanks];         // bf16(master) destinations, each at element 0
+  int n_out;
+  uint16_t* grad_shard;             // zeroed when not null
+  int64_t n_vec;
+};
+
+enum FusedMode { kFusedZ1 = 1, kFusedZ2 = 2, kFusedZ3 = 3 };
+
+// Launchers (return the launch's cudaError_t).
+cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
+
+// Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.
+cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_blocks);
+
+}  // namespace zsm

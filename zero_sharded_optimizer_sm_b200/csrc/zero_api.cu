@@ -1,0 +1,786 @@
+// C ABI of the ZeRO optimizer-step library: validation, arena layout and the
+// executor that sequences the kernels of each stage.  Declarations and the
+// contract of every entry point are in include/zero_sm.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "zero_sm.h"
+#include "kernels.cuh"
+#include "plan.hpp"
+
+static_assert(ZERO_MAX_RANKS == zsm::kMaxRanks, "rank limit mismatch");
+
+namespace {
+
+thread_local std::string g_init_error;
+
+constexpr int64_t kArenaAlign = 256;
+constexpr int64_t kScratchBytes = 80 * 1024;
+
+int64_t align_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
+
+}  // namespace
+
+struct zero_ctx {
+  zsm::Plan plan;
+  int32_t stage = 0;
+  // options
+  bool keep_grad_shards = true;
+  int64_t replica_pad = 0;
+  int blocks_per_sm_opt = 0;
+  // arena layout (bytes)
+  int64_t arena_bytes[ZERO_NUM_ARENAS] = {};
+  int64_t state_pitch = 0;   // bytes between master, m and v
+  int64_t param_pitch = 0;   // bytes between parameter replicas (stage 1, 2)
+  int64_t grad_pitch = 0;    // bytes between gradient buffers
+  int64_t gather_pitch = 0;  // bytes between temporary layer buffers (stage 3)
+  // binding
+  bool bound = false;
+  char* arena[ZERO_NUM_ARENAS] = {};
+  int sm_count = 0;
+  int grid_fused = 0;
+  int grid_simple = 0;
+  // run state
+  bool have_hp = false;
+  zero_adam_hparams hp{};
+  bool loaded = false;
+  int64_t t = 0;
+  int64_t stats_step = 0;
+  bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
+  // fused-kernel timing
+  bool timing = false;
+  std::vector<cudaEvent_t> events;  // pairs (start, end), reused
+  size_t timed = 0;                 // pairs recorded since the last read
+  double timed_bytes = 0.0;
+  std::string err;
+  ~zero_ctx() {
+    for (cudaEvent_t e : events) cudaEventDestroy(e);
+  }
+};
+
+namespace {
+
+zero_status fail(zero_ctx* c, zero_status s, const char* fmt, ...) {
+  if (c) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    c->err = buf;
+  }
+  return s;
+}
+
+zero_status cuda_fail(zero_ctx* c, cudaError_t e, const char* what) {
+  return fail(c, ZERO_ECUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+void compute_layout(zero_ctx* c) {
+  const zsm::Plan& p = c->plan;
+  const int64_t N = p.n_ranks;
+  const int64_t row2 = align_up(p.psi_pad * 2, kArenaAlign);
+  c->state_pitch = align_up(p.psi_pad * 4, kArenaAlign);
+  c->param_pitch = row2 + c->replica_pad;
+  std::fill(c->arena_bytes, c->arena_bytes + ZERO_NUM_ARENAS, 0);
+  c->arena_bytes[ZERO_ARENA_STATES] = 3 * c->state_pitch;
+  c->arena_bytes[ZERO_ARENA_SCRATCH] = kScratchBytes;
+  switch (c->stage) {
+    case ZERO_STAGE_1:
+      c->grad_pitch = c->param_pitch;
+      c->arena_bytes[ZERO_ARENA_PARAMS] = N * c->param_pitch;
+      c->arena_bytes[ZERO_ARENA_GRADS] = N * c->grad_pitch;
+      break;
+    case ZERO_STAGE_2:
+      c->grad_pitch = align_up(p.max_bucket * 2, kArenaAlign) + c->replica_pad;
+      c->arena_bytes[ZERO_ARENA_PARAMS] = N * c->param_pitch;
+      c->arena_bytes[ZERO_ARENA_GRADS] = N * c->grad_pitch;
+      c->arena_bytes[ZERO_ARENA_GRAD_SHARDS] = c->keep_grad_shards ? row2 : 0;
+      break;
+    case ZERO_STAGE_3:
+      c->param_pitch = row2;
+      c->grad_pitch = align_up(p.max_layer * 2, kArenaAlign) + c->replica_pad;
+      c->gather_pitch = c->grad_pitch;
+      c->arena_bytes[ZERO_ARENA_PARAMS] = row2;
+      c->arena_bytes[ZERO_ARENA_GRADS] = N * c->grad_pitch;
+      c->arena_bytes[ZERO_ARENA_GRAD_SHARDS] = c->keep_grad_shards ? row2 : 0;
+      c->arena_bytes[ZERO_ARENA_GATHER] = N * c->gather_pitch;
+      break;
+  }
+}
+
+float* master_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_STATES]); }
+float* m_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_STATES] + c->state_pitch); }
+float* v_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_STATES] + 2 * c->state_pitch); }
+uint16_t* param_ptr(zero_ctx* c, int r) {  // replica r (stage 1, 2) or the shards (stage 3)
+  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_PARAMS] + (c->stage == ZERO_STAGE_3 ? 0 : r * c->param_pitch));
+}
+uint16_t* grad_buf_ptr(zero_ctx* c, int r) {
+  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GRADS] + r * c->grad_pitch);
+}
+uint16_t* grad_shard_ptr(zero_ctx* c) { return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GRAD_SHARDS]); }
+uint16_t* gather_ptr(zero_ctx* c, int r) {
+  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GATHER] + r * c->gather_pitch);
+}
+
+zsm::NormScratch norm_scratch(zero_ctx* c) {
+  char* s = c->arena[ZERO_ARENA_SCRATCH];
+  zsm::NormScratch ns;
+  ns.partial_sq = reinterpret_cast<double*>(s);
+  ns.partial_nf = reinterpret_cast<unsigned long long*>(s + 8 * zsm::kMaxGrid);
+  ns.step_sq = reinterpret_cast<double*>(s + 16 * zsm::kMaxGrid);
+  ns.step_nf = reinterpret_cast<unsigned long long*>(s + 16 * zsm::kMaxGrid + 8);
+  ns.done = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 16);
+  return ns;
+}
+
+zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
+  double p1 = 1.0, p2 = 1.0;
+  for (int64_t k = 0; k < t; ++k) {
+    p1 *= hp.beta1;
+    p2 *= hp.beta2;
+  }
+  zsm::AdamScalars s;
+  s.b1 = (float)hp.beta1;
+  s.b2 = (float)hp.beta2;
+  s.omb1 = (float)(1.0 - hp.beta1);
+  s.omb2 = (float)(1.0 - hp.beta2);
+  s.bc1 = (float)(1.0 - p1);
+  s.bc2 = (float)(1.0 - p2);
+  s.decay = (float)(1.0 - hp.lr * hp.weight_decay);
+  s.lr = (float)hp.lr;
+  s.eps = (float)hp.eps;
+  return s;
+}
+
+constexpr size_t kMaxTimed = 4096;
+
+// Bytes one element moves through HBM in the fused step (the byte model).
+int64_t fused_bytes_per_elem(const zero_ctx* c) {
+  const int64_t N = c->plan.n_ranks;
+  const int64_t keep = c->arena[ZERO_ARENA_GRAD_SHARDS] ? 2 : 0;
+  if (c->stage == ZERO_STAGE_1) return 6 * N + 24;
+  if (c->stage == ZERO_STAGE_2) return 4 * N + 24 + keep;
+  return 4 * N + 26 + keep;
+}
+
+// Event pair for the next timed launch, or nullptr when the record is full.
+cudaEvent_t* timing_pair(zero_ctx* c) {
+  if (c->timed >= kMaxTimed) return nullptr;
+  while (c->events.size() < 2 * (c->timed + 1)) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    c->events.push_back(e);
+  }
+  return &c->events[2 * c->timed];
+}
+
+int grid_for(int64_t n_vec, int cap) {
+  const int64_t want = (n_vec + zsm::kThreads - 1) / zsm::kThreads;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(want, cap));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+zero_status check_interval(zero_ctx* c, int64_t lo, int64_t hi) {
+  if (lo < 0 || hi < lo || hi > c->plan.psi_pad || lo % zsm::kGranule || hi % zsm::kGranule)
+    return fail(c, ZERO_EINVAL, "interval [%lld, %lld) must satisfy 0 <= lo <= hi <= psi_pad=%lld, both multiples of 8",
+                (long long)lo, (long long)hi, (long long)c->plan.psi_pad);
+  return ZERO_OK;
+}
+
+zero_status check_ready(zero_ctx* c, bool need_hp) {
+  if (!c) return ZERO_EINVAL;
+  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
+  if (!c->loaded) return fail(c, ZERO_ESTATE, "state is not initialised (zero_load_master)");
+  if (need_hp && !c->have_hp) return fail(c, ZERO_ESTATE, "hyper-parameters are not set (zero_set_hparams)");
+  return ZERO_OK;
+}
+
+// Which flat ranges a stage's step walks: the bucket schedule (stage 1, 2) or
+// the layers from last to first (stage 3).
+std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
+  std::vector<zsm::Span> out;
+  if (c->stage == ZERO_STAGE_3) {
+    for (auto it = c->plan.layers.rbegin(); it != c->plan.layers.rend(); ++it) out.push_back({it->lo, it->hi});
+  } else {
+    out = c->plan.buckets;
+  }
+  return out;
+}
+
+// One fused launch over [lo, hi).  grad[r] are at flat element lo.
+zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
+                           bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s) {
+  if (hi == lo) return ZERO_OK;
+  const int N = c->plan.n_ranks;
+  zsm::FusedArgs a;
+  std::memset(&a, 0, sizeof a);
+  for (int r = 0; r < N; ++r) {
+    a.grad[r] = grad[r];
+    if (c->stage == ZERO_STAGE_3) {
+      const int64_t off = lo - c->plan.layers[layer_idx].lo;
+      a.out[r] = gather_ptr(c, r) + off;
+    } else {
+      a.out[r] = param_ptr(c, r) + lo;
+    }
+  }
+  a.master = master_ptr(c) + lo;
+  a.m = m_ptr(c) + lo;
+  a.v = v_ptr(c) + lo;
+  a.grad_shard = c->arena[ZERO_ARENA_GRAD_SHARDS] ? grad_shard_ptr(c) + lo : nullptr;
+  a.param_shard = c->stage == ZERO_STAGE_3 ? param_ptr(c, 0) + lo : nullptr;
+  a.n_vec = (hi - lo) / zsm::kVec;
+  a.n_ranks = N;
+  a.accumulate = accumulate ? 1 : 0;
+  a.inv_n = (float)(1.0 / (double)N);
+  a.sc = sc;
+  a.ns = norm_scratch(c);
+  const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
+  cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  cudaError_t e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "fused step kernel launch");
+  if (ev) {
+    cudaEventRecord(ev[1], s);
+    c->timed += 1;
+    c->timed_bytes += (double)fused_bytes_per_elem(c) * (double)(hi - lo);
+  }
+  return ZERO_OK;
+}
+
+zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
+  struct {
+    double sq;
+    unsigned long long nf;
+  } host{};
+  zsm::NormScratch ns = norm_scratch(c);
+  cudaError_t e = cudaMemcpyAsync(&host, ns.step_sq, 16, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "reading step statistics");
+  std::memset(out, 0, sizeof *out);
+  out->grad_norm = std::sqrt(host.sq);
+  out->nonfinite = (int64_t)host.nf;
+  out->step = c->stats_step;
+  zero_comm_elems(c, out->comm_elems);
+  return ZERO_OK;
+}
+
+zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
+                     zero_gather_fn gfn, void* guser, void* stream, zero_step_stats* stats) {
+  zero_status st = check_ready(c, true);
+  if (st != ZERO_OK) return st;
+  const int N = c->plan.n_ranks;
+  if (resident) {
+    for (int r = 0; r < N; ++r)
+      if (!resident[r] || !aligned16(resident[r]))
+        return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
+  } else if (!fn && c->stage != ZERO_STAGE_1) {
+    return fail(c, ZERO_EINVAL, "grad_fn may be NULL only for stage 1");
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t t = c->t + 1;
+  const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+  const std::vector<zsm::Span> iv = step_intervals(c);
+  std::vector<uint16_t*> grad(N), bufs(N);
+  const int n_layers = (int)c->plan.layers.size();
+  for (size_t k = 0; k < iv.size(); ++k) {
+    const int64_t lo = iv[k].lo, hi = iv[k].hi;
+    const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
+    if (resident) {
+      for (int r = 0; r < N; ++r)
+        grad[r] = const_cast<uint16_t*>(static_cast<const uint16_t*>(resident[r])) + lo;
+    } else {
+      for (int r = 0; r < N; ++r)
+        bufs[r] = c->stage == ZERO_STAGE_1 ? grad_buf_ptr(c, r) + lo : grad_buf_ptr(c, r);
+      if (fn) {
+        const int rc = fn(user, t, lo, hi, reinterpret_cast<void* const*>(bufs.data()), stream);
+        if (rc != 0) return fail(c, ZERO_EINVAL, "grad_fn returned %d for [%lld, %lld)", rc, (long long)lo, (long long)hi);
+      }
+      grad = bufs;
+    }
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, k > 0, sc, s);
+    if (st != ZERO_OK) return st;
+    if (c->stage == ZERO_STAGE_3 && gfn) {
+      for (int r = 0; r < N; ++r) bufs[r] = gather_ptr(c, r);
+      const int rc = gfn(guser, c->plan.layers[layer_idx].id, lo, hi, reinterpret_cast<void* const*>(bufs.data()), stream);
+      if (rc != 0) return fail(c, ZERO_EINVAL, "gather_fn returned %d for layer %d", rc, c->plan.layers[layer_idx].id);
+    }
+  }
+  c->t = t;
+  c->stats_step = t;
+  c->norm_fresh = true;
+  if (stats) return finish_stats(c, s, stats);
+  return ZERO_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t zero_version(void) { return ZERO_SM_VERSION; }
+
+zero_status zero_init(const zero_layout* layout, int32_t n_ranks, int32_t stage, int64_t bucket_elems,
+                      zero_ctx** out) {
+  g_init_error.clear();
+  if (!out) return g_init_error = "out is NULL", ZERO_EINVAL;
+  *out = nullptr;
+  if (!layout) return g_init_error = "layout is NULL", ZERO_EINVAL;
+  if (n_ranks < 1 || n_ranks > ZERO_MAX_RANKS)
+    return g_init_error = "n_ranks must be 1.." + std::to_string(ZERO_MAX_RANKS), ZERO_EINVAL;
+  if (stage == ZERO_STAGE_DP) return g_init_error = "stage 0 (plain DP) is not provided on the device", ZERO_ENOTIMPL;
+  if (stage < ZERO_STAGE_1 || stage > ZERO_STAGE_3) return g_init_error = "stage must be 1, 2 or 3", ZERO_EINVAL;
+  zero_ctx* c = new (std::nothrow) zero_ctx();
+  if (!c) return g_init_error = "out of host memory", ZERO_ENOMEM;
+  std::string err;
+  if (!zsm::make_plan(layout->n_tensors, layout->numel, layout->layer_id, n_ranks, bucket_elems, &c->plan, &err)) {
+    delete c;
+    g_init_error = err;
+    return ZERO_EINVAL;
+  }
+  c->stage = stage;
+  compute_layout(c);
+  *out = c;
+  return ZERO_OK;
+}
+
+zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
+  if (!c) return ZERO_EINVAL;
+  if (key == ZERO_OPT_TIMING) {
+    c->timing = value != 0;
+    return ZERO_OK;
+  }
+  if (c->bound) return fail(c, ZERO_ESTATE, "options must be set before zero_bind");
+  switch (key) {
+    case ZERO_OPT_KEEP_GRAD_SHARDS:
+      c->keep_grad_shards = value != 0;
+      break;
+    case ZERO_OPT_REPLICA_PAD:
+      if (value < 0 || value % kArenaAlign || value >= (1 << 20))
+        return fail(c, ZERO_EINVAL, "replica pad must be a multiple of 256 below 1 MiB");
+      c->replica_pad = value;
+      break;
+    case ZERO_OPT_BLOCKS_PER_SM:
+      if (value < 0 || value > 32) return fail(c, ZERO_EINVAL, "blocks per SM must be 0..32");
+      c->blocks_per_sm_opt = (int)value;
+      break;
+    default:
+      return fail(c, ZERO_EINVAL, "unknown option %d", key);
+  }
+  compute_layout(c);
+  return ZERO_OK;
+}
+
+zero_status zero_buffer_sizes(const zero_ctx* c, zero_sizes* out) {
+  if (!c || !out) return ZERO_EINVAL;
+  std::memset(out, 0, sizeof *out);
+  out->psi = c->plan.psi;
+  out->psi_pad = c->plan.psi_pad;
+  out->shard = c->plan.shard;
+  out->max_layer = c->plan.max_layer;
+  out->replica_pitch = c->stage == ZERO_STAGE_3 ? c->gather_pitch : c->param_pitch;
+  out->n_buckets = (int32_t)c->plan.buckets.size();
+  out->n_layers = (int32_t)c->plan.layers.size();
+  for (int k = 0; k < ZERO_NUM_ARENAS; ++k) out->arena_bytes[k] = c->arena_bytes[k];
+  return ZERO_OK;
+}
+
+zero_status zero_tensor_offsets(const zero_ctx* c, int64_t* out, int32_t cap) {
+  if (!c || (!out && cap > 0)) return ZERO_EINVAL;
+  const int32_t n = (int32_t)c->plan.start.size();
+  for (int32_t k = 0; k < std::min(n, cap); ++k) out[k] = c->plan.start[k];
+  return cap < n ? ZERO_EINVAL : ZERO_OK;
+}
+
+zero_status zero_buckets(const zero_ctx* c, int64_t* lo_hi, int32_t cap, int32_t* n_out) {
+  if (!c || !n_out || (!lo_hi && cap > 0)) return ZERO_EINVAL;
+  const int32_t n = (int32_t)c->plan.buckets.size();
+  for (int32_t k = 0; k < std::min(n, cap); ++k) {
+    lo_hi[2 * k] = c->plan.buckets[k].lo;
+    lo_hi[2 * k + 1] = c->plan.buckets[k].hi;
+  }
+  *n_out = n;
+  return ZERO_OK;
+}
+
+zero_status zero_layers(const zero_ctx* c, int64_t* id_lo_hi, int32_t cap, int32_t* n_out) {
+  if (!c || !n_out || (!id_lo_hi && cap > 0)) return ZERO_EINVAL;
+  const int32_t n = (int32_t)c->plan.layers.size();
+  for (int32_t k = 0; k < std::min(n, cap); ++k) {
+    id_lo_hi[3 * k] = c->plan.layers[k].id;
+    id_lo_hi[3 * k + 1] = c->plan.layers[k].lo;
+    id_lo_hi[3 * k + 2] = c->plan.layers[k].hi;
+  }
+  *n_out = n;
+  return ZERO_OK;
+}
+
+zero_status zero_bind(zero_ctx* c, void* const* arenas) {
+  if (!c) return ZERO_EINVAL;
+  if (c->bound) return fail(c, ZERO_ESTATE, "arenas are already bound");
+  if (!arenas) return fail(c, ZERO_EINVAL, "arenas is NULL");
+  for (int k = 0; k < ZERO_NUM_ARENAS; ++k) {
+    if (c->arena_bytes[k] == 0) continue;
+    if (!arenas[k]) return fail(c, ZERO_EINVAL, "arena %d (%lld bytes) is NULL", k, (long long)c->arena_bytes[k]);
+    if (reinterpret_cast<uintptr_t>(arenas[k]) % kArenaAlign)
+      return fail(c, ZERO_EINVAL, "arena %d is not 256-byte aligned", k);
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sm_count, cudaDevAttrMultiProcessorCount, dev);
+  int fused_blocks = 0, simple_blocks = 0;
+  const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
+  if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
+  if (e != cudaSuccess) return cuda_fail(c, e, "device query");
+  if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
+  c->grid_fused = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, fused_blocks)));
+  c->grid_simple = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, simple_blocks)));
+  for (int k = 0; k < ZERO_NUM_ARENAS; ++k) c->arena[k] = c->arena_bytes[k] ? static_cast<char*>(arenas[k]) : nullptr;
+  c->bound = true;
+  return ZERO_OK;
+}
+
+zero_status zero_set_hparams(zero_ctx* c, const zero_adam_hparams* hp) {
+  if (!c || !hp) return ZERO_EINVAL;
+  if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
+      !(hp->eps >= 0.0) || !(hp->weight_decay >= 0.0))
+    return fail(c, ZERO_EINVAL, "hyper-parameters out of range (lr, eps, wd >= 0; 0 <= beta < 1)");
+  c->hp = *hp;
+  c->have_hp = true;
+  return ZERO_OK;
+}
+
+zero_status zero_load_master(zero_ctx* c, const float* master_dev, void* stream) {
+  if (!c) return ZERO_EINVAL;
+  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
+  if (master_dev && !aligned16(master_dev)) return fail(c, ZERO_EINVAL, "master_dev is not 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(c->arena[ZERO_ARENA_SCRATCH], 0, kScratchBytes, s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "clearing scratch");
+  zsm::InitArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.master_src = master_dev ? master_dev : master_ptr(c);
+  a.master = master_ptr(c);
+  a.m = m_ptr(c);
+  a.v = v_ptr(c);
+  a.n_out = c->stage == ZERO_STAGE_3 ? 1 : c->plan.n_ranks;
+  for (int r = 0; r < a.n_out; ++r) a.out[r] = param_ptr(c, r);
+  a.grad_shard = c->arena[ZERO_ARENA_GRAD_SHARDS] ? grad_shard_ptr(c) : nullptr;
+  a.n_vec = c->plan.psi_pad / zsm::kVec;
+  e = zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "init kernel launch");
+  c->t = 0;
+  c->stats_step = 0;
+  c->loaded = true;
+  c->norm_fresh = true;
+  return ZERO_OK;
+}
+
+zero_status zero_get_step(const zero_ctx* c, int64_t* t) {
+  if (!c || !t) return ZERO_EINVAL;
+  *t = c->t;
+  return ZERO_OK;
+}
+
+zero_status zero_set_step(zero_ctx* c, int64_t t) {
+  if (!c || t < 0) return ZERO_EINVAL;
+  c->t = t;
+  return ZERO_OK;
+}
+
+zero_status zero_view(const zero_ctx* cc, int32_t what, int32_t rank, void** ptr, int64_t* n_elems) {
+  zero_ctx* c = const_cast<zero_ctx*>(cc);
+  if (!c || !ptr || !n_elems) return ZERO_EINVAL;
+  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
+  const int N = c->plan.n_ranks;
+  const bool per_rank = what == ZERO_VIEW_GRAD_BUF || what == ZERO_VIEW_GATHER ||
+                        (what == ZERO_VIEW_PARAM && c->stage != ZERO_STAGE_3);
+  if (per_rank && (rank < 0 || rank >= N)) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
+  const int64_t P = c->plan.psi_pad;
+  switch (what) {
+    case ZERO_VIEW_MASTER: *ptr = master_ptr(c); *n_elems = P; break;
+    case ZERO_VIEW_EXP_AVG: *ptr = m_ptr(c); *n_elems = P; break;
+    case ZERO_VIEW_EXP_AVG_SQ: *ptr = v_ptr(c); *n_elems = P; break;
+    case ZERO_VIEW_PARAM: *ptr = param_ptr(c, rank); *n_elems = P; break;
+    case ZERO_VIEW_GRAD_SHARD:
+      if (!c->arena[ZERO_ARENA_GRAD_SHARDS]) return fail(c, ZERO_EINVAL, "stage %d has no gradient shards", c->stage);
+      *ptr = grad_shard_ptr(c);
+      *n_elems = P;
+      break;
+    case ZERO_VIEW_GRAD_BUF:
+      *ptr = grad_buf_ptr(c, rank);
+      *n_elems = c->stage == ZERO_STAGE_1 ? P : c->stage == ZERO_STAGE_2 ? c->plan.max_bucket : c->plan.max_layer;
+      break;
+    case ZERO_VIEW_GATHER:
+      if (c->stage != ZERO_STAGE_3) return fail(c, ZERO_EINVAL, "only stage 3 has gather buffers");
+      *ptr = gather_ptr(c, rank);
+      *n_elems = c->plan.max_layer;
+      break;
+    default:
+      return fail(c, ZERO_EINVAL, "unknown view %d", what);
+  }
+  return ZERO_OK;
+}
+
+zero_status zero_state_bytes(const zero_ctx* c, int32_t rank, int64_t out[3]) {
+  if (!c || !out || rank < 0 || rank >= c->plan.n_ranks) return ZERO_EINVAL;
+  const int64_t P = c->plan.psi_pad, S = c->plan.shard;
+  out[0] = 2 * (c->stage == ZERO_STAGE_3 ? S : P);
+  out[1] = 2 * (c->stage == ZERO_STAGE_1 ? P : S);
+  out[2] = 12 * S;
+  return ZERO_OK;
+}
+
+zero_status zero_comm_elems(const zero_ctx* c, int64_t out[3]) {
+  if (!c || !out) return ZERO_EINVAL;
+  const int64_t N = c->plan.n_ranks;
+  const int64_t one = c->plan.psi_pad * (N - 1) / N;
+  out[0] = c->stage == ZERO_STAGE_1 ? 2 * one : 0;
+  out[1] = c->stage == ZERO_STAGE_1 ? 0 : one;
+  out[2] = c->stage == ZERO_STAGE_3 ? 2 * one : one;
+  return ZERO_OK;
+}
+
+zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void* const* rank_grads, void* stream) {
+  zero_status st = check_ready(c, false);
+  if (st != ZERO_OK) return st;
+  if (c->stage == ZERO_STAGE_1) return fail(c, ZERO_EINVAL, "stage 1 keeps full gradients: use zero_all_reduce");
+  if (!c->arena[ZERO_ARENA_GRAD_SHARDS])
+    return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
+  if ((st = check_interval(c, lo, hi)) != ZERO_OK) return st;
+  const int N = c->plan.n_ranks;
+  zsm::ReduceArgs a;
+  std::memset(&a, 0, sizeof a);
+  if (rank_grads) {
+    for (int r = 0; r < N; ++r) {
+      if (!rank_grads[r] || !aligned16(rank_grads[r]))
+        return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
+      a.grad[r] = static_cast<const uint16_t*>(rank_grads[r]);
+    }
+  } else if (c->stage == ZERO_STAGE_2) {
+    if (hi - lo > c->plan.max_bucket)
+      return fail(c, ZERO_EINVAL, "[%lld, %lld) is larger than the bucket buffer", (long long)lo, (long long)hi);
+    for (int r = 0; r < N; ++r) a.grad[r] = grad_buf_ptr(c, r);
+  } else {
+    const int li = c->plan.layer_of(lo);
+    if (hi > c->plan.layers[li].hi) return fail(c, ZERO_EINVAL, "[%lld, %lld) crosses a layer boundary", (long long)lo, (long long)hi);
+    for (int r = 0; r < N; ++r) a.grad[r] = grad_buf_ptr(c, r) + (lo - c->plan.layers[li].lo);
+  }
+  if (hi == lo) return ZERO_OK;
+  a.shard_out = grad_shard_ptr(c) + lo;
+  a.n_vec = (hi - lo) / zsm::kVec;
+  a.n_ranks = N;
+  a.accumulate = c->norm_fresh ? 0 : 1;
+  a.write_back = 0;
+  a.inv_n = (float)(1.0 / (double)N);
+  a.ns = norm_scratch(c);
+  cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "reduce-scatter kernel launch");
+  c->norm_fresh = false;
+  return ZERO_OK;
+}
+
+zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* rank_grads, void* stream) {
+  zero_status st = check_ready(c, false);
+  if (st != ZERO_OK) return st;
+  if (c->stage != ZERO_STAGE_1) return fail(c, ZERO_EINVAL, "all-reduce keeps full gradients: stage 1 only");
+  if ((st = check_interval(c, lo, hi)) != ZERO_OK) return st;
+  const int N = c->plan.n_ranks;
+  zsm::ReduceArgs a;
+  std::memset(&a, 0, sizeof a);
+  for (int r = 0; r < N; ++r) {
+    const void* p = rank_grads ? rank_grads[r] : static_cast<const void*>(grad_buf_ptr(c, r) + lo);
+    if (!p || !aligned16(p)) return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
+    a.grad[r] = static_cast<const uint16_t*>(p);
+  }
+  if (hi == lo) return ZERO_OK;
+  a.shard_out = nullptr;
+  a.n_vec = (hi - lo) / zsm::kVec;
+  a.n_ranks = N;
+  a.accumulate = c->norm_fresh ? 0 : 1;
+  a.write_back = 1;
+  a.inv_n = (float)(1.0 / (double)N);
+  a.ns = norm_scratch(c);
+  cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(c, e, "all-reduce kernel launch");
+  c->norm_fresh = false;
+  return ZERO_OK;
+}
+
+zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) {
+  zero_status st = check_ready(c, true);
+  if (st != ZERO_OK) return st;
+  const int N = c->plan.n_ranks;
+  if (rank < -1 || rank >= N) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
+  if (t < 1) return fail(c, ZERO_EINVAL, "step t must be >= 1");
+  if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
+    return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
+  const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+  const int64_t S = c->plan.shard;
+  const int r0 = rank < 0 ? 0 : rank, r1 = rank < 0 ? N : rank + 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Stage 2/3 (and stage 1 with one launch for all ranks, since every replica
+  // holds the same reduced gradient): the shards are contiguous, so ranks
+  // r0..r1-1 form one launch over [r0*S, r1*S).  Stage 1 per rank reads the
+  // owner's own replica.
+  const int64_t lo = r0 * S, hi = r1 * S;
+  zsm::AdamArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.sc = sc;
+  a.master = master_ptr(c) + lo;
+  a.m = m_ptr(c) + lo;
+  a.v = v_ptr(c) + lo;
+  a.n_vec = (hi - lo) / zsm::kVec;
+  if (c->stage == ZERO_STAGE_3) {
+    a.grad = grad_shard_ptr(c) + lo;
+    a.out = param_ptr(c, 0) + lo;
+  } else if (c->stage == ZERO_STAGE_2) {
+    a.grad = grad_shard_ptr(c) + lo;
+    if (rank >= 0) {
+      a.out = param_ptr(c, rank) + lo;
+    } else {
+      // every rank writes its own replica's owned segment: one launch per rank
+      for (int r = 0; r < N; ++r) {
+        zsm::AdamArgs b = a;
+        b.master = master_ptr(c) + r * S;
+        b.m = m_ptr(c) + r * S;
+        b.v = v_ptr(c) + r * S;
+        b.grad = grad_shard_ptr(c) + r * S;
+        b.out = param_ptr(c, r) + r * S;
+        b.n_vec = S / zsm::kVec;
+        cudaError_t e = zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
+      }
+      c->norm_fresh = true;
+      c->stats_step = t;
+      return ZERO_OK;
+    }
+  } else {
+    if (rank >= 0) {
+      a.grad = grad_buf_ptr(c, rank) + lo;
+      a.out = param_ptr(c, rank) + lo;
+    } else {
+      for (int r = 0; r < N; ++r) {
+        zsm::AdamArgs b = a;
+        b.master = master_ptr(c) + r * S;
+        b.m = m_ptr(c) + r * S;
+        b.v = v_ptr(c) + r * S;
+        b.grad = grad_buf_ptr(c, r) + r * S;
+        b.out = param_ptr(c, r) + r * S;
+        b.n_vec = S / zsm::kVec;
+        cudaError_t e = zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
+      }
+      c->norm_fresh = true;
+      c->stats_step = t;
+      return ZERO_OK;
+    }
+  }
+  if (a.n_vec > 0) {
+    cudaError_t e = zsm::launch_adam(a, grid_for(a.n_vec, c->grid_simple), s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
+  }
+  c->norm_fresh = true;
+  c->stats_step = t;
+  return ZERO_OK;
+}
+
+zero_status zero_all_gather(zero_ctx* c, int64_t lo, int64_t hi, void* const* rank_out, void* stream) {
+  zero_status st = check_ready(c, false);
+  if (st != ZERO_OK) return st;
+  if ((st = check_interval(c, lo, hi)) != ZERO_OK) return st;
+  if (hi == lo) return ZERO_OK;
+  const int N = c->plan.n_ranks;
+  const int64_t S = c->plan.shard;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<uint16_t*> dst(N);
+  int layer_idx = 0;
+  if (!rank_out && c->stage == ZERO_STAGE_3) {
+    layer_idx = c->plan.layer_of(lo);
+    if (hi > c->plan.layers[layer_idx].hi)
+      return fail(c, ZERO_EINVAL, "[%lld, %lld) crosses a layer boundary", (long long)lo, (long long)hi);
+  }
+  for (int r = 0; r < N; ++r) {
+    if (rank_out) {
+      if (!rank_out[r] || !aligned16(rank_out[r])) return fail(c, ZERO_EINVAL, "rank_out[%d] is null or not 16-byte aligned", r);
+      dst[r] = static_cast<uint16_t*>(rank_out[r]);
+    } else if (c->stage == ZERO_STAGE_3) {
+      dst[r] = gather_ptr(c, r) + (lo - c->plan.layers[layer_idx].lo);
+    } else {
+      dst[r] = param_ptr(c, r) + lo;
+    }
+  }
+  // Each owner's piece of [lo, hi) goes out from the owner's copy.
+  for (int owner = (int)(lo / S); owner < N && owner * S < hi; ++owner) {
+    const int64_t a_lo = std::max(lo, owner * S), a_hi = std::min(hi, (owner + 1) * S);
+    if (a_hi <= a_lo) continue;
+    zsm::GatherArgs g;
+    std::memset(&g, 0, sizeof g);
+    g.src = (c->stage == ZERO_STAGE_3 ? param_ptr(c, 0) : param_ptr(c, owner)) + a_lo;
+    g.n_out = 0;
+    for (int r = 0; r < N; ++r) {
+      // the owner's own replica already holds the source (stage 1, 2)
+      if (!rank_out && c->stage != ZERO_STAGE_3 && r == owner) continue;
+      g.out[g.n_out++] = dst[r] + (a_lo - lo);
+    }
+    g.n_vec = (a_hi - a_lo) / zsm::kVec;
+    if (g.n_out == 0) continue;
+    cudaError_t e = zsm::launch_gather(g, grid_for(g.n_vec, c->grid_simple), s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "all-gather kernel launch");
+  }
+  return ZERO_OK;
+}
+
+zero_status zero_step(zero_ctx* c, zero_grad_fn grad_fn, void* grad_user, zero_gather_fn gather_fn,
+                      void* gather_user, void* stream, zero_step_stats* stats) {
+  if (!c) return ZERO_EINVAL;
+  return run_step(c, grad_fn, grad_user, nullptr, gather_fn, gather_user, stream, stats);
+}
+
+zero_status zero_step_resident(zero_ctx* c, const void* const* rank_grads, zero_gather_fn gather_fn,
+                               void* gather_user, void* stream, zero_step_stats* stats) {
+  if (!c) return ZERO_EINVAL;
+  if (!rank_grads) return fail(c, ZERO_EINVAL, "rank_grads is NULL");
+  return run_step(c, nullptr, nullptr, rank_grads, gather_fn, gather_user, stream, stats);
+}
+
+zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, double* model_bytes) {
+  if (!c || !ms || !launches || !model_bytes) return ZERO_EINVAL;
+  double total = 0.0;
+  if (c->timed > 0) {
+    cudaError_t e = cudaEventSynchronize(c->events[2 * c->timed - 1]);
+    if (e != cudaSuccess) return cuda_fail(c, e, "waiting for timed launches");
+    for (size_t k = 0; k < c->timed; ++k) {
+      float one = 0.f;
+      e = cudaEventElapsedTime(&one, c->events[2 * k], c->events[2 * k + 1]);
+      if (e != cudaSuccess) return cuda_fail(c, e, "reading launch time");
+      total += one;
+    }
+  }
+  *ms = total;
+  *launches = (int64_t)c->timed;
+  *model_bytes = c->timed_bytes;
+  c->timed = 0;
+  c->timed_bytes = 0.0;
+  return ZERO_OK;
+}
+
+zero_status zero_read_stats(zero_ctx* c, void* stream, zero_step_stats* out) {
+  if (!c || !out) return ZERO_EINVAL;
+  if (!c->bound || !c->loaded) return fail(c, ZERO_ESTATE, "nothing to read: not bound or not initialised");
+  return finish_stats(c, static_cast<cudaStream_t>(stream), out);
+}
+
+const char* zero_last_error(const zero_ctx* c) { return c ? c->err.c_str() : g_init_error.c_str(); }
+
+void zero_destroy(zero_ctx* c) { delete c; }
+
+}  // extern "C"
