@@ -52,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--blocks-per-sm", type=int, default=0)
     ap.add_argument("--replica-pad", type=int, default=0)
+    ap.add_argument("--ref-sample-elems", type=int, default=0,
+                    help="reference arm: elements per oracle step (0 = sized to about a minute)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
                     help="gpt-1.2b: the benchmark workload; flat-32m: a 33.5M-param flat buffer, "
                          "N = 8, one bucket (2 GB on the device; for profiler captures)")
@@ -362,13 +364,13 @@ def run_ours(args, world, rank, local):
 
 # --------------------------------------------------------------- reference ----
 
-def reference_sample(w, steps_total: int):
+def reference_sample(w, steps_total: int, elems: int = 0):
     """A contiguous leading slice of the workload's first layer, sized so that
     ``steps_total`` oracle steps take about a minute (the oracle does ~9M
     params/s at N = 8 on one core), at least 8192*N elements."""
     k = w.layer_id.count(0)
     numel = list(w.numel[:k])
-    budget = max(8192 * w.n_ranks, int(5e8 / max(1, steps_total)))
+    budget = elems if elems > 0 else max(8192 * w.n_ranks, int(5e8 / max(1, steps_total)))
     out, total = [], 0
     for n in numel:
         if total >= budget:
@@ -388,7 +390,7 @@ def run_reference(args, world, rank, local):
     import oracle
 
     w = workload()
-    numel, layer = reference_sample(w, args.steps + args.warmup)
+    numel, layer = reference_sample(w, args.steps + args.warmup, args.ref_sample_elems)
     p = oracle.plan(numel, layer, w.n_ranks, w.bucket_elems)
     m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
     grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)

@@ -1,0 +1,74 @@
+"""bench.py's multi-process plumbing on CPU: two ranks over gloo, as
+torch.distributed.run would launch them.  The timing taken is the maximum
+over ranks, every rank makes the same collective calls, and only rank 0
+prints the JSON line (the reference arm runs on rank 0 alone)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r"""
+import json, os, sys
+sys.path.insert(0, {root!r})
+import bench
+world, rank, local = bench.dist_env()
+d = bench.init_dist(world, "gloo")
+m = bench.max_over_ranks(float(10 * rank + 1), d, "cpu")
+bench.barrier(d)
+m2 = bench.max_over_ranks(float(100 - rank), d, "cpu")
+print(json.dumps({{"rank": rank, "max": m, "max2": m2}}))
+d.destroy_process_group()
+"""
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _launch(code_or_args, world=2, timeout=120):
+    port = _free_port()
+    procs = []
+    for r in range(world):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(world),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), CUDA_VISIBLE_DEVICES="")
+        cmd = [sys.executable] + (["-c", code_or_args] if isinstance(code_or_args, str) else code_or_args)
+        procs.append(subprocess.Popen(cmd, env=env, cwd=ROOT, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = []
+    for p in procs:
+        try:
+            o, e = p.communicate(timeout=timeout)
+        except subprocess.TimeoutExpired:
+            for q in procs:
+                q.kill()
+            raise
+        outs.append((p.returncode, o, e))
+    return outs
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    outs = _launch(CHILD.format(root=ROOT))
+    for rc, o, e in outs:
+        assert rc == 0, e
+    got = [json.loads(o.strip().splitlines()[-1]) for _, o, _ in outs]
+    assert all(g["max"] == 11.0 and g["max2"] == 100.0 for g in got)
+
+
+def test_reference_arm_prints_once_on_rank_zero():
+    outs = _launch(["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "2", "--warmup", "1",
+                    "--ref-sample-elems", "65536"], timeout=300)
+    assert all(rc == 0 for rc, _, _ in outs), [e for _, _, e in outs]
+    lines0 = [l for l in outs[0][1].splitlines() if l.startswith("{")]
+    lines1 = [l for l in outs[1][1].splitlines() if l.startswith("{")]
+    assert len(lines0) == 1 and not lines1
+    d = json.loads(lines0[0])
+    assert d["impl"] == "reference" and d["unit"] == "params/s" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] == 1 and d["n_gpus"] == 2

@@ -102,6 +102,8 @@ def _oracle_run(w, stage, bucket):
 
 def _check_against_oracle(w, stage, bucket, exact=True):
     z = _z()
+    if bucket is None:  # one bucket spanning the padded flat space
+        bucket = oracle.plan(w.numel, w.layer_id, w.n_ranks, 1 << 40).psi_pad
     p, ranks, reps = _oracle_run(w, STAGE_OF[stage], bucket)
     ref = oracle.full_view(p, STAGE_OF[stage], ranks)
     opt, fill = make_opt(w, stage, bucket=bucket, keep=True)
