@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--blocks-per-sm", type=int, default=0)
+    ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
+                    help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
@@ -239,7 +241,8 @@ def run_ours(args, world, rank, local):
     s = stream.cuda_stream
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, z.ZERO_STAGE_2, bucket_elems=w.bucket_elems,
                           hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
-                          replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm, device=dev)
+                          replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
+                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], device=dev)
     offsets = opt.offsets()
     mv = opt.view(z.ZERO_VIEW_MASTER)
     b = W.master_base(w)
@@ -342,7 +345,8 @@ def run_ours(args, world, rank, local):
                    "storage": "bf16 grads/params, fp32 master/m/v",
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
-                   "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas"},
+                   "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
+                   "kernel": args.kernel},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak", "kernel": "fused_step_kernel",

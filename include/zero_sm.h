@@ -129,10 +129,26 @@ enum {
   ZERO_OPT_REPLICA_PAD = 2,      /* extra bytes (multiple of 256, < 1 MiB) between consecutive
                                     rank buffers; default 0 */
   ZERO_OPT_BLOCKS_PER_SM = 3,    /* fused-kernel CTAs per SM (0 = occupancy maximum) */
-  ZERO_OPT_TIMING = 4            /* 1: record a CUDA event pair on the launching stream around
+  ZERO_OPT_TIMING = 4,           /* 1: record a CUDA event pair on the launching stream around
                                     every fused-step kernel launch (read with
                                     zero_kernel_timing); may be set at any time; default 0 */
+  ZERO_OPT_KERNEL = 5            /* fused-step kernel: ZERO_KERNEL_AUTO (default),
+                                    ZERO_KERNEL_REGISTER or ZERO_KERNEL_TMA; may be set at any
+                                    time; ZERO_KERNEL_TMA needs N <= 16 (else ZERO_EINVAL) */
 };
+
+/* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.
+ *   REGISTER: each lane loads its 16-byte slices of the N replicas and of
+ *             master/m/v straight into registers (any N).
+ *   TMA:      one CTA per SM; a producer thread streams every 2048-element
+ *             tile of the N replicas and master/m/v into a ring of shared-
+ *             memory stages with bulk copies (mbarrier-counted), consumer
+ *             warps compute from shared memory (N <= 16).  Its waits are
+ *             bounded; one that runs out is reported as ZERO_ECUDA by the next
+ *             synchronising call (zero_read_stats, zero_step with stats,
+ *             zero_kernel_timing).
+ *   AUTO:     the faster of the two for this N, as measured on B200. */
+enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2 };
 
 /* Views (zero_view). */
 enum {

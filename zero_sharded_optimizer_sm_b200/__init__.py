@@ -37,7 +37,8 @@ ZERO_STAGE_DP, ZERO_STAGE_1, ZERO_STAGE_2, ZERO_STAGE_3 = 0, 1, 2, 3
 ZERO_MAX_RANKS = 128
 (ZERO_ARENA_STATES, ZERO_ARENA_PARAMS, ZERO_ARENA_GRADS, ZERO_ARENA_GRAD_SHARDS, ZERO_ARENA_GATHER,
  ZERO_ARENA_SCRATCH, ZERO_NUM_ARENAS) = range(7)
-ZERO_OPT_KEEP_GRAD_SHARDS, ZERO_OPT_REPLICA_PAD, ZERO_OPT_BLOCKS_PER_SM, ZERO_OPT_TIMING = 1, 2, 3, 4
+ZERO_OPT_KEEP_GRAD_SHARDS, ZERO_OPT_REPLICA_PAD, ZERO_OPT_BLOCKS_PER_SM, ZERO_OPT_TIMING, ZERO_OPT_KERNEL = 1, 2, 3, 4, 5
+ZERO_KERNEL_AUTO, ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA = 0, 1, 2
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
 
@@ -145,7 +146,7 @@ class ZeroOptimizer:
     def __init__(self, numel: Sequence[int], layer_id: Sequence[int], n_ranks: int, stage: int,
                  bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
-                 device=None):
+                 kernel: int = ZERO_KERNEL_AUTO, device=None):
         import torch
 
         self._torch = torch
@@ -171,6 +172,8 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_REPLICA_PAD, int(replica_pad)), "zero_set_option")
         if blocks_per_sm:
             self._check(zero_set_option(ctx, ZERO_OPT_BLOCKS_PER_SM, int(blocks_per_sm)), "zero_set_option")
+        if kernel:
+            self._check(zero_set_option(ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
@@ -357,6 +360,9 @@ class ZeroOptimizer:
             raise self._cb_error
         self._check(st, "zero_step_resident")
         return self._stats_dict(out) if stats else None
+
+    def set_kernel(self, kernel: int):
+        self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
 
     def set_timing(self, on: bool):
         self._check(zero_set_option(self.ctx, ZERO_OPT_TIMING, 1 if on else 0), "zero_set_option")

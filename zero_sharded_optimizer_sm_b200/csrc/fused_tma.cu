@@ -1,0 +1,266 @@
+// Fused ZeRO step kernel with the inputs staged through shared memory by the
+// Tensor Memory Accelerator (sm_100a).
+//
+// Same arithmetic and outputs as the register-path fused kernel (kernels.cu),
+// different data movement: one persistent CTA per SM; warp 0 is a producer
+// whose elected lane streams each tile's N gradient slices and its fp32
+// master/m/v slices from HBM into a ring of shared-memory stages with 1-D
+// bulk copies (cp.async.bulk, completion counted in bytes on an mbarrier);
+// two groups of eight consumer warps take alternate tiles, reduce, update
+// and store from shared memory, then release the stage.  Group g owns stages
+// g, g+2, ... (the stage count is even), so each group meets the phases of
+// its stages in order.  With four 56 KB stages per SM (N = 8) up to 224 KB of
+// loads are in flight per SM without holding them in registers.  The bulk copies
+// read only this GPU's memory into the CTA's own shared memory; no cluster
+// multicast is used.
+//
+// Every wait on an mbarrier is bounded (kWaitNs of wall time).  A wait that
+// runs out records an error code in the scratch arena, stops the producer,
+// drains the copies already issued (again bounded) and ends the CTA, so the
+// host sees ZERO_ECUDA instead of a hung GPU.
+#include <cuda_runtime.h>
+
+#include "device_math.cuh"
+#include "kernels.cuh"
+
+namespace zsm {
+namespace {
+
+using namespace dev;
+
+constexpr int kConsumerWarps = 8;                   // warps of one consumer group
+constexpr int kConsumers = kConsumerWarps * 32;     // 256 threads per group, 8 elements each
+constexpr int kGroups = 2;                          // consumer groups, alternate tiles
+constexpr int kTmaThreads = kGroups * kConsumers + 32;  // + one producer warp
+constexpr int kTile = kConsumers * kVec;            // 2048 elements per tile
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (now_ns() - t0 > kWaitNs) return false;
+  return true;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completion on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__host__ __device__ inline unsigned tma_stage_bytes(int n_ranks) {
+  return (unsigned)(kTile * (2 * n_ranks + 12));
+}
+
+// Shared memory: [stages x stage_bytes][full[stages]][empty[stages]][flags]
+template <int MODE>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    fused_step_tma_kernel(const __grid_constant__ FusedArgs a, int stages) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const unsigned stage_bytes = tma_stage_bytes(N);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stage_bytes);
+  uint64_t* empty = full + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* issued_flag = abort_flag + 1;  // tiles issued by the producer
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    *issued_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer --
+    if (lane == 0) {
+      int it = 0;
+      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (*abort_flag) break;
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u)) {
+          atomicOr(a.ns.error, 1u);
+          *abort_flag = 1;
+          break;
+        }
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        unsigned char* st = smem + (size_t)s * stage_bytes;
+        mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s]);
+        unsigned char* stt = st + (size_t)N * 2 * kTile;
+        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &full[s]);
+        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &full[s]);
+        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s]);
+        *issued_flag = it + 1;
+      }
+    }
+  } else {
+    // --------------------------------------------------------- consumers --
+    const int group = (threadIdx.x - 32) / kConsumers;  // 0 or 1
+    const int c = (threadIdx.x - 32) % kConsumers;      // 0..255
+    int it = group;
+    for (int64_t tile = blockIdx.x + (int64_t)group * gridDim.x; tile < n_tiles;
+         tile += (int64_t)kGroups * gridDim.x, it += kGroups) {
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      // warp-uniform decisions, so that no lane is left waiting at __syncwarp
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const unsigned char* st = smem + (size_t)s * stage_bytes;
+      const int j = c * kVec;
+      const bool active = j < cnt;  // the last tile may be ragged
+      float4 p0, p1, m0, m1, v0, v1;
+      float acc[kVec];
+      if (active) {
+        const float* stt = reinterpret_cast<const float*>(st + (size_t)N * 2 * kTile);
+        p0 = *reinterpret_cast<const float4*>(stt + j);
+        p1 = *reinterpret_cast<const float4*>(stt + j + 4);
+        m0 = *reinterpret_cast<const float4*>(stt + kTile + j);
+        m1 = *reinterpret_cast<const float4*>(stt + kTile + j + 4);
+        v0 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j);
+        v1 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j + 4);
+#pragma unroll
+        for (int q = 0; q < kVec; ++q) acc[q] = 0.0f;
+        for (int r = 0; r < N; ++r)
+          add8(acc, *reinterpret_cast<const uint4*>(st + (size_t)r * 2 * kTile + 2 * j));
+      }
+      // every lane of the warp is done reading this stage: release it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (active) {
+        const int64_t e = e0 + j;
+        uint16_t g16[kVec];
+        float g[kVec];
+        mean_bf16(acc, a.inv_n, g16, g, sq, nf);
+        if (MODE == kFusedZ1) {
+          const uint4 gw = pack8(g16);
+          for (int r = 0; r < N; ++r) st_stream(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+        }
+        if (a.grad_shard) st_stream(a.grad_shard + e, pack8(g16));
+        uint16_t p16[kVec];
+        adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        st_stream(a.master + e, p0);
+        st_stream(a.master + e + 4, p1);
+        st_stream(a.m + e, m0);
+        st_stream(a.m + e + 4, m1);
+        st_stream(a.v + e, v0);
+        st_stream(a.v + e + 4, v1);
+        const uint4 pw = pack8(p16);
+        if (MODE == kFusedZ3) st_stream(a.param_shard + e, pw);
+        for (int r = 0; r < N; ++r) st_stream(a.out[r] + e, pw);
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // drain the bulk copies already issued before the CTA's memory goes away
+    const int issued = *issued_flag;
+    for (int s = 0; s < stages && s < issued; ++s) {
+      const int last = ((issued - 1 - s) / stages) * stages + s;  // last tile on stage s
+      if (!mbar_wait(&full[s], (unsigned)(last / stages) & 1u)) atomicOr(a.ns.error, 4u);
+    }
+  }
+  norm_epilogue<kTmaThreads>(a.ns, sq, nf, a.accumulate);
+}
+
+template <int MODE>
+cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, cudaStream_t s) {
+  const size_t bytes = (size_t)stages * tma_stage_bytes(a.n_ranks) + 2 * stages * sizeof(uint64_t) + 16;
+  fused_step_tma_kernel<MODE><<<grid, kTmaThreads, bytes, s>>>(a, stages);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t tma_configure() {
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ3>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+  return e;
+}
+
+int tma_stages_for(int n_ranks) {
+  if (n_ranks < 1 || n_ranks > kTmaMaxRanks) return 0;
+  const size_t per = tma_stage_bytes(n_ranks) + 2 * sizeof(uint64_t);
+  int stages = (int)((kTmaMaxSmem - 16) / per);
+  if (stages > 4) stages = 4;
+  stages -= stages % kGroups;  // each consumer group owns stages g, g+2, ...
+  return stages >= 2 ? stages : 0;
+}
+
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
+  const int stages = tma_stages_for(a.n_ranks);
+  if (stages == 0) return cudaErrorInvalidValue;
+  switch (mode) {
+    case kFusedZ1: return launch_tma_mode<kFusedZ1>(a, grid, stages, s);
+    case kFusedZ2: return launch_tma_mode<kFusedZ2>(a, grid, stages, s);
+    case kFusedZ3: return launch_tma_mode<kFusedZ3>(a, grid, stages, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace zsm

@@ -15,6 +15,8 @@ constexpr int kMaxRanks = 128;   // mirrors ZERO_MAX_RANKS
 constexpr int kVec = 8;          // bf16 elements per 16-byte vector
 constexpr int kThreads = 256;    // threads per CTA for every kernel
 constexpr int kMaxGrid = 4096;   // upper bound on CTAs of a norm-reducing launch
+constexpr int kTmaMaxRanks = 16; // the shared-memory staged kernel handles N <= 16
+constexpr int kTmaMaxSmem = 227 * 1024 - 1024;  // dynamic smem cap (1 KB left for static)
 
 // Binary32 scalars of one Adam step, each rounded once from binary64 on the host.
 struct AdamScalars {
@@ -28,6 +30,7 @@ struct NormScratch {
   unsigned int* done;              // CTAs of the current launch that finished
   double* step_sq;                 // sum over the launches of the current step
   unsigned long long* step_nf;
+  unsigned int* error;             // non-zero after a bounded device wait ran out
 };
 
 // Fused reduce + Adam + broadcast over one interval [lo, hi) of the flat space.
@@ -89,6 +92,7 @@ struct InitArgs {
 };
 
 enum FusedMode { kFusedZ1 = 1, kFusedZ2 = 2, kFusedZ3 = 3 };
+enum FusedKernel { kKernelAuto = 0, kKernelRegister = 1, kKernelTma = 2 };
 
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s);
@@ -96,6 +100,11 @@ cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
+
+// Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM.
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, cudaStream_t s);
+int tma_stages_for(int n_ranks);   // 0 when N is out of its range
+cudaError_t tma_configure();       // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.
 cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_blocks);

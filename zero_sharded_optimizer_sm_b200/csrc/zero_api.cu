@@ -36,6 +36,7 @@ struct zero_ctx {
   bool keep_grad_shards = true;
   int64_t replica_pad = 0;
   int blocks_per_sm_opt = 0;
+  int kernel_opt = ZERO_KERNEL_AUTO;
   // arena layout (bytes)
   int64_t arena_bytes[ZERO_NUM_ARENAS] = {};
   int64_t state_pitch = 0;   // bytes between master, m and v
@@ -139,6 +140,7 @@ zsm::NormScratch norm_scratch(zero_ctx* c) {
   ns.step_sq = reinterpret_cast<double*>(s + 16 * zsm::kMaxGrid);
   ns.step_nf = reinterpret_cast<unsigned long long*>(s + 16 * zsm::kMaxGrid + 8);
   ns.done = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 16);
+  ns.error = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 20);
   return ns;
 }
 
@@ -162,6 +164,15 @@ zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
 }
 
 constexpr size_t kMaxTimed = 4096;
+constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the staged kernel
+
+// Whether the fused step runs the shared-memory staged kernel.
+bool use_tma(const zero_ctx* c) {
+  if (zsm::tma_stages_for(c->plan.n_ranks) == 0) return false;
+  if (c->kernel_opt == ZERO_KERNEL_TMA) return true;
+  if (c->kernel_opt == ZERO_KERNEL_REGISTER) return false;
+  return false;  // AUTO
+}
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
@@ -247,7 +258,13 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  cudaError_t e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
+  cudaError_t e;
+  if (use_tma(c)) {
+    const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
+    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)), s);
+  } else {
+    e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
+  }
   if (e != cudaSuccess) return cuda_fail(c, e, "fused step kernel launch");
   if (ev) {
     cudaEventRecord(ev[1], s);
@@ -257,15 +274,26 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   return ZERO_OK;
 }
 
+// Reads and clears the device error word (a bounded wait that ran out).
+zero_status check_device_error(zero_ctx* c, unsigned int err, cudaStream_t s) {
+  if (err == 0) return ZERO_OK;
+  cudaMemsetAsync(norm_scratch(c).error, 0, sizeof(unsigned int), s);
+  return fail(c, ZERO_ECUDA, "a bounded wait in the staged fused kernel ran out (code %u): results of the step are invalid", err);
+}
+
 zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
   struct {
     double sq;
     unsigned long long nf;
+    unsigned int done;
+    unsigned int error;
   } host{};
   zsm::NormScratch ns = norm_scratch(c);
-  cudaError_t e = cudaMemcpyAsync(&host, ns.step_sq, 16, cudaMemcpyDeviceToHost, s);
+  cudaError_t e = cudaMemcpyAsync(&host, ns.step_sq, sizeof host, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(c, e, "reading step statistics");
+  zero_status st = check_device_error(c, host.error, s);
+  if (st != ZERO_OK) return st;
   std::memset(out, 0, sizeof *out);
   out->grad_norm = std::sqrt(host.sq);
   out->nonfinite = (int64_t)host.nf;
@@ -358,6 +386,13 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     c->timing = value != 0;
     return ZERO_OK;
   }
+  if (key == ZERO_OPT_KERNEL) {
+    if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_TMA) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
+    if (value == ZERO_KERNEL_TMA && zsm::tma_stages_for(c->plan.n_ranks) == 0)
+      return fail(c, ZERO_EINVAL, "the staged kernel handles N <= %d", zsm::kTmaMaxRanks);
+    c->kernel_opt = (int)value;
+    return ZERO_OK;
+  }
   if (c->bound) return fail(c, ZERO_ESTATE, "options must be set before zero_bind");
   switch (key) {
     case ZERO_OPT_KEEP_GRAD_SHARDS:
@@ -439,6 +474,7 @@ zero_status zero_bind(zero_ctx* c, void* const* arenas) {
   int fused_blocks = 0, simple_blocks = 0;
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
+  if (e == cudaSuccess && zsm::tma_stages_for(c->plan.n_ranks) > 0) e = zsm::tma_configure();
   if (e != cudaSuccess) return cuda_fail(c, e, "device query");
   if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
   c->grid_fused = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, fused_blocks)));
@@ -770,6 +806,12 @@ zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, doubl
   *model_bytes = c->timed_bytes;
   c->timed = 0;
   c->timed_bytes = 0.0;
+  if (c->bound) {
+    unsigned int err = 0;
+    cudaError_t e = cudaMemcpy(&err, norm_scratch(c).error, sizeof err, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(c, e, "reading the device error word");
+    return check_device_error(c, err, nullptr);
+  }
   return ZERO_OK;
 }
 
