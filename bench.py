@@ -54,6 +54,11 @@ def parse_args(argv=None):
     ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
                     help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="flat-buffer sweep instead of the bench line: 1K..1G elements (x4) x N in "
+                         "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
+                         "JSON line per cell")
+    ap.add_argument("--sweep-max-gb", type=float, default=150.0)
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
@@ -366,6 +371,79 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------- sweep ----
+
+def run_sweep(args):
+    """Flat-buffer ZeRO-2 sweep: for each (E, N) cell, the fused step (the
+    library's kernel choice) and the unfused reduce-scatter -> Adam ->
+    all-gather sequence over the same resident replicas, timed with CUDA
+    events over enough repetitions for ~50 ms.  GB/s are reported against the
+    (4N+24) B/element model of the fused step; the unfused path's own
+    (4N+32) B/element traffic is reported beside it.  Cells whose working set
+    fits in L2 (126 MB) measure L2 and launch latency, and are labelled so."""
+    import torch
+
+    import synth
+    import zero_sharded_optimizer_sm_b200 as z
+    from synth import workloads as W
+
+    torch.cuda.set_device(0)
+    s = torch.cuda.current_stream().cuda_stream
+    for n_ranks in W.SWEEP_RANKS:
+        for elems in W.SWEEP_ELEMS:
+            resident = (6 * n_ranks + 14) * elems  # replicas in, params out, states, grad shard
+            cell = {"sweep": "flat-zero2", "elems": elems, "n_ranks": n_ranks}
+            if resident > args.sweep_max_gb * 1e9:
+                cell["skipped"] = f"exceeds HBM budget ({resident / 1e9:.0f} GB)"
+                print(json.dumps(cell), flush=True)
+                continue
+            w = W.flat_sweep(elems, n_ranks)
+            opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, z.ZERO_STAGE_2, keep_grad_shards=True,
+                                  grad_buffers=False, kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel])
+            mv = opt.view(z.ZERO_VIEW_MASTER)
+            synth.dev_f32(W.master_base(w), 0, elems, W.MASTER_DIST, mv.data_ptr(), s)
+            opt.load_master(None)
+            reps = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+            for r in range(n_ranks):
+                synth.dev_bf16(W.grad_base(w, 1, r), 0, elems, w.grad_dist, reps[r].data_ptr(), s)
+            rl = list(reps)
+            ptrs = [t.data_ptr() for t in rl]
+            model = (4 * n_ranks + 24) * opt.psi_pad
+            reps_n = int(min(2000, max(3, 5e-2 / max(model / 6.0e12, 3e-6))))
+
+            def fused():
+                opt.step_resident(rl)
+
+            def unfused(t=[0]):
+                t[0] += 1
+                opt.reduce_scatter(0, opt.psi_pad, ptrs)
+                opt.adam_shard(-1, t[0])
+                opt.all_gather(0, opt.psi_pad)
+
+            for name, fn in (("fused", fused), ("unfused", unfused)):
+                for _ in range(3):
+                    fn()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(reps_n):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / reps_n
+                cell[f"{name}_us"] = ms * 1e3
+                cell[f"{name}_gbs_model_4n24"] = model / (ms / 1e3) / 1e9
+            cell["unfused_gbs_own_4n32"] = (4 * n_ranks + 32) * opt.psi_pad / (cell["unfused_us"] / 1e6) / 1e9
+            cell["fused_speedup"] = cell["unfused_us"] / cell["fused_us"]
+            cell["regime"] = "L2-resident / launch-bound" if model < 126e6 * 2 else "HBM"
+            cell["reps"] = reps_n
+            print(json.dumps(cell), flush=True)
+            opt.close()
+            del opt, reps, rl, mv
+            torch.cuda.empty_cache()
+
+
 # --------------------------------------------------------------- reference ----
 
 def reference_sample(w, steps_total: int, elems: int = 0):
@@ -435,6 +513,8 @@ def main(argv=None):
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, world, rank, local)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args, world, rank, local)
 

@@ -132,18 +132,24 @@ enum {
   ZERO_OPT_TIMING = 4,           /* 1: record a CUDA event pair on the launching stream around
                                     every fused-step kernel launch (read with
                                     zero_kernel_timing); may be set at any time; default 0 */
-  ZERO_OPT_KERNEL = 5            /* fused-step kernel: ZERO_KERNEL_AUTO (default),
+  ZERO_OPT_KERNEL = 5,           /* fused-step kernel: ZERO_KERNEL_AUTO (default),
                                     ZERO_KERNEL_REGISTER or ZERO_KERNEL_TMA; may be set at any
                                     time; ZERO_KERNEL_TMA needs N <= 16 (else ZERO_EINVAL) */
+  ZERO_OPT_GRAD_BUFFERS = 6,     /* 1 (default) sizes the GRADS arena; 0 drops it for callers
+                                    that only use zero_step_resident and the calls given explicit
+                                    pointers (zero_step then returns ZERO_ESTATE) */
+  ZERO_OPT_TMA_GROUPS = 7        /* staged kernel: producer/consumer groups per CTA, 1 or 2
+                                    (0 = the library's choice); may be set at any time */
 };
 
 /* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.
  *   REGISTER: each lane loads its 16-byte slices of the N replicas and of
  *             master/m/v straight into registers (any N).
- *   TMA:      one CTA per SM; a producer thread streams every 2048-element
- *             tile of the N replicas and master/m/v into a ring of shared-
- *             memory stages with bulk copies (mbarrier-counted), consumer
- *             warps compute from shared memory (N <= 16).  Its waits are
+ *   TMA:      one CTA per SM with one or two groups, each a producer thread
+ *             that streams its 2048-element tiles of the N replicas and
+ *             master/m/v into its own shared-memory stages with bulk copies
+ *             (mbarrier-counted) and eight consumer warps that compute from
+ *             shared memory (N <= 16).  Its waits are
  *             bounded; one that runs out is reported as ZERO_ECUDA by the next
  *             synchronising call (zero_read_stats, zero_step with stats,
  *             zero_kernel_timing).

@@ -47,15 +47,20 @@ def _hp(w):
 
 
 REG, TMA = 1, 2  # ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA
+# fused-kernel variants: the register path, the staged path with one and two groups
+VARIANTS = {"reg": dict(kernel=REG), "tma1": dict(kernel=TMA, tma_groups=1),
+            "tma2": dict(kernel=TMA, tma_groups=2)}
 
 
 def kernels_for(n_ranks):
-    """Fused kernels that apply at this N (the staged one handles N <= 16)."""
-    return (REG, TMA) if n_ranks <= 16 else (REG,)
+    """Fused-kernel variants that apply at this N (the staged one handles N <= 16)."""
+    return ("reg", "tma1", "tma2") if n_ranks <= 16 else ("reg",)
 
 
-def make_opt(w, stage, bucket=None, keep=True, **kw):
+def make_opt(w, stage, bucket=None, keep=True, variant=None, **kw):
     z = _z()
+    if variant is not None:
+        kw.update(VARIANTS[variant])
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=bucket, hparams=_hp(w),
                           keep_grad_shards=keep, **kw)
     fill = DeviceFill(w, opt.offsets(), opt.psi_pad)
@@ -112,14 +117,14 @@ def _check_against_oracle(w, stage, bucket, exact=True, kernels=None):
     if bucket is None:  # one bucket spanning the padded flat space
         bucket = oracle.plan(w.numel, w.layer_id, w.n_ranks, 1 << 40).psi_pad
     p, ranks, reps = _oracle_run(w, STAGE_OF[stage], bucket)
-    for kernel in (kernels or kernels_for(w.n_ranks)):
-        _check_kernel_against_oracle(w, stage, bucket, p, ranks, reps, kernel, exact)
+    for variant in (kernels or kernels_for(w.n_ranks)):
+        _check_kernel_against_oracle(w, stage, bucket, p, ranks, reps, variant, exact)
 
 
-def _check_kernel_against_oracle(w, stage, bucket, p, ranks, reps, kernel, exact):
+def _check_kernel_against_oracle(w, stage, bucket, p, ranks, reps, variant, exact):
     z = _z()
     ref = oracle.full_view(p, STAGE_OF[stage], ranks)
-    opt, fill = make_opt(w, stage, bucket=bucket, keep=True, kernel=kernel)
+    opt, fill = make_opt(w, stage, bucket=bucket, keep=True, variant=variant)
     assert opt.offsets() == p.offset and opt.buckets() == p.buckets
     gathered = []
 
@@ -350,10 +355,10 @@ def test_transformer_85m_n8_stages_agree_and_match_dp():
     z = _z()
     w = W.gpt_85m_n8()
     opts = {}
-    for stage in (1, 2, 3, "tma1", "tma2", "tma3"):
-        kernel = TMA if isinstance(stage, str) else REG
+    for stage in (1, 2, 3, "tma1-1", "tma1-2", "tma1-3", "tma2-1", "tma2-2", "tma2-3"):
+        variant = stage.split("-")[0] if isinstance(stage, str) else "reg"
         st_ = int(str(stage)[-1])
-        opt, fill = make_opt(w, st_, bucket=20_000_000, kernel=kernel)
+        opt, fill = make_opt(w, st_, bucket=20_000_000, variant=variant)
         gathered_ok = []
 
         def gather(layer, lo, hi, bufs, stream, opt=opt):
@@ -371,8 +376,8 @@ def test_transformer_85m_n8_stages_agree_and_match_dp():
                 assert torch.equal(opt.view(z.ZERO_VIEW_PARAM, 0), opt.view(z.ZERO_VIEW_PARAM, r))
         opts[stage] = opt
     # the staged kernel computes the same bits as the register kernel
-    for st_ in (1, 2, 3):
-        a, b = opts[st_], opts[f"tma{st_}"]
+    for st_, v in [(x, y) for x in (1, 2, 3) for y in ("tma1", "tma2")]:
+        a, b = opts[st_], opts[f"{v}-{st_}"]
         for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ, z.ZERO_VIEW_PARAM):
             assert torch.equal(a.view(what), b.view(what)), (st_, what)
         if st_ == 1:
@@ -440,21 +445,25 @@ def test_transformer_1p2b_n8_zero2_bucket200m():
     del res
     gc.collect()
     torch.cuda.empty_cache()
-    # the staged kernel, resident replicas: the same bits
-    tma, tfill = make_opt(w, 2, bucket=w.bucket_elems, keep=False, kernel=TMA)
-    for t in range(1, w.steps + 1):
+    # the staged kernel (one and two groups), resident replicas: the same bits
+    for variant in ("tma1", "tma2"):
+        tma, tfill = make_opt(w, 2, bucket=w.bucket_elems, keep=False, variant=variant)
+        for t in range(1, w.steps + 1):
+            for r in range(w.n_ranks):
+                tfill.grads_into(t, r, 0, tma.psi_pad, reps[r].data_ptr(), reps[r], s)
+            tma.step_resident(list(reps), stats=True)
+        for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+            assert torch.equal(tma.view(what), keep[what]), variant
         for r in range(w.n_ranks):
-            tfill.grads_into(t, r, 0, tma.psi_pad, reps[r].data_ptr(), reps[r], s)
-        tma.step_resident(list(reps), stats=True)
-    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
-        assert torch.equal(tma.view(what), keep[what])
-    for r in range(w.n_ranks):
-        assert torch.equal(tma.view(z.ZERO_VIEW_PARAM, r), keep["p0"])
-    tma.set_timing(True)
-    tma.step_resident(list(reps))
-    kt = tma.kernel_timing()  # also reads the device error word
-    assert kt["launches"] == 7 and kt["model_bytes"] == 56 * tma.psi_pad
-    tma.close()
+            assert torch.equal(tma.view(z.ZERO_VIEW_PARAM, r), keep["p0"]), variant
+        tma.set_timing(True)
+        tma.step_resident(list(reps))
+        kt = tma.kernel_timing()  # also reads the device error word
+        assert kt["launches"] == 7 and kt["model_bytes"] == 56 * tma.psi_pad
+        tma.close()
+        del tma
+        gc.collect()
+        torch.cuda.empty_cache()
     del reps, keep
     gc.collect()
     torch.cuda.empty_cache()
@@ -511,7 +520,7 @@ def test_flat_sweep_cells_every_element(elems, n_ranks):
 def test_flat_sweep_large_cells_fused_equals_unfused_and_oracle_samples(elems, n_ranks):
     z = _z()
     w = W.flat_sweep(elems, n_ranks)
-    fused, ff = make_opt(w, 2, keep=False, kernel=kernels_for(n_ranks)[-1])
+    fused, ff = make_opt(w, 2, keep=False, variant=kernels_for(n_ranks)[-1])
     s = torch.cuda.current_stream().cuda_stream
     reps = torch.empty((n_ranks, fused.psi_pad), dtype=torch.int16, device="cuda")
     for r in range(n_ranks):

@@ -30,9 +30,11 @@ using namespace dev;
 
 constexpr int kConsumerWarps = 8;                   // warps of one consumer group
 constexpr int kConsumers = kConsumerWarps * 32;     // 256 threads per group, 8 elements each
-constexpr int kGroups = 2;                          // consumer groups, alternate tiles
-constexpr int kTmaThreads = kGroups * kConsumers + 32;  // + one producer warp
 constexpr int kTile = kConsumers * kVec;            // 2048 elements per tile
+
+// G consumer groups, each with its own producer warp: G * (32 + 256) threads.
+template <int G>
+__host__ __device__ constexpr int tma_threads() { return G * (32 + kConsumers); }
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -92,9 +94,15 @@ __host__ __device__ inline unsigned tma_stage_bytes(int n_ranks) {
   return (unsigned)(kTile * (2 * n_ranks + 12));
 }
 
-// Shared memory: [stages x stage_bytes][full[stages]][empty[stages]][flags]
-template <int MODE>
-__global__ void __launch_bounds__(kTmaThreads, 1)
+// Shared memory: [stages x stage_bytes][full[stages]][empty[stages]][abort][last_k[stages]]
+//
+// Warps 0..G-1 are producers (lane 0 works), warps G + 8g .. G + 8g + 7 form
+// consumer group g.  Tile number `it` of this CTA (tile = blockIdx.x + it *
+// gridDim.x) belongs to group it % G and lives in stage it % stages; the
+// stage count is a multiple of G, so every stage belongs to one group and
+// each group's producer and consumers meet its stages' phases in order.
+template <int MODE, int G>
+__global__ void __launch_bounds__(tma_threads<G>(), 1)
     fused_step_tma_kernel(const __grid_constant__ FusedArgs a, int stages) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int N = a.n_ranks;
@@ -102,7 +110,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stage_bytes);
   uint64_t* empty = full + stages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
-  volatile int* issued_flag = abort_flag + 1;  // tiles issued by the producer
+  volatile int* last_k = abort_flag + 1;  // last phase issued on each stage, -1 = none
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_elem = a.n_vec * kVec;
   const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
@@ -111,9 +119,9 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
+      last_k[s] = -1;
     }
     *abort_flag = 0;
-    *issued_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -121,11 +129,13 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   double sq = 0.0;
   unsigned long long nf = 0;
 
-  if (warp == 0) {
+  if (warp < G) {
     // ---------------------------------------------------------- producer --
     if (lane == 0) {
-      int it = 0;
-      for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+      const int g = warp;
+      for (int it = g;; it += G) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
         if (*abort_flag) break;
@@ -144,16 +154,16 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
         bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &full[s]);
         bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &full[s]);
         bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s]);
-        *issued_flag = it + 1;
+        last_k[s] = (int)k;
       }
     }
   } else {
     // --------------------------------------------------------- consumers --
-    const int group = (threadIdx.x - 32) / kConsumers;  // 0 or 1
-    const int c = (threadIdx.x - 32) % kConsumers;      // 0..255
-    int it = group;
-    for (int64_t tile = blockIdx.x + (int64_t)group * gridDim.x; tile < n_tiles;
-         tile += (int64_t)kGroups * gridDim.x, it += kGroups) {
+    const int g = (warp - G) / kConsumerWarps;
+    const int c = (threadIdx.x - 32 * G) % kConsumers;  // 0..255
+    for (int it = g;; it += G) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
       // warp-uniform decisions, so that no lane is left waiting at __syncwarp
@@ -190,15 +200,15 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
       if (active) {
         const int64_t e = e0 + j;
         uint16_t g16[kVec];
-        float g[kVec];
-        mean_bf16(acc, a.inv_n, g16, g, sq, nf);
+        float gv[kVec];
+        mean_bf16(acc, a.inv_n, g16, gv, sq, nf);
         if (MODE == kFusedZ1) {
           const uint4 gw = pack8(g16);
           for (int r = 0; r < N; ++r) st_stream(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         }
         if (a.grad_shard) st_stream(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
-        adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        adam8(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
         st_stream(a.master + e, p0);
         st_stream(a.master + e + 4, p1);
         st_stream(a.m + e, m0);
@@ -214,51 +224,59 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) {
     // drain the bulk copies already issued before the CTA's memory goes away
-    const int issued = *issued_flag;
-    for (int s = 0; s < stages && s < issued; ++s) {
-      const int last = ((issued - 1 - s) / stages) * stages + s;  // last tile on stage s
-      if (!mbar_wait(&full[s], (unsigned)(last / stages) & 1u)) atomicOr(a.ns.error, 4u);
-    }
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
-  norm_epilogue<kTmaThreads>(a.ns, sq, nf, a.accumulate);
+  norm_epilogue<tma_threads<G>()>(a.ns, sq, nf, a.accumulate);
+}
+
+size_t tma_smem_bytes(int n_ranks, int stages) {
+  return (size_t)stages * tma_stage_bytes(n_ranks) + 2 * stages * sizeof(uint64_t) + 4 * (stages + 1);
 }
 
 template <int MODE>
-cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, cudaStream_t s) {
-  const size_t bytes = (size_t)stages * tma_stage_bytes(a.n_ranks) + 2 * stages * sizeof(uint64_t) + 16;
-  fused_step_tma_kernel<MODE><<<grid, kTmaThreads, bytes, s>>>(a, stages);
+cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, int groups, cudaStream_t s) {
+  const size_t bytes = tma_smem_bytes(a.n_ranks, stages);
+  if (groups == 2)
+    fused_step_tma_kernel<MODE, 2><<<grid, tma_threads<2>(), bytes, s>>>(a, stages);
+  else
+    fused_step_tma_kernel<MODE, 1><<<grid, tma_threads<1>(), bytes, s>>>(a, stages);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+template <class K>
+static cudaError_t opt_in(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+}
+
 cudaError_t tma_configure() {
   cudaError_t e = cudaSuccess;
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fused_step_tma_kernel<kFusedZ3>, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 1>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 1>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 1>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 2>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 2>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 2>);
   return e;
 }
 
-int tma_stages_for(int n_ranks) {
-  if (n_ranks < 1 || n_ranks > kTmaMaxRanks) return 0;
-  const size_t per = tma_stage_bytes(n_ranks) + 2 * sizeof(uint64_t);
-  int stages = (int)((kTmaMaxSmem - 16) / per);
-  if (stages > 4) stages = 4;
-  stages -= stages % kGroups;  // each consumer group owns stages g, g+2, ...
+int tma_stages_for(int n_ranks, int groups) {
+  if (n_ranks < 1 || n_ranks > kTmaMaxRanks || (groups != 1 && groups != 2)) return 0;
+  int stages = 4;
+  while (stages > 0 && tma_smem_bytes(n_ranks, stages) > (size_t)kTmaMaxSmem) --stages;
+  stages -= stages % groups;  // every stage belongs to one consumer group
   return stages >= 2 ? stages : 0;
 }
 
-cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
-  const int stages = tma_stages_for(a.n_ranks);
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, cudaStream_t s) {
+  const int stages = tma_stages_for(a.n_ranks, groups);
   if (stages == 0) return cudaErrorInvalidValue;
   switch (mode) {
-    case kFusedZ1: return launch_tma_mode<kFusedZ1>(a, grid, stages, s);
-    case kFusedZ2: return launch_tma_mode<kFusedZ2>(a, grid, stages, s);
-    case kFusedZ3: return launch_tma_mode<kFusedZ3>(a, grid, stages, s);
+    case kFusedZ1: return launch_tma_mode<kFusedZ1>(a, grid, stages, groups, s);
+    case kFusedZ2: return launch_tma_mode<kFusedZ2>(a, grid, stages, groups, s);
+    case kFusedZ3: return launch_tma_mode<kFusedZ3>(a, grid, stages, groups, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -101,9 +101,10 @@ cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
-// Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM.
-cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, cudaStream_t s);
-int tma_stages_for(int n_ranks);   // 0 when N is out of its range
+// Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with
+// `groups` (1 or 2) producer/consumer groups.
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, cudaStream_t s);
+int tma_stages_for(int n_ranks, int groups);  // 0 when N (or groups) is out of range
 cudaError_t tma_configure();       // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.

@@ -34,9 +34,11 @@ struct zero_ctx {
   int32_t stage = 0;
   // options
   bool keep_grad_shards = true;
+  bool grad_buffers = true;
   int64_t replica_pad = 0;
   int blocks_per_sm_opt = 0;
   int kernel_opt = ZERO_KERNEL_AUTO;
+  int tma_groups_opt = 0;  // 0 = the library's choice
   // arena layout (bytes)
   int64_t arena_bytes[ZERO_NUM_ARENAS] = {};
   int64_t state_pitch = 0;   // bytes between master, m and v
@@ -116,6 +118,7 @@ void compute_layout(zero_ctx* c) {
       c->arena_bytes[ZERO_ARENA_GATHER] = N * c->gather_pitch;
       break;
   }
+  if (!c->grad_buffers) c->arena_bytes[ZERO_ARENA_GRADS] = 0;
 }
 
 float* master_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_STATES]); }
@@ -166,9 +169,15 @@ zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
 constexpr size_t kMaxTimed = 4096;
 constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the staged kernel
 
+// Consumer groups of the staged kernel for this context.
+int tma_groups(const zero_ctx* c) {
+  if (c->tma_groups_opt) return c->tma_groups_opt;
+  return zsm::tma_stages_for(c->plan.n_ranks, 2) > 0 ? 2 : 1;
+}
+
 // Whether the fused step runs the shared-memory staged kernel.
 bool use_tma(const zero_ctx* c) {
-  if (zsm::tma_stages_for(c->plan.n_ranks) == 0) return false;
+  if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c)) == 0) return false;
   if (c->kernel_opt == ZERO_KERNEL_TMA) return true;
   if (c->kernel_opt == ZERO_KERNEL_REGISTER) return false;
   return false;  // AUTO
@@ -261,7 +270,8 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   cudaError_t e;
   if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
-    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)), s);
+    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
+                              tma_groups(c), s);
   } else {
     e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
   }
@@ -313,6 +323,8 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
         return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
   } else if (!fn && c->stage != ZERO_STAGE_1) {
     return fail(c, ZERO_EINVAL, "grad_fn may be NULL only for stage 1");
+  } else if (!c->arena[ZERO_ARENA_GRADS]) {
+    return fail(c, ZERO_ESTATE, "no gradient buffers (ZERO_OPT_GRAD_BUFFERS = 0): use zero_step_resident");
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t t = c->t + 1;
@@ -388,9 +400,16 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   }
   if (key == ZERO_OPT_KERNEL) {
     if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_TMA) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
-    if (value == ZERO_KERNEL_TMA && zsm::tma_stages_for(c->plan.n_ranks) == 0)
+    if (value == ZERO_KERNEL_TMA && zsm::tma_stages_for(c->plan.n_ranks, 1) == 0)
       return fail(c, ZERO_EINVAL, "the staged kernel handles N <= %d", zsm::kTmaMaxRanks);
     c->kernel_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_TMA_GROUPS) {
+    if (value < 0 || value > 2) return fail(c, ZERO_EINVAL, "consumer groups must be 0 (auto), 1 or 2");
+    if (value > 0 && zsm::tma_stages_for(c->plan.n_ranks, (int)value) == 0)
+      return fail(c, ZERO_EINVAL, "%lld consumer groups do not fit at N = %d", (long long)value, c->plan.n_ranks);
+    c->tma_groups_opt = (int)value;
     return ZERO_OK;
   }
   if (c->bound) return fail(c, ZERO_ESTATE, "options must be set before zero_bind");
@@ -402,6 +421,9 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
       if (value < 0 || value % kArenaAlign || value >= (1 << 20))
         return fail(c, ZERO_EINVAL, "replica pad must be a multiple of 256 below 1 MiB");
       c->replica_pad = value;
+      break;
+    case ZERO_OPT_GRAD_BUFFERS:
+      c->grad_buffers = value != 0;
       break;
     case ZERO_OPT_BLOCKS_PER_SM:
       if (value < 0 || value > 32) return fail(c, ZERO_EINVAL, "blocks per SM must be 0..32");
@@ -474,7 +496,7 @@ zero_status zero_bind(zero_ctx* c, void* const* arenas) {
   int fused_blocks = 0, simple_blocks = 0;
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
-  if (e == cudaSuccess && zsm::tma_stages_for(c->plan.n_ranks) > 0) e = zsm::tma_configure();
+  if (e == cudaSuccess && zsm::tma_stages_for(c->plan.n_ranks, 1) > 0) e = zsm::tma_configure();
   if (e != cudaSuccess) return cuda_fail(c, e, "device query");
   if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
   c->grid_fused = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, fused_blocks)));
@@ -552,6 +574,7 @@ zero_status zero_view(const zero_ctx* cc, int32_t what, int32_t rank, void** ptr
       *n_elems = P;
       break;
     case ZERO_VIEW_GRAD_BUF:
+      if (!c->arena[ZERO_ARENA_GRADS]) return fail(c, ZERO_EINVAL, "no gradient buffers (ZERO_OPT_GRAD_BUFFERS = 0)");
       *ptr = grad_buf_ptr(c, rank);
       *n_elems = c->stage == ZERO_STAGE_1 ? P : c->stage == ZERO_STAGE_2 ? c->plan.max_bucket : c->plan.max_layer;
       break;
@@ -601,6 +624,8 @@ zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void*
         return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
       a.grad[r] = static_cast<const uint16_t*>(rank_grads[r]);
     }
+  } else if (!c->arena[ZERO_ARENA_GRADS]) {
+    return fail(c, ZERO_EINVAL, "rank_grads is NULL but there are no gradient buffers");
   } else if (c->stage == ZERO_STAGE_2) {
     if (hi - lo > c->plan.max_bucket)
       return fail(c, ZERO_EINVAL, "[%lld, %lld) is larger than the bucket buffer", (long long)lo, (long long)hi);
@@ -632,6 +657,8 @@ zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
   const int N = c->plan.n_ranks;
   zsm::ReduceArgs a;
   std::memset(&a, 0, sizeof a);
+  if (!rank_grads && !c->arena[ZERO_ARENA_GRADS])
+    return fail(c, ZERO_EINVAL, "rank_grads is NULL but there are no gradient buffers");
   for (int r = 0; r < N; ++r) {
     const void* p = rank_grads ? rank_grads[r] : static_cast<const void*>(grad_buf_ptr(c, r) + lo);
     if (!p || !aligned16(p)) return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
@@ -659,6 +686,8 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
   if (t < 1) return fail(c, ZERO_EINVAL, "step t must be >= 1");
   if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
+  if (c->stage == ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRADS])
+    return fail(c, ZERO_ESTATE, "stage 1 Adam reads the gradient buffers, which were dropped");
   const zsm::AdamScalars sc = adam_scalars(c->hp, t);
   const int64_t S = c->plan.shard;
   const int r0 = rank < 0 ? 0 : rank, r1 = rank < 0 ? N : rank + 1;
