@@ -364,6 +364,50 @@ zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
  */
 zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, double* model_bytes);
 
+/*
+ * zero_fused_step_static -- one fused ZeRO-2 step over a single flat interval
+ * that allocates nothing.  The pages have no counterpart to this entry point:
+ * it exists for callers that cannot allocate device memory when they run the
+ * step -- code whose device memory is already entirely owned by another
+ * allocator (a framework's caching allocator that reserved the whole device,
+ * where an extra cudaMalloc fails or fragments that pool), latency-critical
+ * loops that cannot afford the device synchronisation cudaMalloc/cudaFree may
+ * cause, and one-off callers that keep no context object to hold a scratch
+ * arena.  Such a caller passes only the step's inputs and outputs:
+ *   rank_grads   host array of n_ranks device pointers, each to n bf16
+ *                gradient values of that rank (16-byte aligned)
+ *   master, exp_avg, exp_avg_sq
+ *                device fp32 arrays of n values, updated in place
+ *   rank_params  host array of n_ranks device pointers, each receiving the n
+ *                updated bf16 parameters (16-byte aligned)
+ *   hp, t        Adam hyper-parameters and the step number (t >= 1)
+ *   stats_out    NULL, or a device pointer to 16 bytes that receives the
+ *                step's sum of squares of the averaged gradient (double) and
+ *                its non-finite count (uint64)
+ * n must be a multiple of 8 and 1 <= n_ranks <= ZERO_MAX_RANKS.  The values
+ * computed are those of zero_step for a stage-2 context whose single bucket
+ * is this interval.
+ *
+ * The kernel's scratch (per-CTA norm partials, an arrival counter and the
+ * step's sums) is a 32 KiB + 64 B array in the library's device memory,
+ * reserved on every GPU that loads the library until the process exits; it
+ * holds partials for at most 2048 CTAs, and a launch that would need more
+ * returns ZERO_ENOMEM.  Every call on a device shares that array and it keeps
+ * the previous call's contents (the call clears what must start at zero), so
+ * two calls that may run at the same time on the GPU -- on different streams
+ * with no ordering between them -- race and give wrong statistics; calls
+ * ordered on one stream are safe.  The first call on each device looks up the
+ * array's device address with that device current (a one-time set-up); make
+ * that first call before any stream capture begins.
+ * Errors: ZERO_EINVAL (bad size, pointer, alignment or hyper-parameter),
+ * ZERO_ENOMEM (scratch too small for the launch), ZERO_ECUDA (set-up or launch
+ * failed).
+ */
+zero_status zero_fused_step_static(int32_t n_ranks, int64_t n, const void* const* rank_grads,
+                                   float* master, float* exp_avg, float* exp_avg_sq,
+                                   void* const* rank_params, const zero_adam_hparams* hp,
+                                   int64_t t, void* stats_out, void* stream);
+
 /* Synchronise `stream` and read the last step's statistics. */
 zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
 

@@ -101,6 +101,8 @@ _SIGS = {
     "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                   ctypes.POINTER(ctypes.c_double)]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
+    "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
+                                      ctypes.POINTER(zero_adam_hparams), _i64, _vp, _vp]),
     "zero_last_error": (ctypes.c_char_p, [_vp]),
     "zero_destroy": (None, [_vp]),
 }

@@ -11,7 +11,8 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["csrc/zero_api.cu", "csrc/kernels.cu", "csrc/fused_tma.cu", "csrc/plan.cpp"]
+SOURCES = ["csrc/zero_api.cu", "csrc/kernels.cu", "csrc/fused_tma.cu", "csrc/static_scratch.cu",
+           "csrc/plan.cpp"]
 LIB = os.path.join(HERE, "libzero_sm.so")
 
 NVCC_FLAGS = [
