@@ -127,7 +127,9 @@ enum {
                                     registers only and zero_reduce_scatter/zero_adam_shard
                                     return ZERO_ESTATE */
   ZERO_OPT_REPLICA_PAD = 2,      /* extra bytes (multiple of 256, < 1 MiB) between consecutive
-                                    rank buffers; default 0 */
+                                    buffers of an arena (rank replicas, master/m/v), to keep
+                                    streams that are read together off the same DRAM banks when
+                                    the buffers' lengths are large powers of two; default 0 */
   ZERO_OPT_BLOCKS_PER_SM = 3,    /* fused-kernel CTAs per SM (0 = occupancy maximum) */
   ZERO_OPT_TIMING = 4,           /* 1: record a CUDA event pair on the launching stream around
                                     every fused-step kernel launch (read with
@@ -138,8 +140,11 @@ enum {
   ZERO_OPT_GRAD_BUFFERS = 6,     /* 1 (default) sizes the GRADS arena; 0 drops it for callers
                                     that only use zero_step_resident and the calls given explicit
                                     pointers (zero_step then returns ZERO_ESTATE) */
-  ZERO_OPT_TMA_GROUPS = 7        /* staged kernel: producer/consumer groups per CTA, 1 or 2
+  ZERO_OPT_TMA_GROUPS = 7,       /* staged kernel: producer/consumer groups per CTA, 1 or 2
                                     (0 = the library's choice); may be set at any time */
+  ZERO_OPT_TMA_STAGES = 8        /* staged kernel: shared-memory ring depth, at most 8 and at
+                                    most what fits in 227 KB (0 = the library's choice); may be
+                                    set at any time */
 };
 
 /* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.

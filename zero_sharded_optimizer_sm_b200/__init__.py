@@ -41,6 +41,7 @@ ZERO_OPT_KEEP_GRAD_SHARDS, ZERO_OPT_REPLICA_PAD, ZERO_OPT_BLOCKS_PER_SM, ZERO_OP
 ZERO_KERNEL_AUTO, ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA = 0, 1, 2
 ZERO_OPT_GRAD_BUFFERS = 6
 ZERO_OPT_TMA_GROUPS = 7
+ZERO_OPT_TMA_STAGES = 8
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
 
@@ -151,7 +152,7 @@ class ZeroOptimizer:
                  bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
-                 device=None):
+                 tma_stages: int = 0, device=None):
         import torch
 
         self._torch = torch
@@ -183,6 +184,8 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_GRAD_BUFFERS, 0), "zero_set_option")
         if tma_groups:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_GROUPS, int(tma_groups)), "zero_set_option")
+        if tma_stages:
+            self._check(zero_set_option(ctx, ZERO_OPT_TMA_STAGES, int(tma_stages)), "zero_set_option")
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)

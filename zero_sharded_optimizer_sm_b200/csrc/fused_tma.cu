@@ -20,6 +20,8 @@
 // host sees ZERO_ECUDA instead of a hung GPU.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "device_math.cuh"
 #include "kernels.cuh"
 
@@ -262,16 +264,17 @@ cudaError_t tma_configure() {
   return e;
 }
 
-int tma_stages_for(int n_ranks, int groups) {
+int tma_stages_for(int n_ranks, int groups, int max_stages) {
   if (n_ranks < 1 || n_ranks > kTmaMaxRanks || (groups != 1 && groups != 2)) return 0;
-  int stages = 4;
+  int stages = max_stages > 0 ? std::min(max_stages, kTmaMaxStages) : kTmaDefaultStages;
   while (stages > 0 && tma_smem_bytes(n_ranks, stages) > (size_t)kTmaMaxSmem) --stages;
   stages -= stages % groups;  // every stage belongs to one consumer group
   return stages >= 2 ? stages : 0;
 }
 
-cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, cudaStream_t s) {
-  const int stages = tma_stages_for(a.n_ranks, groups);
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, int max_stages,
+                             cudaStream_t s) {
+  const int stages = tma_stages_for(a.n_ranks, groups, max_stages);
   if (stages == 0) return cudaErrorInvalidValue;
   switch (mode) {
     case kFusedZ1: return launch_tma_mode<kFusedZ1>(a, grid, stages, groups, s);

@@ -17,6 +17,8 @@ constexpr int kThreads = 256;    // threads per CTA for every kernel
 constexpr int kMaxGrid = 4096;   // upper bound on CTAs of a norm-reducing launch
 constexpr int kTmaMaxRanks = 16; // the shared-memory staged kernel handles N <= 16
 constexpr int kTmaMaxSmem = 227 * 1024 - 1024;  // dynamic smem cap (1 KB left for static)
+constexpr int kTmaMaxStages = 8;                // ring depth limit of the staged kernel
+constexpr int kTmaDefaultStages = 4;            // ring depth when the caller does not choose
 
 // Binary32 scalars of one Adam step, each rounded once from binary64 on the host.
 struct AdamScalars {
@@ -103,8 +105,10 @@ cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with
 // `groups` (1 or 2) producer/consumer groups.
-cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, cudaStream_t s);
-int tma_stages_for(int n_ranks, int groups);  // 0 when N (or groups) is out of range
+cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, int max_stages,
+                             cudaStream_t s);
+// Ring depth for N and `groups` (max_stages 0 = the default depth), 0 when out of range.
+int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
 cudaError_t tma_configure();       // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.

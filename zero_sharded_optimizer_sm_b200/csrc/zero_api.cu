@@ -39,6 +39,7 @@ struct zero_ctx {
   int blocks_per_sm_opt = 0;
   int kernel_opt = ZERO_KERNEL_AUTO;
   int tma_groups_opt = 0;  // 0 = the library's choice
+  int tma_stages_opt = 0;  // 0 = the library's choice
   // arena layout (bytes)
   int64_t arena_bytes[ZERO_NUM_ARENAS] = {};
   int64_t state_pitch = 0;   // bytes between master, m and v
@@ -91,7 +92,7 @@ void compute_layout(zero_ctx* c) {
   const zsm::Plan& p = c->plan;
   const int64_t N = p.n_ranks;
   const int64_t row2 = align_up(p.psi_pad * 2, kArenaAlign);
-  c->state_pitch = align_up(p.psi_pad * 4, kArenaAlign);
+  c->state_pitch = align_up(p.psi_pad * 4, kArenaAlign) + c->replica_pad;
   c->param_pitch = row2 + c->replica_pad;
   std::fill(c->arena_bytes, c->arena_bytes + ZERO_NUM_ARENAS, 0);
   c->arena_bytes[ZERO_ARENA_STATES] = 3 * c->state_pitch;
@@ -271,7 +272,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
     e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
-                              tma_groups(c), s);
+                              tma_groups(c), c->tma_stages_opt, s);
   } else {
     e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
   }
@@ -403,6 +404,11 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     if (value == ZERO_KERNEL_TMA && zsm::tma_stages_for(c->plan.n_ranks, 1) == 0)
       return fail(c, ZERO_EINVAL, "the staged kernel handles N <= %d", zsm::kTmaMaxRanks);
     c->kernel_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_TMA_STAGES) {
+    if (value < 0 || value > zsm::kTmaMaxStages) return fail(c, ZERO_EINVAL, "stages must be 0..%d", zsm::kTmaMaxStages);
+    c->tma_stages_opt = (int)value;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_TMA_GROUPS) {
