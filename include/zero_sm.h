@@ -142,9 +142,11 @@ enum {
                                     pointers (zero_step then returns ZERO_ESTATE) */
   ZERO_OPT_TMA_GROUPS = 7,       /* staged kernel: producer/consumer groups per CTA, 1 or 2
                                     (0 = the library's choice); may be set at any time */
-  ZERO_OPT_TMA_STAGES = 8        /* staged kernel: shared-memory ring depth, at most 8 and at
+  ZERO_OPT_TMA_STAGES = 8,       /* staged kernel: shared-memory ring depth, at most 8 and at
                                     most what fits in 227 KB (0 = the library's choice); may be
                                     set at any time */
+  ZERO_OPT_TMA_CTAS_PER_SM = 9   /* staged kernel: CTAs per SM, 1..4, capped by what fits in
+                                    shared memory (0 = the library's choice); any time */
 };
 
 /* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.
@@ -255,6 +257,22 @@ zero_status zero_set_hparams(zero_ctx* ctx, const zero_adam_hparams* hp);
  * parameter shards (stage 3), and resets the step counter to 0.
  */
 zero_status zero_load_master(zero_ctx* ctx, const float* master_dev, void* stream);
+
+/*
+ * Resume from a checkpoint, possibly taken with a different N or stage (the
+ * ownership map of [T] section "ZeRO-1" cuts the same flat vector into N
+ * segments, so a re-shard is a reload of the flat state).  master, exp_avg,
+ * exp_avg_sq: device arrays (16-byte aligned) holding the flat fp32 state of
+ * elements [0, n) -- e.g. copies of another context's ZERO_VIEW_MASTER /
+ * _EXP_AVG / _EXP_AVG_SQ; n must be a multiple of 8 that covers every real
+ * element (from the end of the last tensor's 8-element slot, which does not
+ * depend on N, up to psi_pad).  Elements [n, psi_pad) become 0.  Writes
+ * bf16(master) to the parameter replicas (stage 1, 2) or shards (stage 3),
+ * clears the reduced-gradient shards and sets the step counter to t, so the
+ * next step is t + 1.  The sources are read on `stream`.
+ */
+zero_status zero_import_state(zero_ctx* ctx, const float* master, const float* exp_avg,
+                              const float* exp_avg_sq, int64_t n, int64_t t, void* stream);
 
 /* Step counter: the t of the last update (0 after zero_load_master). */
 zero_status zero_get_step(const zero_ctx* ctx, int64_t* t);

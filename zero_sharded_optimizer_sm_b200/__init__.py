@@ -42,6 +42,7 @@ ZERO_KERNEL_AUTO, ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA = 0, 1, 2
 ZERO_OPT_GRAD_BUFFERS = 6
 ZERO_OPT_TMA_GROUPS = 7
 ZERO_OPT_TMA_STAGES = 8
+ZERO_OPT_TMA_CTAS_PER_SM = 9
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
 
@@ -86,6 +87,7 @@ _SIGS = {
     "zero_bind": (_i32, [_vp, _PTRS]),
     "zero_set_hparams": (_i32, [_vp, ctypes.POINTER(zero_adam_hparams)]),
     "zero_load_master": (_i32, [_vp, _vp, _vp]),
+    "zero_import_state": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _vp]),
     "zero_get_step": (_i32, [_vp, ctypes.POINTER(_i64)]),
     "zero_set_step": (_i32, [_vp, _i64]),
     "zero_view": (_i32, [_vp, _i32, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
@@ -152,7 +154,7 @@ class ZeroOptimizer:
                  bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
-                 tma_stages: int = 0, device=None):
+                 tma_stages: int = 0, tma_ctas_per_sm: int = 0, device=None):
         import torch
 
         self._torch = torch
@@ -186,6 +188,8 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_GROUPS, int(tma_groups)), "zero_set_option")
         if tma_stages:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_STAGES, int(tma_stages)), "zero_set_option")
+        if tma_ctas_per_sm:
+            self._check(zero_set_option(ctx, ZERO_OPT_TMA_CTAS_PER_SM, int(tma_ctas_per_sm)), "zero_set_option")
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
@@ -302,6 +306,18 @@ class ZeroOptimizer:
         if master is not None:
             assert master.dtype == self._torch.float32 and master.is_cuda and master.numel() == self.psi_pad
         self._check(zero_load_master(self.ctx, ptr, self._stream(stream)), "zero_load_master")
+
+    def export_state(self) -> dict:
+        """Copies of the flat fp32 state (psi_pad each) and the step counter."""
+        return dict(master=self.view(ZERO_VIEW_MASTER).clone(), exp_avg=self.view(ZERO_VIEW_EXP_AVG).clone(),
+                    exp_avg_sq=self.view(ZERO_VIEW_EXP_AVG_SQ).clone(), t=self.t)
+
+    def import_state(self, state: dict, stream=None):
+        """Resume from ``export_state()`` of any context over the same parameter list."""
+        n = min(int(state["master"].numel()), self.psi_pad)
+        self._check(zero_import_state(self.ctx, state["master"].data_ptr(), state["exp_avg"].data_ptr(),
+                                      state["exp_avg_sq"].data_ptr(), n, int(state["t"]),
+                                      self._stream(stream)), "zero_import_state")
 
     @property
     def t(self) -> int:

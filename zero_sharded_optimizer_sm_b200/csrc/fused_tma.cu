@@ -272,6 +272,19 @@ int tma_stages_for(int n_ranks, int groups, int max_stages) {
   return stages >= 2 ? stages : 0;
 }
 
+int tma_ctas_per_sm(int n_ranks, int groups, int max_stages) {
+  const int stages = tma_stages_for(n_ranks, groups, max_stages);
+  if (stages == 0) return 0;
+  const size_t bytes = tma_smem_bytes(n_ranks, stages);
+  int b = 0;
+  cudaError_t e = groups == 2
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 2>,
+                                                                      tma_threads<2>(), bytes)
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 1>,
+                                                                      tma_threads<1>(), bytes);
+  return e == cudaSuccess ? b : 0;
+}
+
 cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, int max_stages,
                              cudaStream_t s) {
   const int stages = tma_stages_for(a.n_ranks, groups, max_stages);

@@ -114,18 +114,24 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
   }
 }
 
+// Optimizer state from sources (fresh master weights with m = v = 0, or a
+// checkpoint's master/m/v), zeros past the sources, bf16(master) to every
+// parameter destination, reduced-gradient shards cleared.
 __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ InitArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
     const int64_t e = vi * kVec;
-    const float4 p0 = ld_stream(a.master_src + e), p1 = ld_stream(a.master_src + e + 4);
+    const bool src = vi < a.n_src_vec;
+    const float4 p0 = src ? ld_stream(a.master_src + e) : z, p1 = src ? ld_stream(a.master_src + e + 4) : z;
+    const float4 m0 = src && a.m_src ? ld_stream(a.m_src + e) : z, m1 = src && a.m_src ? ld_stream(a.m_src + e + 4) : z;
+    const float4 v0 = src && a.v_src ? ld_stream(a.v_src + e) : z, v1 = src && a.v_src ? ld_stream(a.v_src + e + 4) : z;
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
-    st_stream(a.m + e, z);
-    st_stream(a.m + e + 4, z);
-    st_stream(a.v + e, z);
-    st_stream(a.v + e + 4, z);
+    st_stream(a.m + e, m0);
+    st_stream(a.m + e + 4, m1);
+    st_stream(a.v + e, v0);
+    st_stream(a.v + e + 4, v1);
     const uint16_t h[kVec] = {to_bf16(p0.x), to_bf16(p0.y), to_bf16(p0.z), to_bf16(p0.w),
                               to_bf16(p1.x), to_bf16(p1.y), to_bf16(p1.z), to_bf16(p1.w)};
     const uint4 w = pack8(h);

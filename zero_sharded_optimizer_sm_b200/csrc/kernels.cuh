@@ -83,7 +83,10 @@ struct GatherArgs {
 };
 
 struct InitArgs {
-  const float* master_src;
+  const float* master_src;          // elements [0, n_src_vec*8) come from these sources,
+  const float* m_src;               // m and v are 0 where their source is nullptr,
+  const float* v_src;               // everything beyond the sources is 0
+  int64_t n_src_vec;
   float* master;
   float* m;
   float* v;
@@ -109,6 +112,8 @@ cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups,
                              cudaStream_t s);
 // Ring depth for N and `groups` (max_stages 0 = the default depth), 0 when out of range.
 int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
+// Resident CTAs per SM of the staged kernel in that configuration (0 on error).
+int tma_ctas_per_sm(int n_ranks, int groups, int max_stages);
 cudaError_t tma_configure();       // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.

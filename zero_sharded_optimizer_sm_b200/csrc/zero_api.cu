@@ -40,6 +40,9 @@ struct zero_ctx {
   int kernel_opt = ZERO_KERNEL_AUTO;
   int tma_groups_opt = 0;  // 0 = the library's choice
   int tma_stages_opt = 0;  // 0 = the library's choice
+  int tma_ctas_opt = 0;    // CTAs per SM of the staged kernel, 0 = the library's choice
+  int tma_grid_key = -1;   // configuration the cached grid cap belongs to
+  int tma_grid_cap = 0;
   // arena layout (bytes)
   int64_t arena_bytes[ZERO_NUM_ARENAS] = {};
   int64_t state_pitch = 0;   // bytes between master, m and v
@@ -176,6 +179,19 @@ int tma_groups(const zero_ctx* c) {
   return zsm::tma_stages_for(c->plan.n_ranks, 2) > 0 ? 2 : 1;
 }
 
+// CTAs of a staged-kernel launch: SMs x the CTAs per SM asked for (1 by
+// default), capped by what fits; cached per configuration.
+int tma_grid_cap(zero_ctx* c) {
+  const int want = c->tma_ctas_opt > 0 ? c->tma_ctas_opt : 1;
+  const int key = (tma_groups(c) * 16 + c->tma_stages_opt) * 64 + want;
+  if (key != c->tma_grid_key) {
+    const int fit = zsm::tma_ctas_per_sm(c->plan.n_ranks, tma_groups(c), c->tma_stages_opt);
+    c->tma_grid_cap = c->sm_count * std::max(1, std::min(want, fit));
+    c->tma_grid_key = key;
+  }
+  return c->tma_grid_cap;
+}
+
 // Whether the fused step runs the shared-memory staged kernel.
 bool use_tma(const zero_ctx* c) {
   if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c)) == 0) return false;
@@ -271,7 +287,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   cudaError_t e;
   if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
-    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
+    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, tma_grid_cap(c))),
                               tma_groups(c), c->tma_stages_opt, s);
   } else {
     e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
@@ -406,6 +422,11 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     c->kernel_opt = (int)value;
     return ZERO_OK;
   }
+  if (key == ZERO_OPT_TMA_CTAS_PER_SM) {
+    if (value < 0 || value > 4) return fail(c, ZERO_EINVAL, "CTAs per SM must be 0..4");
+    c->tma_ctas_opt = (int)value;
+    return ZERO_OK;
+  }
   if (key == ZERO_OPT_TMA_STAGES) {
     if (value < 0 || value > zsm::kTmaMaxStages) return fail(c, ZERO_EINVAL, "stages must be 0..%d", zsm::kTmaMaxStages);
     c->tma_stages_opt = (int)value;
@@ -522,16 +543,19 @@ zero_status zero_set_hparams(zero_ctx* c, const zero_adam_hparams* hp) {
   return ZERO_OK;
 }
 
-zero_status zero_load_master(zero_ctx* c, const float* master_dev, void* stream) {
-  if (!c) return ZERO_EINVAL;
-  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
-  if (master_dev && !aligned16(master_dev)) return fail(c, ZERO_EINVAL, "master_dev is not 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+namespace {
+
+// Fills the state from sources (see InitArgs) and resets the run state.
+zero_status load_state(zero_ctx* c, const float* master, const float* m, const float* v, int64_t n,
+                       int64_t t, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(c->arena[ZERO_ARENA_SCRATCH], 0, kScratchBytes, s);
   if (e != cudaSuccess) return cuda_fail(c, e, "clearing scratch");
   zsm::InitArgs a;
   std::memset(&a, 0, sizeof a);
-  a.master_src = master_dev ? master_dev : master_ptr(c);
+  a.master_src = master;
+  a.m_src = m;
+  a.v_src = v;
+  a.n_src_vec = n / zsm::kVec;
   a.master = master_ptr(c);
   a.m = m_ptr(c);
   a.v = v_ptr(c);
@@ -541,11 +565,35 @@ zero_status zero_load_master(zero_ctx* c, const float* master_dev, void* stream)
   a.n_vec = c->plan.psi_pad / zsm::kVec;
   e = zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s);
   if (e != cudaSuccess) return cuda_fail(c, e, "init kernel launch");
-  c->t = 0;
-  c->stats_step = 0;
+  c->t = t;
+  c->stats_step = t;
   c->loaded = true;
   c->norm_fresh = true;
   return ZERO_OK;
+}
+
+}  // namespace
+
+zero_status zero_load_master(zero_ctx* c, const float* master_dev, void* stream) {
+  if (!c) return ZERO_EINVAL;
+  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
+  if (master_dev && !aligned16(master_dev)) return fail(c, ZERO_EINVAL, "master_dev is not 16-byte aligned");
+  return load_state(c, master_dev ? master_dev : master_ptr(c), nullptr, nullptr, c->plan.psi_pad, 0,
+                    static_cast<cudaStream_t>(stream));
+}
+
+zero_status zero_import_state(zero_ctx* c, const float* master, const float* exp_avg, const float* exp_avg_sq,
+                              int64_t n, int64_t t, void* stream) {
+  if (!c) return ZERO_EINVAL;
+  if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
+  if (!aligned16(master) || !aligned16(exp_avg) || !aligned16(exp_avg_sq))
+    return fail(c, ZERO_EINVAL, "master, exp_avg and exp_avg_sq must be 16-byte aligned device pointers");
+  const int64_t flat = c->plan.start.back() + ((c->plan.numel.back() + zsm::kGranule - 1) / zsm::kGranule) * zsm::kGranule;
+  if (n % zsm::kGranule || n < flat || n > c->plan.psi_pad)
+    return fail(c, ZERO_EINVAL, "n = %lld must be a multiple of 8 in [%lld, %lld] (every real element, at most psi_pad)",
+                (long long)n, (long long)flat, (long long)c->plan.psi_pad);
+  if (t < 0) return fail(c, ZERO_EINVAL, "t must be >= 0");
+  return load_state(c, master, exp_avg, exp_avg_sq, n, t, static_cast<cudaStream_t>(stream));
 }
 
 zero_status zero_get_step(const zero_ctx* c, int64_t* t) {
