@@ -37,7 +37,8 @@ if ROOT not in sys.path:
 METRIC = "fused ZeRO step params/sec (1 B200); achieved HBM GB/s vs ~8 TB/s roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCE = os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc", "kernels.cu")
+KERNEL_SOURCES = [os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc", f)
+                  for f in ("kernels.cu", "fused_tma.cu", "device_math.cuh", "kernels.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
 
 
@@ -113,19 +114,24 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_for_current_kernel(stage: int, n_ranks: int, elems_per_launch: float):
-    """Per-launch DRAM bytes from the committed ncu summary, scaled to this
-    launch size, or None when the kernel source changed since the capture."""
+def kernel_sources_digest() -> str:
+    h = hashlib.sha256()
+    for path in KERNEL_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_for_current_kernel(key: str, elems_per_launch: float):
+    """Per-launch DRAM bytes from the committed ncu summary for this kernel
+    configuration, scaled to this launch size, or None when the kernel
+    sources changed since the capture (or there is no capture)."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
-        with open(KERNEL_SOURCE, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-        if d.get("kernels_cu_sha256") != digest:
+        if d.get("kernel_sources_sha256") != kernel_sources_digest():
             return None
-        key = f"stage{stage}_N{n_ranks}"
-        per_elem = d["dram_bytes_per_elem"][key]
-        return per_elem * elems_per_launch
+        return d["dram_bytes_per_elem"][key] * elems_per_launch
     except Exception:
         return None
 
@@ -291,7 +297,9 @@ def run_ours(args, world, rank, local):
     achieved = kt["model_bytes"] / max(1, launches) / (kernel_ms / 1e3) / 1e9 if launches else None
     peak, peak_kind = measured_peaks()
     elems_per_launch = w.psi / max(1, len(opt.buckets()))
-    traffic = traffic_for_current_kernel(2, w.n_ranks, elems_per_launch)
+    fc = opt.fused_config()
+    ckey = f"stage2_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
+    traffic = traffic_for_current_kernel(ckey, elems_per_launch)
 
     # end to end through the C ABI: every bucket's N gradient slices copied
     # from pinned host memory into the fixed-size buffer, then the fused
@@ -351,10 +359,12 @@ def run_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
-                   "kernel": args.kernel},
+                   "kernel": args.kernel, "fused_config": fc},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "peak_kind": f"{peak_kind} copy peak", "kernel": "fused_step_kernel",
+                     "peak_kind": f"{peak_kind} copy peak",
+                     "kernel": "fused_step_tma_kernel" if fc["kernel"] == "tma" else "fused_step_kernel",
+                     "kernel_config": ckey,
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
                      "model_bytes_per_launch": kt["model_bytes"] / max(1, launches),
                      "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None},

@@ -431,6 +431,11 @@ zero_status zero_fused_step_static(int32_t n_ranks, int64_t n, const void* const
                                    void* const* rank_params, const zero_adam_hparams* hp,
                                    int64_t t, void* stats_out, void* stream);
 
+/* The fused-step kernel this context launches: *kernel = ZERO_KERNEL_REGISTER
+ * or ZERO_KERNEL_TMA; for the staged kernel also its consumer groups and ring
+ * depth (0 otherwise).  Host only. */
+zero_status zero_fused_config(const zero_ctx* ctx, int32_t* kernel, int32_t* groups, int32_t* stages);
+
 /* Synchronise `stream` and read the last step's statistics. */
 zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
 

@@ -103,6 +103,7 @@ _SIGS = {
                                   ctypes.POINTER(zero_step_stats)]),
     "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                   ctypes.POINTER(ctypes.c_double)]),
+    "zero_fused_config": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
                                       ctypes.POINTER(zero_adam_hparams), _i64, _vp, _vp]),
@@ -388,6 +389,12 @@ class ZeroOptimizer:
             raise self._cb_error
         self._check(st, "zero_step_resident")
         return self._stats_dict(out) if stats else None
+
+    def fused_config(self) -> dict:
+        k, g, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        self._check(zero_fused_config(self.ctx, ctypes.byref(k), ctypes.byref(g), ctypes.byref(s)),
+                    "zero_fused_config")
+        return dict(kernel={1: "register", 2: "tma"}[k.value], groups=g.value, stages=s.value)
 
     def set_kernel(self, kernel: int):
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")

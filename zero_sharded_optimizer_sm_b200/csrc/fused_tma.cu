@@ -83,14 +83,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
   return true;
 }
 
+// L2 policy for the bulk loads: every input byte is read exactly once, so it
+// is marked first to evict and leaves L2 room for the write-back traffic.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // 1-D bulk copy global -> this CTA's shared memory, completion on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar,
+                                          uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
           smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+
+// Plain (write-back) 16-byte stores for the consumers' outputs; measured ~1 %
+// faster than streaming stores in this kernel on B200.
+__device__ __forceinline__ void st_out(uint16_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
+__device__ __forceinline__ void st_out(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
 __host__ __device__ inline unsigned tma_stage_bytes(int n_ranks) {
   return (unsigned)(kTile * (2 * n_ranks + 12));
@@ -135,6 +149,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
     // ---------------------------------------------------------- producer --
     if (lane == 0) {
       const int g = warp;
+      const uint64_t policy = evict_first_policy();
       for (int it = g;; it += G) {
         const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
         if (tile >= n_tiles) break;
@@ -151,11 +166,11 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         unsigned char* st = smem + (size_t)s * stage_bytes;
         mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
         for (int r = 0; r < N; ++r)
-          bulk_load(st + (size_t)r * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s]);
+          bulk_load(st + (size_t)r * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
         unsigned char* stt = st + (size_t)N * 2 * kTile;
-        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &full[s]);
-        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &full[s]);
-        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s]);
+        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
         last_k[s] = (int)k;
       }
     }
@@ -206,20 +221,20 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         mean_bf16(acc, a.inv_n, g16, gv, sq, nf);
         if (MODE == kFusedZ1) {
           const uint4 gw = pack8(g16);
-          for (int r = 0; r < N; ++r) st_stream(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+          for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         }
-        if (a.grad_shard) st_stream(a.grad_shard + e, pack8(g16));
+        if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
         adam8(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
-        st_stream(a.master + e, p0);
-        st_stream(a.master + e + 4, p1);
-        st_stream(a.m + e, m0);
-        st_stream(a.m + e + 4, m1);
-        st_stream(a.v + e, v0);
-        st_stream(a.v + e + 4, v1);
+        st_out(a.master + e, p0);
+        st_out(a.master + e + 4, p1);
+        st_out(a.m + e, m0);
+        st_out(a.m + e + 4, m1);
+        st_out(a.v + e, v0);
+        st_out(a.v + e + 4, v1);
         const uint4 pw = pack8(p16);
-        if (MODE == kFusedZ3) st_stream(a.param_shard + e, pw);
-        for (int r = 0; r < N; ++r) st_stream(a.out[r] + e, pw);
+        if (MODE == kFusedZ3) st_out(a.param_shard + e, pw);
+        for (int r = 0; r < N; ++r) st_out(a.out[r] + e, pw);
       }
     }
   }

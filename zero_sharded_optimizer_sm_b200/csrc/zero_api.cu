@@ -173,19 +173,42 @@ zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
 constexpr size_t kMaxTimed = 4096;
 constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the staged kernel
 
+// Staged-kernel configuration chosen for N (consumer groups, ring depth),
+// measured on B200 with flat 256M-element buffers and the 1.2B-parameter
+// transformer list: few bytes per element (N <= 4) leave the consumers
+// compute-bound, so two groups win; at N = 5..8 one group with a two-deep
+// ring keeps the fewest copies in flight and moves the most bytes; N = 9..16
+// only fits two stages.  The register kernel wins beyond N = 16 (the staged
+// one does not apply there).
+struct TmaChoice {
+  int groups, stages;
+};
+
+TmaChoice tma_policy(int n_ranks) {
+  if (n_ranks <= 2) return {2, 4};
+  if (n_ranks <= 4) return {2, 2};
+  if (n_ranks <= 8) return {1, 2};
+  return {2, 2};
+}
+
 // Consumer groups of the staged kernel for this context.
 int tma_groups(const zero_ctx* c) {
   if (c->tma_groups_opt) return c->tma_groups_opt;
-  return zsm::tma_stages_for(c->plan.n_ranks, 2) > 0 ? 2 : 1;
+  return tma_policy(c->plan.n_ranks).groups;
+}
+
+int tma_stages(const zero_ctx* c) {
+  if (c->tma_stages_opt) return c->tma_stages_opt;
+  return tma_policy(c->plan.n_ranks).stages;
 }
 
 // CTAs of a staged-kernel launch: SMs x the CTAs per SM asked for (1 by
 // default), capped by what fits; cached per configuration.
 int tma_grid_cap(zero_ctx* c) {
   const int want = c->tma_ctas_opt > 0 ? c->tma_ctas_opt : 1;
-  const int key = (tma_groups(c) * 16 + c->tma_stages_opt) * 64 + want;
+  const int key = (tma_groups(c) * 16 + tma_stages(c)) * 64 + want;
   if (key != c->tma_grid_key) {
-    const int fit = zsm::tma_ctas_per_sm(c->plan.n_ranks, tma_groups(c), c->tma_stages_opt);
+    const int fit = zsm::tma_ctas_per_sm(c->plan.n_ranks, tma_groups(c), tma_stages(c));
     c->tma_grid_cap = c->sm_count * std::max(1, std::min(want, fit));
     c->tma_grid_key = key;
   }
@@ -194,10 +217,10 @@ int tma_grid_cap(zero_ctx* c) {
 
 // Whether the fused step runs the shared-memory staged kernel.
 bool use_tma(const zero_ctx* c) {
-  if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c)) == 0) return false;
+  if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c), tma_stages(c)) == 0) return false;
   if (c->kernel_opt == ZERO_KERNEL_TMA) return true;
   if (c->kernel_opt == ZERO_KERNEL_REGISTER) return false;
-  return false;  // AUTO
+  return true;  // AUTO: the staged kernel wherever it applies (N <= 16)
 }
 
 // Bytes one element moves through HBM in the fused step (the byte model).
@@ -288,7 +311,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
     e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, tma_grid_cap(c))),
-                              tma_groups(c), c->tma_stages_opt, s);
+                              tma_groups(c), tma_stages(c), s);
   } else {
     e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
   }
@@ -894,6 +917,20 @@ zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, doubl
     cudaError_t e = cudaMemcpy(&err, norm_scratch(c).error, sizeof err, cudaMemcpyDeviceToHost);
     if (e != cudaSuccess) return cuda_fail(c, e, "reading the device error word");
     return check_device_error(c, err, nullptr);
+  }
+  return ZERO_OK;
+}
+
+zero_status zero_fused_config(const zero_ctx* c, int32_t* kernel, int32_t* groups, int32_t* stages) {
+  if (!c || !kernel || !groups || !stages) return ZERO_EINVAL;
+  if (use_tma(c)) {
+    *kernel = ZERO_KERNEL_TMA;
+    *groups = tma_groups(c);
+    *stages = zsm::tma_stages_for(c->plan.n_ranks, *groups, tma_stages(c));
+  } else {
+    *kernel = ZERO_KERNEL_REGISTER;
+    *groups = 0;
+    *stages = 0;
   }
   return ZERO_OK;
 }
