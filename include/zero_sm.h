@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SM_VERSION 1
+#define ZERO_SM_VERSION 2
 #define ZERO_MAX_RANKS 128
 
 typedef enum zero_status {
@@ -116,6 +116,8 @@ typedef struct zero_step_stats {
   int64_t step;            /* Adam step number t the statistics belong to */
   int64_t comm_elems[3];   /* logical elements each rank sends per step: all-reduce,
                               reduce-scatter, all-gather (ring convention) */
+  double clip_coef;        /* gradient scale the update used (1 = none; zero_set_clip) */
+  int64_t skipped;         /* 1 when the step was skipped for non-finite gradients */
 } zero_step_stats;
 
 /* Options (zero_set_option, before zero_bind). */
@@ -297,6 +299,26 @@ zero_status zero_state_bytes(const zero_ctx* ctx, int32_t rank, int64_t out[3]);
 zero_status zero_comm_elems(const zero_ctx* ctx, int64_t out[3]);
 
 /* ------------------------------------------------ the step and its parts -- */
+/*
+ * Optional global-norm clipping and overflow skip.  Not on the pages (they
+ * describe no clipping); the conventions of mixed-precision training:
+ *   max_norm > 0     the update uses g * c with c = fp32(max_norm / (||g|| +
+ *                    1e-6)) (the quotient in binary64) whenever c < 1, where
+ *                    ||g|| is the fp64 norm of the whole averaged gradient;
+ *   skip_nonfinite   a step whose averaged gradient holds an Inf or NaN
+ *                    changes no state and does not advance the step counter.
+ * With either enabled the step needs the norm before any update, so zero_step
+ * and zero_step_resident run two passes: every interval is reduced first
+ * (stage 2/3 into the reduced-gradient shards, which must be kept; stage 1
+ * into the replicas, the all-reduce), the stream is synchronised once to read
+ * the norm, and a second kernel runs Adam and the broadcast (per layer at
+ * stage 3, with gather_fn as before).  Bytes per element at stage 2:
+ * (2N+2) + (2+24+2N) = 4N+28.  max_norm = 0 and skip_nonfinite = 0 (the
+ * default) restore the single fused pass.
+ */
+zero_status zero_set_clip(zero_ctx* ctx, double max_norm, int32_t skip_nonfinite);
+
+
 
 /*
  * Reduce-scatter of [lo, hi) ([T] section "ZeRO-2", part on reduce-scatter;

@@ -75,6 +75,8 @@ def _load():
         lib.zo_adam_scalars.argtypes = [f64, f64, f64, f64, f64, i64, vp]
         lib.zo_adam.restype = None
         lib.zo_adam.argtypes = [i64, vp, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
+        lib.zo_adam_coef.restype = None
+        lib.zo_adam_coef.argtypes = [i64, vp, f32, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
         lib.zo_sumsq.restype = ctypes.c_double
         lib.zo_sumsq.argtypes = [i64, vp]
         lib.zo_count_nonfinite.restype = i64
@@ -159,6 +161,31 @@ def adam(g: np.ndarray, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: Ad
         _load().zo_adam(n, g.ctypes.data, master.ctypes.data, m.ctypes.data, v.ctypes.data,
                         out.ctypes.data, hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t)
     return out
+
+
+def adam_coef(g: np.ndarray, coef: float, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: AdamHP,
+              t: int) -> np.ndarray:
+    """Adam with the averaged gradient scaled by a clipping coefficient
+    (applied only when coef < 1)."""
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    n = g.size
+    assert master.size == n and m.size == n and v.size == n
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().zo_adam_coef(n, g.ctypes.data, float(np.float32(coef)), master.ctypes.data, m.ctypes.data,
+                             v.ctypes.data, out.ctypes.data, hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t)
+    return out
+
+
+CLIP_EPS = 1e-6
+
+
+def clip_coef(grad_norm: float, max_norm: float) -> float:
+    """Global-norm clipping coefficient (not on the pages; the usual
+    convention): c = max_norm / (norm + 1e-6) in binary64, rounded once to
+    binary32; 1 when that is not below 1 (no clipping)."""
+    c = float(np.float32(max_norm / (grad_norm + CLIP_EPS)))
+    return c if c < 1.0 else 1.0
 
 
 def sumsq(g: np.ndarray) -> float:
@@ -337,6 +364,8 @@ class StepReport:
     grad_norm: float
     nonfinite: int
     gathered: Optional[List[List[np.ndarray]]] = None  # Z3: per layer (schedule order), per rank
+    skipped: bool = False
+    coef: float = 1.0
 
 
 def init_states(plan_: Plan, stage: int, master0: np.ndarray) -> List[RankState]:
@@ -360,11 +389,26 @@ def init_states(plan_: Plan, stage: int, master0: np.ndarray) -> List[RankState]
 
 
 def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
-         hp: AdamHP) -> StepReport:
-    """One optimizer step, t >= 1, following the pages' flow for ``stage``."""
+         hp: AdamHP, clip_norm: float = 0.0, skip_nonfinite: bool = False) -> StepReport:
+    """One optimizer step, t >= 1, following the pages' flow for ``stage``:
+    every gradient is reduced (and scattered) first, then each rank updates
+    what it owns, then the parameters are gathered.
+
+    Options that are not on the pages (a global-norm clip and an overflow
+    skip): the norm of the whole averaged gradient is known after the
+    reduction, before any update.  With ``skip_nonfinite`` a step whose
+    averaged gradient holds an Inf or NaN changes no state (the caller does not
+    advance t); with ``clip_norm`` > 0 every rank's Adam uses the gradient
+    times clip_coef(norm, clip_norm)."""
     N, S = plan_.n_ranks, plan_.shard
     local = [grads(t, r).astype(np.uint16, copy=True) for r in range(N)]
     assert all(a.size == plan_.psi_pad for a in local)
+
+    def update(g, st):
+        if coef < 1.0:
+            return adam_coef(g, coef, st.master, st.m, st.v, hp, t)
+        return adam(g, st.master, st.m, st.v, hp, t)
+
     if stage in (STAGE_DP, STAGE_Z1):
         # backward ends with a full all-reduce; every rank keeps the full grad
         for lo, hi in plan_.buckets:
@@ -372,37 +416,40 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
         for r in range(N):
             ranks[r].grads = local[r]
         g_full = local[0]
-        if stage == STAGE_DP:
-            # every rank runs the identical update on its full replica
-            for r in range(N):
-                ranks[r].params = adam(local[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t)
+    else:
+        shards = [np.zeros(S, dtype=np.uint16) for _ in range(N)]
+        if stage == STAGE_Z2:
+            # layer-by-layer reduce-scatter through the fixed-size buffer
+            for lo, hi in plan_.buckets:
+                reduce_scatter(local, plan_, lo, hi, shards)
         else:
-            # each rank updates only its owned shard, then all-gather
-            new_shards = []
-            for r in range(N):
-                lo, hi = plan_.owned(r)
-                new_shards.append(adam(local[r][lo:hi], ranks[r].master, ranks[r].m, ranks[r].v, hp, t))
-            all_gather(new_shards, plan_, 0, plan_.psi_pad, [ranks[r].params for r in range(N)])
-        return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full))
-    shards = [np.zeros(S, dtype=np.uint16) for _ in range(N)]
-    if stage == STAGE_Z2:
-        # layer-by-layer reduce-scatter through the fixed-size buffer
-        for lo, hi in plan_.buckets:
-            reduce_scatter(local, plan_, lo, hi, shards)
-        new_shards = []
+            # per layer, last to first: reduce-scatter the layer's gradient
+            for _, lo, hi in reversed(plan_.layers):
+                reduce_scatter(local, plan_, lo, hi, shards)
         for r in range(N):
             ranks[r].grads = shards[r]
-            new_shards.append(adam(shards[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t))
-        all_gather(new_shards, plan_, 0, plan_.psi_pad, [ranks[r].params for r in range(N)])
         g_full = np.concatenate(shards)
-        return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full))
+    norm = float(np.sqrt(sumsq(g_full)))
+    nonfinite = count_nonfinite(g_full)
+    if skip_nonfinite and nonfinite > 0:
+        return StepReport(grad_norm=norm, nonfinite=nonfinite, skipped=True)
+    coef = clip_coef(norm, clip_norm) if clip_norm > 0 else 1.0
+    if stage == STAGE_DP:
+        # every rank runs the identical update on its full replica
+        for r in range(N):
+            ranks[r].params = update(local[r], ranks[r])
+        return StepReport(grad_norm=norm, nonfinite=nonfinite, coef=coef)
+    if stage in (STAGE_Z1, STAGE_Z2):
+        # each rank updates only its owned shard, then all-gather
+        new_shards = []
+        for r in range(N):
+            lo, hi = plan_.owned(r)
+            new_shards.append(update(ranks[r].grads[lo:hi] if stage == STAGE_Z1 else ranks[r].grads, ranks[r]))
+        all_gather(new_shards, plan_, 0, plan_.psi_pad, [ranks[r].params for r in range(N)])
+        return StepReport(grad_norm=norm, nonfinite=nonfinite, coef=coef)
     assert stage == STAGE_Z3
-    # per layer, last to first: reduce-scatter the layer's gradient
-    for _, lo, hi in reversed(plan_.layers):
-        reduce_scatter(local, plan_, lo, hi, shards)
     for r in range(N):
-        ranks[r].grads = shards[r]
-        ranks[r].params = adam(shards[r], ranks[r].master, ranks[r].m, ranks[r].v, hp, t)
+        ranks[r].params = update(ranks[r].grads, ranks[r])
     # per layer, the all-gather of the updated shards into a temporary
     # full-layer buffer on every rank, released after use
     gathered = []
@@ -410,14 +457,22 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
         tmp = [np.zeros(hi - lo, dtype=np.uint16) for _ in range(N)]
         all_gather([ranks[r].params for r in range(N)], plan_, lo, hi, tmp, out_base=lo)
         gathered.append(tmp)
-    g_full = np.concatenate(shards)
-    return StepReport(grad_norm=float(np.sqrt(sumsq(g_full))), nonfinite=count_nonfinite(g_full),
-                      gathered=gathered)
+    return StepReport(grad_norm=norm, nonfinite=nonfinite, gathered=gathered, coef=coef)
 
 
-def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int, hp: AdamHP):
+def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int, hp: AdamHP,
+        clip_norm: float = 0.0, skip_nonfinite: bool = False):
+    """``steps`` optimizer steps; gradients for call k come from grads(k, r).
+    A skipped step does not advance the Adam step counter t, so the Adam
+    step number of call k is 1 + (calls before it that were not skipped)."""
     ranks = init_states(plan_, stage, master0)
-    reports = [step(plan_, stage, ranks, grads, t, hp) for t in range(1, steps + 1)]
+    reports = []
+    t = 0
+    for k in range(1, steps + 1):
+        rep = step(plan_, stage, ranks, lambda _t, r, k=k: grads(k, r), t + 1, hp, clip_norm, skip_nonfinite)
+        if not rep.skipped:
+            t += 1
+        reports.append(rep)
     return ranks, reports
 
 

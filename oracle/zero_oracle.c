@@ -193,6 +193,46 @@ void zo_adam(int64_t n, const uint16_t* g, float* master, float* m, float* v, ui
   }
 }
 
+/*
+ * The same Adam update with the averaged gradient scaled first by a
+ * global-norm clipping coefficient: g_used = fp32(g) * coef (one binary32
+ * rounding) when coef < 1, g_used = fp32(g) otherwise (coef >= 1 means the
+ * norm is within the limit and nothing is scaled).  Not on the pages: the
+ * optional clipping of a mixed-precision step; see the oracle's clip_coef
+ * for the coefficient.
+ */
+void zo_adam_coef(int64_t n, const uint16_t* g, float coef, float* master, float* m, float* v,
+                  uint16_t* p_out, double lr, double beta1, double beta2, double eps,
+                  double weight_decay, int64_t t) {
+  float s[9];
+  zo_adam_scalars(lr, beta1, beta2, eps, weight_decay, t, s);
+  const float b1 = s[0], b2 = s[1], omb1 = s[2], omb2 = s[3], bc1 = s[4], bc2 = s[5];
+  const float decay = s[6], lr_f = s[7], eps_f = s[8];
+  for (int64_t i = 0; i < n; ++i) {
+    float gi = zo_bf16_to_f32(g[i]);
+    if (coef < 1.0f) gi = gi * coef;
+    float p = master[i];
+    p = p * decay;
+    float a = b1 * m[i];
+    float b = omb1 * gi;
+    const float mi = a + b;
+    const float gg = gi * gi;
+    a = b2 * v[i];
+    b = omb2 * gg;
+    const float vi = a + b;
+    const float mh = mi / bc1;
+    const float vh = vi / bc2;
+    const float den = sqrtf(vh) + eps_f;
+    const float ratio = mh / den;
+    const float upd = lr_f * ratio;
+    p = p - upd;
+    master[i] = p;
+    m[i] = mi;
+    v[i] = vi;
+    if (p_out) p_out[i] = zo_bf16_rne(p);
+  }
+}
+
 /* ----------------------------------------------- gradient norm / overflow ---- */
 
 /* Sum of squares of the averaged bf16 gradient, in binary64, index order.

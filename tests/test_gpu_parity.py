@@ -597,3 +597,78 @@ def test_checkpoint_resume_and_reshard():
         assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), c.view(z.ZERO_VIEW_PARAM, r))
     for o in (a, b, c):
         o.close()
+
+
+# ------------------------------------------------------------- clip / skip ----
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_clip_and_overflow_skip_against_oracle(stage):
+    """Two-pass step: clip at a norm the gradients exceed, and skip a step
+    whose gradients hold an Inf (planted in call 2, rank 1).  Every element,
+    every step's statistics, and the step counter against the oracle."""
+    z = _z()
+    numel, layer = W.transformer_layers(2, 64, 256)
+    n_ranks, bucket, clip = 4, 8192, 0.05
+    dist = synth.Dist(synth.NORMAL, 1e-2, zero_mod=11)
+    hp = W.Hyper(weight_decay=0.01)
+    w = W.Workload("clip", numel, layer, n_ranks, (stage,), bucket, dist, W.MASTER_DIST, 3, hp, 0xC1 + stage)
+    p = oracle.plan(numel, layer, n_ranks, bucket)
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def host_grad(k, r):
+        g = W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, k, r), dist)
+        if k == 2 and r == 1:
+            g[7] = 0x7F80
+        return g
+
+    ranks, reps = oracle.run(p, STAGE_OF[stage], m0, host_grad, 3, oracle.AdamHP(**hp.__dict__),
+                             clip_norm=clip, skip_nonfinite=True)
+    assert [r.skipped for r in reps] == [False, True, False] and reps[0].coef < 1.0
+    opt = z.ZeroOptimizer(numel, layer, n_ranks, stage, bucket_elems=bucket, hparams=_hp(w))
+    opt.load_master(torch.from_numpy(m0).cuda())
+    opt.set_clip(clip, True)
+    call = [0]
+
+    def gfn(t, lo, hi, bufs, stream):
+        for r, ptr in enumerate(bufs):
+            opt._tensor_at(ptr, hi - lo, torch.int16).copy_(
+                torch.from_numpy(host_grad(call[0], r)[lo:hi].view(np.int16)))
+        return 0
+
+    for k in range(1, 4):
+        call[0] = k
+        st = opt.step(gfn, stats=True)
+        rep = reps[k - 1]
+        assert st["skipped"] == rep.skipped and st["nonfinite"] == rep.nonfinite
+        assert st["clip_coef"] == (rep.coef if not rep.skipped else 1.0)
+        assert st["grad_norm"] == rep.grad_norm or math.isclose(
+            st["grad_norm"], rep.grad_norm, rel_tol=norm_tol(p.psi_pad))
+    assert opt.t == 2
+    ref = oracle.full_view(p, STAGE_OF[stage], ranks)
+    for name, what in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(opt.view(what)), ref[name], f"clip stage {stage} {name}")
+    for r in (range(n_ranks) if stage != 3 else [0]):
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM, r)), ref["params"], f"clip stage {stage} params {r}")
+    opt.close()
+
+
+def test_inactive_clip_two_pass_equals_fused_step():
+    z = _z()
+    numel, layer = W.transformer_layers(2, 64, 256)
+    w = W.Workload("clip-off", numel, layer, 8, (2,), 16384, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 3,
+                   W.Hyper(), 0xC9)
+    a, fa = make_opt(w, 2, bucket=16384)
+    b, fb = make_opt(w, 2, bucket=16384)
+    b.set_clip(1e9, True)
+    ga, gb = grad_fn_for(a, fa), grad_fn_for(b, fb)
+    for _ in range(3):
+        sa = a.step(ga, stats=True)
+        sb = b.step(gb, stats=True)
+        assert sb["clip_coef"] == 1.0 and not sb["skipped"]
+        assert math.isclose(sa["grad_norm"], sb["grad_norm"], rel_tol=1e-12)
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(a.view(what), b.view(what))
+    for r in range(8):
+        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+    a.close()
+    b.close()

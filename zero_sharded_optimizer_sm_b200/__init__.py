@@ -66,7 +66,7 @@ class zero_sizes(ctypes.Structure):
 
 class zero_step_stats(ctypes.Structure):
     _fields_ = [("grad_norm", ctypes.c_double), ("nonfinite", ctypes.c_int64), ("step", ctypes.c_int64),
-                ("comm_elems", ctypes.c_int64 * 3)]
+                ("comm_elems", ctypes.c_int64 * 3), ("clip_coef", ctypes.c_double), ("skipped", ctypes.c_int64)]
 
 
 zero_grad_fn = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
@@ -103,6 +103,7 @@ _SIGS = {
                                   ctypes.POINTER(zero_step_stats)]),
     "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                   ctypes.POINTER(ctypes.c_double)]),
+    "zero_set_clip": (_i32, [_vp, ctypes.c_double, _i32]),
     "zero_fused_config": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
@@ -334,7 +335,7 @@ class ZeroOptimizer:
     @staticmethod
     def _stats_dict(s: zero_step_stats) -> dict:
         return dict(grad_norm=s.grad_norm, nonfinite=int(s.nonfinite), step=int(s.step),
-                    comm_elems=tuple(s.comm_elems))
+                    comm_elems=tuple(s.comm_elems), clip_coef=s.clip_coef, skipped=bool(s.skipped))
 
     def _wrap_gather(self, gather_fn):
         if gather_fn is None:
@@ -389,6 +390,10 @@ class ZeroOptimizer:
             raise self._cb_error
         self._check(st, "zero_step_resident")
         return self._stats_dict(out) if stats else None
+
+    def set_clip(self, max_norm: float = 0.0, skip_nonfinite: bool = False):
+        """Global-norm clipping (max_norm > 0) and overflow skip; see zero_set_clip."""
+        self._check(zero_set_clip(self.ctx, float(max_norm), 1 if skip_nonfinite else 0), "zero_set_clip")
 
     def fused_config(self) -> dict:
         k, g, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()

@@ -105,6 +105,35 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
   }
 }
 
+__global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_constant__ AdamBcastArgs a) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
+    const int64_t e = vi * kVec;
+    const int64_t i = a.lo + e;  // flat index; the 8 elements share one owner (S % 8 == 0)
+    float4 p0 = ld_stream(a.master + e), p1 = ld_stream(a.master + e + 4);
+    float4 m0 = ld_stream(a.m + e), m1 = ld_stream(a.m + e + 4);
+    float4 v0 = ld_stream(a.v + e), v1 = ld_stream(a.v + e + 4);
+    const uint4 gw = ld_stream(a.gsrc[i / a.shard] + i);
+    float g[kVec] = {bf16_lo(gw.x), bf16_hi(gw.x), bf16_lo(gw.y), bf16_hi(gw.y),
+                     bf16_lo(gw.z), bf16_hi(gw.z), bf16_lo(gw.w), bf16_hi(gw.w)};
+    if (a.apply_coef) {
+#pragma unroll
+      for (int j = 0; j < kVec; ++j) g[j] = __fmul_rn(g[j], a.coef);
+    }
+    uint16_t p16[kVec];
+    adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+    st_stream(a.master + e, p0);
+    st_stream(a.master + e + 4, p1);
+    st_stream(a.m + e, m0);
+    st_stream(a.m + e + 4, m1);
+    st_stream(a.v + e, v0);
+    st_stream(a.v + e + 4, v1);
+    const uint4 pw = pack8(p16);
+    if (a.param_shard) st_stream(a.param_shard + e, pw);
+    for (int r = 0; r < a.n_out; ++r) st_stream(a.out[r] + e, pw);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
@@ -180,6 +209,11 @@ cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s) {
+  adam_bcast_kernel<<<grid, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s) {
   init_kernel<<<grid, kThreads, 0, s>>>(a);
   return cudaGetLastError();
@@ -210,6 +244,7 @@ cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_bloc
   int mn = multi ? blocks_of(reduce_kernel<true>, &e) : blocks_of(reduce_kernel<false>, &e);
   mn = std::min(mn, blocks_of(adam_kernel, &e));
   mn = std::min(mn, blocks_of(gather_kernel, &e));
+  mn = std::min(mn, blocks_of(adam_bcast_kernel, &e));
   mn = std::min(mn, blocks_of(init_kernel, &e));
   *simple_blocks = mn;
   return e;

@@ -75,6 +75,26 @@ struct AdamArgs {
   AdamScalars sc;
 };
 
+// Adam + broadcast from an already reduced gradient (second pass of a clipped
+// or overflow-checked step).  The gradient of flat element i comes from
+// gsrc[i / shard] + i (the owner's copy); every pointer but gsrc is at flat
+// element `lo`.
+struct AdamBcastArgs {
+  const uint16_t* gsrc[kMaxRanks];
+  uint16_t* out[kMaxRanks];
+  float* master;
+  float* m;
+  float* v;
+  uint16_t* param_shard;            // stage 3 bf16 parameter shard, or nullptr
+  int64_t lo;
+  int64_t shard;
+  int64_t n_vec;
+  int n_out;
+  int apply_coef;                   // scale the gradient by coef (coef < 1)
+  float coef;
+  AdamScalars sc;
+};
+
 struct GatherArgs {
   const uint16_t* src;
   uint16_t* out[kMaxRanks];
@@ -104,6 +124,7 @@ cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s)
 cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with

@@ -61,6 +61,10 @@ struct zero_ctx {
   bool loaded = false;
   int64_t t = 0;
   int64_t stats_step = 0;
+  double clip_norm = 0.0;      // > 0: global-norm clipping
+  bool skip_nonfinite = false;
+  double last_coef = 1.0;      // statistics of the last two-pass step
+  int64_t last_skipped = 0;
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
   // fused-kernel timing
   bool timing = false;
@@ -349,6 +353,125 @@ zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
   out->nonfinite = (int64_t)host.nf;
   out->step = c->stats_step;
   zero_comm_elems(c, out->comm_elems);
+  out->clip_coef = c->last_coef;
+  out->skipped = c->last_skipped;
+  return ZERO_OK;
+}
+
+// Reads the step accumulator (norm, non-finite count); synchronises `s`.
+zero_status read_norm(zero_ctx* c, cudaStream_t s, double* sq, unsigned long long* nf) {
+  struct {
+    double sq;
+    unsigned long long nf;
+    unsigned int done;
+    unsigned int error;
+  } host{};
+  cudaError_t e = cudaMemcpyAsync(&host, norm_scratch(c).step_sq, sizeof host, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "reading the gradient norm");
+  zero_status st = check_device_error(c, host.error, s);
+  if (st != ZERO_OK) return st;
+  *sq = host.sq;
+  *nf = host.nf;
+  return ZERO_OK;
+}
+
+// Clipped / overflow-checked step: reduce everything, read the norm, then
+// Adam + broadcast.  `grad` pointers per interval as in run_step.
+zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
+                         zero_gather_fn gfn, void* guser, void* stream, zero_step_stats* stats) {
+  const int N = c->plan.n_ranks;
+  if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
+    return fail(c, ZERO_ESTATE, "clipping / skipping needs the reduced-gradient shards (ZERO_OPT_KEEP_GRAD_SHARDS = 1)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t t = c->t + 1;
+  const std::vector<zsm::Span> iv = step_intervals(c);
+  const int n_layers = (int)c->plan.layers.size();
+  std::vector<void*> bufs(N);
+  // pass 1: reduce every interval
+  for (size_t k = 0; k < iv.size(); ++k) {
+    const int64_t lo = iv[k].lo, hi = iv[k].hi;
+    zsm::ReduceArgs a;
+    std::memset(&a, 0, sizeof a);
+    for (int r = 0; r < N; ++r) {
+      if (resident) {
+        a.grad[r] = static_cast<const uint16_t*>(resident[r]) + lo;
+      } else {
+        uint16_t* b = c->stage == ZERO_STAGE_1 ? grad_buf_ptr(c, r) + lo : grad_buf_ptr(c, r);
+        bufs[r] = b;
+        a.grad[r] = b;
+      }
+    }
+    if (!resident && fn) {
+      const int rc = fn(user, t, lo, hi, bufs.data(), stream);
+      if (rc != 0) return fail(c, ZERO_EINVAL, "grad_fn returned %d for [%lld, %lld)", rc, (long long)lo, (long long)hi);
+    }
+    a.shard_out = c->stage == ZERO_STAGE_1 ? nullptr : grad_shard_ptr(c) + lo;
+    a.write_back = c->stage == ZERO_STAGE_1 ? 1 : 0;
+    a.n_vec = (hi - lo) / zsm::kVec;
+    a.n_ranks = N;
+    a.accumulate = k > 0 ? 1 : 0;
+    a.inv_n = (float)(1.0 / (double)N);
+    a.ns = norm_scratch(c);
+    if (a.n_vec == 0) continue;
+    cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
+  }
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  zero_status st = read_norm(c, s, &sq, &nf);
+  if (st != ZERO_OK) return st;
+  const double norm = std::sqrt(sq);
+  c->last_skipped = (c->skip_nonfinite && nf > 0) ? 1 : 0;
+  c->last_coef = 1.0;
+  if (!c->last_skipped) {
+    float coef = 1.0f;
+    if (c->clip_norm > 0.0) coef = (float)(c->clip_norm / (norm + 1e-6));
+    const bool apply = coef < 1.0f;
+    c->last_coef = apply ? (double)coef : 1.0;
+    const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+    // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3)
+    std::vector<zsm::Span> p2;
+    if (c->stage == ZERO_STAGE_3) p2 = iv;
+    else p2.push_back({0, c->plan.psi_pad});
+    for (size_t k = 0; k < p2.size(); ++k) {
+      const int64_t lo = p2[k].lo, hi = p2[k].hi;
+      const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
+      zsm::AdamBcastArgs b;
+      std::memset(&b, 0, sizeof b);
+      for (int r = 0; r < N; ++r) {
+        if (c->stage == ZERO_STAGE_1)
+          b.gsrc[r] = resident ? static_cast<const uint16_t*>(resident[r]) : grad_buf_ptr(c, r);
+        else
+          b.gsrc[r] = grad_shard_ptr(c);
+        b.out[r] = c->stage == ZERO_STAGE_3 ? gather_ptr(c, r) : param_ptr(c, r) + lo;
+      }
+      b.n_out = N;
+      b.master = master_ptr(c) + lo;
+      b.m = m_ptr(c) + lo;
+      b.v = v_ptr(c) + lo;
+      b.param_shard = c->stage == ZERO_STAGE_3 ? param_ptr(c, 0) + lo : nullptr;
+      b.lo = lo;
+      b.shard = c->plan.shard;
+      b.n_vec = (hi - lo) / zsm::kVec;
+      b.apply_coef = apply ? 1 : 0;
+      b.coef = coef;
+      b.sc = sc;
+      if (b.n_vec > 0) {
+        cudaError_t e = zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
+        if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
+      }
+      if (c->stage == ZERO_STAGE_3 && gfn) {
+        for (int r = 0; r < N; ++r) bufs[r] = gather_ptr(c, r);
+        const int rc = gfn(guser, c->plan.layers[layer_idx].id, lo, hi, bufs.data(), stream);
+        if (rc != 0) return fail(c, ZERO_EINVAL, "gather_fn returned %d for layer %d", rc, c->plan.layers[layer_idx].id);
+      }
+    }
+    c->t = t;
+  }
+  c->stats_step = c->t;
+  c->norm_fresh = true;
+  if (stats) return finish_stats(c, s, stats);
   return ZERO_OK;
 }
 
@@ -366,6 +489,9 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   } else if (!c->arena[ZERO_ARENA_GRADS]) {
     return fail(c, ZERO_ESTATE, "no gradient buffers (ZERO_OPT_GRAD_BUFFERS = 0): use zero_step_resident");
   }
+  if (c->clip_norm > 0.0 || c->skip_nonfinite) return run_two_pass(c, fn, user, resident, gfn, guser, stream, stats);
+  c->last_coef = 1.0;
+  c->last_skipped = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t t = c->t + 1;
   const zsm::AdamScalars sc = adam_scalars(c->hp, t);
@@ -918,6 +1044,14 @@ zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, doubl
     if (e != cudaSuccess) return cuda_fail(c, e, "reading the device error word");
     return check_device_error(c, err, nullptr);
   }
+  return ZERO_OK;
+}
+
+zero_status zero_set_clip(zero_ctx* c, double max_norm, int32_t skip_nonfinite) {
+  if (!c) return ZERO_EINVAL;
+  if (!(max_norm >= 0.0) || std::isinf(max_norm)) return fail(c, ZERO_EINVAL, "max_norm must be finite and >= 0");
+  c->clip_norm = max_norm;
+  c->skip_nonfinite = skip_nonfinite != 0;
   return ZERO_OK;
 }
 
