@@ -37,8 +37,11 @@ if ROOT not in sys.path:
 METRIC = "fused ZeRO step params/sec (1 B200); achieved HBM GB/s vs ~8 TB/s roofline"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = [os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc", f)
-                  for f in ("kernels.cu", "fused_tma.cu", "device_math.cuh", "kernels.cuh")]
+_CSRC = os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc")
+# the sources each fused kernel is compiled from (kernels.cuh holds only
+# declarations and argument structs)
+KERNEL_SOURCES = {"tma": [os.path.join(_CSRC, f) for f in ("fused_tma.cu", "device_math.cuh")],
+                  "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh")]}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
 
 
@@ -114,24 +117,24 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_digest() -> str:
+def kernel_sources_digest(kernel: str) -> str:
     h = hashlib.sha256()
-    for path in KERNEL_SOURCES:
+    for path in KERNEL_SOURCES[kernel]:
         with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def traffic_for_current_kernel(key: str, elems_per_launch: float):
+def traffic_for_current_kernel(kernel: str, key: str, elems_per_launch: float):
     """Per-launch DRAM bytes from the committed ncu summary for this kernel
-    configuration, scaled to this launch size, or None when the kernel
+    configuration, scaled to this launch size, or None when the kernel's
     sources changed since the capture (or there is no capture)."""
     try:
         with open(TRAFFIC_FILE) as f:
-            d = json.load(f)
-        if d.get("kernel_sources_sha256") != kernel_sources_digest():
+            rec = json.load(f)[key]
+        if rec.get("sources_sha256") != kernel_sources_digest(kernel):
             return None
-        return d["dram_bytes_per_elem"][key] * elems_per_launch
+        return rec["dram_bytes_per_elem"] * elems_per_launch
     except Exception:
         return None
 
@@ -299,7 +302,7 @@ def run_ours(args, world, rank, local):
     elems_per_launch = w.psi / max(1, len(opt.buckets()))
     fc = opt.fused_config()
     ckey = f"stage2_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
-    traffic = traffic_for_current_kernel(ckey, elems_per_launch)
+    traffic = traffic_for_current_kernel(fc["kernel"], ckey, elems_per_launch)
 
     # end to end through the C ABI: every bucket's N gradient slices copied
     # from pinned host memory into the fixed-size buffer, then the fused
@@ -401,36 +404,42 @@ def run_sweep(args):
     s = torch.cuda.current_stream().cuda_stream
     for n_ranks in W.SWEEP_RANKS:
         for elems in W.SWEEP_ELEMS:
-            resident = (6 * n_ranks + 14) * elems  # replicas in, params out, states, grad shard
+            resident = (4 * n_ranks + 14) * elems  # replicas in, params out, states, grad shard
             cell = {"sweep": "flat-zero2", "elems": elems, "n_ranks": n_ranks}
             if resident > args.sweep_max_gb * 1e9:
                 cell["skipped"] = f"exceeds HBM budget ({resident / 1e9:.0f} GB)"
                 print(json.dumps(cell), flush=True)
                 continue
             w = W.flat_sweep(elems, n_ranks)
-            opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, z.ZERO_STAGE_2, keep_grad_shards=True,
-                                  grad_buffers=False, kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel])
-            mv = opt.view(z.ZERO_VIEW_MASTER)
-            synth.dev_f32(W.master_base(w), 0, elems, W.MASTER_DIST, mv.data_ptr(), s)
-            opt.load_master(None)
-            reps = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
-            for r in range(n_ranks):
-                synth.dev_bf16(W.grad_base(w, 1, r), 0, elems, w.grad_dist, reps[r].data_ptr(), s)
-            rl = list(reps)
-            ptrs = [t.data_ptr() for t in rl]
-            model = (4 * n_ranks + 24) * opt.psi_pad
-            reps_n = int(min(2000, max(3, 5e-2 / max(model / 6.0e12, 3e-6))))
+            reps = None
+            for name in ("fused", "unfused"):
+                # the fused step keeps the reduced gradient in registers (the
+                # 4N+24 model); the unfused path needs the shard arena
+                opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, z.ZERO_STAGE_2,
+                                      keep_grad_shards=(name == "unfused"), grad_buffers=False,
+                                      kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel])
+                mv = opt.view(z.ZERO_VIEW_MASTER)
+                synth.dev_f32(W.master_base(w), 0, elems, W.MASTER_DIST, mv.data_ptr(), s)
+                opt.load_master(None)
+                if reps is None:
+                    reps = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+                    for r in range(n_ranks):
+                        synth.dev_bf16(W.grad_base(w, 1, r), 0, elems, w.grad_dist, reps[r].data_ptr(), s)
+                rl = list(reps)
+                ptrs = [t.data_ptr() for t in rl]
+                model = (4 * n_ranks + 24) * opt.psi_pad
+                reps_n = int(min(2000, max(3, 5e-2 / max(model / 6.0e12, 3e-6))))
+                if name == "fused":
+                    cell["fused_config"] = opt.fused_config()
 
-            def fused():
-                opt.step_resident(rl)
-
-            def unfused(t=[0]):
-                t[0] += 1
-                opt.reduce_scatter(0, opt.psi_pad, ptrs)
-                opt.adam_shard(-1, t[0])
-                opt.all_gather(0, opt.psi_pad)
-
-            for name, fn in (("fused", fused), ("unfused", unfused)):
+                    def fn(opt=opt, rl=rl):
+                        opt.step_resident(rl)
+                else:
+                    def fn(opt=opt, ptrs=ptrs, t=[0]):
+                        t[0] += 1
+                        opt.reduce_scatter(0, opt.psi_pad, ptrs)
+                        opt.adam_shard(-1, t[0])
+                        opt.all_gather(0, opt.psi_pad)
                 for _ in range(3):
                     fn()
                 e0 = torch.cuda.Event(enable_timing=True)
@@ -444,13 +453,15 @@ def run_sweep(args):
                 ms = e0.elapsed_time(e1) / reps_n
                 cell[f"{name}_us"] = ms * 1e3
                 cell[f"{name}_gbs_model_4n24"] = model / (ms / 1e3) / 1e9
+                opt.close()
+                del opt, mv, fn
+                torch.cuda.empty_cache()
             cell["unfused_gbs_own_4n32"] = (4 * n_ranks + 32) * opt.psi_pad / (cell["unfused_us"] / 1e6) / 1e9
             cell["fused_speedup"] = cell["unfused_us"] / cell["fused_us"]
             cell["regime"] = "L2-resident / launch-bound" if model < 126e6 * 2 else "HBM"
             cell["reps"] = reps_n
             print(json.dumps(cell), flush=True)
-            opt.close()
-            del opt, reps, rl, mv
+            del reps, rl
             torch.cuda.empty_cache()
 
 
