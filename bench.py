@@ -427,7 +427,8 @@ def run_sweep(args):
                         synth.dev_bf16(W.grad_base(w, 1, r), 0, elems, w.grad_dist, reps[r].data_ptr(), s)
                 rl = list(reps)
                 ptrs = [t.data_ptr() for t in rl]
-                model = (4 * n_ranks + 24) * opt.psi_pad
+                psi_pad = opt.psi_pad
+                model = (4 * n_ranks + 24) * psi_pad
                 reps_n = int(min(2000, max(3, 5e-2 / max(model / 6.0e12, 3e-6))))
                 if name == "fused":
                     cell["fused_config"] = opt.fused_config()
@@ -456,7 +457,7 @@ def run_sweep(args):
                 opt.close()
                 del opt, mv, fn
                 torch.cuda.empty_cache()
-            cell["unfused_gbs_own_4n32"] = (4 * n_ranks + 32) * opt.psi_pad / (cell["unfused_us"] / 1e6) / 1e9
+            cell["unfused_gbs_own_4n32"] = (4 * n_ranks + 32) * psi_pad / (cell["unfused_us"] / 1e6) / 1e9
             cell["fused_speedup"] = cell["unfused_us"] / cell["fused_us"]
             cell["regime"] = "L2-resident / launch-bound" if model < 126e6 * 2 else "HBM"
             cell["reps"] = reps_n

@@ -138,11 +138,12 @@ enum {
                                     zero_kernel_timing); may be set at any time; default 0 */
   ZERO_OPT_KERNEL = 5,           /* fused-step kernel: ZERO_KERNEL_AUTO (default),
                                     ZERO_KERNEL_REGISTER or ZERO_KERNEL_TMA; may be set at any
-                                    time; ZERO_KERNEL_TMA needs N <= 16 (else ZERO_EINVAL) */
+                                    time */
   ZERO_OPT_GRAD_BUFFERS = 6,     /* 1 (default) sizes the GRADS arena; 0 drops it for callers
                                     that only use zero_step_resident and the calls given explicit
                                     pointers (zero_step then returns ZERO_ESTATE) */
-  ZERO_OPT_TMA_GROUPS = 7,       /* staged kernel: producer/consumer groups per CTA, 1 or 2
+  ZERO_OPT_TMA_GROUPS = 7,       /* staged kernel: producer/consumer groups per CTA, 1 or 2,
+                                    or 3 = one group of 16 consumer warps of 4 elements each
                                     (0 = the library's choice); may be set at any time */
   ZERO_OPT_TMA_STAGES = 8,       /* staged kernel: shared-memory ring depth, at most 8 and at
                                     most what fits in 227 KB (0 = the library's choice); may be
@@ -158,7 +159,10 @@ enum {
  *             that streams its 2048-element tiles of the N replicas and
  *             master/m/v into its own shared-memory stages with bulk copies
  *             (mbarrier-counted) and eight consumer warps that compute from
- *             shared memory (N <= 16).  Its waits are
+ *             shared memory (N <= 16); above N = 16, one group whose
+ *             producer streams each tile's replicas in chunks of 8 ranks
+ *             through a ring of 32 KB stages and its master/m/v through a
+ *             second ring (ZERO_OPT_TMA_STAGES = chunk-ring depth).  Its waits are
  *             bounded; one that runs out is reported as ZERO_ECUDA by the next
  *             synchronising call (zero_read_stats, zero_step with stats,
  *             zero_kernel_timing).

@@ -49,12 +49,15 @@ def _hp(w):
 REG, TMA = 1, 2  # ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA
 # fused-kernel variants: the register path, the staged path with one and two groups
 VARIANTS = {"reg": dict(kernel=REG), "tma1": dict(kernel=TMA, tma_groups=1),
-            "tma2": dict(kernel=TMA, tma_groups=2)}
+            "tma2": dict(kernel=TMA, tma_groups=2), "tmaw": dict(kernel=TMA, tma_groups=3),
+            "tmac": dict(kernel=TMA)}
 
 
 def kernels_for(n_ranks):
-    """Fused-kernel variants that apply at this N (the staged one handles N <= 16)."""
-    return ("reg", "tma1", "tma2") if n_ranks <= 16 else ("reg",)
+    """Fused-kernel variants at this N: register, and the staged kernel with one
+    group, two groups and one wide group (N <= 16) or its rank-chunked form
+    (N > 16)."""
+    return ("reg", "tma1", "tma2", "tmaw") if n_ranks <= 16 else ("reg", "tmac")
 
 
 def make_opt(w, stage, bucket=None, keep=True, variant=None, **kw):
@@ -187,7 +190,7 @@ def test_tiny_layouts_all_ranks_buckets_stages(layout):
     """Brute force: N = 1..9 and 16, bucket sizes 8/16/24/all, stages 1-3, 3
     steps each, every element against the oracle's literal per-rank run."""
     numel, layer = layout
-    for n_ranks in list(range(1, 10)) + [16]:
+    for n_ranks in list(range(1, 10)) + [16, 17]:
         p0 = oracle.plan(numel, layer, n_ranks, 8)
         for bucket in sorted({8, 16, 24, p0.psi_pad}):
             for stage in (1, 2, 3):
@@ -355,7 +358,8 @@ def test_transformer_85m_n8_stages_agree_and_match_dp():
     z = _z()
     w = W.gpt_85m_n8()
     opts = {}
-    for stage in (1, 2, 3, "tma1-1", "tma1-2", "tma1-3", "tma2-1", "tma2-2", "tma2-3"):
+    for stage in (1, 2, 3, "tma1-1", "tma1-2", "tma1-3", "tma2-1", "tma2-2", "tma2-3", "tmaw-1", "tmaw-2",
+                  "tmaw-3"):
         variant = stage.split("-")[0] if isinstance(stage, str) else "reg"
         st_ = int(str(stage)[-1])
         opt, fill = make_opt(w, st_, bucket=20_000_000, variant=variant)
@@ -376,7 +380,7 @@ def test_transformer_85m_n8_stages_agree_and_match_dp():
                 assert torch.equal(opt.view(z.ZERO_VIEW_PARAM, 0), opt.view(z.ZERO_VIEW_PARAM, r))
         opts[stage] = opt
     # the staged kernel computes the same bits as the register kernel
-    for st_, v in [(x, y) for x in (1, 2, 3) for y in ("tma1", "tma2")]:
+    for st_, v in [(x, y) for x in (1, 2, 3) for y in ("tma1", "tma2", "tmaw")]:
         a, b = opts[st_], opts[f"{v}-{st_}"]
         for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ, z.ZERO_VIEW_PARAM):
             assert torch.equal(a.view(what), b.view(what)), (st_, what)
@@ -446,7 +450,7 @@ def test_transformer_1p2b_n8_zero2_bucket200m():
     gc.collect()
     torch.cuda.empty_cache()
     # the staged kernel (one and two groups), resident replicas: the same bits
-    for variant in ("tma1", "tma2"):
+    for variant in ("tma1", "tma2", "tmaw"):
         tma, tfill = make_opt(w, 2, bucket=w.bucket_elems, keep=False, variant=variant)
         for t in range(1, w.steps + 1):
             for r in range(w.n_ranks):
@@ -469,7 +473,8 @@ def test_transformer_1p2b_n8_zero2_bucket200m():
     torch.cuda.empty_cache()
 
 
-def test_transformer_6p4b_n64_zero3_one_layer_live():
+@pytest.mark.parametrize("variant", ["reg", "tmac"])
+def test_transformer_6p4b_n64_zero3_one_layer_live(variant):
     """32 layers, hidden 4096 (6,444,154,880 params), N = 64, ZeRO-3 with one
     layer's 64 gradient replicas and 64 temporary gathered layers live, 2
     steps: every gathered layer equals the updated shards on every rank, and
@@ -480,7 +485,7 @@ def test_transformer_6p4b_n64_zero3_one_layer_live():
     opt_need = 12 * 6_444_154_880 + 2 * 6_444_154_880 + 4 * 64 * 201_379_840
     if free < opt_need + (4 << 30):
         pytest.skip(f"needs {opt_need / 1e9:.0f} GB free, have {free / 1e9:.0f} GB")
-    opt, fill = make_opt(w, 3, keep=False)
+    opt, fill = make_opt(w, 3, keep=False, variant=variant)
     assert opt.sizes.max_layer == 201_379_840
     ok = []
 

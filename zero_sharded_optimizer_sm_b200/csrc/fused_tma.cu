@@ -247,6 +247,346 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
   norm_epilogue<tma_threads<G>()>(a.ns, sq, nf, a.accumulate);
 }
 
+// ------------------------------------------- 16 consumer warps variant --
+//
+// The same tile (2048 elements) and ring as fused_step_tma_kernel<MODE, 1>,
+// consumed by sixteen warps of four elements each instead of eight warps of
+// eight: twice the warps to hide the latency of the Adam arithmetic, with one
+// producer and one in-order pipeline.
+constexpr int kWideWarps = 16;
+constexpr int kWideThreads = 32 + kWideWarps * 32;  // 544
+
+__device__ __forceinline__ void add4(float (&acc)[4], uint2 w) {
+  acc[0] = __fadd_rn(acc[0], bf16_lo(w.x));
+  acc[1] = __fadd_rn(acc[1], bf16_hi(w.x));
+  acc[2] = __fadd_rn(acc[2], bf16_lo(w.y));
+  acc[3] = __fadd_rn(acc[3], bf16_hi(w.y));
+}
+
+__device__ __forceinline__ void st_out(uint16_t* p, uint2 v) { *reinterpret_cast<uint2*>(p) = v; }
+
+template <int MODE>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    fused_step_tma_wide_kernel(const __grid_constant__ FusedArgs a, int stages) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const unsigned stage_bytes = tma_stage_bytes(N);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stage_bytes);
+  uint64_t* empty = full + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_k = abort_flag + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kWideWarps);
+      last_k[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u)) {
+          atomicOr(a.ns.error, 1u);
+          *abort_flag = 1;
+          break;
+        }
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        unsigned char* st = smem + (size_t)s * stage_bytes;
+        mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
+        unsigned char* stt = st + (size_t)N * 2 * kTile;
+        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
+        last_k[s] = (int)k;
+      }
+    }
+  } else {
+    const int c = threadIdx.x - 32;  // 0..511
+    const int j = c * 4;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const unsigned char* st = smem + (size_t)s * stage_bytes;
+      const bool active = j < cnt;  // cnt is a multiple of 8, so 4-element groups are whole
+      float4 p, m, v;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (active) {
+        const float* stt = reinterpret_cast<const float*>(st + (size_t)N * 2 * kTile);
+        p = *reinterpret_cast<const float4*>(stt + j);
+        m = *reinterpret_cast<const float4*>(stt + kTile + j);
+        v = *reinterpret_cast<const float4*>(stt + 2 * kTile + j);
+        for (int r = 0; r < N; ++r) add4(acc, *reinterpret_cast<const uint2*>(st + (size_t)r * 2 * kTile + 2 * j));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (active) {
+        const int64_t e = e0 + j;
+        uint16_t g16[4];
+        float gv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          g16[q] = to_bf16(__fmul_rn(acc[q], a.inv_n));
+          gv[q] = __uint_as_float((uint32_t)g16[q] << 16);
+          const double d = (double)gv[q];
+          sq = __dadd_rn(sq, __dmul_rn(d, d));
+          nf += isfinite(gv[q]) ? 0ull : 1ull;
+        }
+        const uint2 gw = make_uint2(pack2(g16[0], g16[1]), pack2(g16[2], g16[3]));
+        if (MODE == kFusedZ1)
+          for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+        if (a.grad_shard) st_out(a.grad_shard + e, gw);
+        const uint16_t h0 = to_bf16(adam1(gv[0], p.x, m.x, v.x, a.sc));
+        const uint16_t h1 = to_bf16(adam1(gv[1], p.y, m.y, v.y, a.sc));
+        const uint16_t h2 = to_bf16(adam1(gv[2], p.z, m.z, v.z, a.sc));
+        const uint16_t h3 = to_bf16(adam1(gv[3], p.w, m.w, v.w, a.sc));
+        st_out(a.master + e, p);
+        st_out(a.m + e, m);
+        st_out(a.v + e, v);
+        const uint2 pw = make_uint2(pack2(h0, h1), pack2(h2, h3));
+        if (MODE == kFusedZ3) st_out(a.param_shard + e, pw);
+        for (int r = 0; r < N; ++r) st_out(a.out[r] + e, pw);
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
+  }
+  norm_epilogue<kWideThreads>(a.ns, sq, nf, a.accumulate);
+}
+
+// ------------------------------------------------ rank-chunked variant --
+//
+// For N > 16 a stage holding all N slices of a tile no longer fits, so the
+// replicas travel in chunks of kChunkRanks ranks.  Two rings:
+//   chunk ring (cstages x 32 KB): the producer streams, tile by tile, the
+//                                 rank chunks 0, 1, ... of the tile;
+//   state ring (sstages x 24 KB): the tile's master/m/v slices.
+// The consumers fold every chunk into their fp32 accumulators in rank order
+// (chunk c holds ranks 8c..8c+7), release it, and after the last chunk read the
+// states, update and store.  Phases advance in the same order on both sides
+// (chunk index = tile iteration x chunks per tile + chunk), so the parity of
+// every wait is that of its running index.  One producer, one consumer group.
+constexpr int kChunkRanks = 8;
+constexpr unsigned kChunkBytes = kChunkRanks * 2 * kTile;   // 32 KB
+constexpr unsigned kStateBytes = 12 * kTile;                // 24 KB
+
+__host__ __device__ inline size_t chunked_smem_bytes(int cstages, int sstages) {
+  return (size_t)cstages * kChunkBytes + (size_t)sstages * kStateBytes +
+         2 * (size_t)(cstages + sstages) * sizeof(uint64_t) + 4 * (size_t)(1 + cstages + sstages);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(tma_threads<1>(), 1)
+    fused_step_chunked_kernel(const __grid_constant__ FusedArgs a, int cstages, int sstages) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const int n_chunks = (N + kChunkRanks - 1) / kChunkRanks;
+  unsigned char* chunk_base = smem;
+  unsigned char* state_base = smem + (size_t)cstages * kChunkBytes;
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(state_base + (size_t)sstages * kStateBytes);
+  uint64_t* cempty = cfull + cstages;
+  uint64_t* sfull = cempty + cstages;
+  uint64_t* sempty = sfull + sstages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sempty + sstages);
+  volatile int* last_ck = abort_flag + 1;        // last phase issued per chunk stage
+  volatile int* last_sk = last_ck + cstages;     // last phase issued per state stage
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < cstages; ++s) {
+      mbar_init(&cfull[s], 1);
+      mbar_init(&cempty[s], kConsumerWarps);
+      last_ck[s] = -1;
+    }
+    for (int s = 0; s < sstages; ++s) {
+      mbar_init(&sfull[s], 1);
+      mbar_init(&sempty[s], kConsumerWarps);
+      last_sk[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer --
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *abort_flag) break;
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        // the tile's optimizer state
+        const int ss = it % sstages;
+        const unsigned sk = (unsigned)(it / sstages);
+        if (sk > 0 && !mbar_wait(&sempty[ss], (sk - 1) & 1u)) {
+          atomicOr(a.ns.error, 1u);
+          *abort_flag = 1;
+          break;
+        }
+        unsigned char* stt = state_base + (size_t)ss * kStateBytes;
+        mbar_expect_tx(&sfull[ss], (unsigned)(12 * cnt));
+        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &sfull[ss], policy);
+        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &sfull[ss], policy);
+        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &sfull[ss], policy);
+        last_sk[ss] = (int)sk;
+        // the tile's rank chunks
+        bool stop = false;
+        for (int c = 0; c < n_chunks; ++c) {
+          const int ci = it * n_chunks + c;
+          const int cs = ci % cstages;
+          const unsigned ck = (unsigned)(ci / cstages);
+          if (ck > 0 && !mbar_wait(&cempty[cs], (ck - 1) & 1u)) {
+            atomicOr(a.ns.error, 1u);
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+          const int r0 = c * kChunkRanks;
+          const int r1 = (r0 + kChunkRanks) < N ? (r0 + kChunkRanks) : N;
+          unsigned char* st = chunk_base + (size_t)cs * kChunkBytes;
+          mbar_expect_tx(&cfull[cs], (unsigned)((r1 - r0) * 2 * cnt));
+          for (int r = r0; r < r1; ++r)
+            bulk_load(st + (size_t)(r - r0) * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &cfull[cs], policy);
+          last_ck[cs] = (int)ck;
+        }
+        if (stop) break;
+      }
+    }
+  } else {
+    // --------------------------------------------------------- consumers --
+    const int c_id = threadIdx.x - 32;  // 0..255
+    const int j = c_id * kVec;
+    bool aborted = false;
+    for (int it = 0; !aborted; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const bool active = j < cnt;
+      float acc[kVec];
+#pragma unroll
+      for (int q = 0; q < kVec; ++q) acc[q] = 0.0f;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int ci = it * n_chunks + c;
+        const int cs = ci % cstages;
+        const unsigned ck = (unsigned)(ci / cstages);
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[cs], ck & 1u));
+        if (!ok || __any_sync(0xFFFFFFFFu, *abort_flag != 0)) {
+          if (!ok && lane == 0) atomicOr(a.ns.error, 2u);
+          *abort_flag = 1;
+          aborted = true;
+          break;
+        }
+        const int r0 = c * kChunkRanks;
+        const int r1 = (r0 + kChunkRanks) < N ? (r0 + kChunkRanks) : N;
+        const unsigned char* st = chunk_base + (size_t)cs * kChunkBytes;
+        if (active)
+          for (int r = r0; r < r1; ++r)
+            add8(acc, *reinterpret_cast<const uint4*>(st + (size_t)(r - r0) * 2 * kTile + 2 * j));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cempty[cs]);
+      }
+      if (aborted) break;
+      const int ss = it % sstages;
+      const unsigned sk = (unsigned)(it / sstages);
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfull[ss], sk & 1u));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      float4 p0, p1, m0, m1, v0, v1;
+      if (active) {
+        const float* stt = reinterpret_cast<const float*>(state_base + (size_t)ss * kStateBytes);
+        p0 = *reinterpret_cast<const float4*>(stt + j);
+        p1 = *reinterpret_cast<const float4*>(stt + j + 4);
+        m0 = *reinterpret_cast<const float4*>(stt + kTile + j);
+        m1 = *reinterpret_cast<const float4*>(stt + kTile + j + 4);
+        v0 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j);
+        v1 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j + 4);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sempty[ss]);
+      if (active) {
+        const int64_t e = e0 + j;
+        uint16_t g16[kVec];
+        float gv[kVec];
+        mean_bf16(acc, a.inv_n, g16, gv, sq, nf);
+        if (MODE == kFusedZ1) {
+          const uint4 gw = pack8(g16);
+          for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+        }
+        if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
+        uint16_t p16[kVec];
+        adam8(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        st_out(a.master + e, p0);
+        st_out(a.master + e + 4, p1);
+        st_out(a.m + e, m0);
+        st_out(a.m + e + 4, m1);
+        st_out(a.v + e, v0);
+        st_out(a.v + e + 4, v1);
+        const uint4 pw = pack8(p16);
+        if (MODE == kFusedZ3) st_out(a.param_shard + e, pw);
+        for (int r = 0; r < N; ++r) st_out(a.out[r] + e, pw);
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // drain the bulk copies already issued before the CTA's memory goes away
+    for (int s = 0; s < cstages; ++s)
+      if (last_ck[s] >= 0 && !mbar_wait(&cfull[s], (unsigned)last_ck[s] & 1u)) atomicOr(a.ns.error, 4u);
+    for (int s = 0; s < sstages; ++s)
+      if (last_sk[s] >= 0 && !mbar_wait(&sfull[s], (unsigned)last_sk[s] & 1u)) atomicOr(a.ns.error, 4u);
+  }
+  norm_epilogue<tma_threads<1>()>(a.ns, sq, nf, a.accumulate);
+}
+
+template <int MODE>
+cudaError_t launch_chunked_mode(const FusedArgs& a, int grid, int cstages, int sstages, cudaStream_t s) {
+  fused_step_chunked_kernel<MODE><<<grid, tma_threads<1>(), chunked_smem_bytes(cstages, sstages), s>>>(a, cstages, sstages);
+  return cudaGetLastError();
+}
+
 size_t tma_smem_bytes(int n_ranks, int stages) {
   return (size_t)stages * tma_stage_bytes(n_ranks) + 2 * stages * sizeof(uint64_t) + 4 * (stages + 1);
 }
@@ -254,7 +594,9 @@ size_t tma_smem_bytes(int n_ranks, int stages) {
 template <int MODE>
 cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, int groups, cudaStream_t s) {
   const size_t bytes = tma_smem_bytes(a.n_ranks, stages);
-  if (groups == 2)
+  if (groups == kWideGroup)
+    fused_step_tma_wide_kernel<MODE><<<grid, kWideThreads, bytes, s>>>(a, stages);
+  else if (groups == 2)
     fused_step_tma_kernel<MODE, 2><<<grid, tma_threads<2>(), bytes, s>>>(a, stages);
   else
     fused_step_tma_kernel<MODE, 1><<<grid, tma_threads<1>(), bytes, s>>>(a, stages);
@@ -276,11 +618,30 @@ cudaError_t tma_configure() {
   if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 2>);
   if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 2>);
   if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 2>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ1>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ2>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ3>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ1>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ2>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ3>);
   return e;
 }
 
+cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s) {
+  const int sstages = 2;
+  if (cstages < 2) cstages = 2;
+  while (cstages > 2 && chunked_smem_bytes(cstages, sstages) > (size_t)kTmaMaxSmem) --cstages;
+  switch (mode) {
+    case kFusedZ1: return launch_chunked_mode<kFusedZ1>(a, grid, cstages, sstages, s);
+    case kFusedZ2: return launch_chunked_mode<kFusedZ2>(a, grid, cstages, sstages, s);
+    case kFusedZ3: return launch_chunked_mode<kFusedZ3>(a, grid, cstages, sstages, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 int tma_stages_for(int n_ranks, int groups, int max_stages) {
-  if (n_ranks < 1 || n_ranks > kTmaMaxRanks || (groups != 1 && groups != 2)) return 0;
+  if (n_ranks < 1 || n_ranks > kTmaMaxRanks || (groups != 1 && groups != 2 && groups != kWideGroup)) return 0;
+  if (groups == kWideGroup) groups = 1;  // one pipeline
   int stages = max_stages > 0 ? std::min(max_stages, kTmaMaxStages) : kTmaDefaultStages;
   while (stages > 0 && tma_smem_bytes(n_ranks, stages) > (size_t)kTmaMaxSmem) --stages;
   stages -= stages % groups;  // every stage belongs to one consumer group
@@ -292,7 +653,10 @@ int tma_ctas_per_sm(int n_ranks, int groups, int max_stages) {
   if (stages == 0) return 0;
   const size_t bytes = tma_smem_bytes(n_ranks, stages);
   int b = 0;
-  cudaError_t e = groups == 2
+  cudaError_t e = groups == kWideGroup
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_wide_kernel<kFusedZ2>,
+                                                                      kWideThreads, bytes)
+                  : groups == 2
                       ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 2>,
                                                                       tma_threads<2>(), bytes)
                       : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 1>,

@@ -19,6 +19,7 @@ constexpr int kTmaMaxRanks = 16; // the shared-memory staged kernel handles N <=
 constexpr int kTmaMaxSmem = 227 * 1024 - 1024;  // dynamic smem cap (1 KB left for static)
 constexpr int kTmaMaxStages = 8;                // ring depth limit of the staged kernel
 constexpr int kTmaDefaultStages = 4;            // ring depth when the caller does not choose
+constexpr int kWideGroup = 3;  // "groups" value that selects one group of 16 consumer warps
 
 // Binary32 scalars of one Adam step, each rounded once from binary64 on the host.
 struct AdamScalars {
@@ -133,6 +134,10 @@ cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups,
                              cudaStream_t s);
 // Ring depth for N and `groups` (max_stages 0 = the default depth), 0 when out of range.
 int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
+// Rank-chunked staged kernel (fused_tma.cu) for any N, meant for N > 16: the
+// replicas stream in chunks of 8 ranks through a `cstages`-deep ring.
+cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s);
+
 // Resident CTAs per SM of the staged kernel in that configuration (0 on error).
 int tma_ctas_per_sm(int n_ranks, int groups, int max_stages);
 cudaError_t tma_configure();       // opt in to the large dynamic smem (current device)

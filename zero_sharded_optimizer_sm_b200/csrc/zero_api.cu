@@ -219,13 +219,22 @@ int tma_grid_cap(zero_ctx* c) {
   return c->tma_grid_cap;
 }
 
-// Whether the fused step runs the shared-memory staged kernel.
+// Whether the fused step runs a shared-memory staged kernel: the all-ranks
+// stage kernel for N <= 16, the rank-chunked one above.
+bool use_chunked(const zero_ctx* c) {
+  if (c->plan.n_ranks <= zsm::kTmaMaxRanks) return false;
+  return c->kernel_opt == ZERO_KERNEL_TMA;  // AUTO keeps the register kernel above N = 16
+}
+
 bool use_tma(const zero_ctx* c) {
+  if (use_chunked(c)) return true;
   if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c), tma_stages(c)) == 0) return false;
   if (c->kernel_opt == ZERO_KERNEL_TMA) return true;
   if (c->kernel_opt == ZERO_KERNEL_REGISTER) return false;
   return true;  // AUTO: the staged kernel wherever it applies (N <= 16)
 }
+
+int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages_opt : 4; }
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
@@ -312,7 +321,11 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
   cudaError_t e;
-  if (use_tma(c)) {
+  if (use_chunked(c)) {
+    const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
+    e = zsm::launch_fused_chunked(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
+                                  chunked_stages(c), s);
+  } else if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
     e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, tma_grid_cap(c))),
                               tma_groups(c), tma_stages(c), s);
@@ -566,8 +579,6 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   }
   if (key == ZERO_OPT_KERNEL) {
     if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_TMA) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
-    if (value == ZERO_KERNEL_TMA && zsm::tma_stages_for(c->plan.n_ranks, 1) == 0)
-      return fail(c, ZERO_EINVAL, "the staged kernel handles N <= %d", zsm::kTmaMaxRanks);
     c->kernel_opt = (int)value;
     return ZERO_OK;
   }
@@ -582,7 +593,7 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     return ZERO_OK;
   }
   if (key == ZERO_OPT_TMA_GROUPS) {
-    if (value < 0 || value > 2) return fail(c, ZERO_EINVAL, "consumer groups must be 0 (auto), 1 or 2");
+    if (value < 0 || value > 3) return fail(c, ZERO_EINVAL, "consumer groups must be 0 (auto), 1, 2 or 3 (one wide group)");
     if (value > 0 && zsm::tma_stages_for(c->plan.n_ranks, (int)value) == 0)
       return fail(c, ZERO_EINVAL, "%lld consumer groups do not fit at N = %d", (long long)value, c->plan.n_ranks);
     c->tma_groups_opt = (int)value;
@@ -672,7 +683,7 @@ zero_status zero_bind(zero_ctx* c, void* const* arenas) {
   int fused_blocks = 0, simple_blocks = 0;
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
-  if (e == cudaSuccess && zsm::tma_stages_for(c->plan.n_ranks, 1) > 0) e = zsm::tma_configure();
+  if (e == cudaSuccess) e = zsm::tma_configure();
   if (e != cudaSuccess) return cuda_fail(c, e, "device query");
   if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
   c->grid_fused = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, fused_blocks)));
@@ -1057,7 +1068,11 @@ zero_status zero_set_clip(zero_ctx* c, double max_norm, int32_t skip_nonfinite) 
 
 zero_status zero_fused_config(const zero_ctx* c, int32_t* kernel, int32_t* groups, int32_t* stages) {
   if (!c || !kernel || !groups || !stages) return ZERO_EINVAL;
-  if (use_tma(c)) {
+  if (use_chunked(c)) {
+    *kernel = ZERO_KERNEL_TMA;
+    *groups = 1;
+    *stages = chunked_stages(c);
+  } else if (use_tma(c)) {
     *kernel = ZERO_KERNEL_TMA;
     *groups = tma_groups(c);
     *stages = zsm::tma_stages_for(c->plan.n_ranks, *groups, tma_stages(c));
