@@ -63,11 +63,15 @@ def parse_args(argv=None):
                          "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
                          "JSON line per cell")
     ap.add_argument("--sweep-max-gb", type=float, default=150.0)
+    ap.add_argument("--stages", action="store_true",
+                    help="ZeRO-1/2/3 fused-step throughput on the 1.2B (N=8) and 85M (N=8) workloads "
+                         "and ZeRO-3 on the 6.4B (N=64) workload; one JSON line per cell")
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
                     help="gpt-1.2b: the benchmark workload; flat-32m: a 33.5M-param flat buffer, "
-                         "N = 8, one bucket (2 GB on the device; for profiler captures)")
+                         "N = 8, one bucket (2 GB on the device); flat-8m-n64: 8.4M params, N = 64 "
+                         "(3 GB on the device); the small ones are for profiler captures")
     return ap.parse_args(argv)
 
 
@@ -203,7 +207,15 @@ def _flat_32m():
     return w
 
 
-WORKLOADS = {"gpt-1.2b": _gpt_1p2b, "flat-32m": _flat_32m}
+def _flat_8m_n64():
+    from synth import workloads as W
+
+    w = W.flat_sweep(1 << 23, 64)
+    w.bucket_elems = 1 << 23
+    return w
+
+
+WORKLOADS = {"gpt-1.2b": _gpt_1p2b, "flat-32m": _flat_32m, "flat-8m-n64": _flat_8m_n64}
 _ARGS = None
 
 
@@ -466,6 +478,112 @@ def run_sweep(args):
             torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------------------ stages ----
+
+def run_stages(args):
+    """Fused-step throughput per ZeRO stage.  Byte models per element: ZeRO-1
+    6N+24 (the all-reduce result is written back to the N replicas), ZeRO-2
+    4N+24, ZeRO-3 4N+26 (the parameter shard besides the N temporary layer
+    buffers).  Where the N full replicas fit in HBM they are resident and the
+    step is timed with CUDA events; the 6.4B / N = 64 ZeRO-3 workload keeps one
+    layer's 64 replicas live (filled between launches by the generator), so
+    only the library's kernels are timed there (ZERO_OPT_TIMING)."""
+    import torch
+
+    import synth
+    import zero_sharded_optimizer_sm_b200 as z
+    from synth import workloads as W
+
+    torch.cuda.set_device(0)
+    s = torch.cuda.current_stream().cuda_stream
+    kern = {"auto": 0, "register": 1, "tma": 2}[args.kernel]
+
+    def master_fill(opt, w):
+        mv = opt.view(z.ZERO_VIEW_MASTER)
+        for off, n in zip(opt.offsets(), w.numel):
+            synth.dev_f32(W.master_base(w), off, n, W.MASTER_DIST, mv.data_ptr() + 4 * off, s)
+        opt.load_master(None)
+
+    for w in (W.gpt_1p2b_n8(), W.gpt_85m_n8()):
+        reps = None
+        for stage in (1, 2, 3):
+            opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage,
+                                  bucket_elems=w.bucket_elems or 200_000_000, hparams=z.AdamHParams(),
+                                  keep_grad_shards=False, grad_buffers=False, kernel=kern)
+            master_fill(opt, w)
+            if reps is None:
+                reps = torch.empty((w.n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+                for r in range(w.n_ranks):
+                    for off, n in zip(opt.offsets(), w.numel):
+                        synth.dev_bf16(W.grad_base(w, 1, r), off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
+            rl = list(reps)
+            for _ in range(3):
+                opt.step_resident(rl)
+            steps = max(5, int(2e9 / ((4 * w.n_ranks + 24) * w.psi)) + 5)
+            opt.set_timing(True)
+            opt.kernel_timing()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(steps):
+                opt.step_resident(rl)
+            e1.record()
+            torch.cuda.synchronize()
+            kt = opt.kernel_timing()
+            ms = e0.elapsed_time(e1) / steps
+            per = {1: 6 * w.n_ranks + 24, 2: 4 * w.n_ranks + 24, 3: 4 * w.n_ranks + 26}[stage]
+            print(json.dumps({"stages": w.name, "stage": stage, "n_ranks": w.n_ranks, "params": w.psi,
+                              "ms_per_step": ms, "params_per_s": w.psi / (ms / 1e3),
+                              "bytes_per_elem_model": per,
+                              "step_gbs_model": per * w.psi / (ms / 1e3) / 1e9,
+                              "kernel_gbs_model": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
+                              "launches_per_step": kt["launches"] // steps,
+                              "fused_config": opt.fused_config(), "steps": steps}), flush=True)
+            opt.close()
+            del opt
+            torch.cuda.empty_cache()
+        del reps, rl
+        torch.cuda.empty_cache()
+
+    w = W.gpt_6p4b_n64()
+    free, _ = torch.cuda.mem_get_info()
+    need = 12 * w.psi + 2 * w.psi + 4 * 64 * 201_379_840
+    if free < need + (4 << 30):
+        print(json.dumps({"stages": w.name, "skipped": f"needs {need / 1e9:.0f} GB"}), flush=True)
+        return
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, 3, hparams=z.AdamHParams(), keep_grad_shards=False,
+                          kernel=kern)
+    master_fill(opt, w)
+    offsets = opt.offsets()
+
+    def gfn(t, lo, hi, bufs, stream):
+        for r, ptr in enumerate(bufs):
+            gb = W.grad_base(w, 1, r)
+            for off, n in zip(offsets, w.numel):
+                a, b = max(lo, off), min(hi, off + n)
+                if a < b:
+                    synth.dev_bf16(gb, a, b - a, w.grad_dist, ptr + 2 * (a - lo), stream)
+        return 0
+
+    opt.step(gfn)
+    opt.set_timing(True)
+    opt.kernel_timing()
+    steps = 2
+    for _ in range(steps):
+        opt.step(gfn)
+    kt = opt.kernel_timing()
+    per = 4 * w.n_ranks + 26
+    kms = kt["ms"] / steps
+    print(json.dumps({"stages": w.name, "stage": 3, "n_ranks": w.n_ranks, "params": w.psi,
+                      "kernel_ms_per_step": kms, "params_per_s_kernels": w.psi / (kms / 1e3),
+                      "bytes_per_elem_model": per, "kernel_gbs_model": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
+                      "launches_per_step": kt["launches"] // steps, "fused_config": opt.fused_config(),
+                      "note": "one layer's 64 replicas live; gradients generated between launches (untimed)"}),
+          flush=True)
+    opt.close()
+
+
 # --------------------------------------------------------------- reference ----
 
 def reference_sample(w, steps_total: int, elems: int = 0):
@@ -537,6 +655,8 @@ def main(argv=None):
         run_reference(args, world, rank, local)
     elif args.sweep:
         run_sweep(args)
+    elif args.stages:
+        run_stages(args)
     else:
         run_ours(args, world, rank, local)
 

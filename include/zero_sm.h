@@ -166,7 +166,8 @@ enum {
  *             bounded; one that runs out is reported as ZERO_ECUDA by the next
  *             synchronising call (zero_read_stats, zero_step with stats,
  *             zero_kernel_timing).
- *   AUTO:     the faster of the two for this N, as measured on B200. */
+ *   AUTO:     the staged kernel for every N, in the configuration measured
+ *             fastest on B200 for that N (zero_fused_config reports it). */
 enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2 };
 
 /* Views (zero_view). */

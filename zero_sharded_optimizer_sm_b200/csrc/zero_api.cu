@@ -180,10 +180,10 @@ constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the st
 // Staged-kernel configuration chosen for N (consumer groups, ring depth),
 // measured on B200 with flat 256M-element buffers and the 1.2B-parameter
 // transformer list: few bytes per element (N <= 4) leave the consumers
-// compute-bound, so two groups win; at N = 5..8 one group with a two-deep
-// ring keeps the fewest copies in flight and moves the most bytes; N = 9..16
-// only fits two stages.  The register kernel wins beyond N = 16 (the staged
-// one does not apply there).
+// compute-bound, so two groups win; at N = 5..8 one group of eight warps with
+// a two-deep ring keeps the fewest copies in flight and moves the most bytes;
+// at N = 9..16 (only two stages fit) one group of sixteen warps wins.  Above
+// N = 16 the rank-chunked staged kernel wins over the register kernel.
 struct TmaChoice {
   int groups, stages;
 };
@@ -192,7 +192,7 @@ TmaChoice tma_policy(int n_ranks) {
   if (n_ranks <= 2) return {2, 4};
   if (n_ranks <= 4) return {2, 2};
   if (n_ranks <= 8) return {1, 2};
-  return {2, 2};
+  return {zsm::kWideGroup, 2};
 }
 
 // Consumer groups of the staged kernel for this context.
@@ -223,7 +223,7 @@ int tma_grid_cap(zero_ctx* c) {
 // stage kernel for N <= 16, the rank-chunked one above.
 bool use_chunked(const zero_ctx* c) {
   if (c->plan.n_ranks <= zsm::kTmaMaxRanks) return false;
-  return c->kernel_opt == ZERO_KERNEL_TMA;  // AUTO keeps the register kernel above N = 16
+  return c->kernel_opt != ZERO_KERNEL_REGISTER;  // AUTO and TMA
 }
 
 bool use_tma(const zero_ctx* c) {
