@@ -45,15 +45,35 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
+_lib_path = None  # an alternative build, for the tests that plant mistakes in the oracle
 
 STAGE_DP, STAGE_Z1, STAGE_Z2, STAGE_Z3 = 0, 1, 2, 3
 GRANULE = 8  # every tensor starts on an 8-element boundary (a stated layout choice)
 
 
+class use_library:
+    """Context manager: run the oracle on another build of zero_oracle.c (the
+    mutation tests compile copies with a planted mistake)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib, _lib_path
+        self.saved = (_lib, _lib_path)
+        _lib, _lib_path = None, self.path
+        return self
+
+    def __exit__(self, *exc):
+        global _lib, _lib_path
+        _lib, _lib_path = self.saved
+        return False
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = os.path.join(_HERE, "libzero_oracle.so")
+        path = _lib_path or os.path.join(_HERE, "libzero_oracle.so")
         if not os.path.exists(path):
             raise RuntimeError(f"{path} is missing: run __graft_entry__.build() first")
         lib = ctypes.CDLL(path)

@@ -9,9 +9,9 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def build(verbose: bool = False) -> str:
-    src = os.path.join(HERE, "zero_oracle.c")
-    out = os.path.join(HERE, "libzero_oracle.so")
+def build(verbose: bool = False, src: str = None, out: str = None) -> str:
+    src = src or os.path.join(HERE, "zero_oracle.c")
+    out = out or os.path.join(HERE, "libzero_oracle.so")
     cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
            "-fno-finite-math-only", "-frounding-math", "-Wall", "-Wextra", "-o", out, src, "-lm"]
     if verbose:
