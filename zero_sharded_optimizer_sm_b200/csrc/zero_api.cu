@@ -234,7 +234,7 @@ bool use_tma(const zero_ctx* c) {
   return true;  // AUTO: the staged kernel wherever it applies (N <= 16)
 }
 
-int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages_opt : 4; }
+int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages_opt : 3; }  // measured best at N = 32, 64
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
