@@ -48,6 +48,7 @@ _lib = None
 _lib_path = None  # an alternative build, for the tests that plant mistakes in the oracle
 
 STAGE_DP, STAGE_Z1, STAGE_Z2, STAGE_Z3 = 0, 1, 2, 3
+BF16, F16 = 0, 1  # 16-bit storage formats of gradients and parameters
 GRANULE = 8  # every tensor starts on an 8-element boundary (a stated layout choice)
 
 
@@ -97,6 +98,22 @@ def _load():
         lib.zo_adam.argtypes = [i64, vp, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
         lib.zo_adam_coef.restype = None
         lib.zo_adam_coef.argtypes = [i64, vp, f32, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
+        lib.zo_f16_rne.restype = ctypes.c_uint16
+        lib.zo_f16_rne.argtypes = [f32]
+        lib.zo_f16_to_f32.restype = f32
+        lib.zo_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.zo_f16_rne_array.restype = None
+        lib.zo_f16_rne_array.argtypes = [i64, vp, vp]
+        lib.zo_f16_to_f32_array.restype = None
+        lib.zo_f16_to_f32_array.argtypes = [i64, vp, vp]
+        lib.zo_reduce_mean_fmt.restype = None
+        lib.zo_reduce_mean_fmt.argtypes = [ctypes.c_int, i32, i64, vp, vp]
+        lib.zo_adam_ex.restype = None
+        lib.zo_adam_ex.argtypes = [ctypes.c_int, i64, vp, f32, f32, vp, vp, vp, vp, f64, f64, f64, f64, f64, i64]
+        lib.zo_sumsq_fmt.restype = ctypes.c_double
+        lib.zo_sumsq_fmt.argtypes = [ctypes.c_int, i64, vp]
+        lib.zo_count_nonfinite_fmt.restype = i64
+        lib.zo_count_nonfinite_fmt.argtypes = [ctypes.c_int, i64, vp]
         lib.zo_sumsq.restype = ctypes.c_double
         lib.zo_sumsq.argtypes = [i64, vp]
         lib.zo_count_nonfinite.restype = i64
@@ -124,6 +141,31 @@ def bf16_to_f32(h: np.ndarray) -> np.ndarray:
     return out
 
 
+def f16_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 -> IEEE binary16 bit patterns (uint16), round to nearest even."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint16)
+    if x.size:
+        _load().zo_f16_rne_array(x.size, x.ctypes.data, out.ctypes.data)
+    return out
+
+
+def f16_to_f32(h: np.ndarray) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.empty(h.shape, dtype=np.float32)
+    if h.size:
+        _load().zo_f16_to_f32_array(h.size, h.ctypes.data, out.ctypes.data)
+    return out
+
+
+def fmt_rne(x: np.ndarray, fmt: int) -> np.ndarray:
+    return f16_rne(x) if fmt == F16 else bf16_rne(x)
+
+
+def fmt_to_f32(h: np.ndarray, fmt: int) -> np.ndarray:
+    return f16_to_f32(h) if fmt == F16 else bf16_to_f32(h)
+
+
 def _ptr_array(arrays: Sequence[np.ndarray]):
     ptrs = (ctypes.c_void_p * len(arrays))()
     for r, a in enumerate(arrays):
@@ -139,6 +181,18 @@ def reduce_mean(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
     out = np.empty(n, dtype=np.uint16)
     if n:
         _load().zo_reduce_mean(len(rank_slices), n, _ptr_array(rank_slices), out.ctypes.data)
+    return out
+
+
+def reduce_mean_fmt(rank_slices: Sequence[np.ndarray], fmt: int) -> np.ndarray:
+    """reduce_mean for either 16-bit format (the bf16 path is reduce_mean)."""
+    if fmt == BF16:
+        return reduce_mean(rank_slices)
+    rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
+    n = rank_slices[0].size
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().zo_reduce_mean_fmt(fmt, len(rank_slices), n, _ptr_array(rank_slices), out.ctypes.data)
     return out
 
 
@@ -195,6 +249,30 @@ def adam_coef(g: np.ndarray, coef: float, master: np.ndarray, m: np.ndarray, v: 
         _load().zo_adam_coef(n, g.ctypes.data, float(np.float32(coef)), master.ctypes.data, m.ctypes.data,
                              v.ctypes.data, out.ctypes.data, hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t)
     return out
+
+
+def adam_ex(g: np.ndarray, fmt: int, inv_scale: float, coef: float, master: np.ndarray, m: np.ndarray,
+            v: np.ndarray, hp: AdamHP, t: int) -> np.ndarray:
+    """Adam for either format with a loss-scale unscale (inv_scale != 1) and a
+    clipping coefficient (applied when < 1); returns the 16-bit params."""
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    n = g.size
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load().zo_adam_ex(fmt, n, g.ctypes.data, float(np.float32(inv_scale)), float(np.float32(coef)),
+                           master.ctypes.data, m.ctypes.data, v.ctypes.data, out.ctypes.data,
+                           hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t)
+    return out
+
+
+def sumsq_fmt(g: np.ndarray, fmt: int) -> float:
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    return float(_load().zo_sumsq_fmt(fmt, g.size, g.ctypes.data)) if g.size else 0.0
+
+
+def count_nonfinite_fmt(g: np.ndarray, fmt: int) -> int:
+    g = np.ascontiguousarray(g, dtype=np.uint16)
+    return int(_load().zo_count_nonfinite_fmt(fmt, g.size, g.ctypes.data)) if g.size else 0
 
 
 CLIP_EPS = 1e-6
@@ -328,16 +406,16 @@ def bucket_schedule(p: Plan) -> List[tuple]:
 
 # ------------------------------------------------------------ collectives ----
 
-def all_reduce(rank_grads: Sequence[np.ndarray], lo: int, hi: int) -> None:
+def all_reduce(rank_grads: Sequence[np.ndarray], lo: int, hi: int, fmt: int = BF16) -> None:
     """All-reduce of [lo, hi) in place ([T] section "ZeRO-1", part "2. 反向"):
     every rank's replica receives the same averaged gradient."""
-    g = reduce_mean([a[lo:hi] for a in rank_grads])
+    g = reduce_mean_fmt([a[lo:hi] for a in rank_grads], fmt)
     for a in rank_grads:
         a[lo:hi] = g
 
 
 def reduce_scatter(rank_grads: Sequence[np.ndarray], plan_: Plan, lo: int, hi: int,
-                   grad_shards: List[np.ndarray]) -> None:
+                   grad_shards: List[np.ndarray], fmt: int = BF16) -> None:
     """Reduce-scatter of [lo, hi) ([T] section "ZeRO-2", part "reduce-scatter
     是什么"): rank r receives only the reduced values of the elements it owns,
     written into its shard array (indexed from r*S)."""
@@ -346,7 +424,7 @@ def reduce_scatter(rank_grads: Sequence[np.ndarray], plan_: Plan, lo: int, hi: i
         a, b = max(lo, olo), min(hi, ohi)
         if a >= b:
             continue
-        grad_shards[r][a - olo:b - olo] = reduce_mean([g[a:b] for g in rank_grads])
+        grad_shards[r][a - olo:b - olo] = reduce_mean_fmt([g[a:b] for g in rank_grads], fmt)
 
 
 def all_gather(param_shards: Sequence[np.ndarray], plan_: Plan, lo: int, hi: int,
@@ -388,11 +466,11 @@ class StepReport:
     coef: float = 1.0
 
 
-def init_states(plan_: Plan, stage: int, master0: np.ndarray) -> List[RankState]:
+def init_states(plan_: Plan, stage: int, master0: np.ndarray, fmt: int = BF16) -> List[RankState]:
     """Every rank starts from the same fp32 master (pads 0), m = v = 0 and the
-    16-bit parameter copy equal to bf16(master)."""
+    16-bit parameter copy equal to the master rounded to the format."""
     assert master0.dtype == np.float32 and master0.size == plan_.psi_pad
-    p16 = bf16_rne(master0)
+    p16 = fmt_rne(master0, fmt)
     ranks = []
     for r in range(plan_.n_ranks):
         lo, hi = plan_.owned(r)
@@ -409,7 +487,8 @@ def init_states(plan_: Plan, stage: int, master0: np.ndarray) -> List[RankState]
 
 
 def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
-         hp: AdamHP, clip_norm: float = 0.0, skip_nonfinite: bool = False) -> StepReport:
+         hp: AdamHP, clip_norm: float = 0.0, skip_nonfinite: bool = False, fmt: int = BF16,
+         loss_scale: float = 1.0) -> StepReport:
     """One optimizer step, t >= 1, following the pages' flow for ``stage``:
     every gradient is reduced (and scattered) first, then each rank updates
     what it owns, then the parameters are gathered.
@@ -419,12 +498,22 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
     reduction, before any update.  With ``skip_nonfinite`` a step whose
     averaged gradient holds an Inf or NaN changes no state (the caller does not
     advance t); with ``clip_norm`` > 0 every rank's Adam uses the gradient
-    times clip_coef(norm, clip_norm)."""
+    times clip_coef(norm, clip_norm).
+
+    ``fmt`` = F16 stores gradients and parameters as IEEE binary16; with a
+    ``loss_scale`` S the ranks' gradients are S times the true ones: the
+    averaged gradient is rounded to the format still scaled, the update first
+    multiplies it by fp32(1/S), and the reported norm (and the clip) is that
+    of the unscaled gradient, sqrt(sum g^2) / S."""
     N, S = plan_.n_ranks, plan_.shard
+    generic = fmt != BF16 or loss_scale != 1.0
+    inv_scale = float(np.float32(1.0 / loss_scale))
     local = [grads(t, r).astype(np.uint16, copy=True) for r in range(N)]
     assert all(a.size == plan_.psi_pad for a in local)
 
     def update(g, st):
+        if generic:
+            return adam_ex(g, fmt, inv_scale, coef, st.master, st.m, st.v, hp, t)
         if coef < 1.0:
             return adam_coef(g, coef, st.master, st.m, st.v, hp, t)
         return adam(g, st.master, st.m, st.v, hp, t)
@@ -432,7 +521,7 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
     if stage in (STAGE_DP, STAGE_Z1):
         # backward ends with a full all-reduce; every rank keeps the full grad
         for lo, hi in plan_.buckets:
-            all_reduce(local, lo, hi)
+            all_reduce(local, lo, hi, fmt)
         for r in range(N):
             ranks[r].grads = local[r]
         g_full = local[0]
@@ -441,16 +530,20 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
         if stage == STAGE_Z2:
             # layer-by-layer reduce-scatter through the fixed-size buffer
             for lo, hi in plan_.buckets:
-                reduce_scatter(local, plan_, lo, hi, shards)
+                reduce_scatter(local, plan_, lo, hi, shards, fmt)
         else:
             # per layer, last to first: reduce-scatter the layer's gradient
             for _, lo, hi in reversed(plan_.layers):
-                reduce_scatter(local, plan_, lo, hi, shards)
+                reduce_scatter(local, plan_, lo, hi, shards, fmt)
         for r in range(N):
             ranks[r].grads = shards[r]
         g_full = np.concatenate(shards)
-    norm = float(np.sqrt(sumsq(g_full)))
-    nonfinite = count_nonfinite(g_full)
+    if generic:
+        norm = float(np.sqrt(sumsq_fmt(g_full, fmt))) / loss_scale
+        nonfinite = count_nonfinite_fmt(g_full, fmt)
+    else:
+        norm = float(np.sqrt(sumsq(g_full)))
+        nonfinite = count_nonfinite(g_full)
     if skip_nonfinite and nonfinite > 0:
         return StepReport(grad_norm=norm, nonfinite=nonfinite, skipped=True)
     coef = clip_coef(norm, clip_norm) if clip_norm > 0 else 1.0
@@ -481,15 +574,16 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
 
 
 def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int, hp: AdamHP,
-        clip_norm: float = 0.0, skip_nonfinite: bool = False):
+        clip_norm: float = 0.0, skip_nonfinite: bool = False, fmt: int = BF16, loss_scale: float = 1.0):
     """``steps`` optimizer steps; gradients for call k come from grads(k, r).
     A skipped step does not advance the Adam step counter t, so the Adam
     step number of call k is 1 + (calls before it that were not skipped)."""
-    ranks = init_states(plan_, stage, master0)
+    ranks = init_states(plan_, stage, master0, fmt)
     reports = []
     t = 0
     for k in range(1, steps + 1):
-        rep = step(plan_, stage, ranks, lambda _t, r, k=k: grads(k, r), t + 1, hp, clip_norm, skip_nonfinite)
+        rep = step(plan_, stage, ranks, lambda _t, r, k=k: grads(k, r), t + 1, hp, clip_norm, skip_nonfinite,
+                   fmt, loss_scale)
         if not rep.skipped:
             t += 1
         reports.append(rep)

@@ -79,6 +79,72 @@ void zo_bf16_to_f32_array(int64_t n, const uint16_t* h, float* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = zo_bf16_to_f32(h[i]);
 }
 
+/* -------------------------------------------------------------- binary16 ---- */
+
+/* IEEE-754 binary16 -> fp32 (exact): sign, 5-bit exponent (bias 15), 10-bit
+ * fraction; exponent 0 holds zeros and subnormals (fraction x 2^-24), 31 holds
+ * infinities and NaNs. */
+float zo_f16_to_f32(uint16_t h) {
+  const int sign = (h >> 15) & 1, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+  float mag;
+  if (e == 0) mag = (float)ldexp((double)f, -24);
+  else if (e == 31) mag = f ? NAN : INFINITY;
+  else mag = (float)ldexp((double)(1024 + f), e - 25);
+  return sign ? -mag : mag;
+}
+
+/*
+ * fp32 -> binary16, round to nearest, ties to even (IEEE-754
+ * roundTiesToEven with an 11-bit significand, exponent range -14..15,
+ * subnormals spaced 2^-24): x / q with q the spacing of x's binade (2^(e-10),
+ * at least 2^-24) is exact in binary64; it is rounded to an integer k with
+ * ties to the even one, and k*q is encoded (k = 2048 carries into the next
+ * binade, k = 1024 from the subnormal range is the smallest normal).
+ * Magnitudes at or above 65520 (halfway past the largest finite 65504) round to
+ * infinity.  NaN maps to a quiet NaN with the sign kept.
+ */
+uint16_t zo_f16_rne(float x) {
+  const uint16_t sign = signbit(x) ? 0x8000u : 0u;
+  if (isnan(x)) return (uint16_t)(sign | 0x7E00u);
+  const double a = fabs((double)x);
+  if (a >= 65520.0) return (uint16_t)(sign | 0x7C00u);
+  if (a == 0.0) return sign;
+  int e = (int)floor(log2(a));
+  if (ldexp(1.0, e) > a) --e;           /* guard log2 rounding at binade edges */
+  else if (ldexp(1.0, e + 1) <= a) ++e;
+  if (e < -14) e = -14;                  /* subnormal spacing */
+  const double n = ldexp(a, 10 - e);     /* a / q, exact */
+  double k = floor(n);
+  const double frac = n - k;
+  if (frac > 0.5 || (frac == 0.5 && fmod(k, 2.0) != 0.0)) k += 1.0;
+  int ki = (int)k;
+  int be;                                /* biased exponent */
+  if (ki >= 2048) {                      /* carried into the next binade */
+    ki >>= 1;
+    ++e;
+  }
+  if (ki < 1024) {                       /* subnormal (e == -14) */
+    return (uint16_t)(sign | (uint16_t)ki);
+  }
+  be = e + 15;
+  if (be >= 31) return (uint16_t)(sign | 0x7C00u);
+  return (uint16_t)(sign | (uint16_t)(be << 10) | (uint16_t)(ki - 1024));
+}
+
+void zo_f16_rne_array(int64_t n, const float* x, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = zo_f16_rne(x[i]);
+}
+
+void zo_f16_to_f32_array(int64_t n, const uint16_t* h, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = zo_f16_to_f32(h[i]);
+}
+
+/* 16-bit storage formats of gradients and parameters. */
+enum { ZO_BF16 = 0, ZO_F16 = 1 };
+
+static float fmt_to_f32(int fmt, uint16_t h) { return fmt == ZO_F16 ? zo_f16_to_f32(h) : zo_bf16_to_f32(h); }
+static uint16_t fmt_rne(int fmt, float x) { return fmt == ZO_F16 ? zo_f16_rne(x) : zo_bf16_rne(x); }
+
 /* ------------------------------------------------------------ reduction ---- */
 
 /*
@@ -231,6 +297,75 @@ void zo_adam_coef(int64_t n, const uint16_t* g, float coef, float* master, float
     v[i] = vi;
     if (p_out) p_out[i] = zo_bf16_rne(p);
   }
+}
+
+/*
+ * The reduction and the update for either storage format, with a loss scale.
+ * Mixed-precision training with 16-bit gradients multiplies the loss by a
+ * scale S so that small gradients survive the 16-bit format; the gradients the
+ * ranks hold are S times the true ones.  The averaged gradient is formed and
+ * rounded to the format while still scaled (so an overflow shows as Inf), and
+ * the update multiplies it by inv_scale = fp32(1/S) in binary32 first
+ * (skipped when inv_scale is 1), then by the clipping coefficient when that is
+ * below 1.  Not on the pages beyond their mention of fp16 as the
+ * communication type; these are the usual mixed-precision conventions.
+ */
+void zo_reduce_mean_fmt(int fmt, int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, uint16_t* out) {
+  const float inv_n = (float)(1.0 / (double)n_ranks);
+  for (int64_t i = 0; i < n; ++i) {
+    float acc = 0.0f;
+    for (int32_t r = 0; r < n_ranks; ++r) acc = acc + fmt_to_f32(fmt, rank_grads[r][i]);
+    out[i] = fmt_rne(fmt, acc * inv_n);
+  }
+}
+
+void zo_adam_ex(int fmt, int64_t n, const uint16_t* g, float inv_scale, float coef, float* master, float* m,
+                float* v, uint16_t* p_out, double lr, double beta1, double beta2, double eps,
+                double weight_decay, int64_t t) {
+  float s[9];
+  zo_adam_scalars(lr, beta1, beta2, eps, weight_decay, t, s);
+  const float b1 = s[0], b2 = s[1], omb1 = s[2], omb2 = s[3], bc1 = s[4], bc2 = s[5];
+  const float decay = s[6], lr_f = s[7], eps_f = s[8];
+  for (int64_t i = 0; i < n; ++i) {
+    float gi = fmt_to_f32(fmt, g[i]);
+    if (inv_scale != 1.0f) gi = gi * inv_scale;
+    if (coef < 1.0f) gi = gi * coef;
+    float p = master[i];
+    p = p * decay;
+    float a = b1 * m[i];
+    float b = omb1 * gi;
+    const float mi = a + b;
+    const float gg = gi * gi;
+    a = b2 * v[i];
+    b = omb2 * gg;
+    const float vi = a + b;
+    const float mh = mi / bc1;
+    const float vh = vi / bc2;
+    const float den = sqrtf(vh) + eps_f;
+    const float ratio = mh / den;
+    const float upd = lr_f * ratio;
+    p = p - upd;
+    master[i] = p;
+    m[i] = mi;
+    v[i] = vi;
+    if (p_out) p_out[i] = fmt_rne(fmt, p);
+  }
+}
+
+double zo_sumsq_fmt(int fmt, int64_t n, const uint16_t* g) {
+  double acc = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    const double x = (double)fmt_to_f32(fmt, g[i]);
+    acc = acc + x * x;
+  }
+  return acc;
+}
+
+int64_t zo_count_nonfinite_fmt(int fmt, int64_t n, const uint16_t* g) {
+  int64_t c = 0;
+  for (int64_t i = 0; i < n; ++i)
+    if (!isfinite(fmt_to_f32(fmt, g[i]))) ++c;
+  return c;
 }
 
 /* ----------------------------------------------- gradient norm / overflow ---- */
