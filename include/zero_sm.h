@@ -148,9 +148,17 @@ enum {
   ZERO_OPT_TMA_STAGES = 8,       /* staged kernel: shared-memory ring depth, at most 8 and at
                                     most what fits in 227 KB (0 = the library's choice); may be
                                     set at any time */
-  ZERO_OPT_TMA_CTAS_PER_SM = 9   /* staged kernel: CTAs per SM, 1..4, capped by what fits in
+  ZERO_OPT_TMA_CTAS_PER_SM = 9,  /* staged kernel: CTAs per SM, 1..4, capped by what fits in
                                     shared memory (0 = the library's choice); any time */
+  ZERO_OPT_DTYPE = 10            /* storage format of every 16-bit buffer (gradients,
+                                    parameters, reduced shards): ZERO_DTYPE_BF16 (default) or
+                                    ZERO_DTYPE_F16 (IEEE binary16); before zero_bind */
 };
+
+/* 16-bit storage formats (ZERO_OPT_DTYPE).  The pages account gradients and
+ * parameters at 2 bytes and name fp16 as a communication type ([M] section 3.3
+ * configuration); bf16 is the default. */
+enum { ZERO_DTYPE_BF16 = 0, ZERO_DTYPE_F16 = 1 };
 
 /* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.
  *   REGISTER: each lane loads its 16-byte slices of the N replicas and of
@@ -322,6 +330,18 @@ zero_status zero_comm_elems(const zero_ctx* ctx, int64_t out[3]);
  * default) restore the single fused pass.
  */
 zero_status zero_set_clip(zero_ctx* ctx, double max_norm, int32_t skip_nonfinite);
+
+/*
+ * Loss scale of mixed-precision training with 16-bit gradients (default 1):
+ * the gradients the ranks hold are `scale` times the true ones (so that small
+ * values survive binary16).  The averaged gradient is formed and stored in
+ * the 16-bit format still scaled -- an overflow there shows as Inf, which
+ * zero_set_clip's skip catches -- and the update multiplies it by
+ * fp32(1/scale) in binary32 before any clipping.  The reported grad_norm and
+ * the clip use the norm of the unscaled gradient.  Not on the pages beyond
+ * their mention of fp16 communication; the usual convention.  scale > 0.
+ */
+zero_status zero_set_loss_scale(zero_ctx* ctx, double scale);
 
 
 

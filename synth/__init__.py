@@ -40,7 +40,11 @@ def _load_host():
             fn = getattr(lib, name)
             fn.restype = None
             fn.argtypes = [u64, i64, i64, i32, f64, u32, ctypes.c_void_p]
-        for name in ("synth_host_gather_bf16", "synth_host_gather_f32"):
+        for name in ("synth_host_fill_f16",):
+            fn = getattr(lib, name)
+            fn.restype = None
+            fn.argtypes = [u64, i64, i64, i32, f64, u32, ctypes.c_void_p]
+        for name in ("synth_host_gather_bf16", "synth_host_gather_f32", "synth_host_gather_f16"):
             fn = getattr(lib, name)
             fn.restype = None
             fn.argtypes = [u64, ctypes.c_void_p, i64, i32, f64, u32, ctypes.c_void_p]
@@ -58,7 +62,7 @@ def _load_dev():
         u64, i64, u32, i32, f64 = ctypes.c_uint64, ctypes.c_int64, ctypes.c_uint32, ctypes.c_int, ctypes.c_double
         lib.synth_dev_base.restype = u64
         lib.synth_dev_base.argtypes = [u64, u32, u32, u32]
-        for name in ("synth_dev_fill_bf16", "synth_dev_fill_f32"):
+        for name in ("synth_dev_fill_bf16", "synth_dev_fill_f32", "synth_dev_fill_f16"):
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = [u64, i64, i64, i32, f64, u32, ctypes.c_void_p, ctypes.c_void_p]
@@ -99,6 +103,23 @@ def host_bf16(b: int, idx0: int, n: int, dist: Dist) -> np.ndarray:
     return out
 
 
+def host_f16(b: int, idx0: int, n: int, dist: Dist) -> np.ndarray:
+    """Binary16 patterns (uint16): the fp32 values truncated toward zero."""
+    out = np.empty(n, dtype=np.uint16)
+    if n:
+        _load_host().synth_host_fill_f16(b, idx0, n, dist.kind, dist.scale, dist.zero_mod, out.ctypes.data)
+    return out
+
+
+def host_f16_at(b: int, idx: np.ndarray, dist: Dist) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.int64)
+    out = np.empty(idx.size, dtype=np.uint16)
+    if idx.size:
+        _load_host().synth_host_gather_f16(b, idx.ctypes.data, idx.size, dist.kind, dist.scale,
+                                           dist.zero_mod, out.ctypes.data)
+    return out
+
+
 def host_f32(b: int, idx0: int, n: int, dist: Dist) -> np.ndarray:
     out = np.empty(n, dtype=np.float32)
     if n:
@@ -131,6 +152,12 @@ def dev_bf16(b: int, idx0: int, n: int, dist: Dist, out_ptr: int, stream: int) -
                                          out_ptr, stream)
     if rc != 0:
         raise RuntimeError(f"synth_dev_fill_bf16 failed with cudaError {rc}")
+
+
+def dev_f16(b: int, idx0: int, n: int, dist: Dist, out_ptr: int, stream: int) -> None:
+    rc = _load_dev().synth_dev_fill_f16(b, idx0, n, dist.kind, dist.scale, dist.zero_mod, out_ptr, stream)
+    if rc != 0:
+        raise RuntimeError(f"synth_dev_fill_f16 failed with cudaError {rc}")
 
 
 def dev_f32(b: int, idx0: int, n: int, dist: Dist, out_ptr: int, stream: int) -> None:

@@ -87,4 +87,24 @@ SYNTH_FN uint16_t synth_value_bf16(uint64_t base, int64_t idx, int kind, double 
   return (uint16_t)(synth_f32_bits(synth_value_f32(base, idx, kind, scale, zero_mod)) >> 16);
 }
 
+/* Generated binary16 bit pattern: the fp32 value truncated toward zero to
+ * IEEE binary16 (11-bit significand, subnormals spaced 2^-24, magnitudes from
+ * 65504 up clamped to 65504) -- integer operations on the fp32 bits, this
+ * generator's own definition of its fp16 output. */
+SYNTH_FN uint16_t synth_f32_to_f16_trunc(float f) {
+  const uint32_t u = synth_f32_bits(f);
+  const uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  const uint32_t a = u & 0x7FFFFFFFu;
+  if (a >= 0x477FE000u) return (uint16_t)(sign | 0x7BFFu);
+  const int e = (int)(a >> 23) - 127;
+  if (e >= -14) return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)((a >> 13) & 0x3FFu));
+  if (e < -25) return sign;
+  const uint32_t mant = (a & 0x7FFFFFu) | 0x800000u;
+  return (uint16_t)(sign | (uint16_t)(mant >> (uint32_t)(-(e + 1))));
+}
+
+SYNTH_FN uint16_t synth_value_f16(uint64_t base, int64_t idx, int kind, double scale, uint32_t zero_mod) {
+  return synth_f32_to_f16_trunc(synth_value_f32(base, idx, kind, scale, zero_mod));
+}
+
 #endif /* SYNTH_GEN_H */

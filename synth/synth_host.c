@@ -28,3 +28,13 @@ void synth_host_gather_f32(uint64_t base, const int64_t* idx, int64_t n, int kin
                            uint32_t zero_mod, float* out) {
   for (int64_t j = 0; j < n; ++j) out[j] = synth_value_f32(base, idx[j], kind, scale, zero_mod);
 }
+
+void synth_host_fill_f16(uint64_t base, int64_t idx0, int64_t n, int kind, double scale,
+                         uint32_t zero_mod, uint16_t* out) {
+  for (int64_t j = 0; j < n; ++j) out[j] = synth_value_f16(base, idx0 + j, kind, scale, zero_mod);
+}
+
+void synth_host_gather_f16(uint64_t base, const int64_t* idx, int64_t n, int kind, double scale,
+                           uint32_t zero_mod, uint16_t* out) {
+  for (int64_t j = 0; j < n; ++j) out[j] = synth_value_f16(base, idx[j], kind, scale, zero_mod);
+}

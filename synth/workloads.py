@@ -19,7 +19,7 @@ from typing import List, Optional, Sequence
 
 import numpy as np
 
-from . import NORMAL, STREAM_GRAD, STREAM_MASTER, UNIFORM, Dist, base, host_bf16, host_f32
+from . import NORMAL, STREAM_GRAD, STREAM_MASTER, UNIFORM, Dist, base, host_bf16, host_f16, host_f32
 
 SEED0 = 0x5EED0000
 
@@ -120,11 +120,13 @@ def master_base(w: Workload) -> int:
 
 
 def host_padded(offsets: Sequence[int], numel: Sequence[int], psi_pad: int, b: int, dist: Dist,
-                as_f32: bool = False) -> np.ndarray:
+                as_f32: bool = False, f16: bool = False) -> np.ndarray:
     """Values for a padded flat layout: element at flat position i draws
-    index i; pad positions (between tensors and at the tail) are 0."""
+    index i; pad positions (between tensors and at the tail) are 0.  16-bit
+    patterns are bf16 unless ``f16``."""
     out = np.zeros(psi_pad, dtype=np.float32 if as_f32 else np.uint16)
+    fill = host_f32 if as_f32 else (host_f16 if f16 else host_bf16)
     for off, n in zip(offsets, numel):
         if n:
-            out[off:off + n] = (host_f32 if as_f32 else host_bf16)(b, off, n, dist)
+            out[off:off + n] = fill(b, off, n, dist)
     return out

@@ -89,8 +89,9 @@ def real_segments(offsets: Sequence[int], numel: Sequence[int], lo: int, hi: int
 class DeviceFill:
     """Device-side seeded fills for a workload (pads are written as 0)."""
 
-    def __init__(self, w: W.Workload, offsets: Sequence[int], psi_pad: int):
+    def __init__(self, w: W.Workload, offsets: Sequence[int], psi_pad: int, f16: bool = False):
         self.w, self.offsets, self.psi_pad = w, list(offsets), psi_pad
+        self.fill16 = synth.dev_f16 if f16 else synth.dev_bf16
         self.has_pads = any(o + n != e for o, n, e in zip(self.offsets, w.numel, self.offsets[1:] + [psi_pad]))
 
     def grads_into(self, step: int, rank: int, lo: int, hi: int, buf_ptr: int, buf_tensor, stream: int):
@@ -101,7 +102,7 @@ class DeviceFill:
         if self.has_pads:
             buf_tensor[: hi - lo].zero_()
         for a, e in segs:
-            synth.dev_bf16(b, a, e - a, self.w.grad_dist, buf_ptr + 2 * (a - lo), stream)
+            self.fill16(b, a, e - a, self.w.grad_dist, buf_ptr + 2 * (a - lo), stream)
 
     def master_into(self, master_ptr: int, master_tensor, stream: int):
         b = W.master_base(self.w)

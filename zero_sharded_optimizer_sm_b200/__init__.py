@@ -43,6 +43,8 @@ ZERO_OPT_GRAD_BUFFERS = 6
 ZERO_OPT_TMA_GROUPS = 7
 ZERO_OPT_TMA_STAGES = 8
 ZERO_OPT_TMA_CTAS_PER_SM = 9
+ZERO_OPT_DTYPE = 10
+ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
 
@@ -104,6 +106,7 @@ _SIGS = {
     "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                   ctypes.POINTER(ctypes.c_double)]),
     "zero_set_clip": (_i32, [_vp, ctypes.c_double, _i32]),
+    "zero_set_loss_scale": (_i32, [_vp, ctypes.c_double]),
     "zero_fused_config": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
@@ -156,7 +159,7 @@ class ZeroOptimizer:
                  bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
-                 tma_stages: int = 0, tma_ctas_per_sm: int = 0, device=None):
+                 tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16, device=None):
         import torch
 
         self._torch = torch
@@ -190,6 +193,8 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_GROUPS, int(tma_groups)), "zero_set_option")
         if tma_stages:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_STAGES, int(tma_stages)), "zero_set_option")
+        if dtype != ZERO_DTYPE_BF16:
+            self._check(zero_set_option(ctx, ZERO_OPT_DTYPE, int(dtype)), "zero_set_option")
         if tma_ctas_per_sm:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_CTAS_PER_SM, int(tma_ctas_per_sm)), "zero_set_option")
         self.sizes = zero_sizes()
@@ -394,6 +399,10 @@ class ZeroOptimizer:
     def set_clip(self, max_norm: float = 0.0, skip_nonfinite: bool = False):
         """Global-norm clipping (max_norm > 0) and overflow skip; see zero_set_clip."""
         self._check(zero_set_clip(self.ctx, float(max_norm), 1 if skip_nonfinite else 0), "zero_set_clip")
+
+    def set_loss_scale(self, scale: float):
+        """The ranks' gradients are ``scale`` times the true ones; see zero_set_loss_scale."""
+        self._check(zero_set_loss_scale(self.ctx, float(scale)), "zero_set_loss_scale")
 
     def fused_config(self) -> dict:
         k, g, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()

@@ -15,6 +15,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "kernels.cuh"
@@ -48,6 +49,24 @@ __device__ __forceinline__ uint16_t to_bf16(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// The two 16-bit storage formats: decode the low / high half of a 32-bit word
+// (exact), decode one value, round a binary32 to the format (nearest even).
+struct Bf16 {
+  static __device__ __forceinline__ float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+  static __device__ __forceinline__ float f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+  static __device__ __forceinline__ uint16_t rn(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+};
+
+struct F16 {
+  static __device__ __forceinline__ float lo(uint32_t w) {
+    return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+  }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+  static __device__ __forceinline__ float f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+  static __device__ __forceinline__ uint16_t rn(float x) { return __half_as_ushort(__float2half_rn(x)); }
+};
+
 __device__ __forceinline__ uint32_t pack2(uint16_t lo, uint16_t hi) {
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
@@ -56,15 +75,16 @@ __device__ __forceinline__ uint4 pack8(const uint16_t (&h)[kVec]) {
   return make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
 }
 
+template <class F = Bf16>
 __device__ __forceinline__ void add8(float (&acc)[kVec], uint4 w) {
-  acc[0] = __fadd_rn(acc[0], bf16_lo(w.x));
-  acc[1] = __fadd_rn(acc[1], bf16_hi(w.x));
-  acc[2] = __fadd_rn(acc[2], bf16_lo(w.y));
-  acc[3] = __fadd_rn(acc[3], bf16_hi(w.y));
-  acc[4] = __fadd_rn(acc[4], bf16_lo(w.z));
-  acc[5] = __fadd_rn(acc[5], bf16_hi(w.z));
-  acc[6] = __fadd_rn(acc[6], bf16_lo(w.w));
-  acc[7] = __fadd_rn(acc[7], bf16_hi(w.w));
+  acc[0] = __fadd_rn(acc[0], F::lo(w.x));
+  acc[1] = __fadd_rn(acc[1], F::hi(w.x));
+  acc[2] = __fadd_rn(acc[2], F::lo(w.y));
+  acc[3] = __fadd_rn(acc[3], F::hi(w.y));
+  acc[4] = __fadd_rn(acc[4], F::lo(w.z));
+  acc[5] = __fadd_rn(acc[5], F::hi(w.z));
+  acc[6] = __fadd_rn(acc[6], F::lo(w.w));
+  acc[7] = __fadd_rn(acc[7], F::hi(w.w));
 }
 
 // ------------------------------------------------------- rank-order reduce --
@@ -73,7 +93,7 @@ __device__ __forceinline__ void add8(float (&acc)[kVec], uint4 w) {
 // loaded in groups of 8 (eight 16-byte loads in flight per lane).  With more
 // than 8 ranks (kMulti) the next group's loads are issued before the current
 // group is added, which costs a second 8-vector buffer of registers.
-template <bool kMulti, class PtrArray>
+template <bool kMulti, class F = Bf16, class PtrArray>
 __device__ __forceinline__ void reduce_ranks(const PtrArray& grad, int n, int64_t e,
                                              float (&acc)[kVec]) {
 #pragma unroll
@@ -85,7 +105,7 @@ __device__ __forceinline__ void reduce_ranks(const PtrArray& grad, int n, int64_
   if constexpr (!kMulti) {
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      if (k < n) add8(acc, cur[k]);
+      if (k < n) add8<F>(acc, cur[k]);
   } else {
     uint4 nxt[8];
     for (int r0 = 0; r0 < n; r0 += 8) {
@@ -95,23 +115,25 @@ __device__ __forceinline__ void reduce_ranks(const PtrArray& grad, int n, int64_
         if (r1 + k < n) nxt[k] = ld_stream(grad[r1 + k] + e);
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        if (r0 + k < n) add8(acc, cur[k]);
+        if (r0 + k < n) add8<F>(acc, cur[k]);
 #pragma unroll
       for (int k = 0; k < 8; ++k) cur[k] = nxt[k];
     }
   }
 }
 
-// Mean, bf16 rounding, and the norm / non-finite tallies of one vector.
+// Mean, rounding to the 16-bit format, and the norm / non-finite tallies of
+// one vector (of the stored, still loss-scaled, averaged gradient).
+template <class F = Bf16>
 __device__ __forceinline__ void mean_bf16(const float (&acc)[kVec], float inv_n,
                                           uint16_t (&g16)[kVec], float (&g)[kVec], double& sq,
                                           unsigned long long& nf) {
 #pragma unroll
   for (int j = 0; j < kVec; ++j) {
-    g16[j] = to_bf16(__fmul_rn(acc[j], inv_n));
-    g[j] = __uint_as_float((uint32_t)g16[j] << 16);
+    g16[j] = F::rn(__fmul_rn(acc[j], inv_n));
+    g[j] = F::f32(g16[j]);
     const double d = (double)g[j];
-    sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (8-bit significand)
+    sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
     nf += isfinite(g[j]) ? 0ull : 1ull;
   }
 }
@@ -120,6 +142,8 @@ __device__ __forceinline__ void mean_bf16(const float (&acc)[kVec], float inv_n,
 
 __device__ __forceinline__ float adam1(float g, float& p, float& m, float& v,
                                        const AdamScalars& s) {
+  if (s.flags & kUnscale) g = __fmul_rn(g, s.inv_scale);  // loss scale first,
+  if (s.flags & kClip) g = __fmul_rn(g, s.coef);          // then the clipping coefficient
   p = __fmul_rn(p, s.decay);
   m = __fadd_rn(__fmul_rn(s.b1, m), __fmul_rn(s.omb1, g));
   v = __fadd_rn(__fmul_rn(s.b2, v), __fmul_rn(s.omb2, __fmul_rn(g, g)));
@@ -130,18 +154,19 @@ __device__ __forceinline__ float adam1(float g, float& p, float& m, float& v,
   return p;
 }
 
-// Adam on 8 consecutive elements: state vectors in, bf16 params out.
+// Adam on 8 consecutive elements: state vectors in, 16-bit params out.
+template <class F = Bf16>
 __device__ __forceinline__ void adam8(const float (&g)[kVec], float4& p0, float4& p1, float4& m0,
                                       float4& m1, float4& v0, float4& v1, const AdamScalars& s,
                                       uint16_t (&out)[kVec]) {
-  out[0] = to_bf16(adam1(g[0], p0.x, m0.x, v0.x, s));
-  out[1] = to_bf16(adam1(g[1], p0.y, m0.y, v0.y, s));
-  out[2] = to_bf16(adam1(g[2], p0.z, m0.z, v0.z, s));
-  out[3] = to_bf16(adam1(g[3], p0.w, m0.w, v0.w, s));
-  out[4] = to_bf16(adam1(g[4], p1.x, m1.x, v1.x, s));
-  out[5] = to_bf16(adam1(g[5], p1.y, m1.y, v1.y, s));
-  out[6] = to_bf16(adam1(g[6], p1.z, m1.z, v1.z, s));
-  out[7] = to_bf16(adam1(g[7], p1.w, m1.w, v1.w, s));
+  out[0] = F::rn(adam1(g[0], p0.x, m0.x, v0.x, s));
+  out[1] = F::rn(adam1(g[1], p0.y, m0.y, v0.y, s));
+  out[2] = F::rn(adam1(g[2], p0.z, m0.z, v0.z, s));
+  out[3] = F::rn(adam1(g[3], p0.w, m0.w, v0.w, s));
+  out[4] = F::rn(adam1(g[4], p1.x, m1.x, v1.x, s));
+  out[5] = F::rn(adam1(g[5], p1.y, m1.y, v1.y, s));
+  out[6] = F::rn(adam1(g[6], p1.z, m1.z, v1.z, s));
+  out[7] = F::rn(adam1(g[7], p1.w, m1.w, v1.w, s));
 }
 
 // ------------------------------------------------------- norm epilogue --

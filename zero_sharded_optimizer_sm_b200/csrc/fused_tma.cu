@@ -117,7 +117,7 @@ __host__ __device__ inline unsigned tma_stage_bytes(int n_ranks) {
 // gridDim.x) belongs to group it % G and lives in stage it % stages; the
 // stage count is a multiple of G, so every stage belongs to one group and
 // each group's producer and consumers meet its stages' phases in order.
-template <int MODE, int G>
+template <int MODE, int G, class F>
 __global__ void __launch_bounds__(tma_threads<G>(), 1)
     fused_step_tma_kernel(const __grid_constant__ FusedArgs a, int stages) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
 #pragma unroll
         for (int q = 0; q < kVec; ++q) acc[q] = 0.0f;
         for (int r = 0; r < N; ++r)
-          add8(acc, *reinterpret_cast<const uint4*>(st + (size_t)r * 2 * kTile + 2 * j));
+          add8<F>(acc, *reinterpret_cast<const uint4*>(st + (size_t)r * 2 * kTile + 2 * j));
       }
       // every lane of the warp is done reading this stage: release it
       __syncwarp();
@@ -218,14 +218,14 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         const int64_t e = e0 + j;
         uint16_t g16[kVec];
         float gv[kVec];
-        mean_bf16(acc, a.inv_n, g16, gv, sq, nf);
+        mean_bf16<F>(acc, a.inv_n, g16, gv, sq, nf);
         if (MODE == kFusedZ1) {
           const uint4 gw = pack8(g16);
           for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         }
         if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
-        adam8(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        adam8<F>(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
         st_out(a.master + e, p0);
         st_out(a.master + e + 4, p1);
         st_out(a.m + e, m0);
@@ -256,16 +256,17 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
 constexpr int kWideWarps = 16;
 constexpr int kWideThreads = 32 + kWideWarps * 32;  // 544
 
+template <class F>
 __device__ __forceinline__ void add4(float (&acc)[4], uint2 w) {
-  acc[0] = __fadd_rn(acc[0], bf16_lo(w.x));
-  acc[1] = __fadd_rn(acc[1], bf16_hi(w.x));
-  acc[2] = __fadd_rn(acc[2], bf16_lo(w.y));
-  acc[3] = __fadd_rn(acc[3], bf16_hi(w.y));
+  acc[0] = __fadd_rn(acc[0], F::lo(w.x));
+  acc[1] = __fadd_rn(acc[1], F::hi(w.x));
+  acc[2] = __fadd_rn(acc[2], F::lo(w.y));
+  acc[3] = __fadd_rn(acc[3], F::hi(w.y));
 }
 
 __device__ __forceinline__ void st_out(uint16_t* p, uint2 v) { *reinterpret_cast<uint2*>(p) = v; }
 
-template <int MODE>
+template <int MODE, class F>
 __global__ void __launch_bounds__(kWideThreads, 1)
     fused_step_tma_wide_kernel(const __grid_constant__ FusedArgs a, int stages) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         p = *reinterpret_cast<const float4*>(stt + j);
         m = *reinterpret_cast<const float4*>(stt + kTile + j);
         v = *reinterpret_cast<const float4*>(stt + 2 * kTile + j);
-        for (int r = 0; r < N; ++r) add4(acc, *reinterpret_cast<const uint2*>(st + (size_t)r * 2 * kTile + 2 * j));
+        for (int r = 0; r < N; ++r) add4<F>(acc, *reinterpret_cast<const uint2*>(st + (size_t)r * 2 * kTile + 2 * j));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -355,8 +356,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         float gv[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          g16[q] = to_bf16(__fmul_rn(acc[q], a.inv_n));
-          gv[q] = __uint_as_float((uint32_t)g16[q] << 16);
+          g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
+          gv[q] = F::f32(g16[q]);
           const double d = (double)gv[q];
           sq = __dadd_rn(sq, __dmul_rn(d, d));
           nf += isfinite(gv[q]) ? 0ull : 1ull;
@@ -365,10 +366,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (MODE == kFusedZ1)
           for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         if (a.grad_shard) st_out(a.grad_shard + e, gw);
-        const uint16_t h0 = to_bf16(adam1(gv[0], p.x, m.x, v.x, a.sc));
-        const uint16_t h1 = to_bf16(adam1(gv[1], p.y, m.y, v.y, a.sc));
-        const uint16_t h2 = to_bf16(adam1(gv[2], p.z, m.z, v.z, a.sc));
-        const uint16_t h3 = to_bf16(adam1(gv[3], p.w, m.w, v.w, a.sc));
+        const uint16_t h0 = F::rn(adam1(gv[0], p.x, m.x, v.x, a.sc));
+        const uint16_t h1 = F::rn(adam1(gv[1], p.y, m.y, v.y, a.sc));
+        const uint16_t h2 = F::rn(adam1(gv[2], p.z, m.z, v.z, a.sc));
+        const uint16_t h3 = F::rn(adam1(gv[3], p.w, m.w, v.w, a.sc));
         st_out(a.master + e, p);
         st_out(a.m + e, m);
         st_out(a.v + e, v);
@@ -407,7 +408,7 @@ __host__ __device__ inline size_t chunked_smem_bytes(int cstages, int sstages) {
          2 * (size_t)(cstages + sstages) * sizeof(uint64_t) + 4 * (size_t)(1 + cstages + sstages);
 }
 
-template <int MODE>
+template <int MODE, class F>
 __global__ void __launch_bounds__(tma_threads<1>(), 1)
     fused_step_chunked_kernel(const __grid_constant__ FusedArgs a, int cstages, int sstages) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -521,7 +522,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         const unsigned char* st = chunk_base + (size_t)cs * kChunkBytes;
         if (active)
           for (int r = r0; r < r1; ++r)
-            add8(acc, *reinterpret_cast<const uint4*>(st + (size_t)(r - r0) * 2 * kTile + 2 * j));
+            add8<F>(acc, *reinterpret_cast<const uint4*>(st + (size_t)(r - r0) * 2 * kTile + 2 * j));
         __syncwarp();
         if (lane == 0) mbar_arrive(&cempty[cs]);
       }
@@ -550,14 +551,14 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         const int64_t e = e0 + j;
         uint16_t g16[kVec];
         float gv[kVec];
-        mean_bf16(acc, a.inv_n, g16, gv, sq, nf);
+        mean_bf16<F>(acc, a.inv_n, g16, gv, sq, nf);
         if (MODE == kFusedZ1) {
           const uint4 gw = pack8(g16);
           for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         }
         if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
-        adam8(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        adam8<F>(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
         st_out(a.master + e, p0);
         st_out(a.master + e + 4, p1);
         st_out(a.m + e, m0);
@@ -583,7 +584,11 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
 
 template <int MODE>
 cudaError_t launch_chunked_mode(const FusedArgs& a, int grid, int cstages, int sstages, cudaStream_t s) {
-  fused_step_chunked_kernel<MODE><<<grid, tma_threads<1>(), chunked_smem_bytes(cstages, sstages), s>>>(a, cstages, sstages);
+  const size_t bytes = chunked_smem_bytes(cstages, sstages);
+  if (a.fmt == kFmtF16)
+    fused_step_chunked_kernel<MODE, F16><<<grid, tma_threads<1>(), bytes, s>>>(a, cstages, sstages);
+  else
+    fused_step_chunked_kernel<MODE, Bf16><<<grid, tma_threads<1>(), bytes, s>>>(a, cstages, sstages);
   return cudaGetLastError();
 }
 
@@ -591,15 +596,21 @@ size_t tma_smem_bytes(int n_ranks, int stages) {
   return (size_t)stages * tma_stage_bytes(n_ranks) + 2 * stages * sizeof(uint64_t) + 4 * (stages + 1);
 }
 
+template <int MODE, class F>
+void launch_tma_fmt(const FusedArgs& a, int grid, int stages, int groups, size_t bytes, cudaStream_t s) {
+  if (groups == kWideGroup)
+    fused_step_tma_wide_kernel<MODE, F><<<grid, kWideThreads, bytes, s>>>(a, stages);
+  else if (groups == 2)
+    fused_step_tma_kernel<MODE, 2, F><<<grid, tma_threads<2>(), bytes, s>>>(a, stages);
+  else
+    fused_step_tma_kernel<MODE, 1, F><<<grid, tma_threads<1>(), bytes, s>>>(a, stages);
+}
+
 template <int MODE>
 cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, int groups, cudaStream_t s) {
   const size_t bytes = tma_smem_bytes(a.n_ranks, stages);
-  if (groups == kWideGroup)
-    fused_step_tma_wide_kernel<MODE><<<grid, kWideThreads, bytes, s>>>(a, stages);
-  else if (groups == 2)
-    fused_step_tma_kernel<MODE, 2><<<grid, tma_threads<2>(), bytes, s>>>(a, stages);
-  else
-    fused_step_tma_kernel<MODE, 1><<<grid, tma_threads<1>(), bytes, s>>>(a, stages);
+  if (a.fmt == kFmtF16) launch_tma_fmt<MODE, F16>(a, grid, stages, groups, bytes, s);
+  else launch_tma_fmt<MODE, Bf16>(a, grid, stages, groups, bytes, s);
   return cudaGetLastError();
 }
 
@@ -610,21 +621,27 @@ static cudaError_t opt_in(K kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
 }
 
-cudaError_t tma_configure() {
+template <class F>
+cudaError_t tma_configure_fmt() {
   cudaError_t e = cudaSuccess;
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 1>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 1>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 1>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 2>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 2>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 2>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ1>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ2>);
-  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ3>);
-  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ1>);
-  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ2>);
-  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ3>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 1, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 1, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 1, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ1, 2, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ2, 2, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_kernel<kFusedZ3, 2, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ1, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ2, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_tma_wide_kernel<kFusedZ3, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ1, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ2, F>);
+  if (e == cudaSuccess) e = opt_in(fused_step_chunked_kernel<kFusedZ3, F>);
   return e;
+}
+
+cudaError_t tma_configure() {
+  cudaError_t e = tma_configure_fmt<Bf16>();
+  return e == cudaSuccess ? tma_configure_fmt<F16>() : e;
 }
 
 cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s) {
@@ -654,12 +671,12 @@ int tma_ctas_per_sm(int n_ranks, int groups, int max_stages) {
   const size_t bytes = tma_smem_bytes(n_ranks, stages);
   int b = 0;
   cudaError_t e = groups == kWideGroup
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_wide_kernel<kFusedZ2>,
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_wide_kernel<kFusedZ2, Bf16>,
                                                                       kWideThreads, bytes)
                   : groups == 2
-                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 2>,
+                      ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 2, Bf16>,
                                                                       tma_threads<2>(), bytes)
-                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 1>,
+                      : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, fused_step_tma_kernel<kFusedZ2, 1, Bf16>,
                                                                       tma_threads<1>(), bytes);
   return e == cudaSuccess ? b : 0;
 }

@@ -26,7 +26,7 @@ using namespace dev;
 //             all-gather).
 //   kFusedZ3: parameters to the owner's shard and the N temporary layer
 //             buffers.
-template <int MODE, bool kMulti>
+template <int MODE, bool kMulti, class F>
 __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   double sq = 0.0;
   unsigned long long nf = 0;
@@ -37,17 +37,17 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     float4 m0 = ld_stream(a.m + e), m1 = ld_stream(a.m + e + 4);
     float4 v0 = ld_stream(a.v + e), v1 = ld_stream(a.v + e + 4);
     float acc[kVec];
-    reduce_ranks<kMulti>(a.grad, a.n_ranks, e, acc);
+    reduce_ranks<kMulti, F>(a.grad, a.n_ranks, e, acc);
     uint16_t g16[kVec];
     float g[kVec];
-    mean_bf16(acc, a.inv_n, g16, g, sq, nf);
+    mean_bf16<F>(acc, a.inv_n, g16, g, sq, nf);
     if (MODE == kFusedZ1) {
       const uint4 gw = pack8(g16);
       for (int r = 0; r < a.n_ranks; ++r) st_stream(const_cast<uint16_t*>(a.grad[r]) + e, gw);
     }
     if (a.grad_shard) st_stream(a.grad_shard + e, pack8(g16));
     uint16_t p16[kVec];
-    adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+    adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
     st_stream(a.m + e, m0);
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
 
 // ------------------------------------------------------ unfused kernels --
 
-template <bool kMulti>
+template <bool kMulti, class F>
 __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant__ ReduceArgs a) {
   double sq = 0.0;
   unsigned long long nf = 0;
@@ -71,10 +71,10 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
     const int64_t e = vi * kVec;
     float acc[kVec];
-    reduce_ranks<kMulti>(a.grad, a.n_ranks, e, acc);
+    reduce_ranks<kMulti, F>(a.grad, a.n_ranks, e, acc);
     uint16_t g16[kVec];
     float g[kVec];
-    mean_bf16(acc, a.inv_n, g16, g, sq, nf);
+    mean_bf16<F>(acc, a.inv_n, g16, g, sq, nf);
     const uint4 gw = pack8(g16);
     if (a.shard_out) st_stream(a.shard_out + e, gw);
     if (a.write_back)
@@ -83,6 +83,7 @@ __global__ void __launch_bounds__(kThreads) reduce_kernel(const __grid_constant_
   norm_epilogue<kThreads>(a.ns, sq, nf, a.accumulate);
 }
 
+template <class F>
 __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ AdamArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
@@ -91,10 +92,10 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
     float4 m0 = ld_stream(a.m + e), m1 = ld_stream(a.m + e + 4);
     float4 v0 = ld_stream(a.v + e), v1 = ld_stream(a.v + e + 4);
     const uint4 gw = ld_stream(a.grad + e);
-    float g[kVec] = {bf16_lo(gw.x), bf16_hi(gw.x), bf16_lo(gw.y), bf16_hi(gw.y),
-                     bf16_lo(gw.z), bf16_hi(gw.z), bf16_lo(gw.w), bf16_hi(gw.w)};
+    float g[kVec] = {F::lo(gw.x), F::hi(gw.x), F::lo(gw.y), F::hi(gw.y),
+                     F::lo(gw.z), F::hi(gw.z), F::lo(gw.w), F::hi(gw.w)};
     uint16_t p16[kVec];
-    adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+    adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
     st_stream(a.m + e, m0);
@@ -105,6 +106,7 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
   }
 }
 
+template <class F>
 __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_constant__ AdamBcastArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
@@ -114,14 +116,10 @@ __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_const
     float4 m0 = ld_stream(a.m + e), m1 = ld_stream(a.m + e + 4);
     float4 v0 = ld_stream(a.v + e), v1 = ld_stream(a.v + e + 4);
     const uint4 gw = ld_stream(a.gsrc[i / a.shard] + i);
-    float g[kVec] = {bf16_lo(gw.x), bf16_hi(gw.x), bf16_lo(gw.y), bf16_hi(gw.y),
-                     bf16_lo(gw.z), bf16_hi(gw.z), bf16_lo(gw.w), bf16_hi(gw.w)};
-    if (a.apply_coef) {
-#pragma unroll
-      for (int j = 0; j < kVec; ++j) g[j] = __fmul_rn(g[j], a.coef);
-    }
+    float g[kVec] = {F::lo(gw.x), F::hi(gw.x), F::lo(gw.y), F::hi(gw.y),
+                     F::lo(gw.z), F::hi(gw.z), F::lo(gw.w), F::hi(gw.w)};
     uint16_t p16[kVec];
-    adam8(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+    adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);  // unscale and clip via a.sc.flags
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
     st_stream(a.m + e, m0);
@@ -146,6 +144,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
 // Optimizer state from sources (fresh master weights with m = v = 0, or a
 // checkpoint's master/m/v), zeros past the sources, bf16(master) to every
 // parameter destination, reduced-gradient shards cleared.
+template <class F>
 __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ InitArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -161,8 +160,8 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
     st_stream(a.m + e + 4, m1);
     st_stream(a.v + e, v0);
     st_stream(a.v + e + 4, v1);
-    const uint16_t h[kVec] = {to_bf16(p0.x), to_bf16(p0.y), to_bf16(p0.z), to_bf16(p0.w),
-                              to_bf16(p1.x), to_bf16(p1.y), to_bf16(p1.z), to_bf16(p1.w)};
+    const uint16_t h[kVec] = {F::rn(p0.x), F::rn(p0.y), F::rn(p0.z), F::rn(p0.w),
+                              F::rn(p1.x), F::rn(p1.y), F::rn(p1.z), F::rn(p1.w)};
     const uint4 w = pack8(h);
     for (int r = 0; r < a.n_out; ++r) st_stream(a.out[r] + e, w);
     if (a.grad_shard) st_stream(a.grad_shard + e, make_uint4(0u, 0u, 0u, 0u));
@@ -173,34 +172,46 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
 
 // --------------------------------------------------------------- launchers --
 
-template <int MODE>
+template <int MODE, class F>
 void launch_fused_mode(const FusedArgs& a, int grid, cudaStream_t s) {
   if (a.n_ranks <= 8)
-    fused_step_kernel<MODE, false><<<grid, kThreads, 0, s>>>(a);
+    fused_step_kernel<MODE, false, F><<<grid, kThreads, 0, s>>>(a);
   else
-    fused_step_kernel<MODE, true><<<grid, kThreads, 0, s>>>(a);
+    fused_step_kernel<MODE, true, F><<<grid, kThreads, 0, s>>>(a);
 }
 
-cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
+template <class F>
+cudaError_t launch_fused_fmt(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
   switch (mode) {
-    case kFusedZ1: launch_fused_mode<kFusedZ1>(a, grid, s); break;
-    case kFusedZ2: launch_fused_mode<kFusedZ2>(a, grid, s); break;
-    case kFusedZ3: launch_fused_mode<kFusedZ3>(a, grid, s); break;
+    case kFusedZ1: launch_fused_mode<kFusedZ1, F>(a, grid, s); break;
+    case kFusedZ2: launch_fused_mode<kFusedZ2, F>(a, grid, s); break;
+    case kFusedZ3: launch_fused_mode<kFusedZ3, F>(a, grid, s); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s) {
+cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
+  return a.fmt == kFmtF16 ? launch_fused_fmt<F16>(mode, a, grid, s) : launch_fused_fmt<Bf16>(mode, a, grid, s);
+}
+
+template <class F>
+void launch_reduce_fmt(const ReduceArgs& a, int grid, cudaStream_t s) {
   if (a.n_ranks <= 8)
-    reduce_kernel<false><<<grid, kThreads, 0, s>>>(a);
+    reduce_kernel<false, F><<<grid, kThreads, 0, s>>>(a);
   else
-    reduce_kernel<true><<<grid, kThreads, 0, s>>>(a);
+    reduce_kernel<true, F><<<grid, kThreads, 0, s>>>(a);
+}
+
+cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s) {
+  if (a.fmt == kFmtF16) launch_reduce_fmt<F16>(a, grid, s);
+  else launch_reduce_fmt<Bf16>(a, grid, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s) {
-  adam_kernel<<<grid, kThreads, 0, s>>>(a);
+  if (a.fmt == kFmtF16) adam_kernel<F16><<<grid, kThreads, 0, s>>>(a);
+  else adam_kernel<Bf16><<<grid, kThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -210,12 +221,14 @@ cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s) {
 }
 
 cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s) {
-  adam_bcast_kernel<<<grid, kThreads, 0, s>>>(a);
+  if (a.fmt == kFmtF16) adam_bcast_kernel<F16><<<grid, kThreads, 0, s>>>(a);
+  else adam_bcast_kernel<Bf16><<<grid, kThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s) {
-  init_kernel<<<grid, kThreads, 0, s>>>(a);
+  if (a.fmt == kFmtF16) init_kernel<F16><<<grid, kThreads, 0, s>>>(a);
+  else init_kernel<Bf16><<<grid, kThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -231,21 +244,21 @@ cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_bloc
   const bool multi = n_ranks > 8;
   switch (mode) {
     case kFusedZ1:
-      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ1, true>, &e) : blocks_of(fused_step_kernel<kFusedZ1, false>, &e);
+      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ1, true, Bf16>, &e) : blocks_of(fused_step_kernel<kFusedZ1, false, Bf16>, &e);
       break;
     case kFusedZ2:
-      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ2, true>, &e) : blocks_of(fused_step_kernel<kFusedZ2, false>, &e);
+      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ2, true, Bf16>, &e) : blocks_of(fused_step_kernel<kFusedZ2, false, Bf16>, &e);
       break;
     case kFusedZ3:
-      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ3, true>, &e) : blocks_of(fused_step_kernel<kFusedZ3, false>, &e);
+      *fused_blocks = multi ? blocks_of(fused_step_kernel<kFusedZ3, true, Bf16>, &e) : blocks_of(fused_step_kernel<kFusedZ3, false, Bf16>, &e);
       break;
     default: return cudaErrorInvalidValue;
   }
-  int mn = multi ? blocks_of(reduce_kernel<true>, &e) : blocks_of(reduce_kernel<false>, &e);
-  mn = std::min(mn, blocks_of(adam_kernel, &e));
+  int mn = multi ? blocks_of(reduce_kernel<true, Bf16>, &e) : blocks_of(reduce_kernel<false, Bf16>, &e);
+  mn = std::min(mn, blocks_of(adam_kernel<Bf16>, &e));
   mn = std::min(mn, blocks_of(gather_kernel, &e));
-  mn = std::min(mn, blocks_of(adam_bcast_kernel, &e));
-  mn = std::min(mn, blocks_of(init_kernel, &e));
+  mn = std::min(mn, blocks_of(adam_bcast_kernel<Bf16>, &e));
+  mn = std::min(mn, blocks_of(init_kernel<Bf16>, &e));
   *simple_blocks = mn;
   return e;
 }

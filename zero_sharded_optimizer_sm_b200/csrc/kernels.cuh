@@ -21,10 +21,17 @@ constexpr int kTmaMaxStages = 8;                // ring depth limit of the stage
 constexpr int kTmaDefaultStages = 4;            // ring depth when the caller does not choose
 constexpr int kWideGroup = 3;  // "groups" value that selects one group of 16 consumer warps
 
-// Binary32 scalars of one Adam step, each rounded once from binary64 on the host.
+// Binary32 scalars of one Adam step, each rounded once from binary64 on the host,
+// and the gradient factors applied before the update (flags say which).
+enum AdamFlags { kUnscale = 1, kClip = 2 };
 struct AdamScalars {
   float b1, b2, omb1, omb2, bc1, bc2, decay, lr, eps;
+  float inv_scale;  // fp32(1 / loss scale), applied when flags & kUnscale
+  float coef;       // clipping coefficient, applied when flags & kClip
+  int flags;
 };
+
+enum StorageFormat { kFmtBf16 = 0, kFmtF16 = 1 };
 
 // Gradient-norm / non-finite accumulation in the scratch arena.
 struct NormScratch {
@@ -39,6 +46,7 @@ struct NormScratch {
 // Fused reduce + Adam + broadcast over one interval [lo, hi) of the flat space.
 // Every pointer is already offset to flat element lo of its buffer.
 struct FusedArgs {
+  int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* grad[kMaxRanks];  // rank r's bf16 gradient (stage 1: written back)
   uint16_t* out[kMaxRanks];         // rank r's bf16 parameter destination
   float* master;
@@ -56,6 +64,7 @@ struct FusedArgs {
 
 // Reduce only (reduce-scatter to a shard, or all-reduce written back).
 struct ReduceArgs {
+  int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* grad[kMaxRanks];
   uint16_t* shard_out;              // reduce-scatter destination, or nullptr
   int64_t n_vec;
@@ -67,6 +76,7 @@ struct ReduceArgs {
 };
 
 struct AdamArgs {
+  int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* grad;
   float* master;
   float* m;
@@ -81,6 +91,7 @@ struct AdamArgs {
 // gsrc[i / shard] + i (the owner's copy); every pointer but gsrc is at flat
 // element `lo`.
 struct AdamBcastArgs {
+  int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* gsrc[kMaxRanks];
   uint16_t* out[kMaxRanks];
   float* master;
@@ -91,9 +102,7 @@ struct AdamBcastArgs {
   int64_t shard;
   int64_t n_vec;
   int n_out;
-  int apply_coef;                   // scale the gradient by coef (coef < 1)
-  float coef;
-  AdamScalars sc;
+  AdamScalars sc;                   // including the unscale / clip factors
 };
 
 struct GatherArgs {
@@ -104,6 +113,7 @@ struct GatherArgs {
 };
 
 struct InitArgs {
+  int fmt;                          // StorageFormat of every 16-bit buffer
   const float* master_src;          // elements [0, n_src_vec*8) come from these sources,
   const float* m_src;               // m and v are 0 where their source is nullptr,
   const float* v_src;               // everything beyond the sources is 0

@@ -61,6 +61,8 @@ struct zero_ctx {
   bool loaded = false;
   int64_t t = 0;
   int64_t stats_step = 0;
+  int fmt = zsm::kFmtBf16;     // storage format of gradients and parameters
+  double loss_scale = 1.0;     // the gradients the ranks hold are loss_scale x the true ones
   double clip_norm = 0.0;      // > 0: global-norm clipping
   bool skip_nonfinite = false;
   double last_coef = 1.0;      // statistics of the last two-pass step
@@ -155,6 +157,19 @@ zsm::NormScratch norm_scratch(zero_ctx* c) {
   return ns;
 }
 
+zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t);
+
+// The step's scalars plus the gradient factors: fp32(1/loss_scale) when that
+// is not 1, and a clipping coefficient when below 1.
+zsm::AdamScalars step_scalars(const zero_ctx* c, int64_t t, float coef) {
+  zsm::AdamScalars s = adam_scalars(c->hp, t);
+  s.inv_scale = (float)(1.0 / c->loss_scale);
+  if (s.inv_scale != 1.0f) s.flags |= zsm::kUnscale;
+  s.coef = coef;
+  if (coef < 1.0f) s.flags |= zsm::kClip;
+  return s;
+}
+
 zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
   double p1 = 1.0, p2 = 1.0;
   for (int64_t k = 0; k < t; ++k) {
@@ -171,6 +186,9 @@ zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
   s.decay = (float)(1.0 - hp.lr * hp.weight_decay);
   s.lr = (float)hp.lr;
   s.eps = (float)hp.eps;
+  s.inv_scale = 1.0f;
+  s.coef = 1.0f;
+  s.flags = 0;
   return s;
 }
 
@@ -297,6 +315,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
   std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
   for (int r = 0; r < N; ++r) {
     a.grad[r] = grad[r];
     if (c->stage == ZERO_STAGE_3) {
@@ -362,7 +381,7 @@ zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
   zero_status st = check_device_error(c, host.error, s);
   if (st != ZERO_OK) return st;
   std::memset(out, 0, sizeof *out);
-  out->grad_norm = std::sqrt(host.sq);
+  out->grad_norm = std::sqrt(host.sq) / c->loss_scale;
   out->nonfinite = (int64_t)host.nf;
   out->step = c->stats_step;
   zero_comm_elems(c, out->comm_elems);
@@ -406,6 +425,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     const int64_t lo = iv[k].lo, hi = iv[k].hi;
     zsm::ReduceArgs a;
     std::memset(&a, 0, sizeof a);
+    a.fmt = c->fmt;
     for (int r = 0; r < N; ++r) {
       if (resident) {
         a.grad[r] = static_cast<const uint16_t*>(resident[r]) + lo;
@@ -434,7 +454,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   unsigned long long nf = 0;
   zero_status st = read_norm(c, s, &sq, &nf);
   if (st != ZERO_OK) return st;
-  const double norm = std::sqrt(sq);
+  const double norm = std::sqrt(sq) / c->loss_scale;  // of the unscaled gradient
   c->last_skipped = (c->skip_nonfinite && nf > 0) ? 1 : 0;
   c->last_coef = 1.0;
   if (!c->last_skipped) {
@@ -442,7 +462,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     if (c->clip_norm > 0.0) coef = (float)(c->clip_norm / (norm + 1e-6));
     const bool apply = coef < 1.0f;
     c->last_coef = apply ? (double)coef : 1.0;
-    const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+    const zsm::AdamScalars sc = step_scalars(c, t, apply ? coef : 1.0f);
     // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3)
     std::vector<zsm::Span> p2;
     if (c->stage == ZERO_STAGE_3) p2 = iv;
@@ -452,6 +472,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
       const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
       zsm::AdamBcastArgs b;
       std::memset(&b, 0, sizeof b);
+      b.fmt = c->fmt;
       for (int r = 0; r < N; ++r) {
         if (c->stage == ZERO_STAGE_1)
           b.gsrc[r] = resident ? static_cast<const uint16_t*>(resident[r]) : grad_buf_ptr(c, r);
@@ -467,8 +488,6 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
       b.lo = lo;
       b.shard = c->plan.shard;
       b.n_vec = (hi - lo) / zsm::kVec;
-      b.apply_coef = apply ? 1 : 0;
-      b.coef = coef;
       b.sc = sc;
       if (b.n_vec > 0) {
         cudaError_t e = zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
@@ -507,7 +526,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   c->last_skipped = 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t t = c->t + 1;
-  const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
   const std::vector<zsm::Span> iv = step_intervals(c);
   std::vector<uint16_t*> grad(N), bufs(N);
   const int n_layers = (int)c->plan.layers.size();
@@ -612,6 +631,10 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     case ZERO_OPT_GRAD_BUFFERS:
       c->grad_buffers = value != 0;
       break;
+    case ZERO_OPT_DTYPE:
+      if (value != ZERO_DTYPE_BF16 && value != ZERO_DTYPE_F16) return fail(c, ZERO_EINVAL, "unknown dtype %lld", (long long)value);
+      c->fmt = value == ZERO_DTYPE_F16 ? zsm::kFmtF16 : zsm::kFmtBf16;
+      break;
     case ZERO_OPT_BLOCKS_PER_SM:
       if (value < 0 || value > 32) return fail(c, ZERO_EINVAL, "blocks per SM must be 0..32");
       c->blocks_per_sm_opt = (int)value;
@@ -712,6 +735,7 @@ zero_status load_state(zero_ctx* c, const float* master, const float* m, const f
   if (e != cudaSuccess) return cuda_fail(c, e, "clearing scratch");
   zsm::InitArgs a;
   std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
   a.master_src = master;
   a.m_src = m;
   a.v_src = v;
@@ -832,6 +856,7 @@ zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void*
   const int N = c->plan.n_ranks;
   zsm::ReduceArgs a;
   std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
   if (rank_grads) {
     for (int r = 0; r < N; ++r) {
       if (!rank_grads[r] || !aligned16(rank_grads[r]))
@@ -871,6 +896,7 @@ zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
   const int N = c->plan.n_ranks;
   zsm::ReduceArgs a;
   std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
   if (!rank_grads && !c->arena[ZERO_ARENA_GRADS])
     return fail(c, ZERO_EINVAL, "rank_grads is NULL but there are no gradient buffers");
   for (int r = 0; r < N; ++r) {
@@ -902,7 +928,7 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
     return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
   if (c->stage == ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRADS])
     return fail(c, ZERO_ESTATE, "stage 1 Adam reads the gradient buffers, which were dropped");
-  const zsm::AdamScalars sc = adam_scalars(c->hp, t);
+  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
   const int64_t S = c->plan.shard;
   const int r0 = rank < 0 ? 0 : rank, r1 = rank < 0 ? N : rank + 1;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -913,6 +939,7 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
   const int64_t lo = r0 * S, hi = r1 * S;
   zsm::AdamArgs a;
   std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
   a.sc = sc;
   a.master = master_ptr(c) + lo;
   a.m = m_ptr(c) + lo;
@@ -1055,6 +1082,13 @@ zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, doubl
     if (e != cudaSuccess) return cuda_fail(c, e, "reading the device error word");
     return check_device_error(c, err, nullptr);
   }
+  return ZERO_OK;
+}
+
+zero_status zero_set_loss_scale(zero_ctx* c, double scale) {
+  if (!c) return ZERO_EINVAL;
+  if (!(scale > 0.0) || std::isinf(scale)) return fail(c, ZERO_EINVAL, "the loss scale must be finite and > 0");
+  c->loss_scale = scale;
   return ZERO_OK;
 }
 
