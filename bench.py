@@ -66,6 +66,10 @@ def parse_args(argv=None):
     ap.add_argument("--stages", action="store_true",
                     help="ZeRO-1/2/3 fused-step throughput on the 1.2B (N=8) and 85M (N=8) workloads "
                          "and ZeRO-3 on the 6.4B (N=64) workload; one JSON line per cell")
+    ap.add_argument("--overlap", action="store_true",
+                    help="ZERO_OPT_PIPELINE: step time with the gradient producer (the seeded "
+                         "generator standing in for the backward) run in order vs one interval ahead "
+                         "on the context's stream, on the 1.2B and 85M workloads; one JSON line per cell")
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
@@ -642,6 +646,84 @@ def run_reference(args, world, rank, local):
     }), flush=True)
 
 
+def run_overlap(args):
+    """Overlap of the caller's backward with the step (ZERO_OPT_PIPELINE).
+    grad_fn stands in for the backward: it draws each rank's gradients of the
+    interval with the seeded generator (one launch per rank; an integer-hash
+    kernel, so it competes with the HBM-bound step for issue slots rather than
+    for bandwidth).  Per cell: the step time in order (grad_fn, then the
+    interval's kernel, on one stream) and pipelined (grad_fn one interval
+    ahead on the context's own stream), both CUDA events on the caller's
+    stream around whole steps; the generator alone and the step's kernels
+    alone (from runs in order) bound what overlap can reach: in order costs
+    about their sum, perfect overlap their maximum."""
+    import torch
+
+    import synth
+    import zero_sharded_optimizer_sm_b200 as z
+    from synth import workloads as W
+
+    torch.cuda.set_device(0)
+    s = torch.cuda.current_stream().cuda_stream
+    kern = {"auto": 0, "register": 1, "tma": 2}[args.kernel]
+    cells = [(W.gpt_1p2b_n8(), 3, None), (W.gpt_1p2b_n8(), 2, 200_000_000), (W.gpt_85m_n8(), 3, None),
+             (W.gpt_85m_n8(), 2, 20_000_000)]
+    for w, stage, bucket in cells:
+        res = {}
+        for pipe in (False, True):
+            opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=bucket,
+                                  hparams=z.AdamHParams(), keep_grad_shards=False, kernel=kern, pipeline=pipe)
+            assert opt.psi_pad == w.psi and all(o + n == e for o, n, e in
+                                                zip(opt.offsets(), w.numel, opt.offsets()[1:] + [w.psi]))
+            mv = opt.view(z.ZERO_VIEW_MASTER)
+            synth.dev_f32(W.master_base(w), 0, w.psi, W.MASTER_DIST, mv.data_ptr(), s)
+            opt.load_master(None)
+
+            def gfn(t, lo, hi, bufs, stream):  # no pads in these layouts: one range per rank
+                for r, ptr in enumerate(bufs):
+                    synth.dev_bf16(W.grad_base(w, 1, r), lo, hi - lo, w.grad_dist, ptr, stream)
+                return 0
+
+            for _ in range(3):
+                opt.step(gfn)
+            steps = 5
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            opt.set_timing(not pipe)
+            opt.kernel_timing()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(steps):
+                opt.step(gfn)
+            e1.record()
+            torch.cuda.synchronize()
+            res["pipelined" if pipe else "in_order"] = e0.elapsed_time(e1) / steps
+            if not pipe:
+                kt = opt.kernel_timing()
+                res["kernels_alone"] = kt["ms"] / steps
+                iv = opt.buckets() if stage != 3 else [(lo, hi) for _, lo, hi in reversed(opt.layers())]
+                bufs = [opt.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() for r in range(w.n_ranks)]
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(steps):
+                    for lo, hi in iv:
+                        gfn(1, lo, hi, bufs, s)
+                e1.record()
+                torch.cuda.synchronize()
+                res["grad_fn_alone"] = e0.elapsed_time(e1) / steps
+                res["intervals"] = len(iv)
+            opt.close()
+            del opt, mv
+            torch.cuda.empty_cache()
+        lower = max(res["kernels_alone"], res["grad_fn_alone"])
+        hidden = (res["in_order"] - res["pipelined"]) / min(res["kernels_alone"], res["grad_fn_alone"])
+        print(json.dumps({"overlap": w.name, "stage": stage, "n_ranks": w.n_ranks, "params": w.psi,
+                          "intervals": res["intervals"], "bucket_elems": bucket,
+                          "ms_in_order": res["in_order"], "ms_pipelined": res["pipelined"],
+                          "ms_kernels_alone": res["kernels_alone"], "ms_grad_fn_alone": res["grad_fn_alone"],
+                          "ms_perfect_overlap": lower, "speedup": res["in_order"] / res["pipelined"],
+                          "fraction_of_shorter_phase_hidden": hidden, "steps": steps}), flush=True)
+
+
 def main(argv=None):
     global _ARGS
     args = parse_args(argv)
@@ -657,6 +739,8 @@ def main(argv=None):
         run_sweep(args)
     elif args.stages:
         run_stages(args)
+    elif args.overlap:
+        run_overlap(args)
     else:
         run_ours(args, world, rank, local)
 

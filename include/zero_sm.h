@@ -150,9 +150,21 @@ enum {
                                     set at any time */
   ZERO_OPT_TMA_CTAS_PER_SM = 9,  /* staged kernel: CTAs per SM, 1..4, capped by what fits in
                                     shared memory (0 = the library's choice); any time */
-  ZERO_OPT_DTYPE = 10            /* storage format of every 16-bit buffer (gradients,
+  ZERO_OPT_DTYPE = 10,           /* storage format of every 16-bit buffer (gradients,
                                     parameters, reduced shards): ZERO_DTYPE_BF16 (default) or
                                     ZERO_DTYPE_F16 (IEEE binary16); before zero_bind */
+  ZERO_OPT_PIPELINE = 11         /* 1: zero_step / zero_step_resident run grad_fn and
+                                    gather_fn on a stream of the context's own, one interval
+                                    ahead of the kernels on the caller's stream, so that the
+                                    caller's backward of the next interval and its use of the
+                                    last gathered layer overlap the step's kernel -- the
+                                    overlap and prefetch that ZeRO-3's layer-by-layer gathers
+                                    and reduce-scatters depend on ([T] section "ZeRO-3", part
+                                    on its communication volume; [Q] section 五).  Stages 2 and
+                                    3 then hold two gradient slot sets (GRADS doubles) and
+                                    stage 3 two gather slot sets (GATHER doubles), used
+                                    alternately; stage 1 needs none.  Values are unchanged.
+                                    Default 0; before zero_bind */
 };
 
 /* 16-bit storage formats (ZERO_OPT_DTYPE).  The pages account gradients and
@@ -186,8 +198,11 @@ enum {
   ZERO_VIEW_PARAM = 3,       /* bf16: rank r's replica [psi_pad] (stage 1, 2) or the
                                 shards [psi_pad] (stage 3, rank ignored) */
   ZERO_VIEW_GRAD_SHARD = 4,  /* bf16 [psi_pad] (stage 2, 3) */
-  ZERO_VIEW_GRAD_BUF = 5,    /* bf16: rank r's gradient input buffer */
-  ZERO_VIEW_GATHER = 6       /* bf16: rank r's temporary full-layer buffer (stage 3) */
+  ZERO_VIEW_GRAD_BUF = 5,    /* bf16: rank r's gradient input buffer; with ZERO_OPT_PIPELINE
+                                at stage 2/3, rank r + N is rank r's buffer in the second
+                                slot set */
+  ZERO_VIEW_GATHER = 6       /* bf16: rank r's temporary full-layer buffer (stage 3); with
+                                ZERO_OPT_PIPELINE, rank r + N is the second slot set's */
 };
 
 typedef struct zero_ctx zero_ctx;
@@ -199,7 +214,10 @@ typedef struct zero_ctx zero_ctx;
  * before that interval is reduced.  It must fill, for every rank r, the
  * hi - lo bf16 values of flat elements [lo, hi) at rank_bufs[r] (device
  * pointers into the GRADS arena) with work enqueued on `stream`.  Returns 0
- * on success; any other value aborts the step with ZERO_EINVAL.
+ * on success; any other value aborts the step with ZERO_EINVAL.  With
+ * ZERO_OPT_PIPELINE, `stream` is the context's own stream (not the one given
+ * to zero_step), the call for interval k+1 comes before the step's kernel of
+ * interval k has run, and consecutive intervals get alternating buffers.
  */
 typedef int (*zero_grad_fn)(void* user, int64_t step, int64_t lo, int64_t hi,
                             void* const* rank_bufs, void* stream);
@@ -209,7 +227,11 @@ typedef int (*zero_grad_fn)(void* user, int64_t step, int64_t lo, int64_t hi,
  * parts "1. 前向" and "2. 反向"): called after the layer [lo, hi) has been
  * gathered into every rank's temporary buffer rank_bufs[r] (hi - lo bf16
  * values) and before the buffer is reused for the next layer.  Work must be
- * enqueued on `stream`.  Returns 0 on success.
+ * enqueued on `stream`.  Returns 0 on success.  With ZERO_OPT_PIPELINE,
+ * `stream` is the context's own stream, consecutive layers come in
+ * alternating buffers, and the call for layer k follows the grad_fn call of
+ * the next interval; the buffers stay valid until the work enqueued by the
+ * call has run.
  */
 typedef int (*zero_gather_fn)(void* user, int32_t layer, int64_t lo, int64_t hi,
                               void* const* rank_bufs, void* stream);

@@ -100,7 +100,10 @@ class DeviceFill:
         b = W.grad_base(self.w, step, rank)
         segs = real_segments(self.offsets, self.w.numel, lo, hi)
         if self.has_pads:
-            buf_tensor[: hi - lo].zero_()
+            import torch
+
+            with torch.cuda.stream(torch.cuda.ExternalStream(stream) if stream else torch.cuda.default_stream()):
+                buf_tensor[: hi - lo].zero_()
         for a, e in segs:
             self.fill16(b, a, e - a, self.w.grad_dist, buf_ptr + 2 * (a - lo), stream)
 

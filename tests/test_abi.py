@@ -79,6 +79,7 @@ LAYOUTS = [
     ([7, 0, 11, 13, 2], [0, 0, 1, 2, 2]),
     W.transformer_layers(3, 24, 96),
     ([100], [0]),
+    ([16, 0, 24, 0], [0, 1, 2, 3]),  # empty layers (all-zero tensors), first in reverse order at N = 1, 5
 ]
 
 
@@ -124,6 +125,31 @@ def test_planner_matches_oracle_plan(layout, n_ranks, bucket):
                 pass
         finally:
             z.zero_destroy(ctx)
+
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_pipeline_option_doubles_only_the_slot_arenas(stage):
+    """ZERO_OPT_PIPELINE (set before binding): a second gradient slot set at
+    stage 2/3 and a second gather slot set at stage 3; stage 1 and every other
+    arena unchanged."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    numel, layer = W.transformer_layers(3, 24, 96)
+    sizes = []
+    for pipe in (0, 1):
+        st, ctx = _init(numel, layer, 4, stage, 4096)
+        assert st == 0
+        try:
+            assert z.zero_set_option(ctx, z.ZERO_OPT_PIPELINE, pipe) == 0
+            zs = z.zero_sizes()
+            assert z.zero_buffer_sizes(ctx, ctypes.byref(zs)) == 0
+            sizes.append(list(zs.arena_bytes))
+        finally:
+            z.zero_destroy(ctx)
+    off, on = sizes
+    for k in range(z.ZERO_NUM_ARENAS):
+        doubled = (k == z.ZERO_ARENA_GRADS and stage != 1) or (k == z.ZERO_ARENA_GATHER and stage == 3)
+        assert on[k] == (2 * off[k] if doubled else off[k]), (k, off[k], on[k])
 
 
 def test_init_rejects_bad_arguments():

@@ -182,7 +182,8 @@ def test_flat_1m_n4_zero2_every_element():
 
 
 TINY = [([1], [0]), ([5, 3], [0, 1]), ([8, 16, 9], [0, 0, 1]), ([33, 1, 2, 17], [0, 1, 1, 2]),
-        ([7, 0, 11, 13, 2], [0, 0, 1, 2, 2]), ([3000, 1, 4100], [0, 1, 2])]
+        ([7, 0, 11, 13, 2], [0, 0, 1, 2, 2]), ([3000, 1, 4100], [0, 1, 2]),
+        ([16, 0, 24, 0], [0, 1, 2, 3])]  # empty layers; at N = 1 and 5 the first in reverse order
 
 
 @pytest.mark.parametrize("layout", TINY)

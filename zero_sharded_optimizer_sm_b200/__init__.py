@@ -44,6 +44,7 @@ ZERO_OPT_TMA_GROUPS = 7
 ZERO_OPT_TMA_STAGES = 8
 ZERO_OPT_TMA_CTAS_PER_SM = 9
 ZERO_OPT_DTYPE = 10
+ZERO_OPT_PIPELINE = 11
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -159,7 +160,8 @@ class ZeroOptimizer:
                  bucket_elems: Optional[int] = None, hparams: AdamHParams = AdamHParams(),
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
-                 tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16, device=None):
+                 tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16,
+                 pipeline: bool = False, device=None):
         import torch
 
         self._torch = torch
@@ -197,6 +199,9 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_DTYPE, int(dtype)), "zero_set_option")
         if tma_ctas_per_sm:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_CTAS_PER_SM, int(tma_ctas_per_sm)), "zero_set_option")
+        if pipeline:
+            self._check(zero_set_option(ctx, ZERO_OPT_PIPELINE, 1), "zero_set_option")
+        self.pipeline = bool(pipeline)
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)

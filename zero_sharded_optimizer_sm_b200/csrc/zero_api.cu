@@ -68,6 +68,12 @@ struct zero_ctx {
   double last_coef = 1.0;      // statistics of the last two-pass step
   int64_t last_skipped = 0;
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
+  // callback pipeline (ZERO_OPT_PIPELINE): side stream and ordering events
+  bool pipeline = false;
+  int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_start = nullptr, ev_join = nullptr;
+  cudaEvent_t ev_grads[2] = {}, ev_kernel[2] = {}, ev_consumed[2] = {};
   // fused-kernel timing
   bool timing = false;
   std::vector<cudaEvent_t> events;  // pairs (start, end), reused
@@ -76,6 +82,10 @@ struct zero_ctx {
   std::string err;
   ~zero_ctx() {
     for (cudaEvent_t e : events) cudaEventDestroy(e);
+    for (cudaEvent_t e : {ev_start, ev_join, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
+                          ev_consumed[0], ev_consumed[1]})
+      if (e) cudaEventDestroy(e);
+    if (side) cudaStreamDestroy(side);
   }
 };
 
@@ -106,6 +116,10 @@ void compute_layout(zero_ctx* c) {
   std::fill(c->arena_bytes, c->arena_bytes + ZERO_NUM_ARENAS, 0);
   c->arena_bytes[ZERO_ARENA_STATES] = 3 * c->state_pitch;
   c->arena_bytes[ZERO_ARENA_SCRATCH] = kScratchBytes;
+  // Stage 1's intervals are disjoint ranges of the full replicas, so the
+  // pipeline needs a second slot set only for the stage 2 bucket and the
+  // stage 3 layer buffers.
+  c->slots = (c->pipeline && c->stage != ZERO_STAGE_1) ? 2 : 1;
   switch (c->stage) {
     case ZERO_STAGE_1:
       c->grad_pitch = c->param_pitch;
@@ -115,7 +129,7 @@ void compute_layout(zero_ctx* c) {
     case ZERO_STAGE_2:
       c->grad_pitch = align_up(p.max_bucket * 2, kArenaAlign) + c->replica_pad;
       c->arena_bytes[ZERO_ARENA_PARAMS] = N * c->param_pitch;
-      c->arena_bytes[ZERO_ARENA_GRADS] = N * c->grad_pitch;
+      c->arena_bytes[ZERO_ARENA_GRADS] = c->slots * N * c->grad_pitch;
       c->arena_bytes[ZERO_ARENA_GRAD_SHARDS] = c->keep_grad_shards ? row2 : 0;
       break;
     case ZERO_STAGE_3:
@@ -123,9 +137,9 @@ void compute_layout(zero_ctx* c) {
       c->grad_pitch = align_up(p.max_layer * 2, kArenaAlign) + c->replica_pad;
       c->gather_pitch = c->grad_pitch;
       c->arena_bytes[ZERO_ARENA_PARAMS] = row2;
-      c->arena_bytes[ZERO_ARENA_GRADS] = N * c->grad_pitch;
+      c->arena_bytes[ZERO_ARENA_GRADS] = c->slots * N * c->grad_pitch;
       c->arena_bytes[ZERO_ARENA_GRAD_SHARDS] = c->keep_grad_shards ? row2 : 0;
-      c->arena_bytes[ZERO_ARENA_GATHER] = N * c->gather_pitch;
+      c->arena_bytes[ZERO_ARENA_GATHER] = c->slots * N * c->gather_pitch;
       break;
   }
   if (!c->grad_buffers) c->arena_bytes[ZERO_ARENA_GRADS] = 0;
@@ -137,12 +151,15 @@ float* v_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_
 uint16_t* param_ptr(zero_ctx* c, int r) {  // replica r (stage 1, 2) or the shards (stage 3)
   return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_PARAMS] + (c->stage == ZERO_STAGE_3 ? 0 : r * c->param_pitch));
 }
-uint16_t* grad_buf_ptr(zero_ctx* c, int r) {
-  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GRADS] + r * c->grad_pitch);
+// Rank r's gradient buffer in slot set `slot` (0, or 1 with the pipeline).
+uint16_t* grad_buf_ptr(zero_ctx* c, int r, int slot = 0) {
+  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GRADS] +
+                                     ((int64_t)slot * c->plan.n_ranks + r) * c->grad_pitch);
 }
 uint16_t* grad_shard_ptr(zero_ctx* c) { return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GRAD_SHARDS]); }
-uint16_t* gather_ptr(zero_ctx* c, int r) {
-  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GATHER] + r * c->gather_pitch);
+uint16_t* gather_ptr(zero_ctx* c, int r, int slot = 0) {
+  return reinterpret_cast<uint16_t*>(c->arena[ZERO_ARENA_GATHER] +
+                                     ((int64_t)slot * c->plan.n_ranks + r) * c->gather_pitch);
 }
 
 zsm::NormScratch norm_scratch(zero_ctx* c) {
@@ -310,7 +327,7 @@ std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
 
 // One fused launch over [lo, hi).  grad[r] are at flat element lo.
 zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
-                           bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s) {
+                           bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0) {
   if (hi == lo) return ZERO_OK;
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
@@ -320,7 +337,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
     a.grad[r] = grad[r];
     if (c->stage == ZERO_STAGE_3) {
       const int64_t off = lo - c->plan.layers[layer_idx].lo;
-      a.out[r] = gather_ptr(c, r) + off;
+      a.out[r] = gather_ptr(c, r, slot) + off;
     } else {
       a.out[r] = param_ptr(c, r) + lo;
     }
@@ -408,48 +425,169 @@ zero_status read_norm(zero_ctx* c, cudaStream_t s, double* sq, unsigned long lon
   return ZERO_OK;
 }
 
+// Orders one step's work across the caller's stream `s` (every kernel) and
+// the stream the callbacks get.  Without ZERO_OPT_PIPELINE that is `s`
+// itself and everything runs in program order with one slot set.  With it,
+// the callbacks run on the context's side stream one interval ahead --
+// grad_fn(k+1) and gather_fn(k) overlap the kernel of interval k+1 or k --
+// and events keep each slot set from being refilled before its reader is done:
+//   grad_fn(k)   (side)   after the kernel of k-2 read slot k%2 (stage 2/3)
+//   kernel(k)    (s)      after grad_fn(k), and (stage 3) after gather_fn(k-2)
+//                         finished reading gather slot k%2
+//   gather_fn(k) (side)   after kernel(k)
+// and `s` waits for all of the side stream's work before the step returns.
+struct StepOrder {
+  zero_ctx* c;
+  cudaStream_t s;
+  cudaStream_t q;
+  bool on;
+  bool joined = false;
+  cudaError_t err = cudaSuccess;
+
+  StepOrder(zero_ctx* ctx, cudaStream_t stream) : c(ctx), s(stream), q(stream), on(ctx->pipeline) {
+    if (on) q = c->side;
+  }
+  void record(cudaEvent_t e, cudaStream_t st) {
+    if (err == cudaSuccess) err = cudaEventRecord(e, st);
+  }
+  void wait(cudaStream_t st, cudaEvent_t e) {
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(st, e, 0);
+  }
+  int slot(size_t k) const { return c->slots == 2 ? (int)(k & 1) : 0; }
+  size_t ahead() const { return on ? 1 : 0; }
+  void begin() {
+    if (!on) return;
+    record(c->ev_start, s);
+    wait(q, c->ev_start);
+  }
+  void before_grads(size_t k) {
+    if (on && c->slots == 2 && k >= 2) wait(q, c->ev_kernel[k & 1]);
+  }
+  void after_grads(size_t k) {
+    if (on) record(c->ev_grads[k & 1], q);
+  }
+  void before_kernel(size_t k, bool grads, size_t gather_k) {
+    if (!on) return;
+    if (grads) wait(s, c->ev_grads[k & 1]);
+    if (gather_k != (size_t)-1 && gather_k >= 2) wait(s, c->ev_consumed[gather_k & 1]);
+  }
+  void after_kernel(size_t k) {
+    if (on) record(c->ev_kernel[k & 1], s);
+  }
+  void before_gather(size_t k) {
+    if (on) wait(q, c->ev_kernel[k & 1]);
+  }
+  void after_gather(size_t k) {
+    if (on) record(c->ev_consumed[k & 1], q);
+  }
+  // Joins the side stream into `s`; returns the first CUDA error seen.
+  cudaError_t end() {
+    if (on && !joined) {
+      joined = true;
+      // the join is attempted even after an error, so that `s` never runs ahead
+      // of callback work already enqueued
+      cudaError_t e1 = cudaEventRecord(c->ev_join, q);
+      cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(s, c->ev_join, 0) : e1;
+      if (err == cudaSuccess) err = e2;
+    }
+    return err;
+  }
+};
+
+// Creates the side stream and events of ZERO_OPT_PIPELINE on first use.
+zero_status ensure_pipeline(zero_ctx* c) {
+  if (!c->pipeline || c->side) return ZERO_OK;
+  cudaError_t e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
+  for (cudaEvent_t* ev : {&c->ev_start, &c->ev_join, &c->ev_grads[0], &c->ev_grads[1], &c->ev_kernel[0],
+                          &c->ev_kernel[1], &c->ev_consumed[0], &c->ev_consumed[1]})
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(c, e, "creating the pipeline stream and events");
+  return ZERO_OK;
+}
+
+// The N gradient pointers of interval k (at flat element lo): the caller's
+// resident replicas, the full replicas at stage 1, or slot k's buffers.
+void interval_grads(zero_ctx* c, const void* const* resident, int64_t lo, int slot, uint16_t** out) {
+  const int N = c->plan.n_ranks;
+  for (int r = 0; r < N; ++r) {
+    if (resident)
+      out[r] = const_cast<uint16_t*>(static_cast<const uint16_t*>(resident[r])) + lo;
+    else
+      out[r] = c->stage == ZERO_STAGE_1 ? grad_buf_ptr(c, r) + lo : grad_buf_ptr(c, r, slot);
+  }
+}
+
+// Calls grad_fn for interval k of `iv` (no-op with resident gradients).
+zero_status issue_grads(zero_ctx* c, StepOrder& o, zero_grad_fn fn, void* user, const void* const* resident,
+                        const std::vector<zsm::Span>& iv, size_t k, int64_t t) {
+  if (resident || !fn) return ZERO_OK;
+  const int N = c->plan.n_ranks;
+  std::vector<uint16_t*> bufs(N);
+  interval_grads(c, nullptr, iv[k].lo, o.slot(k), bufs.data());
+  o.before_grads(k);
+  const int rc = fn(user, t, iv[k].lo, iv[k].hi, reinterpret_cast<void* const*>(bufs.data()), o.q);
+  if (rc != 0)
+    return fail(c, ZERO_EINVAL, "grad_fn returned %d for [%lld, %lld)", rc, (long long)iv[k].lo, (long long)iv[k].hi);
+  o.after_grads(k);
+  return ZERO_OK;
+}
+
+// Calls gather_fn for stage-3 layer `layer_idx`, whose gathered copy is in
+// gather slot `slot`.
+zero_status issue_gather(zero_ctx* c, StepOrder& o, zero_gather_fn gfn, void* guser, int layer_idx, size_t k) {
+  const int N = c->plan.n_ranks;
+  std::vector<uint16_t*> bufs(N);
+  for (int r = 0; r < N; ++r) bufs[r] = gather_ptr(c, r, o.slot(k));
+  const zsm::LayerSpan& L = c->plan.layers[layer_idx];
+  o.before_gather(k);
+  const int rc = gfn(guser, L.id, L.lo, L.hi, reinterpret_cast<void* const*>(bufs.data()), o.q);
+  if (rc != 0) return fail(c, ZERO_EINVAL, "gather_fn returned %d for layer %d", rc, L.id);
+  o.after_gather(k);
+  return ZERO_OK;
+}
+
 // Clipped / overflow-checked step: reduce everything, read the norm, then
-// Adam + broadcast.  `grad` pointers per interval as in run_step.
+// Adam + broadcast.
 zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
-                         zero_gather_fn gfn, void* guser, void* stream, zero_step_stats* stats) {
+                         zero_gather_fn gfn, void* guser, StepOrder& o, zero_step_stats* stats) {
   const int N = c->plan.n_ranks;
   if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "clipping / skipping needs the reduced-gradient shards (ZERO_OPT_KEEP_GRAD_SHARDS = 1)");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = o.s;
   const int64_t t = c->t + 1;
   const std::vector<zsm::Span> iv = step_intervals(c);
   const int n_layers = (int)c->plan.layers.size();
-  std::vector<void*> bufs(N);
+  std::vector<uint16_t*> grad(N);
   // pass 1: reduce every interval
+  bool launched = false;  // the first launch of the step starts the norm sum
+  size_t issued = 0;
   for (size_t k = 0; k < iv.size(); ++k) {
+    for (; issued < iv.size() && issued <= k + o.ahead(); ++issued) {
+      zero_status st = issue_grads(c, o, fn, user, resident, iv, issued, t);
+      if (st != ZERO_OK) return st;
+    }
     const int64_t lo = iv[k].lo, hi = iv[k].hi;
     zsm::ReduceArgs a;
     std::memset(&a, 0, sizeof a);
     a.fmt = c->fmt;
-    for (int r = 0; r < N; ++r) {
-      if (resident) {
-        a.grad[r] = static_cast<const uint16_t*>(resident[r]) + lo;
-      } else {
-        uint16_t* b = c->stage == ZERO_STAGE_1 ? grad_buf_ptr(c, r) + lo : grad_buf_ptr(c, r);
-        bufs[r] = b;
-        a.grad[r] = b;
-      }
-    }
-    if (!resident && fn) {
-      const int rc = fn(user, t, lo, hi, bufs.data(), stream);
-      if (rc != 0) return fail(c, ZERO_EINVAL, "grad_fn returned %d for [%lld, %lld)", rc, (long long)lo, (long long)hi);
-    }
+    interval_grads(c, resident, lo, o.slot(k), grad.data());
+    for (int r = 0; r < N; ++r) a.grad[r] = grad[r];
     a.shard_out = c->stage == ZERO_STAGE_1 ? nullptr : grad_shard_ptr(c) + lo;
     a.write_back = c->stage == ZERO_STAGE_1 ? 1 : 0;
     a.n_vec = (hi - lo) / zsm::kVec;
     a.n_ranks = N;
-    a.accumulate = k > 0 ? 1 : 0;
+    a.accumulate = launched ? 1 : 0;
     a.inv_n = (float)(1.0 / (double)N);
     a.ns = norm_scratch(c);
-    if (a.n_vec == 0) continue;
-    cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
-    if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
+    o.before_kernel(k, !resident && fn, (size_t)-1);
+    if (a.n_vec > 0) {
+      cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
+      if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
+      launched = true;
+    }
+    o.after_kernel(k);
   }
+  if (o.err != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
   double sq = 0.0;
   unsigned long long nf = 0;
   zero_status st = read_norm(c, s, &sq, &nf);
@@ -478,7 +616,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
           b.gsrc[r] = resident ? static_cast<const uint16_t*>(resident[r]) : grad_buf_ptr(c, r);
         else
           b.gsrc[r] = grad_shard_ptr(c);
-        b.out[r] = c->stage == ZERO_STAGE_3 ? gather_ptr(c, r) : param_ptr(c, r) + lo;
+        b.out[r] = c->stage == ZERO_STAGE_3 ? gather_ptr(c, r, o.slot(k)) : param_ptr(c, r) + lo;
       }
       b.n_out = N;
       b.master = master_ptr(c) + lo;
@@ -489,18 +627,20 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
       b.shard = c->plan.shard;
       b.n_vec = (hi - lo) / zsm::kVec;
       b.sc = sc;
+      o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
       if (b.n_vec > 0) {
         cudaError_t e = zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
         if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
       }
+      o.after_kernel(k);
       if (c->stage == ZERO_STAGE_3 && gfn) {
-        for (int r = 0; r < N; ++r) bufs[r] = gather_ptr(c, r);
-        const int rc = gfn(guser, c->plan.layers[layer_idx].id, lo, hi, bufs.data(), stream);
-        if (rc != 0) return fail(c, ZERO_EINVAL, "gather_fn returned %d for layer %d", rc, c->plan.layers[layer_idx].id);
+        st = issue_gather(c, o, gfn, guser, layer_idx, k);
+        if (st != ZERO_OK) return st;
       }
     }
     c->t = t;
   }
+  if (o.end() != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
   c->stats_step = c->t;
   c->norm_fresh = true;
   if (stats) return finish_stats(c, s, stats);
@@ -521,38 +661,42 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   } else if (!c->arena[ZERO_ARENA_GRADS]) {
     return fail(c, ZERO_ESTATE, "no gradient buffers (ZERO_OPT_GRAD_BUFFERS = 0): use zero_step_resident");
   }
-  if (c->clip_norm > 0.0 || c->skip_nonfinite) return run_two_pass(c, fn, user, resident, gfn, guser, stream, stats);
+  st = ensure_pipeline(c);
+  if (st != ZERO_OK) return st;
+  StepOrder o(c, static_cast<cudaStream_t>(stream));
+  o.begin();
+  if (c->clip_norm > 0.0 || c->skip_nonfinite) {
+    st = run_two_pass(c, fn, user, resident, gfn, guser, o, stats);
+    o.end();  // joins the side stream also on the error paths
+    return st;
+  }
   c->last_coef = 1.0;
   c->last_skipped = 0;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = o.s;
   const int64_t t = c->t + 1;
   const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
   const std::vector<zsm::Span> iv = step_intervals(c);
-  std::vector<uint16_t*> grad(N), bufs(N);
+  std::vector<uint16_t*> grad(N);
   const int n_layers = (int)c->plan.layers.size();
-  for (size_t k = 0; k < iv.size(); ++k) {
+  const bool gathers = c->stage == ZERO_STAGE_3 && gfn;
+  bool launched = false;  // the first non-empty launch of the step starts the norm sum
+  size_t issued = 0;
+  for (size_t k = 0; k < iv.size() && st == ZERO_OK; ++k) {
+    for (; issued < iv.size() && issued <= k + o.ahead() && st == ZERO_OK; ++issued)
+      st = issue_grads(c, o, fn, user, resident, iv, issued, t);
+    if (st != ZERO_OK) break;
     const int64_t lo = iv[k].lo, hi = iv[k].hi;
     const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
-    if (resident) {
-      for (int r = 0; r < N; ++r)
-        grad[r] = const_cast<uint16_t*>(static_cast<const uint16_t*>(resident[r])) + lo;
-    } else {
-      for (int r = 0; r < N; ++r)
-        bufs[r] = c->stage == ZERO_STAGE_1 ? grad_buf_ptr(c, r) + lo : grad_buf_ptr(c, r);
-      if (fn) {
-        const int rc = fn(user, t, lo, hi, reinterpret_cast<void* const*>(bufs.data()), stream);
-        if (rc != 0) return fail(c, ZERO_EINVAL, "grad_fn returned %d for [%lld, %lld)", rc, (long long)lo, (long long)hi);
-      }
-      grad = bufs;
-    }
-    st = fused_interval(c, lo, hi, grad.data(), layer_idx, k > 0, sc, s);
-    if (st != ZERO_OK) return st;
-    if (c->stage == ZERO_STAGE_3 && gfn) {
-      for (int r = 0; r < N; ++r) bufs[r] = gather_ptr(c, r);
-      const int rc = gfn(guser, c->plan.layers[layer_idx].id, lo, hi, reinterpret_cast<void* const*>(bufs.data()), stream);
-      if (rc != 0) return fail(c, ZERO_EINVAL, "gather_fn returned %d for layer %d", rc, c->plan.layers[layer_idx].id);
-    }
+    interval_grads(c, resident, lo, o.slot(k), grad.data());
+    o.before_kernel(k, !resident && fn, gathers ? k : (size_t)-1);
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k));
+    if (st != ZERO_OK) break;
+    launched = launched || hi > lo;
+    o.after_kernel(k);
+    if (gathers) st = issue_gather(c, o, gfn, guser, layer_idx, k);
   }
+  if (o.end() != cudaSuccess && st == ZERO_OK) st = cuda_fail(c, o.err, "ordering the pipeline streams");
+  if (st != ZERO_OK) return st;
   c->t = t;
   c->stats_step = t;
   c->norm_fresh = true;
@@ -638,6 +782,9 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     case ZERO_OPT_BLOCKS_PER_SM:
       if (value < 0 || value > 32) return fail(c, ZERO_EINVAL, "blocks per SM must be 0..32");
       c->blocks_per_sm_opt = (int)value;
+      break;
+    case ZERO_OPT_PIPELINE:
+      c->pipeline = value != 0;
       break;
     default:
       return fail(c, ZERO_EINVAL, "unknown option %d", key);
@@ -797,9 +944,10 @@ zero_status zero_view(const zero_ctx* cc, int32_t what, int32_t rank, void** ptr
   if (!c || !ptr || !n_elems) return ZERO_EINVAL;
   if (!c->bound) return fail(c, ZERO_ESTATE, "arenas are not bound (zero_bind)");
   const int N = c->plan.n_ranks;
-  const bool per_rank = what == ZERO_VIEW_GRAD_BUF || what == ZERO_VIEW_GATHER ||
-                        (what == ZERO_VIEW_PARAM && c->stage != ZERO_STAGE_3);
-  if (per_rank && (rank < 0 || rank >= N)) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
+  const bool slotted = what == ZERO_VIEW_GRAD_BUF || what == ZERO_VIEW_GATHER;
+  const bool per_rank = slotted || (what == ZERO_VIEW_PARAM && c->stage != ZERO_STAGE_3);
+  const int n_views = slotted ? N * c->slots : N;  // rank + N selects the second slot set
+  if (per_rank && (rank < 0 || rank >= n_views)) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
   const int64_t P = c->plan.psi_pad;
   switch (what) {
     case ZERO_VIEW_MASTER: *ptr = master_ptr(c); *n_elems = P; break;
@@ -813,12 +961,12 @@ zero_status zero_view(const zero_ctx* cc, int32_t what, int32_t rank, void** ptr
       break;
     case ZERO_VIEW_GRAD_BUF:
       if (!c->arena[ZERO_ARENA_GRADS]) return fail(c, ZERO_EINVAL, "no gradient buffers (ZERO_OPT_GRAD_BUFFERS = 0)");
-      *ptr = grad_buf_ptr(c, rank);
+      *ptr = grad_buf_ptr(c, rank % N, rank / N);
       *n_elems = c->stage == ZERO_STAGE_1 ? P : c->stage == ZERO_STAGE_2 ? c->plan.max_bucket : c->plan.max_layer;
       break;
     case ZERO_VIEW_GATHER:
       if (c->stage != ZERO_STAGE_3) return fail(c, ZERO_EINVAL, "only stage 3 has gather buffers");
-      *ptr = gather_ptr(c, rank);
+      *ptr = gather_ptr(c, rank % N, rank / N);
       *n_elems = c->plan.max_layer;
       break;
     default:
