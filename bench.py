@@ -58,6 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
                     help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch the step's fused kernels plainly (no programmatic dependent launch)")
     ap.add_argument("--sweep", action="store_true",
                     help="flat-buffer sweep instead of the bench line: 1K..1G elements (x4) x N in "
                          "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
@@ -286,12 +288,18 @@ def run_ours(args, world, rank, local):
         for off, n in zip(offsets, w.numel):
             synth.dev_bf16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
     rep_list = list(reps)
+    opt.set_pdl(not args.no_pdl)
     torch.cuda.synchronize(dev)
+    # model bytes of one step's fused launches, from the library's own record
+    opt.set_timing(True)
+    opt.kernel_timing()
+    opt.step_resident(rep_list)
+    torch.cuda.synchronize(dev)
+    model_bytes_per_step = opt.kernel_timing()["model_bytes"]
+    opt.set_timing(False)
     for _ in range(args.warmup):
         opt.step_resident(rep_list)
     torch.cuda.synchronize(dev)
-    opt.set_timing(True)
-    opt.kernel_timing()  # empty the record
     sampler = ClockSampler(local)
     sampler.start()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -305,15 +313,28 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     barrier(dist)
     clocks = sampler.stop()
-    kt = opt.kernel_timing()
-    opt.set_timing(False)
     ms_local = e0.elapsed_time(e1)
     ms = max_over_ranks(ms_local, dist, dev)
     stats = opt.read_stats()
     value = world * w.psi * args.steps / (ms / 1e3)
-    launches = kt["launches"]
-    kernel_ms = kt["ms"] / max(1, launches)
-    achieved = kt["model_bytes"] / max(1, launches) / (kernel_ms / 1e3) / 1e9 if launches else None
+    # Only the fused kernels run in the timed region, back to back on this
+    # stream (with programmatic dependent launch each starts as the one before
+    # finishes), so their average launch duration is the region's time over
+    # its launches.
+    launches = args.steps * len(opt.buckets())
+    kernel_ms = ms_local / launches
+    achieved = model_bytes_per_step * args.steps / (ms_local / 1e3) / 1e9
+    # the same kernel timed launch by launch (CUDA events around each launch,
+    # which also turns programmatic dependent launch off)
+    iso_steps = 20
+    opt.set_timing(True)
+    opt.kernel_timing()
+    for _ in range(iso_steps):
+        opt.step_resident(rep_list)
+    torch.cuda.synchronize(dev)
+    kt = opt.kernel_timing()
+    opt.set_timing(False)
+    kernel_ms_isolated = kt["ms"] / max(1, kt["launches"])
     peak, peak_kind = measured_peaks()
     elems_per_launch = w.psi / max(1, len(opt.buckets()))
     fc = opt.fused_config()
@@ -378,14 +399,20 @@ def run_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
-                   "kernel": args.kernel, "fused_config": fc},
+                   "kernel": args.kernel, "fused_config": fc, "pdl": not args.no_pdl},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
                      "kernel": "fused_step_tma_kernel" if fc["kernel"] == "tma" else "fused_step_kernel",
                      "kernel_config": ckey,
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
-                     "model_bytes_per_launch": kt["model_bytes"] / max(1, launches),
+                     "model_bytes_per_launch": model_bytes_per_step / len(opt.buckets()),
+                     "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
+                                     "region (fused launches only, back to back"
+                                     + ("" if args.no_pdl else ", programmatic dependent launch") + ")",
+                     "kernel_ms_per_launch_isolated": kernel_ms_isolated,
+                     "achieved_isolated": kt["model_bytes"] / max(1, kt["launches"])
+                                          / (kernel_ms_isolated / 1e3) / 1e9,
                      "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None},
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -521,11 +548,10 @@ def run_stages(args):
                     for off, n in zip(opt.offsets(), w.numel):
                         synth.dev_bf16(W.grad_base(w, 1, r), off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
             rl = list(reps)
+            opt.set_pdl(not args.no_pdl)
             for _ in range(3):
                 opt.step_resident(rl)
             steps = max(5, int(2e9 / ((4 * w.n_ranks + 24) * w.psi)) + 5)
-            opt.set_timing(True)
-            opt.kernel_timing()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
@@ -534,14 +560,22 @@ def run_stages(args):
                 opt.step_resident(rl)
             e1.record()
             torch.cuda.synchronize()
-            kt = opt.kernel_timing()
             ms = e0.elapsed_time(e1) / steps
+            # the kernels launch by launch (events around each: no programmatic launch)
+            opt.set_timing(True)
+            opt.kernel_timing()
+            for _ in range(steps):
+                opt.step_resident(rl)
+            torch.cuda.synchronize()
+            kt = opt.kernel_timing()
+            opt.set_timing(False)
             per = {1: 6 * w.n_ranks + 24, 2: 4 * w.n_ranks + 24, 3: 4 * w.n_ranks + 26}[stage]
             print(json.dumps({"stages": w.name, "stage": stage, "n_ranks": w.n_ranks, "params": w.psi,
                               "ms_per_step": ms, "params_per_s": w.psi / (ms / 1e3),
                               "bytes_per_elem_model": per,
                               "step_gbs_model": per * w.psi / (ms / 1e3) / 1e9,
-                              "kernel_gbs_model": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
+                              "kernel_gbs_model_isolated": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
+                              "pdl": not args.no_pdl,
                               "launches_per_step": kt["launches"] // steps,
                               "fused_config": opt.fused_config(), "steps": steps}), flush=True)
             opt.close()

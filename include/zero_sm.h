@@ -153,7 +153,7 @@ enum {
   ZERO_OPT_DTYPE = 10,           /* storage format of every 16-bit buffer (gradients,
                                     parameters, reduced shards): ZERO_DTYPE_BF16 (default) or
                                     ZERO_DTYPE_F16 (IEEE binary16); before zero_bind */
-  ZERO_OPT_PIPELINE = 11         /* 1: zero_step / zero_step_resident run grad_fn and
+  ZERO_OPT_PIPELINE = 11,        /* 1: zero_step / zero_step_resident run grad_fn and
                                     gather_fn on a stream of the context's own, one interval
                                     ahead of the kernels on the caller's stream, so that the
                                     caller's backward of the next interval and its use of the
@@ -165,6 +165,13 @@ enum {
                                     stage 3 two gather slot sets (GATHER doubles), used
                                     alternately; stage 1 needs none.  Values are unchanged.
                                     Default 0; before zero_bind */
+  ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
+                                    with no gather_fn) launches its fused kernels with
+                                    programmatic dependent launch, so that each launch's CTAs
+                                    start on the SMs the previous launch leaves and, at stage
+                                    1/2, stream their own interval while it finishes; 0 launches
+                                    them plainly.  Values are unchanged.  Off while
+                                    ZERO_OPT_TIMING is on.  May be set at any time */
 };
 
 /* 16-bit storage formats (ZERO_OPT_DTYPE).  The pages account gradients and

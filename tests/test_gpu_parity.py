@@ -288,6 +288,50 @@ def test_adam_shard_per_rank_equals_all_ranks():
     b.close()
 
 
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_pdl_resident_steps_equal_plain_launches(stage):
+    """Resident steps launch their fused kernels with programmatic dependent
+    launch by default (at stage 1/2 each later launch streams its interval
+    while the one before finishes).  Against the same steps launched plainly:
+    the same bits, for every kernel variant, N = 4, 8, 16 and 17, eight or
+    more intervals per step, 3 steps, and against the oracle."""
+    z = _z()
+    numel, layer = W.transformer_layers(4, 96, 384)
+    for n_ranks in (4, 8, 16, 17):
+        w = W.Workload("pdl", numel, layer, n_ranks, (stage,), 40_000, synth.Dist(synth.NORMAL, 1e-2, zero_mod=13),
+                       W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01), 0x400 + n_ranks)
+        p, ranks, reps = _oracle_run(w, STAGE_OF[stage], 40_000)
+        ref = oracle.full_view(p, STAGE_OF[stage], ranks)
+        host = {t: [W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), w.grad_dist)
+                    for r in range(n_ranks)] for t in range(1, 4)}
+        for variant in kernels_for(n_ranks):
+            a, _ = make_opt(w, stage, bucket=40_000, variant=variant)
+            b, _ = make_opt(w, stage, bucket=40_000, variant=variant)
+            b.set_pdl(False)
+            assert len(a.buckets() if stage != 3 else a.layers()) >= 4
+            for t in range(1, 4):
+                dev = [torch.from_numpy(h.view(np.int16)).cuda() for h in host[t]]
+                devb = [x.clone() for x in dev]
+                sa = a.step_resident(dev, stats=True)
+                sb = b.step_resident(devb, stats=True)
+                assert sa == sb
+                assert math.isclose(sa["grad_norm"], reps[t - 1].grad_norm, rel_tol=norm_tol(p.psi_pad))
+                if stage == 1:
+                    for r in range(n_ranks):
+                        assert torch.equal(dev[r], devb[r])
+            for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+                assert torch.equal(a.view(what), b.view(what))
+            for name, what in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+                assert_bits_equal(to_np(a.view(what)), ref[name], f"pdl {variant} N={n_ranks} {name}")
+            for r in range(n_ranks if stage != 3 else 1):
+                assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+                assert_bits_equal(to_np(a.view(z.ZERO_VIEW_PARAM, r)), ref["params"], f"pdl {variant} params {r}")
+            if stage == 3:
+                assert torch.equal(a.view(z.ZERO_VIEW_GATHER, 0), b.view(z.ZERO_VIEW_GATHER, 0))
+            a.close()
+            b.close()
+
+
 # ------------------------------------------------------------- edge cases ----
 
 def test_nonfinite_gradients_are_counted_and_propagate_like_the_oracle():

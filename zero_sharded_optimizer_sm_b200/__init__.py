@@ -45,6 +45,7 @@ ZERO_OPT_TMA_STAGES = 8
 ZERO_OPT_TMA_CTAS_PER_SM = 9
 ZERO_OPT_DTYPE = 10
 ZERO_OPT_PIPELINE = 11
+ZERO_OPT_PDL = 12
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -417,6 +418,10 @@ class ZeroOptimizer:
 
     def set_kernel(self, kernel: int):
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
+
+    def set_pdl(self, on: bool):
+        """Programmatic dependent launch between a callback-free step's fused launches (default on)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_PDL, 1 if on else 0), "zero_set_option")
 
     def set_timing(self, on: bool):
         self._check(zero_set_option(self.ctx, ZERO_OPT_TIMING, 1 if on else 0), "zero_set_option")

@@ -87,6 +87,17 @@ __device__ __forceinline__ void add8(float (&acc)[kVec], uint4 w) {
   acc[7] = __fadd_rn(acc[7], F::hi(w.w));
 }
 
+// ------------------------------------------ programmatic dependent launch --
+
+// Waits until the grids this one depends on have completed and their memory
+// operations are visible; returns at once for a launch without the
+// programmatic attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the dependent grid launch once every CTA of this grid has issued this
+// or exited (later calls in the same CTA have no further effect).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------- rank-order reduce --
 
 // acc[j] = sum over r = 0..n-1 of grad[r][e + j], in rank order.  Ranks are

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
   unsigned long long nf = 0;
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
         last_k[s] = (int)k;
       }
+      pdl_trigger();  // no more loads to issue: the next fused launch may start
     }
   } else {
     // --------------------------------------------------------- consumers --
@@ -244,6 +246,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
     for (int s = 0; s < stages; ++s)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
+  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<tma_threads<G>()>(a.ns, sq, nf, a.accumulate);
 }
 
@@ -290,6 +293,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
   unsigned long long nf = 0;
@@ -319,6 +323,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
         last_k[s] = (int)k;
       }
+      pdl_trigger();  // no more loads to issue: the next fused launch may start
     }
   } else {
     const int c = threadIdx.x - 32;  // 0..511
@@ -384,6 +389,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     for (int s = 0; s < stages; ++s)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
+  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<kWideThreads>(a.ns, sq, nf, a.accumulate);
 }
 
@@ -442,6 +448,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
   unsigned long long nf = 0;
@@ -491,6 +498,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         }
         if (stop) break;
       }
+      pdl_trigger();  // no more loads to issue: the next fused launch may start
     }
   } else {
     // --------------------------------------------------------- consumers --
@@ -579,17 +587,19 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
     for (int s = 0; s < sstages; ++s)
       if (last_sk[s] >= 0 && !mbar_wait(&sfull[s], (unsigned)last_sk[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
+  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<tma_threads<1>()>(a.ns, sq, nf, a.accumulate);
 }
 
 template <int MODE>
 cudaError_t launch_chunked_mode(const FusedArgs& a, int grid, int cstages, int sstages, cudaStream_t s) {
   const size_t bytes = chunked_smem_bytes(cstages, sstages);
+  const bool pdl = a.pdl != kPdlNone;
   if (a.fmt == kFmtF16)
-    fused_step_chunked_kernel<MODE, F16><<<grid, tma_threads<1>(), bytes, s>>>(a, cstages, sstages);
-  else
-    fused_step_chunked_kernel<MODE, Bf16><<<grid, tma_threads<1>(), bytes, s>>>(a, cstages, sstages);
-  return cudaGetLastError();
+    return launch_kernel(fused_step_chunked_kernel<MODE, F16>, grid, tma_threads<1>(), bytes, s, pdl, a, cstages,
+                         sstages);
+  return launch_kernel(fused_step_chunked_kernel<MODE, Bf16>, grid, tma_threads<1>(), bytes, s, pdl, a, cstages,
+                       sstages);
 }
 
 size_t tma_smem_bytes(int n_ranks, int stages) {
@@ -597,21 +607,20 @@ size_t tma_smem_bytes(int n_ranks, int stages) {
 }
 
 template <int MODE, class F>
-void launch_tma_fmt(const FusedArgs& a, int grid, int stages, int groups, size_t bytes, cudaStream_t s) {
+cudaError_t launch_tma_fmt(const FusedArgs& a, int grid, int stages, int groups, size_t bytes, cudaStream_t s) {
+  const bool pdl = a.pdl != kPdlNone;
   if (groups == kWideGroup)
-    fused_step_tma_wide_kernel<MODE, F><<<grid, kWideThreads, bytes, s>>>(a, stages);
-  else if (groups == 2)
-    fused_step_tma_kernel<MODE, 2, F><<<grid, tma_threads<2>(), bytes, s>>>(a, stages);
-  else
-    fused_step_tma_kernel<MODE, 1, F><<<grid, tma_threads<1>(), bytes, s>>>(a, stages);
+    return launch_kernel(fused_step_tma_wide_kernel<MODE, F>, grid, kWideThreads, bytes, s, pdl, a, stages);
+  if (groups == 2)
+    return launch_kernel(fused_step_tma_kernel<MODE, 2, F>, grid, tma_threads<2>(), bytes, s, pdl, a, stages);
+  return launch_kernel(fused_step_tma_kernel<MODE, 1, F>, grid, tma_threads<1>(), bytes, s, pdl, a, stages);
 }
 
 template <int MODE>
 cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, int groups, cudaStream_t s) {
   const size_t bytes = tma_smem_bytes(a.n_ranks, stages);
-  if (a.fmt == kFmtF16) launch_tma_fmt<MODE, F16>(a, grid, stages, groups, bytes, s);
-  else launch_tma_fmt<MODE, Bf16>(a, grid, stages, groups, bytes, s);
-  return cudaGetLastError();
+  if (a.fmt == kFmtF16) return launch_tma_fmt<MODE, F16>(a, grid, stages, groups, bytes, s);
+  return launch_tma_fmt<MODE, Bf16>(a, grid, stages, groups, bytes, s);
 }
 
 }  // namespace

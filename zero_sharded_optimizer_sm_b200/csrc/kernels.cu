@@ -30,6 +30,10 @@ template <int MODE, bool kMulti, class F>
 __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   double sq = 0.0;
   unsigned long long nf = 0;
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
+  // every CTA is resident from the start (the grid is sized to the SM count),
+  // so the next fused launch may be scheduled as soon as CTAs exit
+  pdl_trigger();
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
     const int64_t e = vi * kVec;
@@ -58,6 +62,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     if (MODE == kFusedZ3) st_stream(a.param_shard + e, pw);
     for (int r = 0; r < a.n_ranks; ++r) st_stream(a.out[r] + e, pw);
   }
+  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<kThreads>(a.ns, sq, nf, a.accumulate);
 }
 
@@ -173,22 +178,20 @@ __global__ void __launch_bounds__(kThreads) init_kernel(const __grid_constant__ 
 // --------------------------------------------------------------- launchers --
 
 template <int MODE, class F>
-void launch_fused_mode(const FusedArgs& a, int grid, cudaStream_t s) {
-  if (a.n_ranks <= 8)
-    fused_step_kernel<MODE, false, F><<<grid, kThreads, 0, s>>>(a);
-  else
-    fused_step_kernel<MODE, true, F><<<grid, kThreads, 0, s>>>(a);
+cudaError_t launch_fused_mode(const FusedArgs& a, int grid, cudaStream_t s) {
+  const bool pdl = a.pdl != kPdlNone;
+  if (a.n_ranks <= 8) return launch_kernel(fused_step_kernel<MODE, false, F>, grid, kThreads, 0, s, pdl, a);
+  return launch_kernel(fused_step_kernel<MODE, true, F>, grid, kThreads, 0, s, pdl, a);
 }
 
 template <class F>
 cudaError_t launch_fused_fmt(int mode, const FusedArgs& a, int grid, cudaStream_t s) {
   switch (mode) {
-    case kFusedZ1: launch_fused_mode<kFusedZ1, F>(a, grid, s); break;
-    case kFusedZ2: launch_fused_mode<kFusedZ2, F>(a, grid, s); break;
-    case kFusedZ3: launch_fused_mode<kFusedZ3, F>(a, grid, s); break;
+    case kFusedZ1: return launch_fused_mode<kFusedZ1, F>(a, grid, s);
+    case kFusedZ2: return launch_fused_mode<kFusedZ2, F>(a, grid, s);
+    case kFusedZ3: return launch_fused_mode<kFusedZ3, F>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s) {

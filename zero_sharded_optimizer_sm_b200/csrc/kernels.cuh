@@ -33,6 +33,37 @@ struct AdamScalars {
 
 enum StorageFormat { kFmtBf16 = 0, kFmtF16 = 1 };
 
+// Programmatic dependent launch of a fused-step kernel.  With kPdlWaitFirst
+// or kPdlEarly the launch carries the programmatic-serialization attribute,
+// so it may start while the grid before it in the stream is still running;
+// each CTA of a fused kernel releases its dependents (griddepcontrol
+// .launch_dependents) once it has no more input loads to issue.
+//   kPdlWaitFirst  the kernel waits for the grid before it (griddepcontrol
+//                  .wait) before touching global memory: safe after anything;
+//   kPdlEarly      the kernel streams its interval at once and waits only
+//                  before the norm epilogue.  Only for a launch whose
+//                  predecessor is a fused kernel of the same step on a
+//                  disjoint interval with disjoint destinations, so that the
+//                  two share nothing but the norm scratch.
+enum PdlMode { kPdlNone = 0, kPdlWaitFirst = 1, kPdlEarly = 2 };
+
+// cudaLaunchKernelEx with the programmatic-serialization attribute when `pdl`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, bool pdl,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // Gradient-norm / non-finite accumulation in the scratch arena.
 struct NormScratch {
   double* partial_sq;              // [kMaxGrid] per-CTA partial sums of g^2
@@ -58,6 +89,7 @@ struct FusedArgs {
   int n_ranks;
   int accumulate;                   // 0: first launch of the step (norm overwrites)
   float inv_n;                      // binary32 1/N
+  int pdl;                          // PdlMode of this launch
   AdamScalars sc;
   NormScratch ns;
 };

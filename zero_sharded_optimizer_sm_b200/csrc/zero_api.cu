@@ -70,6 +70,7 @@ struct zero_ctx {
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
   // callback pipeline (ZERO_OPT_PIPELINE): side stream and ordering events
   bool pipeline = false;
+  bool pdl = true;  // programmatic dependent launch between the step's fused launches
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
   cudaStream_t side = nullptr;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr;
@@ -327,7 +328,8 @@ std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
 
 // One fused launch over [lo, hi).  grad[r] are at flat element lo.
 zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
-                           bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0) {
+                           bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0,
+                           int pdl = zsm::kPdlNone) {
   if (hi == lo) return ZERO_OK;
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
@@ -353,6 +355,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   a.inv_n = (float)(1.0 / (double)N);
   a.sc = sc;
   a.ns = norm_scratch(c);
+  a.pdl = c->timing ? zsm::kPdlNone : pdl;  // an event record between launches ends the overlap
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
@@ -444,7 +447,10 @@ struct StepOrder {
   bool joined = false;
   cudaError_t err = cudaSuccess;
 
-  StepOrder(zero_ctx* ctx, cudaStream_t stream) : c(ctx), s(stream), q(stream), on(ctx->pipeline) {
+  // `callbacks`: the step calls grad_fn or gather_fn (without any there is
+  // nothing to run ahead, and the step stays on `s` alone)
+  StepOrder(zero_ctx* ctx, cudaStream_t stream, bool callbacks)
+      : c(ctx), s(stream), q(stream), on(ctx->pipeline && callbacks) {
     if (on) q = c->side;
   }
   void record(cudaEvent_t e, cudaStream_t st) {
@@ -453,7 +459,7 @@ struct StepOrder {
   void wait(cudaStream_t st, cudaEvent_t e) {
     if (err == cudaSuccess) err = cudaStreamWaitEvent(st, e, 0);
   }
-  int slot(size_t k) const { return c->slots == 2 ? (int)(k & 1) : 0; }
+  int slot(size_t k) const { return (on && c->slots == 2) ? (int)(k & 1) : 0; }
   size_t ahead() const { return on ? 1 : 0; }
   void begin() {
     if (!on) return;
@@ -663,7 +669,8 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   }
   st = ensure_pipeline(c);
   if (st != ZERO_OK) return st;
-  StepOrder o(c, static_cast<cudaStream_t>(stream));
+  const bool callbacks = (!resident && fn) || (c->stage == ZERO_STAGE_3 && gfn);
+  StepOrder o(c, static_cast<cudaStream_t>(stream), callbacks);
   o.begin();
   if (c->clip_norm > 0.0 || c->skip_nonfinite) {
     st = run_two_pass(c, fn, user, resident, gfn, guser, o, stats);
@@ -681,6 +688,13 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   const bool gathers = c->stage == ZERO_STAGE_3 && gfn;
   bool launched = false;  // the first non-empty launch of the step starts the norm sum
   size_t issued = 0;
+  // Programmatic dependent launch only between this step's own back-to-back
+  // launches: with callbacks other work sits between them.  The first launch
+  // follows unknown work and waits for it before touching memory; the later
+  // ones at stage 1/2 touch disjoint intervals and share only the norm
+  // scratch, so they stream at once; stage 3's launches all write the one
+  // temporary gather buffer, so they wait first.
+  const bool pdl_ok = c->pdl && !callbacks;
   for (size_t k = 0; k < iv.size() && st == ZERO_OK; ++k) {
     for (; issued < iv.size() && issued <= k + o.ahead() && st == ZERO_OK; ++issued)
       st = issue_grads(c, o, fn, user, resident, iv, issued, t);
@@ -689,7 +703,10 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
     const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
     interval_grads(c, resident, lo, o.slot(k), grad.data());
     o.before_kernel(k, !resident && fn, gathers ? k : (size_t)-1);
-    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k));
+    const int pdl = !pdl_ok ? zsm::kPdlNone
+                    : (launched && c->stage != ZERO_STAGE_3) ? zsm::kPdlEarly
+                                                             : zsm::kPdlWaitFirst;
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl);
     if (st != ZERO_OK) break;
     launched = launched || hi > lo;
     o.after_kernel(k);
@@ -743,6 +760,10 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   if (key == ZERO_OPT_KERNEL) {
     if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_TMA) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
     c->kernel_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_PDL) {
+    c->pdl = value != 0;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_TMA_CTAS_PER_SM) {
