@@ -58,8 +58,9 @@ def parse_args(argv=None):
     ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
                     help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
-    ap.add_argument("--no-pdl", action="store_true",
-                    help="launch the step's fused kernels plainly (no programmatic dependent launch)")
+    ap.add_argument("--pdl", action="store_true",
+                    help="launch the step's fused kernels with programmatic dependent launch "
+                         "(ZERO_OPT_PDL; off by default, measured slower)")
     ap.add_argument("--sweep", action="store_true",
                     help="flat-buffer sweep instead of the bench line: 1K..1G elements (x4) x N in "
                          "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
@@ -274,7 +275,7 @@ def run_ours(args, world, rank, local):
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, z.ZERO_STAGE_2, bucket_elems=w.bucket_elems,
                           hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
                           replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
-                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], device=dev)
+                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True, device=dev)
     offsets = opt.offsets()
     mv = opt.view(z.ZERO_VIEW_MASTER)
     b = W.master_base(w)
@@ -288,7 +289,7 @@ def run_ours(args, world, rank, local):
         for off, n in zip(offsets, w.numel):
             synth.dev_bf16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
     rep_list = list(reps)
-    opt.set_pdl(not args.no_pdl)
+    opt.set_pdl(args.pdl)
     torch.cuda.synchronize(dev)
     # model bytes of one step's fused launches, from the library's own record
     opt.set_timing(True)
@@ -353,10 +354,11 @@ def run_ours(args, world, rank, local):
 
         def grad_fn(t, lo, hi, bufs, stream_):
             nonlocal h2d
-            for r, ptr in enumerate(bufs):
-                dst = opt._tensor_at(ptr, hi - lo, torch.int16)
-                dst.copy_(host[r, : hi - lo], non_blocking=True)
-                h2d += 2 * (hi - lo)
+            with torch.cuda.stream(torch.cuda.ExternalStream(stream_) if stream_ else stream):
+                for r, ptr in enumerate(bufs):
+                    dst = opt._tensor_at(ptr, hi - lo, torch.int16)
+                    dst.copy_(host[r, : hi - lo], non_blocking=True)
+                    h2d += 2 * (hi - lo)
             return 0
 
         del reps, rep_list
@@ -374,8 +376,9 @@ def run_ours(args, world, rank, local):
         e2e = {"value": world * w.psi * args.e2e_steps / e2e_s, "unit": "params/s",
                "h2d_bytes_per_step": h2d // args.e2e_steps, "d2h_bytes_per_step": 16,
                "steps": args.e2e_steps,
-               "how": "zero_step through the C ABI; grad_fn copies each bucket's N gradient slices "
-                      "from pinned host memory into the 200M-element buffer; stats (grad norm, "
+               "how": "zero_step through the C ABI with ZERO_OPT_PIPELINE; grad_fn copies each "
+                      "bucket's N gradient slices from pinned host memory into one of the two "
+                      "200M-element buffers, one bucket ahead of the fused kernel; stats (grad norm, "
                       "non-finite count) read back every step"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -399,7 +402,7 @@ def run_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
-                   "kernel": args.kernel, "fused_config": fc, "pdl": not args.no_pdl},
+                   "kernel": args.kernel, "fused_config": fc, "pdl": args.pdl},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
@@ -409,7 +412,7 @@ def run_ours(args, world, rank, local):
                      "model_bytes_per_launch": model_bytes_per_step / len(opt.buckets()),
                      "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
                                      "region (fused launches only, back to back"
-                                     + ("" if args.no_pdl else ", programmatic dependent launch") + ")",
+                                     + (", programmatic dependent launch" if args.pdl else "") + ")",
                      "kernel_ms_per_launch_isolated": kernel_ms_isolated,
                      "achieved_isolated": kt["model_bytes"] / max(1, kt["launches"])
                                           / (kernel_ms_isolated / 1e3) / 1e9,
@@ -548,7 +551,7 @@ def run_stages(args):
                     for off, n in zip(opt.offsets(), w.numel):
                         synth.dev_bf16(W.grad_base(w, 1, r), off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
             rl = list(reps)
-            opt.set_pdl(not args.no_pdl)
+            opt.set_pdl(args.pdl)
             for _ in range(3):
                 opt.step_resident(rl)
             steps = max(5, int(2e9 / ((4 * w.n_ranks + 24) * w.psi)) + 5)
@@ -575,7 +578,7 @@ def run_stages(args):
                               "bytes_per_elem_model": per,
                               "step_gbs_model": per * w.psi / (ms / 1e3) / 1e9,
                               "kernel_gbs_model_isolated": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
-                              "pdl": not args.no_pdl,
+                              "pdl": args.pdl,
                               "launches_per_step": kt["launches"] // steps,
                               "fused_config": opt.fused_config(), "steps": steps}), flush=True)
             opt.close()

@@ -165,12 +165,14 @@ enum {
                                     stage 3 two gather slot sets (GATHER doubles), used
                                     alternately; stage 1 needs none.  Values are unchanged.
                                     Default 0; before zero_bind */
-  ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
-                                    with no gather_fn) launches its fused kernels with
-                                    programmatic dependent launch, so that each launch's CTAs
-                                    start on the SMs the previous launch leaves and, at stage
-                                    1/2, stream their own interval while it finishes; 0 launches
-                                    them plainly.  Values are unchanged.  Off while
+  ZERO_OPT_PDL = 12              /* 1: a step without callbacks (zero_step_resident with no
+                                    gather_fn) launches its fused kernels with programmatic
+                                    dependent launch, so that each launch's CTAs start on the
+                                    SMs the previous launch leaves and, at stage 1/2, stream
+                                    their own interval while it finishes.  0 (default): plain
+                                    launches -- faster on B200 for the persistent staged
+                                    kernels, whose one-CTA-per-SM placement the early launch
+                                    breaks.  Values are unchanged either way.  Off while
                                     ZERO_OPT_TIMING is on.  May be set at any time */
 };
 

@@ -290,9 +290,10 @@ def test_adam_shard_per_rank_equals_all_ranks():
 
 @pytest.mark.parametrize("stage", [1, 2, 3])
 def test_pdl_resident_steps_equal_plain_launches(stage):
-    """Resident steps launch their fused kernels with programmatic dependent
-    launch by default (at stage 1/2 each later launch streams its interval
-    while the one before finishes).  Against the same steps launched plainly:
+    """Resident steps with ZERO_OPT_PDL launch their fused kernels with
+    programmatic dependent launch (at stage 1/2 each later launch streams its
+    interval while the one before finishes).  Against the same steps launched
+    plainly:
     the same bits, for every kernel variant, N = 4, 8, 16 and 17, eight or
     more intervals per step, 3 steps, and against the oracle."""
     z = _z()
@@ -307,6 +308,7 @@ def test_pdl_resident_steps_equal_plain_launches(stage):
         for variant in kernels_for(n_ranks):
             a, _ = make_opt(w, stage, bucket=40_000, variant=variant)
             b, _ = make_opt(w, stage, bucket=40_000, variant=variant)
+            a.set_pdl(True)
             b.set_pdl(False)
             assert len(a.buckets() if stage != 3 else a.layers()) >= 4
             for t in range(1, 4):

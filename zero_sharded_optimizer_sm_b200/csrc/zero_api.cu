@@ -70,7 +70,12 @@ struct zero_ctx {
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
   // callback pipeline (ZERO_OPT_PIPELINE): side stream and ordering events
   bool pipeline = false;
-  bool pdl = true;  // programmatic dependent launch between the step's fused launches
+  // Programmatic dependent launch between the step's fused launches.  Off by
+  // default: measured on B200 it made the persistent staged kernels ~17 %
+  // slower -- the next grid's CTAs are placed while the previous grid still
+  // holds SMs, so some SMs receive two of its CTAs and others none, and with
+  // tiles assigned to CTAs statically the doubled SMs set the kernel's time.
+  bool pdl = false;
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
   cudaStream_t side = nullptr;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr;
