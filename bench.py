@@ -707,7 +707,7 @@ def run_overlap(args):
              (W.gpt_85m_n8(), 2, 20_000_000)]
     for w, stage, bucket in cells:
         res = {}
-        for pipe in (False, True):
+        for pipe in (0, 1, 2):
             opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=bucket,
                                   hparams=z.AdamHParams(), keep_grad_shards=False, kernel=kern, pipeline=pipe)
             assert opt.psi_pad == w.psi and all(o + n == e for o, n, e in
@@ -733,7 +733,7 @@ def run_overlap(args):
                 opt.step(gfn)
             e1.record()
             torch.cuda.synchronize()
-            res["pipelined" if pipe else "in_order"] = e0.elapsed_time(e1) / steps
+            res[("in_order", "pipelined", "pipelined_priority")[pipe]] = e0.elapsed_time(e1) / steps
             if not pipe:
                 kt = opt.kernel_timing()
                 res["kernels_alone"] = kt["ms"] / steps
@@ -756,6 +756,8 @@ def run_overlap(args):
         print(json.dumps({"overlap": w.name, "stage": stage, "n_ranks": w.n_ranks, "params": w.psi,
                           "intervals": res["intervals"], "bucket_elems": bucket,
                           "ms_in_order": res["in_order"], "ms_pipelined": res["pipelined"],
+                          "ms_pipelined_priority": res["pipelined_priority"],
+                          "speedup_priority": res["in_order"] / res["pipelined_priority"],
                           "ms_kernels_alone": res["kernels_alone"], "ms_grad_fn_alone": res["grad_fn_alone"],
                           "ms_perfect_overlap": lower, "speedup": res["in_order"] / res["pipelined"],
                           "fraction_of_shorter_phase_hidden": hidden, "steps": steps}), flush=True)

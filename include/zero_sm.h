@@ -163,7 +163,11 @@ enum {
                                     on its communication volume; [Q] section 五).  Stages 2 and
                                     3 then hold two gradient slot sets (GRADS doubles) and
                                     stage 3 two gather slot sets (GATHER doubles), used
-                                    alternately; stage 1 needs none.  Values are unchanged.
+                                    alternately; stage 1 needs none.  2: as 1, and the step's
+                                    kernels run on a stream of the context's own at the
+                                    device's greatest priority (joined into the caller's stream
+                                    at the end), so that their CTAs take the SMs that the
+                                    callbacks' work frees first.  Values are unchanged.
                                     Default 0; before zero_bind */
   ZERO_OPT_PDL = 12              /* 1: a step without callbacks (zero_step_resident with no
                                     gather_fn) launches its fused kernels with programmatic

@@ -102,8 +102,9 @@ def _check_state(opt, p, stage, ranks, what):
 LAYOUTS = [([33, 1, 2, 17], [0, 1, 1, 2]), ([16, 0, 24, 0], [0, 1, 2, 3]), ([3000, 1, 4100], [0, 1, 2])]
 
 
+@pytest.mark.parametrize("mode", [1, 2])
 @pytest.mark.parametrize("layout", LAYOUTS)
-def test_pipeline_every_element_against_the_oracle(layout):
+def test_pipeline_every_element_against_the_oracle(layout, mode):
     """N = 1, 2, 5, 8; stages 1-3; buckets 8 and all; 3 steps; the callbacks
     see the side stream and alternating slot sets, every gathered layer and
     every statistic match the oracle (the empty layers of the second layout
@@ -118,7 +119,7 @@ def test_pipeline_every_element_against_the_oracle(layout):
                                synth.Dist(synth.NORMAL, 1e-2, zero_mod=7), W.MASTER_DIST, 3,
                                W.Hyper(lr=1e-2, weight_decay=0.1), 0x300 + n_ranks)
                 p, ranks, reps = _oracle(w, stage, bucket)
-                opt, fill = make_opt(w, stage, bucket, True)
+                opt, fill = make_opt(w, stage, bucket, mode)
                 caller = torch.cuda.current_stream().cuda_stream
                 for t in range(1, w.steps + 1):
                     seen, gathered = [], []
@@ -145,9 +146,10 @@ def test_pipeline_every_element_against_the_oracle(layout):
                 opt.close()
 
 
+@pytest.mark.parametrize("mode", [1, 2])
 @pytest.mark.parametrize("stage", [1, 2, 3])
 @pytest.mark.parametrize("two_pass", [False, True])
-def test_pipeline_equals_in_order_step(stage, two_pass):
+def test_pipeline_equals_in_order_step(stage, two_pass, mode):
     """2 layers, hidden 768 (14.2M params), N = 8, 3M-element buckets, 4
     steps: with and without the pipeline the same bits everywhere, also in
     the two-pass step (clip at a norm the gradients exceed, overflow skip on)."""
@@ -155,8 +157,8 @@ def test_pipeline_equals_in_order_step(stage, two_pass):
     numel, layer = W.transformer_layers(2, 768, 3072)
     w = W.Workload("pipe-h768", numel, layer, 8, (stage,), 3_000_000, synth.Dist(synth.NORMAL, 1e-2, zero_mod=100),
                    W.MASTER_DIST, 4, W.Hyper(weight_decay=0.01), W.SEED0 + 30)
-    a, fa = make_opt(w, stage, 3_000_000, False)
-    b, fb = make_opt(w, stage, 3_000_000, True)
+    a, fa = make_opt(w, stage, 3_000_000, 0)
+    b, fb = make_opt(w, stage, 3_000_000, mode)
     if two_pass:
         a.set_clip(0.5, True)
         b.set_clip(0.5, True)
@@ -180,13 +182,14 @@ def test_pipeline_equals_in_order_step(stage, two_pass):
     b.close()
 
 
-def test_pipeline_resident_stage3_gathers():
+@pytest.mark.parametrize("mode", [1, 2])
+def test_pipeline_resident_stage3_gathers(mode):
     z = _z()
     numel, layer = W.transformer_layers(4, 128, 512)
     w = W.Workload("pipe-res", numel, layer, 4, (3,), None, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 2,
                    W.Hyper(), 0x340)
-    a, fa = make_opt(w, 3, None, False)
-    b, fb = make_opt(w, 3, None, True)
+    a, fa = make_opt(w, 3, None, 0)
+    b, fb = make_opt(w, 3, None, mode)
     s = torch.cuda.current_stream().cuda_stream
     ga, gb = [], []
     for t in (1, 2):
@@ -210,8 +213,8 @@ def test_pipeline_callback_failure_leaves_the_context_usable():
     numel, layer = W.transformer_layers(3, 64, 256)
     w = W.Workload("pipe-fail", numel, layer, 4, (3,), None, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 1,
                    W.Hyper(), 0x350)
-    ref, fr = make_opt(w, 3, None, False)
-    opt, fill = make_opt(w, 3, None, True)
+    ref, fr = make_opt(w, 3, None, 0)
+    opt, fill = make_opt(w, 3, None, 2)
     good = grad_fn_for(opt, fill)
     calls = [0]
 

@@ -162,7 +162,7 @@ class ZeroOptimizer:
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
                  tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16,
-                 pipeline: bool = False, device=None):
+                 pipeline: int = 0, device=None):
         import torch
 
         self._torch = torch
@@ -201,8 +201,8 @@ class ZeroOptimizer:
         if tma_ctas_per_sm:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_CTAS_PER_SM, int(tma_ctas_per_sm)), "zero_set_option")
         if pipeline:
-            self._check(zero_set_option(ctx, ZERO_OPT_PIPELINE, 1), "zero_set_option")
-        self.pipeline = bool(pipeline)
+            self._check(zero_set_option(ctx, ZERO_OPT_PIPELINE, int(pipeline)), "zero_set_option")
+        self.pipeline = int(pipeline)
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)

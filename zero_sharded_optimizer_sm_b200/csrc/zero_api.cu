@@ -69,7 +69,7 @@ struct zero_ctx {
   int64_t last_skipped = 0;
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
   // callback pipeline (ZERO_OPT_PIPELINE): side stream and ordering events
-  bool pipeline = false;
+  int pipeline = 0;  // ZERO_OPT_PIPELINE: 0, 1 or 2
   // Programmatic dependent launch between the step's fused launches.  Off by
   // default: measured on B200 it made the persistent staged kernels ~17 %
   // slower -- the next grid's CTAs are placed while the previous grid still
@@ -77,8 +77,9 @@ struct zero_ctx {
   // tiles assigned to CTAs statically the doubled SMs set the kernel's time.
   bool pdl = false;
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev_start = nullptr, ev_join = nullptr;
+  cudaStream_t side = nullptr;   // the callbacks' stream
+  cudaStream_t kside = nullptr;  // the kernels' stream at the greatest priority (ZERO_OPT_PIPELINE = 2)
+  cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_kjoin = nullptr;
   cudaEvent_t ev_grads[2] = {}, ev_kernel[2] = {}, ev_consumed[2] = {};
   // fused-kernel timing
   bool timing = false;
@@ -88,10 +89,11 @@ struct zero_ctx {
   std::string err;
   ~zero_ctx() {
     for (cudaEvent_t e : events) cudaEventDestroy(e);
-    for (cudaEvent_t e : {ev_start, ev_join, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
+    for (cudaEvent_t e : {ev_start, ev_join, ev_kjoin, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
                           ev_consumed[0], ev_consumed[1]})
       if (e) cudaEventDestroy(e);
     if (side) cudaStreamDestroy(side);
+    if (kside) cudaStreamDestroy(kside);
   }
 };
 
@@ -433,21 +435,25 @@ zero_status read_norm(zero_ctx* c, cudaStream_t s, double* sq, unsigned long lon
   return ZERO_OK;
 }
 
-// Orders one step's work across the caller's stream `s` (every kernel) and
-// the stream the callbacks get.  Without ZERO_OPT_PIPELINE that is `s`
-// itself and everything runs in program order with one slot set.  With it,
-// the callbacks run on the context's side stream one interval ahead --
-// grad_fn(k+1) and gather_fn(k) overlap the kernel of interval k+1 or k --
-// and events keep each slot set from being refilled before its reader is done:
-//   grad_fn(k)   (side)   after the kernel of k-2 read slot k%2 (stage 2/3)
-//   kernel(k)    (s)      after grad_fn(k), and (stage 3) after gather_fn(k-2)
-//                         finished reading gather slot k%2
-//   gather_fn(k) (side)   after kernel(k)
-// and `s` waits for all of the side stream's work before the step returns.
+// Orders one step's work across the caller's stream `s`, the stream the
+// callbacks get (`q`) and the stream of the step's kernels (`ks`).  Without
+// ZERO_OPT_PIPELINE all three are `s` and everything runs in program order
+// with one slot set.  With it, the callbacks run on the context's side stream
+// one interval ahead -- grad_fn(k+1) and gather_fn(k) overlap the kernel of
+// interval k+1 or k -- and the kernels on `s` (option value 1) or on a
+// stream of the context's own at the device's greatest priority (value 2,
+// so that their CTAs take the SMs the callbacks' work frees first).  Events
+// keep each slot set from being refilled before its reader is done:
+//   grad_fn(k)   (q)    after the kernel of k-2 read slot k%2 (stage 2/3)
+//   kernel(k)    (ks)   after grad_fn(k), and (stage 3) after gather_fn(k-2)
+//                       finished reading gather slot k%2
+//   gather_fn(k) (q)    after kernel(k)
+// and `s` waits for all of q's and ks's work before the step returns.
 struct StepOrder {
   zero_ctx* c;
   cudaStream_t s;
   cudaStream_t q;
+  cudaStream_t ks;
   bool on;
   bool joined = false;
   cudaError_t err = cudaSuccess;
@@ -455,8 +461,9 @@ struct StepOrder {
   // `callbacks`: the step calls grad_fn or gather_fn (without any there is
   // nothing to run ahead, and the step stays on `s` alone)
   StepOrder(zero_ctx* ctx, cudaStream_t stream, bool callbacks)
-      : c(ctx), s(stream), q(stream), on(ctx->pipeline && callbacks) {
+      : c(ctx), s(stream), q(stream), ks(stream), on(ctx->pipeline != 0 && callbacks) {
     if (on) q = c->side;
+    if (on && c->kside) ks = c->kside;
   }
   void record(cudaEvent_t e, cudaStream_t st) {
     if (err == cudaSuccess) err = cudaEventRecord(e, st);
@@ -470,6 +477,7 @@ struct StepOrder {
     if (!on) return;
     record(c->ev_start, s);
     wait(q, c->ev_start);
+    if (ks != s) wait(ks, c->ev_start);
   }
   void before_grads(size_t k) {
     if (on && c->slots == 2 && k >= 2) wait(q, c->ev_kernel[k & 1]);
@@ -479,11 +487,11 @@ struct StepOrder {
   }
   void before_kernel(size_t k, bool grads, size_t gather_k) {
     if (!on) return;
-    if (grads) wait(s, c->ev_grads[k & 1]);
-    if (gather_k != (size_t)-1 && gather_k >= 2) wait(s, c->ev_consumed[gather_k & 1]);
+    if (grads) wait(ks, c->ev_grads[k & 1]);
+    if (gather_k != (size_t)-1 && gather_k >= 2) wait(ks, c->ev_consumed[gather_k & 1]);
   }
   void after_kernel(size_t k) {
-    if (on) record(c->ev_kernel[k & 1], s);
+    if (on) record(c->ev_kernel[k & 1], ks);
   }
   void before_gather(size_t k) {
     if (on) wait(q, c->ev_kernel[k & 1]);
@@ -491,14 +499,20 @@ struct StepOrder {
   void after_gather(size_t k) {
     if (on) record(c->ev_consumed[k & 1], q);
   }
-  // Joins the side stream into `s`; returns the first CUDA error seen.
+  // Joins the callbacks' and the kernels' streams into `s`; returns the
+  // first CUDA error seen.
   cudaError_t end() {
     if (on && !joined) {
       joined = true;
       // the join is attempted even after an error, so that `s` never runs ahead
-      // of callback work already enqueued
+      // of work already enqueued on the other streams
       cudaError_t e1 = cudaEventRecord(c->ev_join, q);
       cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(s, c->ev_join, 0) : e1;
+      if (ks != s) {
+        cudaError_t e3 = cudaEventRecord(c->ev_kjoin, ks);
+        cudaError_t e4 = e3 == cudaSuccess ? cudaStreamWaitEvent(s, c->ev_kjoin, 0) : e3;
+        if (e2 == cudaSuccess) e2 = e4;
+      }
       if (err == cudaSuccess) err = e2;
     }
     return err;
@@ -509,8 +523,13 @@ struct StepOrder {
 zero_status ensure_pipeline(zero_ctx* c) {
   if (!c->pipeline || c->side) return ZERO_OK;
   cudaError_t e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
-  for (cudaEvent_t* ev : {&c->ev_start, &c->ev_join, &c->ev_grads[0], &c->ev_grads[1], &c->ev_kernel[0],
-                          &c->ev_kernel[1], &c->ev_consumed[0], &c->ev_consumed[1]})
+  if (e == cudaSuccess && c->pipeline == 2) {
+    int least = 0, greatest = 0;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&c->kside, cudaStreamNonBlocking, greatest);
+  }
+  for (cudaEvent_t* ev : {&c->ev_start, &c->ev_join, &c->ev_kjoin, &c->ev_grads[0], &c->ev_grads[1],
+                          &c->ev_kernel[0], &c->ev_kernel[1], &c->ev_consumed[0], &c->ev_consumed[1]})
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   if (e != cudaSuccess) return cuda_fail(c, e, "creating the pipeline stream and events");
   return ZERO_OK;
@@ -564,7 +583,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   const int N = c->plan.n_ranks;
   if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "clipping / skipping needs the reduced-gradient shards (ZERO_OPT_KEEP_GRAD_SHARDS = 1)");
-  cudaStream_t s = o.s;
+  cudaStream_t s = o.ks;  // the step's kernels; statistics are read on o.s after the join
   const int64_t t = c->t + 1;
   const std::vector<zsm::Span> iv = step_intervals(c);
   const int n_layers = (int)c->plan.layers.size();
@@ -654,7 +673,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   if (o.end() != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
   c->stats_step = c->t;
   c->norm_fresh = true;
-  if (stats) return finish_stats(c, s, stats);
+  if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
 }
 
@@ -684,7 +703,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   }
   c->last_coef = 1.0;
   c->last_skipped = 0;
-  cudaStream_t s = o.s;
+  cudaStream_t s = o.ks;  // the step's kernels
   const int64_t t = c->t + 1;
   const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
   const std::vector<zsm::Span> iv = step_intervals(c);
@@ -722,7 +741,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   c->t = t;
   c->stats_step = t;
   c->norm_fresh = true;
-  if (stats) return finish_stats(c, s, stats);
+  if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
 }
 
@@ -810,7 +829,8 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
       c->blocks_per_sm_opt = (int)value;
       break;
     case ZERO_OPT_PIPELINE:
-      c->pipeline = value != 0;
+      if (value < 0 || value > 2) return fail(c, ZERO_EINVAL, "pipeline must be 0, 1 or 2");
+      c->pipeline = (int)value;
       break;
     default:
       return fail(c, ZERO_EINVAL, "unknown option %d", key);
