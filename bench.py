@@ -75,6 +75,8 @@ def parse_args(argv=None):
                          "on the context's stream, on the 1.2B and 85M workloads; one JSON line per cell")
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
+    ap.add_argument("--stage", type=int, choices=(1, 2, 3), default=2,
+                    help="ZeRO stage of the bench line (the benchmark is stage 2)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
                     help="gpt-1.2b: the benchmark workload; flat-32m: a 33.5M-param flat buffer, "
                          "N = 8, one bucket (2 GB on the device); flat-8m-n64: 8.4M params, N = 64 "
@@ -206,6 +208,14 @@ def _gpt_1p2b():
     return W.gpt_1p2b_n8()
 
 
+def _gpt_85m():
+    from synth import workloads as W
+
+    w = W.gpt_85m_n8()
+    w.bucket_elems = 20_000_000
+    return w
+
+
 def _flat_32m():
     from synth import workloads as W
 
@@ -222,7 +232,7 @@ def _flat_8m_n64():
     return w
 
 
-WORKLOADS = {"gpt-1.2b": _gpt_1p2b, "flat-32m": _flat_32m, "flat-8m-n64": _flat_8m_n64}
+WORKLOADS = {"gpt-1.2b": _gpt_1p2b, "gpt-85m": _gpt_85m, "flat-32m": _flat_32m, "flat-8m-n64": _flat_8m_n64}
 _ARGS = None
 
 
@@ -230,10 +240,30 @@ def workload():
     return WORKLOADS[_ARGS.workload if _ARGS is not None else "gpt-1.2b"]()
 
 
-def cpu_baseline(w, steps: int = 2) -> dict:
+def fused_kernel_name(fc: dict, n_ranks: int) -> str:
+    """The fused kernel a context launches, from its zero_fused_config."""
+    if fc["kernel"] != "tma":
+        return "fused_step_kernel"
+    if n_ranks > 16:
+        return "fused_step_chunked_kernel"
+    return "fused_step_tma_wide_kernel" if fc["groups"] == 3 else "fused_step_tma_kernel"
+
+
+def bench_stage() -> int:
+    return _ARGS.stage if _ARGS is not None else 2
+
+
+def oracle_stage(stage: int) -> int:
+    import oracle
+
+    return {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2, 3: oracle.STAGE_Z3}[stage]
+
+
+def cpu_baseline(w, steps: int = 2, stage: int = 2) -> dict:
     """The oracle, as it stands (single-threaded), on a bounded sample of the
-    workload: the first transformer layer's tensors (50,358,272 params), the
-    same N, one fixed-size bucket, ``steps`` literal ZeRO-2 steps."""
+    workload: the first transformer layer's tensors (50,358,272 params for the
+    1.2B list), the same N and bucket size, ``steps`` literal steps of the
+    bench's stage."""
     import numpy as np
 
     import oracle
@@ -245,15 +275,16 @@ def cpu_baseline(w, steps: int = 2) -> dict:
     m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
     grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
              for r in range(w.n_ranks)]
-    ranks = oracle.init_states(p, oracle.STAGE_Z2, m0)
+    st = oracle_stage(stage)
+    ranks = oracle.init_states(p, st, m0)
     hp = oracle.AdamHP(**w.hyper.__dict__)
     t0 = time.perf_counter()
     for t in range(1, steps + 1):
-        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
     dt = time.perf_counter() - t0
     return {"value": p.psi * steps / dt, "unit": "params/s", "cores": 1, "kind": "oracle",
             "sample": f"first layer of the workload ({p.psi} params, N={w.n_ranks}), {steps} literal "
-                      f"ZeRO-2 steps, single-threaded C+numpy oracle, input generation untimed",
+                      f"ZeRO-{stage} steps, single-threaded C+numpy oracle, input generation untimed",
             "seconds": dt}
 
 
@@ -272,7 +303,8 @@ def run_ours(args, world, rank, local):
     w = workload()
     stream = torch.cuda.current_stream(dev)
     s = stream.cuda_stream
-    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, z.ZERO_STAGE_2, bucket_elems=w.bucket_elems,
+    stage = bench_stage()
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=w.bucket_elems,
                           hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
                           replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
                           kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True, device=dev)
@@ -322,7 +354,8 @@ def run_ours(args, world, rank, local):
     # stream (with programmatic dependent launch each starts as the one before
     # finishes), so their average launch duration is the region's time over
     # its launches.
-    launches = args.steps * len(opt.buckets())
+    intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
+    launches = args.steps * intervals
     kernel_ms = ms_local / launches
     achieved = model_bytes_per_step * args.steps / (ms_local / 1e3) / 1e9
     # the same kernel timed launch by launch (CUDA events around each launch,
@@ -337,9 +370,9 @@ def run_ours(args, world, rank, local):
     opt.set_timing(False)
     kernel_ms_isolated = kt["ms"] / max(1, kt["launches"])
     peak, peak_kind = measured_peaks()
-    elems_per_launch = w.psi / max(1, len(opt.buckets()))
+    elems_per_launch = w.psi / intervals
     fc = opt.fused_config()
-    ckey = f"stage2_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
+    ckey = f"stage{stage}_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
     traffic = traffic_for_current_kernel(fc["kernel"], ckey, elems_per_launch)
 
     # end to end through the C ABI: every bucket's N gradient slices copied
@@ -348,6 +381,8 @@ def run_ours(args, world, rank, local):
     e2e = None
     if not args.no_e2e:
         max_bucket = max(hi - lo for lo, hi in opt.buckets())
+        if stage == 3:
+            max_bucket = max(hi - lo for _, lo, hi in opt.layers())
         host = torch.empty((w.n_ranks, max_bucket), dtype=torch.int16, pin_memory=True)
         host.copy_(reps[:, :max_bucket])
         h2d = 0
@@ -382,7 +417,7 @@ def run_ours(args, world, rank, local):
                       "non-finite count) read back every step"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w)
+        cpu = cpu_baseline(w, stage=stage)
     out = {
         "metric": METRIC,
         "value": value,
@@ -396,8 +431,8 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "fp32",
         "data": "synthetic (seeded counter-hash gradients and weights, no dataset)",
-        "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks, "stage": 2,
-                   "bucket_elems": w.bucket_elems, "buckets": len(opt.buckets()),
+        "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks, "stage": stage,
+                   "bucket_elems": w.bucket_elems, "buckets": len(opt.buckets()), "launches_per_step": intervals,
                    "storage": "bf16 grads/params, fp32 master/m/v",
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
@@ -406,10 +441,10 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
-                     "kernel": "fused_step_tma_kernel" if fc["kernel"] == "tma" else "fused_step_kernel",
+                     "kernel": fused_kernel_name(fc, w.n_ranks),
                      "kernel_config": ckey,
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
-                     "model_bytes_per_launch": model_bytes_per_step / len(opt.buckets()),
+                     "model_bytes_per_launch": model_bytes_per_step / intervals,
                      "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
                                      "region (fused launches only, back to back"
                                      + (", programmatic dependent launch" if args.pdl else "") + ")",
@@ -658,26 +693,27 @@ def run_reference(args, world, rank, local):
     m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
     grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
              for r in range(w.n_ranks)]
-    ranks = oracle.init_states(p, oracle.STAGE_Z2, m0)
+    st = oracle_stage(args.stage)
+    ranks = oracle.init_states(p, st, m0)
     hp = oracle.AdamHP(**w.hyper.__dict__)
     t = 0
     for _ in range(args.warmup):
         t += 1
-        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         t += 1
-        oracle.step(p, oracle.STAGE_Z2, ranks, lambda t_, r: grads[r], t, hp)
+        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
     dt = time.perf_counter() - t0
     value = p.psi * args.steps / dt
     sample = (f"leading {p.psi} params of the first layer of {w.name} (N={w.n_ranks}) per step, "
-              f"literal ZeRO-2 step of the single-threaded oracle, input generation untimed")
+              f"literal ZeRO-{args.stage} step of the single-threaded oracle, input generation untimed")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic", "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks,
-                                        "stage": 2, "bucket_elems": w.bucket_elems},
+                                        "stage": args.stage, "bucket_elems": w.bucket_elems},
         "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
