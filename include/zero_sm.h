@@ -268,6 +268,20 @@ zero_status zero_init(const zero_layout* layout, int32_t n_ranks, int32_t stage,
 /* Set an option (ZERO_OPT_*) before zero_bind.  ZERO_ESTATE after binding. */
 zero_status zero_set_option(zero_ctx* ctx, int32_t key, int64_t value);
 
+/*
+ * Streams of ZERO_OPT_PIPELINE (host only; before the first pipelined step,
+ * ZERO_ESTATE after it): callback_stream is the stream grad_fn and gather_fn
+ * receive, kernel_stream the one the step's kernels run on at option value 2.
+ * NULL leaves that stream to the context, which then creates it on the first
+ * pipelined step (callbacks: a non-blocking stream; kernels: a non-blocking
+ * stream at the device's greatest priority) and destroys it in zero_destroy
+ * -- so work or bookkeeping of the caller's that still refers to it (for
+ * instance a memory allocator that remembers the streams a block was used
+ * on) must be finished by then.  Streams given here stay the caller's: the
+ * context never destroys them, and they must outlive it.
+ */
+zero_status zero_set_pipeline_streams(zero_ctx* ctx, void* callback_stream, void* kernel_stream);
+
 /* Sizes of the plan and of each arena (bytes).  Host only. */
 zero_status zero_buffer_sizes(const zero_ctx* ctx, zero_sizes* out);
 

@@ -236,3 +236,42 @@ def test_pipeline_callback_failure_leaves_the_context_usable():
         assert torch.equal(ref.view(what), opt.view(what))
     ref.close()
     opt.close()
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_pipeline_pinned_copies_on_the_callback_stream_outlive_the_context(mode):
+    """The callbacks copy from pinned host memory on the stream they are
+    given; torch remembers that stream for the pinned block and records an
+    event on it when the block is freed -- here after the optimizer is closed.
+    The binding hands the library torch's own pooled streams, which stay
+    valid, so the free is harmless; the values equal the in-order step's."""
+    z = _z()
+    numel, layer = W.transformer_layers(2, 64, 256)
+    w = W.Workload("pinned", numel, layer, 4, (2,), 16384, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 2,
+                   W.Hyper(), 0x360)
+    ref, fr = make_opt(w, 2, 16384, 0)
+    opt, _ = make_opt(w, 2, 16384, mode)
+    p = oracle.plan(numel, layer, 4, 16384)
+    host = torch.empty((4, p.psi_pad), dtype=torch.int16, pin_memory=True)
+    for r in range(4):
+        host[r].copy_(torch.from_numpy(W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, 1, r),
+                                                     w.grad_dist).view(np.int16)))
+
+    def gfn(t, lo, hi, bufs, stream):
+        with _on(stream):
+            for r, ptr in enumerate(bufs):
+                opt._tensor_at(ptr, hi - lo, torch.int16).copy_(host[r, lo:hi], non_blocking=True)
+        return 0
+
+    st = opt.step(gfn, stats=True)
+    st_ref = ref.step(lambda t, lo, hi, bufs, s: grad_fn_for(ref, fr)(1, lo, hi, bufs, s), stats=True)
+    assert st == st_ref
+    assert torch.equal(opt.view(z.ZERO_VIEW_MASTER), ref.view(z.ZERO_VIEW_MASTER))
+    opt.close()
+    ref.close()
+    del host
+    gc.collect()
+    torch.cuda.synchronize()
+    x = torch.empty(1 << 20, dtype=torch.int16, pin_memory=True)  # the host allocator runs again
+    del x
+    torch.cuda.synchronize()

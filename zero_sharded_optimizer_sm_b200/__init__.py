@@ -109,6 +109,7 @@ _SIGS = {
                                   ctypes.POINTER(ctypes.c_double)]),
     "zero_set_clip": (_i32, [_vp, ctypes.c_double, _i32]),
     "zero_set_loss_scale": (_i32, [_vp, ctypes.c_double]),
+    "zero_set_pipeline_streams": (_i32, [_vp, _vp, _vp]),
     "zero_fused_config": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
@@ -216,6 +217,15 @@ class ZeroOptimizer:
             ptrs[k] = t.data_ptr() if t is not None else None
         with torch.cuda.device(dev):
             self._check(zero_bind(ctx, ptrs), "zero_bind")
+            if self.pipeline:
+                # torch's pooled streams, which torch never destroys: its own
+                # bookkeeping (pinned-memory blocks remember the streams they
+                # were copied on) may refer to them after this context is gone
+                self._cb_stream = torch.cuda.Stream(device=dev)
+                self._k_stream = torch.cuda.Stream(device=dev, priority=-64) if self.pipeline == 2 else None
+                self._check(zero_set_pipeline_streams(ctx, self._cb_stream.cuda_stream,
+                                                      self._k_stream.cuda_stream if self._k_stream else None),
+                            "zero_set_pipeline_streams")
         self.set_hparams(hparams)
         self._keep = []  # callbacks alive during a call
 

@@ -79,6 +79,8 @@ struct zero_ctx {
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
   cudaStream_t side = nullptr;   // the callbacks' stream
   cudaStream_t kside = nullptr;  // the kernels' stream at the greatest priority (ZERO_OPT_PIPELINE = 2)
+  bool own_side = false, own_kside = false;  // created here (destroyed with the context)
+  bool pipeline_used = false;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_kjoin = nullptr;
   cudaEvent_t ev_grads[2] = {}, ev_kernel[2] = {}, ev_consumed[2] = {};
   // fused-kernel timing
@@ -92,8 +94,8 @@ struct zero_ctx {
     for (cudaEvent_t e : {ev_start, ev_join, ev_kjoin, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
                           ev_consumed[0], ev_consumed[1]})
       if (e) cudaEventDestroy(e);
-    if (side) cudaStreamDestroy(side);
-    if (kside) cudaStreamDestroy(kside);
+    if (side && own_side) cudaStreamDestroy(side);
+    if (kside && own_kside) cudaStreamDestroy(kside);
   }
 };
 
@@ -463,7 +465,7 @@ struct StepOrder {
   StepOrder(zero_ctx* ctx, cudaStream_t stream, bool callbacks)
       : c(ctx), s(stream), q(stream), ks(stream), on(ctx->pipeline != 0 && callbacks) {
     if (on) q = c->side;
-    if (on && c->kside) ks = c->kside;
+    if (on && c->pipeline == 2) ks = c->kside;
   }
   void record(cudaEvent_t e, cudaStream_t st) {
     if (err == cudaSuccess) err = cudaEventRecord(e, st);
@@ -520,18 +522,26 @@ struct StepOrder {
 };
 
 // Creates the side stream and events of ZERO_OPT_PIPELINE on first use.
+// Creates what ZERO_OPT_PIPELINE needs and the caller did not give
+// (zero_set_pipeline_streams) on first use: the streams and the events.
 zero_status ensure_pipeline(zero_ctx* c) {
-  if (!c->pipeline || c->side) return ZERO_OK;
-  cudaError_t e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
-  if (e == cudaSuccess && c->pipeline == 2) {
+  if (!c->pipeline) return ZERO_OK;
+  c->pipeline_used = true;
+  cudaError_t e = cudaSuccess;
+  if (!c->side) {
+    e = cudaStreamCreateWithFlags(&c->side, cudaStreamNonBlocking);
+    c->own_side = e == cudaSuccess;
+  }
+  if (e == cudaSuccess && c->pipeline == 2 && !c->kside) {
     int least = 0, greatest = 0;
     e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&c->kside, cudaStreamNonBlocking, greatest);
+    c->own_kside = e == cudaSuccess;
   }
   for (cudaEvent_t* ev : {&c->ev_start, &c->ev_join, &c->ev_kjoin, &c->ev_grads[0], &c->ev_grads[1],
                           &c->ev_kernel[0], &c->ev_kernel[1], &c->ev_consumed[0], &c->ev_consumed[1]})
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
-  if (e != cudaSuccess) return cuda_fail(c, e, "creating the pipeline stream and events");
+    if (e == cudaSuccess && !*ev) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(c, e, "creating the pipeline streams and events");
   return ZERO_OK;
 }
 
@@ -836,6 +846,16 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
       return fail(c, ZERO_EINVAL, "unknown option %d", key);
   }
   compute_layout(c);
+  return ZERO_OK;
+}
+
+zero_status zero_set_pipeline_streams(zero_ctx* c, void* callback_stream, void* kernel_stream) {
+  if (!c) return ZERO_EINVAL;
+  if (c->pipeline_used) return fail(c, ZERO_ESTATE, "the pipeline streams are set before the first pipelined step");
+  if (!callback_stream && !kernel_stream) return ZERO_OK;
+  c->side = static_cast<cudaStream_t>(callback_stream);
+  c->kside = static_cast<cudaStream_t>(kernel_stream);
+  c->own_side = c->own_kside = false;
   return ZERO_OK;
 }
 
