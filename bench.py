@@ -680,7 +680,7 @@ def reference_sample(w, steps_total: int, elems: int = 0):
 
 
 def run_reference(args, world, rank, local):
-    """The CPU oracle timed on the machine's host cores, same metric and unit."""
+    """The CPU oracle timed on this machine's host cores, same metric and unit."""
     if rank != 0:
         return
     from synth import workloads as W

@@ -57,7 +57,7 @@ typedef enum zero_status {
   ZERO_ENOMEM = 2,   /* an arena the caller sized is too small for this context */
   ZERO_ECUDA = 3,    /* a CUDA runtime error (launch or asynchronous fault) */
   ZERO_ESTATE = 4,   /* call out of order: arenas not bound, hyper-parameters unset */
-  ZERO_ENOTIMPL = 5  /* a combination this build does not provide */
+  ZERO_ENOTIMPL = 5  /* a combination the library does not provide */
 } zero_status;
 
 /* ZeRO stages ([T] section "一张总对比表"; [Q] section 一). */
