@@ -222,18 +222,28 @@ zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t) {
 constexpr size_t kMaxTimed = 4096;
 constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the staged kernel
 
-// Staged-kernel configuration chosen for N (consumer groups, ring depth),
-// measured on B200 with flat 256M-element buffers and the 1.2B-parameter
-// transformer list: few bytes per element (N <= 4) leave the consumers
-// compute-bound, so two groups win; at N = 5..8 one group of eight warps with
-// a two-deep ring keeps the fewest copies in flight and moves the most bytes;
-// at N = 9..16 (only two stages fit) one group of sixteen warps wins.  Above
-// N = 16 the rank-chunked staged kernel wins over the register kernel.
+// Staged-kernel configuration chosen for N and the stage (consumer groups,
+// ring depth), measured on B200 with flat 256M-element buffers and the
+// 1.2B-parameter transformer list.  Stage 2: few bytes per element (N <= 4)
+// leave the consumers compute-bound, so two groups win; at N = 5..8 one group
+// of eight warps with a two-deep ring keeps the fewest copies in flight and
+// moves the most bytes; at N = 9..16 (only two stages fit) one group of
+// sixteen warps wins.  Stages 1 and 3 store more per element (the all-reduce
+// write-back; the parameter shard besides the gather buffers), and there the
+// sixteen-warp group wins from N = 5 (at N = 8 by 4 % for stage 1 and 17 %
+// for stage 3 over one group of eight warps) and two groups with a two-deep
+// ring at N = 2..4.  Above N = 16 the rank-chunked staged kernel wins over
+// the register kernel.
 struct TmaChoice {
   int groups, stages;
 };
 
-TmaChoice tma_policy(int n_ranks) {
+TmaChoice tma_policy(int n_ranks, int stage) {
+  if (stage != ZERO_STAGE_2) {
+    if (n_ranks <= 1) return {2, 4};
+    if (n_ranks <= 4) return {2, 2};
+    return {zsm::kWideGroup, 2};
+  }
   if (n_ranks <= 2) return {2, 4};
   if (n_ranks <= 4) return {2, 2};
   if (n_ranks <= 8) return {1, 2};
@@ -243,12 +253,12 @@ TmaChoice tma_policy(int n_ranks) {
 // Consumer groups of the staged kernel for this context.
 int tma_groups(const zero_ctx* c) {
   if (c->tma_groups_opt) return c->tma_groups_opt;
-  return tma_policy(c->plan.n_ranks).groups;
+  return tma_policy(c->plan.n_ranks, c->stage).groups;
 }
 
 int tma_stages(const zero_ctx* c) {
   if (c->tma_stages_opt) return c->tma_stages_opt;
-  return tma_policy(c->plan.n_ranks).stages;
+  return tma_policy(c->plan.n_ranks, c->stage).stages;
 }
 
 // CTAs of a staged-kernel launch: SMs x the CTAs per SM asked for (1 by
