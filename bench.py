@@ -75,6 +75,8 @@ def parse_args(argv=None):
                          "on the context's stream, on the 1.2B and 85M workloads; one JSON line per cell")
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
+    ap.add_argument("--dtype", choices=("bf16", "f16"), default="bf16",
+                    help="16-bit storage of gradients and parameters (f16: IEEE binary16 with loss scale 1024)")
     ap.add_argument("--stage", type=int, choices=(1, 2, 3), default=2,
                     help="ZeRO stage of the bench line (the benchmark is stage 2)")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
@@ -307,7 +309,12 @@ def run_ours(args, world, rank, local):
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=w.bucket_elems,
                           hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
                           replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
-                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True, device=dev)
+                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True,
+                          dtype=z.ZERO_DTYPE_F16 if args.dtype == "f16" else z.ZERO_DTYPE_BF16, device=dev)
+    if args.dtype == "f16":
+        opt.set_loss_scale(1024.0)
+        w.grad_dist = synth.Dist(w.grad_dist.kind, w.grad_dist.width * 1024.0, w.grad_dist.zero_mod)
+    fill16 = synth.dev_f16 if args.dtype == "f16" else synth.dev_bf16
     offsets = opt.offsets()
     mv = opt.view(z.ZERO_VIEW_MASTER)
     b = W.master_base(w)
@@ -319,7 +326,7 @@ def run_ours(args, world, rank, local):
     for r in range(w.n_ranks):
         gb = W.grad_base(w, 1, r)
         for off, n in zip(offsets, w.numel):
-            synth.dev_bf16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
+            fill16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
     rep_list = list(reps)
     opt.set_pdl(args.pdl)
     torch.cuda.synchronize(dev)
@@ -433,7 +440,8 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded counter-hash gradients and weights, no dataset)",
         "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks, "stage": stage,
                    "bucket_elems": w.bucket_elems, "buckets": len(opt.buckets()), "launches_per_step": intervals,
-                   "storage": "bf16 grads/params, fp32 master/m/v",
+                   "storage": ("binary16 grads/params (loss scale 1024)" if args.dtype == "f16" else "bf16 grads/params")
+                              + ", fp32 master/m/v",
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
