@@ -591,9 +591,21 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
   norm_epilogue<tma_threads<1>()>(a.ns, sq, nf, a.accumulate);
 }
 
+// A programmatic dependent launch may place its CTAs while the grid before
+// it still runs.  These kernels are persistent -- one CTA per SM, tiles dealt
+// out by CTA index -- so an SM must never take two CTAs of one grid: with the
+// attribute the launch asks for at least this much shared memory, more than
+// half of an SM's 228 KB once the 1 KB each block reserves is counted, and a
+// dependent grid's CTAs then land only on SMs the grid before has left.
+constexpr size_t kPdlSoloSmem = 116 * 1024;
+
+size_t pdl_smem(const FusedArgs& a, size_t bytes) {
+  return a.pdl != kPdlNone && bytes < kPdlSoloSmem ? kPdlSoloSmem : bytes;
+}
+
 template <int MODE>
 cudaError_t launch_chunked_mode(const FusedArgs& a, int grid, int cstages, int sstages, cudaStream_t s) {
-  const size_t bytes = chunked_smem_bytes(cstages, sstages);
+  const size_t bytes = pdl_smem(a, chunked_smem_bytes(cstages, sstages));
   const bool pdl = a.pdl != kPdlNone;
   if (a.fmt == kFmtF16)
     return launch_kernel(fused_step_chunked_kernel<MODE, F16>, grid, tma_threads<1>(), bytes, s, pdl, a, cstages,
@@ -618,7 +630,7 @@ cudaError_t launch_tma_fmt(const FusedArgs& a, int grid, int stages, int groups,
 
 template <int MODE>
 cudaError_t launch_tma_mode(const FusedArgs& a, int grid, int stages, int groups, cudaStream_t s) {
-  const size_t bytes = tma_smem_bytes(a.n_ranks, stages);
+  const size_t bytes = pdl_smem(a, tma_smem_bytes(a.n_ranks, stages));
   if (a.fmt == kFmtF16) return launch_tma_fmt<MODE, F16>(a, grid, stages, groups, bytes, s);
   return launch_tma_fmt<MODE, Bf16>(a, grid, stages, groups, bytes, s);
 }

@@ -228,23 +228,23 @@ constexpr int64_t kTmaTile = 2048;  // elements per shared-memory tile of the st
 // leave the consumers compute-bound, so two groups win; at N = 5..8 one group
 // of eight warps with a two-deep ring keeps the fewest copies in flight and
 // moves the most bytes; at N = 9..16 (only two stages fit) one group of
-// sixteen warps wins.  Stages 1 and 3 store more per element (the all-reduce
-// write-back; the parameter shard besides the gather buffers), and there the
-// sixteen-warp group wins from N = 5 (at N = 8 by 4 % for stage 1 and 17 %
-// for stage 3 over one group of eight warps) and two groups with a two-deep
-// ring at N = 2..4.  Above N = 16 the rank-chunked staged kernel wins over
-// the register kernel.
+// sixteen warps wins.  Stage 1 stores 2N more bytes per element (the
+// all-reduce write-back), and there the sixteen-warp group wins from N = 5
+// (by 3.5 % at N = 8); stages 1 and 3 take two groups with a two-deep ring at
+// N = 2.  Above N = 16 the rank-chunked staged kernel wins over the register
+// kernel.
 struct TmaChoice {
   int groups, stages;
 };
 
 TmaChoice tma_policy(int n_ranks, int stage) {
-  if (stage != ZERO_STAGE_2) {
+  if (stage == ZERO_STAGE_1) {
     if (n_ranks <= 1) return {2, 4};
     if (n_ranks <= 4) return {2, 2};
     return {zsm::kWideGroup, 2};
   }
-  if (n_ranks <= 2) return {2, 4};
+  if (n_ranks <= 1) return {2, 4};
+  if (n_ranks <= 2) return stage == ZERO_STAGE_3 ? TmaChoice{2, 2} : TmaChoice{2, 4};
   if (n_ranks <= 4) return {2, 2};
   if (n_ranks <= 8) return {1, 2};
   return {zsm::kWideGroup, 2};
@@ -738,7 +738,9 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   // ones at stage 1/2 touch disjoint intervals and share only the norm
   // scratch, so they stream at once; stage 3's launches all write the one
   // temporary gather buffer, so they wait first.
-  const bool pdl_ok = c->pdl && !callbacks;
+  // (and not with two staged CTAs per SM asked for: a programmatic launch
+  // keeps one per SM)
+  const bool pdl_ok = c->pdl && !callbacks && c->tma_ctas_opt <= 1;
   for (size_t k = 0; k < iv.size() && st == ZERO_OK; ++k) {
     for (; issued < iv.size() && issued <= k + o.ahead() && st == ZERO_OK; ++issued)
       st = issue_grads(c, o, fn, user, resident, iv, issued, t);
