@@ -58,9 +58,8 @@ def parse_args(argv=None):
     ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
                     help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
-    ap.add_argument("--pdl", action="store_true",
-                    help="launch the step's fused kernels with programmatic dependent launch "
-                         "(ZERO_OPT_PDL; off by default, measured slower)")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch the step's fused kernels plainly (no programmatic dependent launch)")
     ap.add_argument("--sweep", action="store_true",
                     help="flat-buffer sweep instead of the bench line: 1K..1G elements (x4) x N in "
                          "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
@@ -328,7 +327,7 @@ def run_ours(args, world, rank, local):
         for off, n in zip(offsets, w.numel):
             fill16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
     rep_list = list(reps)
-    opt.set_pdl(args.pdl)
+    opt.set_pdl(not args.no_pdl)
     torch.cuda.synchronize(dev)
     # model bytes of one step's fused launches, from the library's own record
     opt.set_timing(True)
@@ -445,7 +444,7 @@ def run_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
-                   "kernel": args.kernel, "fused_config": fc, "pdl": args.pdl},
+                   "kernel": args.kernel, "fused_config": fc, "pdl": not args.no_pdl},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
@@ -455,7 +454,7 @@ def run_ours(args, world, rank, local):
                      "model_bytes_per_launch": model_bytes_per_step / intervals,
                      "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
                                      "region (fused launches only, back to back"
-                                     + (", programmatic dependent launch" if args.pdl else "") + ")",
+                                     + ("" if args.no_pdl else ", programmatic dependent launch") + ")",
                      "kernel_ms_per_launch_isolated": kernel_ms_isolated,
                      "achieved_isolated": kt["model_bytes"] / max(1, kt["launches"])
                                           / (kernel_ms_isolated / 1e3) / 1e9,
@@ -594,7 +593,7 @@ def run_stages(args):
                     for off, n in zip(opt.offsets(), w.numel):
                         synth.dev_bf16(W.grad_base(w, 1, r), off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
             rl = list(reps)
-            opt.set_pdl(args.pdl)
+            opt.set_pdl(not args.no_pdl)
             for _ in range(3):
                 opt.step_resident(rl)
             steps = max(5, int(2e9 / ((4 * w.n_ranks + 24) * w.psi)) + 5)
@@ -621,7 +620,7 @@ def run_stages(args):
                               "bytes_per_elem_model": per,
                               "step_gbs_model": per * w.psi / (ms / 1e3) / 1e9,
                               "kernel_gbs_model_isolated": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
-                              "pdl": args.pdl,
+                              "pdl": not args.no_pdl,
                               "launches_per_step": kt["launches"] // steps,
                               "fused_config": opt.fused_config(), "steps": steps}), flush=True)
             opt.close()

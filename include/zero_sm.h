@@ -169,15 +169,16 @@ enum {
                                     at the end), so that their CTAs take the SMs that the
                                     callbacks' work frees first.  Values are unchanged.
                                     Default 0; before zero_bind */
-  ZERO_OPT_PDL = 12              /* 1: a step without callbacks (zero_step_resident with no
-                                    gather_fn) launches its fused kernels with programmatic
-                                    dependent launch, so that each launch's CTAs start on the
-                                    SMs the previous launch leaves and, at stage 1/2, stream
-                                    their own interval while it finishes.  0 (default): plain
-                                    launches -- faster on B200 for the persistent staged
-                                    kernels, whose one-CTA-per-SM placement the early launch
-                                    breaks.  Values are unchanged either way.  Off while
-                                    ZERO_OPT_TIMING is on.  May be set at any time */
+  ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
+                                    with no gather_fn) launches its fused kernels with
+                                    programmatic dependent launch, so that each launch's CTAs
+                                    start on the SMs the previous launch leaves and, at stage
+                                    1/2, stream their own interval while it finishes (a staged
+                                    launch then reserves at least 116 KB of shared memory, so
+                                    that an SM never holds two CTAs of one grid); 0: plain
+                                    launches.  Values are unchanged either way.  Off while
+                                    ZERO_OPT_TIMING is on, and with ZERO_OPT_TMA_CTAS_PER_SM
+                                    above 1.  May be set at any time */
 };
 
 /* 16-bit storage formats (ZERO_OPT_DTYPE).  The pages account gradients and

@@ -430,7 +430,7 @@ class ZeroOptimizer:
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
 
     def set_pdl(self, on: bool):
-        """Programmatic dependent launch between a callback-free step's fused launches (default off)."""
+        """Programmatic dependent launch between a callback-free step's fused launches (default on)."""
         self._check(zero_set_option(self.ctx, ZERO_OPT_PDL, 1 if on else 0), "zero_set_option")
 
     def set_timing(self, on: bool):
