@@ -152,6 +152,25 @@ def test_pipeline_option_doubles_only_the_slot_arenas(stage):
         assert on[k] == (2 * off[k] if doubled else off[k]), (k, off[k], on[k])
 
 
+def test_pipeline_streams_and_option_values_on_the_host():
+    """zero_set_pipeline_streams needs no GPU before the first pipelined step
+    (it only records the handles); ZERO_OPT_PIPELINE takes 0, 1 or 2."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    st, ctx = _init([64, 64], [0, 1], 2, 3, 64)
+    assert st == 0
+    try:
+        assert z.zero_set_pipeline_streams(ctx, None, None) == z.ZERO_OK
+        assert z.zero_set_pipeline_streams(ctx, 0x1000, None) == z.ZERO_OK
+        assert z.zero_set_pipeline_streams(None, None, None) == z.ZERO_EINVAL
+        for v in (0, 1, 2):
+            assert z.zero_set_option(ctx, z.ZERO_OPT_PIPELINE, v) == z.ZERO_OK
+        assert z.zero_set_option(ctx, z.ZERO_OPT_PIPELINE, 3) == z.ZERO_EINVAL
+        assert z.zero_set_option(ctx, z.ZERO_OPT_PDL, 0) == z.ZERO_OK
+    finally:
+        z.zero_destroy(ctx)
+
+
 def test_init_rejects_bad_arguments():
     import zero_sharded_optimizer_sm_b200 as z
 

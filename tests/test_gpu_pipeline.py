@@ -275,3 +275,15 @@ def test_pipeline_pinned_copies_on_the_callback_stream_outlive_the_context(mode)
     x = torch.empty(1 << 20, dtype=torch.int16, pin_memory=True)  # the host allocator runs again
     del x
     torch.cuda.synchronize()
+
+
+def test_pipeline_streams_are_fixed_after_the_first_pipelined_step():
+    z = _z()
+    numel, layer = W.transformer_layers(2, 32, 128)
+    w = W.Workload("streams", numel, layer, 2, (2,), 4096, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 1,
+                   W.Hyper(), 0x370)
+    opt, fill = make_opt(w, 2, 4096, 1)
+    opt.step(grad_fn_for(opt, fill))
+    other = torch.cuda.Stream()
+    assert z.zero_set_pipeline_streams(opt.ctx, other.cuda_stream, None) == z.ZERO_ESTATE
+    opt.close()
