@@ -74,6 +74,9 @@ def parse_args(argv=None):
                          "on the context's stream, on the 1.2B and 85M workloads; one JSON line per cell")
     ap.add_argument("--ref-sample-elems", type=int, default=0,
                     help="reference arm: elements per oracle step (0 = sized to about a minute)")
+    ap.add_argument("--clip", type=float, default=0.0,
+                    help="global-norm clip at this norm with the overflow skip on: the two-pass step "
+                         "(reduce everything, read the norm, then Adam + broadcast)")
     ap.add_argument("--dtype", choices=("bf16", "f16"), default="bf16",
                     help="16-bit storage of gradients and parameters (f16: IEEE binary16 with loss scale 1024)")
     ap.add_argument("--stage", type=int, choices=(1, 2, 3), default=2,
@@ -306,7 +309,7 @@ def run_ours(args, world, rank, local):
     s = stream.cuda_stream
     stage = bench_stage()
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=w.bucket_elems,
-                          hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=False,
+                          hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=args.clip > 0,
                           replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
                           kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True,
                           dtype=z.ZERO_DTYPE_F16 if args.dtype == "f16" else z.ZERO_DTYPE_BF16, device=dev)
@@ -314,6 +317,8 @@ def run_ours(args, world, rank, local):
         opt.set_loss_scale(1024.0)
         w.grad_dist = synth.Dist(w.grad_dist.kind, w.grad_dist.width * 1024.0, w.grad_dist.zero_mod)
     fill16 = synth.dev_f16 if args.dtype == "f16" else synth.dev_bf16
+    if args.clip > 0:
+        opt.set_clip(args.clip, True)
     offsets = opt.offsets()
     mv = opt.view(z.ZERO_VIEW_MASTER)
     b = W.master_base(w)
@@ -336,6 +341,14 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     model_bytes_per_step = opt.kernel_timing()["model_bytes"]
     opt.set_timing(False)
+    if args.clip > 0:
+        # the two-pass step's kernels (reduce, then Adam + broadcast) are not in
+        # the fused-launch record: its byte model per element is the reduce's
+        # 2N+2 plus the update's 2+24+2N (+2 for the stage-3 parameter shard),
+        # and at stage 1 the reduce writes the mean back to the N replicas (4N)
+        n = w.n_ranks
+        per = {1: 4 * n + 2 + 24 + 2 * n, 2: 4 * n + 28, 3: 4 * n + 30}[stage]
+        model_bytes_per_step = per * opt.psi_pad
     for _ in range(args.warmup):
         opt.step_resident(rep_list)
     torch.cuda.synchronize(dev)
@@ -361,12 +374,13 @@ def run_ours(args, world, rank, local):
     # finishes), so their average launch duration is the region's time over
     # its launches.
     intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
-    launches = args.steps * intervals
+    per_step_launches = intervals if args.clip <= 0 else intervals + (1 if stage != 3 else intervals)
+    launches = args.steps * per_step_launches
     kernel_ms = ms_local / launches
     achieved = model_bytes_per_step * args.steps / (ms_local / 1e3) / 1e9
     # the same kernel timed launch by launch (CUDA events around each launch,
     # which also turns programmatic dependent launch off)
-    iso_steps = 20
+    iso_steps = 20 if args.clip <= 0 else 0  # the two-pass kernels are not timed one by one
     opt.set_timing(True)
     opt.kernel_timing()
     for _ in range(iso_steps):
@@ -374,12 +388,12 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     kt = opt.kernel_timing()
     opt.set_timing(False)
-    kernel_ms_isolated = kt["ms"] / max(1, kt["launches"])
+    kernel_ms_isolated = kt["ms"] / kt["launches"] if kt["launches"] else None
     peak, peak_kind = measured_peaks()
     elems_per_launch = w.psi / intervals
     fc = opt.fused_config()
     ckey = f"stage{stage}_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
-    traffic = traffic_for_current_kernel(fc["kernel"], ckey, elems_per_launch)
+    traffic = traffic_for_current_kernel(fc["kernel"], ckey, elems_per_launch) if args.clip <= 0 else None
 
     # end to end through the C ABI: every bucket's N gradient slices copied
     # from pinned host memory into the fixed-size buffer, then the fused
@@ -438,6 +452,7 @@ def run_ours(args, world, rank, local):
         "dtype": "fp32",
         "data": "synthetic (seeded counter-hash gradients and weights, no dataset)",
         "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks, "stage": stage,
+                   "step": (f"two-pass (clip at {args.clip}, overflow skip)" if args.clip > 0 else "fused"),
                    "bucket_elems": w.bucket_elems, "buckets": len(opt.buckets()), "launches_per_step": intervals,
                    "storage": ("binary16 grads/params (loss scale 1024)" if args.dtype == "f16" else "bf16 grads/params")
                               + ", fp32 master/m/v",
@@ -448,16 +463,17 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
-                     "kernel": fused_kernel_name(fc, w.n_ranks),
+                     "kernel": (fused_kernel_name(fc, w.n_ranks) if args.clip <= 0
+                                else "reduce_kernel + adam_bcast_kernel (two-pass step)"),
                      "kernel_config": ckey,
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
-                     "model_bytes_per_launch": model_bytes_per_step / intervals,
+                     "model_bytes_per_launch": model_bytes_per_step / per_step_launches,
                      "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
                                      "region (fused launches only, back to back"
                                      + ("" if args.no_pdl else ", programmatic dependent launch") + ")",
                      "kernel_ms_per_launch_isolated": kernel_ms_isolated,
-                     "achieved_isolated": kt["model_bytes"] / max(1, kt["launches"])
-                                          / (kernel_ms_isolated / 1e3) / 1e9,
+                     "achieved_isolated": (kt["model_bytes"] / kt["launches"] / (kernel_ms_isolated / 1e3) / 1e9
+                                           if kernel_ms_isolated else None),
                      "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None},
         "cpu_baseline": cpu,
         "e2e": e2e,
