@@ -339,16 +339,9 @@ def run_ours(args, world, rank, local):
     opt.kernel_timing()
     opt.step_resident(rep_list)
     torch.cuda.synchronize(dev)
-    model_bytes_per_step = opt.kernel_timing()["model_bytes"]
+    rec = opt.kernel_timing()
+    model_bytes_per_step, per_step_launches = rec["model_bytes"], rec["launches"]
     opt.set_timing(False)
-    if args.clip > 0:
-        # the two-pass step's kernels (reduce, then Adam + broadcast) are not in
-        # the fused-launch record: its byte model per element is the reduce's
-        # 2N+2 plus the update's 2+24+2N (+2 for the stage-3 parameter shard),
-        # and at stage 1 the reduce writes the mean back to the N replicas (4N)
-        n = w.n_ranks
-        per = {1: 4 * n + 2 + 24 + 2 * n, 2: 4 * n + 28, 3: 4 * n + 30}[stage]
-        model_bytes_per_step = per * opt.psi_pad
     for _ in range(args.warmup):
         opt.step_resident(rep_list)
     torch.cuda.synchronize(dev)
@@ -374,13 +367,12 @@ def run_ours(args, world, rank, local):
     # finishes), so their average launch duration is the region's time over
     # its launches.
     intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
-    per_step_launches = intervals if args.clip <= 0 else intervals + (1 if stage != 3 else intervals)
     launches = args.steps * per_step_launches
     kernel_ms = ms_local / launches
     achieved = model_bytes_per_step * args.steps / (ms_local / 1e3) / 1e9
     # the same kernel timed launch by launch (CUDA events around each launch,
     # which also turns programmatic dependent launch off)
-    iso_steps = 20 if args.clip <= 0 else 0  # the two-pass kernels are not timed one by one
+    iso_steps = 20
     opt.set_timing(True)
     opt.kernel_timing()
     for _ in range(iso_steps):

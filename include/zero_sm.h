@@ -134,7 +134,8 @@ enum {
                                     the buffers' lengths are large powers of two; default 0 */
   ZERO_OPT_BLOCKS_PER_SM = 3,    /* fused-kernel CTAs per SM (0 = occupancy maximum) */
   ZERO_OPT_TIMING = 4,           /* 1: record a CUDA event pair on the launching stream around
-                                    every fused-step kernel launch (read with
+                                    every launch of the step's kernels -- the fused kernel, or
+                                    the two passes of a clipped step -- (read with
                                     zero_kernel_timing); may be set at any time; default 0 */
   ZERO_OPT_KERNEL = 5,           /* fused-step kernel: ZERO_KERNEL_AUTO (default),
                                     ZERO_KERNEL_REGISTER or ZERO_KERNEL_TMA; may be set at any
@@ -186,7 +187,9 @@ enum {
  * configuration); bf16 is the default. */
 enum { ZERO_DTYPE_BF16 = 0, ZERO_DTYPE_F16 = 1 };
 
-/* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits.
+/* Fused-step kernels (ZERO_OPT_KERNEL).  Both compute the same bits, and the
+ * choice also applies to the two passes of a clipped step (zero_set_clip),
+ * which TMA stages the same way for N <= 16.
  *   REGISTER: each lane loads its 16-byte slices of the N replicas and of
  *             master/m/v straight into registers (any N).
  *   TMA:      one CTA per SM with one or two groups, each a producer thread
@@ -479,7 +482,9 @@ zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
  * per element, stage 1: 6N+24 (N gradient reads, N all-reduce write-backs,
  * 12 B of state read and written, N parameter writes), stage 2: 4N+24,
  * stage 3: 4N+26 (plus the parameter shard), each +2 when the reduced
- * gradient shard is kept.  Resets the record.  At most 4096 launches are
+ * gradient shard is kept.  A clipped step's passes count the reduce as 2N+2
+ * (4N at stage 1, the all-reduce written back) and the Adam-broadcast as
+ * 2+24+2N (+2 at stage 3).  Resets the record.  At most 4096 launches are
  * recorded between two calls; later ones are not timed.
  */
 zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, double* model_bytes);

@@ -704,6 +704,44 @@ def test_clip_and_overflow_skip_against_oracle(stage):
     opt.close()
 
 
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_two_pass_staged_kernels_equal_register_kernels(stage):
+    """The clipped step's two passes run staged through shared memory for
+    N <= 16 and on the register path when that is asked for: the same bits.
+    Small layouts make the shards 8-64 elements long, so a 2048-element tile
+    reads the reduced gradient from many owners (stage 1: one copy per owner);
+    ragged tails; clip active; 3 steps; both 16-bit formats."""
+    z = _z()
+    for numel, layer in (([3000, 1, 4100], [0, 1, 2]), ([40, 8, 24], [0, 0, 1]), ([70000], [0])):
+        for n_ranks in (1, 2, 3, 5, 8, 16):
+            for dtype in (z.ZERO_DTYPE_BF16, z.ZERO_DTYPE_F16):
+                w = W.Workload("two-pass", numel, layer, n_ranks, (stage,), 16384,
+                               synth.Dist(synth.NORMAL, 1e-2, zero_mod=7), W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01),
+                               0x500 + n_ranks)
+                opts = []
+                for kernel in (TMA, REG):
+                    o, f = make_opt(w, stage, bucket=16384, kernel=kernel, dtype=dtype)
+                    o.set_clip(0.01, True)
+                    opts.append((o, f))
+                for t in range(1, 4):
+                    sts = [o.step(grad_fn_for(o, f), stats=True) for o, f in opts]
+                    assert sts[0]["clip_coef"] < 1.0
+                    assert sts[0]["nonfinite"] == sts[1]["nonfinite"]
+                    assert math.isclose(sts[0]["grad_norm"], sts[1]["grad_norm"], rel_tol=1e-12)
+                (a, _), (b, _) = opts
+                for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+                    assert torch.equal(a.view(what), b.view(what)), (numel, n_ranks, stage, what)
+                for r in range(n_ranks if stage != 3 else 1):
+                    assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+                if stage == 1:
+                    for r in range(n_ranks):
+                        assert torch.equal(a.view(z.ZERO_VIEW_GRAD_BUF, r), b.view(z.ZERO_VIEW_GRAD_BUF, r))
+                else:
+                    assert torch.equal(a.view(z.ZERO_VIEW_GRAD_SHARD), b.view(z.ZERO_VIEW_GRAD_SHARD))
+                a.close()
+                b.close()
+
+
 def test_inactive_clip_two_pass_equals_fused_step():
     z = _z()
     numel, layer = W.transformer_layers(2, 64, 256)

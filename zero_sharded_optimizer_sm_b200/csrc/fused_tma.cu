@@ -24,87 +24,14 @@
 
 #include "device_math.cuh"
 #include "kernels.cuh"
+#include "tma_pipe.cuh"
 
 namespace zsm {
 namespace {
 
 using namespace dev;
+using namespace pipe;
 
-constexpr int kConsumerWarps = 8;                   // warps of one consumer group
-constexpr int kConsumers = kConsumerWarps * 32;     // 256 threads per group, 8 elements each
-constexpr int kTile = kConsumers * kVec;            // 2048 elements per tile
-
-// G consumer groups, each with its own producer warp: G * (32 + 256) threads.
-template <int G>
-__host__ __device__ constexpr int tma_threads() { return G * (32 + kConsumers); }
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s per wait
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long now_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
-  unsigned ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Wait for the phase with the given parity to complete; false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = now_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (now_ns() - t0 > kWaitNs) return false;
-  return true;
-}
-
-// L2 policy for the bulk loads: every input byte is read exactly once, so it
-// is marked first to evict and leaves L2 room for the write-back traffic.
-__device__ __forceinline__ uint64_t evict_first_policy() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-// 1-D bulk copy global -> this CTA's shared memory, completion on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar,
-                                          uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
-}
-
-// Plain (write-back) 16-byte stores for the consumers' outputs; measured ~1 %
-// faster than streaming stores in this kernel on B200.
-__device__ __forceinline__ void st_out(uint16_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }
-__device__ __forceinline__ void st_out(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 
 __host__ __device__ inline unsigned tma_stage_bytes(int n_ranks) {
   return (unsigned)(kTile * (2 * n_ranks + 12));
@@ -267,7 +194,6 @@ __device__ __forceinline__ void add4(float (&acc)[4], uint2 w) {
   acc[3] = __fadd_rn(acc[3], F::hi(w.y));
 }
 
-__device__ __forceinline__ void st_out(uint16_t* p, uint2 v) { *reinterpret_cast<uint2*>(p) = v; }
 
 template <int MODE, class F>
 __global__ void __launch_bounds__(kWideThreads, 1)

@@ -135,6 +135,7 @@ struct AdamBcastArgs {
   int64_t n_vec;
   int n_out;
   AdamScalars sc;                   // including the unscale / clip factors
+  unsigned int* error;              // staged kernel: set when a bounded wait runs out
 };
 
 struct GatherArgs {
@@ -186,5 +187,13 @@ cudaError_t tma_configure();       // opt in to the large dynamic smem (current 
 
 // Resident CTAs per SM of the fused kernel for `mode` and of the simple kernels.
 cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_blocks);
+
+// The two passes of the clipped / overflow-checked step, staged through
+// shared memory (two_pass_tma.cu; N <= 16).  `uniform`: every gsrc[r] is the
+// same array (the reduced-gradient shards), so one copy per tile suffices.
+cudaError_t two_pass_configure();
+cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_adam_bcast_tma(const AdamBcastArgs& a, int grid, bool uniform, cudaStream_t s);
+int64_t two_pass_tile();
 
 }  // namespace zsm

@@ -1,0 +1,323 @@
+// The two passes of the clipped / overflow-checked step with their inputs
+// staged through shared memory by the Tensor Memory Accelerator (sm_100a),
+// for N <= 16.  Same arithmetic, in the same order, as reduce_kernel and
+// adam_bcast_kernel in kernels.cu; different data movement, as in the fused
+// staged kernel: one persistent CTA per SM, warp 0's elected lane streams each
+// 2048-element tile into a ring of shared-memory stages with 1-D bulk copies
+// (completion counted in bytes on an mbarrier), eight consumer warps take
+// their 8 elements from shared memory, release the stage and store.
+//
+// Pass 1 (reduce_tma_kernel): the tile's N gradient slices; the consumers add
+//   them in rank order, take the 1/N mean, store it into the reduced-gradient
+//   shard (stages 2, 3) or back into every replica (stage 1, the all-reduce)
+//   and accumulate the gradient norm.
+// Pass 2 (adam_bcast_tma_kernel): the owners' reduced gradient and the fp32
+//   master, m, v; the consumers run Adam with the loss-scale and clipping
+//   factors and store the 16-bit result to every destination.
+//
+// Every wait is bounded (kWaitNs); one that runs out records an error code,
+// stops the producer, drains the copies in flight and ends the CTA.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "device_math.cuh"
+#include "kernels.cuh"
+#include "tma_pipe.cuh"
+
+namespace zsm {
+namespace {
+
+using namespace dev;
+using namespace pipe;
+
+constexpr int kTpThreads = tma_threads<1>();  // one producer warp + 8 consumer warps
+constexpr int kTpStages = 4;                  // ring depth of both passes
+
+__host__ __device__ inline unsigned reduce_stage_bytes(int n_ranks) { return (unsigned)(kTile * 2 * n_ranks); }
+// pass 2 stage: [16-bit gradient, 2 B][master, 4 B][m, 4 B][v, 4 B] per element
+constexpr unsigned kBcastStageBytes = kTile * 14;
+
+// [stages x stage_bytes][full[stages]][empty[stages]][abort][last_k[stages]]
+inline size_t tp_smem_bytes(unsigned stage_bytes, int stages) {
+  return (size_t)stages * stage_bytes + 2 * stages * sizeof(uint64_t) + 4 * (stages + 1);
+}
+
+struct Ring {
+  uint64_t* full;
+  uint64_t* empty;
+  volatile int* abort_flag;
+  volatile int* last_k;
+};
+
+__device__ __forceinline__ Ring ring_at(unsigned char* smem, unsigned stage_bytes, int stages) {
+  Ring r;
+  r.full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stage_bytes);
+  r.empty = r.full + stages;
+  r.abort_flag = reinterpret_cast<volatile int*>(r.empty + stages);
+  r.last_k = r.abort_flag + 1;
+  return r;
+}
+
+__device__ __forceinline__ void ring_init(const Ring& r, int stages) {
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&r.full[s], 1);
+      mbar_init(&r.empty[s], kConsumerWarps);
+      r.last_k[s] = -1;
+    }
+    *r.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+}
+
+// After the CTA's loops: with an abort, wait (bounded) for the copies already
+// issued before the CTA's shared memory goes away.
+__device__ __forceinline__ void ring_drain(const Ring& r, int stages, unsigned int* error) {
+  __syncthreads();
+  if (*r.abort_flag && threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s)
+      if (r.last_k[s] >= 0 && !mbar_wait(&r.full[s], (unsigned)r.last_k[s] & 1u)) atomicOr(error, 4u);
+  }
+}
+
+// Producer side of one ring slot: wait for the consumers to release stage
+// `s` (phase k - 1); false (abort recorded) when the wait runs out.
+__device__ __forceinline__ bool acquire_stage(const Ring& r, int s, unsigned k, unsigned int* error) {
+  if (k > 0 && !mbar_wait(&r.empty[s], (k - 1) & 1u)) {
+    atomicOr(error, 1u);
+    *r.abort_flag = 1;
+    return false;
+  }
+  return true;
+}
+
+// Consumer side: wait (warp-uniformly) for stage `s` phase k; false to stop.
+__device__ __forceinline__ bool consume_stage(const Ring& r, int s, unsigned k, unsigned int* error, int lane) {
+  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&r.full[s], k & 1u));
+  if (!ok) {
+    if (lane == 0) atomicOr(error, 2u);
+    *r.abort_flag = 1;
+    return false;
+  }
+  return !__any_sync(0xFFFFFFFFu, *r.abort_flag != 0);
+}
+
+// -------------------------------------------------------------- pass 1 --
+
+template <bool kWriteBack, class F>
+__global__ void __launch_bounds__(kTpThreads, 1)
+    reduce_tma_kernel(const __grid_constant__ ReduceArgs a, int stages) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const unsigned stage_bytes = reduce_stage_bytes(N);
+  const Ring ring = ring_at(smem, stage_bytes, stages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+  ring_init(ring, stages);
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *ring.abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (!acquire_stage(ring, s, k, a.ns.error)) break;
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        unsigned char* st = smem + (size_t)s * stage_bytes;
+        mbar_expect_tx(&ring.full[s], (unsigned)(cnt * 2 * N));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &ring.full[s], policy);
+        ring.last_k[s] = (int)k;
+      }
+    }
+  } else {
+    const int j = (threadIdx.x - 32) * kVec;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      if (!consume_stage(ring, s, k, a.ns.error, lane)) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const unsigned char* st = smem + (size_t)s * stage_bytes;
+      const bool active = j < cnt;  // the last tile may be ragged
+      float acc[kVec];
+      if (active) {
+#pragma unroll
+        for (int q = 0; q < kVec; ++q) acc[q] = 0.0f;
+        for (int r = 0; r < N; ++r) add8<F>(acc, *reinterpret_cast<const uint4*>(st + (size_t)r * 2 * kTile + 2 * j));
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring.empty[s]);
+      if (active) {
+        const int64_t e = e0 + j;
+        uint16_t g16[kVec];
+        float g[kVec];
+        mean_bf16<F>(acc, a.inv_n, g16, g, sq, nf);
+        const uint4 gw = pack8(g16);
+        if (kWriteBack) {
+          for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+        } else {
+          st_out(a.shard_out + e, gw);
+        }
+      }
+    }
+  }
+  ring_drain(ring, stages, a.ns.error);
+  norm_epilogue<kTpThreads>(a.ns, sq, nf, a.accumulate);
+}
+
+// -------------------------------------------------------------- pass 2 --
+
+// gsrc[r] are flat-element-0 pointers; element i's reduced gradient is read
+// from its owner's copy, gsrc[i / shard] (all the same pointer when the
+// owners' copies are the one reduced-gradient shard array: `uniform`).
+template <class F>
+__global__ void __launch_bounds__(kTpThreads, 1)
+    adam_bcast_tma_kernel(const __grid_constant__ AdamBcastArgs a, int stages, int uniform) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const Ring ring = ring_at(smem, kBcastStageBytes, stages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+  ring_init(ring, stages);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *ring.abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (!acquire_stage(ring, s, k, a.error)) break;
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        unsigned char* st = smem + (size_t)s * kBcastStageBytes;
+        mbar_expect_tx(&ring.full[s], (unsigned)(cnt * 14));
+        const int64_t i0 = a.lo + e0;  // flat index of the tile's first element
+        if (uniform) {
+          bulk_load(st, a.gsrc[0] + i0, (unsigned)(2 * cnt), &ring.full[s], policy);
+        } else {
+          // one copy per owner: owners change every `shard` elements (a multiple of 8)
+          for (int64_t e = 0; e < cnt;) {
+            const int64_t owner = (i0 + e) / a.shard;
+            const int64_t next = (owner + 1) * a.shard - i0;
+            const int64_t end = next < cnt ? next : cnt;
+            bulk_load(st + 2 * e, a.gsrc[owner] + i0 + e, (unsigned)(2 * (end - e)), &ring.full[s], policy);
+            e = end;
+          }
+        }
+        unsigned char* stt = st + 2 * kTile;
+        bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &ring.full[s], policy);
+        bulk_load(stt + 4 * kTile, a.m + e0, (unsigned)(4 * cnt), &ring.full[s], policy);
+        bulk_load(stt + 8 * kTile, a.v + e0, (unsigned)(4 * cnt), &ring.full[s], policy);
+        ring.last_k[s] = (int)k;
+      }
+    }
+  } else {
+    const int j = (threadIdx.x - 32) * kVec;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      if (!consume_stage(ring, s, k, a.error, lane)) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const unsigned char* st = smem + (size_t)s * kBcastStageBytes;
+      const bool active = j < cnt;
+      float4 p0, p1, m0, m1, v0, v1;
+      uint4 gw;
+      if (active) {
+        gw = *reinterpret_cast<const uint4*>(st + 2 * j);
+        const float* stt = reinterpret_cast<const float*>(st + 2 * kTile);
+        p0 = *reinterpret_cast<const float4*>(stt + j);
+        p1 = *reinterpret_cast<const float4*>(stt + j + 4);
+        m0 = *reinterpret_cast<const float4*>(stt + kTile + j);
+        m1 = *reinterpret_cast<const float4*>(stt + kTile + j + 4);
+        v0 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j);
+        v1 = *reinterpret_cast<const float4*>(stt + 2 * kTile + j + 4);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring.empty[s]);
+      if (active) {
+        const int64_t e = e0 + j;
+        float g[kVec] = {F::lo(gw.x), F::hi(gw.x), F::lo(gw.y), F::hi(gw.y),
+                         F::lo(gw.z), F::hi(gw.z), F::lo(gw.w), F::hi(gw.w)};
+        uint16_t p16[kVec];
+        adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);  // loss-scale and clip factors via a.sc.flags
+        st_out(a.master + e, p0);
+        st_out(a.master + e + 4, p1);
+        st_out(a.m + e, m0);
+        st_out(a.m + e + 4, m1);
+        st_out(a.v + e, v0);
+        st_out(a.v + e + 4, v1);
+        const uint4 pw = pack8(p16);
+        if (a.param_shard) st_out(a.param_shard + e, pw);
+        for (int r = 0; r < a.n_out; ++r) st_out(a.out[r] + e, pw);
+      }
+    }
+  }
+  ring_drain(ring, stages, a.error);
+}
+
+template <class K>
+cudaError_t opt_in(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+}
+
+int reduce_stages(int n_ranks) {
+  int stages = kTpStages;
+  while (stages > 2 && tp_smem_bytes(reduce_stage_bytes(n_ranks), stages) > (size_t)kTmaMaxSmem) --stages;
+  return stages;
+}
+
+}  // namespace
+
+cudaError_t two_pass_configure() {
+  cudaError_t e = cudaSuccess;
+  if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<false, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<true, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<false, F16>);
+  if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<true, F16>);
+  if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<Bf16>);
+  if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<F16>);
+  return e;
+}
+
+cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s) {
+  if (a.n_ranks < 1 || a.n_ranks > kTmaMaxRanks) return cudaErrorInvalidValue;
+  const int stages = reduce_stages(a.n_ranks);
+  const size_t bytes = tp_smem_bytes(reduce_stage_bytes(a.n_ranks), stages);
+  if (a.fmt == kFmtF16) {
+    if (a.write_back) reduce_tma_kernel<true, F16><<<grid, kTpThreads, bytes, s>>>(a, stages);
+    else reduce_tma_kernel<false, F16><<<grid, kTpThreads, bytes, s>>>(a, stages);
+  } else {
+    if (a.write_back) reduce_tma_kernel<true, Bf16><<<grid, kTpThreads, bytes, s>>>(a, stages);
+    else reduce_tma_kernel<false, Bf16><<<grid, kTpThreads, bytes, s>>>(a, stages);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adam_bcast_tma(const AdamBcastArgs& a, int grid, bool uniform, cudaStream_t s) {
+  const size_t bytes = tp_smem_bytes(kBcastStageBytes, kTpStages);
+  if (a.fmt == kFmtF16)
+    adam_bcast_tma_kernel<F16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages, uniform ? 1 : 0);
+  else
+    adam_bcast_tma_kernel<Bf16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages, uniform ? 1 : 0);
+  return cudaGetLastError();
+}
+
+int64_t two_pass_tile() { return kTile; }
+
+}  // namespace zsm

@@ -594,6 +594,46 @@ zero_status issue_gather(zero_ctx* c, StepOrder& o, zero_gather_fn gfn, void* gu
   return ZERO_OK;
 }
 
+// The two-pass step's kernels: staged through shared memory for N <= 16
+// unless the register path is asked for; timed (ZERO_OPT_TIMING) like the
+// fused launches, with their own byte models.
+bool use_two_pass_tma(const zero_ctx* c) {
+  return c->plan.n_ranks <= zsm::kTmaMaxRanks && c->kernel_opt != ZERO_KERNEL_REGISTER;
+}
+
+int two_pass_grid(const zero_ctx* c, int64_t elems) {
+  const int64_t tiles = (elems + zsm::two_pass_tile() - 1) / zsm::two_pass_tile();
+  return (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count));
+}
+
+cudaError_t launch_pass1(zero_ctx* c, const zsm::ReduceArgs& a, cudaStream_t s) {
+  const int64_t elems = a.n_vec * zsm::kVec;
+  cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  const cudaError_t e = use_two_pass_tma(c) ? zsm::launch_reduce_tma(a, two_pass_grid(c, elems), s)
+                                            : zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
+  if (e == cudaSuccess && ev) {
+    cudaEventRecord(ev[1], s);
+    c->timed += 1;
+    c->timed_bytes += (double)(a.write_back ? 4 * a.n_ranks : 2 * a.n_ranks + 2) * (double)elems;
+  }
+  return e;
+}
+
+cudaError_t launch_pass2(zero_ctx* c, const zsm::AdamBcastArgs& b, bool uniform, cudaStream_t s) {
+  const int64_t elems = b.n_vec * zsm::kVec;
+  cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  const cudaError_t e = use_two_pass_tma(c) ? zsm::launch_adam_bcast_tma(b, two_pass_grid(c, elems), uniform, s)
+                                            : zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
+  if (e == cudaSuccess && ev) {
+    cudaEventRecord(ev[1], s);
+    c->timed += 1;
+    c->timed_bytes += (double)(2 + 24 + 2 * b.n_out + (b.param_shard ? 2 : 0)) * (double)elems;
+  }
+  return e;
+}
+
 // Clipped / overflow-checked step: reduce everything, read the norm, then
 // Adam + broadcast.
 zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
@@ -629,7 +669,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     a.ns = norm_scratch(c);
     o.before_kernel(k, !resident && fn, (size_t)-1);
     if (a.n_vec > 0) {
-      cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
+      cudaError_t e = launch_pass1(c, a, s);
       if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
       launched = true;
     }
@@ -675,9 +715,11 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
       b.shard = c->plan.shard;
       b.n_vec = (hi - lo) / zsm::kVec;
       b.sc = sc;
+      b.error = norm_scratch(c).error;
       o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
       if (b.n_vec > 0) {
-        cudaError_t e = zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
+        // stages 2 and 3 read every owner's reduced gradient from the one shard array
+        cudaError_t e = launch_pass2(c, b, c->stage != ZERO_STAGE_1, s);
         if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
       }
       o.after_kernel(k);
@@ -930,6 +972,7 @@ zero_status zero_bind(zero_ctx* c, void* const* arenas) {
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
   if (e == cudaSuccess) e = zsm::tma_configure();
+  if (e == cudaSuccess) e = zsm::two_pass_configure();
   if (e != cudaSuccess) return cuda_fail(c, e, "device query");
   if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
   c->grid_fused = std::max(1, std::min(zsm::kMaxGrid, c->sm_count * std::max(1, fused_blocks)));
