@@ -1149,7 +1149,7 @@ zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void*
   a.write_back = 0;
   a.inv_n = (float)(1.0 / (double)N);
   a.ns = norm_scratch(c);
-  cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_pass1(c, a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "reduce-scatter kernel launch");
   c->norm_fresh = false;
   return ZERO_OK;
@@ -1179,7 +1179,7 @@ zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
   a.write_back = 1;
   a.inv_n = (float)(1.0 / (double)N);
   a.ns = norm_scratch(c);
-  cudaError_t e = zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_pass1(c, a, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(c, e, "all-reduce kernel launch");
   c->norm_fresh = false;
   return ZERO_OK;
