@@ -706,14 +706,15 @@ def test_clip_and_overflow_skip_against_oracle(stage):
 
 @pytest.mark.parametrize("stage", [1, 2, 3])
 def test_two_pass_staged_kernels_equal_register_kernels(stage):
-    """The clipped step's two passes run staged through shared memory for
-    N <= 16 and on the register path when that is asked for: the same bits.
+    """The clipped step's two passes run staged through shared memory (the
+    reduce in chunks of 8 ranks above 16) and on the register path when that
+    is asked for: the same bits.
     Small layouts make the shards 8-64 elements long, so a 2048-element tile
     reads the reduced gradient from many owners (stage 1: one copy per owner);
     ragged tails; clip active; 3 steps; both 16-bit formats."""
     z = _z()
     for numel, layer in (([3000, 1, 4100], [0, 1, 2]), ([40, 8, 24], [0, 0, 1]), ([70000], [0])):
-        for n_ranks in (1, 2, 3, 5, 8, 16):
+        for n_ranks in (1, 2, 3, 5, 8, 16, 17, 40):  # above 16 the reduce streams rank chunks
             for dtype in (z.ZERO_DTYPE_BF16, z.ZERO_DTYPE_F16):
                 w = W.Workload("two-pass", numel, layer, n_ranks, (stage,), 16384,
                                synth.Dist(synth.NORMAL, 1e-2, zero_mod=7), W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01),

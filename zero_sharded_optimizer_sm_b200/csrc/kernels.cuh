@@ -189,8 +189,9 @@ cudaError_t tma_configure();       // opt in to the large dynamic smem (current 
 cudaError_t occupancy(int mode, int n_ranks, int* fused_blocks, int* simple_blocks);
 
 // The two passes of the clipped / overflow-checked step, staged through
-// shared memory (two_pass_tma.cu; N <= 16).  `uniform`: every gsrc[r] is the
-// same array (the reduced-gradient shards), so one copy per tile suffices.
+// shared memory (two_pass_tma.cu; the reduce streams the ranks in chunks of 8
+// above 16 ranks).  `uniform`: every gsrc[r] is the same array (the
+// reduced-gradient shards), so one copy per tile suffices.
 cudaError_t two_pass_configure();
 cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam_bcast_tma(const AdamBcastArgs& a, int grid, bool uniform, cudaStream_t s);

@@ -1,6 +1,5 @@
 // The two passes of the clipped / overflow-checked step with their inputs
-// staged through shared memory by the Tensor Memory Accelerator (sm_100a),
-// for N <= 16.  Same arithmetic, in the same order, as reduce_kernel and
+// staged through shared memory by the Tensor Memory Accelerator (sm_100a).  Same arithmetic, in the same order, as reduce_kernel and
 // adam_bcast_kernel in kernels.cu; different data movement, as in the fused
 // staged kernel: one persistent CTA per SM, warp 0's elected lane streams each
 // 2048-element tile into a ring of shared-memory stages with 1-D bulk copies
@@ -176,6 +175,101 @@ __global__ void __launch_bounds__(kTpThreads, 1)
   norm_epilogue<kTpThreads>(a.ns, sq, nf, a.accumulate);
 }
 
+// Pass 1 above 16 ranks: a tile's N slices do not fit a stage, so the
+// producer streams them in chunks of kChunk ranks (32 KB stages) and the
+// consumers add each chunk in rank order -- the same sequence of additions.
+constexpr int kChunk = 8;
+constexpr unsigned kChunkStageBytes = kChunk * 2 * kTile;
+
+template <bool kWriteBack, class F>
+__global__ void __launch_bounds__(kTpThreads, 1)
+    reduce_chunked_tma_kernel(const __grid_constant__ ReduceArgs a, int stages) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const int n_chunks = (N + kChunk - 1) / kChunk;
+  const Ring ring = ring_at(smem, kChunkStageBytes, stages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
+  ring_init(ring, stages);
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      bool stop = false;
+      for (int it = 0; !stop; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *ring.abort_flag) break;
+        const int64_t e0 = tile * kTile;
+        const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+        for (int c = 0; c < n_chunks; ++c) {
+          const int ci = it * n_chunks + c;
+          const int s = ci % stages;
+          const unsigned k = (unsigned)(ci / stages);
+          if (!acquire_stage(ring, s, k, a.ns.error)) {
+            stop = true;
+            break;
+          }
+          const int r0 = c * kChunk;
+          const int r1 = (r0 + kChunk) < N ? (r0 + kChunk) : N;
+          unsigned char* st = smem + (size_t)s * kChunkStageBytes;
+          mbar_expect_tx(&ring.full[s], (unsigned)(cnt * 2 * (r1 - r0)));
+          for (int r = r0; r < r1; ++r)
+            bulk_load(st + (size_t)(r - r0) * 2 * kTile, a.grad[r] + e0, (unsigned)(2 * cnt), &ring.full[s], policy);
+          ring.last_k[s] = (int)k;
+        }
+      }
+    }
+  } else {
+    const int j = (threadIdx.x - 32) * kVec;
+    bool stop = false;
+    for (int it = 0; !stop; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int64_t e0 = tile * kTile;
+      const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
+      const bool active = j < cnt;
+      float acc[kVec];
+#pragma unroll
+      for (int q = 0; q < kVec; ++q) acc[q] = 0.0f;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int ci = it * n_chunks + c;
+        const int s = ci % stages;
+        const unsigned k = (unsigned)(ci / stages);
+        if (!consume_stage(ring, s, k, a.ns.error, lane)) {
+          stop = true;
+          break;
+        }
+        const int r0 = c * kChunk;
+        const int r1 = (r0 + kChunk) < N ? (r0 + kChunk) : N;
+        const unsigned char* st = smem + (size_t)s * kChunkStageBytes;
+        if (active)
+          for (int r = r0; r < r1; ++r)
+            add8<F>(acc, *reinterpret_cast<const uint4*>(st + (size_t)(r - r0) * 2 * kTile + 2 * j));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);
+      }
+      if (stop) break;
+      if (active) {
+        const int64_t e = e0 + j;
+        uint16_t g16[kVec];
+        float g[kVec];
+        mean_bf16<F>(acc, a.inv_n, g16, g, sq, nf);
+        const uint4 gw = pack8(g16);
+        if (kWriteBack) {
+          for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
+        } else {
+          st_out(a.shard_out + e, gw);
+        }
+      }
+    }
+  }
+  ring_drain(ring, stages, a.ns.error);
+  norm_epilogue<kTpThreads>(a.ns, sq, nf, a.accumulate);
+}
+
 // -------------------------------------------------------------- pass 2 --
 
 // gsrc[r] are flat-element-0 pointers; element i's reduced gradient is read
@@ -290,13 +384,28 @@ cudaError_t two_pass_configure() {
   if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<true, Bf16>);
   if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<false, F16>);
   if (e == cudaSuccess) e = opt_in(reduce_tma_kernel<true, F16>);
+  if (e == cudaSuccess) e = opt_in(reduce_chunked_tma_kernel<false, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_chunked_tma_kernel<true, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_chunked_tma_kernel<false, F16>);
+  if (e == cudaSuccess) e = opt_in(reduce_chunked_tma_kernel<true, F16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<Bf16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<F16>);
   return e;
 }
 
 cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s) {
-  if (a.n_ranks < 1 || a.n_ranks > kTmaMaxRanks) return cudaErrorInvalidValue;
+  if (a.n_ranks < 1 || a.n_ranks > kMaxRanks) return cudaErrorInvalidValue;
+  if (a.n_ranks > kTmaMaxRanks) {
+    const size_t bytes = tp_smem_bytes(kChunkStageBytes, kTpStages);
+    if (a.fmt == kFmtF16) {
+      if (a.write_back) reduce_chunked_tma_kernel<true, F16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages);
+      else reduce_chunked_tma_kernel<false, F16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages);
+    } else {
+      if (a.write_back) reduce_chunked_tma_kernel<true, Bf16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages);
+      else reduce_chunked_tma_kernel<false, Bf16><<<grid, kTpThreads, bytes, s>>>(a, kTpStages);
+    }
+    return cudaGetLastError();
+  }
   const int stages = reduce_stages(a.n_ranks);
   const size_t bytes = tp_smem_bytes(reduce_stage_bytes(a.n_ranks), stages);
   if (a.fmt == kFmtF16) {

@@ -594,12 +594,10 @@ zero_status issue_gather(zero_ctx* c, StepOrder& o, zero_gather_fn gfn, void* gu
   return ZERO_OK;
 }
 
-// The two-pass step's kernels: staged through shared memory for N <= 16
-// unless the register path is asked for; timed (ZERO_OPT_TIMING) like the
-// fused launches, with their own byte models.
-bool use_two_pass_tma(const zero_ctx* c) {
-  return c->plan.n_ranks <= zsm::kTmaMaxRanks && c->kernel_opt != ZERO_KERNEL_REGISTER;
-}
+// The two-pass step's kernels (and the unfused reduce calls): staged through
+// shared memory unless the register path is asked for; timed
+// (ZERO_OPT_TIMING) like the fused launches, with their own byte models.
+bool use_two_pass_tma(const zero_ctx* c) { return c->kernel_opt != ZERO_KERNEL_REGISTER; }
 
 int two_pass_grid(const zero_ctx* c, int64_t elems) {
   const int64_t tiles = (elems + zsm::two_pass_tile() - 1) / zsm::two_pass_tile();
