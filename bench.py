@@ -263,33 +263,96 @@ def oracle_stage(stage: int) -> int:
     return {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2, 3: oracle.STAGE_Z3}[stage]
 
 
-def cpu_baseline(w, steps: int = 2, stage: int = 2) -> dict:
-    """The oracle, as it stands (single-threaded), on a bounded sample of the
-    workload: the first transformer layer's tensors (50,358,272 params for the
-    1.2B list), the same N and bucket size, ``steps`` literal steps of the
-    bench's stage."""
+def usable_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+_SLICE_BARRIER = None
+
+
+def _slice_init(barrier):
+    global _SLICE_BARRIER
+    _SLICE_BARRIER = barrier
+
+
+def _oracle_slice(job):
+    """One worker of the parallel oracle timing (a spawned process): literal
+    steps of the oracle on flat elements [a, a + n) of the workload (their
+    values are the workload's: every input is drawn by its flat index), timed
+    after all workers have their inputs."""
     import numpy as np
 
     import oracle
+    import synth
     from synth import workloads as W
 
-    k = w.layer_id.count(0)
-    numel, layer = w.numel[:k], w.layer_id[:k]
-    p = oracle.plan(numel, layer, w.n_ranks, w.bucket_elems)
-    m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
-    grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
-             for r in range(w.n_ranks)]
+    w, stage, a, n, warmup, steps = job
+    p = oracle.plan([n], [0], w.n_ranks, w.bucket_elems or (1 << 40))
+    m0 = np.zeros(p.psi_pad, np.float32)
+    m0[:n] = synth.host_f32(W.master_base(w), a, n, W.MASTER_DIST)
+    grads = []
+    for r in range(w.n_ranks):
+        g = np.zeros(p.psi_pad, np.uint16)
+        g[:n] = synth.host_bf16(W.grad_base(w, 1, r), a, n, w.grad_dist)
+        grads.append(g)
     st = oracle_stage(stage)
     ranks = oracle.init_states(p, st, m0)
     hp = oracle.AdamHP(**w.hyper.__dict__)
-    t0 = time.perf_counter()
-    for t in range(1, steps + 1):
+    t = 0
+    for _ in range(warmup):
+        t += 1
         oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
-    dt = time.perf_counter() - t0
-    return {"value": p.psi * steps / dt, "unit": "params/s", "cores": 1, "kind": "oracle",
-            "sample": f"first layer of the workload ({p.psi} params, N={w.n_ranks}), {steps} literal "
-                      f"ZeRO-{stage} steps, single-threaded C+numpy oracle, input generation untimed",
-            "seconds": dt}
+    if _SLICE_BARRIER is not None:
+        _SLICE_BARRIER.wait()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        t += 1
+        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
+    return n, time.perf_counter() - t0
+
+
+def oracle_parallel(w, stage: int, total: int, warmup: int, steps: int, procs: int):
+    """The oracle as it stands over `total` leading elements, split into
+    `procs` contiguous slices timed in as many spawned processes, released
+    together by a barrier.  Returns (params/s, seconds per step of the
+    slowest slice, elements)."""
+    import multiprocessing as mp
+
+    procs = max(1, min(procs, total // 8))
+    per = max(8, total // procs // 8 * 8)
+    jobs = [(w, stage, k * per, per, warmup, steps) for k in range(procs)]
+    ctx = mp.get_context("spawn")
+    if procs == 1:
+        res = [_oracle_slice(jobs[0])]
+    else:
+        barrier = ctx.Manager().Barrier(procs)
+        with ctx.Pool(procs, initializer=_slice_init, initargs=(barrier,)) as pool:
+            res = pool.map(_oracle_slice, jobs, chunksize=1)
+    elems = sum(n for n, _ in res)
+    worst = max(dt for _, dt in res)
+    return elems * steps / worst, worst / steps, elems
+
+
+def cpu_baseline(w, steps: int = 2, stage: int = 2) -> dict:
+    """The oracle, as it stands, on a bounded sample of the workload: the
+    first transformer layer's elements (50,358,272 params for the 1.2B list),
+    the same N and bucket size, ``steps`` literal steps of the bench's stage
+    -- on one core, and split over every usable core."""
+    k = w.layer_id.count(0)
+    total = int(sum(w.numel[:k])) // 8 * 8
+    one, one_s, _ = oracle_parallel(w, stage, total, 0, steps, 1)
+    cores = usable_cores()
+    allc, all_s, elems = oracle_parallel(w, stage, total, 1, steps, cores)
+    return {"value": allc, "unit": "params/s", "cores": cores, "kind": "oracle",
+            "sample": f"first layer of the workload ({elems} params, N={w.n_ranks}) split into {cores} "
+                      f"contiguous slices, one spawned process per usable core, {steps} literal "
+                      f"ZeRO-{stage} steps each after one warm-up, timed together; C+numpy oracle, "
+                      f"input generation untimed",
+            "single_core": {"value": one, "unit": "params/s", "cores": 1, "seconds_per_step": one_s,
+                            "sample": f"the same {total} params in one process, {steps} steps"}}
 
 
 # -------------------------------------------------------------------- ours ----
@@ -677,59 +740,34 @@ def run_stages(args):
 
 # --------------------------------------------------------------- reference ----
 
-def reference_sample(w, steps_total: int, elems: int = 0):
-    """A contiguous leading slice of the workload's first layer, sized so that
-    ``steps_total`` oracle steps take about a minute (the oracle does ~9M
-    params/s at N = 8 on one core), at least 8192*N elements."""
-    k = w.layer_id.count(0)
-    numel = list(w.numel[:k])
-    budget = elems if elems > 0 else max(8192 * w.n_ranks, int(5e8 / max(1, steps_total)))
-    out, total = [], 0
-    for n in numel:
-        if total >= budget:
-            break
-        take = min(n, budget - total)
-        out.append(take)
-        total += take
-    return out, [0] * len(out)
-
-
 def run_reference(args, world, rank, local):
-    """The CPU oracle timed on this machine's host cores, same metric and unit."""
+    """The CPU oracle timed on this machine's host cores, same metric and unit:
+    each step a bounded sample of the workload (leading elements of its first
+    layer), split over every usable core."""
     if rank != 0:
         return
-    from synth import workloads as W
-
-    import oracle
-
     w = workload()
-    numel, layer = reference_sample(w, args.steps + args.warmup, args.ref_sample_elems)
-    p = oracle.plan(numel, layer, w.n_ranks, w.bucket_elems)
-    m0 = W.host_padded(p.offset, numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
-    grads = [W.host_padded(p.offset, numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist)
-             for r in range(w.n_ranks)]
-    st = oracle_stage(args.stage)
-    ranks = oracle.init_states(p, st, m0)
-    hp = oracle.AdamHP(**w.hyper.__dict__)
-    t = 0
-    for _ in range(args.warmup):
-        t += 1
-        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        t += 1
-        oracle.step(p, st, ranks, lambda t_, r: grads[r], t, hp)
-    dt = time.perf_counter() - t0
-    value = p.psi * args.steps / dt
-    sample = (f"leading {p.psi} params of the first layer of {w.name} (N={w.n_ranks}) per step, "
-              f"literal ZeRO-{args.stage} step of the single-threaded oracle, input generation untimed")
+    procs = usable_cores()
+    k = w.layer_id.count(0)
+    layer_elems = int(sum(w.numel[:k])) // 8 * 8
+    if args.ref_sample_elems > 0:
+        total = args.ref_sample_elems
+    else:  # about a minute of oracle work per core for the whole run
+        per_core = max(8192 * w.n_ranks, int(5e8 / max(1, args.steps + args.warmup)))
+        total = min(layer_elems, procs * per_core)
+    total = max(8, total // 8 * 8)
+    value, s_per_step, elems = oracle_parallel(w, args.stage, total, args.warmup, args.steps, procs)
+    cores = max(1, min(procs, total // 8))
+    sample = (f"leading {elems} params of the first layer of {w.name} (N={w.n_ranks}) per step, split into "
+              f"{cores} contiguous slices in as many spawned processes; literal ZeRO-{args.stage} steps of "
+              f"the C+numpy oracle, input generation untimed")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "params/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic", "config": {"workload": w.name, "params": w.psi, "n_ranks": w.n_ranks,
                                         "stage": args.stage, "bucket_elems": w.bucket_elems},
-        "cpu_baseline": {"value": value, "unit": "params/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "params/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "params/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 

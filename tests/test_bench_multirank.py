@@ -71,4 +71,4 @@ def test_reference_arm_prints_once_on_rank_zero():
     d = json.loads(lines0[0])
     assert d["impl"] == "reference" and d["unit"] == "params/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
-    assert d["cpu_baseline"]["cores"] == 1 and d["n_gpus"] == 2
+    assert d["cpu_baseline"]["cores"] >= 1 and d["n_gpus"] == 2
