@@ -40,8 +40,11 @@ FALLBACK_HBM_GBS = 6650.0
 _CSRC = os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc")
 # the sources each fused kernel is compiled from (kernels.cuh holds only
 # declarations and argument structs)
-KERNEL_SOURCES = {"tma": [os.path.join(_CSRC, f) for f in ("fused_tma.cu", "device_math.cuh")],
-                  "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh")]}
+# the files a fused kernel's device code comes from (its traffic record is
+# void once any of them changes)
+KERNEL_SOURCES = {"tma": [os.path.join(_CSRC, f) for f in ("fused_tma.cu", "tma_pipe.cuh", "device_math.cuh",
+                                                            "kernels.cuh")],
+                  "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh", "kernels.cuh")]}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
 
 
