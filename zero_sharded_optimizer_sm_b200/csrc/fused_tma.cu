@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
 
   double sq = 0.0;
   unsigned long long nf = 0;
+  bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
 
   if (warp < G) {
     // ---------------------------------------------------------- producer --
@@ -145,6 +146,10 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
       if (lane == 0) mbar_arrive(&empty[s]);
       if (active) {
         const int64_t e = e0 + j;
+        if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+          pdl_wait();
+          waited = true;
+        }
         uint16_t g16[kVec];
         float gv[kVec];
         mean_bf16<F>(acc, a.inv_n, g16, gv, sq, nf);
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
     for (int s = 0; s < stages; ++s)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
-  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<tma_threads<G>()>(a.ns, sq, nf, a.accumulate);
 }
 
@@ -223,6 +228,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
   double sq = 0.0;
   unsigned long long nf = 0;
+  bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -283,6 +289,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       if (lane == 0) mbar_arrive(&empty[s]);
       if (active) {
         const int64_t e = e0 + j;
+        if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+          pdl_wait();
+          waited = true;
+        }
         uint16_t g16[4];
         float gv[4];
 #pragma unroll
@@ -315,7 +325,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     for (int s = 0; s < stages; ++s)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
-  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<kWideThreads>(a.ns, sq, nf, a.accumulate);
 }
 
@@ -378,6 +388,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
 
   double sq = 0.0;
   unsigned long long nf = 0;
+  bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer --
@@ -483,6 +494,10 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
       if (lane == 0) mbar_arrive(&sempty[ss]);
       if (active) {
         const int64_t e = e0 + j;
+        if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+          pdl_wait();
+          waited = true;
+        }
         uint16_t g16[kVec];
         float gv[kVec];
         mean_bf16<F>(acc, a.inv_n, g16, gv, sq, nf);
@@ -513,7 +528,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
     for (int s = 0; s < sstages; ++s)
       if (last_sk[s] >= 0 && !mbar_wait(&sfull[s], (unsigned)last_sk[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
-  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<tma_threads<1>()>(a.ns, sq, nf, a.accumulate);
 }
 

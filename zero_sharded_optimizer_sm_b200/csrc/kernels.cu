@@ -31,6 +31,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
   double sq = 0.0;
   unsigned long long nf = 0;
   if (a.pdl == kPdlWaitFirst) pdl_wait();
+  bool waited = false;
   // every CTA is resident from the start (the grid is sized to the SM count),
   // so the next fused launch may be scheduled as soon as CTAs exit
   pdl_trigger();
@@ -45,6 +46,10 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     uint16_t g16[kVec];
     float g[kVec];
     mean_bf16<F>(acc, a.inv_n, g16, g, sq, nf);
+    if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+      pdl_wait();
+      waited = true;
+    }
     if (MODE == kFusedZ1) {
       const uint4 gw = pack8(g16);
       for (int r = 0; r < a.n_ranks; ++r) st_stream(const_cast<uint16_t*>(a.grad[r]) + e, gw);
@@ -62,7 +67,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     if (MODE == kFusedZ3) st_stream(a.param_shard + e, pw);
     for (int r = 0; r < a.n_ranks; ++r) st_stream(a.out[r] + e, pw);
   }
-  if (a.pdl == kPdlEarly) pdl_wait();  // the norm scratch is shared with the grid before
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
   norm_epilogue<kThreads>(a.ns, sq, nf, a.accumulate);
 }
 

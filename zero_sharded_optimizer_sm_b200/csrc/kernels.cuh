@@ -45,7 +45,11 @@ enum StorageFormat { kFmtBf16 = 0, kFmtF16 = 1 };
 //                  predecessor is a fused kernel of the same step on a
 //                  disjoint interval with disjoint destinations, so that the
 //                  two share nothing but the norm scratch.
-enum PdlMode { kPdlNone = 0, kPdlWaitFirst = 1, kPdlEarly = 2 };
+//   kPdlEarlyLoads the kernel loads and computes at once but each thread
+//                  waits before its first store (and before the epilogue):
+//                  for a predecessor on a disjoint interval that writes the
+//                  same destination buffer (stage 3's temporary layer buffer).
+enum PdlMode { kPdlNone = 0, kPdlWaitFirst = 1, kPdlEarly = 2, kPdlEarlyLoads = 3 };
 
 // cudaLaunchKernelEx with the programmatic-serialization attribute when `pdl`.
 template <typename... KArgs, typename... Args>

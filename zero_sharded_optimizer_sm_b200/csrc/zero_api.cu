@@ -775,7 +775,8 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   // follows unknown work and waits for it before touching memory; the later
   // ones at stage 1/2 touch disjoint intervals and share only the norm
   // scratch, so they stream at once; stage 3's launches all write the one
-  // temporary gather buffer, so they wait first.
+  // temporary gather buffer, so they load and compute at once but store only
+  // after the launch before has finished.
   // (and not with two staged CTAs per SM asked for: a programmatic launch
   // keeps one per SM)
   const bool pdl_ok = c->pdl && !callbacks && c->tma_ctas_opt <= 1;
@@ -788,8 +789,9 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
     interval_grads(c, resident, lo, o.slot(k), grad.data());
     o.before_kernel(k, !resident && fn, gathers ? k : (size_t)-1);
     const int pdl = !pdl_ok ? zsm::kPdlNone
-                    : (launched && c->stage != ZERO_STAGE_3) ? zsm::kPdlEarly
-                                                             : zsm::kPdlWaitFirst;
+                    : !launched ? zsm::kPdlWaitFirst
+                    : c->stage != ZERO_STAGE_3 ? zsm::kPdlEarly
+                                               : zsm::kPdlEarlyLoads;
     st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl);
     if (st != ZERO_OK) break;
     launched = launched || hi > lo;
