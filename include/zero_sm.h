@@ -376,11 +376,16 @@ zero_status zero_comm_elems(const zero_ctx* ctx, int64_t out[3]);
  * With either enabled the step needs the norm before any update, so zero_step
  * and zero_step_resident run two passes: every interval is reduced first
  * (stage 2/3 into the reduced-gradient shards, which must be kept; stage 1
- * into the replicas, the all-reduce), the stream is synchronised once to read
- * the norm, and a second kernel runs Adam and the broadcast (per layer at
- * stage 3, with gather_fn as before).  Bytes per element at stage 2:
- * (2N+2) + (2+24+2N) = 4N+28.  max_norm = 0 and skip_nonfinite = 0 (the
- * default) restore the single fused pass.
+ * into the replicas, the all-reduce), a one-thread kernel takes the decision
+ * (norm, skip, coefficient) on the device, and a second kernel runs Adam and
+ * the broadcast (per layer at stage 3, with gather_fn as before) reading that
+ * decision -- no host synchronisation between the passes.  A skipped step
+ * writes no state and broadcasts the unchanged parameters.  The host learns
+ * the decision when it next needs it (the statistics, zero_get_step, the next
+ * step), which advances the step counter only for a step that was not
+ * skipped.  Bytes per element at stage 2: (2N+2) + (2+24+2N) = 4N+28.
+ * max_norm = 0 and skip_nonfinite = 0 (the default) restore the single fused
+ * pass.
  */
 zero_status zero_set_clip(zero_ctx* ctx, double max_norm, int32_t skip_nonfinite);
 

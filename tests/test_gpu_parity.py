@@ -743,6 +743,48 @@ def test_two_pass_staged_kernels_equal_register_kernels(stage):
                 b.close()
 
 
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_clipped_steps_back_to_back_without_statistics(stage):
+    """The clipped step's decision is taken on the device, so steps issued
+    back to back without reading statistics never wait on the host; the state,
+    the step count (a skipped step, call 2, does not advance it) and the last
+    statistics equal those of steps read one at a time."""
+    z = _z()
+    numel, layer = W.transformer_layers(2, 64, 256)
+    n_ranks, bucket = 4, 8192
+    dist = synth.Dist(synth.NORMAL, 1e-2, zero_mod=11)
+    w = W.Workload("clip-async", numel, layer, n_ranks, (stage,), bucket, dist, W.MASTER_DIST, 4,
+                   W.Hyper(weight_decay=0.01), 0xCA + stage)
+    p = oracle.plan(numel, layer, n_ranks, bucket)
+
+    def host_grad(k, r):
+        g = W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, k, r), dist)
+        if k == 2 and r == 1:
+            g[7] = 0x7F80
+        return g
+
+    dev = {k: [torch.from_numpy(host_grad(k, r).view(np.int16)).cuda() for r in range(n_ranks)] for k in range(1, 5)}
+    opts = []
+    for _ in range(2):
+        o, _f = make_opt(w, stage, bucket=bucket)
+        o.set_clip(0.05, True)
+        opts.append(o)
+    a, b = opts
+    for k in range(1, 5):
+        sa = a.step_resident([x.clone() for x in dev[k]], stats=True)
+        b.step_resident([x.clone() for x in dev[k]])           # no statistics: nothing waits
+        if k == 2:
+            assert sa["skipped"] == 1
+    assert b.t == a.t == 3
+    assert b.read_stats() == a.read_stats()
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(a.view(what), b.view(what))
+    for r in range(n_ranks if stage != 3 else 1):
+        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+    a.close()
+    b.close()
+
+
 def test_inactive_clip_two_pass_equals_fused_step():
     z = _z()
     numel, layer = W.transformer_layers(2, 64, 256)

@@ -151,6 +151,27 @@ __device__ __forceinline__ void mean_bf16(const float (&acc)[kVec], float inv_n,
 
 // ------------------------------------------------------------------- Adam --
 
+// The 16-bit rounding of 8 fp32 values (the parameters of unchanged masters).
+template <class F>
+__device__ __forceinline__ uint4 round8(const float4& p0, const float4& p1) {
+  return make_uint4((uint32_t)F::rn(p0.x) | ((uint32_t)F::rn(p0.y) << 16),
+                    (uint32_t)F::rn(p0.z) | ((uint32_t)F::rn(p0.w) << 16),
+                    (uint32_t)F::rn(p1.x) | ((uint32_t)F::rn(p1.y) << 16),
+                    (uint32_t)F::rn(p1.z) | ((uint32_t)F::rn(p1.w) << 16));
+}
+
+// Folds the clipped step's decision into the scalars: the coefficient when
+// below 1; returns whether the step is skipped.  `dec` may be null.
+__device__ __forceinline__ bool apply_decision(const ClipDecision* dec, AdamScalars& sc) {
+  if (!dec) return false;
+  const float coef = dec->coef;
+  if (coef < 1.0f) {
+    sc.coef = coef;
+    sc.flags |= kClip;
+  }
+  return dec->skip != 0;
+}
+
 __device__ __forceinline__ float adam1(float g, float& p, float& m, float& v,
                                        const AdamScalars& s) {
   if (s.flags & kUnscale) g = __fmul_rn(g, s.inv_scale);  // loss scale first,

@@ -119,17 +119,25 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
 template <class F>
 __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_constant__ AdamBcastArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
+  AdamScalars sc = a.sc;
+  const bool skip = apply_decision(a.dec, sc);
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
     const int64_t e = vi * kVec;
     const int64_t i = a.lo + e;  // flat index; the 8 elements share one owner (S % 8 == 0)
     float4 p0 = ld_stream(a.master + e), p1 = ld_stream(a.master + e + 4);
+    if (skip) {  // a skipped step: the unchanged parameters, no state written
+      const uint4 pw = round8<F>(p0, p1);
+      if (a.param_shard) st_stream(a.param_shard + e, pw);
+      for (int r = 0; r < a.n_out; ++r) st_stream(a.out[r] + e, pw);
+      continue;
+    }
     float4 m0 = ld_stream(a.m + e), m1 = ld_stream(a.m + e + 4);
     float4 v0 = ld_stream(a.v + e), v1 = ld_stream(a.v + e + 4);
     const uint4 gw = ld_stream(a.gsrc[i / a.shard] + i);
     float g[kVec] = {F::lo(gw.x), F::hi(gw.x), F::lo(gw.y), F::hi(gw.y),
                      F::lo(gw.z), F::hi(gw.z), F::lo(gw.w), F::hi(gw.w)};
     uint16_t p16[kVec];
-    adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);  // unscale and clip via a.sc.flags
+    adam8<F>(g, p0, p1, m0, m1, v0, v1, sc, p16);  // unscale and clip via sc.flags
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
     st_stream(a.m + e, m0);
@@ -140,6 +148,21 @@ __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_const
     if (a.param_shard) st_stream(a.param_shard + e, pw);
     for (int r = 0; r < a.n_out; ++r) st_stream(a.out[r] + e, pw);
   }
+}
+
+// The clipped step's decision (ClipDecision), one thread, from the step's sums.
+__global__ void clip_decide_kernel(const NormScratch ns, const ClipParams p, ClipDecision* out) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  ClipDecision d;
+  d.nonfinite = *ns.step_nf;
+  d.norm = __ddiv_rn(__dsqrt_rn(*ns.step_sq), p.loss_scale);
+  d.skip = (p.skip_nonfinite && d.nonfinite > 0) ? 1 : 0;
+  d.coef = 1.0f;
+  if (!d.skip && p.max_norm > 0.0) {
+    const float c = __double2float_rn(__ddiv_rn(p.max_norm, __dadd_rn(d.norm, 1e-6)));
+    if (c < 1.0f) d.coef = c;  // false for a NaN norm: no clipping
+  }
+  *out = d;
 }
 
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherArgs a) {
@@ -231,6 +254,11 @@ cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s) {
 cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s) {
   if (a.fmt == kFmtF16) adam_bcast_kernel<F16><<<grid, kThreads, 0, s>>>(a);
   else adam_bcast_kernel<Bf16><<<grid, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, cudaStream_t s) {
+  clip_decide_kernel<<<1, 32, 0, s>>>(ns, p, out);
   return cudaGetLastError();
 }
 

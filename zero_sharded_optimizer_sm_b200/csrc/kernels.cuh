@@ -126,6 +126,24 @@ struct AdamArgs {
 // or overflow-checked step).  The gradient of flat element i comes from
 // gsrc[i / shard] + i (the owner's copy); every pointer but gsrc is at flat
 // element `lo`.
+// The clipped step's decision, taken on the device between the two passes
+// from the step's gradient sums: norm = sqrt(sum of squares) / loss scale,
+// skip when the overflow skip is on and a value is not finite, and the
+// clipping coefficient fp32(max_norm / (norm + 1e-6)) (binary64 quotient),
+// applied when below 1 -- the host's formula, the same binary64 operations.
+struct ClipDecision {
+  double norm;
+  unsigned long long nonfinite;
+  float coef;    // 1 when no clipping applies
+  int skip;
+};
+
+struct ClipParams {
+  double max_norm;     // 0: no clipping
+  double loss_scale;
+  int skip_nonfinite;
+};
+
 struct AdamBcastArgs {
   int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* gsrc[kMaxRanks];
@@ -138,7 +156,8 @@ struct AdamBcastArgs {
   int64_t shard;
   int64_t n_vec;
   int n_out;
-  AdamScalars sc;                   // including the unscale / clip factors
+  AdamScalars sc;                   // including the unscale factor
+  const ClipDecision* dec;          // the step's decision (clip coefficient, skip), or nullptr
   unsigned int* error;              // staged kernel: set when a bounded wait runs out
 };
 
@@ -173,6 +192,7 @@ cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s);
+cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with

@@ -280,6 +280,8 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     adam_bcast_tma_kernel(const __grid_constant__ AdamBcastArgs a, int stages, int uniform) {
   extern __shared__ __align__(128) unsigned char smem[];
   const Ring ring = ring_at(smem, kBcastStageBytes, stages);
+  AdamScalars sc = a.sc;
+  const bool skip = apply_decision(a.dec, sc);  // a skipped step writes the unchanged parameters only
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_elem = a.n_vec * kVec;
   const int64_t n_tiles = (n_elem + kTile - 1) / kTile;
@@ -344,12 +346,17 @@ __global__ void __launch_bounds__(kTpThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ring.empty[s]);
-      if (active) {
+      if (active && skip) {
+        const int64_t e = e0 + j;
+        const uint4 pw = round8<F>(p0, p1);
+        if (a.param_shard) st_out(a.param_shard + e, pw);
+        for (int r = 0; r < a.n_out; ++r) st_out(a.out[r] + e, pw);
+      } else if (active) {
         const int64_t e = e0 + j;
         float g[kVec] = {F::lo(gw.x), F::hi(gw.x), F::lo(gw.y), F::hi(gw.y),
                          F::lo(gw.z), F::hi(gw.z), F::lo(gw.w), F::hi(gw.w)};
         uint16_t p16[kVec];
-        adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);  // loss-scale and clip factors via a.sc.flags
+        adam8<F>(g, p0, p1, m0, m1, v0, v1, sc, p16);  // loss-scale and clip factors via sc.flags
         st_out(a.master + e, p0);
         st_out(a.master + e + 4, p1);
         st_out(a.m + e, m0);

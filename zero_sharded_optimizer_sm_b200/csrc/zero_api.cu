@@ -24,6 +24,8 @@ thread_local std::string g_init_error;
 
 constexpr int64_t kArenaAlign = 256;
 constexpr int64_t kScratchBytes = 80 * 1024;
+static_assert(16 * zsm::kMaxGrid + 64 + sizeof(zsm::ClipDecision) <= kScratchBytes,
+              "the scratch arena holds the norm partials, the step sums and the clip decision");
 
 int64_t align_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
 
@@ -79,6 +81,12 @@ struct zero_ctx {
   cudaStream_t kside = nullptr;  // the kernels' stream at the greatest priority (ZERO_OPT_PIPELINE = 2)
   bool own_side = false, own_kside = false;  // created here (destroyed with the context)
   bool pipeline_used = false;
+  // the clipped step's decision: device copy in the scratch arena, host copy
+  // in pinned memory, resolved into t and the statistics when next needed
+  bool pending = false;
+  int64_t pending_t = 0;
+  cudaEvent_t ev_decision = nullptr;
+  zsm::ClipDecision* host_dec = nullptr;
   cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_kjoin = nullptr;
   cudaEvent_t ev_grads[2] = {}, ev_kernel[2] = {}, ev_consumed[2] = {};
   // fused-kernel timing
@@ -92,6 +100,8 @@ struct zero_ctx {
     for (cudaEvent_t e : {ev_start, ev_join, ev_kjoin, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
                           ev_consumed[0], ev_consumed[1]})
       if (e) cudaEventDestroy(e);
+    if (ev_decision) cudaEventDestroy(ev_decision);
+    if (host_dec) cudaFreeHost(host_dec);
     if (side && own_side) cudaStreamDestroy(side);
     if (kside && own_kside) cudaStreamDestroy(kside);
   }
@@ -180,6 +190,34 @@ zsm::NormScratch norm_scratch(zero_ctx* c) {
   ns.done = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 16);
   ns.error = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 20);
   return ns;
+}
+
+// The clipped step's decision in the scratch arena (after the norm sums).
+zsm::ClipDecision* decision_ptr(zero_ctx* c) {
+  return reinterpret_cast<zsm::ClipDecision*>(c->arena[ZERO_ARENA_SCRATCH] + 16 * zsm::kMaxGrid + 64);
+}
+
+zero_status ensure_decision(zero_ctx* c) {
+  cudaError_t e = cudaSuccess;
+  if (!c->ev_decision) e = cudaEventCreateWithFlags(&c->ev_decision, cudaEventDisableTiming);
+  if (e == cudaSuccess && !c->host_dec) e = cudaMallocHost(&c->host_dec, sizeof(zsm::ClipDecision));
+  if (e != cudaSuccess) return cuda_fail(c, e, "creating the decision event and pinned host copy");
+  return ZERO_OK;
+}
+
+// Folds a clipped step's decision, once it has reached the host, into the
+// step counter (advanced unless the step was skipped) and the statistics.
+zero_status resolve_decision(zero_ctx* c) {
+  if (!c->pending) return ZERO_OK;
+  c->pending = false;
+  const cudaError_t e = cudaEventSynchronize(c->ev_decision);
+  if (e != cudaSuccess) return cuda_fail(c, e, "waiting for the clipped step's decision");
+  const zsm::ClipDecision d = *c->host_dec;
+  c->last_skipped = d.skip ? 1 : 0;
+  c->last_coef = d.coef < 1.0f ? (double)d.coef : 1.0;
+  if (!d.skip) c->t = c->pending_t;
+  c->stats_step = c->t;
+  return ZERO_OK;
 }
 
 zsm::AdamScalars adam_scalars(const zero_adam_hparams& hp, int64_t t);
@@ -416,6 +454,7 @@ zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(c, e, "reading step statistics");
   zero_status st = check_device_error(c, host.error, s);
+  if (st == ZERO_OK) st = resolve_decision(c);
   if (st != ZERO_OK) return st;
   std::memset(out, 0, sizeof *out);
   out->grad_norm = std::sqrt(host.sq) / c->loss_scale;
@@ -424,24 +463,6 @@ zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
   zero_comm_elems(c, out->comm_elems);
   out->clip_coef = c->last_coef;
   out->skipped = c->last_skipped;
-  return ZERO_OK;
-}
-
-// Reads the step accumulator (norm, non-finite count); synchronises `s`.
-zero_status read_norm(zero_ctx* c, cudaStream_t s, double* sq, unsigned long long* nf) {
-  struct {
-    double sq;
-    unsigned long long nf;
-    unsigned int done;
-    unsigned int error;
-  } host{};
-  cudaError_t e = cudaMemcpyAsync(&host, norm_scratch(c).step_sq, sizeof host, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(c, e, "reading the gradient norm");
-  zero_status st = check_device_error(c, host.error, s);
-  if (st != ZERO_OK) return st;
-  *sq = host.sq;
-  *nf = host.nf;
   return ZERO_OK;
 }
 
@@ -674,62 +695,65 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     o.after_kernel(k);
   }
   if (o.err != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
-  double sq = 0.0;
-  unsigned long long nf = 0;
-  zero_status st = read_norm(c, s, &sq, &nf);
+  // The decision -- norm, skip, clipping coefficient -- is taken on the device
+  // from the sums pass 1 left and read there by pass 2, so nothing waits
+  // between the passes; the host learns it later (resolve_decision).
+  zero_status st = ensure_decision(c);
   if (st != ZERO_OK) return st;
-  const double norm = std::sqrt(sq) / c->loss_scale;  // of the unscaled gradient
-  c->last_skipped = (c->skip_nonfinite && nf > 0) ? 1 : 0;
-  c->last_coef = 1.0;
-  if (!c->last_skipped) {
-    float coef = 1.0f;
-    if (c->clip_norm > 0.0) coef = (float)(c->clip_norm / (norm + 1e-6));
-    const bool apply = coef < 1.0f;
-    c->last_coef = apply ? (double)coef : 1.0;
-    const zsm::AdamScalars sc = step_scalars(c, t, apply ? coef : 1.0f);
-    // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3)
-    std::vector<zsm::Span> p2;
-    if (c->stage == ZERO_STAGE_3) p2 = iv;
-    else p2.push_back({0, c->plan.psi_pad});
-    for (size_t k = 0; k < p2.size(); ++k) {
-      const int64_t lo = p2[k].lo, hi = p2[k].hi;
-      const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
-      zsm::AdamBcastArgs b;
-      std::memset(&b, 0, sizeof b);
-      b.fmt = c->fmt;
-      for (int r = 0; r < N; ++r) {
-        if (c->stage == ZERO_STAGE_1)
-          b.gsrc[r] = resident ? static_cast<const uint16_t*>(resident[r]) : grad_buf_ptr(c, r);
-        else
-          b.gsrc[r] = grad_shard_ptr(c);
-        b.out[r] = c->stage == ZERO_STAGE_3 ? gather_ptr(c, r, o.slot(k)) : param_ptr(c, r) + lo;
-      }
-      b.n_out = N;
-      b.master = master_ptr(c) + lo;
-      b.m = m_ptr(c) + lo;
-      b.v = v_ptr(c) + lo;
-      b.param_shard = c->stage == ZERO_STAGE_3 ? param_ptr(c, 0) + lo : nullptr;
-      b.lo = lo;
-      b.shard = c->plan.shard;
-      b.n_vec = (hi - lo) / zsm::kVec;
-      b.sc = sc;
-      b.error = norm_scratch(c).error;
-      o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
-      if (b.n_vec > 0) {
-        // stages 2 and 3 read every owner's reduced gradient from the one shard array
-        cudaError_t e = launch_pass2(c, b, c->stage != ZERO_STAGE_1, s);
-        if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
-      }
-      o.after_kernel(k);
-      if (c->stage == ZERO_STAGE_3 && gfn) {
-        st = issue_gather(c, o, gfn, guser, layer_idx, k);
-        if (st != ZERO_OK) return st;
-      }
+  zsm::ClipParams cp;
+  cp.max_norm = c->clip_norm;
+  cp.loss_scale = c->loss_scale;
+  cp.skip_nonfinite = c->skip_nonfinite ? 1 : 0;
+  zsm::ClipDecision* dec = decision_ptr(c);
+  cudaError_t e = zsm::launch_clip_decide(norm_scratch(c), cp, dec, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(c->host_dec, dec, sizeof *dec, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaEventRecord(c->ev_decision, s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "the clipped step's decision");
+  c->pending = true;
+  c->pending_t = t;
+  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);  // the coefficient comes from the decision
+  // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3);
+  // a skipped step writes the unchanged parameters only
+  std::vector<zsm::Span> p2;
+  if (c->stage == ZERO_STAGE_3) p2 = iv;
+  else p2.push_back({0, c->plan.psi_pad});
+  for (size_t k = 0; k < p2.size(); ++k) {
+    const int64_t lo = p2[k].lo, hi = p2[k].hi;
+    const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
+    zsm::AdamBcastArgs b;
+    std::memset(&b, 0, sizeof b);
+    b.fmt = c->fmt;
+    for (int r = 0; r < N; ++r) {
+      if (c->stage == ZERO_STAGE_1)
+        b.gsrc[r] = resident ? static_cast<const uint16_t*>(resident[r]) : grad_buf_ptr(c, r);
+      else
+        b.gsrc[r] = grad_shard_ptr(c);
+      b.out[r] = c->stage == ZERO_STAGE_3 ? gather_ptr(c, r, o.slot(k)) : param_ptr(c, r) + lo;
     }
-    c->t = t;
+    b.n_out = N;
+    b.master = master_ptr(c) + lo;
+    b.m = m_ptr(c) + lo;
+    b.v = v_ptr(c) + lo;
+    b.param_shard = c->stage == ZERO_STAGE_3 ? param_ptr(c, 0) + lo : nullptr;
+    b.lo = lo;
+    b.shard = c->plan.shard;
+    b.n_vec = (hi - lo) / zsm::kVec;
+    b.sc = sc;
+    b.dec = dec;
+    b.error = norm_scratch(c).error;
+    o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
+    if (b.n_vec > 0) {
+      // stages 2 and 3 read every owner's reduced gradient from the one shard array
+      e = launch_pass2(c, b, c->stage != ZERO_STAGE_1, s);
+      if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
+    }
+    o.after_kernel(k);
+    if (c->stage == ZERO_STAGE_3 && gfn) {
+      st = issue_gather(c, o, gfn, guser, layer_idx, k);
+      if (st != ZERO_OK) return st;
+    }
   }
   if (o.end() != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
-  c->stats_step = c->t;
   c->norm_fresh = true;
   if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
@@ -738,6 +762,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
 zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
                      zero_gather_fn gfn, void* guser, void* stream, zero_step_stats* stats) {
   zero_status st = check_ready(c, true);
+  if (st == ZERO_OK) st = resolve_decision(c);  // t after the last clipped step
   if (st != ZERO_OK) return st;
   const int N = c->plan.n_ranks;
   if (resident) {
@@ -997,6 +1022,8 @@ namespace {
 // Fills the state from sources (see InitArgs) and resets the run state.
 zero_status load_state(zero_ctx* c, const float* master, const float* m, const float* v, int64_t n,
                        int64_t t, cudaStream_t s) {
+  const zero_status st = resolve_decision(c);  // a pending decision must not overwrite the new t
+  if (st != ZERO_OK) return st;
   cudaError_t e = cudaMemsetAsync(c->arena[ZERO_ARENA_SCRATCH], 0, kScratchBytes, s);
   if (e != cudaSuccess) return cuda_fail(c, e, "clearing scratch");
   zsm::InitArgs a;
@@ -1046,14 +1073,19 @@ zero_status zero_import_state(zero_ctx* c, const float* master, const float* exp
   return load_state(c, master, exp_avg, exp_avg_sq, n, t, static_cast<cudaStream_t>(stream));
 }
 
-zero_status zero_get_step(const zero_ctx* c, int64_t* t) {
+zero_status zero_get_step(const zero_ctx* cc, int64_t* t) {
+  zero_ctx* c = const_cast<zero_ctx*>(cc);
   if (!c || !t) return ZERO_EINVAL;
+  const zero_status st = resolve_decision(c);
+  if (st != ZERO_OK) return st;
   *t = c->t;
   return ZERO_OK;
 }
 
 zero_status zero_set_step(zero_ctx* c, int64_t t) {
   if (!c || t < 0) return ZERO_EINVAL;
+  const zero_status st = resolve_decision(c);
+  if (st != ZERO_OK) return st;
   c->t = t;
   return ZERO_OK;
 }
