@@ -113,7 +113,7 @@ typedef struct zero_sizes {
 typedef struct zero_step_stats {
   double grad_norm;        /* sqrt(sum of squares of the averaged bf16 gradient), fp64 */
   int64_t nonfinite;       /* averaged gradient elements that are Inf or NaN */
-  int64_t step;            /* Adam step number t the statistics belong to */
+  int64_t step;            /* the step counter after the step (unchanged by a skipped step) */
   int64_t comm_elems[3];   /* logical elements each rank sends per step: all-reduce,
                               reduce-scatter, all-gather (ring convention) */
   double clip_coef;        /* gradient scale the update used (1 = none; zero_set_clip) */
@@ -230,11 +230,15 @@ typedef struct zero_ctx zero_ctx;
  * finishes).  Called once per interval of the schedule, in schedule order,
  * before that interval is reduced.  It must fill, for every rank r, the
  * hi - lo bf16 values of flat elements [lo, hi) at rank_bufs[r] (device
- * pointers into the GRADS arena) with work enqueued on `stream`.  Returns 0
- * on success; any other value aborts the step with ZERO_EINVAL.  With
- * ZERO_OPT_PIPELINE, `stream` is the context's own stream (not the one given
- * to zero_step), the call for interval k+1 comes before the step's kernel of
- * interval k has run, and consecutive intervals get alternating buffers.
+ * pointers into the GRADS arena) with work enqueued on `stream`.  `step` is
+ * the number of this step call since the step counter was last set (loaded,
+ * imported or zero_set_step): the counter + 1, unless an earlier clipped step
+ * was skipped.  Returns 0 on success; any other value aborts the step with
+ * ZERO_EINVAL (intervals already updated stay updated; the step counter does
+ * not advance).  With ZERO_OPT_PIPELINE, `stream` is the context's own stream
+ * (not the one given to zero_step), the call for interval k+1 comes before
+ * the step's kernel of interval k has run, and consecutive intervals get
+ * alternating buffers.
  */
 typedef int (*zero_grad_fn)(void* user, int64_t step, int64_t lo, int64_t hi,
                             void* const* rank_bufs, void* stream);
@@ -342,7 +346,15 @@ zero_status zero_load_master(zero_ctx* ctx, const float* master_dev, void* strea
 zero_status zero_import_state(zero_ctx* ctx, const float* master, const float* exp_avg,
                               const float* exp_avg_sq, int64_t n, int64_t t, void* stream);
 
-/* Step counter: the t of the last update (0 after zero_load_master). */
+/*
+ * Step counter: the t of the last update (0 after zero_load_master).  The
+ * device holds it, with the bias-correction powers beta^t (t successive
+ * binary64 products), and each step's first kernel forms that step's scalars
+ * from it -- so a step enqueues nothing but kernels and a step captured in a
+ * CUDA graph advances it on every replay.  Both calls wait for the device
+ * once the state is loaded.  Changing the betas (zero_set_hparams) rebuilds
+ * the powers for the current t.
+ */
 zero_status zero_get_step(const zero_ctx* ctx, int64_t* t);
 zero_status zero_set_step(zero_ctx* ctx, int64_t t);
 
@@ -462,6 +474,11 @@ zero_status zero_all_gather(zero_ctx* ctx, int64_t lo, int64_t hi, void* const* 
  * grad_fn may be NULL for stage 1 only (the replicas are already filled).
  * stats (may be NULL): when given, the call synchronises `stream` and fills
  * it; otherwise nothing synchronises (zero_read_stats reads it later).
+ * The step's scalars come from the device step counter (zero_get_step), so
+ * with stats = NULL and ZERO_OPT_TIMING off a step enqueues only kernels and
+ * may be captured in a CUDA graph on `stream` and replayed (each replay is
+ * one more step; the callbacks run at capture time only, so a captured step
+ * replays the work they enqueued then).
  */
 zero_status zero_step(zero_ctx* ctx, zero_grad_fn grad_fn, void* grad_user,
                       zero_gather_fn gather_fn, void* gather_user, void* stream,

@@ -785,6 +785,47 @@ def test_clipped_steps_back_to_back_without_statistics(stage):
     b.close()
 
 
+@pytest.mark.parametrize("stage", [2, 3])
+@pytest.mark.parametrize("clip", [False, True])
+def test_resident_step_captured_in_a_cuda_graph(stage, clip):
+    """A step enqueues only kernels (its scalars come from the device step
+    counter), so it can be captured once in a CUDA graph and replayed: four
+    replays equal four eager steps bit for bit -- the fused step and the
+    clipped two-pass step -- and the device step counter advances with each."""
+    z = _z()
+    numel, layer = W.transformer_layers(3, 64, 256)
+    w = W.Workload("graph", numel, layer, 4, (stage,), 16384, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 1,
+                   W.Hyper(weight_decay=0.01), 0xD7 + stage)
+    p = oracle.plan(numel, layer, 4, 16384)
+    host = [W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, 1, r), w.grad_dist) for r in range(4)]
+    a, _ = make_opt(w, stage, bucket=16384)
+    b, _ = make_opt(w, stage, bucket=16384)
+    if clip:
+        a.set_clip(0.05, True)
+        b.set_clip(0.05, True)
+    ga = [torch.from_numpy(h.view(np.int16)).cuda() for h in host]
+    gb = [x.clone() for x in ga]
+    torch.cuda.synchronize()
+    for _ in range(4):
+        a.step_resident(ga)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        b.step_resident(gb)
+    assert b.t == 0  # capturing runs nothing
+    for _ in range(4):
+        g.replay()
+    torch.cuda.synchronize()
+    assert a.t == b.t == 4
+    assert a.read_stats() == b.read_stats()
+    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+        assert torch.equal(a.view(what), b.view(what))
+    for r in range(4 if stage != 3 else 1):
+        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+    del g
+    a.close()
+    b.close()
+
+
 def test_inactive_clip_two_pass_equals_fused_step():
     z = _z()
     numel, layer = W.transformer_layers(2, 64, 256)

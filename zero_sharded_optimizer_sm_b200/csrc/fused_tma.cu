@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
   double sq = 0.0;
   unsigned long long nf = 0;
   bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp < G) {
     // ---------------------------------------------------------- producer --
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         }
         if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
-        adam8<F>(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        adam8<F>(gv, p0, p1, m0, m1, v0, v1, sc, p16);
         st_out(a.master + e, p0);
         st_out(a.master + e + 4, p1);
         st_out(a.m + e, m0);
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   double sq = 0.0;
   unsigned long long nf = 0;
   bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -307,10 +309,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (MODE == kFusedZ1)
           for (int r = 0; r < N; ++r) st_out(const_cast<uint16_t*>(a.grad[r]) + e, gw);
         if (a.grad_shard) st_out(a.grad_shard + e, gw);
-        const uint16_t h0 = F::rn(adam1(gv[0], p.x, m.x, v.x, a.sc));
-        const uint16_t h1 = F::rn(adam1(gv[1], p.y, m.y, v.y, a.sc));
-        const uint16_t h2 = F::rn(adam1(gv[2], p.z, m.z, v.z, a.sc));
-        const uint16_t h3 = F::rn(adam1(gv[3], p.w, m.w, v.w, a.sc));
+        const uint16_t h0 = F::rn(adam1(gv[0], p.x, m.x, v.x, sc));
+        const uint16_t h1 = F::rn(adam1(gv[1], p.y, m.y, v.y, sc));
+        const uint16_t h2 = F::rn(adam1(gv[2], p.z, m.z, v.z, sc));
+        const uint16_t h3 = F::rn(adam1(gv[3], p.w, m.w, v.w, sc));
         st_out(a.master + e, p);
         st_out(a.m + e, m);
         st_out(a.v + e, v);
@@ -389,6 +391,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
   double sq = 0.0;
   unsigned long long nf = 0;
   bool waited = false;  // this thread has waited for the grid before (kPdlEarlyLoads)
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer --
@@ -507,7 +510,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         }
         if (a.grad_shard) st_out(a.grad_shard + e, pack8(g16));
         uint16_t p16[kVec];
-        adam8<F>(gv, p0, p1, m0, m1, v0, v1, a.sc, p16);
+        adam8<F>(gv, p0, p1, m0, m1, v0, v1, sc, p16);
         st_out(a.master + e, p0);
         st_out(a.master + e + 4, p1);
         st_out(a.m + e, m0);

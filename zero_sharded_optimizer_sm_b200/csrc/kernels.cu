@@ -30,7 +30,8 @@ template <int MODE, bool kMulti, class F>
 __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_constant__ FusedArgs a) {
   double sq = 0.0;
   unsigned long long nf = 0;
-  if (a.pdl == kPdlWaitFirst) pdl_wait();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();  // before any global access, the step's scalars included
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
   bool waited = false;
   // every CTA is resident from the start (the grid is sized to the SM count),
   // so the next fused launch may be scheduled as soon as CTAs exit
@@ -56,7 +57,7 @@ __global__ void __launch_bounds__(kThreads) fused_step_kernel(const __grid_const
     }
     if (a.grad_shard) st_stream(a.grad_shard + e, pack8(g16));
     uint16_t p16[kVec];
-    adam8<F>(g, p0, p1, m0, m1, v0, v1, a.sc, p16);
+    adam8<F>(g, p0, p1, m0, m1, v0, v1, sc, p16);
     st_stream(a.master + e, p0);
     st_stream(a.master + e + 4, p1);
     st_stream(a.m + e, m0);
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) adam_kernel(const __grid_constant__ 
 template <class F>
 __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_constant__ AdamBcastArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  AdamScalars sc = a.sc;
+  AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
   const bool skip = apply_decision(a.dec, sc);
   for (int64_t vi = (int64_t)blockIdx.x * kThreads + threadIdx.x; vi < a.n_vec; vi += stride) {
     const int64_t e = vi * kVec;
@@ -150,8 +151,47 @@ __global__ void __launch_bounds__(kThreads) adam_bcast_kernel(const __grid_const
   }
 }
 
-// The clipped step's decision (ClipDecision), one thread, from the step's sums.
-__global__ void clip_decide_kernel(const NormScratch ns, const ClipParams p, ClipDecision* out) {
+// A step's first kernel, one thread: the powers beta^(t+1) as one more
+// binary64 product each, and the step's binary32 scalars from them -- each
+// derived scalar rounded once from binary64, as the host computes them.
+__global__ void step_begin_kernel(StepState* st, const StepHparams hp, ClipDecision* dec) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  const double q1 = __dmul_rn(st->p1, hp.beta1);
+  const double q2 = __dmul_rn(st->p2, hp.beta2);
+  AdamScalars s;
+  s.b1 = __double2float_rn(hp.beta1);
+  s.b2 = __double2float_rn(hp.beta2);
+  s.omb1 = __double2float_rn(__dsub_rn(1.0, hp.beta1));
+  s.omb2 = __double2float_rn(__dsub_rn(1.0, hp.beta2));
+  s.bc1 = __double2float_rn(__dsub_rn(1.0, q1));
+  s.bc2 = __double2float_rn(__dsub_rn(1.0, q2));
+  s.decay = __double2float_rn(__dsub_rn(1.0, __dmul_rn(hp.lr, hp.weight_decay)));
+  s.lr = __double2float_rn(hp.lr);
+  s.eps = __double2float_rn(hp.eps);
+  s.inv_scale = __double2float_rn(__ddiv_rn(1.0, hp.loss_scale));
+  s.coef = 1.0f;
+  s.flags = s.inv_scale != 1.0f ? kUnscale : 0;
+  st->sc = s;
+  st->t_next = st->t + 1;
+  st->p1_next = q1;
+  st->p2_next = q2;
+  if (dec) {
+    dec->coef = 1.0f;
+    dec->skip = 0;
+  }
+}
+
+// A completed (fused) step: t and the powers advance.
+__global__ void step_commit_kernel(StepState* st) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  st->t = st->t_next;
+  st->p1 = st->p1_next;
+  st->p2 = st->p2_next;
+}
+
+// The clipped step's decision (ClipDecision), one thread, from the step's
+// sums; commits the step state unless the step is skipped.
+__global__ void clip_decide_kernel(const NormScratch ns, const ClipParams p, ClipDecision* out, StepState* st) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   ClipDecision d;
   d.nonfinite = *ns.step_nf;
@@ -163,6 +203,11 @@ __global__ void clip_decide_kernel(const NormScratch ns, const ClipParams p, Cli
     if (c < 1.0f) d.coef = c;  // false for a NaN norm: no clipping
   }
   *out = d;
+  if (!d.skip) {
+    st->t = st->t_next;
+    st->p1 = st->p1_next;
+    st->p2 = st->p2_next;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherArgs a) {
@@ -257,8 +302,19 @@ cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s) 
   return cudaGetLastError();
 }
 
-cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, cudaStream_t s) {
-  clip_decide_kernel<<<1, 32, 0, s>>>(ns, p, out);
+cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, StepState* state,
+                               cudaStream_t s) {
+  clip_decide_kernel<<<1, 32, 0, s>>>(ns, p, out, state);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_step_begin(StepState* state, const StepHparams& hp, ClipDecision* dec, cudaStream_t s) {
+  step_begin_kernel<<<1, 32, 0, s>>>(state, hp, dec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_step_commit(StepState* state, cudaStream_t s) {
+  step_commit_kernel<<<1, 32, 0, s>>>(state);
   return cudaGetLastError();
 }
 

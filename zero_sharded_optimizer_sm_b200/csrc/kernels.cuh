@@ -95,6 +95,7 @@ struct FusedArgs {
   float inv_n;                      // binary32 1/N
   int pdl;                          // PdlMode of this launch
   AdamScalars sc;
+  const AdamScalars* sc_dev;        // when set, the scalars are read here instead (StepState::sc)
   NormScratch ns;
 };
 
@@ -144,6 +145,25 @@ struct ClipParams {
   int skip_nonfinite;
 };
 
+// The optimizer's step state on the device: t and beta1^t, beta2^t as t
+// successive binary64 products (the host's definition of the bias-correction
+// powers, so the same bits), and the binary32 scalars of the step being run.
+// A step's first kernel forms the scalars for t + 1; the update kernels read
+// them here, so a step enqueues nothing but kernels and can be captured in a
+// CUDA graph and replayed.
+struct StepState {
+  long long t;        // completed steps
+  double p1, p2;      // beta1^t, beta2^t
+  long long t_next;   // the step being run (committed when it completes unskipped)
+  double p1_next, p2_next;
+  AdamScalars sc;     // its scalars
+};
+
+// Hyper-parameters as the user gave them (binary64) and the loss scale.
+struct StepHparams {
+  double lr, beta1, beta2, eps, weight_decay, loss_scale;
+};
+
 struct AdamBcastArgs {
   int fmt;                          // StorageFormat of every 16-bit buffer
   const uint16_t* gsrc[kMaxRanks];
@@ -157,6 +177,7 @@ struct AdamBcastArgs {
   int64_t n_vec;
   int n_out;
   AdamScalars sc;                   // including the unscale factor
+  const AdamScalars* sc_dev;        // when set, the scalars are read here instead (StepState::sc)
   const ClipDecision* dec;          // the step's decision (clip coefficient, skip), or nullptr
   unsigned int* error;              // staged kernel: set when a bounded wait runs out
 };
@@ -192,7 +213,15 @@ cudaError_t launch_reduce(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam(const AdamArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_gather(const GatherArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam_bcast(const AdamBcastArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, cudaStream_t s);
+// The clipped step's decision; commits the step state's t_next when the step
+// is not skipped.
+cudaError_t launch_clip_decide(const NormScratch& ns, const ClipParams& p, ClipDecision* out, StepState* state,
+                               cudaStream_t s);
+// A step's first kernel: the scalars of step t + 1 into state->sc (t and the
+// powers advance when the step completes: step_commit, or the clipped step's
+// decision); `dec`, when given, is reset to "no clipping, not skipped".
+cudaError_t launch_step_begin(StepState* state, const StepHparams& hp, ClipDecision* dec, cudaStream_t s);
+cudaError_t launch_step_commit(StepState* state, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with

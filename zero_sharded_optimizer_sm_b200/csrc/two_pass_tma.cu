@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     adam_bcast_tma_kernel(const __grid_constant__ AdamBcastArgs a, int stages, int uniform) {
   extern __shared__ __align__(128) unsigned char smem[];
   const Ring ring = ring_at(smem, kBcastStageBytes, stages);
-  AdamScalars sc = a.sc;
+  AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
   const bool skip = apply_decision(a.dec, sc);  // a skipped step writes the unchanged parameters only
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t n_elem = a.n_vec * kVec;

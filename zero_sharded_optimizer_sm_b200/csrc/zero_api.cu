@@ -24,8 +24,8 @@ thread_local std::string g_init_error;
 
 constexpr int64_t kArenaAlign = 256;
 constexpr int64_t kScratchBytes = 80 * 1024;
-static_assert(16 * zsm::kMaxGrid + 64 + sizeof(zsm::ClipDecision) <= kScratchBytes,
-              "the scratch arena holds the norm partials, the step sums and the clip decision");
+static_assert(16 * zsm::kMaxGrid + 128 + sizeof(zsm::StepState) <= kScratchBytes,
+              "the scratch arena holds the norm partials, the step sums, the clip decision and the step state");
 
 int64_t align_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
 
@@ -61,14 +61,12 @@ struct zero_ctx {
   bool have_hp = false;
   zero_adam_hparams hp{};
   bool loaded = false;
-  int64_t t = 0;
-  int64_t stats_step = 0;
+  int64_t t = 0;      // the step counter as the host last learnt it (the device holds it)
+  int64_t calls = 0;  // step calls since the counter was last set: the callbacks' step number
   int fmt = zsm::kFmtBf16;     // storage format of gradients and parameters
   double loss_scale = 1.0;     // the gradients the ranks hold are loss_scale x the true ones
   double clip_norm = 0.0;      // > 0: global-norm clipping
   bool skip_nonfinite = false;
-  double last_coef = 1.0;      // statistics of the last two-pass step
-  int64_t last_skipped = 0;
   bool norm_fresh = true;  // next norm-producing launch starts a new step's sum
   // callback pipeline (ZERO_OPT_PIPELINE): side stream and ordering events
   int pipeline = 0;  // ZERO_OPT_PIPELINE: 0, 1 or 2
@@ -81,12 +79,7 @@ struct zero_ctx {
   cudaStream_t kside = nullptr;  // the kernels' stream at the greatest priority (ZERO_OPT_PIPELINE = 2)
   bool own_side = false, own_kside = false;  // created here (destroyed with the context)
   bool pipeline_used = false;
-  // the clipped step's decision: device copy in the scratch arena, host copy
-  // in pinned memory, resolved into t and the statistics when next needed
-  bool pending = false;
-  int64_t pending_t = 0;
-  cudaEvent_t ev_decision = nullptr;
-  zsm::ClipDecision* host_dec = nullptr;
+
   cudaEvent_t ev_start = nullptr, ev_join = nullptr, ev_kjoin = nullptr;
   cudaEvent_t ev_grads[2] = {}, ev_kernel[2] = {}, ev_consumed[2] = {};
   // fused-kernel timing
@@ -100,8 +93,6 @@ struct zero_ctx {
     for (cudaEvent_t e : {ev_start, ev_join, ev_kjoin, ev_grads[0], ev_grads[1], ev_kernel[0], ev_kernel[1],
                           ev_consumed[0], ev_consumed[1]})
       if (e) cudaEventDestroy(e);
-    if (ev_decision) cudaEventDestroy(ev_decision);
-    if (host_dec) cudaFreeHost(host_dec);
     if (side && own_side) cudaStreamDestroy(side);
     if (kside && own_kside) cudaStreamDestroy(kside);
   }
@@ -192,31 +183,78 @@ zsm::NormScratch norm_scratch(zero_ctx* c) {
   return ns;
 }
 
-// The clipped step's decision in the scratch arena (after the norm sums).
+// The scratch arena past the norm partials: the step's sums, then (at +64)
+// the clipped step's decision and (at +128) the device step state; one copy
+// of this block gives the host every statistic of the last step.
+constexpr int64_t kDecisionOffset = 64, kStateOffset = 128;
+struct StatsBlock {
+  double sq;
+  unsigned long long nf;
+  unsigned int done;
+  unsigned int error;
+  char pad0[kDecisionOffset - 24];
+  zsm::ClipDecision dec;
+  char pad1[kStateOffset - kDecisionOffset - sizeof(zsm::ClipDecision)];
+  zsm::StepState state;
+};
+static_assert(offsetof(StatsBlock, dec) == kDecisionOffset && offsetof(StatsBlock, state) == kStateOffset,
+              "stats block layout");
+
+char* stats_block(zero_ctx* c) { return c->arena[ZERO_ARENA_SCRATCH] + 16 * zsm::kMaxGrid; }
 zsm::ClipDecision* decision_ptr(zero_ctx* c) {
-  return reinterpret_cast<zsm::ClipDecision*>(c->arena[ZERO_ARENA_SCRATCH] + 16 * zsm::kMaxGrid + 64);
+  return reinterpret_cast<zsm::ClipDecision*>(stats_block(c) + kDecisionOffset);
+}
+zsm::StepState* state_ptr(zero_ctx* c) { return reinterpret_cast<zsm::StepState*>(stats_block(c) + kStateOffset); }
+
+zsm::StepHparams step_hparams(const zero_ctx* c) {
+  zsm::StepHparams h;
+  h.lr = c->hp.lr;
+  h.beta1 = c->hp.beta1;
+  h.beta2 = c->hp.beta2;
+  h.eps = c->hp.eps;
+  h.weight_decay = c->hp.weight_decay;
+  h.loss_scale = c->loss_scale;
+  return h;
 }
 
-zero_status ensure_decision(zero_ctx* c) {
-  cudaError_t e = cudaSuccess;
-  if (!c->ev_decision) e = cudaEventCreateWithFlags(&c->ev_decision, cudaEventDisableTiming);
-  if (e == cudaSuccess && !c->host_dec) e = cudaMallocHost(&c->host_dec, sizeof(zsm::ClipDecision));
-  if (e != cudaSuccess) return cuda_fail(c, e, "creating the decision event and pinned host copy");
+// The device step state for t completed steps: beta^t by t successive
+// binary64 products, as the step kernels continue them.
+zsm::StepState host_state(const zero_adam_hparams& hp, int64_t t) {
+  zsm::StepState st;
+  std::memset(&st, 0, sizeof st);
+  double p1 = 1.0, p2 = 1.0;
+  for (int64_t k = 0; k < t; ++k) {
+    p1 *= hp.beta1;
+    p2 *= hp.beta2;
+  }
+  st.t = t;
+  st.p1 = p1;
+  st.p2 = p2;
+  st.t_next = t;
+  st.p1_next = p1;
+  st.p2_next = p2;
+  return st;
+}
+
+// Reads the device step counter (waits for the device).
+zero_status read_device_t(zero_ctx* c, int64_t* t) {
+  long long v = 0;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(&v, &state_ptr(c)->t, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(c, e, "reading the step counter");
+  *t = (int64_t)v;
+  c->t = *t;
   return ZERO_OK;
 }
 
-// Folds a clipped step's decision, once it has reached the host, into the
-// step counter (advanced unless the step was skipped) and the statistics.
-zero_status resolve_decision(zero_ctx* c) {
-  if (!c->pending) return ZERO_OK;
-  c->pending = false;
-  const cudaError_t e = cudaEventSynchronize(c->ev_decision);
-  if (e != cudaSuccess) return cuda_fail(c, e, "waiting for the clipped step's decision");
-  const zsm::ClipDecision d = *c->host_dec;
-  c->last_skipped = d.skip ? 1 : 0;
-  c->last_coef = d.coef < 1.0f ? (double)d.coef : 1.0;
-  if (!d.skip) c->t = c->pending_t;
-  c->stats_step = c->t;
+// Writes the device step state for t completed steps (waits for the device).
+zero_status write_device_t(zero_ctx* c, int64_t t) {
+  const zsm::StepState st = host_state(c->hp, t);
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(state_ptr(c), &st, sizeof st, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(c, e, "writing the step counter");
+  c->t = t;
+  c->calls = t;
   return ZERO_OK;
 }
 
@@ -384,7 +422,7 @@ std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
 // One fused launch over [lo, hi).  grad[r] are at flat element lo.
 zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
                            bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0,
-                           int pdl = zsm::kPdlNone) {
+                           int pdl = zsm::kPdlNone, const zsm::AdamScalars* sc_dev = nullptr) {
   if (hi == lo) return ZERO_OK;
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
@@ -409,6 +447,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   a.accumulate = accumulate ? 1 : 0;
   a.inv_n = (float)(1.0 / (double)N);
   a.sc = sc;
+  a.sc_dev = sc_dev;
   a.ns = norm_scratch(c);
   a.pdl = c->timing ? zsm::kPdlNone : pdl;  // an event record between launches ends the overlap
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
@@ -442,27 +481,23 @@ zero_status check_device_error(zero_ctx* c, unsigned int err, cudaStream_t s) {
   return fail(c, ZERO_ECUDA, "a bounded wait in the staged fused kernel ran out (code %u): results of the step are invalid", err);
 }
 
+// Synchronises `s` and reads the last step's statistics, its decision and
+// the step counter from the device in one copy.
 zero_status finish_stats(zero_ctx* c, cudaStream_t s, zero_step_stats* out) {
-  struct {
-    double sq;
-    unsigned long long nf;
-    unsigned int done;
-    unsigned int error;
-  } host{};
-  zsm::NormScratch ns = norm_scratch(c);
-  cudaError_t e = cudaMemcpyAsync(&host, ns.step_sq, sizeof host, cudaMemcpyDeviceToHost, s);
+  StatsBlock host;
+  cudaError_t e = cudaMemcpyAsync(&host, stats_block(c), sizeof host, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(c, e, "reading step statistics");
   zero_status st = check_device_error(c, host.error, s);
-  if (st == ZERO_OK) st = resolve_decision(c);
   if (st != ZERO_OK) return st;
+  c->t = (int64_t)host.state.t;
   std::memset(out, 0, sizeof *out);
   out->grad_norm = std::sqrt(host.sq) / c->loss_scale;
   out->nonfinite = (int64_t)host.nf;
-  out->step = c->stats_step;
+  out->step = c->t;
   zero_comm_elems(c, out->comm_elems);
-  out->clip_coef = c->last_coef;
-  out->skipped = c->last_skipped;
+  out->clip_coef = host.dec.coef < 1.0f ? (double)host.dec.coef : 1.0;
+  out->skipped = host.dec.skip ? 1 : 0;
   return ZERO_OK;
 }
 
@@ -661,10 +696,15 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "clipping / skipping needs the reduced-gradient shards (ZERO_OPT_KEEP_GRAD_SHARDS = 1)");
   cudaStream_t s = o.ks;  // the step's kernels; statistics are read on o.s after the join
-  const int64_t t = c->t + 1;
+  const int64_t t = c->calls + 1;  // the callbacks' step number (the kernels use the device's count)
   const std::vector<zsm::Span> iv = step_intervals(c);
   const int n_layers = (int)c->plan.layers.size();
   std::vector<uint16_t*> grad(N);
+  // the scalars of step t + 1 from the device step state, committed by the decision
+  {
+    const cudaError_t e = zsm::launch_step_begin(state_ptr(c), step_hparams(c), nullptr, s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
+  }
   // pass 1: reduce every interval
   bool launched = false;  // the first launch of the step starts the norm sum
   size_t issued = 0;
@@ -697,21 +737,17 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   if (o.err != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
   // The decision -- norm, skip, clipping coefficient -- is taken on the device
   // from the sums pass 1 left and read there by pass 2, so nothing waits
-  // between the passes; the host learns it later (resolve_decision).
-  zero_status st = ensure_decision(c);
-  if (st != ZERO_OK) return st;
+  // between the passes; it also commits the step counter unless the step is
+  // skipped.
+  zero_status st = ZERO_OK;
   zsm::ClipParams cp;
   cp.max_norm = c->clip_norm;
   cp.loss_scale = c->loss_scale;
   cp.skip_nonfinite = c->skip_nonfinite ? 1 : 0;
   zsm::ClipDecision* dec = decision_ptr(c);
-  cudaError_t e = zsm::launch_clip_decide(norm_scratch(c), cp, dec, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(c->host_dec, dec, sizeof *dec, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaEventRecord(c->ev_decision, s);
+  cudaError_t e = zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s);
   if (e != cudaSuccess) return cuda_fail(c, e, "the clipped step's decision");
-  c->pending = true;
-  c->pending_t = t;
-  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);  // the coefficient comes from the decision
+  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);  // by value; the kernels read the device copy
   // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3);
   // a skipped step writes the unchanged parameters only
   std::vector<zsm::Span> p2;
@@ -739,6 +775,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     b.shard = c->plan.shard;
     b.n_vec = (hi - lo) / zsm::kVec;
     b.sc = sc;
+    b.sc_dev = &state_ptr(c)->sc;
     b.dec = dec;
     b.error = norm_scratch(c).error;
     o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
@@ -754,6 +791,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     }
   }
   if (o.end() != cudaSuccess) return cuda_fail(c, o.err, "ordering the pipeline streams");
+  c->calls = t;
   c->norm_fresh = true;
   if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
@@ -762,7 +800,6 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
 zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
                      zero_gather_fn gfn, void* guser, void* stream, zero_step_stats* stats) {
   zero_status st = check_ready(c, true);
-  if (st == ZERO_OK) st = resolve_decision(c);  // t after the last clipped step
   if (st != ZERO_OK) return st;
   const int N = c->plan.n_ranks;
   if (resident) {
@@ -784,11 +821,14 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
     o.end();  // joins the side stream also on the error paths
     return st;
   }
-  c->last_coef = 1.0;
-  c->last_skipped = 0;
   cudaStream_t s = o.ks;  // the step's kernels
-  const int64_t t = c->t + 1;
+  const int64_t t = c->calls + 1;  // the callbacks' step number (the kernels use the device's count)
   const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
+  // the step's scalars from the device step state (committed when the step completes)
+  {
+    const cudaError_t e = zsm::launch_step_begin(state_ptr(c), step_hparams(c), decision_ptr(c), s);
+    if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
+  }
   const std::vector<zsm::Span> iv = step_intervals(c);
   std::vector<uint16_t*> grad(N);
   const int n_layers = (int)c->plan.layers.size();
@@ -817,16 +857,20 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
                     : !launched ? zsm::kPdlWaitFirst
                     : c->stage != ZERO_STAGE_3 ? zsm::kPdlEarly
                                                : zsm::kPdlEarlyLoads;
-    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl);
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl, &state_ptr(c)->sc);
     if (st != ZERO_OK) break;
     launched = launched || hi > lo;
     o.after_kernel(k);
     if (gathers) st = issue_gather(c, o, gfn, guser, layer_idx, k);
   }
+  if (st == ZERO_OK) {
+    const cudaError_t e = zsm::launch_step_commit(state_ptr(c), s);
+    if (e != cudaSuccess) st = cuda_fail(c, e, "step-commit kernel launch");
+  }
   if (o.end() != cudaSuccess && st == ZERO_OK) st = cuda_fail(c, o.err, "ordering the pipeline streams");
   if (st != ZERO_OK) return st;
+  c->calls = t;
   c->t = t;
-  c->stats_step = t;
   c->norm_fresh = true;
   if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
@@ -1012,8 +1056,16 @@ zero_status zero_set_hparams(zero_ctx* c, const zero_adam_hparams* hp) {
   if (!(hp->lr >= 0.0) || !(hp->beta1 >= 0.0 && hp->beta1 < 1.0) || !(hp->beta2 >= 0.0 && hp->beta2 < 1.0) ||
       !(hp->eps >= 0.0) || !(hp->weight_decay >= 0.0))
     return fail(c, ZERO_EINVAL, "hyper-parameters out of range (lr, eps, wd >= 0; 0 <= beta < 1)");
+  const bool new_betas = c->have_hp && (hp->beta1 != c->hp.beta1 || hp->beta2 != c->hp.beta2);
   c->hp = *hp;
   c->have_hp = true;
+  if (new_betas && c->bound && c->loaded) {
+    // the bias corrections are the new betas to the power t: rebuild the
+    // device powers for the current t (waits for the device)
+    int64_t t = 0;
+    const zero_status st = read_device_t(c, &t);
+    return st != ZERO_OK ? st : write_device_t(c, t);
+  }
   return ZERO_OK;
 }
 
@@ -1022,9 +1074,17 @@ namespace {
 // Fills the state from sources (see InitArgs) and resets the run state.
 zero_status load_state(zero_ctx* c, const float* master, const float* m, const float* v, int64_t n,
                        int64_t t, cudaStream_t s) {
-  const zero_status st = resolve_decision(c);  // a pending decision must not overwrite the new t
-  if (st != ZERO_OK) return st;
   cudaError_t e = cudaMemsetAsync(c->arena[ZERO_ARENA_SCRATCH], 0, kScratchBytes, s);
+  if (e == cudaSuccess) {
+    // the step state for t completed steps and a decision of "no clipping, not
+    // skipped" (pageable sources: copied before the calls return)
+    const zsm::StepState st = host_state(c->hp, t);
+    e = cudaMemcpyAsync(state_ptr(c), &st, sizeof st, cudaMemcpyHostToDevice, s);
+    zsm::ClipDecision d;
+    std::memset(&d, 0, sizeof d);
+    d.coef = 1.0f;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(decision_ptr(c), &d, sizeof d, cudaMemcpyHostToDevice, s);
+  }
   if (e != cudaSuccess) return cuda_fail(c, e, "clearing scratch");
   zsm::InitArgs a;
   std::memset(&a, 0, sizeof a);
@@ -1043,7 +1103,7 @@ zero_status load_state(zero_ctx* c, const float* master, const float* m, const f
   e = zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s);
   if (e != cudaSuccess) return cuda_fail(c, e, "init kernel launch");
   c->t = t;
-  c->stats_step = t;
+  c->calls = t;
   c->loaded = true;
   c->norm_fresh = true;
   return ZERO_OK;
@@ -1076,18 +1136,21 @@ zero_status zero_import_state(zero_ctx* c, const float* master, const float* exp
 zero_status zero_get_step(const zero_ctx* cc, int64_t* t) {
   zero_ctx* c = const_cast<zero_ctx*>(cc);
   if (!c || !t) return ZERO_EINVAL;
-  const zero_status st = resolve_decision(c);
-  if (st != ZERO_OK) return st;
-  *t = c->t;
-  return ZERO_OK;
+  if (!c->bound || !c->loaded) {
+    *t = c->t;
+    return ZERO_OK;
+  }
+  return read_device_t(c, t);
 }
 
 zero_status zero_set_step(zero_ctx* c, int64_t t) {
   if (!c || t < 0) return ZERO_EINVAL;
-  const zero_status st = resolve_decision(c);
-  if (st != ZERO_OK) return st;
-  c->t = t;
-  return ZERO_OK;
+  if (!c->bound || !c->loaded) {
+    c->t = t;
+    c->calls = t;
+    return ZERO_OK;
+  }
+  return write_device_t(c, t);
 }
 
 zero_status zero_view(const zero_ctx* cc, int32_t what, int32_t rank, void** ptr, int64_t* n_elems) {
@@ -1265,7 +1328,6 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
         if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
       }
       c->norm_fresh = true;
-      c->stats_step = t;
       return ZERO_OK;
     }
   } else {
@@ -1285,7 +1347,6 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
         if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
       }
       c->norm_fresh = true;
-      c->stats_step = t;
       return ZERO_OK;
     }
   }
@@ -1294,7 +1355,6 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
     if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
   }
   c->norm_fresh = true;
-  c->stats_step = t;
   return ZERO_OK;
 }
 
