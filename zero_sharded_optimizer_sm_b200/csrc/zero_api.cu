@@ -747,7 +747,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   zsm::ClipDecision* dec = decision_ptr(c);
   cudaError_t e = zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s);
   if (e != cudaSuccess) return cuda_fail(c, e, "the clipped step's decision");
-  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);  // by value; the kernels read the device copy
+  const zsm::AdamScalars sc{};  // the kernels read the step's scalars from the device step state
   // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3);
   // a skipped step writes the unchanged parameters only
   std::vector<zsm::Span> p2;
@@ -823,8 +823,9 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   }
   cudaStream_t s = o.ks;  // the step's kernels
   const int64_t t = c->calls + 1;  // the callbacks' step number (the kernels use the device's count)
-  const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
-  // the step's scalars from the device step state (committed when the step completes)
+  // the kernels read the step's scalars from the device step state (no host
+  // copy: forming beta^t on the host would cost t multiplications a step)
+  const zsm::AdamScalars sc{};
   {
     const cudaError_t e = zsm::launch_step_begin(state_ptr(c), step_hparams(c), decision_ptr(c), s);
     if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
