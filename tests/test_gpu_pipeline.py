@@ -287,3 +287,33 @@ def test_pipeline_streams_are_fixed_after_the_first_pipelined_step():
     other = torch.cuda.Stream()
     assert z.zero_set_pipeline_streams(opt.ctx, other.cuda_stream, None) == z.ZERO_ESTATE
     opt.close()
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_clipped_pipelined_stage3_repeated_equals_in_order(mode):
+    """A clipped ZeRO-3 step with the callbacks (and a gather consumer) on the
+    side stream, repeated: the staged Adam-broadcast pass must not see a stage
+    refilled while its shared-memory reads are still in flight -- the
+    producer's proxy fence orders them (without it this case differed in
+    scattered elements in every repetition on B200)."""
+    z = _z()
+    numel, layer = W.transformer_layers(2, 768, 3072)
+    w = W.Workload("pipe-race", numel, layer, 8, (3,), 3_000_000, synth.Dist(synth.NORMAL, 1e-2, zero_mod=100),
+                   W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01), W.SEED0 + 31)
+    for _ in range(4):
+        a, fa = make_opt(w, 3, 3_000_000, 0)
+        b, fb = make_opt(w, 3, 3_000_000, mode)
+        a.set_clip(0.5, True)
+        b.set_clip(0.5, True)
+        ga, gb = [], []
+        for t in range(1, w.steps + 1):
+            ga.clear()
+            gb.clear()
+            a.step(grad_fn_for(a, fa), gather_recorder(a, ga), stats=True)
+            b.step(grad_fn_for(b, fb), gather_recorder(b, gb), stats=True)
+            for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ, z.ZERO_VIEW_PARAM):
+                assert torch.equal(a.view(what), b.view(what)), (t, what)
+            for (_, _, _, x), (_, _, _, y) in zip(ga, gb):
+                assert all(torch.equal(u, v) for u, v in zip(x, y))
+        a.close()
+        b.close()

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
           *abort_flag = 1;
           break;
         }
+        fence_proxy_async_smem();  // the consumers' reads of this stage before the copies refill it
         const int64_t e0 = tile * kTile;
         const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
         unsigned char* st = smem + (size_t)s * stage_bytes;
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           *abort_flag = 1;
           break;
         }
+        fence_proxy_async_smem();  // the consumers' reads of this stage before the copies refill it
         const int64_t e0 = tile * kTile;
         const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
         unsigned char* st = smem + (size_t)s * stage_bytes;
@@ -410,6 +412,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
           *abort_flag = 1;
           break;
         }
+        fence_proxy_async_smem();
         unsigned char* stt = state_base + (size_t)ss * kStateBytes;
         mbar_expect_tx(&sfull[ss], (unsigned)(12 * cnt));
         bulk_load(stt, a.master + e0, (unsigned)(4 * cnt), &sfull[ss], policy);
@@ -428,6 +431,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
             stop = true;
             break;
           }
+          fence_proxy_async_smem();
           const int r0 = c * kChunkRanks;
           const int r1 = (r0 + kChunkRanks) < N ? (r0 + kChunkRanks) : N;
           unsigned char* st = chunk_base + (size_t)cs * kChunkBytes;

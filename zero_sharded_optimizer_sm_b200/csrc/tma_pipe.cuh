@@ -69,6 +69,16 @@ static __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity)
   return true;
 }
 
+// A stage is refilled by bulk copies (async proxy) after its consumers'
+// ordinary shared-memory reads (generic proxy) -- ordered by the empty
+// barrier the producer has just waited on, which orders generic-proxy
+// accesses only.  This fence orders those reads before the async-proxy
+// writes that follow; without it a consumer's read still in flight when it
+// released the stage could return the next tile's data.
+static __device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // L2 policy for the bulk loads: every input byte is read exactly once, so it
 // is marked first to evict and leaves L2 room for the write-back traffic.
 static __device__ __forceinline__ uint64_t evict_first_policy() {

@@ -89,6 +89,7 @@ __device__ __forceinline__ bool acquire_stage(const Ring& r, int s, unsigned k, 
     *r.abort_flag = 1;
     return false;
   }
+  fence_proxy_async_smem();  // the consumers' reads of this stage before the copies refill it
   return true;
 }
 
