@@ -512,6 +512,20 @@ zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
 zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, double* model_bytes);
 
 /*
+ * zero_launch_count -- the number of kernels this context has enqueued since
+ * zero_init: every fused, staged, two-pass, Adam, all-gather and
+ * initialisation launch, and the one-thread kernels that form and commit the
+ * step's device-held counter and scalars.  A zero_step / zero_step_resident
+ * enqueues the launches zero_kernel_timing times (one fused launch per
+ * non-empty interval; a clipped step its reduce launches and its
+ * Adam-broadcast launches, one over the whole buffer at stage 1/2, one per
+ * layer at stage 3) plus two of those one-thread kernels.  Host only: reads a
+ * counter kept by the launching calls, no device work and no wait.
+ * ZERO_EINVAL for a NULL argument.
+ */
+zero_status zero_launch_count(const zero_ctx* ctx, int64_t* n);
+
+/*
  * zero_fused_step_static -- one fused ZeRO-2 step over a single flat interval
  * that allocates nothing.  The pages have no counterpart to this entry point:
  * it exists for callers that cannot allocate device memory when they run the

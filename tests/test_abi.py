@@ -171,6 +171,25 @@ def test_pipeline_streams_and_option_values_on_the_host():
         z.zero_destroy(ctx)
 
 
+def test_launch_count_starts_at_zero_and_refused_calls_launch_nothing():
+    """zero_launch_count is a host counter: 0 after zero_init, unchanged by
+    calls that are refused before any launch, EINVAL for NULL arguments."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    st, ctx = _init([64, 64], [0, 1], 4, 2, 64)
+    assert st == 0
+    try:
+        n = ctypes.c_int64(-1)
+        assert z.zero_launch_count(ctx, ctypes.byref(n)) == z.ZERO_OK and n.value == 0
+        assert z.zero_reduce_scatter(ctx, 0, 64, None, None) == z.ZERO_ESTATE
+        assert z.zero_adam_shard(ctx, -1, 1, None) == z.ZERO_ESTATE
+        assert z.zero_launch_count(ctx, ctypes.byref(n)) == z.ZERO_OK and n.value == 0
+        assert z.zero_launch_count(ctx, None) == z.ZERO_EINVAL
+        assert z.zero_launch_count(None, ctypes.byref(n)) == z.ZERO_EINVAL
+    finally:
+        z.zero_destroy(ctx)
+
+
 def test_init_rejects_bad_arguments():
     import zero_sharded_optimizer_sm_b200 as z
 

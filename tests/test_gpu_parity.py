@@ -289,6 +289,35 @@ def test_adam_shard_per_rank_equals_all_ranks():
 
 
 @pytest.mark.parametrize("stage", [1, 2, 3])
+@pytest.mark.parametrize("clip", [0.0, 0.5])
+def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
+    """zero_launch_count advances by exactly the launches zero_kernel_timing
+    records plus the two one-thread step kernels, per step, plain and clipped."""
+    numel, layer = W.transformer_layers(3, 64, 256)
+    w = W.Workload("count", numel, layer, 4, (stage,), 16_000, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 2,
+                   W.Hyper(), 0x600 + stage)
+    opt, fill = make_opt(w, stage, bucket=16_000)
+    p = oracle.plan(w.numel, w.layer_id, w.n_ranks, 16_000)
+    if clip > 0:
+        opt.set_clip(clip, True)
+    dev = [torch.from_numpy(W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, 1, r),
+                                          w.grad_dist).view(np.int16)).cuda() for r in range(w.n_ranks)]
+    opt.set_timing(True)
+    opt.kernel_timing()
+    for _ in range(2):
+        n0 = opt.launch_count()
+        opt.step_resident(dev)
+        torch.cuda.synchronize()
+        timed = opt.kernel_timing()["launches"]
+        intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
+        expect = intervals if clip == 0 else intervals + (intervals if stage == 3 else 1)
+        assert timed == expect, (timed, expect)
+        assert opt.launch_count() - n0 == timed + 2
+    opt.set_timing(False)
+    opt.close()
+
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
 def test_pdl_resident_steps_equal_plain_launches(stage):
     """Resident steps with ZERO_OPT_PDL launch their fused kernels with
     programmatic dependent launch (at stage 1/2 each later launch streams its

@@ -107,6 +107,7 @@ _SIGS = {
                                   ctypes.POINTER(zero_step_stats)]),
     "zero_kernel_timing": (_i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                   ctypes.POINTER(ctypes.c_double)]),
+    "zero_launch_count": (_i32, [_vp, ctypes.POINTER(_i64)]),
     "zero_set_clip": (_i32, [_vp, ctypes.c_double, _i32]),
     "zero_set_loss_scale": (_i32, [_vp, ctypes.c_double]),
     "zero_set_pipeline_streams": (_i32, [_vp, _vp, _vp]),
@@ -445,6 +446,12 @@ class ZeroOptimizer:
         self._check(zero_kernel_timing(self.ctx, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(b)),
                     "zero_kernel_timing")
         return dict(ms=ms.value, launches=n.value, model_bytes=b.value)
+
+    def launch_count(self) -> int:
+        """Kernels this context has enqueued since it was created."""
+        n = ctypes.c_int64()
+        self._check(zero_launch_count(self.ctx, ctypes.byref(n)), "zero_launch_count")
+        return n.value
 
     def read_stats(self, stream=None) -> dict:
         out = zero_step_stats()

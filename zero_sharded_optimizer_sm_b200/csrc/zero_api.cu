@@ -87,6 +87,7 @@ struct zero_ctx {
   std::vector<cudaEvent_t> events;  // pairs (start, end), reused
   size_t timed = 0;                 // pairs recorded since the last read
   double timed_bytes = 0.0;
+  int64_t launched = 0;             // kernels this context has enqueued (zero_launch_count)
   std::string err;
   ~zero_ctx() {
     for (cudaEvent_t e : events) cudaEventDestroy(e);
@@ -374,6 +375,13 @@ int64_t fused_bytes_per_elem(const zero_ctx* c) {
   return 4 * N + 26 + keep;
 }
 
+// Counts a kernel the context enqueued (zero_launch_count) and passes the
+// launch status through.
+cudaError_t counted(zero_ctx* c, cudaError_t e) {
+  if (e == cudaSuccess) ++c->launched;
+  return e;
+}
+
 // Event pair for the next timed launch, or nullptr when the record is full.
 cudaEvent_t* timing_pair(zero_ctx* c) {
   if (c->timed >= kMaxTimed) return nullptr;
@@ -456,14 +464,14 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   cudaError_t e;
   if (use_chunked(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
-    e = zsm::launch_fused_chunked(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
-                                  chunked_stages(c), s);
+    e = counted(c, zsm::launch_fused_chunked(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
+                                  chunked_stages(c), s));
   } else if (use_tma(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
-    e = zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, tma_grid_cap(c))),
-                              tma_groups(c), tma_stages(c), s);
+    e = counted(c, zsm::launch_fused_tma(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, tma_grid_cap(c))),
+                              tma_groups(c), tma_stages(c), s));
   } else {
-    e = zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s);
+    e = counted(c, zsm::launch_fused(mode, a, grid_for(a.n_vec, c->grid_fused), s));
   }
   if (e != cudaSuccess) return cuda_fail(c, e, "fused step kernel launch");
   if (ev) {
@@ -664,8 +672,8 @@ cudaError_t launch_pass1(zero_ctx* c, const zsm::ReduceArgs& a, cudaStream_t s) 
   const int64_t elems = a.n_vec * zsm::kVec;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  const cudaError_t e = use_two_pass_tma(c) ? zsm::launch_reduce_tma(a, two_pass_grid(c, elems), s)
-                                            : zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s);
+  const cudaError_t e = counted(c, use_two_pass_tma(c) ? zsm::launch_reduce_tma(a, two_pass_grid(c, elems), s)
+                                                       : zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s));
   if (e == cudaSuccess && ev) {
     cudaEventRecord(ev[1], s);
     c->timed += 1;
@@ -678,8 +686,9 @@ cudaError_t launch_pass2(zero_ctx* c, const zsm::AdamBcastArgs& b, bool uniform,
   const int64_t elems = b.n_vec * zsm::kVec;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  const cudaError_t e = use_two_pass_tma(c) ? zsm::launch_adam_bcast_tma(b, two_pass_grid(c, elems), uniform, s)
-                                            : zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s);
+  const cudaError_t e = counted(c, use_two_pass_tma(c)
+                                       ? zsm::launch_adam_bcast_tma(b, two_pass_grid(c, elems), uniform, s)
+                                       : zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s));
   if (e == cudaSuccess && ev) {
     cudaEventRecord(ev[1], s);
     c->timed += 1;
@@ -702,7 +711,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   std::vector<uint16_t*> grad(N);
   // the scalars of step t + 1 from the device step state, committed by the decision
   {
-    const cudaError_t e = zsm::launch_step_begin(state_ptr(c), step_hparams(c), nullptr, s);
+    const cudaError_t e = counted(c, zsm::launch_step_begin(state_ptr(c), step_hparams(c), nullptr, s));
     if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
   }
   // pass 1: reduce every interval
@@ -745,7 +754,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   cp.loss_scale = c->loss_scale;
   cp.skip_nonfinite = c->skip_nonfinite ? 1 : 0;
   zsm::ClipDecision* dec = decision_ptr(c);
-  cudaError_t e = zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s);
+  cudaError_t e = counted(c, zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s));
   if (e != cudaSuccess) return cuda_fail(c, e, "the clipped step's decision");
   const zsm::AdamScalars sc{};  // the kernels read the step's scalars from the device step state
   // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3);
@@ -827,7 +836,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   // copy: forming beta^t on the host would cost t multiplications a step)
   const zsm::AdamScalars sc{};
   {
-    const cudaError_t e = zsm::launch_step_begin(state_ptr(c), step_hparams(c), decision_ptr(c), s);
+    const cudaError_t e = counted(c, zsm::launch_step_begin(state_ptr(c), step_hparams(c), decision_ptr(c), s));
     if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
   }
   const std::vector<zsm::Span> iv = step_intervals(c);
@@ -865,7 +874,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
     if (gathers) st = issue_gather(c, o, gfn, guser, layer_idx, k);
   }
   if (st == ZERO_OK) {
-    const cudaError_t e = zsm::launch_step_commit(state_ptr(c), s);
+    const cudaError_t e = counted(c, zsm::launch_step_commit(state_ptr(c), s));
     if (e != cudaSuccess) st = cuda_fail(c, e, "step-commit kernel launch");
   }
   if (o.end() != cudaSuccess && st == ZERO_OK) st = cuda_fail(c, o.err, "ordering the pipeline streams");
@@ -1101,7 +1110,7 @@ zero_status load_state(zero_ctx* c, const float* master, const float* m, const f
   for (int r = 0; r < a.n_out; ++r) a.out[r] = param_ptr(c, r);
   a.grad_shard = c->arena[ZERO_ARENA_GRAD_SHARDS] ? grad_shard_ptr(c) : nullptr;
   a.n_vec = c->plan.psi_pad / zsm::kVec;
-  e = zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s);
+  e = counted(c, zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s));
   if (e != cudaSuccess) return cuda_fail(c, e, "init kernel launch");
   c->t = t;
   c->calls = t;
@@ -1325,7 +1334,7 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
         b.grad = grad_shard_ptr(c) + r * S;
         b.out = param_ptr(c, r) + r * S;
         b.n_vec = S / zsm::kVec;
-        cudaError_t e = zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s);
+        cudaError_t e = counted(c, zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s));
         if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
       }
       c->norm_fresh = true;
@@ -1344,7 +1353,7 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
         b.grad = grad_buf_ptr(c, r) + r * S;
         b.out = param_ptr(c, r) + r * S;
         b.n_vec = S / zsm::kVec;
-        cudaError_t e = zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s);
+        cudaError_t e = counted(c, zsm::launch_adam(b, grid_for(b.n_vec, c->grid_simple), s));
         if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
       }
       c->norm_fresh = true;
@@ -1352,7 +1361,7 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
     }
   }
   if (a.n_vec > 0) {
-    cudaError_t e = zsm::launch_adam(a, grid_for(a.n_vec, c->grid_simple), s);
+    cudaError_t e = counted(c, zsm::launch_adam(a, grid_for(a.n_vec, c->grid_simple), s));
     if (e != cudaSuccess) return cuda_fail(c, e, "adam kernel launch");
   }
   c->norm_fresh = true;
@@ -1399,7 +1408,7 @@ zero_status zero_all_gather(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
     }
     g.n_vec = (a_hi - a_lo) / zsm::kVec;
     if (g.n_out == 0) continue;
-    cudaError_t e = zsm::launch_gather(g, grid_for(g.n_vec, c->grid_simple), s);
+    cudaError_t e = counted(c, zsm::launch_gather(g, grid_for(g.n_vec, c->grid_simple), s));
     if (e != cudaSuccess) return cuda_fail(c, e, "all-gather kernel launch");
   }
   return ZERO_OK;
@@ -1475,6 +1484,12 @@ zero_status zero_fused_config(const zero_ctx* c, int32_t* kernel, int32_t* group
     *groups = 0;
     *stages = 0;
   }
+  return ZERO_OK;
+}
+
+zero_status zero_launch_count(const zero_ctx* c, int64_t* n) {
+  if (!c || !n) return ZERO_EINVAL;
+  *n = c->launched;
   return ZERO_OK;
 }
 
