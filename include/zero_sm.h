@@ -581,7 +581,13 @@ zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
  * ctx == NULL: the reason the calling thread's last zero_init failed. */
 const char* zero_last_error(const zero_ctx* ctx);
 
-/* Release a context (the arenas stay the caller's). NULL is a no-op. */
+/* Release a context (the arenas stay the caller's). NULL is a no-op.  Does
+ * not wait for the device: work already enqueued keeps using the arenas, so
+ * the caller frees them only after the stream given to the last call has
+ * reached that point (every call joins its side streams back into that
+ * stream before it returns).  Streams and events the context created are
+ * released once their work completes; streams given by
+ * zero_set_pipeline_streams stay the caller's. */
 void zero_destroy(zero_ctx* ctx);
 
 #ifdef __cplusplus
