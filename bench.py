@@ -531,8 +531,9 @@ def run_ours(args, world, rank, local):
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
                      "model_bytes_per_launch": model_bytes_per_step / per_step_launches,
                      "achieved_how": "model bytes of the timed launches / CUDA-event time of the timed "
-                                     "region (fused launches only, back to back"
-                                     + ("" if args.no_pdl else ", programmatic dependent launch") + ")",
+                                     "region (the fused launches back to back"
+                                     + ("" if args.no_pdl else ", programmatic dependent launch")
+                                     + "; the region also holds two one-thread step-state kernels a step)",
                      "kernel_ms_per_launch_isolated": kernel_ms_isolated,
                      "achieved_isolated": (kt["model_bytes"] / kt["launches"] / (kernel_ms_isolated / 1e3) / 1e9
                                            if kernel_ms_isolated else None),
