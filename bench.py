@@ -159,6 +159,28 @@ def traffic_for_current_kernel(kernel: str, key: str, elems_per_launch: float):
         return None
 
 
+def nvsmi_index(device_index: int) -> int:
+    """nvidia-smi's index of CUDA device `device_index`: the two numberings
+    differ when CUDA_VISIBLE_DEVICES selects or reorders devices, so the GPU
+    is matched by its PCI domain, bus and device numbers (the CUDA index when
+    nothing matches)."""
+    try:
+        import torch
+
+        p = torch.cuda.get_device_properties(device_index)
+        want = (int(p.pci_domain_id), int(p.pci_bus_id), int(p.pci_device_id))
+        out = subprocess.run(["nvidia-smi", "--query-gpu=index,pci.bus_id", "--format=csv,noheader"],
+                             capture_output=True, text=True, timeout=30).stdout
+        for line in out.splitlines():
+            idx, bus = [x.strip() for x in line.split(",")[:2]]
+            dom, b, dev_fn = bus.split(":")
+            if (int(dom, 16), int(b, 16), int(dev_fn.split(".")[0], 16)) == want:
+                return int(idx)
+    except Exception:
+        pass
+    return device_index
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -204,7 +226,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "nvidia_smi_index": self.gpu}
 
 
 # ---------------------------------------------------------------- workload ----
@@ -411,7 +433,7 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         opt.step_resident(rep_list)
     torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local)
+    sampler = ClockSampler(nvsmi_index(local))
     sampler.start()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
