@@ -72,3 +72,30 @@ def test_reference_arm_prints_once_on_rank_zero():
     assert d["impl"] == "reference" and d["unit"] == "params/s" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["cpu_baseline"]["cores"] >= 1 and d["n_gpus"] == 2
+
+
+def test_clock_sampler_matches_the_gpu_by_pci_bus_id(monkeypatch):
+    """nvidia-smi numbers GPUs by PCI order, CUDA by what CUDA_VISIBLE_DEVICES
+    leaves: the sampler's index is the nvidia-smi row with the CUDA device's
+    PCI domain/bus/device, else the CUDA index."""
+    import types
+
+    import torch
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    props = types.SimpleNamespace(pci_domain_id=0, pci_bus_id=0x9C, pci_device_id=0)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda i: props)
+    rows = "0, 00000000:1B:00.0\n1, 00000000:43:00.0\n2, 00000000:9C:00.0\n"
+    monkeypatch.setattr(bench.subprocess, "run",
+                        lambda *a, **k: types.SimpleNamespace(stdout=rows, returncode=0))
+    assert bench.nvsmi_index(0) == 2
+    props.pci_bus_id = 0x55  # no such row: the CUDA index
+    assert bench.nvsmi_index(1) == 1
+
+    def no_smi(*a, **k):
+        raise FileNotFoundError("nvidia-smi")
+
+    monkeypatch.setattr(bench.subprocess, "run", no_smi)
+    assert bench.nvsmi_index(3) == 3
