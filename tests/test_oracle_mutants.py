@@ -9,6 +9,7 @@ import oracle
 from oracle import build as obuild
 
 import test_oracle_adam as A
+import test_oracle_adam_invariants as I
 import test_oracle_bf16 as B
 import test_oracle_reduce as R
 
@@ -51,6 +52,18 @@ MUTANTS = [
      "    const float gi = zo_bf16_to_f32(g[i]);\n    float p = master[i];\n    p = p * decay;",
      "    const float gi = zo_bf16_to_f32(g[i]);\n    float p = master[i];",
      A.test_weight_decay_alone_scales_weights_by_one_minus_lr_wd),
+    ("second moment from |g| instead of g^2",
+     "    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     "    const float gg = fabsf(gi);\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(3, 0.0)),
+    ("square root of the second moment dropped",
+     "    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     "    const float den = vh + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(-1, 0.0)),
+    ("first moment from |g|",
+     "    float b = omb1 * gi;\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     "    float b = omb1 * fabsf(gi);\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
+     lambda: I.test_negated_gradients_negate_weights_and_first_moment_exactly(0.0)),
     ("bias-correction power off by one step",
      "  for (int64_t k = 0; k < t; ++k) {\n    p1 = p1 * beta1;",
      "  for (int64_t k = 0; k < t - 1; ++k) {\n    p1 = p1 * beta1;",
