@@ -125,7 +125,11 @@ def _load():
 # ------------------------------------------------------------ elementwise ----
 
 def bf16_rne(x: np.ndarray) -> np.ndarray:
-    """fp32 -> bf16 bit patterns (uint16), round to nearest even."""
+    """fp32 -> bf16 bit patterns (uint16), IEEE round to nearest even,
+    overflow to infinity.  The 2-byte format of the gradients and parameter
+    copies that the pages account everywhere ([M] section 1, memory
+    composition; [Q] sections 二, 四.2, 五.2); the pages name no rounding, and
+    round-to-nearest-even is the reading taken."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     out = np.empty(x.shape, dtype=np.uint16)
     if x.size:
@@ -134,6 +138,7 @@ def bf16_rne(x: np.ndarray) -> np.ndarray:
 
 
 def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> fp32, exact (the 2-byte format of [M] section 1)."""
     h = np.ascontiguousarray(h, dtype=np.uint16)
     out = np.empty(h.shape, dtype=np.float32)
     if h.size:
@@ -142,7 +147,10 @@ def bf16_to_f32(h: np.ndarray) -> np.ndarray:
 
 
 def f16_rne(x: np.ndarray) -> np.ndarray:
-    """fp32 -> IEEE binary16 bit patterns (uint16), round to nearest even."""
+    """fp32 -> IEEE binary16 bit patterns (uint16), round to nearest even,
+    overflow to infinity, subnormals kept.  The FP16 the pages name for
+    gradients and parameters ([M] section 1) as the alternative storage
+    format to bf16."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     out = np.empty(x.shape, dtype=np.uint16)
     if x.size:
@@ -151,6 +159,7 @@ def f16_rne(x: np.ndarray) -> np.ndarray:
 
 
 def f16_to_f32(h: np.ndarray) -> np.ndarray:
+    """IEEE binary16 bit patterns -> fp32, exact ([M] section 1's FP16)."""
     h = np.ascontiguousarray(h, dtype=np.uint16)
     out = np.empty(h.shape, dtype=np.float32)
     if h.size:
@@ -159,10 +168,12 @@ def f16_to_f32(h: np.ndarray) -> np.ndarray:
 
 
 def fmt_rne(x: np.ndarray, fmt: int) -> np.ndarray:
+    """``bf16_rne`` or ``f16_rne`` by the storage format."""
     return f16_rne(x) if fmt == F16 else bf16_rne(x)
 
 
 def fmt_to_f32(h: np.ndarray, fmt: int) -> np.ndarray:
+    """``bf16_to_f32`` or ``f16_to_f32`` by the storage format."""
     return f16_to_f32(h) if fmt == F16 else bf16_to_f32(h)
 
 
@@ -174,7 +185,11 @@ def _ptr_array(arrays: Sequence[np.ndarray]):
 
 
 def reduce_mean(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
-    """Averaged bf16 gradient of N equal-length rank slices (uint16 arrays)."""
+    """Averaged bf16 gradient of N equal-length rank slices (uint16 arrays):
+    the reduction of [T] section "ZeRO-2" (reduce-scatter of the ranks'
+    gradients, averaged over the N ranks).  The pages fix neither order nor
+    precision; the reading taken: a binary32 sum from +0 in rank order
+    0..N-1, multiplied by the binary32 reciprocal of N, rounded to bf16."""
     rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
     n = rank_slices[0].size
     assert all(a.size == n for a in rank_slices)
@@ -185,7 +200,9 @@ def reduce_mean(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
 
 
 def reduce_mean_fmt(rank_slices: Sequence[np.ndarray], fmt: int) -> np.ndarray:
-    """reduce_mean for either 16-bit format (the bf16 path is reduce_mean)."""
+    """reduce_mean for either 16-bit format (the bf16 path is reduce_mean):
+    [T] section "ZeRO-2"'s averaged gradient, the mean rounded once to the
+    storage format."""
     if fmt == BF16:
         return reduce_mean(rank_slices)
     rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
@@ -197,6 +214,8 @@ def reduce_mean_fmt(rank_slices: Sequence[np.ndarray], fmt: int) -> np.ndarray:
 
 
 def rank_sum_f32(rank_slices: Sequence[np.ndarray]) -> np.ndarray:
+    """The binary32 rank-order sum inside ``reduce_mean``, before the mean
+    ([T] section "ZeRO-2", the reduce of the reduce-scatter)."""
     rank_slices = [np.ascontiguousarray(a, dtype=np.uint16) for a in rank_slices]
     n = rank_slices[0].size
     out = np.empty(n, dtype=np.float32)
@@ -215,7 +234,13 @@ class AdamHP:
 
 
 def adam_scalars(hp: AdamHP, t: int) -> np.ndarray:
-    """float32[9]: beta1, beta2, 1-beta1, 1-beta2, bc1, bc2, decay, lr, eps."""
+    """float32[9]: beta1, beta2, 1-beta1, 1-beta2, bc1, bc2, decay, lr, eps.
+    The per-step scalars of bias-corrected Adam with decoupled weight decay,
+    the optimizer every page names without writing it out ([T] sections
+    "ZeRO-1" to "ZeRO-3", part "3. 更新"; the definition is Kingma & Ba's
+    Algorithm 1 plus Loshchilov & Hutter's decoupled decay): each formed in
+    binary64 from the hyper-parameters (beta^t by t multiplications) and
+    rounded once to binary32."""
     out = np.empty(9, dtype=np.float32)
     _load().zo_adam_scalars(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, t,
                             out.ctypes.data)
@@ -224,7 +249,12 @@ def adam_scalars(hp: AdamHP, t: int) -> np.ndarray:
 
 def adam(g: np.ndarray, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: AdamHP,
          t: int) -> np.ndarray:
-    """In-place Adam on fp32 master/m/v from the bf16 grad g; returns the bf16 params."""
+    """In-place Adam on fp32 master/m/v from the bf16 grad g; returns the bf16 params.
+
+    The owner's update of its shard in every ZeRO stage ([T] sections
+    "ZeRO-1" to "ZeRO-3", part "3. 更新"), on the fp32 master weights and
+    moments the pages keep per parameter ([M] section 1: 4 + 4 + 4 bytes),
+    followed by the cast of the new master to the 2-byte parameter copy."""
     assert master.dtype == np.float32 and m.dtype == np.float32 and v.dtype == np.float32
     assert master.flags.c_contiguous and m.flags.c_contiguous and v.flags.c_contiguous
     g = np.ascontiguousarray(g, dtype=np.uint16)
@@ -240,7 +270,9 @@ def adam(g: np.ndarray, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: Ad
 def adam_coef(g: np.ndarray, coef: float, master: np.ndarray, m: np.ndarray, v: np.ndarray, hp: AdamHP,
               t: int) -> np.ndarray:
     """Adam with the averaged gradient scaled by a clipping coefficient
-    (applied only when coef < 1)."""
+    (applied only when coef < 1): ``adam``'s update ([T] sections "ZeRO-1" to
+    "ZeRO-3", part "3. 更新") on fp32(g) * coef.  Clipping itself is not on
+    the pages; see ``clip_coef``."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     n = g.size
     assert master.size == n and m.size == n and v.size == n
@@ -254,7 +286,11 @@ def adam_coef(g: np.ndarray, coef: float, master: np.ndarray, m: np.ndarray, v: 
 def adam_ex(g: np.ndarray, fmt: int, inv_scale: float, coef: float, master: np.ndarray, m: np.ndarray,
             v: np.ndarray, hp: AdamHP, t: int) -> np.ndarray:
     """Adam for either format with a loss-scale unscale (inv_scale != 1) and a
-    clipping coefficient (applied when < 1); returns the 16-bit params."""
+    clipping coefficient (applied when < 1); returns the 16-bit params.
+    ``adam``'s update ([T] sections "ZeRO-1" to "ZeRO-3", part "3. 更新") on
+    the FP16 storage the pages name ([M] section 1), whose gradients carry the
+    loss scale that fp16 training needs (not on the pages): fp32(g) times
+    fp32(1/S), then the coefficient, each one binary32 multiplication."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     n = g.size
     out = np.empty(n, dtype=np.uint16)
@@ -266,11 +302,15 @@ def adam_ex(g: np.ndarray, fmt: int, inv_scale: float, coef: float, master: np.n
 
 
 def sumsq_fmt(g: np.ndarray, fmt: int) -> float:
+    """Sum of squares of a 16-bit gradient in binary64, in element order: the
+    squared norm for the clip and overflow checks (not on the pages)."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     return float(_load().zo_sumsq_fmt(fmt, g.size, g.ctypes.data)) if g.size else 0.0
 
 
 def count_nonfinite_fmt(g: np.ndarray, fmt: int) -> int:
+    """Number of infinite or NaN elements of a 16-bit gradient (the overflow
+    check; not on the pages)."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     return int(_load().zo_count_nonfinite_fmt(fmt, g.size, g.ctypes.data)) if g.size else 0
 
@@ -287,11 +327,13 @@ def clip_coef(grad_norm: float, max_norm: float) -> float:
 
 
 def sumsq(g: np.ndarray) -> float:
+    """``sumsq_fmt`` for bf16 (not on the pages: the gradient norm's square)."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     return float(_load().zo_sumsq(g.size, g.ctypes.data)) if g.size else 0.0
 
 
 def count_nonfinite(g: np.ndarray) -> int:
+    """``count_nonfinite_fmt`` for bf16 (the overflow check; not on the pages)."""
     g = np.ascontiguousarray(g, dtype=np.uint16)
     return int(_load().zo_count_nonfinite(g.size, g.ctypes.data)) if g.size else 0
 
@@ -339,6 +381,10 @@ class Plan:
 
 
 def plan(numel: Sequence[int], layer_id: Sequence[int], n_ranks: int, bucket_elems: int) -> Plan:
+    """The flat layout, the N-way ownership partition ([T] section "ZeRO-1",
+    part "optimizer state 怎么切分"; reading in ``Plan``), the layers' flat
+    ranges ([T] section "ZeRO-3", one layer gathered at a time) and the
+    fixed-size buffer schedule (``bucket_schedule``: [M] section 3.3 "CB")."""
     assert n_ranks >= 1 and bucket_elems > 0 and bucket_elems % GRANULE == 0
     assert len(numel) == len(layer_id) and len(numel) >= 1
     assert all(n >= 0 for n in numel)
@@ -468,7 +514,10 @@ class StepReport:
 
 def init_states(plan_: Plan, stage: int, master0: np.ndarray, fmt: int = BF16) -> List[RankState]:
     """Every rank starts from the same fp32 master (pads 0), m = v = 0 and the
-    16-bit parameter copy equal to the master rounded to the format."""
+    16-bit parameter copy equal to the master rounded to the format: plain
+    DP's identical replicas ([T] section "先立一个基线"), each ZeRO stage
+    keeping of the fp32 states only the owned shard ([T] sections "ZeRO-1"
+    to "ZeRO-3") and stage 3 only the owned parameter shard."""
     assert master0.dtype == np.float32 and master0.size == plan_.psi_pad
     p16 = fmt_rne(master0, fmt)
     ranks = []
@@ -576,8 +625,11 @@ def step(plan_: Plan, stage: int, ranks: List[RankState], grads: GradFn, t: int,
 def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int, hp: AdamHP,
         clip_norm: float = 0.0, skip_nonfinite: bool = False, fmt: int = BF16, loss_scale: float = 1.0):
     """``steps`` optimizer steps; gradients for call k come from grads(k, r).
-    A skipped step does not advance the Adam step counter t, so the Adam
-    step number of call k is 1 + (calls before it that were not skipped)."""
+    Each step follows ``step``'s flow for the stage ([T] sections
+    "先立一个基线", "ZeRO-1", "ZeRO-2", "ZeRO-3").  A skipped step (the
+    overflow skip, not on the pages) does not advance the Adam step counter
+    t, so the Adam step number of call k is 1 + (calls before it that were
+    not skipped)."""
     ranks = init_states(plan_, stage, master0, fmt)
     reports = []
     t = 0
@@ -592,7 +644,8 @@ def run(plan_: Plan, stage: int, master0: np.ndarray, grads: GradFn, steps: int,
 
 def full_view(plan_: Plan, stage: int, ranks: List[RankState]) -> dict:
     """Assemble the flat master/m/v/params/grad (psi_pad each) from the ranks:
-    owned shards concatenated in rank order (rank 0's copy for DP)."""
+    owned shards concatenated in rank order (rank 0's copy for DP) -- the
+    inverse of the ownership partition of [T] section "ZeRO-1"."""
     if stage == STAGE_DP:
         r0 = ranks[0]
         return dict(master=r0.master, m=r0.m, v=r0.v, params=r0.params, grad=r0.grads)

@@ -182,7 +182,8 @@ void zo_rank_sum_f32(int32_t n_ranks, int64_t n, const uint16_t* const* rank_gra
 /* ----------------------------------------------------------------- Adam ---- */
 
 /*
- * Host scalars of Adam step t (t >= 1).  The hyper-parameters arrive as
+ * Host scalars of Adam step t (t >= 1), for the owner's update below ([T]
+ * sections "ZeRO-1" to "ZeRO-3", part "3. 更新").  The hyper-parameters arrive as
  * binary64 numbers (as a user writes them); every scalar the per-element
  * update uses is computed in binary64 and rounded once to binary32:
  *   out[0] = beta1            out[1] = beta2
@@ -352,6 +353,8 @@ void zo_adam_ex(int fmt, int64_t n, const uint16_t* g, float inv_scale, float co
   }
 }
 
+/* zo_sumsq and zo_count_nonfinite below for either 16-bit format (not on the
+ * pages: the norm and the overflow count of the optional clip and skip). */
 double zo_sumsq_fmt(int fmt, int64_t n, const uint16_t* g) {
   double acc = 0.0;
   for (int64_t i = 0; i < n; ++i) {
@@ -371,7 +374,8 @@ int64_t zo_count_nonfinite_fmt(int fmt, int64_t n, const uint16_t* g) {
 /* ----------------------------------------------- gradient norm / overflow ---- */
 
 /* Sum of squares of the averaged bf16 gradient, in binary64, index order.
- * (Not on the pages: a norm / overflow report, never a skip or a clip.) */
+ * (Not on the pages: the reported norm, which the optional global-norm clip
+ * and the overflow skip of the step flows also use.) */
 double zo_sumsq(int64_t n, const uint16_t* g) {
   double s = 0.0;
   for (int64_t i = 0; i < n; ++i) {
@@ -381,6 +385,8 @@ double zo_sumsq(int64_t n, const uint16_t* g) {
   return s;
 }
 
+/* Number of infinite or NaN elements of the averaged bf16 gradient (not on
+ * the pages: the overflow report and the optional skip's test). */
 int64_t zo_count_nonfinite(int64_t n, const uint16_t* g) {
   int64_t c = 0;
   for (int64_t i = 0; i < n; ++i)
