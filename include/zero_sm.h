@@ -273,7 +273,13 @@ int32_t zero_version(void);
 zero_status zero_init(const zero_layout* layout, int32_t n_ranks, int32_t stage,
                       int64_t bucket_elems, zero_ctx** out);
 
-/* Set an option (ZERO_OPT_*) before zero_bind.  ZERO_ESTATE after binding. */
+/* Set an option (ZERO_OPT_*).  ZERO_OPT_TIMING, ZERO_OPT_KERNEL, ZERO_OPT_PDL
+ * and the staged-kernel options (ZERO_OPT_TMA_GROUPS, ZERO_OPT_TMA_STAGES,
+ * ZERO_OPT_TMA_CTAS_PER_SM) may be set at any time; the others size or shape
+ * the arenas and are refused with ZERO_ESTATE once the context is bound.
+ * ZERO_EINVAL for an unknown key or a value out of range.
+ * Library plumbing: no passage of the pages defines it.
+ */
 zero_status zero_set_option(zero_ctx* ctx, int32_t key, int64_t value);
 
 /*
@@ -287,13 +293,23 @@ zero_status zero_set_option(zero_ctx* ctx, int32_t key, int64_t value);
  * instance a memory allocator that remembers the streams a block was used
  * on) must be finished by then.  Streams given here stay the caller's: the
  * context never destroys them, and they must outlive it.
+ * The overlap it serves is [T] section "ZeRO-2"'s reduce-scatter of a bucket
+ * while the backward of the next layers runs, and [T] section "ZeRO-3"'s
+ * per-layer gathers; the streams themselves are library plumbing.
  */
 zero_status zero_set_pipeline_streams(zero_ctx* ctx, void* callback_stream, void* kernel_stream);
 
-/* Sizes of the plan and of each arena (bytes).  Host only. */
+/* Sizes of the plan and of each arena (bytes).  Host only.
+ * The arenas are [M] section 3.4 "MD"'s one pre-allocated pool; the gradient
+ * arena's size is [M] section 3.3 "CB"'s fixed buffer, the gather arena [T]
+ * section "ZeRO-3"'s temporary full-layer buffer.
+ */
 zero_status zero_buffer_sizes(const zero_ctx* ctx, zero_sizes* out);
 
-/* Flat start of every tensor (host array of n_tensors). */
+/* Flat start of every tensor (host array of n_tensors).
+ * The flat layout behind [T] section "ZeRO-1"'s partition of the parameter
+ * vector (part "optimizer state 怎么切分").
+ */
 zero_status zero_tensor_offsets(const zero_ctx* ctx, int64_t* out, int32_t cap);
 
 /* The bucket schedule ([M] section 3.3; [T] section "ZeRO-2"): tensors
@@ -302,7 +318,10 @@ zero_status zero_tensor_offsets(const zero_ctx* ctx, int64_t* out, int32_t cap);
  * Writes min(cap, n) (lo, hi) pairs to lo_hi and returns n through *n_out. */
 zero_status zero_buckets(const zero_ctx* ctx, int64_t* lo_hi, int32_t cap, int32_t* n_out);
 
-/* Layer spans in layer order: (layer id, lo, hi) triples as int64. */
+/* Layer spans in layer order: (layer id, lo, hi) triples as int64.
+ * The layers of [T] section "ZeRO-3" (one layer's parameters gathered at a
+ * time).
+ */
 zero_status zero_layers(const zero_ctx* ctx, int64_t* id_lo_hi, int32_t cap, int32_t* n_out);
 
 /*
@@ -313,10 +332,14 @@ zero_status zero_layers(const zero_ctx* ctx, int64_t* id_lo_hi, int32_t cap, int
  * caller's; the library uses it until zero_destroy.
  * Errors: ZERO_EINVAL (null or misaligned), ZERO_ESTATE (already bound),
  * ZERO_ECUDA (device query failed).
+ * [M] section 3.4 "MD": one caller-owned pool, lifetimes managed inside it.
  */
 zero_status zero_bind(zero_ctx* ctx, void* const* arenas);
 
-/* Adam hyper-parameters (required before any update). */
+/* Adam hyper-parameters (required before any update).
+ * The Adam every page names ([T] sections "ZeRO-1" to "ZeRO-3", part "3.
+ * 更新").
+ */
 zero_status zero_set_hparams(zero_ctx* ctx, const zero_adam_hparams* hp);
 
 /*
@@ -327,6 +350,8 @@ zero_status zero_set_hparams(zero_ctx* ctx, const zero_adam_hparams* hp);
  * zeroes m, v and the reduced-gradient shards, writes bf16(master) (round to
  * nearest even) to every rank's parameter replica (stage 1, 2) or to the
  * parameter shards (stage 3), and resets the step counter to 0.
+ * Plain DP's identical starting replicas ([T] section "先立一个基线"), with the
+ * fp32 master, m and v of [M] section 1's state set.
  */
 zero_status zero_load_master(zero_ctx* ctx, const float* master_dev, void* stream);
 
@@ -354,11 +379,17 @@ zero_status zero_import_state(zero_ctx* ctx, const float* master, const float* e
  * CUDA graph advances it on every replay.  Both calls wait for the device
  * once the state is loaded.  Changing the betas (zero_set_hparams) rebuilds
  * the powers for the current t.
+ * The t of Adam's bias correction (the Adam of [T] sections "ZeRO-1" to
+ * "ZeRO-3", part "3. 更新").
  */
 zero_status zero_get_step(const zero_ctx* ctx, int64_t* t);
 zero_status zero_set_step(zero_ctx* ctx, int64_t t);
 
-/* Device pointer and element count of a view (ZERO_VIEW_*) for rank r. */
+/* Device pointer and element count of a view (ZERO_VIEW_*) for rank r.
+ * Which rank holds which state follows [T] sections "ZeRO-1" to "ZeRO-3"
+ * (owned shards of master, m, v; replicas or shards of the 16-bit
+ * parameters).
+ */
 zero_status zero_view(const zero_ctx* ctx, int32_t what, int32_t rank, void** ptr,
                       int64_t* n_elems);
 
@@ -491,6 +522,7 @@ zero_status zero_step(zero_ctx* ctx, zero_grad_fn grad_fn, void* grad_user,
  * zero_step; the intervals index straight into the replicas instead of
  * passing through the fixed-size buffer.  Stage 1 writes the all-reduced
  * gradient back into these replicas.
+ * The step of [T] sections "ZeRO-1" to "ZeRO-3", as zero_step.
  */
 zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
                                zero_gather_fn gather_fn, void* gather_user, void* stream,
@@ -508,6 +540,7 @@ zero_status zero_step_resident(zero_ctx* ctx, const void* const* rank_grads,
  * (4N at stage 1, the all-reduce written back) and the Adam-broadcast as
  * 2+24+2N (+2 at stage 3).  Resets the record.  At most 4096 launches are
  * recorded between two calls; later ones are not timed.
+ * Measurement plumbing: no passage of the pages defines it.
  */
 zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, double* model_bytes);
 
@@ -522,6 +555,7 @@ zero_status zero_kernel_timing(zero_ctx* ctx, double* ms, int64_t* launches, dou
  * layer at stage 3) plus two of those one-thread kernels.  Host only: reads a
  * counter kept by the launching calls, no device work and no wait.
  * ZERO_EINVAL for a NULL argument.
+ * Measurement plumbing: no passage of the pages defines it.
  */
 zero_status zero_launch_count(const zero_ctx* ctx, int64_t* n);
 
@@ -571,14 +605,21 @@ zero_status zero_fused_step_static(int32_t n_ranks, int64_t n, const void* const
 
 /* The fused-step kernel this context launches: *kernel = ZERO_KERNEL_REGISTER
  * or ZERO_KERNEL_TMA; for the staged kernel also its consumer groups and ring
- * depth (0 otherwise).  Host only. */
+ * depth (0 otherwise).  Host only.
+ * Library plumbing: no passage of the pages defines it.
+ */
 zero_status zero_fused_config(const zero_ctx* ctx, int32_t* kernel, int32_t* groups, int32_t* stages);
 
-/* Synchronise `stream` and read the last step's statistics. */
+/* Synchronise `stream` and read the last step's statistics.
+ * The norm and overflow count are not on the pages (the usual mixed-
+ * precision checks).
+ */
 zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
 
 /* Message of the last failure on ctx (never NULL; "" when none).  With
- * ctx == NULL: the reason the calling thread's last zero_init failed. */
+ * ctx == NULL: the reason the calling thread's last zero_init failed.
+ * Library plumbing: no passage of the pages defines it.
+ */
 const char* zero_last_error(const zero_ctx* ctx);
 
 /* Release a context (the arenas stay the caller's). NULL is a no-op.  Does
@@ -587,7 +628,9 @@ const char* zero_last_error(const zero_ctx* ctx);
  * reached that point (every call joins its side streams back into that
  * stream before it returns).  Streams and events the context created are
  * released once their work completes; streams given by
- * zero_set_pipeline_streams stay the caller's. */
+ * zero_set_pipeline_streams stay the caller's.
+ * Library plumbing: no passage of the pages defines it.
+ */
 void zero_destroy(zero_ctx* ctx);
 
 #ifdef __cplusplus
