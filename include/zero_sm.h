@@ -276,8 +276,9 @@ zero_status zero_init(const zero_layout* layout, int32_t n_ranks, int32_t stage,
 /* Set an option (ZERO_OPT_*).  ZERO_OPT_TIMING, ZERO_OPT_KERNEL, ZERO_OPT_PDL
  * and the staged-kernel options (ZERO_OPT_TMA_GROUPS, ZERO_OPT_TMA_STAGES,
  * ZERO_OPT_TMA_CTAS_PER_SM) may be set at any time; the others size or shape
- * the arenas and are refused with ZERO_ESTATE once the context is bound.
- * ZERO_EINVAL for an unknown key or a value out of range.
+ * the arenas and are refused with ZERO_ESTATE once the context is bound (so
+ * is an unknown key then).  ZERO_EINVAL for a value out of range, and before
+ * binding for an unknown key.
  * Library plumbing: no passage of the pages defines it.
  */
 zero_status zero_set_option(zero_ctx* ctx, int32_t key, int64_t value);
