@@ -2,6 +2,16 @@
 // for any N (loads straight into registers), the unfused reduce-scatter /
 // all-reduce, Adam, all-gather and the state initialisation.  Arithmetic and
 // helpers are in device_math.cuh.
+//
+// What each computes follows "ZERO训练技术": the all-reduce of section
+// "ZeRO-1" (part "2. 反向") and the reduce-scatter of section "ZeRO-2"
+// (the N ranks' gradients summed and averaged, each owner keeping its
+// shard), the owner's Adam update of its shard (sections "ZeRO-1" to
+// "ZeRO-3", part "3. 更新") and the all-gather of the updated 16-bit
+// parameters into every rank's copy (section "ZeRO-1", part "all-gather 是
+// 什么"; section "ZeRO-3" for the temporary full-layer buffers).  The fused
+// kernel does the three in one pass per element, since the N ranks are
+// buffers of one GPU.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

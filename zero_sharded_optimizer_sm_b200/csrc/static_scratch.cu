@@ -1,5 +1,6 @@
 // zero_fused_step_static: one fused ZeRO-2 step over a caller-described
-// interval that allocates nothing.
+// interval that allocates nothing ("ZERO训练技术" section "ZeRO-2":
+// reduce-scatter, update of the owned shard, all-gather, fused into one pass).
 //
 // Why it exists: the context-based entry points need the caller to allocate
 // and lend a scratch arena (zero_buffer_sizes / zero_bind).  Some callers

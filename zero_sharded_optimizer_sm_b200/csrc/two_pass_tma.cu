@@ -16,6 +16,11 @@
 //
 // Every wait is bounded (kWaitNs); one that runs out records an error code,
 // stops the producer, drains the copies in flight and ends the CTA.
+//
+// The passes compute the reduce-scatter / all-reduce and the update +
+// all-gather of "ZERO训练技术" sections "ZeRO-1" to "ZeRO-3"; the split into
+// two passes is for the global-norm clip and the overflow skip, which are not
+// on the pages (both need the whole step's norm before any update).
 #include <cuda_runtime.h>
 
 #include <algorithm>

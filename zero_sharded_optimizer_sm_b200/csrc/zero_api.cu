@@ -1,6 +1,13 @@
 // C ABI of the ZeRO optimizer-step library: validation, arena layout and the
 // executor that sequences the kernels of each stage.  Declarations and the
 // contract of every entry point are in include/zero_sm.h.
+//
+// The stage flows follow "ZERO训练技术" sections "ZeRO-1" (all-reduce, update
+// of the owned shard, all-gather), "ZeRO-2" (bucketed reduce-scatter as the
+// backward produces gradients, update, all-gather) and "ZeRO-3" (per-layer
+// gather into a temporary full-layer buffer that the next layer reuses); the
+// fixed-size gradient buffer and the one caller-owned pool are sections 3.3
+// "CB" and 3.4 "MD" of "ZeRO：从优化器状态到残差状态的显存优化".
 #include <cuda_runtime.h>
 
 #include <algorithm>
