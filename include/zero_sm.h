@@ -120,7 +120,7 @@ typedef struct zero_step_stats {
   int64_t skipped;         /* 1 when the step was skipped for non-finite gradients */
 } zero_step_stats;
 
-/* Options (zero_set_option, before zero_bind). */
+/* Options (zero_set_option): before zero_bind unless an entry says otherwise. */
 enum {
   ZERO_OPT_KEEP_GRAD_SHARDS = 1, /* stage 2/3: 1 (default) keeps the reduced bf16 gradient
                                     shards (GRAD_SHARDS arena; the fused step stores them and

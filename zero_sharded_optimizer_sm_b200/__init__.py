@@ -124,7 +124,7 @@ for _name, (_res, _args) in _SIGS.items():
     _fn.argtypes = _args
     globals()[_name] = _fn
 
-__all__ = list(_SIGS) + ["ZeroOptimizer", "AdamHParams", "ZeroError", "lib", "LIB_PATH"]
+__all__ = list(_SIGS) + ["ZeroOptimizer", "AdamHParams", "ZeroError", "lib", "LIB_PATH", "options_from_config"]
 
 
 class ZeroError(RuntimeError):
@@ -149,6 +149,60 @@ class AdamHParams:
     beta2: float = 0.999
     eps: float = 1e-8
     weight_decay: float = 0.0
+
+
+def options_from_config(cfg: dict) -> dict:
+    """``ZeroOptimizer`` keyword arguments from a DeepSpeed-style JSON config.
+
+    Reads the keys of the fixed-buffer snippet in "ZeRO：从优化器状态到残差状态
+    的显存优化" section 3.3 "CB" -- ``reduce_bucket_size``,
+    ``allgather_bucket_size`` (elements) and ``communication_data_type`` --
+    and the ZeRO ``stage``, either at the top level or under
+    ``zero_optimization``; every other key is left alone.
+
+    * ``reduce_bucket_size`` -> ``bucket_elems``, rounded up to a multiple of 8
+      (the granule every interval starts on).
+    * ``allgather_bucket_size``: the fused step gathers each interval in the
+      pass that reduces and updates it, so the gather bucket is the reduce
+      bucket; a different value raises ``ValueError`` instead of being
+      silently ignored (alone, it sets the bucket).
+    * ``communication_data_type``: "fp16" -> ZERO_DTYPE_F16, "bf16" /
+      "bfloat16" -> ZERO_DTYPE_BF16; anything else raises ``ValueError``
+      (the gradients and parameter copies are 16-bit here).
+    * ``stage``: 1, 2 or 3; 0 (plain data parallelism) raises, as
+      ``zero_init`` has no stage 0.
+    """
+    z = cfg.get("zero_optimization", {}) if isinstance(cfg.get("zero_optimization"), dict) else {}
+
+    def key(name):
+        return z[name] if name in z else cfg.get(name)
+
+    out = {}
+    stage = key("stage")
+    if stage is not None:
+        if int(stage) not in (1, 2, 3):
+            raise ValueError(f"stage {stage}: the library implements ZeRO stages 1, 2 and 3")
+        out["stage"] = int(stage)
+    rb, ab = key("reduce_bucket_size"), key("allgather_bucket_size")
+    if rb is not None and ab is not None and int(float(rb)) != int(float(ab)):
+        raise ValueError(f"allgather_bucket_size {ab} != reduce_bucket_size {rb}: the fused step gathers "
+                         "each interval as it reduces it, so the two buckets are one")
+    bucket = rb if rb is not None else ab
+    if bucket is not None:
+        b = int(float(bucket))
+        if b <= 0:
+            raise ValueError(f"bucket size {bucket} must be positive")
+        out["bucket_elems"] = (b + 7) // 8 * 8
+    dt = key("communication_data_type")
+    if dt is not None:
+        name = str(dt).lower()
+        if name in ("fp16", "float16", "half"):
+            out["dtype"] = ZERO_DTYPE_F16
+        elif name in ("bf16", "bfloat16"):
+            out["dtype"] = ZERO_DTYPE_BF16
+        else:
+            raise ValueError(f"communication_data_type {dt!r}: gradients and parameters are bf16 or fp16")
+    return out
 
 
 class ZeroOptimizer:
