@@ -243,3 +243,46 @@ def test_calls_out_of_order_and_bad_pointers_fail_cleanly():
     finally:
         z.zero_destroy(ctx)
     z.zero_destroy(None)
+
+
+def test_planner_matches_oracle_plan_on_random_layouts():
+    """Seeded random parameter lists (1-12 tensors, zero-size ones included,
+    random layer grouping), N in 1..128 and any bucket that is a multiple of
+    8: the library's flat offsets, padding, shard size, layer spans and
+    bucket schedule equal the oracle's."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    import zero_sharded_optimizer_sm_b200 as z
+
+    @st.composite
+    def layouts(draw):
+        n = draw(st.integers(1, 12))
+        numel = draw(st.lists(st.one_of(st.just(0), st.integers(1, 5000)), min_size=n, max_size=n))
+        if sum(numel) == 0:
+            numel[0] = draw(st.integers(1, 64))
+        steps = draw(st.lists(st.booleans(), min_size=n, max_size=n))
+        layer, cur = [], 0
+        for k in range(n):
+            cur += 1 if (k and steps[k]) else 0
+            layer.append(cur)
+        return numel, layer
+
+    @settings(max_examples=300, deadline=None, derandomize=True)
+    @given(layouts(), st.integers(1, 128), st.integers(1, 2500).map(lambda b: 8 * b), st.integers(1, 3))
+    def check(layout, n_ranks, bucket, stage):
+        numel, layer = layout
+        status, ctx = _init(numel, layer, n_ranks, stage, bucket)
+        assert status == 0
+        try:
+            sizes, buckets, layers = _plan_of(ctx)
+            p = oracle.plan(numel, layer, n_ranks, bucket)
+            assert (sizes.psi, sizes.psi_pad, sizes.shard) == (p.psi, p.psi_pad, p.shard)
+            assert buckets == p.buckets and layers == p.layers
+            offs = (ctypes.c_int64 * len(numel))()
+            assert z.zero_tensor_offsets(ctx, offs, len(numel)) == 0
+            assert list(offs) == p.offset
+        finally:
+            z.zero_destroy(ctx)
+
+    check()
