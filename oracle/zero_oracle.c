@@ -160,23 +160,31 @@ static uint16_t fmt_rne(int fmt, float x) { return fmt == ZO_F16 ? zo_f16_rne(x)
  *
  * rank_grads[r] points at element 0 of rank r's slice; n elements each.
  */
-void zo_reduce_mean(int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, uint16_t* out) {
+static float rank_sum(int fmt, int32_t n_ranks, const uint16_t* const* rank_grads, int64_t i) {
+  float acc = 0.0f;
+  for (int32_t r = 0; r < n_ranks; ++r) acc = acc + fmt_to_f32(fmt, rank_grads[r][i]);
+  return acc;
+}
+
+/* The averaged gradient in either 16-bit format (zo_reduce_mean is this
+ * function with ZO_BF16): the mean rounded once to the format.  Under a loss
+ * scale the ranks' gradients are S times the true ones and the mean is
+ * formed and rounded while still scaled, so that an overflow shows as Inf
+ * (mixed-precision convention; the pages only name fp16 as a communication
+ * type, [M] section 3.3). */
+void zo_reduce_mean_fmt(int fmt, int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, uint16_t* out) {
   const float inv_n = (float)(1.0 / (double)n_ranks);
-  for (int64_t i = 0; i < n; ++i) {
-    float acc = 0.0f;
-    for (int32_t r = 0; r < n_ranks; ++r) acc = acc + zo_bf16_to_f32(rank_grads[r][i]);
-    out[i] = zo_bf16_rne(acc * inv_n);
-  }
+  for (int64_t i = 0; i < n; ++i) out[i] = fmt_rne(fmt, rank_sum(fmt, n_ranks, rank_grads, i) * inv_n);
+}
+
+void zo_reduce_mean(int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, uint16_t* out) {
+  zo_reduce_mean_fmt(ZO_BF16, n_ranks, n, rank_grads, out);
 }
 
 /* Same sum in fp32 without the mean and the bf16 rounding, for the tests that
  * bound the accumulation error against the exact sum. */
 void zo_rank_sum_f32(int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, float* out) {
-  for (int64_t i = 0; i < n; ++i) {
-    float acc = 0.0f;
-    for (int32_t r = 0; r < n_ranks; ++r) acc = acc + zo_bf16_to_f32(rank_grads[r][i]);
-    out[i] = acc;
-  }
+  for (int64_t i = 0; i < n; ++i) out[i] = rank_sum(ZO_BF16, n_ranks, rank_grads, i);
 }
 
 /* ----------------------------------------------------------------- Adam ---- */
@@ -215,111 +223,28 @@ void zo_adam_scalars(double lr, double beta1, double beta2, double eps, double w
 /*
  * Mixed-precision Adam on one rank's owned elements ([T] section "ZeRO-1",
  * part "3. 更新"; [M] section 1 table for the state set: fp32 master weight,
- * fp32 first moment m, fp32 second moment v, 16-bit parameter copy).
+ * fp32 first moment m, fp32 second moment v, 16-bit parameter copy).  This is
+ * the oracle's only update loop; zo_adam and zo_adam_coef below call it.
  *
  * The pages name Adam but print no equation.  Reading: Adam with bias
  * correction (Kingma & Ba 2015, Algorithm 1) with decoupled weight decay
  * (Loshchilov & Hutter, AdamW), eps added after the square root of the
  * bias-corrected second moment.  Per element, each line one binary32 op
  * rounded to nearest even, in this order (scalars from zo_adam_scalars):
+ *   g  = fp32(g16) [* inv_scale when inv_scale != 1] [* coef when coef < 1]
  *   p  = p * decay
  *   m  = beta1*m + (1-beta1)*g        (both products rounded before the sum)
  *   v  = beta2*v + (1-beta2)*(g*g)
  *   mh = m / bc1 ;  vh = v / bc2
  *   p  = p - lr * (mh / (sqrt(vh) + eps))
- *   out = bf16(p)
- * g is the averaged bf16 gradient; master, m, v are updated in place.
+ *   out = 16-bit(p)
+ * g16 is the averaged gradient in storage format `fmt`; master, m, v are
+ * updated in place.  The two optional factors are the usual mixed-precision
+ * conventions, not on the pages beyond their mention of fp16 as the
+ * communication type: the ranks' gradients are S times the true ones under a
+ * loss scale S (inv_scale = fp32(1/S)), and a global-norm clipping
+ * coefficient scales the gradient when below 1 (see the oracle's clip_coef).
  */
-void zo_adam(int64_t n, const uint16_t* g, float* master, float* m, float* v, uint16_t* p_out,
-             double lr, double beta1, double beta2, double eps, double weight_decay, int64_t t) {
-  float s[9];
-  zo_adam_scalars(lr, beta1, beta2, eps, weight_decay, t, s);
-  const float b1 = s[0], b2 = s[1], omb1 = s[2], omb2 = s[3], bc1 = s[4], bc2 = s[5];
-  const float decay = s[6], lr_f = s[7], eps_f = s[8];
-  for (int64_t i = 0; i < n; ++i) {
-    const float gi = zo_bf16_to_f32(g[i]);
-    float p = master[i];
-    p = p * decay;
-    float a = b1 * m[i];
-    float b = omb1 * gi;
-    const float mi = a + b;
-    const float gg = gi * gi;
-    a = b2 * v[i];
-    b = omb2 * gg;
-    const float vi = a + b;
-    const float mh = mi / bc1;
-    const float vh = vi / bc2;
-    const float den = sqrtf(vh) + eps_f;
-    const float ratio = mh / den;
-    const float upd = lr_f * ratio;
-    p = p - upd;
-    master[i] = p;
-    m[i] = mi;
-    v[i] = vi;
-    if (p_out) p_out[i] = zo_bf16_rne(p);
-  }
-}
-
-/*
- * The same Adam update with the averaged gradient scaled first by a
- * global-norm clipping coefficient: g_used = fp32(g) * coef (one binary32
- * rounding) when coef < 1, g_used = fp32(g) otherwise (coef >= 1 means the
- * norm is within the limit and nothing is scaled).  Not on the pages: the
- * optional clipping of a mixed-precision step; see the oracle's clip_coef
- * for the coefficient.
- */
-void zo_adam_coef(int64_t n, const uint16_t* g, float coef, float* master, float* m, float* v,
-                  uint16_t* p_out, double lr, double beta1, double beta2, double eps,
-                  double weight_decay, int64_t t) {
-  float s[9];
-  zo_adam_scalars(lr, beta1, beta2, eps, weight_decay, t, s);
-  const float b1 = s[0], b2 = s[1], omb1 = s[2], omb2 = s[3], bc1 = s[4], bc2 = s[5];
-  const float decay = s[6], lr_f = s[7], eps_f = s[8];
-  for (int64_t i = 0; i < n; ++i) {
-    float gi = zo_bf16_to_f32(g[i]);
-    if (coef < 1.0f) gi = gi * coef;
-    float p = master[i];
-    p = p * decay;
-    float a = b1 * m[i];
-    float b = omb1 * gi;
-    const float mi = a + b;
-    const float gg = gi * gi;
-    a = b2 * v[i];
-    b = omb2 * gg;
-    const float vi = a + b;
-    const float mh = mi / bc1;
-    const float vh = vi / bc2;
-    const float den = sqrtf(vh) + eps_f;
-    const float ratio = mh / den;
-    const float upd = lr_f * ratio;
-    p = p - upd;
-    master[i] = p;
-    m[i] = mi;
-    v[i] = vi;
-    if (p_out) p_out[i] = zo_bf16_rne(p);
-  }
-}
-
-/*
- * The reduction and the update for either storage format, with a loss scale.
- * Mixed-precision training with 16-bit gradients multiplies the loss by a
- * scale S so that small gradients survive the 16-bit format; the gradients the
- * ranks hold are S times the true ones.  The averaged gradient is formed and
- * rounded to the format while still scaled (so an overflow shows as Inf), and
- * the update multiplies it by inv_scale = fp32(1/S) in binary32 first
- * (skipped when inv_scale is 1), then by the clipping coefficient when that is
- * below 1.  Not on the pages beyond their mention of fp16 as the
- * communication type; these are the usual mixed-precision conventions.
- */
-void zo_reduce_mean_fmt(int fmt, int32_t n_ranks, int64_t n, const uint16_t* const* rank_grads, uint16_t* out) {
-  const float inv_n = (float)(1.0 / (double)n_ranks);
-  for (int64_t i = 0; i < n; ++i) {
-    float acc = 0.0f;
-    for (int32_t r = 0; r < n_ranks; ++r) acc = acc + fmt_to_f32(fmt, rank_grads[r][i]);
-    out[i] = fmt_rne(fmt, acc * inv_n);
-  }
-}
-
 void zo_adam_ex(int fmt, int64_t n, const uint16_t* g, float inv_scale, float coef, float* master, float* m,
                 float* v, uint16_t* p_out, double lr, double beta1, double beta2, double eps,
                 double weight_decay, int64_t t) {
@@ -351,6 +276,20 @@ void zo_adam_ex(int fmt, int64_t n, const uint16_t* g, float inv_scale, float co
     v[i] = vi;
     if (p_out) p_out[i] = fmt_rne(fmt, p);
   }
+}
+
+/* The bf16 update without a loss scale or a clipping coefficient. */
+void zo_adam(int64_t n, const uint16_t* g, float* master, float* m, float* v, uint16_t* p_out,
+             double lr, double beta1, double beta2, double eps, double weight_decay, int64_t t) {
+  zo_adam_ex(ZO_BF16, n, g, 1.0f, 1.0f, master, m, v, p_out, lr, beta1, beta2, eps, weight_decay, t);
+}
+
+/* The bf16 update with the averaged gradient scaled first by a global-norm
+ * clipping coefficient (when coef < 1; coef >= 1 scales nothing). */
+void zo_adam_coef(int64_t n, const uint16_t* g, float coef, float* master, float* m, float* v,
+                  uint16_t* p_out, double lr, double beta1, double beta2, double eps,
+                  double weight_decay, int64_t t) {
+  zo_adam_ex(ZO_BF16, n, g, 1.0f, coef, master, m, v, p_out, lr, beta1, beta2, eps, weight_decay, t);
 }
 
 /* zo_sumsq and zo_count_nonfinite below for either 16-bit format (not on the

@@ -109,3 +109,26 @@ def test_stages_agree_under_clip_and_skip(clip):
     for v in views[1:]:
         for k in ("master", "m", "v", "params", "grad"):
             assert np.array_equal(v[k], views[0][k]), k
+
+
+def test_three_clipped_steps_match_torch():
+    """Three clipped steps against torch (clip_grad_norm_ on each step's
+    averaged gradient, then AdamW): from the second step on the moments are
+    non-zero, so a mistake in how the old moments enter the update shows
+    (step one starts from m = v = 0 and cannot see it)."""
+    p, m0, g = _setup([20000], [0], 4, 20000, 34, synth.Dist(synth.NORMAL, 1e-2))
+    hp = oracle.AdamHP(lr=1e-3, weight_decay=0.01)
+    w = torch.nn.Parameter(torch.from_numpy(m0.copy()))
+    opt = torch.optim.AdamW([w], lr=hp.lr, betas=(hp.beta1, hp.beta2), eps=hp.eps, weight_decay=0.01,
+                            foreach=False, fused=False)
+    for steps in (1, 2, 3):
+        ranks, reps = oracle.run(p, oracle.STAGE_Z2, m0, g, steps, hp, clip_norm=0.05)
+        assert reps[-1].coef < 0.5
+        view = oracle.full_view(p, oracle.STAGE_Z2, ranks)
+        w.grad = torch.from_numpy(oracle.bf16_to_f32(view["grad"]).copy())
+        torch.nn.utils.clip_grad_norm_([w], 0.05, foreach=False)
+        opt.step()
+        np.testing.assert_allclose(view["m"], opt.state[w]["exp_avg"].numpy(), rtol=1e-4, atol=1e-10)
+        np.testing.assert_allclose(view["v"], opt.state[w]["exp_avg_sq"].numpy(), rtol=1e-4, atol=1e-14)
+        np.testing.assert_allclose(view["master"], w.detach().numpy(), rtol=1e-6, atol=1e-6)
+        w.data.copy_(torch.from_numpy(view["master"].copy()))  # keep the two on the oracle's weights

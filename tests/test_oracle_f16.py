@@ -143,6 +143,11 @@ def test_fp16_adam_matches_torch_adamw_on_unscaled_gradient():
     opt.step()
     np.testing.assert_allclose(view["m"], opt.state[w]["exp_avg"].numpy(), rtol=2e-6, atol=1e-9)
     np.testing.assert_allclose(view["v"], opt.state[w]["exp_avg_sq"].numpy(), rtol=2e-6, atol=1e-13)
+    # the update itself: the weights' change against torch's (torch orders
+    # the same operations differently, hence a relative bound, not bits)
+    d_or = view["master"].astype(np.float64) - m0
+    d_tc = w.detach().numpy().astype(np.float64) - m0
+    assert np.all(np.abs(d_or - d_tc) <= 1e-4 * np.abs(d_tc) + np.spacing(np.abs(view["master"])) + 1e-10)
     assert np.array_equal(view["params"], oracle.f16_rne(view["master"]))
     assert math.isclose(reps[0].grad_norm, float(np.sqrt(np.sum(gavg.astype(np.float64) ** 2))), rel_tol=1e-12)
 
@@ -160,3 +165,25 @@ def test_fp16_stages_agree(scale):
     for v in views[1:]:
         for k in ("master", "m", "v", "params", "grad"):
             assert np.array_equal(v[k], views[0][k]), k
+
+
+def test_fp16_three_steps_match_torch_adamw():
+    """Three binary16 steps with loss scale 256 against torch's AdamW on the
+    unscaled averaged gradients: the second and third steps start from
+    non-zero moments, so a mistake in how the old moments enter shows."""
+    p, m0, g = _setup([20000], [0], 4, 20000, 74, 1e-2)
+    hp = oracle.AdamHP(lr=1e-3, weight_decay=0.01)
+    S = 256.0
+    w = torch.nn.Parameter(torch.from_numpy(m0.copy()))
+    opt = torch.optim.AdamW([w], lr=hp.lr, betas=(hp.beta1, hp.beta2), eps=hp.eps, weight_decay=0.01,
+                            foreach=False, fused=False)
+    for steps in (1, 2, 3):
+        ranks, _ = oracle.run(p, oracle.STAGE_Z2, m0, lambda k, r: g(k, r, S), steps, hp, fmt=oracle.F16,
+                              loss_scale=S)
+        view = oracle.full_view(p, oracle.STAGE_Z2, ranks)
+        w.grad = torch.from_numpy((oracle.f16_to_f32(view["grad"]) / np.float32(S)).astype(np.float32))
+        opt.step()
+        np.testing.assert_allclose(view["m"], opt.state[w]["exp_avg"].numpy(), rtol=1e-4, atol=1e-10)
+        np.testing.assert_allclose(view["v"], opt.state[w]["exp_avg_sq"].numpy(), rtol=1e-4, atol=1e-14)
+        np.testing.assert_allclose(view["master"], w.detach().numpy(), rtol=1e-6, atol=1e-6)
+        w.data.copy_(torch.from_numpy(view["master"].copy()))

@@ -15,74 +15,111 @@ import test_oracle_reduce as R
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "zero_oracle.c")
 
+import test_oracle_clip as C  # noqa: E402
+import test_oracle_f16 as F  # noqa: E402
+
+# Each arithmetic mistake is planted once: the oracle has one rank-order sum
+# (rank_sum) and one update loop (zo_adam_ex, which zo_adam and zo_adam_coef
+# call).  The update's mistakes are checked through each entry point's own
+# pins -- the plain bf16 update (zo_adam), the clipped one (zo_adam_coef) and
+# the binary16 one with a loss scale (zo_adam_ex) -- and every listed pin must
+# fail; the last mistakes break the forwarding of the entry points.
+def CLIP_PIN():
+    C.test_active_clip_matches_torch_clip_grad_norm_and_adamw()
+    C.test_three_clipped_steps_match_torch()
+
+
+def F16_PIN():
+    F.test_fp16_adam_matches_torch_adamw_on_unscaled_gradient()
+    F.test_fp16_three_steps_match_torch_adamw()
+
+
 MUTANTS = [
     ("bf16 truncates instead of rounding",
      "  if (d_tz < d_aw) return toward_zero;\n  if (d_aw < d_tz) return away;",
      "  return toward_zero;",
-     lambda: R.test_mean_exact_when_accumulation_exact(8)),
+     [lambda: R.test_mean_exact_when_accumulation_exact(8)]),
     ("ties round up instead of to even",
      "  return (toward_zero & 1u) ? away : toward_zero;",
      "  return away;",
-     lambda: B.test_bf16_rne_worked_cases(1.0 + 2.0**-8, 0x3F80)),
+     [lambda: B.test_bf16_rne_worked_cases(1.0 + 2.0**-8, 0x3F80)]),
     ("rank order reversed",
-     "    for (int32_t r = 0; r < n_ranks; ++r) acc = acc + zo_bf16_to_f32(rank_grads[r][i]);\n    out[i] = acc;",
-     "    for (int32_t r = n_ranks - 1; r >= 0; --r) acc = acc + zo_bf16_to_f32(rank_grads[r][i]);\n    out[i] = acc;",
-     R.test_rank_order_matters_and_is_zero_to_n_minus_1),
+     "  for (int32_t r = 0; r < n_ranks; ++r) acc = acc + fmt_to_f32(fmt, rank_grads[r][i]);",
+     "  for (int32_t r = n_ranks - 1; r >= 0; --r) acc = acc + fmt_to_f32(fmt, rank_grads[r][i]);",
+     [R.test_rank_order_matters_and_is_zero_to_n_minus_1]),
     ("mean not divided by N",
-     "    out[i] = zo_bf16_rne(acc * inv_n);",
-     "    out[i] = zo_bf16_rne(acc);",
-     lambda: R.test_mean_exact_when_accumulation_exact(4)),
+     "rank_sum(fmt, n_ranks, rank_grads, i) * inv_n)",
+     "rank_sum(fmt, n_ranks, rank_grads, i))",
+     [lambda: R.test_mean_exact_when_accumulation_exact(4), lambda: F.test_f16_mean_exact_when_accumulation_exact(4)]),
     ("bias correction of m dropped",
-     "    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    const float mh = mi;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     lambda: A.test_adam_matches_torch_adamw(0.0)),
+     "    const float mh = mi / bc1;",
+     "    const float mh = mi;",
+     [lambda: A.test_adam_matches_torch_adamw(0.0), CLIP_PIN, F16_PIN]),
     ("update sign flipped",
-     "    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    p = p + upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     A.test_first_step_moves_each_weight_by_lr_against_the_gradient_sign),
+     "    p = p - upd;",
+     "    p = p + upd;",
+     [A.test_first_step_moves_each_weight_by_lr_against_the_gradient_sign, CLIP_PIN, F16_PIN]),
     ("beta2 used for the first moment",
-     "    float a = b1 * m[i];\n    float b = omb1 * gi;\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    float a = b2 * m[i];\n    float b = omb1 * gi;\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     lambda: A.test_adam_matches_torch_adamw(0.0)),
+     "    float a = b1 * m[i];",
+     "    float a = b2 * m[i];",
+     [lambda: A.test_adam_matches_torch_adamw(0.0), CLIP_PIN, F16_PIN]),
     ("eps inside the square root",
-     "    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    const float den = sqrtf(vh + eps_f);\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     A.test_first_step_moves_each_weight_by_lr_against_the_gradient_sign),
+     "    const float den = sqrtf(vh) + eps_f;",
+     "    const float den = sqrtf(vh + eps_f);",
+     [A.test_first_step_moves_each_weight_by_lr_against_the_gradient_sign, CLIP_PIN, F16_PIN]),
     ("weight decay dropped",
-     "    const float gi = zo_bf16_to_f32(g[i]);\n    float p = master[i];\n    p = p * decay;",
-     "    const float gi = zo_bf16_to_f32(g[i]);\n    float p = master[i];",
-     A.test_weight_decay_alone_scales_weights_by_one_minus_lr_wd),
+     "    p = p * decay;\n",
+     "",
+     [A.test_weight_decay_alone_scales_weights_by_one_minus_lr_wd, CLIP_PIN, F16_PIN]),
     ("second moment from |g| instead of g^2",
-     "    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    const float gg = fabsf(gi);\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(3, 0.0)),
+     "    const float gg = gi * gi;",
+     "    const float gg = fabsf(gi);",
+     [lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(3, 0.0), CLIP_PIN, F16_PIN]),
     ("square root of the second moment dropped",
-     "    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    const float den = vh + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(-1, 0.0)),
+     "    const float den = sqrtf(vh) + eps_f;",
+     "    const float den = vh + eps_f;",
+     [lambda: I.test_power_of_two_gradient_scale_leaves_the_update_bits_unchanged(-1, 0.0), CLIP_PIN, F16_PIN]),
     ("first moment from |g|",
-     "    float b = omb1 * gi;\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     "    float b = omb1 * fabsf(gi);\n    const float mi = a + b;\n    const float gg = gi * gi;\n    a = b2 * v[i];\n    b = omb2 * gg;\n    const float vi = a + b;\n    const float mh = mi / bc1;\n    const float vh = vi / bc2;\n    const float den = sqrtf(vh) + eps_f;\n    const float ratio = mh / den;\n    const float upd = lr_f * ratio;\n    p = p - upd;\n    master[i] = p;\n    m[i] = mi;\n    v[i] = vi;\n    if (p_out) p_out[i] = zo_bf16_rne(p);\n  }\n}\n\n/*\n * The same Adam",
-     lambda: I.test_negated_gradients_negate_weights_and_first_moment_exactly(0.0)),
+     "    float b = omb1 * gi;",
+     "    float b = omb1 * fabsf(gi);",
+     [lambda: I.test_negated_gradients_negate_weights_and_first_moment_exactly(0.0), CLIP_PIN, F16_PIN]),
     ("bias-correction power off by one step",
      "  for (int64_t k = 0; k < t; ++k) {\n    p1 = p1 * beta1;",
      "  for (int64_t k = 0; k < t - 1; ++k) {\n    p1 = p1 * beta1;",
-     A.test_bias_correction_scalars),
+     [A.test_bias_correction_scalars]),
+    ("clipping coefficient not forwarded by zo_adam_coef",
+     "zo_adam_ex(ZO_BF16, n, g, 1.0f, coef,",
+     "zo_adam_ex(ZO_BF16, n, g, 1.0f, 1.0f,",
+     [CLIP_PIN]),
+    ("loss scale not applied",
+     "    if (inv_scale != 1.0f) gi = gi * inv_scale;\n",
+     "",
+     [F16_PIN]),
+    ("averaged gradient rounded to bf16 whatever the format",
+     "out[i] = fmt_rne(fmt, rank_sum(fmt, n_ranks, rank_grads, i) * inv_n);",
+     "out[i] = zo_bf16_rne(rank_sum(fmt, n_ranks, rank_grads, i) * inv_n);",
+     [lambda: F.test_f16_mean_exact_when_accumulation_exact(2)]),
+    ("parameters rounded to bf16 whatever the format",
+     "    if (p_out) p_out[i] = fmt_rne(fmt, p);",
+     "    if (p_out) p_out[i] = zo_bf16_rne(p);",
+     [F16_PIN]),
 ]
 
 
-@pytest.mark.parametrize("name,old,new,pin", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pin_catches_planted_mistake(tmp_path, name, old, new, pin):
+@pytest.mark.parametrize("name,old,new,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pin_catches_planted_mistake(tmp_path, name, old, new, pins):
     src = open(SRC).read()
     assert src.count(old) == 1, f"mutation site for '{name}' not found exactly once"
     mutant = tmp_path / "zero_oracle_mutant.c"
     mutant.write_text(src.replace(old, new))
     lib = obuild.build(src=str(mutant), out=str(tmp_path / "libzero_oracle_mutant.so"))
     with oracle.use_library(lib):
-        with pytest.raises(AssertionError):
-            pin()
-    # and the unmutated oracle passes the same pin
-    pin()
+        for pin in pins:
+            with pytest.raises(AssertionError):
+                pin()
+    # and the unmutated oracle passes the same pins
+    for pin in pins:
+        pin()
 
 
 # --- mistakes planted in the oracle's plan and collectives (Python side) ---
