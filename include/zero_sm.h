@@ -170,6 +170,13 @@ enum {
                                     at the end), so that their CTAs take the SMs that the
                                     callbacks' work frees first.  Values are unchanged.
                                     Default 0; before zero_bind */
+  ZERO_OPT_TMA_TILE = 13,        /* bulk-store kernel: elements per tile, 1024 or 2048 (0 = the
+                                    library's choice); may be set at any time */
+  ZERO_OPT_TMA_WARPS = 14,       /* bulk-store kernel: consumer warps, 4, 8 or 16, with 8 or 4
+                                    elements per lane (0 = the library's choice); the built
+                                    (tile, warps) pairs are 2048 x 8, 2048 x 16, 1024 x 4,
+                                    1024 x 8 and 1024 x 16; another pair makes the next fused
+                                    launch fail with ZERO_ECUDA; may be set at any time */
   ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
                                     with no gather_fn) launches its fused kernels with
                                     programmatic dependent launch, so that each launch's CTAs
@@ -203,9 +210,18 @@ enum { ZERO_DTYPE_BF16 = 0, ZERO_DTYPE_F16 = 1 };
  *             bounded; one that runs out is reported as ZERO_ECUDA by the next
  *             synchronising call (zero_read_stats, zero_step with stats,
  *             zero_kernel_timing).
+ *   BULK:     (N <= 16) the staged loads of TMA with bulk stores: one CTA
+ *             per SM, a producer thread streaming tiles (ZERO_OPT_TMA_TILE) of
+ *             the N replicas and master/m/v into a ring of shared-memory
+ *             stages, consumer warps (ZERO_OPT_TMA_WARPS) that compute and
+ *             write every result back into the stage, and a storer thread
+ *             that copies the stage's results to master/m/v and the N
+ *             destinations with bulk copies (shared -> global), so that no
+ *             consumer lane issues a global store.  Bounded waits as TMA.
+ *             Above N = 16 the rank-chunked TMA kernel runs instead.
  *   AUTO:     the staged kernel for every N, in the configuration measured
  *             fastest on B200 for that N (zero_fused_config reports it). */
-enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2 };
+enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2, ZERO_KERNEL_BULK = 3 };
 
 /* Views (zero_view). */
 enum {
@@ -266,7 +282,8 @@ int32_t zero_version(void);
  * Plan a context for `layout` over n_ranks logical ranks (1..ZERO_MAX_RANKS)
  * at `stage` (ZERO_STAGE_1..3; ZERO_STAGE_DP returns ZERO_ENOTIMPL), with the
  * fixed communication buffer of bucket_elems elements per rank ([M] section
- * 3.3 "CB"; > 0, multiple of 8).  Host only, no device work.  *out receives
+ * 3.3 "CB"; a positive multiple of 8, or 0 for one bucket spanning the whole
+ * padded flat space).  Host only, no device work.  *out receives
  * a context owned by the caller (free with zero_destroy).
  * Errors: ZERO_EINVAL for null pointers, bad sizes or decreasing layer ids.
  */
@@ -476,8 +493,23 @@ zero_status zero_all_reduce(zero_ctx* ctx, int64_t lo, int64_t hi, void* const* 
  *   p = p - lr*((m/(1-b1^t)) / (sqrt(v/(1-b2^t)) + eps));  out = bf16(p).
  * g is the reduced bf16 gradient (stage 2/3: GRAD_SHARDS; stage 1: the
  * owner's full replica in GRADS).  out goes to the owner's own parameter
- * replica (stage 1/2) or to the parameter shards (stage 3).  Does not change
- * the context's step counter (zero_set_step does).
+ * replica (stage 1/2) or to the parameter shards (stage 3).
+ * The step number and the context's step counter (the count of completed
+ * steps that zero_step / zero_step_resident use and advance, kept on the
+ * device):
+ *   t >= 1  the caller's step number is used; the counter is neither read
+ *           nor changed.  A caller that mixes explicit-t calls with fused
+ *           steps sets the counter with zero_set_step(ctx, k) after its k-th
+ *           unfused step, so that the next zero_step runs step k + 1.
+ *   t = 0   the step after the counter's value is used (the device is
+ *           synchronised to read it); with rank = -1 the call completes that
+ *           step and advances the counter by one (again synchronising), with
+ *           rank >= 0 the counter is left for the caller to advance
+ *           (zero_set_step, or a final rank = -1 call of the same step is NOT
+ *           the way: it would update every shard a second time).
+ * Errors: ZERO_EINVAL (rank out of range, t < 0), ZERO_ESTATE (not bound,
+ * not initialised, hyper-parameters not set, or the gradient buffers it reads
+ * were dropped), ZERO_ECUDA (launch, or reading / writing the counter).
  */
 zero_status zero_adam_shard(zero_ctx* ctx, int32_t rank, int64_t t, void* stream);
 
@@ -580,36 +612,69 @@ zero_status zero_launch_count(const zero_ctx* ctx, int64_t* n);
  *   stats_out    NULL, or a device pointer to 16 bytes that receives the
  *                step's sum of squares of the averaged gradient (double) and
  *                its non-finite count (uint64)
- * n must be a multiple of 8 and 1 <= n_ranks <= ZERO_MAX_RANKS.  The values
- * computed are those of zero_step for a stage-2 context whose single bucket
- * is this interval.
+ * n must be a multiple of 8 and 1 <= n_ranks <= ZERO_MAX_RANKS.  master, m,
+ * v and the parameters are those of zero_step for a stage-2 context whose
+ * single bucket is this interval, bit for bit; the sum of squares in
+ * stats_out is the same sum added in another order (per CTA of this call's
+ * own grid), so it may differ from the context step's in the last bits; the
+ * non-finite count is exact.  beta^t is formed on the host by t binary64
+ * products on every call (no state survives between calls), so a call at
+ * step t costs O(t) host time until both powers reach 0.
  *
  * The kernel's scratch (per-CTA norm partials, an arrival counter and the
  * step's sums) is a 32 KiB + 64 B array in the library's device memory,
  * reserved on every GPU that loads the library until the process exits; it
- * holds partials for at most 2048 CTAs, and a launch that would need more
- * returns ZERO_ENOMEM.  Every call on a device shares that array and it keeps
- * the previous call's contents (the call clears what must start at zero), so
- * two calls that may run at the same time on the GPU -- on different streams
- * with no ordering between them -- race and give wrong statistics; calls
+ * holds partials for 2048 CTAs, and a launch takes at most that many CTAs
+ * (the kernel loops over any n).  Every call on a device shares that array
+ * and it keeps the previous call's contents (the call clears what must start
+ * at zero), so two calls that may run at the same time on the GPU -- on
+ * different streams with no ordering between them -- race: the statistics
+ * are wrong, and stats_out may receive an earlier call's sums with nothing
+ * to tell them apart (master, m, v and the parameters are unaffected); calls
  * ordered on one stream are safe.  The first call on each device looks up the
  * array's device address with that device current (a one-time set-up); make
  * that first call before any stream capture begins.
  * Errors: ZERO_EINVAL (bad size, pointer, alignment or hyper-parameter),
- * ZERO_ENOMEM (scratch too small for the launch), ZERO_ECUDA (set-up or launch
- * failed).
+ * ZERO_ECUDA (set-up or launch failed).
  */
 zero_status zero_fused_step_static(int32_t n_ranks, int64_t n, const void* const* rank_grads,
                                    float* master, float* exp_avg, float* exp_avg_sq,
                                    void* const* rank_params, const zero_adam_hparams* hp,
                                    int64_t t, void* stats_out, void* stream);
 
-/* The fused-step kernel this context launches: *kernel = ZERO_KERNEL_REGISTER
- * or ZERO_KERNEL_TMA; for the staged kernel also its consumer groups and ring
- * depth (0 otherwise).  Host only.
+/* The fused-step kernel this context launches: *kernel = ZERO_KERNEL_REGISTER,
+ * ZERO_KERNEL_TMA or ZERO_KERNEL_BULK; for a staged kernel also its consumer
+ * groups (BULK: its consumer warps) and ring depth (0 otherwise).  Host only.
  * Library plumbing: no passage of the pages defines it.
  */
 zero_status zero_fused_config(const zero_ctx* ctx, int32_t* kernel, int32_t* groups, int32_t* stages);
+
+/* Elements per tile of the staged kernel this context launches (0 for the
+ * register kernel).  Host only.  Library plumbing: no passage defines it. */
+zero_status zero_fused_tile(const zero_ctx* ctx, int32_t* tile);
+
+/*
+ * zero_probe_pattern -- the ceiling of the step's own memory traffic on this
+ * device.  Enqueues on `stream`, for every interval of the step in the step's
+ * order and launch chaining, the movement-only twin of the bulk-store kernel
+ * in this context's configuration: the same bulk loads of the N gradient
+ * slices (rank_grads, as for zero_step_resident) and of master/m/v, the same
+ * shared-memory reads and writes, the same bulk stores of master/m/v, of the
+ * N parameter destinations, of the ZeRO-3 shard and of the ZeRO-1 write-back
+ * or reduced shard -- with no reduction and no Adam: master/m/v are stored
+ * back unchanged and the destinations receive the 16-bit rounding of the
+ * unchanged master weights.  So a probe leaves the optimizer state and the
+ * parameters as a step left them (the ZeRO-1 write-back and the reduced
+ * shards receive an XOR of the gradient slices; the step statistics are
+ * overwritten with zeros); the step counter does not move.  Timed against
+ * the step's byte model it gives the fraction of the traffic pattern's own
+ * ceiling that the step reaches.  Not part of the method: no passage of the
+ * pages defines it; measurement plumbing.
+ * Errors: ZERO_EINVAL (NULL or misaligned pointers), ZERO_ESTATE (not bound
+ * or not initialised), ZERO_ENOTIMPL (N > 16, or the configuration of
+ * ZERO_OPT_TMA_TILE / ZERO_OPT_TMA_WARPS is not built), ZERO_ECUDA (launch).
+ */
+zero_status zero_probe_pattern(zero_ctx* ctx, const void* const* rank_grads, void* stream);
 
 /* Synchronise `stream` and read the last step's statistics.
  * The norm and overflow count are not on the pages (the usual mixed-
@@ -633,6 +698,141 @@ const char* zero_last_error(const zero_ctx* ctx);
  * Library plumbing: no passage of the pages defines it.
  */
 void zero_destroy(zero_ctx* ctx);
+
+/* ------------------------------------------------ one logical rank per GPU -- */
+/*
+ * The same step with each data-parallel rank on its own GPU, one process per
+ * GPU ([T] sections "ZeRO-1" and "ZeRO-2"; the pages tie ZeRO's cost to the
+ * bandwidth between the ranks' devices: [T] section "ZeRO-3", the list of
+ * what it is sensitive to, and [M] section 6).  Rank r keeps, in its own
+ * GPU's memory and in arenas the caller allocates:
+ *   GRAD    its 16-bit gradient replica, psi_pad elements (its backward's
+ *           output; stage 1 also receives the all-reduced gradient here)
+ *   PARAM   its 16-bit parameter replica, psi_pad elements
+ *   STATES  fp32 master, m and v of its owned shard [rS, (r+1)S)
+ *   SCRATCH the step's norm partials and counters
+ * Every rank exports its GRAD and PARAM arenas as CUDA IPC records
+ * (zero_dist_export), the caller exchanges the records (for instance with
+ * torch.distributed all_gather_object) and every rank opens the others'
+ * (zero_dist_open_peers).  zero_dist_step then launches, on this GPU, one
+ * kernel over the owned shard that reads the N ranks' gradient slices (the
+ * peers' through the peer mapping) with plain 16-byte loads, sums them in
+ * rank order 0..N-1 in binary32, multiplies by fp32(1/N), rounds to bf16,
+ * runs Adam (zero_adam_shard's equations) on the owned fp32 states, and
+ * stores bf16(master) into the shard's range of every rank's PARAM replica
+ * (stage 1: also the averaged gradient into every rank's GRAD replica): the
+ * reduce-scatter, the update and the all-gather in one pass, the same bits
+ * as the single-device step and the oracle.  No bulk copy or multicast reads
+ * another GPU's memory.
+ *
+ * Ordering between the ranks is the caller's, on the host: every rank's GRAD
+ * replica of the step is complete before any rank calls zero_dist_step (for
+ * instance: synchronise the stream of the backward, then a barrier), and no
+ * rank reads its PARAM replica or writes its GRAD replica again before every
+ * rank's step has completed (synchronise the step's stream, then a barrier).
+ * zero_dist_load_master has the same contract as a step.  No kernel of this
+ * API waits on another rank.
+ *
+ * Errors as for the single-device context: status codes, the text in
+ * zero_dist_last_error.  Stages 1 and 2; stage 3 returns ZERO_ENOTIMPL.
+ */
+typedef struct zero_dist zero_dist;
+
+enum {
+  ZERO_DIST_ARENA_GRAD = 0,
+  ZERO_DIST_ARENA_PARAM = 1,
+  ZERO_DIST_ARENA_STATES = 2,
+  ZERO_DIST_ARENA_SCRATCH = 3,
+  ZERO_DIST_NUM_ARENAS = 4
+};
+
+/* Bytes of one rank's export record (two CUDA IPC handles with the arenas'
+ * offsets in their allocations and their lengths; zero padded). */
+#define ZERO_DIST_HANDLE_BYTES 192
+
+/* Plan rank `rank` of `world` ranks (1..ZERO_MAX_RANKS) at `stage` (1 or 2):
+ * the same partition as zero_init (S = psi_pad / world).  Host only.
+ * ZERO_EINVAL for bad arguments, ZERO_ENOTIMPL for stage 3 or DP. */
+zero_status zero_dist_init(const zero_layout* layout, int32_t world, int32_t rank, int32_t stage,
+                           zero_dist** out);
+
+/* plan = {psi, psi_pad, shard}; arena_bytes[ZERO_DIST_NUM_ARENAS].  Either
+ * may be NULL.  Host only. */
+zero_status zero_dist_sizes(const zero_dist* d, int64_t plan[3], int64_t arena_bytes[ZERO_DIST_NUM_ARENAS]);
+
+/* Flat offset of every tensor (cap >= n_tensors).  Host only. */
+zero_status zero_dist_tensor_offsets(const zero_dist* d, int64_t* out, int32_t cap);
+
+/* Bind this rank's arenas: device pointers on the current device, 256-byte
+ * aligned, caller-owned, at least zero_dist_sizes bytes each.  GRAD and PARAM
+ * must come from device allocations that CUDA IPC can export (cudaMalloc and
+ * allocators built on it; not virtual-memory-managed pools).  Zeroes SCRATCH
+ * (synchronously).  With world = 1 no peer needs opening. */
+zero_status zero_dist_bind(zero_dist* d, void* const* arenas);
+
+/* Write this rank's export record (ZERO_DIST_HANDLE_BYTES bytes) to `record`:
+ * the IPC handles of the allocations holding its GRAD and PARAM arenas and
+ * the arenas' offsets in them.  The allocations must stay alive while any
+ * peer has them open. */
+zero_status zero_dist_export(zero_dist* d, void* record);
+
+/* Open the peers' arenas from `records`: world records in rank order, each
+ * ZERO_DIST_HANDLE_BYTES bytes (this rank's own is ignored).  Each distinct
+ * allocation is opened once (cudaIpcOpenMemHandle with lazy peer access) and
+ * closed by zero_dist_destroy.  ZERO_EINVAL when a record does not describe
+ * arenas of this layout's sizes, ZERO_ECUDA when a handle cannot be opened. */
+zero_status zero_dist_open_peers(zero_dist* d, const void* records);
+
+/* Adam hyper-parameters (as zero_set_hparams). */
+zero_status zero_dist_set_hparams(zero_dist* d, const zero_adam_hparams* hp);
+
+/* Initialise from fp32 master weights: master_full is a device array of
+ * psi_pad fp32 values on this GPU (pads 0); the rank copies its shard into
+ * STATES, sets m = v = 0 and the step counter to 0, and writes bf16(master)
+ * of its shard into every rank's PARAM replica (so that, once every rank has
+ * loaded, every replica holds all of them).  Enqueued on `stream`. */
+zero_status zero_dist_load_master(zero_dist* d, const float* master_full, void* stream);
+
+/* One fused step (t = completed steps + 1) over this rank's shard, enqueued
+ * on `stream`, as described above; records this rank's share of the
+ * gradient norm (sum of squares and non-finite count of its shard's
+ * averaged gradient) for zero_dist_read_partial.  The global norm is the
+ * square root of the ranks' sums, added in rank order. */
+zero_status zero_dist_step(zero_dist* d, void* stream);
+
+/* Adam on this rank's shard from an already reduced 16-bit gradient shard
+ * (grad_shard: S values on this GPU, 16-byte aligned) -- for a caller whose
+ * reduce-scatter and all-gather are collective-library calls (NCCL): the
+ * update writes bf16(master) into this rank's own PARAM replica at [rS,
+ * (r+1)S) only, and advances the step counter. */
+zero_status zero_dist_adam_shard(zero_dist* d, const void* grad_shard, void* stream);
+
+/* Synchronise `stream` and read the last step's partial statistics (sum of
+ * squares of this shard's averaged gradient, its non-finite count) and the
+ * step counter (step may be NULL). */
+zero_status zero_dist_read_partial(zero_dist* d, void* stream, double* sumsq, int64_t* nonfinite, int64_t* step);
+
+/* The step's global statistics from the ranks' partials (host only, no
+ * device work): norm = sqrt of sumsq[0] + ... + sumsq[world-1] added in rank
+ * order in binary64, and the non-finite counts summed -- the same bits on
+ * every rank that passes the same partials.  Not on the pages (the usual
+ * mixed-precision norm and overflow report). */
+zero_status zero_dist_combine_partials(int32_t world, const double* sumsq, const int64_t* nonfinite, double* norm,
+                                       int64_t* nonfinite_total);
+
+/* Local device pointer and length of ZERO_VIEW_MASTER / _EXP_AVG /
+ * _EXP_AVG_SQ (the owned shard, S) or ZERO_VIEW_PARAM / ZERO_VIEW_GRAD_BUF
+ * (this rank's replicas, psi_pad). */
+zero_status zero_dist_view(const zero_dist* d, int32_t what, void** ptr, int64_t* n_elems);
+
+/* Message of the last failure (d == NULL: of the calling thread's last
+ * zero_dist_init). */
+const char* zero_dist_last_error(const zero_dist* d);
+
+/* Close the peers' mappings and release the context (the arenas stay the
+ * caller's).  Does not wait for the device: the caller synchronises first,
+ * and no peer may still run a step that writes this rank's replicas. */
+void zero_dist_destroy(zero_dist* d);
 
 #ifdef __cplusplus
 }

@@ -198,7 +198,7 @@ def test_init_rejects_bad_arguments():
     assert _init([8], [0], 2, 4, 8)[0] == z.ZERO_EINVAL            # no such stage
     assert _init([8], [0], 2, 0, 8)[0] == z.ZERO_ENOTIMPL          # plain DP is oracle-only
     assert _init([8], [0], 2, 2, 12)[0] == z.ZERO_EINVAL           # bucket not a multiple of 8
-    assert _init([8], [0], 2, 2, 0)[0] == z.ZERO_EINVAL
+    assert _init([8], [0], 2, 2, -8)[0] == z.ZERO_EINVAL           # negative bucket (0 = one bucket)
     assert _init([8, 8], [1, 0], 2, 2, 8)[0] == z.ZERO_EINVAL      # decreasing layer ids
     assert b"non-decreasing" in z.zero_last_error(None)
     assert _init([8, -1], [0, 0], 2, 2, 8)[0] == z.ZERO_EINVAL     # negative size
@@ -286,3 +286,28 @@ def test_planner_matches_oracle_plan_on_random_layouts():
             z.zero_destroy(ctx)
 
     check()
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("n_ranks", [1, 3, 8, 64])
+def test_bucket_zero_is_one_bucket_over_the_padded_space(layout, n_ranks):
+    """bucket_elems = 0 asks the library for one bucket spanning the padded
+    flat space: the same plan as the oracle's with a bucket of psi_pad
+    elements (the binding passes 0 when no bucket is given)."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    numel, layer = layout
+    for stage in (1, 2, 3):
+        st, ctx = _init(numel, layer, n_ranks, stage, 0)
+        assert st == 0
+        try:
+            sizes, buckets, layers = _plan_of(ctx)
+            p_any = oracle.plan(numel, layer, n_ranks, 8)
+            p = oracle.plan(numel, layer, n_ranks, p_any.psi_pad)
+            assert buckets == p.buckets
+            assert len(buckets) == 1 and buckets[0][1] - buckets[0][0] <= p.psi_pad
+            assert layers == p.layers and sizes.psi_pad == p.psi_pad
+            if stage == 2:
+                assert sizes.arena_bytes[z.ZERO_ARENA_GRADS] >= 2 * p.psi_pad * n_ranks
+        finally:
+            z.zero_destroy(ctx)

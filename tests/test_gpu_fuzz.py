@@ -50,9 +50,14 @@ def _case(k):
     f16 = bool(rng.random() < 0.4)
     scale = float(rng.choice([1.0, 256.0])) if f16 else 1.0
     clip = float(rng.choice([0.0, 0.0, 0.02, 1e9]))
-    return dict(numel=numel, layer=layer, n_ranks=n_ranks, stage=stage, bucket=bucket, f16=f16, scale=scale,
-                clip=clip, pipeline=int(rng.integers(0, 3)), pdl=bool(rng.random() < 0.5),
-                kernel=int(rng.choice([0, 0, 1])), seed=0xF100 + k)
+    c = dict(numel=numel, layer=layer, n_ranks=n_ranks, stage=stage, bucket=bucket, f16=f16, scale=scale,
+             clip=clip, pipeline=int(rng.integers(0, 3)), pdl=bool(rng.random() < 0.5),
+             kernel=int(rng.choice([0, 0, 1])), seed=0xF100 + k, tile=0, warps=0)
+    # drawn last, so that the fields above stay those of the seed
+    if rng.random() < 0.4:
+        c["kernel"] = 3  # the bulk-store staged kernel, in one of its built configurations
+        c["tile"], c["warps"] = [(2048, 8), (2048, 16), (1024, 4), (1024, 8), (1024, 16)][int(rng.integers(0, 5))]
+    return c
 
 
 @pytest.mark.parametrize("k", range(N_CASES))
@@ -76,6 +81,7 @@ def test_random_configuration_against_the_oracle(k):
 
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, c["stage"], bucket_elems=c["bucket"],
                           hparams=z.AdamHParams(**w.hyper.__dict__), kernel=c["kernel"], pipeline=c["pipeline"],
+                          tma_tile=c["tile"], tma_warps=c["warps"],
                           dtype=z.ZERO_DTYPE_F16 if c["f16"] else z.ZERO_DTYPE_BF16)
     opt.set_pdl(c["pdl"])
     if c["scale"] != 1.0:

@@ -46,18 +46,21 @@ def _hp(w):
     return z.AdamHParams(**w.hyper.__dict__)
 
 
-REG, TMA = 1, 2  # ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA
-# fused-kernel variants: the register path, the staged path with one and two groups
+REG, TMA, BULK = 1, 2, 3  # ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA, ZERO_KERNEL_BULK
+# fused-kernel variants: the register path, the staged path with one and two
+# groups, one wide group, the rank-chunked form; the bulk-store staged kernel
 VARIANTS = {"reg": dict(kernel=REG), "tma1": dict(kernel=TMA, tma_groups=1),
             "tma2": dict(kernel=TMA, tma_groups=2), "tmaw": dict(kernel=TMA, tma_groups=3),
-            "tmac": dict(kernel=TMA)}
+            "tmac": dict(kernel=TMA), "blk": dict(kernel=BULK),
+            "blk2k16": dict(kernel=BULK, tma_tile=2048, tma_warps=16)}
 
 
 def kernels_for(n_ranks):
-    """Fused-kernel variants at this N: register, and the staged kernel with one
-    group, two groups and one wide group (N <= 16) or its rank-chunked form
+    """Fused-kernel variants at this N: register, the staged kernel with one
+    group, two groups and one wide group, and the bulk-store kernel in two
+    configurations (N <= 16); register and the rank-chunked staged kernel
     (N > 16)."""
-    return ("reg", "tma1", "tma2", "tmaw") if n_ranks <= 16 else ("reg", "tmac")
+    return ("reg", "tma1", "tma2", "tmaw", "blk", "blk2k16") if n_ranks <= 16 else ("reg", "tmac")
 
 
 def make_opt(w, stage, bucket=None, keep=True, variant=None, **kw):
@@ -264,6 +267,46 @@ def test_unfused_calls_equal_fused_step(stage):
             assert torch.equal(fused.view(z.ZERO_VIEW_GATHER, r)[: hi - lo], split.view(z.ZERO_VIEW_GATHER, r)[: hi - lo])
     fused.close()
     split.close()
+
+
+@pytest.mark.parametrize("stage", [1, 2, 3])
+def test_adam_shard_step_counter_mixed_with_fused_steps(stage):
+    """Unfused steps that take the context's step counter (t = 0, every
+    shard) advance it, so a fused step after two of them is step 3; explicit
+    steps t = 1, 2 leave it, and zero_set_step(2) puts it in line.  Both
+    mixes end bit for bit on the oracle's three steps."""
+    z = _z()
+    numel, layer = W.transformer_layers(2, 64, 256)
+    w = W.Workload("mixed-t", numel, layer, 4, (stage,), 8192, synth.Dist(synth.NORMAL, 1e-2, zero_mod=9),
+                   W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01), 0x7A0 + stage)
+    p, ranks, reps = _oracle_run(w, stage, 8192)
+    ref = oracle.full_view(p, STAGE_OF[stage], ranks)
+    s = torch.cuda.current_stream().cuda_stream
+    for explicit in (False, True):
+        opt, fill = make_opt(w, stage, bucket=8192)
+        gfn = grad_fn_for(opt, fill)
+        intervals = opt.buckets() if stage != 3 else [(lo, hi) for _, lo, hi in reversed(opt.layers())]
+        for t in (1, 2):
+            for lo, hi in intervals:
+                if stage == 1:
+                    bufs = [opt.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() + 2 * lo for r in range(w.n_ranks)]
+                    gfn(t, lo, hi, bufs, s)
+                    opt.all_reduce(lo, hi)
+                else:
+                    bufs = [opt.view(z.ZERO_VIEW_GRAD_BUF, r).data_ptr() for r in range(w.n_ranks)]
+                    gfn(t, lo, hi, bufs, s)
+                    opt.reduce_scatter(lo, hi)
+            opt.adam_shard(-1, t if explicit else 0)
+            for lo, hi in intervals:
+                opt.all_gather(lo, hi)
+            assert opt.t == (0 if explicit else t)
+        if explicit:
+            opt.t = 2
+        st = opt.step(gfn, stats=True)
+        assert st["step"] == 3 and st["nonfinite"] == reps[2].nonfinite
+        for k, view in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+            assert_bits_equal(to_np(opt.view(view)), ref[k], f"stage {stage} explicit {explicit} {k}")
+        opt.close()
 
 
 def test_adam_shard_per_rank_equals_all_ranks():

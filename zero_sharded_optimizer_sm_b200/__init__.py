@@ -38,7 +38,7 @@ ZERO_MAX_RANKS = 128
 (ZERO_ARENA_STATES, ZERO_ARENA_PARAMS, ZERO_ARENA_GRADS, ZERO_ARENA_GRAD_SHARDS, ZERO_ARENA_GATHER,
  ZERO_ARENA_SCRATCH, ZERO_NUM_ARENAS) = range(7)
 ZERO_OPT_KEEP_GRAD_SHARDS, ZERO_OPT_REPLICA_PAD, ZERO_OPT_BLOCKS_PER_SM, ZERO_OPT_TIMING, ZERO_OPT_KERNEL = 1, 2, 3, 4, 5
-ZERO_KERNEL_AUTO, ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA = 0, 1, 2
+ZERO_KERNEL_AUTO, ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA, ZERO_KERNEL_BULK = 0, 1, 2, 3
 ZERO_OPT_GRAD_BUFFERS = 6
 ZERO_OPT_TMA_GROUPS = 7
 ZERO_OPT_TMA_STAGES = 8
@@ -46,6 +46,8 @@ ZERO_OPT_TMA_CTAS_PER_SM = 9
 ZERO_OPT_DTYPE = 10
 ZERO_OPT_PIPELINE = 11
 ZERO_OPT_PDL = 12
+ZERO_OPT_TMA_TILE = 13
+ZERO_OPT_TMA_WARPS = 14
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -112,9 +114,28 @@ _SIGS = {
     "zero_set_loss_scale": (_i32, [_vp, ctypes.c_double]),
     "zero_set_pipeline_streams": (_i32, [_vp, _vp, _vp]),
     "zero_fused_config": (_i32, [_vp, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32)]),
+    "zero_fused_tile": (_i32, [_vp, ctypes.POINTER(_i32)]),
+    "zero_probe_pattern": (_i32, [_vp, _PTRS, _vp]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
                                       ctypes.POINTER(zero_adam_hparams), _i64, _vp, _vp]),
+    "zero_dist_init": (_i32, [ctypes.POINTER(zero_layout), _i32, _i32, _i32, ctypes.POINTER(_vp)]),
+    "zero_dist_sizes": (_i32, [_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64)]),
+    "zero_dist_tensor_offsets": (_i32, [_vp, ctypes.POINTER(_i64), _i32]),
+    "zero_dist_bind": (_i32, [_vp, _PTRS]),
+    "zero_dist_export": (_i32, [_vp, _vp]),
+    "zero_dist_open_peers": (_i32, [_vp, _vp]),
+    "zero_dist_set_hparams": (_i32, [_vp, ctypes.POINTER(zero_adam_hparams)]),
+    "zero_dist_load_master": (_i32, [_vp, _vp, _vp]),
+    "zero_dist_step": (_i32, [_vp, _vp]),
+    "zero_dist_adam_shard": (_i32, [_vp, _vp, _vp]),
+    "zero_dist_read_partial": (_i32, [_vp, _vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
+                                      ctypes.POINTER(_i64)]),
+    "zero_dist_view": (_i32, [_vp, _i32, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
+    "zero_dist_combine_partials": (_i32, [_i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
+                                          ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)]),
+    "zero_dist_last_error": (ctypes.c_char_p, [_vp]),
+    "zero_dist_destroy": (None, [_vp]),
     "zero_last_error": (ctypes.c_char_p, [_vp]),
     "zero_destroy": (None, [_vp]),
 }
@@ -124,7 +145,11 @@ for _name, (_res, _args) in _SIGS.items():
     _fn.argtypes = _args
     globals()[_name] = _fn
 
-__all__ = list(_SIGS) + ["ZeroOptimizer", "AdamHParams", "ZeroError", "lib", "LIB_PATH", "options_from_config"]
+__all__ = list(_SIGS) + ["ZeroOptimizer", "ZeroDist", "AdamHParams", "ZeroError", "lib", "LIB_PATH",
+                         "options_from_config", "exchange_records", "rank_ordered_norm", "ordered_step"]
+ZERO_DIST_ARENA_GRAD, ZERO_DIST_ARENA_PARAM, ZERO_DIST_ARENA_STATES, ZERO_DIST_ARENA_SCRATCH = 0, 1, 2, 3
+ZERO_DIST_NUM_ARENAS = 4
+ZERO_DIST_HANDLE_BYTES = 192
 
 
 class ZeroError(RuntimeError):
@@ -218,7 +243,7 @@ class ZeroOptimizer:
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
                  tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16,
-                 pipeline: int = 0, device=None):
+                 pipeline: int = 0, tma_tile: int = 0, tma_warps: int = 0, device=None):
         import torch
 
         self._torch = torch
@@ -227,12 +252,8 @@ class ZeroOptimizer:
         self._numel = (ctypes.c_int64 * n)(*[int(x) for x in numel])
         self._layer = (ctypes.c_int32 * n)(*[int(x) for x in layer_id])
         lay = zero_layout(n, self._numel, self._layer)
-        if bucket_elems is None:
-            total = 0
-            for x in numel:
-                total = (total + int(x) + 7) // 8 * 8
-            bucket_elems = max(8, (total + 8 * n_ranks - 1) // (8 * n_ranks) * 8 * n_ranks)
-        self.bucket_elems = int(bucket_elems)
+        # None / 0: the library's one bucket spanning the padded flat space
+        self.bucket_elems = 0 if bucket_elems is None else int(bucket_elems)
         ctx = ctypes.c_void_p()
         st = zero_init(ctypes.byref(lay), self.n_ranks, self.stage, self.bucket_elems, ctypes.byref(ctx))
         if st != ZERO_OK:
@@ -256,6 +277,10 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_DTYPE, int(dtype)), "zero_set_option")
         if tma_ctas_per_sm:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_CTAS_PER_SM, int(tma_ctas_per_sm)), "zero_set_option")
+        if tma_tile:
+            self._check(zero_set_option(ctx, ZERO_OPT_TMA_TILE, int(tma_tile)), "zero_set_option")
+        if tma_warps:
+            self._check(zero_set_option(ctx, ZERO_OPT_TMA_WARPS, int(tma_warps)), "zero_set_option")
         if pipeline:
             self._check(zero_set_option(ctx, ZERO_OPT_PIPELINE, int(pipeline)), "zero_set_option")
         self.pipeline = int(pipeline)
@@ -479,7 +504,21 @@ class ZeroOptimizer:
         k, g, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
         self._check(zero_fused_config(self.ctx, ctypes.byref(k), ctypes.byref(g), ctypes.byref(s)),
                     "zero_fused_config")
-        return dict(kernel={1: "register", 2: "tma"}[k.value], groups=g.value, stages=s.value)
+        tile = ctypes.c_int32()
+        self._check(zero_fused_tile(self.ctx, ctypes.byref(tile)), "zero_fused_tile")
+        return dict(kernel={1: "register", 2: "tma", 3: "bulk"}[k.value], groups=g.value, stages=s.value,
+                    tile=tile.value)
+
+    def set_staged(self, tile: int = 0, warps: int = 0, stages: int = 0):
+        """Tile, consumer warps and ring depth of the staged kernels (0 = the library's choice)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_TMA_TILE, int(tile)), "zero_set_option")
+        self._check(zero_set_option(self.ctx, ZERO_OPT_TMA_WARPS, int(warps)), "zero_set_option")
+        self._check(zero_set_option(self.ctx, ZERO_OPT_TMA_STAGES, int(stages)), "zero_set_option")
+
+    def probe_pattern(self, rank_grads, stream=None):
+        """The movement-only twin of the step's bulk-store launches (zero_probe_pattern)."""
+        ptrs = (ctypes.c_void_p * self.n_ranks)(*[int(g.data_ptr()) for g in rank_grads])
+        self._check(zero_probe_pattern(self.ctx, ptrs, self._stream(stream)), "zero_probe_pattern")
 
     def set_kernel(self, kernel: int):
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
@@ -521,9 +560,160 @@ class ZeroOptimizer:
         ptrs = None if rank_grads is None else _ptr_array(rank_grads)
         self._check(zero_all_reduce(self.ctx, lo, hi, ptrs, self._stream(stream)), "zero_all_reduce")
 
-    def adam_shard(self, rank: int, t: int, stream=None):
+    def adam_shard(self, rank: int, t: int = 0, stream=None):
+        """Adam on rank's shard (-1 = all) for step t; t = 0 takes the
+        context's counter + 1 and, with rank = -1, advances the counter."""
         self._check(zero_adam_shard(self.ctx, rank, t, self._stream(stream)), "zero_adam_shard")
 
     def all_gather(self, lo: int, hi: int, rank_out: Optional[Sequence[int]] = None, stream=None):
         ptrs = None if rank_out is None else _ptr_array(rank_out)
         self._check(zero_all_gather(self.ctx, lo, hi, ptrs, self._stream(stream)), "zero_all_gather")
+
+
+# ------------------------------------------------ one logical rank per GPU ----
+#
+# Host-side plumbing of the rank-per-GPU step (zero_dist_* in
+# include/zero_sm.h): the exchange of the ranks' IPC records, the ordering
+# of a step between the ranks (barriers around the kernel), and the global
+# gradient norm from the ranks' partial sums.  These three helpers take the
+# torch.distributed module and group, so that they run as written over gloo
+# on CPU.
+
+def exchange_records(dist, record: bytes, group=None) -> List[bytes]:
+    """Every rank's export record, in rank order (all_gather_object)."""
+    if len(record) != ZERO_DIST_HANDLE_BYTES:
+        raise ValueError(f"a rank's record is {ZERO_DIST_HANDLE_BYTES} bytes, got {len(record)}")
+    out: List = [None] * dist.get_world_size(group)
+    dist.all_gather_object(out, record, group=group)
+    for q, r in enumerate(out):
+        if not isinstance(r, (bytes, bytearray)) or len(r) != ZERO_DIST_HANDLE_BYTES:
+            raise RuntimeError(f"rank {q} sent a malformed record")
+    return [bytes(r) for r in out]
+
+
+def rank_ordered_norm(dist, sumsq: float, nonfinite: int, group=None):
+    """(global norm, non-finite count) from the ranks' partial sums, added in
+    rank order 0..N-1 in binary64 (every rank gets the same bits)."""
+    world = dist.get_world_size(group)
+    parts: List = [None] * world
+    dist.all_gather_object(parts, (float(sumsq), int(nonfinite)), group=group)
+    sq = (ctypes.c_double * world)(*[p[0] for p in parts])
+    nf = (ctypes.c_int64 * world)(*[p[1] for p in parts])
+    norm, total = ctypes.c_double(), ctypes.c_int64()
+    st = zero_dist_combine_partials(world, sq, nf, ctypes.byref(norm), ctypes.byref(total))
+    if st != ZERO_OK:
+        raise ZeroError(st, "zero_dist_combine_partials", "bad partials")
+    return norm.value, total.value
+
+
+def ordered_step(dist, sync: Callable[[], None], launch: Callable[[], None], group=None):
+    """The cross-rank order of one step: this rank's pending work on its
+    replicas done and every rank past that point (barrier) before the
+    launch; the launch done and every rank past that point before return."""
+    sync()
+    dist.barrier(group=group)
+    launch()
+    sync()
+    dist.barrier(group=group)
+
+
+class ZeroDist:
+    """Rank ``dist.get_rank(group)`` of a ZeRO step with one logical rank per
+    GPU (stage 1 or 2): allocates this rank's arenas with torch on ``device``,
+    binds them, exchanges IPC records with the other ranks and opens theirs.
+    Every call below is collective (every rank calls it, in the same order)."""
+
+    def __init__(self, numel: Sequence[int], layer_id: Sequence[int], stage: int = ZERO_STAGE_2,
+                 hparams: AdamHParams = AdamHParams(), group=None, device=None):
+        import torch
+        import torch.distributed as dist
+
+        self._torch, self._dist, self.group = torch, dist, group
+        self.world, self.rank = dist.get_world_size(group), dist.get_rank(group)
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        n = len(numel)
+        self._numel = (ctypes.c_int64 * n)(*[int(x) for x in numel])
+        self._layer = (ctypes.c_int32 * n)(*[int(x) for x in layer_id])
+        lay = zero_layout(n, self._numel, self._layer)
+        ctx = ctypes.c_void_p()
+        st = zero_dist_init(ctypes.byref(lay), self.world, self.rank, int(stage), ctypes.byref(ctx))
+        if st != ZERO_OK:
+            raise ZeroError(st, "zero_dist_init", zero_dist_last_error(None).decode())
+        self.ctx, self.stage = ctx, int(stage)
+        plan = (ctypes.c_int64 * 3)()
+        ab = (ctypes.c_int64 * ZERO_DIST_NUM_ARENAS)()
+        self._check(zero_dist_sizes(ctx, plan, ab), "zero_dist_sizes")
+        self.psi, self.psi_pad, self.shard = int(plan[0]), int(plan[1]), int(plan[2])
+        self.arenas = [torch.empty(int(ab[k]), dtype=torch.uint8, device=self.device)
+                       for k in range(ZERO_DIST_NUM_ARENAS)]
+        ptrs = (ctypes.c_void_p * ZERO_DIST_NUM_ARENAS)(*[a.data_ptr() for a in self.arenas])
+        with torch.cuda.device(self.device):
+            self._check(zero_dist_bind(ctx, ptrs), "zero_dist_bind")
+            if self.world > 1:
+                rec = ctypes.create_string_buffer(ZERO_DIST_HANDLE_BYTES)
+                self._check(zero_dist_export(ctx, rec), "zero_dist_export")
+                records = exchange_records(dist, rec.raw, group)
+                allrec = ctypes.create_string_buffer(b"".join(records), ZERO_DIST_HANDLE_BYTES * self.world)
+                self._check(zero_dist_open_peers(ctx, allrec), "zero_dist_open_peers")
+                dist.barrier(group=group)  # every rank has mapped every other before anyone writes
+        hp = zero_adam_hparams(hparams.lr, hparams.beta1, hparams.beta2, hparams.eps, hparams.weight_decay)
+        self._check(zero_dist_set_hparams(ctx, ctypes.byref(hp)), "zero_dist_set_hparams")
+
+    def _check(self, st: int, where: str):
+        if st != ZERO_OK:
+            raise ZeroError(st, where, zero_dist_last_error(self.ctx).decode())
+
+    def _stream(self) -> int:
+        return self._torch.cuda.current_stream(self.device).cuda_stream
+
+    def _sync(self):
+        self._torch.cuda.current_stream(self.device).synchronize()
+
+    def offsets(self) -> List[int]:
+        out = (ctypes.c_int64 * len(self._numel))()
+        self._check(zero_dist_tensor_offsets(self.ctx, out, len(self._numel)), "zero_dist_tensor_offsets")
+        return list(out)
+
+    def view(self, what: int):
+        """Tensor view of ZERO_VIEW_MASTER/_EXP_AVG/_EXP_AVG_SQ (the owned
+        shard) or ZERO_VIEW_PARAM/ZERO_VIEW_GRAD_BUF (this rank's replicas)."""
+        ptr, n = ctypes.c_void_p(), ctypes.c_int64()
+        self._check(zero_dist_view(self.ctx, int(what), ctypes.byref(ptr), ctypes.byref(n)), "zero_dist_view")
+        dt = self._torch.float32 if what in (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ) \
+            else self._torch.int16
+        item = 4 if dt == self._torch.float32 else 2
+        arena = self.arenas[ZERO_DIST_ARENA_STATES if item == 4 else
+                            (ZERO_DIST_ARENA_PARAM if what == ZERO_VIEW_PARAM else ZERO_DIST_ARENA_GRAD)]
+        off = (ptr.value - arena.data_ptr())
+        return arena[off: off + item * n.value].view(dt)
+
+    def load_master(self, master_full):
+        """master_full: fp32 CUDA tensor of psi_pad values on this rank's device."""
+        ordered_step(self._dist, self._sync,
+                     lambda: self._check(zero_dist_load_master(self.ctx, master_full.data_ptr(), self._stream()),
+                                         "zero_dist_load_master"), self.group)
+
+    def step(self, stats: bool = False):
+        """One step; with ``stats`` the global gradient norm and non-finite
+        count (rank-ordered sum of the ranks' partials) and the step number."""
+        ordered_step(self._dist, self._sync,
+                     lambda: self._check(zero_dist_step(self.ctx, self._stream()), "zero_dist_step"), self.group)
+        if not stats:
+            return None
+        sq, nf, t = ctypes.c_double(), ctypes.c_int64(), ctypes.c_int64()
+        self._check(zero_dist_read_partial(self.ctx, self._stream(), ctypes.byref(sq), ctypes.byref(nf),
+                                           ctypes.byref(t)), "zero_dist_read_partial")
+        norm, nft = rank_ordered_norm(self._dist, sq.value, nf.value, self.group)
+        return {"grad_norm": norm, "nonfinite": nft, "step": t.value}
+
+    def adam_shard(self, grad_shard):
+        """Adam on the owned shard from an already reduced bf16 shard (S
+        values): the update of a step whose collectives are NCCL calls."""
+        self._check(zero_dist_adam_shard(self.ctx, grad_shard.data_ptr(), self._stream()), "zero_dist_adam_shard")
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            self._sync()
+            self._dist.barrier(group=self.group)  # no peer still writes this rank's replicas
+            zero_dist_destroy(self.ctx)
+            self.ctx = None

@@ -11,8 +11,8 @@ import subprocess
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = ["csrc/zero_api.cu", "csrc/kernels.cu", "csrc/fused_tma.cu", "csrc/static_scratch.cu",
-           "csrc/two_pass_tma.cu",
+SOURCES = ["csrc/zero_api.cu", "csrc/kernels.cu", "csrc/fused_tma.cu", "csrc/fused_bulk.cu", "csrc/static_scratch.cu",
+           "csrc/two_pass_tma.cu", "csrc/dist.cu",
            "csrc/plan.cpp"]
 LIB = os.path.join(HERE, "libzero_sm.so")
 
@@ -30,9 +30,11 @@ def nvcc() -> str:
 
 
 def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    objs = []
+    from concurrent.futures import ThreadPoolExecutor
+
     bdir = os.path.join(HERE, "_build")
     os.makedirs(bdir, exist_ok=True)
+    cmds, objs = [], []
     for src in SOURCES:
         obj = os.path.join(bdir, os.path.basename(src) + ".o")
         cmd = [nvcc(), *NVCC_FLAGS]
@@ -43,8 +45,16 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
             cmd += ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd))
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # the translation units are independent: compile them side by side
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as pool:
+        for res in pool.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds):
+            if verbose or ptxas_verbose or res.returncode != 0:
+                print(res.stdout, end="")
+                print(res.stderr, end="")
+            if res.returncode != 0:
+                raise subprocess.CalledProcessError(res.returncode, res.args, res.stdout, res.stderr)
     link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs]
     if verbose:
         print(" ".join(link))

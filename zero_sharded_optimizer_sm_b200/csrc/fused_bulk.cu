@@ -1,0 +1,436 @@
+// Fused ZeRO step kernel whose loads AND stores are bulk copies (sm_100a).
+//
+// The same arithmetic and outputs as the other fused kernels (reduce in rank
+// order, mean, Adam, broadcast of the 16-bit parameters -- "ZERO训练技术",
+// sections "ZeRO-1"/"ZeRO-2"/"ZeRO-3", parts "2. 反向" and "3. 更新"), with
+// both directions of data movement handed to the Tensor Memory Accelerator:
+//
+//   warp 0 (producer)  its elected lane streams tile after tile -- the N
+//                      gradient slices and the fp32 master/m/v slices of T
+//                      elements -- into a ring of shared-memory stages
+//                      (cp.async.bulk, completion counted in bytes on the
+//                      stage's `full` mbarrier);
+//   warps 2..W+1       (consumers) reduce, update, and write every result
+//                      back into the same stage: master/m/v in place, the
+//                      16-bit parameters over rank 0's gradient slice, the
+//                      averaged gradient (stage 1 write-back or the reduced
+//                      shard) into a slice of its own; then fence the async
+//                      proxy and arrive on the stage's `computed` mbarrier;
+//   warp 1 (storer)    its elected lane waits for `computed`, issues the
+//                      stage's bulk stores (shared -> global: master, m, v,
+//                      the N parameter replicas, the ZeRO-3 shard, the
+//                      ZeRO-1 write-back), waits until they have read the
+//                      stage and releases it to the producer (`empty`).
+//
+// A lane of the consumers therefore issues no global store at all: the 2N + 6
+// sixteen-byte stores per lane per tile of the register-store kernels become
+// N + 3 (+ N at ZeRO-1) bulk copies per tile from one thread.  Every copy
+// reads or writes only this GPU's memory and this CTA's shared memory; no
+// cluster multicast.
+//
+// Every mbarrier wait is bounded (kWaitNs); a role whose wait runs out sets an
+// error bit in the scratch arena and the CTA's abort flag, the other roles
+// leave their loops, the copies already issued are drained (loads: bounded
+// wait on their barriers; stores: the issuing thread's bulk-group wait, which
+// depends on no other thread) and the CTA ends.
+//
+// kMove builds the movement-only twin used to measure what this exact pattern
+// of streams can move on the device: identical copies and shared-memory
+// traffic, the arithmetic replaced by an XOR fold of the gradients and the
+// 16-bit rounding of the unchanged master weights (so a twin pass leaves a
+// context's master/m/v and parameters as they were).  No step entry point
+// launches it.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "device_math.cuh"
+#include "kernels.cuh"
+#include "tma_pipe.cuh"
+
+namespace zsm {
+namespace {
+
+using namespace dev;
+using namespace pipe;
+
+// ------------------------------------------------ per-thread smem vectors --
+
+template <int EPT>
+struct H16 {  // EPT 16-bit values, two per word
+  uint32_t w[EPT / 2];
+};
+template <int EPT>
+struct V32 {  // EPT fp32 values
+  float f[EPT];
+};
+
+template <int EPT>
+__device__ __forceinline__ H16<EPT> lds16(const unsigned char* p);
+template <>
+__device__ __forceinline__ H16<8> lds16<8>(const unsigned char* p) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  return {{v.x, v.y, v.z, v.w}};
+}
+template <>
+__device__ __forceinline__ H16<4> lds16<4>(const unsigned char* p) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  return {{v.x, v.y}};
+}
+template <>
+__device__ __forceinline__ H16<2> lds16<2>(const unsigned char* p) {
+  return {{*reinterpret_cast<const uint32_t*>(p)}};
+}
+
+template <int EPT>
+__device__ __forceinline__ void sts16(unsigned char* p, const H16<EPT>& h);
+template <>
+__device__ __forceinline__ void sts16<8>(unsigned char* p, const H16<8>& h) {
+  *reinterpret_cast<uint4*>(p) = make_uint4(h.w[0], h.w[1], h.w[2], h.w[3]);
+}
+template <>
+__device__ __forceinline__ void sts16<4>(unsigned char* p, const H16<4>& h) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(h.w[0], h.w[1]);
+}
+template <>
+__device__ __forceinline__ void sts16<2>(unsigned char* p, const H16<2>& h) {
+  *reinterpret_cast<uint32_t*>(p) = h.w[0];
+}
+
+template <int EPT>
+__device__ __forceinline__ V32<EPT> ldsf(const unsigned char* p) {
+  V32<EPT> r;
+#pragma unroll
+  for (int q = 0; q < EPT; q += 4) {
+    if constexpr (EPT >= 4) {
+      const float4 v = *reinterpret_cast<const float4*>(p + 4 * q);
+      r.f[q] = v.x;
+      r.f[q + 1] = v.y;
+      r.f[q + 2] = v.z;
+      r.f[q + 3] = v.w;
+    } else {
+      const float2 v = *reinterpret_cast<const float2*>(p + 4 * q);
+      r.f[q] = v.x;
+      r.f[q + 1] = v.y;
+    }
+  }
+  return r;
+}
+
+template <int EPT>
+__device__ __forceinline__ void stsf(unsigned char* p, const V32<EPT>& r) {
+#pragma unroll
+  for (int q = 0; q < EPT; q += 4) {
+    if constexpr (EPT >= 4) {
+      *reinterpret_cast<float4*>(p + 4 * q) = make_float4(r.f[q], r.f[q + 1], r.f[q + 2], r.f[q + 3]);
+    } else {
+      *reinterpret_cast<float2*>(p + 4 * q) = make_float2(r.f[q], r.f[q + 1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------ stage layout --
+//
+// One stage of T elements: [N gradient slices, 2T bytes each][master 4T][m 4T]
+// [v 4T][averaged gradient 2T, only when stored].  Consumers overwrite the
+// state slices in place and rank 0's gradient slice with the parameters.
+__host__ __device__ inline unsigned bulk_stage_bytes(int n_ranks, int tile, bool need_g) {
+  return (unsigned)tile * (unsigned)(2 * n_ranks + 12 + (need_g ? 2 : 0));
+}
+
+__host__ __device__ inline size_t bulk_smem_bytes(int n_ranks, int tile, bool need_g, int stages) {
+  return (size_t)stages * bulk_stage_bytes(n_ranks, tile, need_g) + 3 * (size_t)stages * sizeof(uint64_t) +
+         4 * (size_t)(stages + 1);
+}
+
+template <int MODE, class F, int T, int W, bool kMove>
+__global__ void __launch_bounds__(32 * (W + 2), 1)
+    fused_bulk_kernel(const __grid_constant__ FusedArgs a, int stages, uint32_t opaque) {
+  constexpr int EPT = T / (32 * W);
+  static_assert(EPT == 2 || EPT == 4 || EPT == 8, "2, 4 or 8 elements per consumer lane");
+  constexpr int NT = 32 * (W + 2);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const bool need_g = MODE == kFusedZ1 || a.grad_shard != nullptr;
+  const unsigned sb = bulk_stage_bytes(N, T, need_g);
+  const unsigned off_state = 2u * (unsigned)N * T;  // master; m at +4T, v at +8T
+  const unsigned off_g = off_state + 12u * T;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * sb);
+  uint64_t* computed = full + stages;
+  uint64_t* empty = computed + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_k = abort_flag + 1;  // last phase of `full` issued per stage, -1 = none
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + T - 1) / T;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&computed[s], W);
+      mbar_init(&empty[s], 1);
+      last_k[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (k > 0) {
+          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag);
+          if (w != 0) {
+            if (w == 1) atomicOr(a.ns.error, 1u);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        fence_proxy_async_smem();  // the stage's last reads (consumers, stores) before the refill
+        const int64_t e0 = tile * T;
+        const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+        unsigned char* st = smem + (size_t)s * sb;
+        mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * T, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
+        bulk_load(st + off_state, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + off_state + 4 * T, a.m + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + off_state + 8 * T, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
+        last_k[s] = (int)k;
+      }
+      pdl_trigger();  // no more loads to issue: the next fused launch may start
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- storer --
+    if (lane == 0) {
+      bool waited = false;
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag);
+        if (w != 0) {
+          if (w == 1) atomicOr(a.ns.error, 8u);
+          *abort_flag = 1;
+          break;
+        }
+        if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+          pdl_wait();
+          waited = true;
+        }
+        const int64_t e0 = tile * T;
+        const unsigned cnt = (unsigned)((n_elem - e0) < T ? (n_elem - e0) : T);
+        const unsigned char* st = smem + (size_t)s * sb;
+        bulk_store(a.master + e0, st + off_state, 4 * cnt);
+        bulk_store(a.m + e0, st + off_state + 4 * T, 4 * cnt);
+        bulk_store(a.v + e0, st + off_state + 8 * T, 4 * cnt);
+        if (MODE == kFusedZ3) bulk_store(a.param_shard + e0, st, 2 * cnt);
+        for (int r = 0; r < N; ++r) bulk_store(a.out[r] + e0, st, 2 * cnt);
+        if (MODE == kFusedZ1)
+          for (int r = 0; r < N; ++r) bulk_store(const_cast<uint16_t*>(a.grad[r]) + e0, st + off_g, 2 * cnt);
+        if (a.grad_shard) bulk_store(a.grad_shard + e0, st + off_g, 2 * cnt);
+        bulk_commit();
+        bulk_wait_read<0>();  // the copies have read the stage: hand it back to the producer
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait<0>();  // every store of this CTA performed before the CTA ends
+    }
+  } else {
+    // ----------------------------------------------------------- consumers --
+    const int c = threadIdx.x - 64;  // 0 .. 32W-1
+    const int j = c * EPT;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      // warp-uniform decisions, so that no lane is left waiting at __syncwarp
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      const int64_t e0 = tile * T;
+      const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+      unsigned char* st = smem + (size_t)s * sb;
+      if (j < cnt) {  // cnt is a multiple of 8, so a lane's EPT elements are whole
+        V32<EPT> p = ldsf<EPT>(st + off_state + 4 * j);
+        V32<EPT> m = ldsf<EPT>(st + off_state + 4 * T + 4 * j);
+        V32<EPT> v = ldsf<EPT>(st + off_state + 8 * T + 4 * j);
+        H16<EPT> par, gout;
+        if constexpr (kMove) {
+          // movement only: every slice read, nothing computed but a fold
+          uint32_t fold[EPT / 2];
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) fold[q] = 0u;
+          for (int r = 0; r < N; ++r) {
+            const H16<EPT> h = lds16<EPT>(st + (size_t)r * 2 * T + 2 * j);
+#pragma unroll
+            for (int q = 0; q < EPT / 2; ++q) fold[q] ^= h.w[q];
+          }
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) {
+            par.w[q] = pack2(F::rn(p.f[2 * q]), F::rn(p.f[2 * q + 1])) ^ (fold[q] & opaque);
+            gout.w[q] = fold[q];
+          }
+        } else {
+          float acc[EPT];
+#pragma unroll
+          for (int q = 0; q < EPT; ++q) acc[q] = 0.0f;
+          for (int r = 0; r < N; ++r) {
+            const H16<EPT> h = lds16<EPT>(st + (size_t)r * 2 * T + 2 * j);
+#pragma unroll
+            for (int q = 0; q < EPT / 2; ++q) {
+              acc[2 * q] = __fadd_rn(acc[2 * q], F::lo(h.w[q]));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], F::hi(h.w[q]));
+            }
+          }
+          uint16_t g16[EPT], p16[EPT];
+#pragma unroll
+          for (int q = 0; q < EPT; ++q) {
+            g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
+            const float g = F::f32(g16[q]);
+            const double d = (double)g;
+            sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
+            nf += isfinite(g) ? 0ull : 1ull;
+            p16[q] = F::rn(adam1(g, p.f[q], m.f[q], v.f[q], sc));
+          }
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) {
+            par.w[q] = pack2(p16[2 * q], p16[2 * q + 1]);
+            gout.w[q] = pack2(g16[2 * q], g16[2 * q + 1]);
+          }
+        }
+        stsf<EPT>(st + off_state + 4 * j, p);
+        stsf<EPT>(st + off_state + 4 * T + 4 * j, m);
+        stsf<EPT>(st + off_state + 8 * T + 4 * j, v);
+        sts16<EPT>(st + 2 * j, par);  // over rank 0's slice, which this lane alone read here
+        if (need_g) sts16<EPT>(st + off_g + 2 * j, gout);
+      }
+      fence_proxy_async_smem();  // this lane's stage writes before the storer's bulk copies read them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&computed[s]);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // drain the bulk loads already issued before the CTA's memory goes away
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
+  }
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
+  norm_epilogue<NT>(a.ns, sq, nf, a.accumulate);
+}
+
+// A programmatic dependent launch may place its CTAs while the grid before it
+// still runs; these kernels are persistent (tiles dealt by CTA index), so a
+// launch with the attribute asks for more than half an SM's shared memory and
+// a dependent grid's CTAs land only on SMs the grid before has left.
+constexpr size_t kPdlSoloSmemBulk = 116 * 1024;
+
+template <int MODE, class F, int T, int W, bool kMove>
+cudaError_t launch_cfg(const FusedArgs& a, int grid, int stages, size_t bytes, uint32_t opaque, cudaStream_t s) {
+  return launch_kernel(fused_bulk_kernel<MODE, F, T, W, kMove>, grid, 32 * (W + 2), bytes, s, a.pdl != kPdlNone,
+                       a, stages, opaque);
+}
+
+// The (tile, consumer warps) configurations built: 2048 x 8 and 1024 x 4
+// (8 elements a lane), 2048 x 16 and 1024 x 8 (4 a lane), 1024 x 16 (2).
+#define ZSM_BULK_CONFIGS(X) X(2048, 8) X(2048, 16) X(1024, 4) X(1024, 8) X(1024, 16)
+
+template <int MODE, class F, bool kMove>
+cudaError_t launch_mode_fmt(const FusedArgs& a, int grid, int tile, int warps, int stages, size_t bytes,
+                            uint32_t opaque, cudaStream_t s) {
+#define ZSM_BULK_CASE(TT, WW) \
+  if (tile == TT && warps == WW) return launch_cfg<MODE, F, TT, WW, kMove>(a, grid, stages, bytes, opaque, s);
+  ZSM_BULK_CONFIGS(ZSM_BULK_CASE)
+#undef ZSM_BULK_CASE
+  return cudaErrorInvalidValue;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const FusedArgs& a, int grid, int tile, int warps, int stages, size_t bytes, bool move,
+                        uint32_t opaque, cudaStream_t s) {
+  if (move) return launch_mode_fmt<MODE, Bf16, true>(a, grid, tile, warps, stages, bytes, opaque, s);
+  if (a.fmt == kFmtF16) return launch_mode_fmt<MODE, F16, false>(a, grid, tile, warps, stages, bytes, opaque, s);
+  return launch_mode_fmt<MODE, Bf16, false>(a, grid, tile, warps, stages, bytes, opaque, s);
+}
+
+template <class K>
+cudaError_t opt_in(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
+}
+
+template <int MODE, class F, bool kMove>
+cudaError_t configure_mode_fmt() {
+  cudaError_t e = cudaSuccess;
+#define ZSM_BULK_OPT(TT, WW) \
+  if (e == cudaSuccess) e = opt_in(fused_bulk_kernel<MODE, F, TT, WW, kMove>);
+  ZSM_BULK_CONFIGS(ZSM_BULK_OPT)
+#undef ZSM_BULK_OPT
+  return e;
+}
+
+template <int MODE>
+cudaError_t configure_mode() {
+  cudaError_t e = configure_mode_fmt<MODE, Bf16, false>();
+  if (e == cudaSuccess) e = configure_mode_fmt<MODE, F16, false>();
+  if (e == cudaSuccess) e = configure_mode_fmt<MODE, Bf16, true>();
+  return e;
+}
+
+}  // namespace
+
+bool bulk_config_valid(int tile, int warps) {
+#define ZSM_BULK_VALID(TT, WW) \
+  if (tile == TT && warps == WW) return true;
+  ZSM_BULK_CONFIGS(ZSM_BULK_VALID)
+#undef ZSM_BULK_VALID
+  return false;
+}
+
+int bulk_stages_for(int n_ranks, int tile, bool need_g, int max_stages) {
+  if (n_ranks < 1 || n_ranks > kTmaMaxRanks) return 0;
+  int stages = max_stages > 0 ? std::min(max_stages, kTmaMaxStages) : kTmaMaxStages;
+  while (stages > 0 && bulk_smem_bytes(n_ranks, tile, need_g, stages) > (size_t)kTmaMaxSmem) --stages;
+  return stages >= 2 ? stages : 0;
+}
+
+cudaError_t bulk_configure() {
+  cudaError_t e = configure_mode<kFusedZ1>();
+  if (e == cudaSuccess) e = configure_mode<kFusedZ2>();
+  if (e == cudaSuccess) e = configure_mode<kFusedZ3>();
+  return e;
+}
+
+cudaError_t launch_fused_bulk(int mode, const FusedArgs& a, int grid, int tile, int warps, int max_stages, bool move,
+                              uint32_t opaque, cudaStream_t s) {
+  const bool need_g = mode == kFusedZ1 || a.grad_shard != nullptr;
+  const int stages = bulk_stages_for(a.n_ranks, tile, need_g, max_stages);
+  if (stages == 0 || !bulk_config_valid(tile, warps)) return cudaErrorInvalidValue;
+  size_t bytes = bulk_smem_bytes(a.n_ranks, tile, need_g, stages);
+  if (a.pdl != kPdlNone && bytes < kPdlSoloSmemBulk) bytes = kPdlSoloSmemBulk;
+  switch (mode) {
+    case kFusedZ1: return launch_mode<kFusedZ1>(a, grid, tile, warps, stages, bytes, move, opaque, s);
+    case kFusedZ2: return launch_mode<kFusedZ2>(a, grid, tile, warps, stages, bytes, move, opaque, s);
+    case kFusedZ3: return launch_mode<kFusedZ3>(a, grid, tile, warps, stages, bytes, move, opaque, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace zsm

@@ -205,7 +205,7 @@ struct InitArgs {
 };
 
 enum FusedMode { kFusedZ1 = 1, kFusedZ2 = 2, kFusedZ3 = 3 };
-enum FusedKernel { kKernelAuto = 0, kKernelRegister = 1, kKernelTma = 2 };
+enum FusedKernel { kKernelAuto = 0, kKernelRegister = 1, kKernelTma = 2, kKernelBulk = 3 };
 
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_fused(int mode, const FusedArgs& a, int grid, cudaStream_t s);
@@ -233,6 +233,19 @@ int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
 // Rank-chunked staged kernel (fused_tma.cu) for any N, meant for N > 16: the
 // replicas stream in chunks of 8 ranks through a `cstages`-deep ring.
 cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s);
+
+// Staged kernel with bulk stores (fused_bulk.cu), N <= 16: tiles of `tile`
+// elements, `warps` consumer warps, a ring of at most `max_stages` stages (0 =
+// as many as fit); one CTA per SM.  `move` launches the movement-only twin
+// (same copies, no arithmetic; `opaque` must be 0), which measures the
+// pattern's ceiling and is never part of a step.
+cudaError_t launch_fused_bulk(int mode, const FusedArgs& a, int grid, int tile, int warps, int max_stages, bool move,
+                              uint32_t opaque, cudaStream_t s);
+// Ring depth of that kernel for N, the tile and whether the averaged gradient
+// is stored (0 when nothing fits); whether (tile, warps) is a built configuration.
+int bulk_stages_for(int n_ranks, int tile, bool need_g, int max_stages);
+bool bulk_config_valid(int tile, int warps);
+cudaError_t bulk_configure();  // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the staged kernel in that configuration (0 on error).
 int tma_ctas_per_sm(int n_ranks, int groups, int max_stages);

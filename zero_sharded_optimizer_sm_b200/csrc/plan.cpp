@@ -23,8 +23,8 @@ bool make_plan(int32_t n_tensors, const int64_t* numel, const int32_t* layer_id,
     *err = "layout needs n_tensors >= 1 and non-null numel/layer_id";
     return false;
   }
-  if (bucket_elems <= 0 || bucket_elems % kGranule != 0) {
-    *err = "bucket_elems must be a positive multiple of 8";
+  if (bucket_elems < 0 || bucket_elems % kGranule != 0) {
+    *err = "bucket_elems must be 0 (one bucket) or a positive multiple of 8";
     return false;
   }
   Plan p;
@@ -64,8 +64,10 @@ bool make_plan(int32_t n_tensors, const int64_t* numel, const int32_t* layer_id,
     k = j + 1;
   }
 
-  // Bucket schedule, last tensor to first.
-  const int64_t B = bucket_elems;
+  // Bucket schedule, last tensor to first; 0 = one bucket spanning the padded
+  // flat space.
+  if (bucket_elems == 0) p.bucket_elems = p.psi_pad;
+  const int64_t B = p.bucket_elems;
   bool open = false;
   Span cur{0, 0};
   for (int32_t k = n_tensors - 1; k >= 0; --k) {

@@ -97,6 +97,50 @@ static __device__ __forceinline__ void bulk_load(void* dst, const void* src, uns
       : "memory");
 }
 
+// Wait for the phase with the given parity, giving up when `abort_flag` is set
+// (another role of the CTA stopped) or after kWaitNs: 0 = done, 1 = timed
+// out, 2 = aborted.
+static __device__ __forceinline__ int mbar_wait_or_abort(uint64_t* bar, unsigned parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return 0;
+  const unsigned long long t0 = now_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return 2;
+    if (now_ns() - t0 > kWaitNs) return 1;
+  }
+  return 0;
+}
+
+// 1-D bulk copy from this CTA's shared memory to this GPU's global memory,
+// tracked in the issuing thread's bulk async-group.  The shared-memory
+// source must have been written before a fence.proxy.async by its writers.
+static __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
+               : "memory");
+}
+
+static __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned bytes, uint64_t policy) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes), "l"(policy)
+               : "memory");
+}
+
+static __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Until at most `Pending` of this thread's committed bulk groups still read
+// their shared-memory source (the source may then be overwritten).
+template <int Pending>
+static __device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(Pending) : "memory");
+}
+
+// Until at most `Pending` of this thread's committed bulk groups are incomplete
+// (their writes to global memory performed).
+template <int Pending>
+static __device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(Pending) : "memory");
+}
+
 // Plain (write-back) 16-byte stores for the consumers' outputs; measured ~1 %
 // faster than streaming stores in this kernel on B200.
 static __device__ __forceinline__ void st_out(uint16_t* p, uint4 v) { *reinterpret_cast<uint4*>(p) = v; }

@@ -50,6 +50,8 @@ struct zero_ctx {
   int tma_groups_opt = 0;  // 0 = the library's choice
   int tma_stages_opt = 0;  // 0 = the library's choice
   int tma_ctas_opt = 0;    // CTAs per SM of the staged kernel, 0 = the library's choice
+  int tma_tile_opt = 0;    // bulk-store kernel: elements per tile, 0 = the library's choice
+  int tma_warps_opt = 0;   // bulk-store kernel: consumer warps, 0 = the library's choice
   int tma_grid_key = -1;   // configuration the cached grid cap belongs to
   int tma_grid_cap = 0;
   // arena layout (bytes)
@@ -360,11 +362,14 @@ int tma_grid_cap(zero_ctx* c) {
 // stage kernel for N <= 16, the rank-chunked one above.
 bool use_chunked(const zero_ctx* c) {
   if (c->plan.n_ranks <= zsm::kTmaMaxRanks) return false;
-  return c->kernel_opt != ZERO_KERNEL_REGISTER;  // AUTO and TMA
+  return c->kernel_opt != ZERO_KERNEL_REGISTER;  // AUTO, TMA and BULK
 }
+
+bool use_bulk(const zero_ctx* c);
 
 bool use_tma(const zero_ctx* c) {
   if (use_chunked(c)) return true;
+  if (use_bulk(c)) return false;
   if (zsm::tma_stages_for(c->plan.n_ranks, tma_groups(c), tma_stages(c)) == 0) return false;
   if (c->kernel_opt == ZERO_KERNEL_TMA) return true;
   if (c->kernel_opt == ZERO_KERNEL_REGISTER) return false;
@@ -372,6 +377,23 @@ bool use_tma(const zero_ctx* c) {
 }
 
 int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages_opt : 3; }  // measured best at N = 32, 64
+
+// The bulk-store staged kernel (fused_bulk.cu): its tile, consumer warps and
+// ring depth for this context.
+int bulk_tile(const zero_ctx* c) { return c->tma_tile_opt ? c->tma_tile_opt : 1024; }
+int bulk_warps(const zero_ctx* c) { return c->tma_warps_opt ? c->tma_warps_opt : 8; }
+bool bulk_need_g(const zero_ctx* c) {
+  return c->stage == ZERO_STAGE_1 || c->arena[ZERO_ARENA_GRAD_SHARDS] != nullptr;
+}
+int bulk_stages(const zero_ctx* c) {
+  return zsm::bulk_stages_for(c->plan.n_ranks, bulk_tile(c), bulk_need_g(c), c->tma_stages_opt);
+}
+bool bulk_fits(const zero_ctx* c) {
+  return c->plan.n_ranks <= zsm::kTmaMaxRanks && zsm::bulk_config_valid(bulk_tile(c), bulk_warps(c)) &&
+         bulk_stages(c) > 0;
+}
+// Asked for and N <= 16; a (tile, warps) pair that is not built fails at launch.
+bool use_bulk(const zero_ctx* c) { return c->kernel_opt == ZERO_KERNEL_BULK && c->plan.n_ranks <= zsm::kTmaMaxRanks; }
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
@@ -437,7 +459,7 @@ std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
 // One fused launch over [lo, hi).  grad[r] are at flat element lo.
 zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
                            bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0,
-                           int pdl = zsm::kPdlNone, const zsm::AdamScalars* sc_dev = nullptr) {
+                           int pdl = zsm::kPdlNone, const zsm::AdamScalars* sc_dev = nullptr, bool twin = false) {
   if (hi == lo) return ZERO_OK;
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
@@ -469,7 +491,11 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
   cudaError_t e;
-  if (use_chunked(c)) {
+  if (twin || use_bulk(c)) {
+    const int64_t tiles = (hi - lo + bulk_tile(c) - 1) / bulk_tile(c);
+    e = counted(c, zsm::launch_fused_bulk(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
+                                          bulk_tile(c), bulk_warps(c), c->tma_stages_opt, twin, 0u, s));
+  } else if (use_chunked(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
     e = counted(c, zsm::launch_fused_chunked(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
                                   chunked_stages(c), s));
@@ -930,7 +956,7 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     return ZERO_OK;
   }
   if (key == ZERO_OPT_KERNEL) {
-    if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_TMA) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
+    if (value < ZERO_KERNEL_AUTO || value > ZERO_KERNEL_BULK) return fail(c, ZERO_EINVAL, "unknown kernel %lld", (long long)value);
     c->kernel_opt = (int)value;
     return ZERO_OK;
   }
@@ -946,6 +972,17 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   if (key == ZERO_OPT_TMA_STAGES) {
     if (value < 0 || value > zsm::kTmaMaxStages) return fail(c, ZERO_EINVAL, "stages must be 0..%d", zsm::kTmaMaxStages);
     c->tma_stages_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_TMA_TILE) {
+    if (value != 0 && value != 1024 && value != 2048) return fail(c, ZERO_EINVAL, "tile must be 0 (auto), 1024 or 2048");
+    c->tma_tile_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_TMA_WARPS) {
+    if (value != 0 && value != 4 && value != 8 && value != 16)
+      return fail(c, ZERO_EINVAL, "consumer warps must be 0 (auto), 4, 8 or 16");
+    c->tma_warps_opt = (int)value;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_TMA_GROUPS) {
@@ -1058,6 +1095,7 @@ zero_status zero_bind(zero_ctx* c, void* const* arenas) {
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   if (e == cudaSuccess) e = zsm::occupancy(mode, c->plan.n_ranks, &fused_blocks, &simple_blocks);
   if (e == cudaSuccess) e = zsm::tma_configure();
+  if (e == cudaSuccess) e = zsm::bulk_configure();
   if (e == cudaSuccess) e = zsm::two_pass_configure();
   if (e != cudaSuccess) return cuda_fail(c, e, "device query");
   if (c->blocks_per_sm_opt > 0) fused_blocks = std::min(fused_blocks, c->blocks_per_sm_opt);
@@ -1297,20 +1335,47 @@ zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
   return ZERO_OK;
 }
 
+}  // extern "C"
+
+namespace {
+zero_status adam_shard_launch(zero_ctx* c, int32_t rank, int64_t t, cudaStream_t s);
+}  // namespace
+
+extern "C" {
+
 zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) {
   zero_status st = check_ready(c, true);
   if (st != ZERO_OK) return st;
   const int N = c->plan.n_ranks;
   if (rank < -1 || rank >= N) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
-  if (t < 1) return fail(c, ZERO_EINVAL, "step t must be >= 1");
+  if (t < 0) return fail(c, ZERO_EINVAL, "step t must be >= 1, or 0 for the context's counter + 1");
   if (c->stage != ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
   if (c->stage == ZERO_STAGE_1 && !c->arena[ZERO_ARENA_GRADS])
     return fail(c, ZERO_ESTATE, "stage 1 Adam reads the gradient buffers, which were dropped");
+  // t = 0: the step after the context's counter; a call for every shard
+  // (rank = -1) then completes that step and advances the counter
+  const bool from_counter = t == 0;
+  if (from_counter) {
+    int64_t done = 0;
+    st = read_device_t(c, &done);
+    if (st != ZERO_OK) return st;
+    t = done + 1;
+  }
+  st = adam_shard_launch(c, rank, t, static_cast<cudaStream_t>(stream));
+  if (st == ZERO_OK && from_counter && rank < 0) st = write_device_t(c, t);
+  return st;
+}
+
+}  // extern "C"
+
+namespace {
+
+zero_status adam_shard_launch(zero_ctx* c, int32_t rank, int64_t t, cudaStream_t s) {
+  const int N = c->plan.n_ranks;
   const zsm::AdamScalars sc = step_scalars(c, t, 1.0f);
   const int64_t S = c->plan.shard;
   const int r0 = rank < 0 ? 0 : rank, r1 = rank < 0 ? N : rank + 1;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Stage 2/3 (and stage 1 with one launch for all ranks, since every replica
   // holds the same reduced gradient): the shards are contiguous, so ranks
   // r0..r1-1 form one launch over [r0*S, r1*S).  Stage 1 per rank reads the
@@ -1374,6 +1439,10 @@ zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) 
   c->norm_fresh = true;
   return ZERO_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 zero_status zero_all_gather(zero_ctx* c, int64_t lo, int64_t hi, void* const* rank_out, void* stream) {
   zero_status st = check_ready(c, false);
@@ -1478,7 +1547,11 @@ zero_status zero_set_clip(zero_ctx* c, double max_norm, int32_t skip_nonfinite) 
 
 zero_status zero_fused_config(const zero_ctx* c, int32_t* kernel, int32_t* groups, int32_t* stages) {
   if (!c || !kernel || !groups || !stages) return ZERO_EINVAL;
-  if (use_chunked(c)) {
+  if (use_bulk(c)) {
+    *kernel = ZERO_KERNEL_BULK;
+    *groups = bulk_warps(c);
+    *stages = bulk_stages(c);
+  } else if (use_chunked(c)) {
     *kernel = ZERO_KERNEL_TMA;
     *groups = 1;
     *stages = chunked_stages(c);
@@ -1491,6 +1564,44 @@ zero_status zero_fused_config(const zero_ctx* c, int32_t* kernel, int32_t* group
     *groups = 0;
     *stages = 0;
   }
+  return ZERO_OK;
+}
+
+zero_status zero_fused_tile(const zero_ctx* c, int32_t* tile) {
+  if (!c || !tile) return ZERO_EINVAL;
+  *tile = use_bulk(c) ? bulk_tile(c) : use_tma(c) ? (int32_t)kTmaTile : 0;
+  return ZERO_OK;
+}
+
+zero_status zero_probe_pattern(zero_ctx* c, const void* const* rank_grads, void* stream) {
+  zero_status st = check_ready(c, false);
+  if (st != ZERO_OK) return st;
+  if (!rank_grads) return fail(c, ZERO_EINVAL, "rank_grads is NULL");
+  const int N = c->plan.n_ranks;
+  for (int r = 0; r < N; ++r)
+    if (!rank_grads[r] || !aligned16(rank_grads[r]))
+      return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
+  if (!bulk_fits(c))
+    return fail(c, ZERO_ENOTIMPL, "the movement-only pass exists for the bulk-store kernel's configurations (N <= 16)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const std::vector<zsm::Span> iv = step_intervals(c);
+  std::vector<uint16_t*> grad(N);
+  const int n_layers = (int)c->plan.layers.size();
+  const bool pdl_ok = c->pdl && c->tma_ctas_opt <= 1;
+  bool launched = false;
+  for (size_t k = 0; k < iv.size(); ++k) {
+    const int64_t lo = iv[k].lo, hi = iv[k].hi;
+    const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
+    interval_grads(c, rank_grads, lo, 0, grad.data());
+    const int pdl = !pdl_ok ? zsm::kPdlNone
+                    : !launched ? zsm::kPdlWaitFirst
+                    : c->stage != ZERO_STAGE_3 ? zsm::kPdlEarly
+                                               : zsm::kPdlEarlyLoads;
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, zsm::AdamScalars{}, s, 0, pdl, nullptr, true);
+    if (st != ZERO_OK) return st;
+    launched = launched || hi > lo;
+  }
+  c->norm_fresh = true;
   return ZERO_OK;
 }
 
