@@ -84,6 +84,13 @@ def parse_args(argv=None):
                     help="16-bit storage of gradients and parameters (f16: IEEE binary16 with loss scale 1024)")
     ap.add_argument("--stage", type=int, choices=(1, 2, 3), default=2,
                     help="ZeRO stage of the bench line (the benchmark is stage 2)")
+    ap.add_argument("--rank-per-gpu", action="store_true",
+                    help="ZeRO with one logical rank per GPU (zero_dist_*: N = --gpus processes, each GPU "
+                         "holding its gradient and parameter replicas and its fp32 shard); one JSON line "
+                         "from rank 0")
+    ap.add_argument("--arm", choices=("fused", "nccl"), default="fused",
+                    help="with --rank-per-gpu: the library's fused peer-memory kernel, or NCCL "
+                         "reduce-scatter + the library's shard update + NCCL all-gather")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gpt-1.2b",
                     help="gpt-1.2b: the benchmark workload; flat-32m: a 33.5M-param flat buffer, "
                          "N = 8, one bucket (2 GB on the device); flat-8m-n64: 8.4M params, N = 64 "
@@ -802,6 +809,97 @@ def run_reference(args, world, rank, local):
     }), flush=True)
 
 
+def run_rank_per_gpu(args, world, rank, local):
+    """ZeRO-2 with one logical rank per GPU on the workload's layout (N = the
+    number of GPUs, not the workload's logical N): every step each rank
+    reduces its shard from the N gradient replicas (peers' over NVLink),
+    updates it and writes the result into every rank's parameter replica
+    (arm "fused"), or does the same with NCCL reduce-scatter and all-gather
+    around the library's shard update (arm "nccl").  Time = the max over
+    ranks of the CUDA-event time of the timed steps (host barriers between
+    the ranks inside the fused arm's steps are part of it)."""
+    import datetime
+
+    import torch
+    import torch.distributed as tdist
+
+    import synth
+    import zero_sharded_optimizer_sm_b200 as z
+    from synth import workloads as W
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist = init_dist(world, "nccl")
+    else:  # a one-rank group for the library's host protocol
+        import socket
+
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        tdist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                 timeout=datetime.timedelta(seconds=120))
+        dist = None
+    w = workload()
+    opt = z.ZeroDist(w.numel, w.layer_id, bench_stage(), z.AdamHParams(**w.hyper.__dict__), device=dev)
+    stream = torch.cuda.current_stream(dev)
+    s = stream.cuda_stream
+    offs = opt.offsets()
+    master = torch.zeros(opt.psi_pad, dtype=torch.float32, device=dev)
+    for off, n in zip(offs, w.numel):
+        synth.dev_f32(W.master_base(w), off, n, W.MASTER_DIST, master.data_ptr() + 4 * off, s)
+    opt.load_master(master)
+    del master
+    grads = opt.view(z.ZERO_VIEW_GRAD_BUF)
+    for off, n in zip(offs, w.numel):
+        synth.dev_bf16(W.grad_base(w, 1, rank), off, n, w.grad_dist, grads.data_ptr() + 2 * off, s)
+    torch.cuda.synchronize(dev)
+    nccl = args.arm == "nccl" and world > 1
+    if nccl:
+        shard = torch.empty(opt.shard, dtype=torch.bfloat16, device=dev)
+        gin = grads.view(torch.bfloat16)
+        pout = opt.view(z.ZERO_VIEW_PARAM).view(torch.bfloat16)
+        mine = pout[rank * opt.shard:(rank + 1) * opt.shard]
+
+        def one():
+            tdist.reduce_scatter_tensor(shard, gin, op=tdist.ReduceOp.AVG)
+            opt.adam_shard(shard)
+            tdist.all_gather_into_tensor(pout, mine)
+    else:
+        def one():
+            opt.step()
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier(dist if world > 1 else None)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, dist if world > 1 else None, dev)
+    S, N = opt.shard, world
+    nvlink_bytes = 2 * 2 * S * (N - 1)  # per rank per step: peers' gradient slices in, its result out
+    hbm_bytes = (4 * N + 24) * S        # per rank per step, every access counted once where it lands
+    out = {"metric": METRIC + " -- one logical rank per GPU", "value": w.psi * args.steps / (ms / 1e3),
+           "unit": "params/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+           "dtype": "fp32", "data": "synthetic (seeded counter-hash gradients and weights, no dataset)",
+           "config": {"workload": w.name, "params": w.psi, "n_ranks": N, "stage": bench_stage(),
+                      "arm": args.arm if world > 1 else "fused", "parallelism": f"dp{N}, one rank per GPU",
+                      "shard": S},
+           "per_rank": {"nvlink_bytes_per_step": nvlink_bytes, "hbm_bytes_per_step": hbm_bytes,
+                        "nvlink_GBps": nvlink_bytes / (ms / args.steps / 1e3) / 1e9,
+                        "hbm_GBps": hbm_bytes / (ms / args.steps / 1e3) / 1e9}}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    opt.close()
+    tdist.destroy_process_group()
+
+
 def run_overlap(args):
     """Overlap of the caller's backward with the step (ZERO_OPT_PIPELINE).
     grad_fn stands in for the backward: it draws each rank's gradients of the
@@ -899,6 +997,8 @@ def main(argv=None):
         run_stages(args)
     elif args.overlap:
         run_overlap(args)
+    elif args.rank_per_gpu:
+        run_rank_per_gpu(args, world, rank, local)
     else:
         run_ours(args, world, rank, local)
 
