@@ -4,10 +4,15 @@ It is for callers that cannot allocate device memory when they run the step
 (their device memory is owned by another allocator, or a cudaMalloc's
 possible device synchronisation is not acceptable where they run, or they
 keep no context to hold a scratch arena).  Its scratch is a fixed array in the
-library's own device memory.  This test calls it through the C ABI and checks
-its results against the context-based fused step (zero_step_resident of a
-stage-2 context with one bucket) on two calls in a row, within the
-tolerances the parity tests use.  The file name makes pytest collect it last.
+library's own device memory.  These tests call it through the C ABI and check
+it, on two calls in a row, against the context-based fused step
+(zero_step_resident of a stage-2 context with one bucket) within the
+tolerances the parity tests use, and against the CPU oracle's literal ZeRO-2
+run bit for bit: at N = 1, 3, 8, 17 and 64 on an interval that is not a
+multiple of a CTA's 2048 elements, with and without statistics; on an
+interval larger than one pass of the capped grid (the kernel's grid-stride
+loop); and with planted infinities and NaNs (the exact non-finite count).
+The file name makes pytest collect it last.
 """
 import ctypes
 import gc
@@ -20,6 +25,7 @@ torch = pytest.importorskip("torch")
 
 from harness import assert_bf16_close, assert_f32_close, to_np  # noqa: E402
 
+import oracle  # noqa: E402
 import synth  # noqa: E402
 from synth import workloads as W  # noqa: E402
 
@@ -105,3 +111,127 @@ def test_static_scratch_step_rejects_bad_arguments():
     assert call(8, hp=bad) == z.ZERO_EINVAL
     assert call(0) == z.ZERO_OK                       # an empty interval is a no-op
     torch.cuda.synchronize()
+
+
+def _bits_or_both_nan(got, ref, what):
+    """Equal bit patterns, except that two NaNs match whatever their payloads
+    (a NaN's payload is not part of the method's result)."""
+    g = np.ascontiguousarray(got)
+    r = np.ascontiguousarray(ref)
+    if g.dtype == np.float32:
+        gn, rn = np.isnan(g), np.isnan(r)
+        gb, rb = g.view(np.uint32), r.view(np.uint32)
+    else:
+        gb, rb = g.view(np.uint16), r.view(np.uint16)
+        gn = ((gb & 0x7F80) == 0x7F80) & ((gb & 0x7F) != 0)
+        rn = ((rb & 0x7F80) == 0x7F80) & ((rb & 0x7F) != 0)
+    ok = (gb == rb) | (gn & rn)
+    if not np.all(ok):
+        i = int(np.flatnonzero(~ok)[0])
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements differ; first at {i}: "
+                             f"got {hex(int(gb[i]))} ref {hex(int(rb[i]))}")
+
+
+def _oracle_and_static(n_ranks, n, seed, plant=None, stats_on=(True, False)):
+    """Two calls (t = 1, 2) of the allocation-free step on the caller's own
+    buffers, and the oracle's literal ZeRO-2 run of the same flat interval;
+    `plant(t, r, host_grad)` may overwrite gradient values on the host."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    w = W.Workload("no-alloc-oracle", [n], [0], n_ranks, (2,), None, synth.Dist(synth.NORMAL, 1e-2, zero_mod=37),
+                   W.MASTER_DIST, 2, W.Hyper(lr=2e-3, weight_decay=0.02), seed)
+    p = oracle.plan(w.numel, w.layer_id, n_ranks, 1 << 40)
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def g(t, r):
+        x = W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), w.grad_dist)
+        if plant is not None:
+            plant(t, r, x)
+        return x
+
+    ranks, reps = oracle.run(p, oracle.STAGE_Z2, m0, g, 2, oracle.AdamHP(**w.hyper.__dict__))
+    ref = oracle.full_view(p, oracle.STAGE_Z2, ranks)
+
+    hp = z.zero_adam_hparams(w.hyper.lr, w.hyper.beta1, w.hyper.beta2, w.hyper.eps, w.hyper.weight_decay)
+    s = torch.cuda.current_stream().cuda_stream
+    master = torch.from_numpy(m0[:n].copy()).cuda()
+    m = torch.zeros_like(master)
+    v = torch.zeros_like(master)
+    params = torch.full((n_ranks, n), 0x5555, dtype=torch.int16, device="cuda")
+    grads = torch.empty((n_ranks, n), dtype=torch.int16, device="cuda")
+    stats = torch.full((2,), float("nan"), dtype=torch.float64, device="cuda")
+    got_stats = []
+    for t in (1, 2):
+        for r in range(n_ranks):
+            grads[r].copy_(torch.from_numpy(g(t, r)[:n].view(np.int16)))
+        with_stats = stats_on[t - 1]
+        st = z.zero_fused_step_static(n_ranks, n, _ptrs([x.data_ptr() for x in grads]), master.data_ptr(),
+                                      m.data_ptr(), v.data_ptr(), _ptrs([x.data_ptr() for x in params]),
+                                      ctypes.byref(hp), t, stats.data_ptr() if with_stats else None, s)
+        assert st == z.ZERO_OK, z.STATUS_NAMES.get(st, st)
+        torch.cuda.synchronize()
+        if with_stats:
+            got_stats.append((float(stats[0].item()), int(stats[1:].view(torch.int64).item())))
+        else:
+            got_stats.append(None)
+    for key, dev in (("master", master), ("m", m), ("v", v)):
+        _bits_or_both_nan(to_np(dev), ref[key][:n], f"N={n_ranks} {key}")
+    for r in range(n_ranks):
+        _bits_or_both_nan(to_np(params[r]).view(np.uint16), ref["params"][:n], f"N={n_ranks} params {r}")
+    for t, gs in zip((1, 2), got_stats):
+        if gs is None:
+            continue
+        sq, nf = gs
+        assert nf == reps[t - 1].nonfinite, (t, nf, reps[t - 1].nonfinite)
+        if nf == 0:
+            tol = 2 * p.psi_pad * 2.0**-53 + 1e-15
+            assert abs(math.sqrt(sq) - reps[t - 1].grad_norm) <= tol * reps[t - 1].grad_norm
+    del master, m, v, params, grads, stats
+    return reps
+
+
+@pytest.mark.parametrize("n_ranks", [1, 3, 8, 17, 64])
+def test_static_step_equals_the_oracle_bit_for_bit(n_ranks):
+    """10,264 elements (five 2048-element CTA spans and a ragged 24), two calls
+    in a row, statistics on the first call and stats_out = NULL on the
+    second: master, m, v and every rank's parameters bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    _oracle_and_static(n_ranks, 5 * 2048 + 24, 0xAC0 + n_ranks, stats_on=(True, False))
+
+
+def test_static_step_grid_stride_over_a_long_interval():
+    """16,777,216 elements at N = 2: more than the capped grid covers in one
+    pass (148 SMs x resident CTAs x 2048 elements), so every CTA loops;
+    bit for bit against the oracle, statistics on both calls."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    _oracle_and_static(2, 1 << 24, 0xAD0, stats_on=(True, True))
+
+
+def test_static_step_counts_planted_nonfinite_values():
+    """Infinities, NaNs, opposite infinities in one element and a sum that
+    overflows bf16 planted in the ranks' gradients: the exact non-finite
+    count of the averaged gradient, and the states (NaN where the oracle's are
+    NaN) bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+
+    def plant(t, r, x):
+        if t != 2:
+            return
+        if r == 1:
+            x[100] = 0x7F80           # +inf
+        if r == 2:
+            x[2000] = 0x7FC1          # NaN
+        if r == 0:
+            x[5000] = 0x7F80          # +inf ...
+        if r == 3:
+            x[5000] = 0xFF80          # ... and -inf in the same element: NaN
+        x[7000] = 0x7F7F              # the largest finite bf16 on every rank: the sum overflows
+
+    reps = _oracle_and_static(4, 65536, 0xAE0, plant=plant, stats_on=(True, True))
+    assert reps[1].nonfinite == 4 and reps[0].nonfinite == 0

@@ -13,11 +13,12 @@
 // scratch the kernel needs (per-CTA gradient-norm partials, an arrival counter
 // and the step's sums) live in a file-scope __device__ array instead.
 //
-// The array is a fixed 32 KiB + 64 B (room for the partials of 2048 CTAs),
-// held on every GPU that loads the library until the process exits.  Every
-// call on a device shares it and it keeps the last call's contents, so calls
-// that overlap on the GPU (different streams, no ordering between them) race
-// on it; calls ordered on one stream do not.
+// The array is a fixed 32 KiB + 64 B (room for the partials of 2048 CTAs; a
+// launch never takes more CTAs than that, and the kernel's grid-stride loop
+// covers any interval), held on every GPU that loads the library until the
+// process exits.  Every call on a device shares it and it keeps the last
+// call's contents, so calls that overlap on the GPU (different streams, no
+// ordering between them) race on it; calls ordered on one stream do not.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -147,14 +148,17 @@ extern "C" zero_status zero_fused_step_static(int32_t n_ranks, int64_t n, const 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t n_vec = n / kVec;
   const int64_t want = std::max<int64_t>(1, (n_vec + kThreads - 1) / kThreads);
-  const int grid = (int)std::min<int64_t>(want, d->grid_cap);
-  if (grid > kStaticMaxCtas) return ZERO_ENOMEM;  // more CTAs than the scratch has partials for
+  // at most the CTAs the scratch has partials for (the loop is grid-stride)
+  const int grid = (int)std::min<int64_t>(std::min<int64_t>(want, d->grid_cap), kStaticMaxCtas);
   // what must start at zero: the arrival counter and the error word
   if (cudaMemsetAsync(d->scratch + kOffDone, 0, 8, s) != cudaSuccess) return ZERO_ECUDA;
   if (n_vec > 0) {
-    // binary32 scalars of step t, each rounded once from binary64
+    // binary32 scalars of step t, each rounded once from binary64; beta^t
+    // is t successive binary64 products (no state survives between calls
+    // to keep a running product in), left early once both have reached 0,
+    // where every further product stays exactly 0
     double p1 = 1.0, p2 = 1.0;
-    for (int64_t k = 0; k < t; ++k) {
+    for (int64_t k = 0; k < t && (p1 != 0.0 || p2 != 0.0); ++k) {
       p1 *= hp->beta1;
       p2 *= hp->beta2;
     }
