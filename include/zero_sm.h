@@ -177,6 +177,17 @@ enum {
                                     (tile, warps) pairs are 2048 x 8, 2048 x 16, 1024 x 4,
                                     1024 x 8 and 1024 x 16; another pair makes the next fused
                                     launch fail with ZERO_ECUDA; may be set at any time */
+  ZERO_OPT_WAIT_LIMIT_NS = 15,   /* limit, in ns of wall time, of each wait of the staged
+                                    kernels on their shared-memory ring (default 2e9, at most
+                                    60e9).  0 makes every ring wait one non-blocking test: a
+                                    wait whose copies have not already landed runs out at once,
+                                    so the kernel takes its failure path (error word, drain of
+                                    the copies in flight -- those waits keep 2 s -- and a
+                                    ZERO_ECUDA from the next synchronising call) without
+                                    anything stalling; it exists to test that path.  The
+                                    parameters and states of a step that ran out are partly
+                                    updated: restore them (zero_import_state) before going on.
+                                    May be set at any time */
   ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
                                     with no gather_fn) launches its fused kernels with
                                     programmatic dependent launch, so that each launch's CTAs

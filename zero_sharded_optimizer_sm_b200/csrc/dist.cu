@@ -116,6 +116,7 @@ zsm::NormScratch scratch_of(zero_dist* d) {
   ns.error = reinterpret_cast<unsigned int*>(tail + 4);
   ns.step_sq = reinterpret_cast<double*>(tail + 8);
   ns.step_nf = reinterpret_cast<unsigned long long*>(tail + 16);
+  ns.wait_ns = 2000000000ull;  // the register kernel it serves has no waits
   return ns;
 }
 

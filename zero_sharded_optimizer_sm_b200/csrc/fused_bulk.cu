@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
         if (k > 0) {
-          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag);
+          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag, a.ns.wait_ns);
           if (w != 0) {
             if (w == 1) atomicOr(a.ns.error, 1u);
             *abort_flag = 1;
@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
         if (tile >= n_tiles) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
-        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag);
+        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag, a.ns.wait_ns);
         if (w != 0) {
           if (w == 1) atomicOr(a.ns.error, 8u);
           *abort_flag = 1;
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
       // warp-uniform decisions, so that no lane is left waiting at __syncwarp
-      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.ns.wait_ns));
       if (!ok) {
         if (lane == 0) atomicOr(a.ns.error, 2u);
         *abort_flag = 1;

@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
         if (*abort_flag) break;
-        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u)) {
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u, a.ns.wait_ns)) {
           atomicOr(a.ns.error, 1u);
           *abort_flag = 1;
           break;
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(tma_threads<G>(), 1)
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
       // warp-uniform decisions, so that no lane is left waiting at __syncwarp
-      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.ns.wait_ns));
       if (!ok) {
         if (lane == 0) atomicOr(a.ns.error, 2u);
         *abort_flag = 1;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (tile >= n_tiles || *abort_flag) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
-        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u)) {
+        if (k > 0 && !mbar_wait(&empty[s], (k - 1) & 1u, a.ns.wait_ns)) {
           atomicOr(a.ns.error, 1u);
           *abort_flag = 1;
           break;
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       if (tile >= n_tiles) break;
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
-      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u));
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.ns.wait_ns));
       if (!ok) {
         if (lane == 0) atomicOr(a.ns.error, 2u);
         *abort_flag = 1;
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         // the tile's optimizer state
         const int ss = it % sstages;
         const unsigned sk = (unsigned)(it / sstages);
-        if (sk > 0 && !mbar_wait(&sempty[ss], (sk - 1) & 1u)) {
+        if (sk > 0 && !mbar_wait(&sempty[ss], (sk - 1) & 1u, a.ns.wait_ns)) {
           atomicOr(a.ns.error, 1u);
           *abort_flag = 1;
           break;
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
           const int ci = it * n_chunks + c;
           const int cs = ci % cstages;
           const unsigned ck = (unsigned)(ci / cstages);
-          if (ck > 0 && !mbar_wait(&cempty[cs], (ck - 1) & 1u)) {
+          if (ck > 0 && !mbar_wait(&cempty[cs], (ck - 1) & 1u, a.ns.wait_ns)) {
             atomicOr(a.ns.error, 1u);
             *abort_flag = 1;
             stop = true;
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
         const int ci = it * n_chunks + c;
         const int cs = ci % cstages;
         const unsigned ck = (unsigned)(ci / cstages);
-        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[cs], ck & 1u));
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&cfull[cs], ck & 1u, a.ns.wait_ns));
         if (!ok || __any_sync(0xFFFFFFFFu, *abort_flag != 0)) {
           if (!ok && lane == 0) atomicOr(a.ns.error, 2u);
           *abort_flag = 1;
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(tma_threads<1>(), 1)
       if (aborted) break;
       const int ss = it % sstages;
       const unsigned sk = (unsigned)(it / sstages);
-      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfull[ss], sk & 1u));
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&sfull[ss], sk & 1u, a.ns.wait_ns));
       if (!ok) {
         if (lane == 0) atomicOr(a.ns.error, 2u);
         *abort_flag = 1;

@@ -76,6 +76,7 @@ struct NormScratch {
   double* step_sq;                 // sum over the launches of the current step
   unsigned long long* step_nf;
   unsigned int* error;             // non-zero after a bounded device wait ran out
+  unsigned long long wait_ns;      // limit of a staged kernel's ring waits (0: one non-blocking test)
 };
 
 // Fused reduce + Adam + broadcast over one interval [lo, hi) of the flat space.
@@ -180,6 +181,7 @@ struct AdamBcastArgs {
   const AdamScalars* sc_dev;        // when set, the scalars are read here instead (StepState::sc)
   const ClipDecision* dec;          // the step's decision (clip coefficient, skip), or nullptr
   unsigned int* error;              // staged kernel: set when a bounded wait runs out
+  unsigned long long wait_ns;       // staged kernel: limit of its ring waits (0: one non-blocking test)
 };
 
 struct GatherArgs {

@@ -60,12 +60,30 @@ static __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned par
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false after kWaitNs.
-static __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+// Non-blocking test of whether the phase with the given parity has completed.
+static __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after `limit`
+// nanoseconds of %globaltimer.  limit = 0 tests once without blocking (a
+// phase not already complete counts as run out: the tests' way to make a
+// bounded wait expire without stalling anything).
+static __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity,
+                                                 unsigned long long limit = kWaitNs) {
+  if (limit == 0) return mbar_test_wait(bar, parity);
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
   while (!mbar_try_wait(bar, parity))
-    if (now_ns() - t0 > kWaitNs) return false;
+    if (now_ns() - t0 > limit) return false;
   return true;
 }
 
@@ -98,14 +116,16 @@ static __device__ __forceinline__ void bulk_load(void* dst, const void* src, uns
 }
 
 // Wait for the phase with the given parity, giving up when `abort_flag` is set
-// (another role of the CTA stopped) or after kWaitNs: 0 = done, 1 = timed
-// out, 2 = aborted.
-static __device__ __forceinline__ int mbar_wait_or_abort(uint64_t* bar, unsigned parity, volatile int* abort_flag) {
+// (another role of the CTA stopped) or after `limit` ns (0: one non-blocking
+// test): 0 = done, 1 = timed out, 2 = aborted.
+static __device__ __forceinline__ int mbar_wait_or_abort(uint64_t* bar, unsigned parity, volatile int* abort_flag,
+                                                         unsigned long long limit) {
+  if (limit == 0) return mbar_test_wait(bar, parity) ? 0 : 1;
   if (mbar_try_wait(bar, parity)) return 0;
   const unsigned long long t0 = now_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return 2;
-    if (now_ns() - t0 > kWaitNs) return 1;
+    if (now_ns() - t0 > limit) return 1;
   }
   return 0;
 }

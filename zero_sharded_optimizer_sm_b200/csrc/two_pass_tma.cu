@@ -88,8 +88,9 @@ __device__ __forceinline__ void ring_drain(const Ring& r, int stages, unsigned i
 
 // Producer side of one ring slot: wait for the consumers to release stage
 // `s` (phase k - 1); false (abort recorded) when the wait runs out.
-__device__ __forceinline__ bool acquire_stage(const Ring& r, int s, unsigned k, unsigned int* error) {
-  if (k > 0 && !mbar_wait(&r.empty[s], (k - 1) & 1u)) {
+__device__ __forceinline__ bool acquire_stage(const Ring& r, int s, unsigned k, unsigned int* error,
+                                              unsigned long long limit) {
+  if (k > 0 && !mbar_wait(&r.empty[s], (k - 1) & 1u, limit)) {
     atomicOr(error, 1u);
     *r.abort_flag = 1;
     return false;
@@ -99,8 +100,9 @@ __device__ __forceinline__ bool acquire_stage(const Ring& r, int s, unsigned k, 
 }
 
 // Consumer side: wait (warp-uniformly) for stage `s` phase k; false to stop.
-__device__ __forceinline__ bool consume_stage(const Ring& r, int s, unsigned k, unsigned int* error, int lane) {
-  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&r.full[s], k & 1u));
+__device__ __forceinline__ bool consume_stage(const Ring& r, int s, unsigned k, unsigned int* error, int lane,
+                                              unsigned long long limit) {
+  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&r.full[s], k & 1u, limit));
   if (!ok) {
     if (lane == 0) atomicOr(error, 2u);
     *r.abort_flag = 1;
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
         if (tile >= n_tiles || *ring.abort_flag) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
-        if (!acquire_stage(ring, s, k, a.ns.error)) break;
+        if (!acquire_stage(ring, s, k, a.ns.error, a.ns.wait_ns)) break;
         const int64_t e0 = tile * kTile;
         const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
         unsigned char* st = smem + (size_t)s * stage_bytes;
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
       if (tile >= n_tiles) break;
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
-      if (!consume_stage(ring, s, k, a.ns.error, lane)) break;
+      if (!consume_stage(ring, s, k, a.ns.error, lane, a.ns.wait_ns)) break;
       const int64_t e0 = tile * kTile;
       const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
       const unsigned char* st = smem + (size_t)s * stage_bytes;
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           const int ci = it * n_chunks + c;
           const int s = ci % stages;
           const unsigned k = (unsigned)(ci / stages);
-          if (!acquire_stage(ring, s, k, a.ns.error)) {
+          if (!acquire_stage(ring, s, k, a.ns.error, a.ns.wait_ns)) {
             stop = true;
             break;
           }
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
         const int ci = it * n_chunks + c;
         const int s = ci % stages;
         const unsigned k = (unsigned)(ci / stages);
-        if (!consume_stage(ring, s, k, a.ns.error, lane)) {
+        if (!consume_stage(ring, s, k, a.ns.error, lane, a.ns.wait_ns)) {
           stop = true;
           break;
         }
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
         if (tile >= n_tiles || *ring.abort_flag) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
-        if (!acquire_stage(ring, s, k, a.error)) break;
+        if (!acquire_stage(ring, s, k, a.error, a.wait_ns)) break;
         const int64_t e0 = tile * kTile;
         const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
         unsigned char* st = smem + (size_t)s * kBcastStageBytes;
@@ -333,7 +335,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
       if (tile >= n_tiles) break;
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
-      if (!consume_stage(ring, s, k, a.error, lane)) break;
+      if (!consume_stage(ring, s, k, a.error, lane, a.wait_ns)) break;
       const int64_t e0 = tile * kTile;
       const int64_t cnt = (n_elem - e0) < kTile ? (n_elem - e0) : kTile;
       const unsigned char* st = smem + (size_t)s * kBcastStageBytes;

@@ -52,6 +52,7 @@ struct zero_ctx {
   int tma_ctas_opt = 0;    // CTAs per SM of the staged kernel, 0 = the library's choice
   int tma_tile_opt = 0;    // bulk-store kernel: elements per tile, 0 = the library's choice
   int tma_warps_opt = 0;   // bulk-store kernel: consumer warps, 0 = the library's choice
+  unsigned long long wait_ns = 2000000000ull;  // limit of the staged kernels' ring waits (ZERO_OPT_WAIT_LIMIT_NS)
   int tma_grid_key = -1;   // configuration the cached grid cap belongs to
   int tma_grid_cap = 0;
   // arena layout (bytes)
@@ -190,6 +191,7 @@ zsm::NormScratch norm_scratch(zero_ctx* c) {
   ns.step_nf = reinterpret_cast<unsigned long long*>(s + 16 * zsm::kMaxGrid + 8);
   ns.done = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 16);
   ns.error = reinterpret_cast<unsigned int*>(s + 16 * zsm::kMaxGrid + 20);
+  ns.wait_ns = c->wait_ns;
   return ns;
 }
 
@@ -820,6 +822,7 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     b.sc_dev = &state_ptr(c)->sc;
     b.dec = dec;
     b.error = norm_scratch(c).error;
+    b.wait_ns = c->wait_ns;
     o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
     if (b.n_vec > 0) {
       // stages 2 and 3 read every owner's reduced gradient from the one shard array
@@ -972,6 +975,11 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   if (key == ZERO_OPT_TMA_STAGES) {
     if (value < 0 || value > zsm::kTmaMaxStages) return fail(c, ZERO_EINVAL, "stages must be 0..%d", zsm::kTmaMaxStages);
     c->tma_stages_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_WAIT_LIMIT_NS) {
+    if (value < 0 || value > 60000000000ll) return fail(c, ZERO_EINVAL, "wait limit must be 0..60e9 ns");
+    c->wait_ns = (unsigned long long)value;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_TMA_TILE) {
