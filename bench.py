@@ -44,7 +44,9 @@ _CSRC = os.path.join(ROOT, "zero_sharded_optimizer_sm_b200", "csrc")
 # void once any of them changes)
 KERNEL_SOURCES = {"tma": [os.path.join(_CSRC, f) for f in ("fused_tma.cu", "tma_pipe.cuh", "device_math.cuh",
                                                             "kernels.cuh")],
-                  "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh", "kernels.cuh")]}
+                  "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh", "kernels.cuh")],
+                  "bulk": [os.path.join(_CSRC, f) for f in ("fused_bulk.cu", "tma_pipe.cuh", "device_math.cuh",
+                                                            "kernels.cuh")]}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
 
 
@@ -58,9 +60,12 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--blocks-per-sm", type=int, default=0)
-    ap.add_argument("--kernel", choices=("auto", "register", "tma"), default="auto",
+    ap.add_argument("--kernel", choices=("auto", "register", "tma", "bulk"), default="auto",
                     help="fused-step kernel (auto = the library's choice for this N)")
     ap.add_argument("--replica-pad", type=int, default=0)
+    ap.add_argument("--tile", type=int, default=0, help="bulk-store kernel: elements per tile (0 = library's choice)")
+    ap.add_argument("--warps", type=int, default=0, help="bulk-store kernel: consumer warps (0 = library's choice)")
+    ap.add_argument("--ring", type=int, default=0, help="staged kernels: ring depth (0 = library's choice)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch the step's fused kernels plainly (no programmatic dependent launch)")
     ap.add_argument("--sweep", action="store_true",
@@ -278,6 +283,8 @@ def workload():
 
 def fused_kernel_name(fc: dict, n_ranks: int) -> str:
     """The fused kernel a context launches, from its zero_fused_config."""
+    if fc["kernel"] == "bulk":
+        return "fused_bulk_kernel"
     if fc["kernel"] != "tma":
         return "fused_step_kernel"
     if n_ranks > 16:
@@ -406,7 +413,8 @@ def run_ours(args, world, rank, local):
     opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, stage, bucket_elems=w.bucket_elems,
                           hparams=z.AdamHParams(**w.hyper.__dict__), keep_grad_shards=args.clip > 0,
                           replica_pad=args.replica_pad, blocks_per_sm=args.blocks_per_sm,
-                          kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel], pipeline=True,
+                          kernel={"auto": 0, "register": 1, "tma": 2, "bulk": 3}[args.kernel], pipeline=True,
+                          tma_tile=args.tile, tma_warps=args.warps, tma_stages=args.ring,
                           dtype=z.ZERO_DTYPE_F16 if args.dtype == "f16" else z.ZERO_DTYPE_BF16, device=dev)
     if args.dtype == "f16":
         opt.set_loss_scale(1024.0)
@@ -481,9 +489,13 @@ def run_ours(args, world, rank, local):
     opt.set_timing(False)
     kernel_ms_isolated = kt["ms"] / kt["launches"] if kt["launches"] else None
     peak, peak_kind = measured_peaks()
+    pattern = pattern_ceiling(opt, rep_list, stream, model_bytes_per_step, args) if args.clip <= 0 else None
+    copy_gbs = same_box_copy(dev)
     elems_per_launch = w.psi / intervals
     fc = opt.fused_config()
-    ckey = f"stage{stage}_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else "")
+    ckey = f"stage{stage}_N{w.n_ranks}_{fc['kernel']}" + (f"_g{fc['groups']}_s{fc['stages']}" if fc["kernel"] == "tma" else
+                                                          f"_t{fc['tile']}_w{fc['groups']}_s{fc['stages']}"
+                                                          if fc["kernel"] == "bulk" else "")
     traffic = traffic_for_current_kernel(fc["kernel"], ckey, elems_per_launch) if args.clip <= 0 else None
 
     # end to end through the C ABI: every bucket's N gradient slices copied
@@ -566,7 +578,12 @@ def run_ours(args, world, rank, local):
                      "kernel_ms_per_launch_isolated": kernel_ms_isolated,
                      "achieved_isolated": (kt["model_bytes"] / kt["launches"] / (kernel_ms_isolated / 1e3) / 1e9
                                            if kernel_ms_isolated else None),
-                     "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None},
+                     "frac_of_nominal_8tbs": (achieved / NOMINAL_HBM_GBS) if achieved else None,
+                     "pattern_peak": pattern["GBps"] if pattern else None,
+                     "frac_of_pattern": (achieved / pattern["GBps"]) if pattern else None,
+                     "pattern_how": pattern["how"] if pattern else None,
+                     "copy_same_box": copy_gbs,
+                     "frac_of_copy_same_box": (achieved / copy_gbs) if copy_gbs else None},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": region_launches,
@@ -578,6 +595,65 @@ def run_ours(args, world, rank, local):
     opt.close()
     if dist is not None:
         dist.destroy_process_group()
+
+
+def pattern_ceiling(opt, rep_list, stream, model_bytes_per_step, args, steps=None):
+    """The step's own traffic pattern with no arithmetic: the movement-only
+    twin of the bulk-store kernel (zero_probe_pattern) over the same
+    intervals, in the same launch chaining, timed like the step.  GB/s of the
+    step's byte model over its time; None where no twin exists (N > 16)."""
+    import torch
+
+    import zero_sharded_optimizer_sm_b200 as z
+
+    steps = steps or max(20, min(args.steps, 100))
+    try:
+        for _ in range(3):
+            opt.probe_pattern(rep_list)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            opt.probe_pattern(rep_list)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    except z.ZeroError:
+        return None
+    ms = e0.elapsed_time(e1) / steps
+    fc = opt.fused_config()
+    return {"GBps": model_bytes_per_step / (ms / 1e3) / 1e9, "ms_per_step": ms, "steps": steps,
+            "how": f"zero_probe_pattern: the bulk-store kernel's movement-only twin (same bulk loads, "
+                   f"shared-memory traffic and bulk stores, no reduction or Adam) over the step's "
+                   f"intervals, tile {fc.get('tile')}, same launch chaining; the step's byte model over its "
+                   f"CUDA-event time"}
+
+
+def same_box_copy(dev, gib: int = 4, reps: int = 20):
+    """Device-to-device copy of a 4 GiB buffer on this GPU (torch's copy
+    kernel), read + write bytes over CUDA-event time: the plain-copy ceiling
+    of the box the step ran on."""
+    import torch
+
+    try:
+        a = torch.empty(gib << 30, dtype=torch.uint8, device=dev)
+        b = torch.empty_like(a)
+    except RuntimeError:
+        return None
+    for _ in range(3):
+        b.copy_(a)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        b.copy_(a)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    del a, b
+    torch.cuda.empty_cache()
+    return 2 * (gib << 30) / (ms / 1e3) / 1e9
 
 
 # ------------------------------------------------------------------- sweep ----
@@ -613,7 +689,7 @@ def run_sweep(args):
                 # 4N+24 model); the unfused path needs the shard arena
                 opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, z.ZERO_STAGE_2,
                                       keep_grad_shards=(name == "unfused"), grad_buffers=False,
-                                      kernel={"auto": 0, "register": 1, "tma": 2}[args.kernel])
+                                      kernel={"auto": 0, "register": 1, "tma": 2, "bulk": 3}[args.kernel])
                 mv = opt.view(z.ZERO_VIEW_MASTER)
                 synth.dev_f32(W.master_base(w), 0, elems, W.MASTER_DIST, mv.data_ptr(), s)
                 opt.load_master(None)
@@ -680,7 +756,7 @@ def run_stages(args):
 
     torch.cuda.set_device(0)
     s = torch.cuda.current_stream().cuda_stream
-    kern = {"auto": 0, "register": 1, "tma": 2}[args.kernel]
+    kern = {"auto": 0, "register": 1, "tma": 2, "bulk": 3}[args.kernel]
 
     def master_fill(opt, w):
         mv = opt.view(z.ZERO_VIEW_MASTER)
@@ -919,7 +995,7 @@ def run_overlap(args):
 
     torch.cuda.set_device(0)
     s = torch.cuda.current_stream().cuda_stream
-    kern = {"auto": 0, "register": 1, "tma": 2}[args.kernel]
+    kern = {"auto": 0, "register": 1, "tma": 2, "bulk": 3}[args.kernel]
     cells = [(W.gpt_1p2b_n8(), 3, None), (W.gpt_1p2b_n8(), 2, 200_000_000), (W.gpt_85m_n8(), 3, None),
              (W.gpt_85m_n8(), 2, 20_000_000)]
     for w, stage, bucket in cells:

@@ -172,11 +172,15 @@ enum {
                                     Default 0; before zero_bind */
   ZERO_OPT_TMA_TILE = 13,        /* bulk-store kernel: elements per tile, 1024 or 2048 (0 = the
                                     library's choice); may be set at any time */
-  ZERO_OPT_TMA_WARPS = 14,       /* bulk-store kernel: consumer warps, 4, 8 or 16, with 8 or 4
-                                    elements per lane (0 = the library's choice); the built
+  ZERO_OPT_TMA_WARPS = 14,       /* bulk-store kernel: consumer warps, 4, 8 or 16 (8, 4 or 2
+                                    elements per lane; 0 = the library's choice); the built
                                     (tile, warps) pairs are 2048 x 8, 2048 x 16, 1024 x 4,
-                                    1024 x 8 and 1024 x 16; another pair makes the next fused
-                                    launch fail with ZERO_ECUDA; may be set at any time */
+                                    1024 x 8 and 1024 x 16 for N <= 16, 2048 x 8 and 1024 x 8
+                                    above; another pair makes the next fused launch fail with
+                                    ZERO_ECUDA; may be set at any time */
+  ZERO_OPT_STORE_HINT = 16,      /* bulk-store kernel: 1 marks its bulk stores L2 evict-first
+                                    (written lines leave L2 first), 0 (default) plain; values
+                                    are unchanged either way; may be set at any time */
   ZERO_OPT_WAIT_LIMIT_NS = 15,   /* limit, in ns of wall time, of each wait of the staged
                                     kernels on their shared-memory ring (default 2e9, at most
                                     60e9).  0 makes every ring wait one non-blocking test: a
@@ -221,15 +225,15 @@ enum { ZERO_DTYPE_BF16 = 0, ZERO_DTYPE_F16 = 1 };
  *             bounded; one that runs out is reported as ZERO_ECUDA by the next
  *             synchronising call (zero_read_stats, zero_step with stats,
  *             zero_kernel_timing).
- *   BULK:     (N <= 16) the staged loads of TMA with bulk stores: one CTA
- *             per SM, a producer thread streaming tiles (ZERO_OPT_TMA_TILE) of
- *             the N replicas and master/m/v into a ring of shared-memory
- *             stages, consumer warps (ZERO_OPT_TMA_WARPS) that compute and
- *             write every result back into the stage, and a storer thread
- *             that copies the stage's results to master/m/v and the N
+ *   BULK:     the staged loads of TMA with bulk stores: one CTA per SM, a
+ *             producer thread streaming tiles (ZERO_OPT_TMA_TILE) of the N
+ *             replicas and master/m/v into a ring of shared-memory stages
+ *             (above N = 16 the replicas in chunks of 8 ranks through a ring
+ *             of their own), consumer warps (ZERO_OPT_TMA_WARPS) that
+ *             compute and write every result back into shared memory, and a
+ *             storer thread that copies the results to master/m/v and the N
  *             destinations with bulk copies (shared -> global), so that no
  *             consumer lane issues a global store.  Bounded waits as TMA.
- *             Above N = 16 the rank-chunked TMA kernel runs instead.
  *   AUTO:     the staged kernel for every N, in the configuration measured
  *             fastest on B200 for that N (zero_fused_config reports it). */
 enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2, ZERO_KERNEL_BULK = 3 };
@@ -682,8 +686,9 @@ zero_status zero_fused_tile(const zero_ctx* ctx, int32_t* tile);
  * ceiling that the step reaches.  Not part of the method: no passage of the
  * pages defines it; measurement plumbing.
  * Errors: ZERO_EINVAL (NULL or misaligned pointers), ZERO_ESTATE (not bound
- * or not initialised), ZERO_ENOTIMPL (N > 16, or the configuration of
- * ZERO_OPT_TMA_TILE / ZERO_OPT_TMA_WARPS is not built), ZERO_ECUDA (launch).
+ * or not initialised), ZERO_ENOTIMPL (the configuration of
+ * ZERO_OPT_TMA_TILE / ZERO_OPT_TMA_WARPS is not built at this N), ZERO_ECUDA
+ * (launch).
  */
 zero_status zero_probe_pattern(zero_ctx* ctx, const void* const* rank_grads, void* stream);
 

@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
 STAGE_OF = {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2, 3: oracle.STAGE_Z3}
 BULK = 3  # ZERO_KERNEL_BULK
 CONFIGS = [(2048, 8), (2048, 16), (1024, 4), (1024, 8), (1024, 16)]
+CHUNKED_CONFIGS = [(2048, 8), (1024, 8)]  # N > 16: the rank-chunked form
 # ragged layout: a zero-size tensor, tensors that are not multiples of 8, and
 # 220,000 elements in all (over a hundred 1024-element tiles, a ragged last
 # tile, several tiles per CTA at the small bucket)
@@ -120,20 +121,21 @@ def _run_steps(opt, fill, w, stage, p, reps, tag, gathered=None):
         assert abs(st["grad_norm"] - reps[t - 1].grad_norm) <= (2 * n * 2.0**-53 + 1e-15) * reps[t - 1].grad_norm, tag
 
 
-@pytest.mark.parametrize("n_ranks", [1, 3, 8, 16])
+@pytest.mark.parametrize("n_ranks", [1, 3, 8, 16, 17, 33])
 @pytest.mark.parametrize("stage", [1, 2, 3])
 @pytest.mark.parametrize("small_bucket", [False, True])
 def test_every_bulk_configuration_against_the_oracle(n_ranks, stage, small_bucket):
     """Every built (tile, warps) pair, with and without the reduced-gradient
     shards, on a ragged 220K-element layout: one bucket, or 8192-element
     buckets (many intervals shorter than a tile); ZeRO-3 also checks every
-    gathered layer buffer of the last step."""
+    gathered layer buffer of the last step.  Above 16 ranks the rank-chunked
+    form (8 ranks a chunk; 33 ranks end on a chunk of one)."""
     numel, layer = RAGGED
     p_all = oracle.plan(numel, layer, n_ranks, 1 << 40)
     bucket = 8192 if small_bucket else p_all.psi_pad
     w = _workload(numel, layer, n_ranks, stage, bucket)
     p, ranks, reps, ref = _oracle(w, stage, bucket)
-    for tile, warps in CONFIGS:
+    for tile, warps in (CONFIGS if n_ranks <= 16 else CHUNKED_CONFIGS):
         for keep in (True, False):
             tag = f"N={n_ranks} stage {stage} bucket {bucket} tile {tile} warps {warps} keep {keep}"
             opt, fill = _make(w, stage, bucket, keep, tile, warps)
@@ -221,13 +223,13 @@ def test_resident_steps_chained_launches(stage, pdl):
 
 
 @pytest.mark.parametrize("stage", [1, 2, 3])
-def test_probe_pattern_leaves_the_state(stage):
+@pytest.mark.parametrize("n_ranks", [4, 17])
+def test_probe_pattern_leaves_the_state(stage, n_ranks):
     """The movement-only pass between two steps changes no bit of master, m,
     v or the parameters and does not move the step counter: the second step
-    still equals the oracle's second step."""
+    still equals the oracle's second step (one-stage and rank-chunked twins)."""
     z = _z()
     numel, layer = RAGGED
-    n_ranks = 4
     w = _workload(numel, layer, n_ranks, stage, 16384, steps=2)
     p, ranks, reps, ref = _oracle(w, stage, 16384)
     opt, fill = _make(w, stage, 16384, True, 1024, 8)
@@ -250,13 +252,18 @@ def test_probe_pattern_leaves_the_state(stage):
     opt.close()
 
 
-def test_probe_pattern_refuses_beyond_16_ranks():
+def test_probe_pattern_refuses_a_configuration_that_is_not_built():
+    """Four consumer warps exist for the one-stage kernel only: at 17 ranks
+    the probe refuses them (ZERO_ENOTIMPL) and a step fails at launch."""
     z = _z()
     numel, layer = [4096], [0]
     w = _workload(numel, layer, 17, 2, 1 << 20, steps=1)
-    opt, _ = _make(w, 2, None, True, 1024, 8)
+    opt, _ = _make(w, 2, None, True, 1024, 4)
     reps_t = torch.zeros((17, opt.psi_pad), dtype=torch.int16, device="cuda")
     with pytest.raises(z.ZeroError) as e:
         opt.probe_pattern(list(reps_t))
     assert e.value.status == z.ZERO_ENOTIMPL
+    with pytest.raises(z.ZeroError) as e:
+        opt.step_resident(list(reps_t))
+    assert e.value.status == z.ZERO_ECUDA
     opt.close()

@@ -49,6 +49,7 @@ ZERO_OPT_PDL = 12
 ZERO_OPT_TMA_TILE = 13
 ZERO_OPT_TMA_WARPS = 14
 ZERO_OPT_WAIT_LIMIT_NS = 15
+ZERO_OPT_STORE_HINT = 16
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -523,6 +524,10 @@ class ZeroOptimizer:
 
     def set_kernel(self, kernel: int):
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
+
+    def set_store_hint(self, on: bool):
+        """Bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_STORE_HINT, 1 if on else 0), "zero_set_option")
 
     def set_wait_limit(self, ns: int):
         """Limit of the staged kernels' ring waits in ns (0: one non-blocking test; see ZERO_OPT_WAIT_LIMIT_NS)."""

@@ -55,10 +55,14 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
                 print(res.stderr, end="")
             if res.returncode != 0:
                 raise subprocess.CalledProcessError(res.returncode, res.args, res.stdout, res.stderr)
-    link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs]
+    # link beside the library and rename over it: a reader never sees a
+    # half-written file
+    tmp = LIB + ".tmp"
+    link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(link))
     subprocess.run(link, check=True)
+    os.replace(tmp, LIB)
     return LIB
 
 

@@ -95,6 +95,7 @@ struct FusedArgs {
   int accumulate;                   // 0: first launch of the step (norm overwrites)
   float inv_n;                      // binary32 1/N
   int pdl;                          // PdlMode of this launch
+  int store_hint;                   // bulk-store kernel: 1 = its stores carry an L2 evict-first hint
   AdamScalars sc;
   const AdamScalars* sc_dev;        // when set, the scalars are read here instead (StepState::sc)
   NormScratch ns;
@@ -236,17 +237,19 @@ int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
 // replicas stream in chunks of 8 ranks through a `cstages`-deep ring.
 cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s);
 
-// Staged kernel with bulk stores (fused_bulk.cu), N <= 16: tiles of `tile`
-// elements, `warps` consumer warps, a ring of at most `max_stages` stages (0 =
-// as many as fit); one CTA per SM.  `move` launches the movement-only twin
-// (same copies, no arithmetic; `opaque` must be 0), which measures the
-// pattern's ceiling and is never part of a step.
+// Staged kernel with bulk stores (fused_bulk.cu): tiles of `tile` elements,
+// `warps` consumer warps, a ring of at most `max_stages` stages (0 = the
+// default depth); above N = 16 the rank-chunked form (max_stages bounds its
+// chunk ring).  One CTA per SM.  `move` launches the movement-only twin (same
+// copies, no arithmetic; `opaque` must be 0), which measures the pattern's
+// ceiling and is never part of a step.
 cudaError_t launch_fused_bulk(int mode, const FusedArgs& a, int grid, int tile, int warps, int max_stages, bool move,
                               uint32_t opaque, cudaStream_t s);
 // Ring depth of that kernel for N, the tile and whether the averaged gradient
-// is stored (0 when nothing fits); whether (tile, warps) is a built configuration.
+// is stored (the chunk ring above N = 16; 0 when nothing fits); whether
+// (tile, warps) is a built configuration at that N.
 int bulk_stages_for(int n_ranks, int tile, bool need_g, int max_stages);
-bool bulk_config_valid(int tile, int warps);
+bool bulk_config_valid(int n_ranks, int tile, int warps);
 cudaError_t bulk_configure();  // opt in to the large dynamic smem (current device)
 
 // Resident CTAs per SM of the staged kernel in that configuration (0 on error).

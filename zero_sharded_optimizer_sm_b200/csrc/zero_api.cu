@@ -53,6 +53,7 @@ struct zero_ctx {
   int tma_tile_opt = 0;    // bulk-store kernel: elements per tile, 0 = the library's choice
   int tma_warps_opt = 0;   // bulk-store kernel: consumer warps, 0 = the library's choice
   unsigned long long wait_ns = 2000000000ull;  // limit of the staged kernels' ring waits (ZERO_OPT_WAIT_LIMIT_NS)
+  int store_hint = 0;      // bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)
   int tma_grid_key = -1;   // configuration the cached grid cap belongs to
   int tma_grid_cap = 0;
   // arena layout (bytes)
@@ -362,12 +363,12 @@ int tma_grid_cap(zero_ctx* c) {
 
 // Whether the fused step runs a shared-memory staged kernel: the all-ranks
 // stage kernel for N <= 16, the rank-chunked one above.
-bool use_chunked(const zero_ctx* c) {
-  if (c->plan.n_ranks <= zsm::kTmaMaxRanks) return false;
-  return c->kernel_opt != ZERO_KERNEL_REGISTER;  // AUTO, TMA and BULK
-}
-
 bool use_bulk(const zero_ctx* c);
+
+bool use_chunked(const zero_ctx* c) {
+  if (c->plan.n_ranks <= zsm::kTmaMaxRanks || use_bulk(c)) return false;
+  return c->kernel_opt != ZERO_KERNEL_REGISTER;  // AUTO and TMA
+}
 
 bool use_tma(const zero_ctx* c) {
   if (use_chunked(c)) return true;
@@ -391,11 +392,11 @@ int bulk_stages(const zero_ctx* c) {
   return zsm::bulk_stages_for(c->plan.n_ranks, bulk_tile(c), bulk_need_g(c), c->tma_stages_opt);
 }
 bool bulk_fits(const zero_ctx* c) {
-  return c->plan.n_ranks <= zsm::kTmaMaxRanks && zsm::bulk_config_valid(bulk_tile(c), bulk_warps(c)) &&
-         bulk_stages(c) > 0;
+  return zsm::bulk_config_valid(c->plan.n_ranks, bulk_tile(c), bulk_warps(c)) && bulk_stages(c) > 0;
 }
-// Asked for and N <= 16; a (tile, warps) pair that is not built fails at launch.
-bool use_bulk(const zero_ctx* c) { return c->kernel_opt == ZERO_KERNEL_BULK && c->plan.n_ranks <= zsm::kTmaMaxRanks; }
+// Asked for (any N; the rank-chunked form above 16); a (tile, warps) pair
+// that is not built fails at launch.
+bool use_bulk(const zero_ctx* c) { return c->kernel_opt == ZERO_KERNEL_BULK; }
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
@@ -489,6 +490,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   a.sc_dev = sc_dev;
   a.ns = norm_scratch(c);
   a.pdl = c->timing ? zsm::kPdlNone : pdl;  // an event record between launches ends the overlap
+  a.store_hint = c->store_hint;
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
@@ -975,6 +977,11 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
   if (key == ZERO_OPT_TMA_STAGES) {
     if (value < 0 || value > zsm::kTmaMaxStages) return fail(c, ZERO_EINVAL, "stages must be 0..%d", zsm::kTmaMaxStages);
     c->tma_stages_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_STORE_HINT) {
+    if (value != 0 && value != 1) return fail(c, ZERO_EINVAL, "store hint must be 0 or 1");
+    c->store_hint = (int)value;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_WAIT_LIMIT_NS) {
@@ -1590,7 +1597,7 @@ zero_status zero_probe_pattern(zero_ctx* c, const void* const* rank_grads, void*
     if (!rank_grads[r] || !aligned16(rank_grads[r]))
       return fail(c, ZERO_EINVAL, "rank_grads[%d] is null or not 16-byte aligned", r);
   if (!bulk_fits(c))
-    return fail(c, ZERO_ENOTIMPL, "the movement-only pass exists for the bulk-store kernel's configurations (N <= 16)");
+    return fail(c, ZERO_ENOTIMPL, "the movement-only pass exists for the bulk-store kernel's built configurations");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const std::vector<zsm::Span> iv = step_intervals(c);
   std::vector<uint16_t*> grad(N);
