@@ -582,6 +582,7 @@ def run_ours(args, world, rank, local):
                      "pattern_peak": pattern["GBps"] if pattern else None,
                      "frac_of_pattern": (achieved / pattern["GBps"]) if pattern else None,
                      "pattern_how": pattern["how"] if pattern else None,
+                     "pattern_by_config": pattern["by_config"] if pattern else None,
                      "copy_same_box": copy_gbs,
                      "frac_of_copy_same_box": (achieved / copy_gbs) if copy_gbs else None},
         "cpu_baseline": cpu,
@@ -600,33 +601,48 @@ def run_ours(args, world, rank, local):
 def pattern_ceiling(opt, rep_list, stream, model_bytes_per_step, args, steps=None):
     """The step's own traffic pattern with no arithmetic: the movement-only
     twin of the bulk-store kernel (zero_probe_pattern) over the same
-    intervals, in the same launch chaining, timed like the step.  GB/s of the
-    step's byte model over its time; None where no twin exists (N > 16)."""
+    intervals, in the same launch chaining, timed like the step, in the
+    step's configuration and in four others (tiles of 1024 and 2048
+    elements, 8 or 16 consumer warps, 2-4 stages).  The twin's pace depends
+    on its configuration -- without arithmetic its copies bunch up -- so the
+    ceiling is the fastest of them.  GB/s of the step's byte model over the
+    twin's time; None where no twin exists."""
     import torch
 
     import zero_sharded_optimizer_sm_b200 as z
 
-    steps = steps or max(20, min(args.steps, 100))
-    try:
-        for _ in range(3):
-            opt.probe_pattern(rep_list)
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            opt.probe_pattern(rep_list)
-        e1.record(stream)
-        torch.cuda.synchronize()
-    except z.ZeroError:
-        return None
-    ms = e0.elapsed_time(e1) / steps
+    steps = steps or max(20, min(args.steps, 60))
     fc = opt.fused_config()
-    return {"GBps": model_bytes_per_step / (ms / 1e3) / 1e9, "ms_per_step": ms, "steps": steps,
-            "how": f"zero_probe_pattern: the bulk-store kernel's movement-only twin (same bulk loads, "
-                   f"shared-memory traffic and bulk stores, no reduction or Adam) over the step's "
-                   f"intervals, tile {fc.get('tile')}, same launch chaining; the step's byte model over its "
-                   f"CUDA-event time"}
+    own = (fc["tile"], fc["groups"], fc["stages"]) if fc["kernel"] == "bulk" else None
+    configs = [own] if own else []
+    configs += [c for c in ((1024, 8, 3), (1024, 8, 4), (2048, 8, 2), (2048, 16, 2)) if c != own]
+    results = {}
+    for cfg in configs:
+        try:
+            opt.set_staged(*cfg)
+            for _ in range(3):
+                opt.probe_pattern(rep_list)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                opt.probe_pattern(rep_list)
+            e1.record(stream)
+            torch.cuda.synchronize()
+        except z.ZeroError:
+            continue
+        results["x".join(map(str, cfg))] = model_bytes_per_step / (e0.elapsed_time(e1) / steps / 1e3) / 1e9
+    opt.set_staged(args.tile, args.warps, args.ring)  # the step's own configuration again
+    if not results:
+        return None
+    best = max(results, key=results.get)
+    return {"GBps": results[best], "by_config": results, "best_config": best,
+            "own_config": "x".join(map(str, own)) if own else None,
+            "how": "zero_probe_pattern: the bulk-store kernel's movement-only twin (same bulk loads, shared-memory "
+                   "traffic and bulk stores, no reduction or Adam) over the step's intervals with the same launch "
+                   "chaining, in the step's configuration and four others (tile x consumer warps x stages); the "
+                   "fastest, as the step's byte model over its CUDA-event time"}
 
 
 def same_box_copy(dev, gib: int = 4, reps: int = 20):

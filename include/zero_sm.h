@@ -138,8 +138,8 @@ enum {
                                     the two passes of a clipped step -- (read with
                                     zero_kernel_timing); may be set at any time; default 0 */
   ZERO_OPT_KERNEL = 5,           /* fused-step kernel: ZERO_KERNEL_AUTO (default),
-                                    ZERO_KERNEL_REGISTER or ZERO_KERNEL_TMA; may be set at any
-                                    time */
+                                    ZERO_KERNEL_REGISTER, ZERO_KERNEL_TMA or ZERO_KERNEL_BULK;
+                                    may be set at any time */
   ZERO_OPT_GRAD_BUFFERS = 6,     /* 1 (default) sizes the GRADS arena; 0 drops it for callers
                                     that only use zero_step_resident and the calls given explicit
                                     pointers (zero_step then returns ZERO_ESTATE) */
@@ -178,9 +178,10 @@ enum {
                                     1024 x 8 and 1024 x 16 for N <= 16, 2048 x 8 and 1024 x 8
                                     above; another pair makes the next fused launch fail with
                                     ZERO_ECUDA; may be set at any time */
-  ZERO_OPT_STORE_HINT = 16,      /* bulk-store kernel: 1 marks its bulk stores L2 evict-first
-                                    (written lines leave L2 first), 0 (default) plain; values
-                                    are unchanged either way; may be set at any time */
+  ZERO_OPT_STORE_HINT = 16,      /* bulk-store kernel: 1 (default) marks its bulk stores L2
+                                    evict-first (written lines leave L2 first; measured 0.5-4 %
+                                    faster on B200), 0 plain; values are unchanged either way;
+                                    may be set at any time */
   ZERO_OPT_WAIT_LIMIT_NS = 15,   /* limit, in ns of wall time, of each wait of the staged
                                     kernels on their shared-memory ring (default 2e9, at most
                                     60e9).  0 makes every ring wait one non-blocking test: a
@@ -234,8 +235,9 @@ enum { ZERO_DTYPE_BF16 = 0, ZERO_DTYPE_F16 = 1 };
  *             storer thread that copies the results to master/m/v and the N
  *             destinations with bulk copies (shared -> global), so that no
  *             consumer lane issues a global store.  Bounded waits as TMA.
- *   AUTO:     the staged kernel for every N, in the configuration measured
- *             fastest on B200 for that N (zero_fused_config reports it). */
+ *   AUTO:     the bulk-store staged kernel (BULK) for every N, in the
+ *             configuration measured fastest on B200 for that N and stage
+ *             (zero_fused_config and zero_fused_tile report it). */
 enum { ZERO_KERNEL_AUTO = 0, ZERO_KERNEL_REGISTER = 1, ZERO_KERNEL_TMA = 2, ZERO_KERNEL_BULK = 3 };
 
 /* Views (zero_view). */

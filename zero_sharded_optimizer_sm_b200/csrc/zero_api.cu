@@ -53,7 +53,7 @@ struct zero_ctx {
   int tma_tile_opt = 0;    // bulk-store kernel: elements per tile, 0 = the library's choice
   int tma_warps_opt = 0;   // bulk-store kernel: consumer warps, 0 = the library's choice
   unsigned long long wait_ns = 2000000000ull;  // limit of the staged kernels' ring waits (ZERO_OPT_WAIT_LIMIT_NS)
-  int store_hint = 0;      // bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)
+  int store_hint = 1;      // bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)
   int tma_grid_key = -1;   // configuration the cached grid cap belongs to
   int tma_grid_cap = 0;
   // arena layout (bytes)
@@ -381,22 +381,66 @@ bool use_tma(const zero_ctx* c) {
 
 int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages_opt : 3; }  // measured best at N = 32, 64
 
+// The bulk-store staged kernel's configuration (tile, consumer warps, ring
+// depth -- above 16 ranks the chunk ring's) chosen for N and the stage,
+// measured on B200: flat 256M-element buffers at N = 1, 2, 4, 8, 16, flat
+// 64M at N = 17, 32, 64, and the 1.2B-parameter transformer list at N = 8,
+// every stage, two or three interleaved repetitions per cell, with the L2
+// evict-first hint on the stores.  Few ranks leave each tile short and the
+// arithmetic dominant: 2048-element tiles with sixteen warps.  From N = 5 the
+// copies dominate: eight warps, 1024-element tiles, with the ring as deep as
+// measured best (three stages at ZeRO-1, which also stages the averaged
+// gradient, four otherwise; at N = 9..16, where a stage is twice as large,
+// three).  Above 16 ranks the rank-chunked form; at N = 17..31 (a chunk ring
+// of three 2048-element stages) the last chunk is short.  tile = 0: the TMA
+// kernel measured faster there (N = 2 at ZeRO-3, by 4 %).
+struct BulkChoice {
+  int tile, warps, stages;
+};
+
+BulkChoice bulk_policy(int n_ranks, int stage) {
+  const bool z1 = stage == ZERO_STAGE_1;
+  if (n_ranks <= 1) return {2048, 16, 3};
+  if (n_ranks == 2) return stage == ZERO_STAGE_3 ? BulkChoice{0, 0, 0} : BulkChoice{2048, 16, 3};
+  if (n_ranks <= 4) return z1 ? BulkChoice{2048, 16, 2} : BulkChoice{2048, 16, 3};
+  if (n_ranks <= 8) return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{1024, 8, 4};
+  if (n_ranks <= 16) return z1 ? BulkChoice{2048, 8, 2} : BulkChoice{1024, 8, 3};
+  if (n_ranks < 32) return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{2048, 8, 3};
+  return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{1024, 8, 4};
+}
+
 // The bulk-store staged kernel (fused_bulk.cu): its tile, consumer warps and
-// ring depth for this context.
-int bulk_tile(const zero_ctx* c) { return c->tma_tile_opt ? c->tma_tile_opt : 1024; }
-int bulk_warps(const zero_ctx* c) { return c->tma_warps_opt ? c->tma_warps_opt : 8; }
+// ring depth for this context (the options where set, else the policy).
+int bulk_tile(const zero_ctx* c) {
+  if (c->tma_tile_opt) return c->tma_tile_opt;
+  const int t = bulk_policy(c->plan.n_ranks, c->stage).tile;
+  return t ? t : 2048;  // BULK asked for where the policy prefers TMA
+}
+int bulk_warps(const zero_ctx* c) {
+  if (c->tma_warps_opt) return c->tma_warps_opt;
+  const int w = bulk_policy(c->plan.n_ranks, c->stage).warps;
+  return w ? w : 16;
+}
 bool bulk_need_g(const zero_ctx* c) {
   return c->stage == ZERO_STAGE_1 || c->arena[ZERO_ARENA_GRAD_SHARDS] != nullptr;
 }
+int bulk_ring(const zero_ctx* c) {
+  if (c->tma_stages_opt) return c->tma_stages_opt;
+  const int st = bulk_policy(c->plan.n_ranks, c->stage).stages;
+  return st ? st : 3;
+}
 int bulk_stages(const zero_ctx* c) {
-  return zsm::bulk_stages_for(c->plan.n_ranks, bulk_tile(c), bulk_need_g(c), c->tma_stages_opt);
+  return zsm::bulk_stages_for(c->plan.n_ranks, bulk_tile(c), bulk_need_g(c), bulk_ring(c));
 }
 bool bulk_fits(const zero_ctx* c) {
   return zsm::bulk_config_valid(c->plan.n_ranks, bulk_tile(c), bulk_warps(c)) && bulk_stages(c) > 0;
 }
-// Asked for (any N; the rank-chunked form above 16); a (tile, warps) pair
-// that is not built fails at launch.
-bool use_bulk(const zero_ctx* c) { return c->kernel_opt == ZERO_KERNEL_BULK; }
+// Asked for, or AUTO where the policy picks it (any N; the rank-chunked form
+// above 16); a (tile, warps) pair that is not built fails at launch.
+bool use_bulk(const zero_ctx* c) {
+  if (c->kernel_opt == ZERO_KERNEL_BULK) return true;
+  return c->kernel_opt == ZERO_KERNEL_AUTO && bulk_policy(c->plan.n_ranks, c->stage).tile != 0;
+}
 
 // Bytes one element moves through HBM in the fused step (the byte model).
 int64_t fused_bytes_per_elem(const zero_ctx* c) {
@@ -498,7 +542,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   if (twin || use_bulk(c)) {
     const int64_t tiles = (hi - lo + bulk_tile(c) - 1) / bulk_tile(c);
     e = counted(c, zsm::launch_fused_bulk(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
-                                          bulk_tile(c), bulk_warps(c), c->tma_stages_opt, twin, 0u, s));
+                                          bulk_tile(c), bulk_warps(c), bulk_ring(c), twin, 0u, s));
   } else if (use_chunked(c)) {
     const int64_t tiles = (hi - lo + kTmaTile - 1) / kTmaTile;
     e = counted(c, zsm::launch_fused_chunked(mode, a, (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count)),
