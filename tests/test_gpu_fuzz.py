@@ -56,7 +56,11 @@ def _case(k):
     # drawn last, so that the fields above stay those of the seed
     if rng.random() < 0.4:
         c["kernel"] = 3  # the bulk-store staged kernel, in one of its built configurations
-        c["tile"], c["warps"] = [(2048, 8), (2048, 16), (1024, 4), (1024, 8), (1024, 16)][int(rng.integers(0, 5))]
+        pick = int(rng.integers(0, 5))
+        if n_ranks <= 16:
+            c["tile"], c["warps"] = [(2048, 8), (2048, 16), (1024, 4), (1024, 8), (1024, 16)][pick]
+        else:  # the rank-chunked form's configurations
+            c["tile"], c["warps"] = [(2048, 8), (1024, 8)][pick % 2]
     return c
 
 
