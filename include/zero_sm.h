@@ -178,10 +178,11 @@ enum {
                                     1024 x 8 and 1024 x 16 for N <= 16, 2048 x 8 and 1024 x 8
                                     above; another pair makes the next fused launch fail with
                                     ZERO_ECUDA; may be set at any time */
-  ZERO_OPT_STORE_HINT = 16,      /* bulk-store kernel: 1 (default) marks its bulk stores L2
-                                    evict-first (written lines leave L2 first; measured 0.5-4 %
-                                    faster on B200), 0 plain; values are unchanged either way;
-                                    may be set at any time */
+  ZERO_OPT_STORE_HINT = 16,      /* bulk-store kernel: 1 marks its bulk stores L2 evict-first
+                                    (written lines leave L2 first), 0 plain, -1 (default) the
+                                    library's measured choice for N and the stage (on at stages
+                                    2 and 3, where it gained up to 4 % on B200); values are
+                                    unchanged either way; may be set at any time */
   ZERO_OPT_WAIT_LIMIT_NS = 15,   /* limit, in ns of wall time, of each wait of the staged
                                     kernels on their shared-memory ring (default 2e9, at most
                                     60e9).  0 makes every ring wait one non-blocking test: a

@@ -525,9 +525,11 @@ class ZeroOptimizer:
     def set_kernel(self, kernel: int):
         self._check(zero_set_option(self.ctx, ZERO_OPT_KERNEL, int(kernel)), "zero_set_option")
 
-    def set_store_hint(self, on: bool):
-        """Bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)."""
-        self._check(zero_set_option(self.ctx, ZERO_OPT_STORE_HINT, 1 if on else 0), "zero_set_option")
+    def set_store_hint(self, on):
+        """Bulk-store kernel: L2 evict-first hint on its stores (True / False;
+        None = the library's choice; ZERO_OPT_STORE_HINT)."""
+        v = -1 if on is None else (1 if on else 0)
+        self._check(zero_set_option(self.ctx, ZERO_OPT_STORE_HINT, v), "zero_set_option")
 
     def set_wait_limit(self, ns: int):
         """Limit of the staged kernels' ring waits in ns (0: one non-blocking test; see ZERO_OPT_WAIT_LIMIT_NS)."""

@@ -53,7 +53,7 @@ struct zero_ctx {
   int tma_tile_opt = 0;    // bulk-store kernel: elements per tile, 0 = the library's choice
   int tma_warps_opt = 0;   // bulk-store kernel: consumer warps, 0 = the library's choice
   unsigned long long wait_ns = 2000000000ull;  // limit of the staged kernels' ring waits (ZERO_OPT_WAIT_LIMIT_NS)
-  int store_hint = 1;      // bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT)
+  int store_hint = -1;     // bulk-store kernel: L2 evict-first hint on its stores (ZERO_OPT_STORE_HINT, -1 = policy)
   int tma_grid_key = -1;   // configuration the cached grid cap belongs to
   int tma_grid_cap = 0;
   // arena layout (bytes)
@@ -393,20 +393,23 @@ int chunked_stages(const zero_ctx* c) { return c->tma_stages_opt ? c->tma_stages
 // gradient, four otherwise; at N = 9..16, where a stage is twice as large,
 // three).  Above 16 ranks the rank-chunked form; at N = 17..31 (a chunk ring
 // of three 2048-element stages) the last chunk is short.  tile = 0: the TMA
-// kernel measured faster there (N = 2 at ZeRO-3, by 4 %).
+// kernel measured faster there (N = 2 at ZeRO-3, by 4 %).  The stores' L2
+// evict-first hint gained up to 4 % at stages 2 and 3 everywhere and is on
+// there; at stage 1 it lost about 1 % at N = 5..8 and from N = 32 on (where
+// it is off) and gained about as much at N = 3..4 and 9..31.
 struct BulkChoice {
-  int tile, warps, stages;
+  int tile, warps, stages, hint;
 };
 
 BulkChoice bulk_policy(int n_ranks, int stage) {
   const bool z1 = stage == ZERO_STAGE_1;
-  if (n_ranks <= 1) return {2048, 16, 3};
-  if (n_ranks == 2) return stage == ZERO_STAGE_3 ? BulkChoice{0, 0, 0} : BulkChoice{2048, 16, 3};
-  if (n_ranks <= 4) return z1 ? BulkChoice{2048, 16, 2} : BulkChoice{2048, 16, 3};
-  if (n_ranks <= 8) return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{1024, 8, 4};
-  if (n_ranks <= 16) return z1 ? BulkChoice{2048, 8, 2} : BulkChoice{1024, 8, 3};
-  if (n_ranks < 32) return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{2048, 8, 3};
-  return z1 ? BulkChoice{1024, 8, 3} : BulkChoice{1024, 8, 4};
+  if (n_ranks <= 1) return {2048, 16, 3, 1};
+  if (n_ranks == 2) return stage == ZERO_STAGE_3 ? BulkChoice{0, 0, 0, 1} : BulkChoice{2048, 16, 3, 1};
+  if (n_ranks <= 4) return z1 ? BulkChoice{2048, 16, 2, 1} : BulkChoice{2048, 16, 3, 1};
+  if (n_ranks <= 8) return z1 ? BulkChoice{1024, 8, 3, 0} : BulkChoice{1024, 8, 4, 1};
+  if (n_ranks <= 16) return z1 ? BulkChoice{2048, 8, 2, 1} : BulkChoice{1024, 8, 3, 1};
+  if (n_ranks < 32) return z1 ? BulkChoice{1024, 8, 3, 1} : BulkChoice{2048, 8, 3, 1};
+  return z1 ? BulkChoice{1024, 8, 3, 0} : BulkChoice{1024, 8, 4, 1};
 }
 
 // The bulk-store staged kernel (fused_bulk.cu): its tile, consumer warps and
@@ -534,7 +537,7 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   a.sc_dev = sc_dev;
   a.ns = norm_scratch(c);
   a.pdl = c->timing ? zsm::kPdlNone : pdl;  // an event record between launches ends the overlap
-  a.store_hint = c->store_hint;
+  a.store_hint = c->store_hint >= 0 ? c->store_hint : bulk_policy(c->plan.n_ranks, c->stage).hint;
   const int mode = c->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : c->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
@@ -1024,7 +1027,7 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     return ZERO_OK;
   }
   if (key == ZERO_OPT_STORE_HINT) {
-    if (value != 0 && value != 1) return fail(c, ZERO_EINVAL, "store hint must be 0 or 1");
+    if (value < -1 || value > 1) return fail(c, ZERO_EINVAL, "store hint must be -1 (the library's choice), 0 or 1");
     c->store_hint = (int)value;
     return ZERO_OK;
   }
