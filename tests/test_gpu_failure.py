@@ -7,7 +7,8 @@ synchronising call returns ZERO_ECUDA and clears the word; the context stays
 usable, and after the state is restored (zero_import_state) the next step
 equals the oracle bit for bit.  Each staged family: one and two producer /
 consumer groups, the sixteen-warp group, the rank-chunked kernel (N > 16),
-the bulk-store kernel, and the two passes of a clipped step."""
+the bulk-store kernel, and the two passes of a clipped step (the second pass
+with per-lane stores and with bulk stores)."""
 import gc
 
 import numpy as np
@@ -32,6 +33,7 @@ FAMILIES = {
     "rank-chunked": (17, dict(kernel=TMA), False),
     "bulk-store": (8, dict(kernel=BULK), False),
     "two-pass": (8, dict(kernel=TMA), True),
+    "two-pass-bulk-store": (8, dict(kernel=BULK), True),
 }
 
 

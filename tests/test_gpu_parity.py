@@ -792,27 +792,29 @@ def test_two_pass_staged_kernels_equal_register_kernels(stage):
                                synth.Dist(synth.NORMAL, 1e-2, zero_mod=7), W.MASTER_DIST, 3, W.Hyper(weight_decay=0.01),
                                0x500 + n_ranks)
                 opts = []
-                for kernel in (TMA, REG):
+                for kernel in (TMA, REG, BULK):  # BULK: pass 2 with bulk stores
                     o, f = make_opt(w, stage, bucket=16384, kernel=kernel, dtype=dtype)
                     o.set_clip(0.01, True)
                     opts.append((o, f))
                 for t in range(1, 4):
                     sts = [o.step(grad_fn_for(o, f), stats=True) for o, f in opts]
                     assert sts[0]["clip_coef"] < 1.0
-                    assert sts[0]["nonfinite"] == sts[1]["nonfinite"]
-                    assert math.isclose(sts[0]["grad_norm"], sts[1]["grad_norm"], rel_tol=1e-12)
-                (a, _), (b, _) = opts
-                for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
-                    assert torch.equal(a.view(what), b.view(what)), (numel, n_ranks, stage, what)
-                for r in range(n_ranks if stage != 3 else 1):
-                    assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+                    for other in sts[1:]:
+                        assert sts[0]["nonfinite"] == other["nonfinite"]
+                        assert math.isclose(sts[0]["grad_norm"], other["grad_norm"], rel_tol=1e-12)
+                (b, _) = opts[1]
+                for a, _ in (opts[0], opts[2]):
+                    for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
+                        assert torch.equal(a.view(what), b.view(what)), (numel, n_ranks, stage, what)
+                    for r in range(n_ranks if stage != 3 else 1):
+                        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
                 if stage == 1:
                     for r in range(n_ranks):
                         assert torch.equal(a.view(z.ZERO_VIEW_GRAD_BUF, r), b.view(z.ZERO_VIEW_GRAD_BUF, r))
                 else:
                     assert torch.equal(a.view(z.ZERO_VIEW_GRAD_SHARD), b.view(z.ZERO_VIEW_GRAD_SHARD))
-                a.close()
-                b.close()
+                for o, _ in opts:
+                    o.close()
 
 
 @pytest.mark.parametrize("stage", [1, 2, 3])

@@ -267,5 +267,11 @@ cudaError_t two_pass_configure();
 cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam_bcast_tma(const AdamBcastArgs& a, int grid, bool uniform, cudaStream_t s);
 int64_t two_pass_tile();
+// Pass 2 with bulk stores (two_pass_tma.cu): 1024-element tiles, eight
+// consumer warps, a ring of `stages` (2..8, fitted to shared memory); the
+// stores carry the L2 evict-first hint when `store_hint`.
+cudaError_t launch_adam_bcast_bulk(const AdamBcastArgs& a, int grid, bool uniform, int stages, int store_hint,
+                                   cudaStream_t s);
+int64_t bulk_bcast_tile();
 
 }  // namespace zsm

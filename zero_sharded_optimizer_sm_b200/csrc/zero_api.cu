@@ -770,9 +770,17 @@ cudaError_t launch_pass2(zero_ctx* c, const zsm::AdamBcastArgs& b, bool uniform,
   const int64_t elems = b.n_vec * zsm::kVec;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  const cudaError_t e = counted(c, use_two_pass_tma(c)
-                                       ? zsm::launch_adam_bcast_tma(b, two_pass_grid(c, elems), uniform, s)
+  cudaError_t e;
+  if (use_bulk(c)) {
+    // the bulk-store pass 2: four 1024-element stages unless the ring depth is set
+    const int64_t tiles = (elems + zsm::bulk_bcast_tile() - 1) / zsm::bulk_bcast_tile();
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count));
+    e = counted(c, zsm::launch_adam_bcast_bulk(b, grid, uniform, c->tma_stages_opt ? c->tma_stages_opt : 4,
+                                               c->store_hint >= 0 ? c->store_hint : 1, s));
+  } else {
+    e = counted(c, use_two_pass_tma(c) ? zsm::launch_adam_bcast_tma(b, two_pass_grid(c, elems), uniform, s)
                                        : zsm::launch_adam_bcast(b, grid_for(b.n_vec, c->grid_simple), s));
+  }
   if (e == cudaSuccess && ev) {
     cudaEventRecord(ev[1], s);
     c->timed += 1;
