@@ -726,11 +726,16 @@ void zero_destroy(zero_ctx* ctx);
  * what it is sensitive to, and [M] section 6).  Rank r keeps, in its own
  * GPU's memory and in arenas the caller allocates:
  *   GRAD    its 16-bit gradient replica, psi_pad elements (its backward's
- *           output; stage 1 also receives the all-reduced gradient here)
- *   PARAM   its 16-bit parameter replica, psi_pad elements
+ *           output; stage 1 also receives the all-reduced gradient here);
+ *           at stage 3 one layer's gradient, the largest layer's length
+ *   PARAM   its 16-bit parameter replica, psi_pad elements; at stage 3 its
+ *           parameter shard, S elements
  *   STATES  fp32 master, m and v of its owned shard [rS, (r+1)S)
  *   SCRATCH the step's norm partials and counters
- * Every rank exports its GRAD and PARAM arenas as CUDA IPC records
+ *   GATHER  stage 3 only: the temporary gathered layer, the largest layer's
+ *           length ([T] section "ZeRO-3": each layer's parameters are
+ *           gathered into a temporary full buffer for its use)
+ * Every rank exports its GRAD, PARAM and GATHER arenas as CUDA IPC records
  * (zero_dist_export), the caller exchanges the records (for instance with
  * torch.distributed all_gather_object) and every rank opens the others'
  * (zero_dist_open_peers).  zero_dist_step then launches, on this GPU, one
@@ -741,7 +746,12 @@ void zero_destroy(zero_ctx* ctx);
  * stores bf16(master) into the shard's range of every rank's PARAM replica
  * (stage 1: also the averaged gradient into every rank's GRAD replica): the
  * reduce-scatter, the update and the all-gather in one pass, the same bits
- * as the single-device step and the oracle.  No bulk copy or multicast reads
+ * as the single-device step and the oracle.  At stage 3 the step goes layer
+ * by layer (zero_dist_step_layer): every rank's GRAD buffer holds that
+ * layer's gradient, the kernel covers the layer's part of the owned shard,
+ * writes the rank's own PARAM shard and stores the result into that part of
+ * every rank's GATHER buffer, so that once every rank has run the layer each
+ * GATHER buffer holds the whole layer.  No bulk copy or multicast reads
  * another GPU's memory.
  *
  * Ordering between the ranks is the caller's, on the host: every rank's GRAD
@@ -749,11 +759,13 @@ void zero_destroy(zero_ctx* ctx);
  * instance: synchronise the stream of the backward, then a barrier), and no
  * rank reads its PARAM replica or writes its GRAD replica again before every
  * rank's step has completed (synchronise the step's stream, then a barrier).
- * zero_dist_load_master has the same contract as a step.  No kernel of this
- * API waits on another rank.
+ * zero_dist_load_master has the same contract as a step, and so does each
+ * layer of a stage-3 step (its GRAD buffers filled before, its GATHER buffers
+ * used and GRAD refilled only after every rank has run it).  No kernel of
+ * this API waits on another rank.
  *
  * Errors as for the single-device context: status codes, the text in
- * zero_dist_last_error.  Stages 1 and 2; stage 3 returns ZERO_ENOTIMPL.
+ * zero_dist_last_error.  Stages 1, 2 and 3; DP returns ZERO_ENOTIMPL.
  */
 typedef struct zero_dist zero_dist;
 
@@ -762,16 +774,18 @@ enum {
   ZERO_DIST_ARENA_PARAM = 1,
   ZERO_DIST_ARENA_STATES = 2,
   ZERO_DIST_ARENA_SCRATCH = 3,
-  ZERO_DIST_NUM_ARENAS = 4
+  ZERO_DIST_ARENA_GATHER = 4,  /* stage 3 only (0 bytes otherwise) */
+  ZERO_DIST_NUM_ARENAS = 5
 };
 
-/* Bytes of one rank's export record (two CUDA IPC handles with the arenas'
- * offsets in their allocations and their lengths; zero padded). */
-#define ZERO_DIST_HANDLE_BYTES 192
+/* Bytes of one rank's export record (three CUDA IPC handles -- GRAD, PARAM,
+ * GATHER -- with the arenas' offsets in their allocations and their lengths;
+ * an empty arena's entry is zero; zero padded). */
+#define ZERO_DIST_HANDLE_BYTES 256
 
-/* Plan rank `rank` of `world` ranks (1..ZERO_MAX_RANKS) at `stage` (1 or 2):
- * the same partition as zero_init (S = psi_pad / world).  Host only.
- * ZERO_EINVAL for bad arguments, ZERO_ENOTIMPL for stage 3 or DP. */
+/* Plan rank `rank` of `world` ranks (1..ZERO_MAX_RANKS) at `stage` (1, 2 or
+ * 3): the same partition and layers as zero_init (S = psi_pad / world).
+ * Host only.  ZERO_EINVAL for bad arguments, ZERO_ENOTIMPL for DP. */
 zero_status zero_dist_init(const zero_layout* layout, int32_t world, int32_t rank, int32_t stage,
                            zero_dist** out);
 
@@ -783,7 +797,8 @@ zero_status zero_dist_sizes(const zero_dist* d, int64_t plan[3], int64_t arena_b
 zero_status zero_dist_tensor_offsets(const zero_dist* d, int64_t* out, int32_t cap);
 
 /* Bind this rank's arenas: device pointers on the current device, 256-byte
- * aligned, caller-owned, at least zero_dist_sizes bytes each.  GRAD and PARAM
+ * aligned, caller-owned, at least zero_dist_sizes bytes each (an arena of 0
+ * bytes may be NULL).  GRAD and PARAM
  * must come from device allocations that CUDA IPC can export (cudaMalloc and
  * allocators built on it; not virtual-memory-managed pools).  Zeroes SCRATCH
  * (synchronously).  With world = 1 no peer needs opening. */
@@ -809,7 +824,8 @@ zero_status zero_dist_set_hparams(zero_dist* d, const zero_adam_hparams* hp);
  * psi_pad fp32 values on this GPU (pads 0); the rank copies its shard into
  * STATES, sets m = v = 0 and the step counter to 0, and writes bf16(master)
  * of its shard into every rank's PARAM replica (so that, once every rank has
- * loaded, every replica holds all of them).  Enqueued on `stream`. */
+ * loaded, every replica holds all of them); at stage 3 into its own PARAM
+ * shard.  Enqueued on `stream`. */
 zero_status zero_dist_load_master(zero_dist* d, const float* master_full, void* stream);
 
 /* One fused step (t = completed steps + 1) over this rank's shard, enqueued
@@ -818,6 +834,19 @@ zero_status zero_dist_load_master(zero_dist* d, const float* master_full, void* 
  * averaged gradient) for zero_dist_read_partial.  The global norm is the
  * square root of the ranks' sums, added in rank order. */
 zero_status zero_dist_step(zero_dist* d, void* stream);
+
+/* One layer of a stage-3 step (t = completed steps + 1), enqueued on
+ * `stream`: `layer` in layer order (zero_layers of a context with the same
+ * layout lists them); every rank's GRAD buffer holds that layer's gradient
+ * from element 0.  The rank updates the layer's part of its shard (none when
+ * it owns no part of the layer) and stores the result into its PARAM shard
+ * and into every rank's GATHER buffer at the part's offset in the layer.
+ * The call with `last` != 0 completes the step: the step counter advances
+ * and zero_dist_read_partial then gives the step's partial sums (all layers
+ * of the step added).  Layers may come in any order ([T] section "ZeRO-3"
+ * walks them from the last).  ZERO_ESTATE at stages 1 and 2, ZERO_EINVAL for
+ * a layer out of range. */
+zero_status zero_dist_step_layer(zero_dist* d, int32_t layer, int32_t last, void* stream);
 
 /* Adam on this rank's shard from an already reduced 16-bit gradient shard
  * (grad_shard: S values on this GPU, 16-byte aligned) -- for a caller whose
@@ -840,8 +869,9 @@ zero_status zero_dist_combine_partials(int32_t world, const double* sumsq, const
                                        int64_t* nonfinite_total);
 
 /* Local device pointer and length of ZERO_VIEW_MASTER / _EXP_AVG /
- * _EXP_AVG_SQ (the owned shard, S) or ZERO_VIEW_PARAM / ZERO_VIEW_GRAD_BUF
- * (this rank's replicas, psi_pad). */
+ * _EXP_AVG_SQ (the owned shard, S), ZERO_VIEW_PARAM / ZERO_VIEW_GRAD_BUF
+ * (this rank's replicas, psi_pad; at stage 3 the parameter shard, S, and the
+ * layer gradient buffer) or ZERO_VIEW_GATHER (stage 3: the gathered layer). */
 zero_status zero_dist_view(const zero_dist* d, int32_t what, void** ptr, int64_t* n_elems);
 
 /* Message of the last failure (d == NULL: of the calling thread's last

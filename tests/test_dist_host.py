@@ -115,8 +115,19 @@ def test_dist_argument_checks_need_no_device():
     ctx = ctypes.c_void_p()
     assert z.zero_dist_init(ctypes.byref(lay), 0, 0, 2, ctypes.byref(ctx)) == z.ZERO_EINVAL
     assert z.zero_dist_init(ctypes.byref(lay), 4, 4, 2, ctypes.byref(ctx)) == z.ZERO_EINVAL
-    assert z.zero_dist_init(ctypes.byref(lay), 4, 1, 3, ctypes.byref(ctx)) == z.ZERO_ENOTIMPL
-    assert b"stages 1 and 2" in z.zero_dist_last_error(None)
+    assert z.zero_dist_init(ctypes.byref(lay), 4, 1, 0, ctypes.byref(ctx)) == z.ZERO_ENOTIMPL  # plain DP
+    assert b"oracle" in z.zero_dist_last_error(None)
+    assert z.zero_dist_init(ctypes.byref(lay), 4, 1, 5, ctypes.byref(ctx)) == z.ZERO_EINVAL
+    # stage 3: one layer's gradient, the parameter shard, one gathered layer
+    assert z.zero_dist_init(ctypes.byref(lay), 4, 1, 3, ctypes.byref(ctx)) == z.ZERO_OK
+    try:
+        ab = (ctypes.c_int64 * z.ZERO_DIST_NUM_ARENAS)()
+        assert z.zero_dist_sizes(ctx, None, ab) == z.ZERO_OK
+        assert ab[z.ZERO_DIST_ARENA_GRAD] >= 2 * 104 and ab[z.ZERO_DIST_ARENA_GATHER] >= 2 * 104  # largest layer
+        assert 2 * 40 <= ab[z.ZERO_DIST_ARENA_PARAM] < 2 * 160                                     # the shard
+        assert z.zero_dist_step_layer(ctx, 0, 1, None) == z.ZERO_ESTATE  # not bound
+    finally:
+        z.zero_dist_destroy(ctx)
     assert z.zero_dist_init(None, 4, 1, 2, ctypes.byref(ctx)) == z.ZERO_EINVAL
     assert z.zero_dist_init(ctypes.byref(lay), 4, 1, 2, ctypes.byref(ctx)) == z.ZERO_OK
     try:
@@ -127,6 +138,7 @@ def test_dist_argument_checks_need_no_device():
         assert tuple(plan) == (128, 160, 40)
         assert ab[z.ZERO_DIST_ARENA_GRAD] >= 2 * 160 and ab[z.ZERO_DIST_ARENA_PARAM] >= 2 * 160
         assert ab[z.ZERO_DIST_ARENA_STATES] >= 12 * 40
+        assert ab[z.ZERO_DIST_ARENA_GATHER] == 0  # stage 3 only
         offs = (ctypes.c_int64 * 2)()
         assert z.zero_dist_tensor_offsets(ctx, offs, 2) == z.ZERO_OK and list(offs) == [0, 104]
         # calls out of order fail cleanly before any device work

@@ -24,7 +24,7 @@ from synth import workloads as W  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
-STAGE_OF = {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2}
+STAGE_OF = {1: oracle.STAGE_Z1, 2: oracle.STAGE_Z2, 3: oracle.STAGE_Z3}
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -76,6 +76,42 @@ def _rank_main(rank, world, port, stage, outdir, nccl_style):
     opt.load_master(master)
     grads = opt.view(z.ZERO_VIEW_GRAD_BUF)
     stats = []
+    gathered = []
+    if stage == 3:
+        # layer by layer from the last: this rank's gradient of the layer, then
+        # the layer's step on every rank; the gathered layer is kept on the last step
+        import oracle as o
+
+        p = o.plan(w.numel, w.layer_id, world, 1 << 40)
+        for step in range(1, w.steps + 1):
+            order = list(reversed(range(len(p.layers))))
+            for k, li in enumerate(order):
+                _, l_lo, l_hi = p.layers[li]
+                grads.zero_()
+                for off, n in zip(offs, w.numel):
+                    if l_lo <= off < l_hi and n:
+                        sy.dev_bf16(WW.grad_base(w, step, rank), off, n, w.grad_dist,
+                                    grads.data_ptr() + 2 * (off - l_lo), s)
+                st = opt.step_layer(li, k == len(order) - 1, stats=True)
+                if step == w.steps:
+                    g = opt.view(z.ZERO_VIEW_GATHER)[: l_hi - l_lo].cpu().numpy().view(np.uint16).copy()
+                    gathered.append((li, g))
+                if st is not None:
+                    stats.append(st)
+        t.cuda.synchronize()
+        np.savez(os.path.join(outdir, f"rank{rank}.npz"),
+                 master=opt.view(z.ZERO_VIEW_MASTER).cpu().numpy(), m=opt.view(z.ZERO_VIEW_EXP_AVG).cpu().numpy(),
+                 v=opt.view(z.ZERO_VIEW_EXP_AVG_SQ).cpu().numpy(),
+                 params=opt.view(z.ZERO_VIEW_PARAM).cpu().numpy().view(np.uint16),
+                 grads=np.zeros(1, np.uint16),
+                 gathered_ids=np.array([li for li, _ in gathered], dtype=np.int64),
+                 **{f"gathered{li}": g for li, g in gathered},
+                 norms=np.array([x["grad_norm"] for x in stats], dtype=np.float64),
+                 nfs=np.array([x["nonfinite"] for x in stats], dtype=np.int64),
+                 steps=np.array([x["step"] for x in stats], dtype=np.int64))
+        opt.close()
+        dist.destroy_process_group()
+        return
     for step in range(1, w.steps + 1):
         grads.zero_()
         for off, n in zip(offs, w.numel):
@@ -145,7 +181,15 @@ def _compare(got, w, stage, p, ranks, reps, ref, with_stats=True):
         lo, hi = r * S, (r + 1) * S
         for k in ("master", "m", "v"):
             assert np.array_equal(d[k].view(np.uint32), ref[k][lo:hi].view(np.uint32)), (r, k)
-        assert np.array_equal(d["params"], ref["params"]), f"rank {r} parameter replica"
+        if stage == 3:
+            assert np.array_equal(d["params"], ref["params"][lo:hi]), f"rank {r} parameter shard"
+            # every layer of the last step, gathered on every rank: the oracle's temporary buffers
+            want = {lid: tmp for (lid, _, _), tmp in zip(reversed(p.layers), reps[-1].gathered)}
+            for li in d["gathered_ids"]:
+                lid = p.layers[int(li)][0]
+                assert np.array_equal(d[f"gathered{int(li)}"], want[lid][r]), f"rank {r} gathered layer {lid}"
+        else:
+            assert np.array_equal(d["params"], ref["params"]), f"rank {r} parameter replica"
         if stage == 1:
             assert np.array_equal(d["grads"], ranks[r].grads), f"rank {r} all-reduced gradient"
         if with_stats:
@@ -160,7 +204,7 @@ def _compare(got, w, stage, p, ranks, reps, ref, with_stats=True):
 
 
 @pytest.mark.parametrize("world", [2, 3])
-@pytest.mark.parametrize("stage", [1, 2])
+@pytest.mark.parametrize("stage", [1, 2, 3])
 def test_ranks_as_processes_against_the_oracle(world, stage, tmp_path):
     w = _workload(world, stage)
     p, ranks, reps, ref = _oracle(w, stage)

@@ -130,6 +130,7 @@ _SIGS = {
     "zero_dist_set_hparams": (_i32, [_vp, ctypes.POINTER(zero_adam_hparams)]),
     "zero_dist_load_master": (_i32, [_vp, _vp, _vp]),
     "zero_dist_step": (_i32, [_vp, _vp]),
+    "zero_dist_step_layer": (_i32, [_vp, _i32, _i32, _vp]),
     "zero_dist_adam_shard": (_i32, [_vp, _vp, _vp]),
     "zero_dist_read_partial": (_i32, [_vp, _vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64),
                                       ctypes.POINTER(_i64)]),
@@ -150,8 +151,9 @@ for _name, (_res, _args) in _SIGS.items():
 __all__ = list(_SIGS) + ["ZeroOptimizer", "ZeroDist", "AdamHParams", "ZeroError", "lib", "LIB_PATH",
                          "options_from_config", "exchange_records", "rank_ordered_norm", "ordered_step"]
 ZERO_DIST_ARENA_GRAD, ZERO_DIST_ARENA_PARAM, ZERO_DIST_ARENA_STATES, ZERO_DIST_ARENA_SCRATCH = 0, 1, 2, 3
-ZERO_DIST_NUM_ARENAS = 4
-ZERO_DIST_HANDLE_BYTES = 192
+ZERO_DIST_ARENA_GATHER = 4
+ZERO_DIST_NUM_ARENAS = 5
+ZERO_DIST_HANDLE_BYTES = 256
 
 
 class ZeroError(RuntimeError):
@@ -631,7 +633,7 @@ def ordered_step(dist, sync: Callable[[], None], launch: Callable[[], None], gro
 
 class ZeroDist:
     """Rank ``dist.get_rank(group)`` of a ZeRO step with one logical rank per
-    GPU (stage 1 or 2): allocates this rank's arenas with torch on ``device``,
+    GPU (stage 1, 2 or 3): allocates this rank's arenas with torch on ``device``,
     binds them, exchanges IPC records with the other ranks and opens theirs.
     Every call below is collective (every rank calls it, in the same order)."""
 
@@ -656,9 +658,10 @@ class ZeroDist:
         ab = (ctypes.c_int64 * ZERO_DIST_NUM_ARENAS)()
         self._check(zero_dist_sizes(ctx, plan, ab), "zero_dist_sizes")
         self.psi, self.psi_pad, self.shard = int(plan[0]), int(plan[1]), int(plan[2])
-        self.arenas = [torch.empty(int(ab[k]), dtype=torch.uint8, device=self.device)
+        self.arenas = [torch.empty(int(ab[k]), dtype=torch.uint8, device=self.device) if int(ab[k]) else None
                        for k in range(ZERO_DIST_NUM_ARENAS)]
-        ptrs = (ctypes.c_void_p * ZERO_DIST_NUM_ARENAS)(*[a.data_ptr() for a in self.arenas])
+        ptrs = (ctypes.c_void_p * ZERO_DIST_NUM_ARENAS)(*[a.data_ptr() if a is not None else None
+                                                          for a in self.arenas])
         with torch.cuda.device(self.device):
             self._check(zero_dist_bind(ctx, ptrs), "zero_dist_bind")
             if self.world > 1:
@@ -695,7 +698,8 @@ class ZeroDist:
             else self._torch.int16
         item = 4 if dt == self._torch.float32 else 2
         arena = self.arenas[ZERO_DIST_ARENA_STATES if item == 4 else
-                            (ZERO_DIST_ARENA_PARAM if what == ZERO_VIEW_PARAM else ZERO_DIST_ARENA_GRAD)]
+                            ZERO_DIST_ARENA_PARAM if what == ZERO_VIEW_PARAM else
+                            ZERO_DIST_ARENA_GATHER if what == ZERO_VIEW_GATHER else ZERO_DIST_ARENA_GRAD]
         off = (ptr.value - arena.data_ptr())
         return arena[off: off + item * n.value].view(dt)
 
@@ -711,6 +715,20 @@ class ZeroDist:
         ordered_step(self._dist, self._sync,
                      lambda: self._check(zero_dist_step(self.ctx, self._stream()), "zero_dist_step"), self.group)
         if not stats:
+            return None
+        sq, nf, t = ctypes.c_double(), ctypes.c_int64(), ctypes.c_int64()
+        self._check(zero_dist_read_partial(self.ctx, self._stream(), ctypes.byref(sq), ctypes.byref(nf),
+                                           ctypes.byref(t)), "zero_dist_read_partial")
+        norm, nft = rank_ordered_norm(self._dist, sq.value, nf.value, self.group)
+        return {"grad_norm": norm, "nonfinite": nft, "step": t.value}
+
+    def step_layer(self, layer: int, last: bool, stats: bool = False):
+        """Stage 3: one layer of the step (every rank's GRAD buffer holds the
+        layer's gradient); ``last`` completes the step.  Statistics as step()."""
+        ordered_step(self._dist, self._sync,
+                     lambda: self._check(zero_dist_step_layer(self.ctx, int(layer), 1 if last else 0, self._stream()),
+                                         "zero_dist_step_layer"), self.group)
+        if not (stats and last):
             return None
         sq, nf, t = ctypes.c_double(), ctypes.c_int64(), ctypes.c_int64()
         self._check(zero_dist_read_partial(self.ctx, self._stream(), ctypes.byref(sq), ctypes.byref(nf),

@@ -53,7 +53,9 @@ struct IpcEntry {
   int64_t offset;
   int64_t bytes;
 };
-static_assert(2 * sizeof(IpcEntry) <= ZERO_DIST_HANDLE_BYTES, "two exported arenas fit a rank's record");
+constexpr int kExported = 3;  // GRAD, PARAM, GATHER (an empty arena's entry is zero)
+constexpr int kExportedArena[kExported] = {ZERO_DIST_ARENA_GRAD, ZERO_DIST_ARENA_PARAM, ZERO_DIST_ARENA_GATHER};
+static_assert(kExported * sizeof(IpcEntry) <= ZERO_DIST_HANDLE_BYTES, "the exported arenas fit a rank's record");
 
 thread_local std::string g_dist_init_error;
 
@@ -67,14 +69,16 @@ struct zero_dist {
   char* arena[ZERO_DIST_NUM_ARENAS] = {};
   bool bound = false;
   bool peers_open = false;
-  uint16_t* peer_grad[zsm::kMaxRanks] = {};   // every rank's gradient replica, element 0 (own: local)
-  uint16_t* peer_param[zsm::kMaxRanks] = {};  // every rank's parameter replica, element 0
+  uint16_t* peer_grad[zsm::kMaxRanks] = {};    // every rank's gradient replica (stage 3: layer buffer), element 0
+  uint16_t* peer_param[zsm::kMaxRanks] = {};   // every rank's parameter replica, element 0 (stage 1, 2)
+  uint16_t* peer_gather[zsm::kMaxRanks] = {};  // every rank's temporary gathered-layer buffer (stage 3)
   std::vector<void*> mapped;                  // IPC mappings this context opened
   int sm_count = 0, grid = 0, grid_simple = 0;
   zero_adam_hparams hp{};
   bool have_hp = false;
   bool loaded = false;
   int64_t t = 0;            // completed steps
+  int layers_in_step = 0;   // stage 3: layer launches of the step in progress
   double p1 = 1.0, p2 = 1.0;  // beta1^t, beta2^t: t binary64 multiplications, one per step
   std::string err;
   ~zero_dist() {
@@ -178,11 +182,11 @@ zero_status zero_dist_init(const zero_layout* layout, int32_t world, int32_t ran
     g_dist_init_error = "need 1 <= world <= ZERO_MAX_RANKS and 0 <= rank < world";
     return ZERO_EINVAL;
   }
-  if (stage == ZERO_STAGE_3 || stage == ZERO_STAGE_DP) {
-    g_dist_init_error = "one rank per GPU is built for stages 1 and 2";
+  if (stage == ZERO_STAGE_DP) {
+    g_dist_init_error = "plain data parallelism exists only in the oracle";
     return ZERO_ENOTIMPL;
   }
-  if (stage != ZERO_STAGE_1 && stage != ZERO_STAGE_2) {
+  if (stage != ZERO_STAGE_1 && stage != ZERO_STAGE_2 && stage != ZERO_STAGE_3) {
     g_dist_init_error = "unknown stage";
     return ZERO_EINVAL;
   }
@@ -196,10 +200,16 @@ zero_status zero_dist_init(const zero_layout* layout, int32_t world, int32_t ran
   d->world = world;
   d->rank = rank;
   d->stage = stage;
-  const int64_t S = d->plan.shard, P = d->plan.psi_pad;
+  const int64_t S = d->plan.shard, P = d->plan.psi_pad, L = d->plan.max_layer;
   d->state_pitch = align_up(4 * S, kAlign);
-  d->arena_bytes[ZERO_DIST_ARENA_GRAD] = align_up(2 * P, kAlign);
-  d->arena_bytes[ZERO_DIST_ARENA_PARAM] = align_up(2 * P, kAlign);
+  if (stage == ZERO_STAGE_3) {  // one layer's gradient, the parameter shard, one gathered layer
+    d->arena_bytes[ZERO_DIST_ARENA_GRAD] = align_up(2 * std::max<int64_t>(L, 8), kAlign);
+    d->arena_bytes[ZERO_DIST_ARENA_PARAM] = align_up(2 * S, kAlign);
+    d->arena_bytes[ZERO_DIST_ARENA_GATHER] = align_up(2 * std::max<int64_t>(L, 8), kAlign);
+  } else {
+    d->arena_bytes[ZERO_DIST_ARENA_GRAD] = align_up(2 * P, kAlign);
+    d->arena_bytes[ZERO_DIST_ARENA_PARAM] = align_up(2 * P, kAlign);
+  }
   d->arena_bytes[ZERO_DIST_ARENA_STATES] = 3 * d->state_pitch;
   d->arena_bytes[ZERO_DIST_ARENA_SCRATCH] = kDistScratch;
   *out = d;
@@ -230,6 +240,7 @@ zero_status zero_dist_bind(zero_dist* d, void* const* arenas) {
   if (d->bound) return dfail(d, ZERO_ESTATE, "arenas are already bound");
   if (!arenas) return dfail(d, ZERO_EINVAL, "arenas is NULL");
   for (int k = 0; k < ZERO_DIST_NUM_ARENAS; ++k) {
+    if (d->arena_bytes[k] == 0) continue;
     if (!arenas[k]) return dfail(d, ZERO_EINVAL, "arena %d is NULL", k);
     if (reinterpret_cast<uintptr_t>(arenas[k]) % kAlign) return dfail(d, ZERO_EINVAL, "arena %d is not 256-byte aligned", k);
   }
@@ -237,13 +248,15 @@ zero_status zero_dist_bind(zero_dist* d, void* const* arenas) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
-    e = zsm::occupancy(d->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : zsm::kFusedZ2, d->world, &fused, &simple);
+    e = zsm::occupancy(d->stage == ZERO_STAGE_1 ? zsm::kFusedZ1 : d->stage == ZERO_STAGE_2 ? zsm::kFusedZ2 : zsm::kFusedZ3,
+                       d->world, &fused, &simple);
   if (e != cudaSuccess) return dcuda(d, e, "device query");
   d->grid = std::max(1, std::min(zsm::kMaxGrid, d->sm_count * std::max(1, fused)));
   d->grid_simple = std::max(1, std::min(zsm::kMaxGrid, d->sm_count * std::max(1, simple)));
-  for (int k = 0; k < ZERO_DIST_NUM_ARENAS; ++k) d->arena[k] = static_cast<char*>(arenas[k]);
+  for (int k = 0; k < ZERO_DIST_NUM_ARENAS; ++k) d->arena[k] = d->arena_bytes[k] ? static_cast<char*>(arenas[k]) : nullptr;
   d->peer_grad[d->rank] = reinterpret_cast<uint16_t*>(d->arena[ZERO_DIST_ARENA_GRAD]);
   d->peer_param[d->rank] = reinterpret_cast<uint16_t*>(d->arena[ZERO_DIST_ARENA_PARAM]);
+  d->peer_gather[d->rank] = reinterpret_cast<uint16_t*>(d->arena[ZERO_DIST_ARENA_GATHER]);
   e = cudaMemset(d->arena[ZERO_DIST_ARENA_SCRATCH], 0, kDistScratch);
   if (e != cudaSuccess) return dcuda(d, e, "clearing the scratch arena");
   d->bound = true;
@@ -254,24 +267,28 @@ zero_status zero_dist_bind(zero_dist* d, void* const* arenas) {
 zero_status zero_dist_export(zero_dist* d, void* record) {
   if (!d || !record) return ZERO_EINVAL;
   if (!d->bound) return dfail(d, ZERO_ESTATE, "arenas are not bound (zero_dist_bind)");
-  IpcEntry ent[2];
+  IpcEntry ent[kExported];
   std::memset(ent, 0, sizeof ent);
-  const int which[2] = {ZERO_DIST_ARENA_GRAD, ZERO_DIST_ARENA_PARAM};
-  CUdeviceptr bases[2] = {0, 0};
-  for (int k = 0; k < 2; ++k) {
+  CUdeviceptr bases[kExported] = {};
+  for (int k = 0; k < kExported; ++k) {
+    const int which = kExportedArena[k];
+    if (d->arena_bytes[which] == 0) continue;  // zero entry: nothing to map
     size_t size = 0;
-    cudaError_t e = allocation_of(d->arena[which[k]], &bases[k], &size);
+    cudaError_t e = allocation_of(d->arena[which], &bases[k], &size);
     if (e != cudaSuccess) return dcuda(d, e, "finding the allocation of an exported arena");
     const CUdeviceptr base = bases[k];
-    if (k == 1 && bases[1] == bases[0]) {
-      ent[1].handle = ent[0].handle;  // one allocation holds both: one handle, opened once
+    int same = -1;  // an earlier arena in the same allocation: one handle, opened once
+    for (int q = 0; q < k; ++q)
+      if (ent[q].bytes && bases[q] == base) same = q;
+    if (same >= 0) {
+      ent[k].handle = ent[same].handle;
     } else {
       e = cudaIpcGetMemHandle(&ent[k].handle, reinterpret_cast<void*>(base));
       if (e != cudaSuccess)
         return dcuda(d, e, "cudaIpcGetMemHandle (arenas must come from cudaMalloc-style allocations)");
     }
-    ent[k].offset = (int64_t)(reinterpret_cast<uintptr_t>(d->arena[which[k]]) - (uintptr_t)base);
-    ent[k].bytes = d->arena_bytes[which[k]];
+    ent[k].offset = (int64_t)(reinterpret_cast<uintptr_t>(d->arena[which]) - (uintptr_t)base);
+    ent[k].bytes = d->arena_bytes[which];
   }
   std::memset(record, 0, ZERO_DIST_HANDLE_BYTES);
   std::memcpy(record, ent, sizeof ent);
@@ -287,12 +304,13 @@ zero_status zero_dist_open_peers(zero_dist* d, const void* records) {
   std::vector<std::pair<cudaIpcMemHandle_t, char*>> opened;
   for (int q = 0; q < d->world; ++q) {
     if (q == d->rank) continue;
-    IpcEntry ent[2];
+    IpcEntry ent[kExported];
     std::memcpy(ent, rec + (size_t)q * ZERO_DIST_HANDLE_BYTES, sizeof ent);
-    for (int k = 0; k < 2; ++k) {
-      if (ent[k].bytes != d->arena_bytes[k == 0 ? ZERO_DIST_ARENA_GRAD : ZERO_DIST_ARENA_PARAM] || ent[k].offset < 0 ||
-          ent[k].offset % kAlign)
+    for (int k = 0; k < kExported; ++k) {
+      const int which = kExportedArena[k];
+      if (ent[k].bytes != d->arena_bytes[which] || ent[k].offset < 0 || ent[k].offset % kAlign)
         return dfail(d, ZERO_EINVAL, "rank %d's record does not describe this layout's arenas", q);
+      if (ent[k].bytes == 0) continue;
       char* base = nullptr;
       for (auto& o : opened)
         if (std::memcmp(&o.first, &ent[k].handle, sizeof(cudaIpcMemHandle_t)) == 0) base = o.second;
@@ -305,8 +323,9 @@ zero_status zero_dist_open_peers(zero_dist* d, const void* records) {
         opened.push_back({ent[k].handle, base});
       }
       uint16_t* arena = reinterpret_cast<uint16_t*>(base + ent[k].offset);
-      if (k == 0) d->peer_grad[q] = arena;
-      else d->peer_param[q] = arena;
+      if (which == ZERO_DIST_ARENA_GRAD) d->peer_grad[q] = arena;
+      else if (which == ZERO_DIST_ARENA_PARAM) d->peer_param[q] = arena;
+      else d->peer_gather[q] = arena;
     }
   }
   d->peers_open = true;
@@ -337,8 +356,13 @@ zero_status zero_dist_load_master(zero_dist* d, const float* master_full, void* 
   a.master = master_of(d);
   a.m = m_of(d);
   a.v = v_of(d);
-  for (int q = 0; q < d->world; ++q) a.out[q] = d->peer_param[q] + lo;
-  a.n_out = d->world;
+  if (d->stage == ZERO_STAGE_3) {  // the rank's own parameter shard
+    a.out[0] = d->peer_param[d->rank];
+    a.n_out = 1;
+  } else {
+    for (int q = 0; q < d->world; ++q) a.out[q] = d->peer_param[q] + lo;
+    a.n_out = d->world;
+  }
   a.n_vec = S / zsm::kVec;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (a.n_vec > 0) {
@@ -347,6 +371,7 @@ zero_status zero_dist_load_master(zero_dist* d, const float* master_full, void* 
   }
   d->t = 0;
   d->p1 = d->p2 = 1.0;
+  d->layers_in_step = 0;
   d->loaded = true;
   return ZERO_OK;
 }
@@ -356,6 +381,7 @@ zero_status zero_dist_step(zero_dist* d, void* stream) {
   if (st != ZERO_OK) return st;
   if (!d->have_hp) return dfail(d, ZERO_ESTATE, "hyper-parameters are not set (zero_dist_set_hparams)");
   if (!d->loaded) return dfail(d, ZERO_ESTATE, "state is not initialised (zero_dist_load_master)");
+  if (d->stage == ZERO_STAGE_3) return dfail(d, ZERO_ESTATE, "stage 3 steps layer by layer (zero_dist_step_layer)");
   const int N = d->world;
   const int64_t S = d->plan.shard, lo = d->rank * S;
   const double p1 = d->p1 * d->hp.beta1, p2 = d->p2 * d->hp.beta2;
@@ -386,6 +412,59 @@ zero_status zero_dist_step(zero_dist* d, void* stream) {
   return ZERO_OK;
 }
 
+zero_status zero_dist_step_layer(zero_dist* d, int32_t layer, int32_t last, void* stream) {
+  zero_status st = check_ready(d);
+  if (st != ZERO_OK) return st;
+  if (!d->have_hp) return dfail(d, ZERO_ESTATE, "hyper-parameters are not set (zero_dist_set_hparams)");
+  if (!d->loaded) return dfail(d, ZERO_ESTATE, "state is not initialised (zero_dist_load_master)");
+  if (d->stage != ZERO_STAGE_3) return dfail(d, ZERO_ESTATE, "layer-by-layer steps are stage 3's (zero_dist_step)");
+  if (layer < 0 || layer >= (int32_t)d->plan.layers.size())
+    return dfail(d, ZERO_EINVAL, "layer %d out of range", layer);
+  const int N = d->world;
+  const int64_t S = d->plan.shard, own_lo = d->rank * S, own_hi = own_lo + S;
+  const int64_t l_lo = d->plan.layers[layer].lo, l_hi = d->plan.layers[layer].hi;
+  const int64_t lo = std::max(l_lo, own_lo), hi = std::min(l_hi, own_hi);  // the layer's part of this shard
+  const double p1 = d->p1 * d->hp.beta1, p2 = d->p2 * d->hp.beta2;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (hi > lo) {
+    zsm::FusedArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.fmt = zsm::kFmtBf16;
+    for (int q = 0; q < N; ++q) {
+      a.grad[q] = d->peer_grad[q] + (lo - l_lo);   // every rank's layer gradient, at this part
+      a.out[q] = d->peer_gather[q] + (lo - l_lo);  // every rank's gathered layer, at this part
+    }
+    a.param_shard = d->peer_param[d->rank] + (lo - own_lo);
+    a.master = master_of(d) + (lo - own_lo);
+    a.m = m_of(d) + (lo - own_lo);
+    a.v = v_of(d) + (lo - own_lo);
+    a.n_vec = (hi - lo) / zsm::kVec;
+    a.n_ranks = N;
+    a.accumulate = d->layers_in_step > 0 ? 1 : 0;
+    a.inv_n = (float)(1.0 / (double)N);
+    a.pdl = zsm::kPdlNone;
+    a.sc = scalars_of(d->hp, p1, p2);
+    a.ns = scratch_of(d);
+    const int64_t want = (a.n_vec + zsm::kThreads - 1) / zsm::kThreads;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, d->grid));
+    cudaError_t e = zsm::launch_fused(zsm::kFusedZ3, a, grid, s);
+    if (e != cudaSuccess) return dcuda(d, e, "fused step kernel launch");
+    d->layers_in_step += 1;
+  }
+  if (last) {
+    if (d->layers_in_step == 0) {  // no part of any layer on this rank: the step's sums are zero
+      const zsm::NormScratch ns = scratch_of(d);
+      cudaError_t e = cudaMemsetAsync(ns.step_sq, 0, 16, s);
+      if (e != cudaSuccess) return dcuda(d, e, "clearing the step's sums");
+    }
+    d->t += 1;
+    d->p1 = p1;
+    d->p2 = p2;
+    d->layers_in_step = 0;
+  }
+  return ZERO_OK;
+}
+
 zero_status zero_dist_adam_shard(zero_dist* d, const void* grad_shard, void* stream) {
   zero_status st = check_ready(d);
   if (st != ZERO_OK) return st;
@@ -402,7 +481,7 @@ zero_status zero_dist_adam_shard(zero_dist* d, const void* grad_shard, void* str
   a.master = master_of(d);
   a.m = m_of(d);
   a.v = v_of(d);
-  a.out = d->peer_param[d->rank] + lo;
+  a.out = d->stage == ZERO_STAGE_3 ? d->peer_param[d->rank] : d->peer_param[d->rank] + lo;
   a.n_vec = S / zsm::kVec;
   a.sc = scalars_of(d->hp, p1, p2);
   if (a.n_vec > 0) {
@@ -442,8 +521,19 @@ zero_status zero_dist_view(const zero_dist* dc, int32_t what, void** ptr, int64_
     case ZERO_VIEW_MASTER: *ptr = master_of(d); *n_elems = d->plan.shard; return ZERO_OK;
     case ZERO_VIEW_EXP_AVG: *ptr = m_of(d); *n_elems = d->plan.shard; return ZERO_OK;
     case ZERO_VIEW_EXP_AVG_SQ: *ptr = v_of(d); *n_elems = d->plan.shard; return ZERO_OK;
-    case ZERO_VIEW_PARAM: *ptr = d->arena[ZERO_DIST_ARENA_PARAM]; *n_elems = d->plan.psi_pad; return ZERO_OK;
-    case ZERO_VIEW_GRAD_BUF: *ptr = d->arena[ZERO_DIST_ARENA_GRAD]; *n_elems = d->plan.psi_pad; return ZERO_OK;
+    case ZERO_VIEW_PARAM:
+      *ptr = d->arena[ZERO_DIST_ARENA_PARAM];
+      *n_elems = d->stage == ZERO_STAGE_3 ? d->plan.shard : d->plan.psi_pad;
+      return ZERO_OK;
+    case ZERO_VIEW_GRAD_BUF:
+      *ptr = d->arena[ZERO_DIST_ARENA_GRAD];
+      *n_elems = d->stage == ZERO_STAGE_3 ? d->plan.max_layer : d->plan.psi_pad;
+      return ZERO_OK;
+    case ZERO_VIEW_GATHER:
+      if (d->stage != ZERO_STAGE_3) return dfail(d, ZERO_EINVAL, "the gathered-layer buffer is stage 3's");
+      *ptr = d->arena[ZERO_DIST_ARENA_GATHER];
+      *n_elems = d->plan.max_layer;
+      return ZERO_OK;
     default: return dfail(d, ZERO_EINVAL, "view %d does not exist for one rank per GPU", what);
   }
 }
