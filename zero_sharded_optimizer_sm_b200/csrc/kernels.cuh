@@ -273,5 +273,8 @@ int64_t two_pass_tile();
 cudaError_t launch_adam_bcast_bulk(const AdamBcastArgs& a, int grid, bool uniform, int stages, int store_hint,
                                    cudaStream_t s);
 int64_t bulk_bcast_tile();
+// Pass 1 with bulk stores (two_pass_tma.cu), N <= 16: 1024-element tiles,
+// eight consumer warps, a ring of `stages` (fitted to shared memory).
+cudaError_t launch_reduce_bulk(const ReduceArgs& a, int grid, int stages, int store_hint, cudaStream_t s);
 
 }  // namespace zsm

@@ -183,6 +183,165 @@ __global__ void __launch_bounds__(kTpThreads, 1)
   norm_epilogue<kTpThreads>(a.ns, sq, nf, a.accumulate);
 }
 
+// Pass 1 with bulk stores (N <= 16): the consumers add the tile's N slices
+// in rank order and write the rounded mean over rank 0's slice in the stage
+// (each lane over the elements it alone read); a storer warp's elected lane
+// copies it out with bulk stores -- to the reduced-gradient shard, or back to
+// all N replicas (the all-reduce) -- and releases the stage once the copies
+// have read it.  Tiles of 1024 elements, eight consumer warps.
+constexpr int kBulkRedTile = 1024;
+constexpr int kBulkRedWarps = 8;
+constexpr int kBulkRedThreads = 32 * (kBulkRedWarps + 2);
+
+inline size_t bulk_reduce_smem_bytes(int n_ranks, int stages) {
+  return (size_t)stages * (size_t)(2 * n_ranks * kBulkRedTile) + 3 * (size_t)stages * sizeof(uint64_t) +
+         4 * (size_t)(stages + 1);
+}
+
+template <bool kWriteBack, class F>
+__global__ void __launch_bounds__(kBulkRedThreads, 1)
+    reduce_bulk_kernel(const __grid_constant__ ReduceArgs a, int stages, int store_hint) {
+  constexpr int T = kBulkRedTile;
+  constexpr int W = kBulkRedWarps;
+  constexpr int EPT = T / (32 * W);
+  static_assert(EPT == 4, "four elements per consumer lane");
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const unsigned sb = (unsigned)(2 * N * T);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * sb);
+  uint64_t* computed = full + stages;
+  uint64_t* empty = computed + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_k = abort_flag + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + T - 1) / T;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&computed[s], W);
+      mbar_init(&empty[s], 1);
+      last_k[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (k > 0) {
+          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag, a.ns.wait_ns);
+          if (w != 0) {
+            if (w == 1) atomicOr(a.ns.error, 1u);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        fence_proxy_async_smem();
+        const int64_t e0 = tile * T;
+        const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+        unsigned char* st = smem + (size_t)s * sb;
+        mbar_expect_tx(&full[s], (unsigned)(cnt * 2 * N));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * T, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
+        last_k[s] = (int)k;
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- storer --
+    if (lane == 0) {
+      const uint64_t spol = evict_first_policy();
+      auto put = [&](void* dst, const void* src, unsigned bytes) {
+        if (store_hint) bulk_store(dst, src, bytes, spol);
+        else bulk_store(dst, src, bytes);
+      };
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag, a.ns.wait_ns);
+        if (w != 0) {
+          if (w == 1) atomicOr(a.ns.error, 8u);
+          *abort_flag = 1;
+          break;
+        }
+        const int64_t e0 = tile * T;
+        const unsigned cnt = (unsigned)((n_elem - e0) < T ? (n_elem - e0) : T);
+        const unsigned char* st = smem + (size_t)s * sb;
+        if (kWriteBack) {
+          for (int r = 0; r < N; ++r) put(const_cast<uint16_t*>(a.grad[r]) + e0, st, 2 * cnt);
+        } else {
+          put(a.shard_out + e0, st, 2 * cnt);
+        }
+        bulk_commit();
+        bulk_wait_read<0>();  // the copies have read the stage: hand it back to the producer
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait<0>();  // every store of this CTA performed before the CTA ends
+    }
+  } else {
+    // ----------------------------------------------------------- consumers --
+    const int j = (threadIdx.x - 64) * EPT;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.ns.wait_ns));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      const int64_t e0 = tile * T;
+      const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+      unsigned char* st = smem + (size_t)s * sb;
+      if (j < cnt) {  // cnt is a multiple of 8, so a lane's four elements are whole
+        float acc[EPT] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int r = 0; r < N; ++r) {
+          const uint2 w2 = *reinterpret_cast<const uint2*>(st + (size_t)r * 2 * T + 2 * j);
+          acc[0] = __fadd_rn(acc[0], F::lo(w2.x));
+          acc[1] = __fadd_rn(acc[1], F::hi(w2.x));
+          acc[2] = __fadd_rn(acc[2], F::lo(w2.y));
+          acc[3] = __fadd_rn(acc[3], F::hi(w2.y));
+        }
+        uint16_t g16[EPT];
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+          g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
+          const float g = F::f32(g16[q]);
+          const double d = (double)g;
+          sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
+          nf += isfinite(g) ? 0ull : 1ull;
+        }
+        *reinterpret_cast<uint2*>(st + 2 * j) = make_uint2(pack2(g16[0], g16[1]), pack2(g16[2], g16[3]));
+      }
+      fence_proxy_async_smem();  // this lane's stage writes before the storer's bulk copies read them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&computed[s]);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
+  }
+  norm_epilogue<kBulkRedThreads>(a.ns, sq, nf, a.accumulate);
+}
+
 // Pass 1 above 16 ranks: a tile's N slices do not fit a stage, so the
 // producer streams them in chunks of kChunk ranks (32 KB stages) and the
 // consumers add each chunk in rank order -- the same sequence of additions.
@@ -586,6 +745,10 @@ cudaError_t two_pass_configure() {
   if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<F16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_kernel<Bf16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_kernel<F16>);
+  if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<false, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<true, Bf16>);
+  if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<false, F16>);
+  if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<true, F16>);
   return e;
 }
 
@@ -633,6 +796,22 @@ cudaError_t launch_adam_bcast_bulk(const AdamBcastArgs& a, int grid, bool unifor
     adam_bcast_bulk_kernel<F16><<<grid, kBulkBcastThreads, bytes, s>>>(a, stages, uniform ? 1 : 0, store_hint);
   else
     adam_bcast_bulk_kernel<Bf16><<<grid, kBulkBcastThreads, bytes, s>>>(a, stages, uniform ? 1 : 0, store_hint);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_bulk(const ReduceArgs& a, int grid, int stages, int store_hint, cudaStream_t s) {
+  if (a.n_ranks < 1 || a.n_ranks > kTmaMaxRanks) return cudaErrorInvalidValue;
+  if (stages < 2) stages = 2;
+  if (stages > kTmaMaxStages) stages = kTmaMaxStages;
+  while (stages > 2 && bulk_reduce_smem_bytes(a.n_ranks, stages) > (size_t)kTmaMaxSmem) --stages;
+  const size_t bytes = bulk_reduce_smem_bytes(a.n_ranks, stages);
+  if (a.fmt == kFmtF16) {
+    if (a.write_back) reduce_bulk_kernel<true, F16><<<grid, kBulkRedThreads, bytes, s>>>(a, stages, store_hint);
+    else reduce_bulk_kernel<false, F16><<<grid, kBulkRedThreads, bytes, s>>>(a, stages, store_hint);
+  } else {
+    if (a.write_back) reduce_bulk_kernel<true, Bf16><<<grid, kBulkRedThreads, bytes, s>>>(a, stages, store_hint);
+    else reduce_bulk_kernel<false, Bf16><<<grid, kBulkRedThreads, bytes, s>>>(a, stages, store_hint);
+  }
   return cudaGetLastError();
 }
 

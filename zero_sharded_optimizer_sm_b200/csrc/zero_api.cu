@@ -756,8 +756,17 @@ cudaError_t launch_pass1(zero_ctx* c, const zsm::ReduceArgs& a, cudaStream_t s) 
   const int64_t elems = a.n_vec * zsm::kVec;
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  const cudaError_t e = counted(c, use_two_pass_tma(c) ? zsm::launch_reduce_tma(a, two_pass_grid(c, elems), s)
-                                                       : zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s));
+  cudaError_t e;
+  if (use_bulk(c) && a.n_ranks <= zsm::kTmaMaxRanks) {
+    // the bulk-store pass 1: four 1024-element stages unless the ring depth is set
+    const int64_t tiles = (elems + 1023) / 1024;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(tiles, c->sm_count));
+    e = counted(c, zsm::launch_reduce_bulk(a, grid, c->tma_stages_opt ? c->tma_stages_opt : 4,
+                                           c->store_hint >= 0 ? c->store_hint : 1, s));
+  } else {
+    e = counted(c, use_two_pass_tma(c) ? zsm::launch_reduce_tma(a, two_pass_grid(c, elems), s)
+                                       : zsm::launch_reduce(a, grid_for(a.n_vec, c->grid_simple), s));
+  }
   if (e == cudaSuccess && ev) {
     cudaEventRecord(ev[1], s);
     c->timed += 1;
