@@ -536,8 +536,9 @@ def run_ours(args, world, rank, local):
                "steps": args.e2e_steps,
                "how": "zero_step through the C ABI with ZERO_OPT_PIPELINE; grad_fn copies each "
                       "bucket's N gradient slices from pinned host memory into one of the two "
-                      "200M-element buffers, one bucket ahead of the fused kernel; stats (grad norm, "
-                      "non-finite count) read back every step"}
+                      "200M-element buffers, one bucket ahead of the fused kernel; only the step's "
+                      "16-byte statistics (sum of squares, non-finite count) come back to the host "
+                      "each step -- the updated parameters stay on the device for the next forward"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, stage=stage)
