@@ -267,3 +267,46 @@ def test_probe_pattern_refuses_a_configuration_that_is_not_built():
         opt.step_resident(list(reps_t))
     assert e.value.status == z.ZERO_ECUDA
     opt.close()
+
+
+@pytest.mark.parametrize("n_ranks", [4, 8])
+def test_zero3_chained_layers_order_their_shared_buffer_stores(n_ranks):
+    """ZeRO-3 resident steps with chained launches.  Every layer writes the
+    same temporary layer buffers, so a launch's stores wait until the launch
+    before has finished; its loads and arithmetic may start earlier.  The
+    test uses three layers of about 3.1M elements (more than 16 tiles per
+    CTA).  It compares them with the same steps launched plainly, on every
+    view and every rank's layer buffer.  It also compares them with the
+    oracle: states, parameter shards, and the last gathered layer (the first
+    layer, which ends in the buffers)."""
+    z = _z()
+    numel, layer = W.transformer_layers(3, 512, 2048)
+    w = _workload(numel, layer, n_ranks, 3, 1 << 30, steps=2)
+    p, ranks, reps, ref = _oracle(w, 3, 1 << 30)
+    s = torch.cuda.current_stream().cuda_stream
+    opts = []
+    for pdl in (True, False):
+        opt, fill = _make(w, 3, None, True, 1024, 8)
+        opt.set_pdl(pdl)
+        opts.append((opt, fill))
+    for t in range(1, w.steps + 1):
+        for opt, fill in opts:
+            reps_t = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+            for r in range(n_ranks):
+                fill.grads_into(t, r, 0, opt.psi_pad, reps_t[r].data_ptr(), reps_t[r], s)
+            opt.step_resident(list(reps_t))
+        torch.cuda.synchronize()
+    (a, _), (b, _) = opts
+    assert len(a.layers()) == 3 and all(hi - lo > 16 * 148 * 1024 for _, lo, hi in a.layers())
+    for k, view in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert torch.equal(a.view(view), b.view(view))
+        assert_bits_equal(to_np(a.view(view)), ref[k], f"chained ZeRO-3 {k}")
+    assert torch.equal(a.view(z.ZERO_VIEW_PARAM), b.view(z.ZERO_VIEW_PARAM))
+    assert_bits_equal(to_np(a.view(z.ZERO_VIEW_PARAM)), ref["params"], "chained ZeRO-3 param shards")
+    _, lo0, hi0 = a.layers()[0]
+    for r in range(n_ranks):
+        assert torch.equal(a.view(z.ZERO_VIEW_GATHER, r), b.view(z.ZERO_VIEW_GATHER, r)), r
+        assert_bits_equal(to_np(a.view(z.ZERO_VIEW_GATHER, r))[: hi0 - lo0], ref["params"][lo0:hi0],
+                          f"chained ZeRO-3 last gathered layer, rank {r}")
+    a.close()
+    b.close()
