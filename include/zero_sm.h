@@ -57,7 +57,8 @@ typedef enum zero_status {
   ZERO_ENOMEM = 2,   /* an arena the caller sized is too small for this context */
   ZERO_ECUDA = 3,    /* a CUDA runtime error (launch or asynchronous fault) */
   ZERO_ESTATE = 4,   /* call out of order: arenas not bound, hyper-parameters unset */
-  ZERO_ENOTIMPL = 5  /* a combination the library does not provide */
+  ZERO_ENOTIMPL = 5, /* a combination the library does not provide */
+  ZERO_EGUARD = 6    /* a guard byte of an arena changed (ZERO_OPT_GUARD, zero_check_guards) */
 } zero_status;
 
 /* ZeRO stages ([T] section "一张总对比表"; [Q] section 一). */
@@ -194,6 +195,27 @@ enum {
                                     parameters and states of a step that ran out are partly
                                     updated: restore them (zero_import_state) before going on.
                                     May be set at any time */
+  ZERO_OPT_NVTX = 18,            /* 1: NVTX ranges on the domain "zero_sm" around the host side
+                                    of each step ("step t (stage s, N = n)"), of each of its
+                                    launches ("bucket k [lo, hi)", "layer id [lo, hi)"; a
+                                    clipped step: "reduce ...", "clip decision", "update
+                                    ..."), and of each unfused call, so that a profiler
+                                    attributes the kernels to buckets and layers; without a
+                                    tool attached a range costs a function call.  Default 0;
+                                    may be set at any time */
+  ZERO_OPT_GUARD = 17,           /* guard bytes around the library's buffers, a stand-in for a
+                                    bounds-checking sanitizer: 1 adds 256 bytes after each
+                                    arena (arena_bytes grows by 256 for every arena in use) and
+                                    makes the unused end of every row of an arena -- each rank
+                                    replica, master / m / v, gradient or layer buffer: the
+                                    pitch's 256-byte alignment slack and ZERO_OPT_REPLICA_PAD --
+                                    a guard too.  zero_load_master and zero_import_state fill
+                                    them with the byte 0xA5; zero_check_guards finds bytes
+                                    that changed.  2: as 1, and zero_step / zero_step_resident
+                                    check them after every step (waiting for the step) and
+                                    return ZERO_EGUARD when one changed.  Values are
+                                    unchanged.  Default 0; 0 <-> 1 or 2 before zero_bind, 1 <->
+                                    2 at any time */
   ZERO_OPT_PDL = 12              /* 1 (default): a step without callbacks (zero_step_resident
                                     with no gather_fn) launches its fused kernels with
                                     programmatic dependent launch, so that each launch's CTAs
@@ -700,6 +722,17 @@ zero_status zero_probe_pattern(zero_ctx* ctx, const void* const* rank_grads, voi
  * precision checks).
  */
 zero_status zero_read_stats(zero_ctx* ctx, void* stream, zero_step_stats* out);
+
+/* Check the guard bytes (ZERO_OPT_GUARD) on `stream` and wait for the
+ * result.  Every guard byte that is not 0xA5 is counted and written back,
+ * so a later check reports only later changes.  out (may be NULL) =
+ * {changed bytes, arena of the first changed byte (ZERO_ARENA_*), its byte
+ * offset in that arena}, or {0, -1, -1}.  Returns ZERO_OK when none changed,
+ * ZERO_EGUARD when some did (the message names the arena and the row or the
+ * tail), ZERO_ESTATE when the context has no guard bytes or its state is
+ * not loaded.  A check made while a step is still running on another stream
+ * may see that step's stores in progress, never outside its buffers. */
+zero_status zero_check_guards(zero_ctx* ctx, void* stream, int64_t out[3]);
 
 /* Message of the last failure on ctx (never NULL; "" when none).  With
  * ctx == NULL: the reason the calling thread's last zero_init failed.

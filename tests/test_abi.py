@@ -152,6 +152,63 @@ def test_pipeline_option_doubles_only_the_slot_arenas(stage):
         assert on[k] == (2 * off[k] if doubled else off[k]), (k, off[k], on[k])
 
 
+@pytest.mark.parametrize("stage", [1, 2, 3])
+@pytest.mark.parametrize("extra", [{}, {"pipe": 1, "pad": 512}, {"keep": 0}])
+def test_guard_option_adds_a_tail_to_every_arena_in_use(stage, extra):
+    """ZERO_OPT_GUARD (before binding) grows every arena in use by its
+    256-byte tail and leaves the rows' pitches alone; unused arenas stay 0."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    numel, layer = W.transformer_layers(3, 24, 96)
+    got = []
+    for guard in (0, 1, 2):
+        st, ctx = _init(numel, layer, 4, stage, 4096)
+        assert st == 0
+        try:
+            if "pipe" in extra:
+                assert z.zero_set_option(ctx, z.ZERO_OPT_PIPELINE, extra["pipe"]) == 0
+            if "pad" in extra:
+                assert z.zero_set_option(ctx, z.ZERO_OPT_REPLICA_PAD, extra["pad"]) == 0
+            if "keep" in extra:
+                assert z.zero_set_option(ctx, z.ZERO_OPT_KEEP_GRAD_SHARDS, extra["keep"]) == 0
+            assert z.zero_set_option(ctx, z.ZERO_OPT_GUARD, guard) == 0
+            zs = z.zero_sizes()
+            assert z.zero_buffer_sizes(ctx, ctypes.byref(zs)) == 0
+            got.append((list(zs.arena_bytes), zs.replica_pitch))
+        finally:
+            z.zero_destroy(ctx)
+    (off, pitch0), (on1, pitch1), (on2, pitch2) = got
+    assert pitch0 == pitch1 == pitch2
+    assert on1 == on2
+    for k in range(z.ZERO_NUM_ARENAS):
+        assert on1[k] == (off[k] + 256 if off[k] else 0), (k, off[k], on1[k])
+
+
+def test_guard_and_nvtx_option_values_and_the_check_without_a_device():
+    """ZERO_OPT_GUARD takes 0, 1 or 2 and ZERO_OPT_NVTX any value at any
+    time; zero_check_guards refuses a context without guard bytes or not yet
+    bound, before any device work, and leaves {0, -1, -1}."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    st, ctx = _init([100, 28], [0, 1], 2, 2, 64)
+    assert st == 0
+    try:
+        out = (ctypes.c_int64 * 3)(7, 7, 7)
+        assert z.zero_check_guards(ctx, None, out) == z.ZERO_ESTATE and list(out) == [0, -1, -1]
+        assert b"ZERO_OPT_GUARD" in z.zero_last_error(ctx)
+        assert z.zero_set_option(ctx, z.ZERO_OPT_GUARD, 3) == z.ZERO_EINVAL
+        assert z.zero_set_option(ctx, z.ZERO_OPT_GUARD, -1) == z.ZERO_EINVAL
+        assert z.zero_set_option(ctx, z.ZERO_OPT_GUARD, 2) == z.ZERO_OK
+        assert z.zero_check_guards(ctx, None, out) == z.ZERO_ESTATE  # not bound
+        assert b"armed" in z.zero_last_error(ctx)
+        assert z.zero_check_guards(ctx, None, None) == z.ZERO_ESTATE
+        for v in (1, 0, 5):
+            assert z.zero_set_option(ctx, z.ZERO_OPT_NVTX, v) == z.ZERO_OK
+    finally:
+        z.zero_destroy(ctx)
+    assert z.zero_check_guards(None, None, None) == z.ZERO_EINVAL
+
+
 def test_pipeline_streams_and_option_values_on_the_host():
     """zero_set_pipeline_streams needs no GPU before the first pipelined step
     (it only records the handles); ZERO_OPT_PIPELINE takes 0, 1 or 2."""

@@ -30,9 +30,9 @@ lib = ctypes.CDLL(LIB_PATH)
 
 # ------------------------------------------------------------------ C ABI ----
 
-ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ENOTIMPL = range(6)
+ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ENOTIMPL, ZERO_EGUARD = range(7)
 STATUS_NAMES = {0: "ZERO_OK", 1: "ZERO_EINVAL", 2: "ZERO_ENOMEM", 3: "ZERO_ECUDA", 4: "ZERO_ESTATE",
-                5: "ZERO_ENOTIMPL"}
+                5: "ZERO_ENOTIMPL", 6: "ZERO_EGUARD"}
 ZERO_STAGE_DP, ZERO_STAGE_1, ZERO_STAGE_2, ZERO_STAGE_3 = 0, 1, 2, 3
 ZERO_MAX_RANKS = 128
 (ZERO_ARENA_STATES, ZERO_ARENA_PARAMS, ZERO_ARENA_GRADS, ZERO_ARENA_GRAD_SHARDS, ZERO_ARENA_GATHER,
@@ -50,6 +50,8 @@ ZERO_OPT_TMA_TILE = 13
 ZERO_OPT_TMA_WARPS = 14
 ZERO_OPT_WAIT_LIMIT_NS = 15
 ZERO_OPT_STORE_HINT = 16
+ZERO_OPT_GUARD = 17
+ZERO_OPT_NVTX = 18
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -119,6 +121,7 @@ _SIGS = {
     "zero_fused_tile": (_i32, [_vp, ctypes.POINTER(_i32)]),
     "zero_probe_pattern": (_i32, [_vp, _PTRS, _vp]),
     "zero_read_stats": (_i32, [_vp, _vp, ctypes.POINTER(zero_step_stats)]),
+    "zero_check_guards": (_i32, [_vp, _vp, ctypes.POINTER(ctypes.c_int64)]),
     "zero_fused_step_static": (_i32, [_i32, _i64, _PTRS, _vp, _vp, _vp, _PTRS,
                                       ctypes.POINTER(zero_adam_hparams), _i64, _vp, _vp]),
     "zero_dist_init": (_i32, [ctypes.POINTER(zero_layout), _i32, _i32, _i32, ctypes.POINTER(_vp)]),
@@ -247,7 +250,7 @@ class ZeroOptimizer:
                  keep_grad_shards: bool = True, replica_pad: int = 0, blocks_per_sm: int = 0,
                  kernel: int = ZERO_KERNEL_AUTO, grad_buffers: bool = True, tma_groups: int = 0,
                  tma_stages: int = 0, tma_ctas_per_sm: int = 0, dtype: int = ZERO_DTYPE_BF16,
-                 pipeline: int = 0, tma_tile: int = 0, tma_warps: int = 0, device=None):
+                 pipeline: int = 0, tma_tile: int = 0, tma_warps: int = 0, guard: int = 0, device=None):
         import torch
 
         self._torch = torch
@@ -287,6 +290,8 @@ class ZeroOptimizer:
             self._check(zero_set_option(ctx, ZERO_OPT_TMA_WARPS, int(tma_warps)), "zero_set_option")
         if pipeline:
             self._check(zero_set_option(ctx, ZERO_OPT_PIPELINE, int(pipeline)), "zero_set_option")
+        if guard:
+            self._check(zero_set_option(ctx, ZERO_OPT_GUARD, int(guard)), "zero_set_option")
         self.pipeline = int(pipeline)
         self.sizes = zero_sizes()
         self._check(zero_buffer_sizes(ctx, ctypes.byref(self.sizes)), "zero_buffer_sizes")
@@ -559,6 +564,29 @@ class ZeroOptimizer:
         n = ctypes.c_int64()
         self._check(zero_launch_count(self.ctx, ctypes.byref(n)), "zero_launch_count")
         return n.value
+
+    def check_guards(self, stream=None) -> dict:
+        """Check the arenas' guard bytes (ZERO_OPT_GUARD; waits for the
+        stream).  Returns {"changed": bytes, "arena": first's arena, "offset":
+        its byte offset} ({0, -1, -1} when clean, "message" naming the row or
+        tail otherwise); other failures raise."""
+        out = (ctypes.c_int64 * 3)()
+        st = zero_check_guards(self.ctx, self._stream(stream), out)
+        if st not in (ZERO_OK, ZERO_EGUARD):
+            self._check(st, "zero_check_guards")
+        res = dict(changed=out[0], arena=out[1], offset=out[2])
+        if st == ZERO_EGUARD:
+            res["message"] = zero_last_error(self.ctx).decode()
+        return res
+
+    def set_nvtx(self, on: bool):
+        """NVTX ranges per step, launch and unfused call on the domain "zero_sm" (ZERO_OPT_NVTX)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_NVTX, 1 if on else 0), "zero_set_option")
+
+    def set_guard(self, mode: int):
+        """1: guards checked on request; 2: also after every step (ZERO_OPT_GUARD; the
+        context must have been made with guard bytes)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_GUARD, int(mode)), "zero_set_option")
 
     def read_stats(self, stream=None) -> dict:
         out = zero_step_stats()

@@ -12,7 +12,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = ["csrc/zero_api.cu", "csrc/kernels.cu", "csrc/fused_tma.cu", "csrc/fused_bulk.cu", "csrc/static_scratch.cu",
-           "csrc/two_pass_tma.cu", "csrc/dist.cu",
+           "csrc/two_pass_tma.cu", "csrc/dist.cu", "csrc/guards.cu",
            "csrc/plan.cpp"]
 LIB = os.path.join(HERE, "libzero_sm.so")
 

@@ -227,6 +227,24 @@ cudaError_t launch_step_begin(StepState* state, const StepHparams& hp, ClipDecis
 cudaError_t launch_step_commit(StepState* state, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
+// Guard bytes (guards.cu): per arena, `rows` rows of `pitch` bytes from
+// `base` whose bytes [used, pitch) are guards, then `tail` guard bytes after
+// the last row (rows = tail = 0: no arena).  The check counts the guard
+// bytes that differ from kGuardByte into result[0], the least
+// (arena << 56 | byte offset) of them into result[1] (the caller sets 0 and
+// ~0 first), and restores them.
+constexpr int kGuardSets = 6;
+constexpr unsigned char kGuardByte = 0xA5;
+struct GuardSet {
+  unsigned char* base;
+  long long pitch, used, rows, tail;
+};
+struct GuardArgs {
+  GuardSet set[kGuardSets];
+  unsigned long long* result;
+};
+cudaError_t launch_guards(const GuardArgs& a, bool check, cudaStream_t s);
+
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with
 // `groups` (1 or 2) producer/consumer groups.
 cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, int max_stages,

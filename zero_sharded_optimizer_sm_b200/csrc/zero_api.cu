@@ -9,6 +9,7 @@
 // fixed-size gradient buffer and the one caller-owned pool are sections 3.3
 // "CB" and 3.4 "MD" of "ZeRO：从优化器状态到残差状态的显存优化".
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -33,8 +34,51 @@ constexpr int64_t kArenaAlign = 256;
 constexpr int64_t kScratchBytes = 80 * 1024;
 static_assert(16 * zsm::kMaxGrid + 128 + sizeof(zsm::StepState) <= kScratchBytes,
               "the scratch arena holds the norm partials, the step sums, the clip decision and the step state");
+// Guard bytes (ZERO_OPT_GUARD): the tail after each arena; the guard check's
+// two result words sit in the scratch arena past the step state.
+constexpr int64_t kGuardBytes = 256;
+constexpr int64_t kGuardResultOffset = 72 * 1024;
+static_assert(16 * zsm::kMaxGrid + 128 + sizeof(zsm::StepState) <= kGuardResultOffset &&
+                  kGuardResultOffset + 16 <= kScratchBytes,
+              "the guard check's result words follow the step state in the scratch arena");
 
 int64_t align_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
+
+// NVTX ranges on the library's own domain "zero_sm" (ZERO_OPT_NVTX): host
+// ranges around the enqueueing of a step and of each of its launches, which
+// a profiler projects onto the kernels they enqueue.  Without a tool
+// attached each call returns at once.
+nvtxDomainHandle_t nvtx_domain() {
+  static const nvtxDomainHandle_t d = nvtxDomainCreateA("zero_sm");
+  return d;
+}
+
+class NvtxRange {
+ public:
+  NvtxRange(bool on, const char* fmt, ...) : on_(on) {
+    if (!on_) return;
+    char msg[128];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(msg, sizeof msg, fmt, ap);
+    va_end(ap);
+    nvtxEventAttributes_t a;
+    std::memset(&a, 0, sizeof a);
+    a.version = NVTX_VERSION;
+    a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    a.message.ascii = msg;
+    nvtxDomainRangePushEx(nvtx_domain(), &a);
+  }
+  ~NvtxRange() {
+    if (on_) nvtxDomainRangePop(nvtx_domain());
+  }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+
+ private:
+  bool on_;
+};
 
 }  // namespace
 
@@ -85,6 +129,8 @@ struct zero_ctx {
   // staged launches then reserve enough shared memory that a grid never puts
   // two CTAs on one SM); measured 0.5-2 % faster per step on B200.
   bool pdl = true;
+  bool nvtx = false;  // ZERO_OPT_NVTX: ranges per step and per launch
+  int guard = 0;  // ZERO_OPT_GUARD: 0, 1 (laid out, armed at load, checked on request) or 2 (checked after each step)
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
   cudaStream_t side = nullptr;   // the callbacks' stream
   cudaStream_t kside = nullptr;  // the kernels' stream at the greatest priority (ZERO_OPT_PIPELINE = 2)
@@ -164,6 +210,9 @@ void compute_layout(zero_ctx* c) {
       break;
   }
   if (!c->grad_buffers) c->arena_bytes[ZERO_ARENA_GRADS] = 0;
+  if (c->guard)
+    for (int k = 0; k < ZERO_NUM_ARENAS; ++k)
+      if (c->arena_bytes[k]) c->arena_bytes[k] += kGuardBytes;
 }
 
 float* master_ptr(zero_ctx* c) { return reinterpret_cast<float*>(c->arena[ZERO_ARENA_STATES]); }
@@ -218,6 +267,34 @@ zsm::ClipDecision* decision_ptr(zero_ctx* c) {
   return reinterpret_cast<zsm::ClipDecision*>(stats_block(c) + kDecisionOffset);
 }
 zsm::StepState* state_ptr(zero_ctx* c) { return reinterpret_cast<zsm::StepState*>(stats_block(c) + kStateOffset); }
+
+// The guard bytes of each bound arena: the end of every row past the bytes
+// the library's buffers use, and the tail.  Returns false when the rows and
+// the tail do not add up to the arena's size (a layout this code does not
+// describe).
+bool guard_args(zero_ctx* c, zsm::GuardArgs* g) {
+  std::memset(g, 0, sizeof *g);
+  const zsm::Plan& p = c->plan;
+  const int64_t N = p.n_ranks;
+  const int64_t row2 = align_up(p.psi_pad * 2, kArenaAlign);
+  const int64_t grad_used = c->stage == ZERO_STAGE_1   ? p.psi_pad * 2
+                            : c->stage == ZERO_STAGE_2 ? p.max_bucket * 2
+                                                       : p.max_layer * 2;
+  const int64_t grad_rows = c->stage == ZERO_STAGE_1 ? N : c->slots * N;
+  const int64_t rows[ZERO_NUM_ARENAS] = {3, c->stage == ZERO_STAGE_3 ? 1 : N, grad_rows, 1, c->slots * N, 1};
+  const int64_t pitch[ZERO_NUM_ARENAS] = {c->state_pitch, c->param_pitch, c->grad_pitch, row2, c->gather_pitch,
+                                          kScratchBytes};
+  const int64_t used[ZERO_NUM_ARENAS] = {p.psi_pad * 4, p.psi_pad * 2, grad_used, p.psi_pad * 2, p.max_layer * 2,
+                                         kScratchBytes};
+  static_assert(ZERO_NUM_ARENAS == zsm::kGuardSets, "one guard set per arena");
+  for (int k = 0; k < ZERO_NUM_ARENAS; ++k) {
+    if (!c->arena[k]) continue;
+    if (rows[k] * pitch[k] + kGuardBytes != c->arena_bytes[k] || used[k] > pitch[k]) return false;
+    g->set[k] = zsm::GuardSet{reinterpret_cast<unsigned char*>(c->arena[k]), pitch[k], used[k], rows[k], kGuardBytes};
+  }
+  g->result = reinterpret_cast<unsigned long long*>(c->arena[ZERO_ARENA_SCRATCH] + kGuardResultOffset);
+  return true;
+}
 
 zsm::StepHparams step_hparams(const zero_ctx* c) {
   zsm::StepHparams h;
@@ -841,6 +918,9 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     a.ns = norm_scratch(c);
     o.before_kernel(k, !resident && fn, (size_t)-1);
     if (a.n_vec > 0) {
+      const NvtxRange range(c->nvtx, "reduce %s %d [%lld, %lld)", c->stage == ZERO_STAGE_3 ? "layer" : "bucket",
+                            c->stage == ZERO_STAGE_3 ? c->plan.layers[n_layers - 1 - (int)k].id : (int)k,
+                            (long long)lo, (long long)hi);
       cudaError_t e = launch_pass1(c, a, s);
       if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
       launched = true;
@@ -858,7 +938,11 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   cp.loss_scale = c->loss_scale;
   cp.skip_nonfinite = c->skip_nonfinite ? 1 : 0;
   zsm::ClipDecision* dec = decision_ptr(c);
-  cudaError_t e = counted(c, zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s));
+  cudaError_t e;
+  {
+    const NvtxRange range(c->nvtx, "clip decision");
+    e = counted(c, zsm::launch_clip_decide(norm_scratch(c), cp, dec, state_ptr(c), s));
+  }
   if (e != cudaSuccess) return cuda_fail(c, e, "the clipped step's decision");
   const zsm::AdamScalars sc{};  // the kernels read the step's scalars from the device step state
   // pass 2: Adam + broadcast, over everything (stage 1/2) or per layer (stage 3);
@@ -894,6 +978,9 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     b.wait_ns = c->wait_ns;
     o.before_kernel(k, false, c->stage == ZERO_STAGE_3 && gfn ? k : (size_t)-1);
     if (b.n_vec > 0) {
+      const NvtxRange range(c->nvtx, "update %s %d [%lld, %lld)", c->stage == ZERO_STAGE_3 ? "layer" : "all",
+                            c->stage == ZERO_STAGE_3 ? c->plan.layers[layer_idx].id : 0, (long long)lo,
+                            (long long)hi);
       // stages 2 and 3 read every owner's reduced gradient from the one shard array
       e = launch_pass2(c, b, c->stage != ZERO_STAGE_1, s);
       if (e != cudaSuccess) return cuda_fail(c, e, "adam-broadcast kernel launch");
@@ -909,6 +996,34 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   c->norm_fresh = true;
   if (stats) return finish_stats(c, o.s, stats);
   return ZERO_OK;
+}
+
+// Checks the guard bytes on `s` and waits for the result; out = {changed
+// bytes, arena of the first, its byte offset in the arena} (-1, -1 when none).
+zero_status check_guards(zero_ctx* c, cudaStream_t s, int64_t out[3]) {
+  out[0] = 0;
+  out[1] = out[2] = -1;
+  zsm::GuardArgs g;
+  if (!guard_args(c, &g)) return fail(c, ZERO_EINVAL, "guard layout does not match the arenas");
+  unsigned long long h[2] = {0ull, ~0ull};
+  cudaError_t e = cudaMemcpyAsync(g.result, h, sizeof h, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = counted(c, zsm::launch_guards(g, true, s));
+  if (e == cudaSuccess) e = cudaMemcpyAsync(h, g.result, sizeof h, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "guard check");
+  if (h[0] == 0) return ZERO_OK;
+  const int arena = (int)(h[1] >> 56);
+  const int64_t off = (int64_t)(h[1] & ((1ull << 56) - 1));
+  out[0] = (int64_t)h[0];
+  out[1] = arena;
+  out[2] = off;
+  const zsm::GuardSet& gs = g.set[arena];
+  if (off >= gs.rows * gs.pitch)
+    return fail(c, ZERO_EGUARD, "%lld guard bytes changed; the first: arena %d, byte %lld of its %lld-byte tail",
+                (long long)h[0], arena, (long long)(off - gs.rows * gs.pitch), (long long)gs.tail);
+  return fail(c, ZERO_EGUARD, "%lld guard bytes changed; the first: arena %d, row %lld, byte %lld past its %lld used bytes",
+              (long long)h[0], arena, (long long)(off / gs.pitch), (long long)(off % gs.pitch - gs.used),
+              (long long)gs.used);
 }
 
 zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
@@ -929,6 +1044,7 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   if (st != ZERO_OK) return st;
   const bool callbacks = (!resident && fn) || (c->stage == ZERO_STAGE_3 && gfn);
   StepOrder o(c, static_cast<cudaStream_t>(stream), callbacks);
+  const NvtxRange step_range(c->nvtx, "step %lld (stage %d, N = %d)", (long long)(c->calls + 1), c->stage, N);
   o.begin();
   if (c->clip_norm > 0.0 || c->skip_nonfinite) {
     st = run_two_pass(c, fn, user, resident, gfn, guser, o, stats);
@@ -972,6 +1088,9 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
                     : !launched ? zsm::kPdlWaitFirst
                     : c->stage != ZERO_STAGE_3 ? zsm::kPdlEarly
                                                : zsm::kPdlEarlyLoads;
+    const NvtxRange range(c->nvtx, "%s %d [%lld, %lld)", c->stage == ZERO_STAGE_3 ? "layer" : "bucket",
+                          c->stage == ZERO_STAGE_3 ? c->plan.layers[layer_idx].id : (int)k, (long long)lo,
+                          (long long)hi);
     st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl, &state_ptr(c)->sc);
     if (st != ZERO_OK) break;
     launched = launched || hi > lo;
@@ -1072,6 +1191,18 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     if (value > 0 && zsm::tma_stages_for(c->plan.n_ranks, (int)value) == 0)
       return fail(c, ZERO_EINVAL, "%lld consumer groups do not fit at N = %d", (long long)value, c->plan.n_ranks);
     c->tma_groups_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_NVTX) {
+    c->nvtx = value != 0;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_GUARD) {
+    if (value < 0 || value > 2) return fail(c, ZERO_EINVAL, "guard must be 0, 1 or 2");
+    if (c->bound && (value != 0) != (c->guard != 0))
+      return fail(c, ZERO_ESTATE, "guard bytes are laid out before zero_bind (after it only 1 <-> 2)");
+    c->guard = (int)value;
+    if (!c->bound) compute_layout(c);
     return ZERO_OK;
   }
   if (c->bound) return fail(c, ZERO_ESTATE, "options must be set before zero_bind");
@@ -1239,6 +1370,12 @@ zero_status load_state(zero_ctx* c, const float* master, const float* m, const f
   a.n_vec = c->plan.psi_pad / zsm::kVec;
   e = counted(c, zsm::launch_init(a, grid_for(a.n_vec, c->grid_simple), s));
   if (e != cudaSuccess) return cuda_fail(c, e, "init kernel launch");
+  if (c->guard) {  // arm the guard bytes
+    zsm::GuardArgs g;
+    if (!guard_args(c, &g)) return fail(c, ZERO_EINVAL, "guard layout does not match the arenas");
+    e = counted(c, zsm::launch_guards(g, false, s));
+    if (e != cudaSuccess) return cuda_fail(c, e, "guard fill launch");
+  }
   c->t = t;
   c->calls = t;
   c->loaded = true;
@@ -1348,6 +1485,7 @@ zero_status zero_comm_elems(const zero_ctx* c, int64_t out[3]) {
 zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void* const* rank_grads, void* stream) {
   zero_status st = check_ready(c, false);
   if (st != ZERO_OK) return st;
+  const NvtxRange range(c->nvtx, "reduce-scatter [%lld, %lld)", (long long)lo, (long long)hi);
   if (c->stage == ZERO_STAGE_1) return fail(c, ZERO_EINVAL, "stage 1 keeps full gradients: use zero_all_reduce");
   if (!c->arena[ZERO_ARENA_GRAD_SHARDS])
     return fail(c, ZERO_ESTATE, "gradient shards were dropped (ZERO_OPT_KEEP_GRAD_SHARDS = 0)");
@@ -1390,6 +1528,7 @@ zero_status zero_reduce_scatter(zero_ctx* c, int64_t lo, int64_t hi, const void*
 zero_status zero_all_reduce(zero_ctx* c, int64_t lo, int64_t hi, void* const* rank_grads, void* stream) {
   zero_status st = check_ready(c, false);
   if (st != ZERO_OK) return st;
+  const NvtxRange range(c->nvtx, "all-reduce [%lld, %lld)", (long long)lo, (long long)hi);
   if (c->stage != ZERO_STAGE_1) return fail(c, ZERO_EINVAL, "all-reduce keeps full gradients: stage 1 only");
   if ((st = check_interval(c, lo, hi)) != ZERO_OK) return st;
   const int N = c->plan.n_ranks;
@@ -1428,6 +1567,7 @@ extern "C" {
 zero_status zero_adam_shard(zero_ctx* c, int32_t rank, int64_t t, void* stream) {
   zero_status st = check_ready(c, true);
   if (st != ZERO_OK) return st;
+  const NvtxRange range(c->nvtx, "adam shard %d", rank);
   const int N = c->plan.n_ranks;
   if (rank < -1 || rank >= N) return fail(c, ZERO_EINVAL, "rank %d out of range", rank);
   if (t < 0) return fail(c, ZERO_EINVAL, "step t must be >= 1, or 0 for the context's counter + 1");
@@ -1529,6 +1669,7 @@ extern "C" {
 zero_status zero_all_gather(zero_ctx* c, int64_t lo, int64_t hi, void* const* rank_out, void* stream) {
   zero_status st = check_ready(c, false);
   if (st != ZERO_OK) return st;
+  const NvtxRange range(c->nvtx, "all-gather [%lld, %lld)", (long long)lo, (long long)hi);
   if ((st = check_interval(c, lo, hi)) != ZERO_OK) return st;
   if (hi == lo) return ZERO_OK;
   const int N = c->plan.n_ranks;
@@ -1575,14 +1716,30 @@ zero_status zero_all_gather(zero_ctx* c, int64_t lo, int64_t hi, void* const* ra
 zero_status zero_step(zero_ctx* c, zero_grad_fn grad_fn, void* grad_user, zero_gather_fn gather_fn,
                       void* gather_user, void* stream, zero_step_stats* stats) {
   if (!c) return ZERO_EINVAL;
-  return run_step(c, grad_fn, grad_user, nullptr, gather_fn, gather_user, stream, stats);
+  const zero_status st = run_step(c, grad_fn, grad_user, nullptr, gather_fn, gather_user, stream, stats);
+  int64_t g[3];
+  return st == ZERO_OK && c->guard == 2 ? check_guards(c, static_cast<cudaStream_t>(stream), g) : st;
 }
 
 zero_status zero_step_resident(zero_ctx* c, const void* const* rank_grads, zero_gather_fn gather_fn,
                                void* gather_user, void* stream, zero_step_stats* stats) {
   if (!c) return ZERO_EINVAL;
   if (!rank_grads) return fail(c, ZERO_EINVAL, "rank_grads is NULL");
-  return run_step(c, nullptr, nullptr, rank_grads, gather_fn, gather_user, stream, stats);
+  const zero_status st = run_step(c, nullptr, nullptr, rank_grads, gather_fn, gather_user, stream, stats);
+  int64_t g[3];
+  return st == ZERO_OK && c->guard == 2 ? check_guards(c, static_cast<cudaStream_t>(stream), g) : st;
+}
+
+zero_status zero_check_guards(zero_ctx* c, void* stream, int64_t out[3]) {
+  if (!c) return ZERO_EINVAL;
+  int64_t local[3];
+  if (!out) out = local;
+  out[0] = 0;
+  out[1] = out[2] = -1;
+  if (!c->guard) return fail(c, ZERO_ESTATE, "the arenas have no guard bytes (ZERO_OPT_GUARD before zero_bind)");
+  if (!c->bound || !c->loaded)
+    return fail(c, ZERO_ESTATE, "the guard bytes are armed by zero_load_master / zero_import_state");
+  return check_guards(c, static_cast<cudaStream_t>(stream), out);
 }
 
 zero_status zero_kernel_timing(zero_ctx* c, double* ms, int64_t* launches, double* model_bytes) {
