@@ -269,6 +269,75 @@ def test_probe_pattern_refuses_a_configuration_that_is_not_built():
     opt.close()
 
 
+# stage-3 layer lengths in flat order (the schedule runs from the last
+# layer to the first), chosen for what the launches leave in the shared layer
+# buffers: only the last launch ("last-longest"); the longest layer
+# mid-schedule leaves its tail, the launches before it nothing ("mixed");
+# every launch leaves a part ("falling")
+UNEQUAL_LAYERS = {
+    "last-longest": [3_000_000, 1_000_000, 2_000_000, 500_000],
+    "mixed": [1_000_000, 3_000_000, 500_000, 2_000_000],
+    "falling": [300_008, 700_000, 1_500_000, 2_500_000],
+}
+_UNEQUAL_REF = {}
+
+
+@pytest.mark.parametrize("layout", list(UNEQUAL_LAYERS))
+@pytest.mark.parametrize("kernel", [1, 2, 3])
+def test_zero3_chained_launches_leave_each_buffer_byte_of_its_last_writer(layout, kernel):
+    """Chained stage-3 launches of unequal layers into the one set of shared
+    layer buffers.  Every byte of every rank's buffer after the step must
+    hold the parameter of the layer scheduled last among those that write it
+    (the serialised step's result), with programmatic launches and with plain
+    ones, in every kernel family, against the oracle."""
+    z = _z()
+    sizes = UNEQUAL_LAYERS[layout]
+    numel, layer = list(sizes), list(range(len(sizes)))
+    n_ranks = 8
+    w = _workload(numel, layer, n_ranks, 3, 1 << 30, steps=2)
+    if layout not in _UNEQUAL_REF:  # one oracle run per layout, shared by the kernels
+        _UNEQUAL_REF[layout] = _oracle(w, 3, 1 << 30)[3]
+    ref = _UNEQUAL_REF[layout]
+    s = torch.cuda.current_stream().cuda_stream
+    opts = []
+    for pdl in (True, False):
+        opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, 3, bucket_elems=1 << 30,
+                              hparams=z.AdamHParams(**w.hyper.__dict__), kernel=kernel)
+        fill = DeviceFill(w, opt.offsets(), opt.psi_pad)
+        mv = opt.view(z.ZERO_VIEW_MASTER)
+        fill.master_into(mv.data_ptr(), mv, s)
+        opt.load_master(None)
+        opt.set_pdl(pdl)
+        opts.append((opt, fill))
+    for t in range(1, w.steps + 1):
+        for opt, fill in opts:
+            reps_t = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+            for r in range(n_ranks):
+                fill.grads_into(t, r, 0, opt.psi_pad, reps_t[r].data_ptr(), reps_t[r], s)
+            opt.step_resident(list(reps_t))
+        torch.cuda.synchronize()
+    (a, _), (b, _) = opts
+    layers = a.layers()
+    width = max(hi - lo for _, lo, hi in layers)
+    # the byte each position ends with: the last launch of the schedule (the
+    # first layer in flat order) long enough to write it
+    want = np.zeros(width, dtype=ref["params"].dtype)
+    done = np.zeros(width, dtype=bool)
+    for _, lo, hi in layers:  # flat order = the schedule's last launch first
+        fresh = ~done[: hi - lo]
+        want[: hi - lo][fresh] = ref["params"][lo:hi][fresh]
+        done[: hi - lo] = True
+    assert done.all()
+    for key, view in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(a.view(view)), ref[key], f"{layout} kernel {kernel} {key}")
+    assert_bits_equal(to_np(a.view(z.ZERO_VIEW_PARAM)), ref["params"], f"{layout} param shards")
+    for r in range(n_ranks):
+        for opt, tag in ((a, "chained"), (b, "plain")):
+            assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GATHER, r))[:width], want, f"{layout} {tag} buffer {r}")
+    a.close()
+    b.close()
+
+
 @pytest.mark.parametrize("n_ranks", [4, 8])
 def test_zero3_chained_layers_order_their_shared_buffer_stores(n_ranks):
     """ZeRO-3 resident steps with chained launches.  Every layer writes the
