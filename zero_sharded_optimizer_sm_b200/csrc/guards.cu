@@ -9,7 +9,7 @@
 // the first of them, and writes the value back.
 #include <cuda_runtime.h>
 
-#include "kernels.cuh"
+#include "guards.cuh"
 
 namespace zsm {
 namespace {

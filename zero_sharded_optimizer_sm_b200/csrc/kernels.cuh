@@ -227,24 +227,6 @@ cudaError_t launch_step_begin(StepState* state, const StepHparams& hp, ClipDecis
 cudaError_t launch_step_commit(StepState* state, cudaStream_t s);
 cudaError_t launch_init(const InitArgs& a, int grid, cudaStream_t s);
 
-// Guard bytes (guards.cu): per arena, `rows` rows of `pitch` bytes from
-// `base` whose bytes [used, pitch) are guards, then `tail` guard bytes after
-// the last row (rows = tail = 0: no arena).  The check counts the guard
-// bytes that differ from kGuardByte into result[0], the least
-// (arena << 56 | byte offset) of them into result[1] (the caller sets 0 and
-// ~0 first), and restores them.
-constexpr int kGuardSets = 6;
-constexpr unsigned char kGuardByte = 0xA5;
-struct GuardSet {
-  unsigned char* base;
-  long long pitch, used, rows, tail;
-};
-struct GuardArgs {
-  GuardSet set[kGuardSets];
-  unsigned long long* result;
-};
-cudaError_t launch_guards(const GuardArgs& a, bool check, cudaStream_t s);
-
 // Shared-memory staged fused kernel (fused_tma.cu): one CTA per SM with
 // `groups` (1 or 2) producer/consumer groups.
 cudaError_t launch_fused_tma(int mode, const FusedArgs& a, int grid, int groups, int max_stages,
@@ -285,14 +267,5 @@ cudaError_t two_pass_configure();
 cudaError_t launch_reduce_tma(const ReduceArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_adam_bcast_tma(const AdamBcastArgs& a, int grid, bool uniform, cudaStream_t s);
 int64_t two_pass_tile();
-// Pass 2 with bulk stores (two_pass_tma.cu): 1024-element tiles, eight
-// consumer warps, a ring of `stages` (2..8, fitted to shared memory); the
-// stores carry the L2 evict-first hint when `store_hint`.
-cudaError_t launch_adam_bcast_bulk(const AdamBcastArgs& a, int grid, bool uniform, int stages, int store_hint,
-                                   cudaStream_t s);
-int64_t bulk_bcast_tile();
-// Pass 1 with bulk stores (two_pass_tma.cu), N <= 16: 1024-element tiles,
-// eight consumer warps, a ring of `stages` (fitted to shared memory).
-cudaError_t launch_reduce_bulk(const ReduceArgs& a, int grid, int stages, int store_hint, cudaStream_t s);
 
 }  // namespace zsm

@@ -27,6 +27,7 @@
 
 #include "device_math.cuh"
 #include "kernels.cuh"
+#include "two_pass_bulk.cuh"
 #include "tma_pipe.cuh"
 
 namespace zsm {

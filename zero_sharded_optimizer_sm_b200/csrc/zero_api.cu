@@ -21,7 +21,9 @@
 #include <vector>
 
 #include "zero_sm.h"
+#include "guards.cuh"
 #include "kernels.cuh"
+#include "two_pass_bulk.cuh"
 #include "plan.hpp"
 
 static_assert(ZERO_MAX_RANKS == zsm::kMaxRanks, "rank limit mismatch");
