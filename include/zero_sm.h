@@ -195,6 +195,20 @@ enum {
                                     parameters and states of a step that ran out are partly
                                     updated: restore them (zero_import_state) before going on.
                                     May be set at any time */
+  ZERO_OPT_LAYERED = 19,         /* 1 (default): a stage-3 step without callbacks
+                                    (zero_step_resident with no gather_fn) on the bulk-store
+                                    kernel at N <= 16, with 2..64 non-empty layers, runs as
+                                    one cooperative launch.  Its CTAs take the layers in the
+                                    schedule's order (last to first), their shared-memory
+                                    rings running on across the layer boundaries.  A layer's
+                                    stores into the temporary layer buffers go out only after
+                                    every CTA has finished storing the layers before it -- the
+                                    order of one launch per layer, without a launch boundary at
+                                    each layer.  The gradient norm is summed over the whole
+                                    step at once (the same value up to rounding order, the same
+                                    bits run to run).  0: one launch per layer.  The movement-
+                                    only pass (zero_probe_pattern) follows the same choice.
+                                    May be set at any time */
   ZERO_OPT_NVTX = 18,            /* 1: NVTX ranges on the domain "zero_sm" around the host side
                                     of each step ("step t (stage s, N = n)"), of each of its
                                     launches ("bucket k [lo, hi)", "layer id [lo, hi)"; a

@@ -283,13 +283,15 @@ _UNEQUAL_REF = {}
 
 
 @pytest.mark.parametrize("layout", list(UNEQUAL_LAYERS))
-@pytest.mark.parametrize("kernel", [1, 2, 3])
-def test_zero3_chained_launches_leave_each_buffer_byte_of_its_last_writer(layout, kernel):
-    """Chained stage-3 launches of unequal layers into the one set of shared
-    layer buffers.  Every byte of every rank's buffer after the step must
-    hold the parameter of the layer scheduled last among those that write it
-    (the serialised step's result), with programmatic launches and with plain
-    ones, in every kernel family, against the oracle."""
+@pytest.mark.parametrize("kernel,layered", [(1, False), (2, False), (3, False), (3, True)])
+def test_zero3_chained_launches_leave_each_buffer_byte_of_its_last_writer(layout, kernel, layered):
+    """Stage-3 steps of unequal layers into the one set of shared layer
+    buffers: chained launches (programmatic and plain) in every kernel
+    family, and the bulk-store kernel's single layered launch (every layer in
+    one cooperative launch, each layer's buffer stores after every CTA's
+    stores of the layers before).  Every byte of every rank's buffer after
+    the step must hold the parameter of the layer scheduled last among those
+    that write it (the serialised step's result), against the oracle."""
     z = _z()
     sizes = UNEQUAL_LAYERS[layout]
     numel, layer = list(sizes), list(range(len(sizes)))
@@ -308,14 +310,20 @@ def test_zero3_chained_launches_leave_each_buffer_byte_of_its_last_writer(layout
         fill.master_into(mv.data_ptr(), mv, s)
         opt.load_master(None)
         opt.set_pdl(pdl)
+        opt.set_layered(layered)
         opts.append((opt, fill))
+    launches = []
     for t in range(1, w.steps + 1):
         for opt, fill in opts:
             reps_t = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
             for r in range(n_ranks):
                 fill.grads_into(t, r, 0, opt.psi_pad, reps_t[r].data_ptr(), reps_t[r], s)
+            before = opt.launch_count()
             opt.step_resident(list(reps_t))
+            launches.append(opt.launch_count() - before)
         torch.cuda.synchronize()
+    # begin + commit around the fused launches: one when layered, one per layer otherwise
+    assert set(launches) == {2 + (1 if layered else len(sizes))}, launches
     (a, _), (b, _) = opts
     layers = a.layers()
     width = max(hi - lo for _, lo, hi in layers)

@@ -105,3 +105,63 @@ def test_expired_ring_wait_reports_and_the_context_recovers(family, stage):
         assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM)), ref["params"], f"{family} param shards")
     opt.close()
     assert np.isfinite(reps[1].grad_norm)
+
+
+@pytest.mark.parametrize("n_ranks", [4, 8])
+def test_layered_launch_wait_runs_out_and_the_context_recovers(n_ranks):
+    """The stage-3 step as one layered launch (resident gradients, no
+    callbacks): with ZERO_OPT_WAIT_LIMIT_NS = 0 a ring wait or a storer's
+    wait for the other CTAs' layer stores runs out.  The CTA aborts, still
+    arrives for the layers it has left (so the other CTAs' waits end), and
+    the next synchronising call returns ZERO_ECUDA.  After the state is
+    restored, the next step equals the oracle bit for bit, layer buffers
+    included."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    numel, layer = W.transformer_layers(3, 128, 512)
+    w = W.Workload("failure-layered", numel, layer, n_ranks, (3,), 65536, synth.Dist(synth.NORMAL, 1e-2, zero_mod=17),
+                   W.MASTER_DIST, 2, W.Hyper(weight_decay=0.01), 0xFB0 + n_ranks)
+    p = oracle.plan(w.numel, w.layer_id, n_ranks, 65536)
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def g(t, r):
+        return W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), w.grad_dist)
+
+    ranks, reps = oracle.run(p, oracle.STAGE_Z3, m0, g, 2, oracle.AdamHP(**w.hyper.__dict__))
+    ref = oracle.full_view(p, oracle.STAGE_Z3, ranks)
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, 3, bucket_elems=65536,
+                          hparams=z.AdamHParams(**w.hyper.__dict__), kernel=BULK)
+    fill = DeviceFill(w, opt.offsets(), opt.psi_pad)
+    mv = opt.view(z.ZERO_VIEW_MASTER)
+    s = torch.cuda.current_stream().cuda_stream
+    fill.master_into(mv.data_ptr(), mv, s)
+    opt.load_master(None)
+
+    def grads(t):
+        rp = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+        for r in range(n_ranks):
+            fill.grads_into(t, r, 0, opt.psi_pad, rp[r].data_ptr(), rp[r], s)
+        return list(rp)
+
+    before = opt.launch_count()
+    assert opt.step_resident(grads(1), stats=True)["step"] == 1
+    assert opt.launch_count() - before == 3  # step begin, one layered launch, step commit
+    saved = opt.export_state()
+    g2 = grads(2)
+    opt.set_wait_limit(0)
+    with pytest.raises(z.ZeroError) as err:
+        opt.step_resident(g2, stats=True)
+    assert err.value.status == z.ZERO_ECUDA and "bounded wait" in str(err.value)
+    opt.set_wait_limit(2_000_000_000)
+    opt.read_stats()
+    opt.import_state(saved)
+    st = opt.step_resident(g2, stats=True)
+    assert st["step"] == 2 and st["nonfinite"] == reps[1].nonfinite
+    for k, view in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(opt.view(view)), ref[k], f"layered N={n_ranks} {k} after recovery")
+    assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM)), ref["params"], "layered param shards")
+    _, lo0, hi0 = opt.layers()[0]
+    for r in range(n_ranks):
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GATHER, r))[: hi0 - lo0], ref["params"][lo0:hi0],
+                          f"layered last gathered layer, rank {r}")
+    opt.close()

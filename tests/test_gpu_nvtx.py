@@ -4,7 +4,8 @@ child process runs steps with the ranges on and off, and the recorded
 domain "zero_sm" holds, in order, one range per step with one nested range
 per launch naming its bucket or layer and its [lo, hi) -- the intervals of
 the step's schedule --, the clipped step's reduce / decision / update
-ranges, a range per unfused call, and nothing while the option is off."""
+ranges, the stage-3 step's single range when its layers run as one launch,
+a range per unfused call, and nothing while the option is off."""
 import json
 import os
 import subprocess
@@ -35,11 +36,15 @@ for stage in (2, 3):
     opt.load_master(torch.randn(opt.psi_pad, device="cuda", generator=g) * 0.1)
     reps = (torch.randn(N, opt.psi_pad, device="cuda", generator=g) * 1e-2).to(torch.bfloat16).view(torch.int16)
     rl = list(reps)
+    opt.set_layered(False)
     opt.set_nvtx(True)
     opt.step_resident(rl)
     opt.set_clip(1e-3, True)
     opt.step_resident(rl)
     opt.set_clip(0.0, False)
+    if stage == 3:
+        opt.set_layered(True)
+        opt.step_resident(rl)
     lo, hi = (opt.buckets()[0] if stage == 2 else opt.layers()[-1][1:])
     opt.reduce_scatter(lo, hi, [int(t.data_ptr()) + 2 * lo for t in rl])
     opt.adam_shard(-1, 3)
@@ -74,6 +79,11 @@ def _expected(stage, info):
         for kind, k, lo, hi in sched:
             lines += [f"push zero_sm update layer {k} [{lo}, {hi})", "pop zero_sm"]
     lines.append("pop zero_sm")
+    if stage == 3:  # the stage-3 step as one layered launch
+        layers = info["layers"]
+        lines += [f"push zero_sm step 3 (stage 3, N = 4)",
+                  f"push zero_sm layers x {len(layers)} [{layers[0][1]}, {layers[-1][2]}) in one launch",
+                  "pop zero_sm", "pop zero_sm"]
     lo, hi = info["unfused"]
     lines += [f"push zero_sm reduce-scatter [{lo}, {hi})", "pop zero_sm", "push zero_sm adam shard -1", "pop zero_sm",
               f"push zero_sm all-gather [{lo}, {hi})", "pop zero_sm"]

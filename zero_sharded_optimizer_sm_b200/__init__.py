@@ -52,6 +52,7 @@ ZERO_OPT_WAIT_LIMIT_NS = 15
 ZERO_OPT_STORE_HINT = 16
 ZERO_OPT_GUARD = 17
 ZERO_OPT_NVTX = 18
+ZERO_OPT_LAYERED = 19
 ZERO_DTYPE_BF16, ZERO_DTYPE_F16 = 0, 1
 (ZERO_VIEW_MASTER, ZERO_VIEW_EXP_AVG, ZERO_VIEW_EXP_AVG_SQ, ZERO_VIEW_PARAM, ZERO_VIEW_GRAD_SHARD,
  ZERO_VIEW_GRAD_BUF, ZERO_VIEW_GATHER) = range(7)
@@ -578,6 +579,10 @@ class ZeroOptimizer:
         if st == ZERO_EGUARD:
             res["message"] = zero_last_error(self.ctx).decode()
         return res
+
+    def set_layered(self, on: bool):
+        """A callback-free stage-3 step as one launch over its layers (ZERO_OPT_LAYERED, default on)."""
+        self._check(zero_set_option(self.ctx, ZERO_OPT_LAYERED, 1 if on else 0), "zero_set_option")
 
     def set_nvtx(self, on: bool):
         """NVTX ranges per step, launch and unfused call on the domain "zero_sm" (ZERO_OPT_NVTX)."""

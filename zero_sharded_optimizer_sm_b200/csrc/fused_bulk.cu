@@ -43,6 +43,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "device_math.cuh"
 #include "kernels.cuh"
@@ -143,9 +144,81 @@ __host__ __device__ inline size_t bulk_smem_bytes(int n_ranks, int tile, bool ne
          4 * (size_t)(stages + 1);
 }
 
-template <int MODE, class F, int T, int W, bool kMove>
+// ------------------------------------------------------------ tile walk --
+//
+// A CTA's tiles in launch order.  One interval: tiles blockIdx.x,
+// blockIdx.x + G, ... of [0, n_elem).  Layered (a stage-3 step's layers in one
+// launch): the same walk through each segment in turn.  e_src is the tile's
+// flat start (gradients, states, shards), e_dst its offset in the N
+// destination buffers (the same for one interval; from the layer's start for
+// a segment).
+struct TileCursor {
+  int seg = 0;      // segment of the current tile
+  long long t = -1; // tile index inside the segment (-1: before the first)
+};
+
+template <int T, bool kLayered>
+__device__ __forceinline__ bool cursor_next(TileCursor& c, const SegTable& g, long long n_tiles, long long n_elem,
+                                            long long& e_src, long long& e_dst, unsigned& cnt) {
+  c.t = c.t < 0 ? (long long)blockIdx.x : c.t + gridDim.x;
+  long long rest;
+  if constexpr (kLayered) {
+    while (c.seg < g.n && c.t * T >= g.len[c.seg]) {
+      ++c.seg;
+      c.t = blockIdx.x;
+    }
+    if (c.seg >= g.n) return false;
+    e_dst = c.t * T;
+    e_src = g.lo[c.seg] + e_dst;
+    rest = g.len[c.seg] - e_dst;
+  } else {
+    if (c.t >= n_tiles) return false;
+    e_dst = e_src = c.t * T;
+    rest = n_elem - e_src;
+  }
+  cnt = (unsigned)(rest < T ? rest : T);
+  return true;
+}
+
+// The layered storers' ordering: a storer that has finished a segment's
+// stores waits until their global writes are performed, orders them before
+// its generic release (proxy fence) and arrives on the counter; a storer
+// about to store segment k waits until all G CTAs have arrived k times and
+// orders its bulk stores after that acquire.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+__device__ __forceinline__ void segment_arrive(unsigned* counter) {
+  bulk_wait<0>();
+  fence_proxy_async_global();
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded like the ring waits (limit 0: one test); false when it ran out or
+// the CTA aborted.
+__device__ __forceinline__ bool segment_wait(const unsigned* counter, unsigned target, volatile int* abort_flag,
+                                             unsigned long long limit) {
+  bool ok = ld_acquire_gpu(counter) >= target;
+  if (!ok && limit > 0) {
+    const unsigned long long t0 = now_ns();
+    while (!(ok = ld_acquire_gpu(counter) >= target)) {
+      if (*abort_flag || now_ns() - t0 > limit) break;
+      __nanosleep(32);
+    }
+  }
+  if (ok) fence_proxy_async_global();
+  return ok;
+}
+
+template <int MODE, class F, int T, int W, bool kMove, bool kLayered>
 __global__ void __launch_bounds__(32 * (W + 2), 1)
-    fused_bulk_kernel(const __grid_constant__ FusedArgs a, int stages, uint32_t opaque) {
+    fused_bulk_kernel(const __grid_constant__ FusedArgs a, int stages, uint32_t opaque,
+                      const __grid_constant__ SegTable g) {
   constexpr int EPT = T / (32 * W);
   static_assert(EPT == 2 || EPT == 4 || EPT == 8, "2, 4 or 8 elements per consumer lane");
   constexpr int NT = 32 * (W + 2);
@@ -185,9 +258,11 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       const uint64_t policy = evict_first_policy();
+      TileCursor cur;
       for (int it = 0;; ++it) {
-        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
-        if (tile >= n_tiles || *abort_flag) break;
+        long long e0, ed;
+        unsigned cnt;
+        if (!cursor_next<T, kLayered>(cur, g, n_tiles, n_elem, e0, ed, cnt) || *abort_flag) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
         if (k > 0) {
@@ -199,10 +274,8 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
           }
         }
         fence_proxy_async_smem();  // the stage's last reads (consumers, stores) before the refill
-        const int64_t e0 = tile * T;
-        const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
         unsigned char* st = smem + (size_t)s * sb;
-        mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
+        mbar_expect_tx(&full[s], cnt * (unsigned)(2 * N + 12));
         for (int r = 0; r < N; ++r)
           bulk_load(st + (size_t)r * 2 * T, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
         bulk_load(st + off_state, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
@@ -222,9 +295,12 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
         if (hint) bulk_store(dst, src, bytes, spol);
         else bulk_store(dst, src, bytes);
       };
+      TileCursor cur;
+      int arrived = 0;  // layered: segments this storer has finished and arrived for
       for (int it = 0;; ++it) {
-        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
-        if (tile >= n_tiles) break;
+        long long e0, ed;
+        unsigned cnt;
+        if (!cursor_next<T, kLayered>(cur, g, n_tiles, n_elem, e0, ed, cnt)) break;
         const int s = it % stages;
         const unsigned k = (unsigned)(it / stages);
         const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag, a.ns.wait_ns);
@@ -237,14 +313,26 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
           pdl_wait();
           waited = true;
         }
-        const int64_t e0 = tile * T;
-        const unsigned cnt = (unsigned)((n_elem - e0) < T ? (n_elem - e0) : T);
+        if constexpr (kLayered) {
+          // a new layer: every CTA's stores of the layers before it first
+          if (cur.seg > arrived) {
+            while (arrived < cur.seg) {
+              segment_arrive(g.counter);
+              ++arrived;
+            }
+            if (!segment_wait(g.counter, gridDim.x * (unsigned)cur.seg, abort_flag, a.ns.wait_ns)) {
+              atomicOr(a.ns.error, 16u);
+              *abort_flag = 1;
+              break;
+            }
+          }
+        }
         const unsigned char* st = smem + (size_t)s * sb;
         put(a.master + e0, st + off_state, 4 * cnt);
         put(a.m + e0, st + off_state + 4 * T, 4 * cnt);
         put(a.v + e0, st + off_state + 8 * T, 4 * cnt);
         if (MODE == kFusedZ3) put(a.param_shard + e0, st, 2 * cnt);
-        for (int r = 0; r < N; ++r) put(a.out[r] + e0, st, 2 * cnt);
+        for (int r = 0; r < N; ++r) put(a.out[r] + ed, st, 2 * cnt);
         if (MODE == kFusedZ1)
           for (int r = 0; r < N; ++r) put(const_cast<uint16_t*>(a.grad[r]) + e0, st + off_g, 2 * cnt);
         if (a.grad_shard) put(a.grad_shard + e0, st + off_g, 2 * cnt);
@@ -252,15 +340,22 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
         bulk_wait_read<0>();  // the copies have read the stage: hand it back to the producer
         mbar_arrive(&empty[s]);
       }
+      if constexpr (kLayered) {
+        // arrive for the layers left (also after an abort: the other CTAs
+        // then end without waiting out their limit; the step has failed)
+        for (; arrived < g.n; ++arrived) segment_arrive(g.counter);
+      }
       bulk_wait<0>();  // every store of this CTA performed before the CTA ends
     }
   } else {
     // ----------------------------------------------------------- consumers --
     const int c = threadIdx.x - 64;  // 0 .. 32W-1
     const int j = c * EPT;
+    TileCursor cur;
     for (int it = 0;; ++it) {
-      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
-      if (tile >= n_tiles) break;
+      long long e0, ed;
+      unsigned cnt;
+      if (!cursor_next<T, kLayered>(cur, g, n_tiles, n_elem, e0, ed, cnt)) break;
       const int s = it % stages;
       const unsigned k = (unsigned)(it / stages);
       // warp-uniform decisions, so that no lane is left waiting at __syncwarp
@@ -271,10 +366,8 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
         break;
       }
       if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
-      const int64_t e0 = tile * T;
-      const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
       unsigned char* st = smem + (size_t)s * sb;
-      if (j < cnt) {  // cnt is a multiple of 8, so a lane's EPT elements are whole
+      if (j < (int)cnt) {  // cnt is a multiple of 8, so a lane's EPT elements are whole
         V32<EPT> p = ldsf<EPT>(st + off_state + 4 * j);
         V32<EPT> m = ldsf<EPT>(st + off_state + 4 * T + 4 * j);
         V32<EPT> v = ldsf<EPT>(st + off_state + 8 * T + 4 * j);
@@ -629,8 +722,28 @@ template <int MODE, class F, int T, int W, bool kMove>
 cudaError_t launch_cfg(const FusedArgs& a, int grid, int stages, int sstages, size_t bytes, uint32_t opaque,
                        cudaStream_t s) {
   (void)sstages;
-  return launch_kernel(fused_bulk_kernel<MODE, F, T, W, kMove>, grid, 32 * (W + 2), bytes, s, a.pdl != kPdlNone,
-                       a, stages, opaque);
+  SegTable none;
+  std::memset(&none, 0, sizeof none);
+  return launch_kernel(fused_bulk_kernel<MODE, F, T, W, kMove, false>, grid, 32 * (W + 2), bytes, s,
+                       a.pdl != kPdlNone, a, stages, opaque, none);
+}
+
+// The layered stage-3 launch: cooperative, so that every CTA is resident at
+// once (its storers wait on one another's progress), and one CTA per SM.
+template <class F, int T, int W, bool kMove>
+cudaError_t launch_layered_cfg(const FusedArgs& a, const SegTable& g, int grid, int stages, size_t bytes,
+                               cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)(32 * (W + 2)));
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fused_bulk_kernel<kFusedZ3, F, T, W, kMove, true>, a, stages, 0u, g);
 }
 
 template <int MODE, class F, int T, int W, bool kMove>
@@ -681,8 +794,9 @@ cudaError_t opt_in(K kernel) {
 template <int MODE, class F, bool kMove>
 cudaError_t configure_mode_fmt() {
   cudaError_t e = cudaSuccess;
-#define ZSM_BULK_OPT(TT, WW) \
-  if (e == cudaSuccess) e = opt_in(fused_bulk_kernel<MODE, F, TT, WW, kMove>);
+#define ZSM_BULK_OPT(TT, WW)                                                                   \
+  if (e == cudaSuccess) e = opt_in(fused_bulk_kernel<MODE, F, TT, WW, kMove, false>);          \
+  if (MODE == kFusedZ3 && e == cudaSuccess) e = opt_in(fused_bulk_kernel<kFusedZ3, F, TT, WW, kMove, true>);
   ZSM_BULK_CONFIGS(ZSM_BULK_OPT)
 #undef ZSM_BULK_OPT
 #define ZSM_BULK_OPT(TT, WW) \
@@ -769,6 +883,27 @@ cudaError_t launch_fused_bulk(int mode, const FusedArgs& a, int grid, int tile, 
     case kFusedZ3: return launch_mode<kFusedZ3>(a, grid, tile, warps, stages, sstages, bytes, move, opaque, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_fused_bulk_layered(const FusedArgs& a, const SegTable& g, int grid, int tile, int warps,
+                                      int max_stages, bool move, cudaStream_t s) {
+  if (a.n_ranks < 1 || a.n_ranks > kTmaMaxRanks || g.n < 1 || g.n > kMaxSegments || !g.counter ||
+      a.pdl != kPdlNone)
+    return cudaErrorInvalidValue;
+  const bool need_g = a.grad_shard != nullptr;
+  const int stages = bulk_stages_for(a.n_ranks, tile, need_g, max_stages);
+  if (stages == 0) return cudaErrorInvalidValue;
+  size_t bytes = bulk_smem_bytes(a.n_ranks, tile, need_g, stages);
+  if (bytes < kPdlSoloSmemBulk) bytes = kPdlSoloSmemBulk;  // one CTA per SM: tiles are dealt by CTA index
+#define ZSM_BULK_CASE(TT, WW)                                                                   \
+  if (tile == TT && warps == WW) {                                                              \
+    if (move) return launch_layered_cfg<Bf16, TT, WW, true>(a, g, grid, stages, bytes, s);      \
+    if (a.fmt == kFmtF16) return launch_layered_cfg<F16, TT, WW, false>(a, g, grid, stages, bytes, s); \
+    return launch_layered_cfg<Bf16, TT, WW, false>(a, g, grid, stages, bytes, s);               \
+  }
+  ZSM_BULK_CONFIGS(ZSM_BULK_CASE)
+#undef ZSM_BULK_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace zsm

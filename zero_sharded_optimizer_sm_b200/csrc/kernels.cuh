@@ -237,6 +237,20 @@ int tma_stages_for(int n_ranks, int groups, int max_stages = 0);
 // replicas stream in chunks of 8 ranks through a `cstages`-deep ring.
 cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cstages, cudaStream_t s);
 
+// A stage-3 step's layers as one launch of the bulk-store kernel
+// (launch_fused_bulk_layered): segment k is one layer's flat range
+// [lo[k], lo[k] + len[k]), in the schedule's order, whose parameters go to
+// the temporary layer buffers from their start.  `counter` (zero before the
+// launch) counts the storers' arrivals: one per CTA for each segment whose
+// stores it has finished.
+constexpr int kMaxSegments = 64;
+struct SegTable {
+  int n;
+  unsigned* counter;
+  long long lo[kMaxSegments];
+  long long len[kMaxSegments];
+};
+
 // Staged kernel with bulk stores (fused_bulk.cu): tiles of `tile` elements,
 // `warps` consumer warps, a ring of at most `max_stages` stages (0 = the
 // default depth); above N = 16 the rank-chunked form (max_stages bounds its
@@ -245,6 +259,14 @@ cudaError_t launch_fused_chunked(int mode, const FusedArgs& a, int grid, int cst
 // ceiling and is never part of a step.
 cudaError_t launch_fused_bulk(int mode, const FusedArgs& a, int grid, int tile, int warps, int max_stages, bool move,
                               uint32_t opaque, cudaStream_t s);
+// Stage 3, N <= 16: every segment of `g` in one cooperative launch of that
+// kernel (`a`'s pointers at flat element 0, its layer-buffer pointers at the
+// buffers' start, no programmatic launch).  Each CTA walks its tiles layer
+// after layer with its ring running on across the boundaries; its storer
+// issues a layer's stores only after every CTA has finished storing the
+// layers before (g.counter).
+cudaError_t launch_fused_bulk_layered(const FusedArgs& a, const SegTable& g, int grid, int tile, int warps,
+                                      int max_stages, bool move, cudaStream_t s);
 // Ring depth of that kernel for N, the tile and whether the averaged gradient
 // is stored (the chunk ring above N = 16; 0 when nothing fits); whether
 // (tile, warps) is a built configuration at that N.

@@ -43,6 +43,9 @@ constexpr int64_t kGuardResultOffset = 72 * 1024;
 static_assert(16 * zsm::kMaxGrid + 128 + sizeof(zsm::StepState) <= kGuardResultOffset &&
                   kGuardResultOffset + 16 <= kScratchBytes,
               "the guard check's result words follow the step state in the scratch arena");
+// The layered stage-3 launch's arrival counter, past the guard result.
+constexpr int64_t kSegCounterOffset = kGuardResultOffset + 64;
+static_assert(kSegCounterOffset + 4 <= kScratchBytes, "the layered launch's counter fits the scratch arena");
 
 int64_t align_up(int64_t x, int64_t m) { return ((x + m - 1) / m) * m; }
 
@@ -132,6 +135,7 @@ struct zero_ctx {
   // two CTAs on one SM); measured 0.5-2 % faster per step on B200.
   bool pdl = true;
   bool nvtx = false;  // ZERO_OPT_NVTX: ranges per step and per launch
+  bool layered = true;  // ZERO_OPT_LAYERED: a callback-free stage-3 step as one launch
   int guard = 0;  // ZERO_OPT_GUARD: 0, 1 (laid out, armed at load, checked on request) or 2 (checked after each step)
   int slots = 1;  // gradient / gather slot sets: 2 with the pipeline at stage 2/3
   cudaStream_t side = nullptr;   // the callbacks' stream
@@ -645,6 +649,77 @@ zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const*
   return ZERO_OK;
 }
 
+// A callback-free stage-3 step as one launch (ZERO_OPT_LAYERED): the
+// bulk-store kernel at N <= 16, at least two non-empty layers, at most
+// kMaxSegments, and one CTA per SM.
+bool layered_ok(const zero_ctx* c, bool callbacks, const std::vector<zsm::Span>& iv) {
+  if (!c->layered || callbacks || c->stage != ZERO_STAGE_3 || !use_bulk(c) || !bulk_fits(c) ||
+      c->plan.n_ranks > zsm::kTmaMaxRanks || c->tma_ctas_opt > 1)
+    return false;
+  int n = 0;
+  for (const zsm::Span& sp : iv) n += sp.hi > sp.lo ? 1 : 0;
+  return n >= 2 && n <= zsm::kMaxSegments;
+}
+
+// Every layer of the schedule in one cooperative launch of the bulk-store
+// kernel: the layers in schedule order (last to first), each CTA's ring
+// running on across layer boundaries, and each layer's stores into the
+// temporary layer buffers issued only after every CTA has finished storing
+// the layers before it -- the order of the per-layer launches, without a
+// launch boundary at each layer.  grad0[r] are the ranks' full replicas.
+zero_status fused_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, uint16_t* const* grad0, cudaStream_t s,
+                          const zsm::AdamScalars* sc_dev, bool twin) {
+  const int N = c->plan.n_ranks;
+  zsm::FusedArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.fmt = c->fmt;
+  for (int r = 0; r < N; ++r) {
+    a.grad[r] = grad0[r];
+    a.out[r] = gather_ptr(c, r, 0);
+  }
+  a.master = master_ptr(c);
+  a.m = m_ptr(c);
+  a.v = v_ptr(c);
+  a.grad_shard = c->arena[ZERO_ARENA_GRAD_SHARDS] ? grad_shard_ptr(c) : nullptr;
+  a.param_shard = param_ptr(c, 0);
+  a.n_vec = c->plan.psi_pad / zsm::kVec;
+  a.n_ranks = N;
+  a.accumulate = 0;
+  a.inv_n = (float)(1.0 / (double)N);
+  a.sc_dev = sc_dev;
+  a.ns = norm_scratch(c);
+  a.pdl = zsm::kPdlNone;
+  a.store_hint = c->store_hint >= 0 ? c->store_hint : bulk_policy(c->plan.n_ranks, c->stage).hint;
+  zsm::SegTable g;
+  std::memset(&g, 0, sizeof g);
+  g.counter = reinterpret_cast<unsigned*>(c->arena[ZERO_ARENA_SCRATCH] + kSegCounterOffset);
+  int64_t elems = 0, max_tiles = 1;
+  const int64_t tile = bulk_tile(c);
+  for (const zsm::Span& sp : iv) {
+    if (sp.hi == sp.lo) continue;
+    g.lo[g.n] = sp.lo;
+    g.len[g.n] = sp.hi - sp.lo;
+    ++g.n;
+    elems += sp.hi - sp.lo;
+    max_tiles = std::max(max_tiles, (sp.hi - sp.lo + tile - 1) / tile);
+  }
+  const NvtxRange range(c->nvtx, "layers x %d [%lld, %lld) in one launch", g.n, (long long)g.lo[g.n - 1],
+                        (long long)(g.lo[0] + g.len[0]));
+  cudaError_t e = cudaMemsetAsync(g.counter, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "clearing the layered launch's counter");
+  cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  e = counted(c, zsm::launch_fused_bulk_layered(a, g, (int)std::min<int64_t>(max_tiles, c->sm_count), (int)tile,
+                                                bulk_warps(c), bulk_ring(c), twin, s));
+  if (e != cudaSuccess) return cuda_fail(c, e, "layered fused step kernel launch");
+  if (ev) {
+    cudaEventRecord(ev[1], s);
+    c->timed += 1;
+    c->timed_bytes += (double)fused_bytes_per_elem(c) * (double)elems;
+  }
+  return ZERO_OK;
+}
+
 // Reads and clears the device error word (a bounded wait that ran out).
 zero_status check_device_error(zero_ctx* c, unsigned int err, cudaStream_t s) {
   if (err == 0) return ZERO_OK;
@@ -1078,7 +1153,12 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   // (and not with two staged CTAs per SM asked for: a programmatic launch
   // keeps one per SM)
   const bool pdl_ok = c->pdl && !callbacks && c->tma_ctas_opt <= 1;
-  for (size_t k = 0; k < iv.size() && st == ZERO_OK; ++k) {
+  const bool one_launch = layered_ok(c, callbacks, iv);  // every layer in one launch
+  if (one_launch) {
+    interval_grads(c, resident, 0, 0, grad.data());
+    st = fused_layered(c, iv, grad.data(), s, &state_ptr(c)->sc, false);
+  }
+  for (size_t k = 0; k < iv.size() && st == ZERO_OK && !one_launch; ++k) {
     for (; issued < iv.size() && issued <= k + o.ahead() && st == ZERO_OK; ++issued)
       st = issue_grads(c, o, fn, user, resident, iv, issued, t);
     if (st != ZERO_OK) break;
@@ -1193,6 +1273,10 @@ zero_status zero_set_option(zero_ctx* c, int32_t key, int64_t value) {
     if (value > 0 && zsm::tma_stages_for(c->plan.n_ranks, (int)value) == 0)
       return fail(c, ZERO_EINVAL, "%lld consumer groups do not fit at N = %d", (long long)value, c->plan.n_ranks);
     c->tma_groups_opt = (int)value;
+    return ZERO_OK;
+  }
+  if (key == ZERO_OPT_LAYERED) {
+    c->layered = value != 0;
     return ZERO_OK;
   }
   if (key == ZERO_OPT_NVTX) {
@@ -1829,6 +1913,13 @@ zero_status zero_probe_pattern(zero_ctx* c, const void* const* rank_grads, void*
   std::vector<uint16_t*> grad(N);
   const int n_layers = (int)c->plan.layers.size();
   const bool pdl_ok = c->pdl && c->tma_ctas_opt <= 1;
+  if (layered_ok(c, false, iv)) {  // the step's own form: every layer in one launch
+    interval_grads(c, rank_grads, 0, 0, grad.data());
+    st = fused_layered(c, iv, grad.data(), s, nullptr, true);
+    if (st != ZERO_OK) return st;
+    c->norm_fresh = true;
+    return ZERO_OK;
+  }
   bool launched = false;
   for (size_t k = 0; k < iv.size(); ++k) {
     const int64_t lo = iv[k].lo, hi = iv[k].hi;
