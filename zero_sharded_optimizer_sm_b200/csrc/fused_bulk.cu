@@ -43,7 +43,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <cstring>
 
 #include "device_math.cuh"
 #include "kernels.cuh"
@@ -215,10 +214,216 @@ __device__ __forceinline__ bool segment_wait(const unsigned* counter, unsigned t
   return ok;
 }
 
-template <int MODE, class F, int T, int W, bool kMove, bool kLayered>
+template <int MODE, class F, int T, int W, bool kMove>
 __global__ void __launch_bounds__(32 * (W + 2), 1)
-    fused_bulk_kernel(const __grid_constant__ FusedArgs a, int stages, uint32_t opaque,
-                      const __grid_constant__ SegTable g) {
+    fused_bulk_kernel(const __grid_constant__ FusedArgs a, int stages, uint32_t opaque) {
+  constexpr int EPT = T / (32 * W);
+  static_assert(EPT == 2 || EPT == 4 || EPT == 8, "2, 4 or 8 elements per consumer lane");
+  constexpr int NT = 32 * (W + 2);
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int N = a.n_ranks;
+  const bool need_g = MODE == kFusedZ1 || a.grad_shard != nullptr;
+  const unsigned sb = bulk_stage_bytes(N, T, need_g);
+  const unsigned off_state = 2u * (unsigned)N * T;  // master; m at +4T, v at +8T
+  const unsigned off_g = off_state + 12u * T;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * sb);
+  uint64_t* computed = full + stages;
+  uint64_t* empty = computed + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_k = abort_flag + 1;  // last phase of `full` issued per stage, -1 = none
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t n_elem = a.n_vec * kVec;
+  const int64_t n_tiles = (n_elem + T - 1) / T;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&computed[s], W);
+      mbar_init(&empty[s], 1);
+      last_k[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (a.pdl == kPdlWaitFirst) pdl_wait();
+
+  double sq = 0.0;
+  unsigned long long nf = 0;
+  const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles || *abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (k > 0) {
+          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag, a.ns.wait_ns);
+          if (w != 0) {
+            if (w == 1) atomicOr(a.ns.error, 1u);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        fence_proxy_async_smem();  // the stage's last reads (consumers, stores) before the refill
+        const int64_t e0 = tile * T;
+        const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+        unsigned char* st = smem + (size_t)s * sb;
+        mbar_expect_tx(&full[s], (unsigned)(cnt * (2 * N + 12)));
+        for (int r = 0; r < N; ++r)
+          bulk_load(st + (size_t)r * 2 * T, a.grad[r] + e0, (unsigned)(2 * cnt), &full[s], policy);
+        bulk_load(st + off_state, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + off_state + 4 * T, a.m + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + off_state + 8 * T, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
+        last_k[s] = (int)k;
+      }
+      pdl_trigger();  // no more loads to issue: the next fused launch may start
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- storer --
+    if (lane == 0) {
+      bool waited = false;
+      const uint64_t spol = evict_first_policy();
+      const bool hint = a.store_hint != 0;
+      auto put = [&](void* dst, const void* src, unsigned bytes) {
+        if (hint) bulk_store(dst, src, bytes, spol);
+        else bulk_store(dst, src, bytes);
+      };
+      for (int it = 0;; ++it) {
+        const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+        if (tile >= n_tiles) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag, a.ns.wait_ns);
+        if (w != 0) {
+          if (w == 1) atomicOr(a.ns.error, 8u);
+          *abort_flag = 1;
+          break;
+        }
+        if (a.pdl == kPdlEarlyLoads && !waited) {  // the first store waits for the grid before
+          pdl_wait();
+          waited = true;
+        }
+        const int64_t e0 = tile * T;
+        const unsigned cnt = (unsigned)((n_elem - e0) < T ? (n_elem - e0) : T);
+        const unsigned char* st = smem + (size_t)s * sb;
+        put(a.master + e0, st + off_state, 4 * cnt);
+        put(a.m + e0, st + off_state + 4 * T, 4 * cnt);
+        put(a.v + e0, st + off_state + 8 * T, 4 * cnt);
+        if (MODE == kFusedZ3) put(a.param_shard + e0, st, 2 * cnt);
+        for (int r = 0; r < N; ++r) put(a.out[r] + e0, st, 2 * cnt);
+        if (MODE == kFusedZ1)
+          for (int r = 0; r < N; ++r) put(const_cast<uint16_t*>(a.grad[r]) + e0, st + off_g, 2 * cnt);
+        if (a.grad_shard) put(a.grad_shard + e0, st + off_g, 2 * cnt);
+        bulk_commit();
+        bulk_wait_read<0>();  // the copies have read the stage: hand it back to the producer
+        mbar_arrive(&empty[s]);
+      }
+      bulk_wait<0>();  // every store of this CTA performed before the CTA ends
+    }
+  } else {
+    // ----------------------------------------------------------- consumers --
+    const int c = threadIdx.x - 64;  // 0 .. 32W-1
+    const int j = c * EPT;
+    for (int it = 0;; ++it) {
+      const int64_t tile = blockIdx.x + (int64_t)it * gridDim.x;
+      if (tile >= n_tiles) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      // warp-uniform decisions, so that no lane is left waiting at __syncwarp
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.ns.wait_ns));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.ns.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      const int64_t e0 = tile * T;
+      const int64_t cnt = (n_elem - e0) < T ? (n_elem - e0) : T;
+      unsigned char* st = smem + (size_t)s * sb;
+      if (j < cnt) {  // cnt is a multiple of 8, so a lane's EPT elements are whole
+        V32<EPT> p = ldsf<EPT>(st + off_state + 4 * j);
+        V32<EPT> m = ldsf<EPT>(st + off_state + 4 * T + 4 * j);
+        V32<EPT> v = ldsf<EPT>(st + off_state + 8 * T + 4 * j);
+        H16<EPT> par, gout;
+        if constexpr (kMove) {
+          // movement only: every slice read, nothing computed but a fold
+          uint32_t fold[EPT / 2];
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) fold[q] = 0u;
+          for (int r = 0; r < N; ++r) {
+            const H16<EPT> h = lds16<EPT>(st + (size_t)r * 2 * T + 2 * j);
+#pragma unroll
+            for (int q = 0; q < EPT / 2; ++q) fold[q] ^= h.w[q];
+          }
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) {
+            par.w[q] = pack2(F::rn(p.f[2 * q]), F::rn(p.f[2 * q + 1])) ^ (fold[q] & opaque);
+            gout.w[q] = fold[q];
+          }
+        } else {
+          float acc[EPT];
+#pragma unroll
+          for (int q = 0; q < EPT; ++q) acc[q] = 0.0f;
+          for (int r = 0; r < N; ++r) {
+            const H16<EPT> h = lds16<EPT>(st + (size_t)r * 2 * T + 2 * j);
+#pragma unroll
+            for (int q = 0; q < EPT / 2; ++q) {
+              acc[2 * q] = __fadd_rn(acc[2 * q], F::lo(h.w[q]));
+              acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], F::hi(h.w[q]));
+            }
+          }
+          uint16_t g16[EPT], p16[EPT];
+#pragma unroll
+          for (int q = 0; q < EPT; ++q) {
+            g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
+            const float g = F::f32(g16[q]);
+            const double d = (double)g;
+            sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
+            nf += isfinite(g) ? 0ull : 1ull;
+            p16[q] = F::rn(adam1(g, p.f[q], m.f[q], v.f[q], sc));
+          }
+#pragma unroll
+          for (int q = 0; q < EPT / 2; ++q) {
+            par.w[q] = pack2(p16[2 * q], p16[2 * q + 1]);
+            gout.w[q] = pack2(g16[2 * q], g16[2 * q + 1]);
+          }
+        }
+        stsf<EPT>(st + off_state + 4 * j, p);
+        stsf<EPT>(st + off_state + 4 * T + 4 * j, m);
+        stsf<EPT>(st + off_state + 8 * T + 4 * j, v);
+        sts16<EPT>(st + 2 * j, par);  // over rank 0's slice, which this lane alone read here
+        if (need_g) sts16<EPT>(st + off_g + 2 * j, gout);
+      }
+      fence_proxy_async_smem();  // this lane's stage writes before the storer's bulk copies read them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&computed[s]);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // drain the bulk loads already issued before the CTA's memory goes away
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
+  }
+  if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
+  norm_epilogue<NT>(a.ns, sq, nf, a.accumulate);
+}
+
+// The layered stage-3 launch: the kernel above with the tile walk through
+// the segments of `g` and the storers' ordering between segments.  A kernel
+// of its own: sharing the walk with the one-interval kernel (a template flag)
+// made that kernel's stage-1 and stage-2 launches 1.5-6 % slower on B200.
+template <class F, int T, int W, bool kMove>
+__global__ void __launch_bounds__(32 * (W + 2), 1)
+    fused_bulk_layered_kernel(const __grid_constant__ FusedArgs a, int stages, const __grid_constant__ SegTable g) {
+  constexpr int MODE = kFusedZ3;
+  constexpr bool kLayered = true;
+  constexpr uint32_t opaque = 0u;
   constexpr int EPT = T / (32 * W);
   static_assert(EPT == 2 || EPT == 4 || EPT == 8, "2, 4 or 8 elements per consumer lane");
   constexpr int NT = 32 * (W + 2);
@@ -722,10 +927,8 @@ template <int MODE, class F, int T, int W, bool kMove>
 cudaError_t launch_cfg(const FusedArgs& a, int grid, int stages, int sstages, size_t bytes, uint32_t opaque,
                        cudaStream_t s) {
   (void)sstages;
-  SegTable none;
-  std::memset(&none, 0, sizeof none);
-  return launch_kernel(fused_bulk_kernel<MODE, F, T, W, kMove, false>, grid, 32 * (W + 2), bytes, s,
-                       a.pdl != kPdlNone, a, stages, opaque, none);
+  return launch_kernel(fused_bulk_kernel<MODE, F, T, W, kMove>, grid, 32 * (W + 2), bytes, s, a.pdl != kPdlNone,
+                       a, stages, opaque);
 }
 
 // The layered stage-3 launch: cooperative, so that every CTA is resident at
@@ -743,7 +946,7 @@ cudaError_t launch_layered_cfg(const FusedArgs& a, const SegTable& g, int grid, 
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fused_bulk_kernel<kFusedZ3, F, T, W, kMove, true>, a, stages, 0u, g);
+  return cudaLaunchKernelEx(&cfg, fused_bulk_layered_kernel<F, T, W, kMove>, a, stages, g);
 }
 
 template <int MODE, class F, int T, int W, bool kMove>
@@ -794,9 +997,9 @@ cudaError_t opt_in(K kernel) {
 template <int MODE, class F, bool kMove>
 cudaError_t configure_mode_fmt() {
   cudaError_t e = cudaSuccess;
-#define ZSM_BULK_OPT(TT, WW)                                                                   \
-  if (e == cudaSuccess) e = opt_in(fused_bulk_kernel<MODE, F, TT, WW, kMove, false>);          \
-  if (MODE == kFusedZ3 && e == cudaSuccess) e = opt_in(fused_bulk_kernel<kFusedZ3, F, TT, WW, kMove, true>);
+#define ZSM_BULK_OPT(TT, WW)                                                          \
+  if (e == cudaSuccess) e = opt_in(fused_bulk_kernel<MODE, F, TT, WW, kMove>);        \
+  if (MODE == kFusedZ3 && e == cudaSuccess) e = opt_in(fused_bulk_layered_kernel<F, TT, WW, kMove>);
   ZSM_BULK_CONFIGS(ZSM_BULK_OPT)
 #undef ZSM_BULK_OPT
 #define ZSM_BULK_OPT(TT, WW) \
