@@ -68,6 +68,8 @@ def parse_args(argv=None):
     ap.add_argument("--ring", type=int, default=0, help="staged kernels: ring depth (0 = library's choice)")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch the step's fused kernels plainly (no programmatic dependent launch)")
+    ap.add_argument("--no-layered", action="store_true",
+                    help="stage 3: one launch per layer instead of the layered launch over all layers")
     ap.add_argument("--sweep", action="store_true",
                     help="flat-buffer sweep instead of the bench line: 1K..1G elements (x4) x N in "
                          "{2,4,8,16,64}, fused step vs unfused reduce-scatter + Adam + all-gather; one "
@@ -281,10 +283,13 @@ def workload():
     return WORKLOADS[_ARGS.workload if _ARGS is not None else "gpt-1.2b"]()
 
 
-def fused_kernel_name(fc: dict, n_ranks: int) -> str:
-    """The fused kernel a context launches, from its zero_fused_config."""
+def fused_kernel_name(fc: dict, n_ranks: int, layered: bool = False) -> str:
+    """The fused kernel a context launches, from its zero_fused_config
+    (layered: a callback-free stage-3 step as one launch over its layers)."""
     if fc["kernel"] == "bulk":
-        return "fused_bulk_kernel"
+        if n_ranks > 16:
+            return "fused_bulk_chunked_kernel"
+        return "fused_bulk_layered_kernel" if layered else "fused_bulk_kernel"
     if fc["kernel"] != "tma":
         return "fused_step_kernel"
     if n_ranks > 16:
@@ -436,6 +441,7 @@ def run_ours(args, world, rank, local):
             fill16(gb, off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
     rep_list = list(reps)
     opt.set_pdl(not args.no_pdl)
+    opt.set_layered(not args.no_layered)
     torch.cuda.synchronize(dev)
     # model bytes of one step's fused launches, from the library's own record
     opt.set_timing(True)
@@ -563,11 +569,13 @@ def run_ours(args, world, rank, local):
                    "l2": f"inputs larger than L2: {(4 * w.n_ranks + 24) * w.psi / 1e9:.1f} GB moved "
                          f"per step vs 126 MB L2",
                    "parallelism": f"{w.n_ranks} logical ranks per GPU x {world} GPU replicas",
-                   "kernel": args.kernel, "fused_config": fc, "pdl": not args.no_pdl},
+                   "kernel": args.kernel, "fused_config": fc, "pdl": not args.no_pdl,
+                   "layered": args.stage == 3 and not args.no_layered},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                      "peak_kind": f"{peak_kind} copy peak",
-                     "kernel": (fused_kernel_name(fc, w.n_ranks) if args.clip <= 0
+                     "kernel": (fused_kernel_name(fc, w.n_ranks, args.stage == 3 and not args.no_layered)
+                                if args.clip <= 0
                                 else "reduce_kernel + adam_bcast_kernel (two-pass step)"),
                      "kernel_config": ckey,
                      "kernel_ms_per_launch": kernel_ms, "launches": launches,
@@ -795,6 +803,7 @@ def run_stages(args):
                         synth.dev_bf16(W.grad_base(w, 1, r), off, n, w.grad_dist, reps[r].data_ptr() + 2 * off, s)
             rl = list(reps)
             opt.set_pdl(not args.no_pdl)
+            opt.set_layered(not args.no_layered)
             for _ in range(3):
                 opt.step_resident(rl)
             steps = max(5, int(2e9 / ((4 * w.n_ranks + 24) * w.psi)) + 5)
@@ -821,7 +830,7 @@ def run_stages(args):
                               "bytes_per_elem_model": per,
                               "step_gbs_model": per * w.psi / (ms / 1e3) / 1e9,
                               "kernel_gbs_model_isolated": kt["model_bytes"] / (kt["ms"] / 1e3) / 1e9,
-                              "pdl": not args.no_pdl,
+                              "pdl": not args.no_pdl, "layered": stage == 3 and not args.no_layered,
                               "launches_per_step": kt["launches"] // steps,
                               "fused_config": opt.fused_config(), "steps": steps}), flush=True)
             opt.close()

@@ -335,7 +335,9 @@ def test_adam_shard_per_rank_equals_all_ranks():
 @pytest.mark.parametrize("clip", [0.0, 0.5])
 def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
     """zero_launch_count advances by exactly the launches zero_kernel_timing
-    records plus the two one-thread step kernels, per step, plain and clipped."""
+    records plus the two one-thread step kernels, per step, plain and clipped;
+    a plain stage-3 step is one layered launch, or one launch per layer with
+    ZERO_OPT_LAYERED off."""
     numel, layer = W.transformer_layers(3, 64, 256)
     w = W.Workload("count", numel, layer, 4, (stage,), 16_000, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 2,
                    W.Hyper(), 0x600 + stage)
@@ -347,15 +349,21 @@ def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
                                           w.grad_dist).view(np.int16)).cuda() for r in range(w.n_ranks)]
     opt.set_timing(True)
     opt.kernel_timing()
-    for _ in range(2):
-        n0 = opt.launch_count()
-        opt.step_resident(dev)
-        torch.cuda.synchronize()
-        timed = opt.kernel_timing()["launches"]
-        intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
-        expect = intervals if clip == 0 else intervals + (intervals if stage == 3 else 1)
-        assert timed == expect, (timed, expect)
-        assert opt.launch_count() - n0 == timed + 2
+    assert opt.fused_config()["kernel"] == "bulk"  # AUTO's kernel at N = 4
+    for layered in ((True, False) if stage == 3 else (True,)):
+        opt.set_layered(layered)
+        for _ in range(2):
+            n0 = opt.launch_count()
+            opt.step_resident(dev)
+            torch.cuda.synchronize()
+            timed = opt.kernel_timing()["launches"]
+            intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
+            if clip == 0:
+                expect = 1 if stage == 3 and layered else intervals
+            else:
+                expect = intervals + (intervals if stage == 3 else 1)
+            assert timed == expect, (layered, timed, expect)
+            assert opt.launch_count() - n0 == timed + 2
     opt.set_timing(False)
     opt.close()
 
