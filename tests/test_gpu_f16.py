@@ -278,15 +278,19 @@ def test_f16_clip_and_overflow_skip(stage):
     opt.close()
 
 
-def test_f16_resident_step_equals_callback_step():
-    """step_resident on fp16 replicas (the bench's path) equals the callback step."""
+@pytest.mark.parametrize("stage", [2, 3])
+def test_f16_resident_step_equals_callback_step(stage):
+    """step_resident on fp16 replicas (the bench's path) equals the callback
+    step; at stage 3 the resident step is the layered launch (every layer in
+    one launch) and the callback step one launch per layer, layer buffers
+    included."""
     z = _z()
-    numel, layer = [65536, 4096], [0, 1]
-    w = W.Workload("resident-f16", numel, layer, 8, (2,), None, synth.Dist(synth.NORMAL, 4.0), W.MASTER_DIST, 2,
-                   W.Hyper(), 0x190)
+    numel, layer = [65536, 4096, 30_000], [0, 1, 2]
+    w = W.Workload("resident-f16", numel, layer, 8, (stage,), None, synth.Dist(synth.NORMAL, 4.0), W.MASTER_DIST, 2,
+                   W.Hyper(), 0x190 + stage)
     bucket = oracle.plan(numel, layer, 8, 1 << 40).psi_pad
-    a, fa = make_opt(w, 2, bucket, 1024.0)
-    b, fb = make_opt(w, 2, bucket, 1024.0)
+    a, fa = make_opt(w, stage, bucket, 1024.0)
+    b, fb = make_opt(w, stage, bucket, 1024.0)
     ga = grad_fn_for(a, fa)
     stream = torch.cuda.current_stream().cuda_stream
     for t in (1, 2):
@@ -297,7 +301,12 @@ def test_f16_resident_step_equals_callback_step():
         b.step_resident(reps)
     for what in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ):
         assert torch.equal(a.view(what), b.view(what))
-    for r in range(8):
-        assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
+    if stage == 3:
+        assert torch.equal(a.view(z.ZERO_VIEW_PARAM), b.view(z.ZERO_VIEW_PARAM))
+        for r in range(8):
+            assert torch.equal(a.view(z.ZERO_VIEW_GATHER, r), b.view(z.ZERO_VIEW_GATHER, r))
+    else:
+        for r in range(8):
+            assert torch.equal(a.view(z.ZERO_VIEW_PARAM, r), b.view(z.ZERO_VIEW_PARAM, r))
     a.close()
     b.close()

@@ -667,8 +667,12 @@ bool layered_ok(const zero_ctx* c, bool callbacks, const std::vector<zsm::Span>&
 // temporary layer buffers issued only after every CTA has finished storing
 // the layers before it -- the order of the per-layer launches, without a
 // launch boundary at each layer.  grad0[r] are the ranks' full replicas.
+// *refused: the device could not hold every CTA at once (a cooperative launch
+// refused, e.g. with fewer SMs available to this process); nothing was
+// launched, and the caller runs one launch per layer instead.
 zero_status fused_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, uint16_t* const* grad0, cudaStream_t s,
-                          const zsm::AdamScalars* sc_dev, bool twin) {
+                          const zsm::AdamScalars* sc_dev, bool twin, bool* refused) {
+  *refused = false;
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
   std::memset(&a, 0, sizeof a);
@@ -709,8 +713,14 @@ zero_status fused_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, uint16_
   if (e != cudaSuccess) return cuda_fail(c, e, "clearing the layered launch's counter");
   cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
   if (ev) cudaEventRecord(ev[0], s);
-  e = counted(c, zsm::launch_fused_bulk_layered(a, g, (int)std::min<int64_t>(max_tiles, c->sm_count), (int)tile,
-                                                bulk_warps(c), bulk_ring(c), twin, s));
+  e = zsm::launch_fused_bulk_layered(a, g, (int)std::min<int64_t>(max_tiles, c->sm_count), (int)tile,
+                                     bulk_warps(c), bulk_ring(c), twin, s);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();  // a launch-configuration error: the context stays usable
+    *refused = true;            // (an event pair recorded above is re-recorded by the next timed launch)
+    return ZERO_OK;
+  }
+  e = counted(c, e);
   if (e != cudaSuccess) return cuda_fail(c, e, "layered fused step kernel launch");
   if (ev) {
     cudaEventRecord(ev[1], s);
@@ -1153,10 +1163,12 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
   // (and not with two staged CTAs per SM asked for: a programmatic launch
   // keeps one per SM)
   const bool pdl_ok = c->pdl && !callbacks && c->tma_ctas_opt <= 1;
-  const bool one_launch = layered_ok(c, callbacks, iv);  // every layer in one launch
+  bool one_launch = layered_ok(c, callbacks, iv);  // every layer in one launch
   if (one_launch) {
     interval_grads(c, resident, 0, 0, grad.data());
-    st = fused_layered(c, iv, grad.data(), s, &state_ptr(c)->sc, false);
+    bool refused = false;
+    st = fused_layered(c, iv, grad.data(), s, &state_ptr(c)->sc, false, &refused);
+    one_launch = !refused;
   }
   for (size_t k = 0; k < iv.size() && st == ZERO_OK && !one_launch; ++k) {
     for (; issued < iv.size() && issued <= k + o.ahead() && st == ZERO_OK; ++issued)
@@ -1915,10 +1927,13 @@ zero_status zero_probe_pattern(zero_ctx* c, const void* const* rank_grads, void*
   const bool pdl_ok = c->pdl && c->tma_ctas_opt <= 1;
   if (layered_ok(c, false, iv)) {  // the step's own form: every layer in one launch
     interval_grads(c, rank_grads, 0, 0, grad.data());
-    st = fused_layered(c, iv, grad.data(), s, nullptr, true);
+    bool refused = false;
+    st = fused_layered(c, iv, grad.data(), s, nullptr, true, &refused);
     if (st != ZERO_OK) return st;
-    c->norm_fresh = true;
-    return ZERO_OK;
+    if (!refused) {
+      c->norm_fresh = true;
+      return ZERO_OK;
+    }
   }
   bool launched = false;
   for (size_t k = 0; k < iv.size(); ++k) {
