@@ -3,8 +3,8 @@ test recorder (tests/nvtx_recorder.c) loaded as the process's NVTX tool: a
 child process runs steps with the ranges on and off, and the recorded
 domain "zero_sm" holds, in order, one range per step with one nested range
 per launch naming its bucket or layer and its [lo, hi) -- the intervals of
-the step's schedule --, the clipped step's reduce / decision / update
-ranges, the stage-3 step's single range when its layers run as one launch,
+the step's schedule --, the clipped step's reduce (one launch over the
+resident replicas) / decision / update ranges, the stage-3 step's single range when its layers run as one launch,
 a range per unfused call, and nothing while the option is off."""
 import json
 import os
@@ -70,8 +70,8 @@ def _expected(stage, info):
         lines += [f"push zero_sm {kind} {k} [{lo}, {hi})", "pop zero_sm"]
     lines.append("pop zero_sm")
     lines.append(f"push zero_sm step 2 (stage {stage}, N = 4)")
-    for kind, k, lo, hi in sched:
-        lines += [f"push zero_sm reduce {kind} {k} [{lo}, {hi})", "pop zero_sm"]
+    # the resident replicas' first pass: one launch over the flat space
+    lines += [f"push zero_sm reduce all 0 [0, {info['psi_pad']})", "pop zero_sm"]
     lines += ["push zero_sm clip decision", "pop zero_sm"]
     if stage == 2:
         lines += [f"push zero_sm update all 0 [0, {info['psi_pad']})", "pop zero_sm"]

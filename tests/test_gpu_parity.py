@@ -337,7 +337,8 @@ def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
     """zero_launch_count advances by exactly the launches zero_kernel_timing
     records plus the two one-thread step kernels, per step, plain and clipped;
     a plain stage-3 step is one layered launch, or one launch per layer with
-    ZERO_OPT_LAYERED off."""
+    ZERO_OPT_LAYERED off; a clipped step's first pass over resident replicas
+    is one launch."""
     numel, layer = W.transformer_layers(3, 64, 256)
     w = W.Workload("count", numel, layer, 4, (stage,), 16_000, synth.Dist(synth.NORMAL, 1e-2), W.MASTER_DIST, 2,
                    W.Hyper(), 0x600 + stage)
@@ -360,8 +361,8 @@ def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
             intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
             if clip == 0:
                 expect = 1 if stage == 3 and layered else intervals
-            else:
-                expect = intervals + (intervals if stage == 3 else 1)
+            else:  # pass 1 over the resident replicas in one launch, pass 2 per layer at stage 3
+                expect = 1 + (intervals if stage == 3 else 1)
             assert timed == expect, (layered, timed, expect)
             assert opt.launch_count() - n0 == timed + 2
     opt.set_timing(False)

@@ -982,15 +982,19 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     const cudaError_t e = counted(c, zsm::launch_step_begin(state_ptr(c), step_hparams(c), nullptr, s));
     if (e != cudaSuccess) return cuda_fail(c, e, "step-begin kernel launch");
   }
-  // pass 1: reduce every interval
+  // pass 1: reduce every interval.  Resident gradients are all there at
+  // once and pass 1 writes only the flat shard (or, at stage 1, each
+  // replica in place), so the whole flat space is reduced in one launch; the
+  // intervals are for gradients that arrive interval by interval.
+  const std::vector<zsm::Span> p1 = resident ? std::vector<zsm::Span>{zsm::Span{0, c->plan.psi_pad}} : iv;
   bool launched = false;  // the first launch of the step starts the norm sum
   size_t issued = 0;
-  for (size_t k = 0; k < iv.size(); ++k) {
-    for (; issued < iv.size() && issued <= k + o.ahead(); ++issued) {
+  for (size_t k = 0; k < p1.size(); ++k) {
+    for (; !resident && issued < iv.size() && issued <= k + o.ahead(); ++issued) {
       zero_status st = issue_grads(c, o, fn, user, resident, iv, issued, t);
       if (st != ZERO_OK) return st;
     }
-    const int64_t lo = iv[k].lo, hi = iv[k].hi;
+    const int64_t lo = p1[k].lo, hi = p1[k].hi;
     zsm::ReduceArgs a;
     std::memset(&a, 0, sizeof a);
     a.fmt = c->fmt;
@@ -1005,8 +1009,9 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
     a.ns = norm_scratch(c);
     o.before_kernel(k, !resident && fn, (size_t)-1);
     if (a.n_vec > 0) {
-      const NvtxRange range(c->nvtx, "reduce %s %d [%lld, %lld)", c->stage == ZERO_STAGE_3 ? "layer" : "bucket",
-                            c->stage == ZERO_STAGE_3 ? c->plan.layers[n_layers - 1 - (int)k].id : (int)k,
+      const NvtxRange range(c->nvtx, "reduce %s %d [%lld, %lld)",
+                            resident ? "all" : c->stage == ZERO_STAGE_3 ? "layer" : "bucket",
+                            resident ? 0 : c->stage == ZERO_STAGE_3 ? c->plan.layers[n_layers - 1 - (int)k].id : (int)k,
                             (long long)lo, (long long)hi);
       cudaError_t e = launch_pass1(c, a, s);
       if (e != cudaSuccess) return cuda_fail(c, e, "reduce kernel launch");
