@@ -46,7 +46,7 @@ KERNEL_SOURCES = {"tma": [os.path.join(_CSRC, f) for f in ("fused_tma.cu", "tma_
                                                             "kernels.cuh")],
                   "register": [os.path.join(_CSRC, f) for f in ("kernels.cu", "device_math.cuh", "kernels.cuh")],
                   "bulk": [os.path.join(_CSRC, f) for f in ("fused_bulk.cu", "tma_pipe.cuh", "device_math.cuh",
-                                                            "kernels.cuh")]}
+                                                            "kernels.cuh", "layered_walk.cuh")]}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fused_step_traffic.json")
 
 

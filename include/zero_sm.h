@@ -206,9 +206,12 @@ enum {
                                     order of one launch per layer, without a launch boundary at
                                     each layer.  The gradient norm is summed over the whole
                                     step at once (the same value up to rounding order, the same
-                                    bits run to run).  Where the device cannot hold every CTA
-                                    at once (a cooperative launch refused), the step runs one
-                                    launch per layer instead.  0: one launch per layer.  The movement-
+                                    bits run to run).  The same holds for the update pass of a
+                                    clipped stage-3 step without gather_fn (zero_set_clip),
+                                    on the bulk-store kernel at any N.  Where the device cannot
+                                    hold every CTA at once (a cooperative launch refused), the
+                                    step runs one launch per layer instead.  0: one launch per
+                                    layer.  The movement-
                                     only pass (zero_probe_pattern) follows the same choice.
                                     May be set at any time */
   ZERO_OPT_NVTX = 18,            /* 1: NVTX ranges on the domain "zero_sm" around the host side

@@ -361,8 +361,8 @@ def test_launch_count_is_the_timed_launches_plus_the_step_kernels(stage, clip):
             intervals = len(opt.buckets()) if stage != 3 else len(opt.layers())
             if clip == 0:
                 expect = 1 if stage == 3 and layered else intervals
-            else:  # pass 1 over the resident replicas in one launch, pass 2 per layer at stage 3
-                expect = 1 + (intervals if stage == 3 else 1)
+            else:  # pass 1 over the resident replicas in one launch; pass 2 per layer at stage 3 unless layered
+                expect = 1 + (1 if stage != 3 or layered else intervals)
             assert timed == expect, (layered, timed, expect)
             assert opt.launch_count() - n0 == timed + 2
     opt.set_timing(False)
@@ -782,6 +782,60 @@ def test_clip_and_overflow_skip_against_oracle(stage):
         assert_bits_equal(to_np(opt.view(what)), ref[name], f"clip stage {stage} {name}")
     for r in (range(n_ranks) if stage != 3 else [0]):
         assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM, r)), ref["params"], f"clip stage {stage} params {r}")
+    if stage == 3:  # the update pass's layers in one launch: the buffers end with the first layer
+        _, lo0, hi0 = opt.layers()[0]
+        for r in range(n_ranks):
+            assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GATHER, r))[: hi0 - lo0], ref["params"][lo0:hi0],
+                              f"clip stage 3 last gathered layer, rank {r}")
+    opt.close()
+
+
+@pytest.mark.parametrize("layered", [True, False])
+def test_clipped_zero3_update_pass_layered_equals_per_layer(layered):
+    """The clipped stage-3 step's update pass, every layer in one cooperative
+    launch (layered) or one launch per layer, on unequal layers: states,
+    parameter shards and every rank's layer buffers against the oracle, bit
+    for bit, over two steps whose norms are clipped."""
+    z = _z()
+    numel, layer = [1_000_000, 3_000_000, 500_000, 2_000_000], [0, 1, 2, 3]
+    n_ranks, clip = 8, 0.05
+    w = W.Workload("clip-layered", numel, layer, n_ranks, (3,), 1 << 30, synth.Dist(synth.NORMAL, 1e-2, zero_mod=7),
+                   W.MASTER_DIST, 2, W.Hyper(weight_decay=0.01), 0xC7)
+    p = oracle.plan(numel, layer, n_ranks, 1 << 30)
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def g(t, r):
+        return W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), w.grad_dist)
+
+    ranks, reps = oracle.run(p, oracle.STAGE_Z3, m0, g, 2, oracle.AdamHP(**w.hyper.__dict__), clip_norm=clip,
+                             skip_nonfinite=True)
+    assert all(r.coef < 1.0 for r in reps)
+    ref = oracle.full_view(p, oracle.STAGE_Z3, ranks)
+    opt, fill = make_opt(w, 3, bucket=1 << 30)
+    opt.set_clip(clip, True)
+    opt.set_layered(layered)
+    s = torch.cuda.current_stream().cuda_stream
+    for t in (1, 2):
+        rp = torch.empty((n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+        for r in range(n_ranks):
+            fill.grads_into(t, r, 0, opt.psi_pad, rp[r].data_ptr(), rp[r], s)
+        before = opt.launch_count()
+        st = opt.step_resident(list(rp), stats=True)
+        # begin, pass 1 (one launch), decision, pass 2 (one or four launches)
+        assert opt.launch_count() - before == 3 + (1 if layered else len(numel))
+        assert st["clip_coef"] == reps[t - 1].coef
+    for name, what in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(opt.view(what)), ref[name], f"clipped layered={layered} {name}")
+    assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM)), ref["params"], f"clipped layered={layered} shards")
+    width = max(hi - lo for _, lo, hi in opt.layers())
+    want = np.zeros(width, dtype=ref["params"].dtype)
+    done = np.zeros(width, dtype=bool)
+    for _, lo, hi in opt.layers():  # flat order = the schedule's last launch first
+        fresh = ~done[: hi - lo]
+        want[: hi - lo][fresh] = ref["params"][lo:hi][fresh]
+        done[: hi - lo] = True
+    for r in range(n_ranks):
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GATHER, r))[:width], want, f"clipped layered={layered} buffer {r}")
     opt.close()
 
 

@@ -29,6 +29,7 @@
 #include "kernels.cuh"
 #include "two_pass_bulk.cuh"
 #include "tma_pipe.cuh"
+#include "layered_walk.cuh"
 
 namespace zsm {
 namespace {
@@ -719,6 +720,185 @@ __global__ void __launch_bounds__(kBulkBcastThreads, 1)
   }
 }
 
+// The same pass over every layer of a stage-3 step in one cooperative launch
+// (layered_walk.cuh): `a`'s sources, states and shard at flat element 0
+// (a.lo = 0), its N destinations at the temporary layer buffers' start; a
+// layer's stores into those buffers follow every CTA's stores of the layers
+// before it.  A kernel of its own, so that the one-interval kernel above
+// keeps its measured code.
+template <class F>
+__global__ void __launch_bounds__(kBulkBcastThreads, 1)
+    adam_bcast_bulk_layered_kernel(const __grid_constant__ AdamBcastArgs a, int stages, int uniform, int store_hint,
+                                   const __grid_constant__ SegTable g) {
+  constexpr int T = kBulkBcastTile;
+  constexpr int W = kBulkBcastWarps;
+  constexpr int EPT = T / (32 * W);
+  static_assert(EPT == 4, "four elements per consumer lane");
+  extern __shared__ __align__(128) unsigned char smem[];
+  const unsigned sb = kBulkBcastStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * sb);
+  uint64_t* computed = full + stages;
+  uint64_t* empty = computed + stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+  volatile int* last_k = abort_flag + 1;
+  AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
+  const bool skip = apply_decision(a.dec, sc);  // a skipped step writes the unchanged parameters only
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&computed[s], W);
+      mbar_init(&empty[s], 1);
+      last_k[s] = -1;
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      TileCursor cur;
+      for (int it = 0;; ++it) {
+        long long e0, ed;
+        unsigned cnt;
+        if (!cursor_next<T, true>(cur, g, 0, 0, e0, ed, cnt) || *abort_flag) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        if (k > 0) {
+          const int w = mbar_wait_or_abort(&empty[s], (k - 1) & 1u, abort_flag, a.wait_ns);
+          if (w != 0) {
+            if (w == 1) atomicOr(a.error, 1u);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        fence_proxy_async_smem();  // the stage's last reads (consumers, stores) before the refill
+        unsigned char* st = smem + (size_t)s * sb;
+        mbar_expect_tx(&full[s], cnt * 14u);
+        const int64_t i0 = e0;  // flat index of the tile's first element
+        if (uniform) {
+          bulk_load(st, a.gsrc[0] + i0, (unsigned)(2 * cnt), &full[s], policy);
+        } else {
+          // one copy per owner: owners change every `shard` elements (a multiple of 8)
+          for (int64_t e = 0; e < (int64_t)cnt;) {
+            const int64_t owner = (i0 + e) / a.shard;
+            const int64_t next = (owner + 1) * a.shard - i0;
+            const int64_t end = next < (int64_t)cnt ? next : (int64_t)cnt;
+            bulk_load(st + 2 * e, a.gsrc[owner] + i0 + e, (unsigned)(2 * (end - e)), &full[s], policy);
+            e = end;
+          }
+        }
+        bulk_load(st + 2 * T, a.master + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + 6 * T, a.m + e0, (unsigned)(4 * cnt), &full[s], policy);
+        bulk_load(st + 10 * T, a.v + e0, (unsigned)(4 * cnt), &full[s], policy);
+        last_k[s] = (int)k;
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- storer --
+    if (lane == 0) {
+      const uint64_t spol = evict_first_policy();
+      auto put = [&](void* dst, const void* src, unsigned bytes) {
+        if (store_hint) bulk_store(dst, src, bytes, spol);
+        else bulk_store(dst, src, bytes);
+      };
+      TileCursor cur;
+      int arrived = 0;  // layers this storer has finished and arrived for
+      for (int it = 0;; ++it) {
+        long long e0, ed;
+        unsigned cnt;
+        if (!cursor_next<T, true>(cur, g, 0, 0, e0, ed, cnt)) break;
+        const int s = it % stages;
+        const unsigned k = (unsigned)(it / stages);
+        const int w = mbar_wait_or_abort(&computed[s], k & 1u, abort_flag, a.wait_ns);
+        if (w != 0) {
+          if (w == 1) atomicOr(a.error, 8u);
+          *abort_flag = 1;
+          break;
+        }
+        if (cur.seg > arrived) {  // a new layer: every CTA's stores of the layers before it first
+          while (arrived < cur.seg) {
+            segment_arrive(g.counter);
+            ++arrived;
+          }
+          if (!segment_wait(g.counter, gridDim.x * (unsigned)cur.seg, abort_flag, a.wait_ns)) {
+            atomicOr(a.error, 16u);
+            *abort_flag = 1;
+            break;
+          }
+        }
+        const unsigned char* st = smem + (size_t)s * sb;
+        if (!skip) {
+          put(a.master + e0, st + 2 * T, 4 * cnt);
+          put(a.m + e0, st + 6 * T, 4 * cnt);
+          put(a.v + e0, st + 10 * T, 4 * cnt);
+        }
+        if (a.param_shard) put(a.param_shard + e0, st, 2 * cnt);
+        for (int r = 0; r < a.n_out; ++r) put(a.out[r] + ed, st, 2 * cnt);
+        bulk_commit();
+        bulk_wait_read<0>();  // the copies have read the stage: hand it back to the producer
+        mbar_arrive(&empty[s]);
+      }
+      // arrive for the layers left (also after an abort: the other CTAs'
+      // waits then end; the step has failed)
+      for (; arrived < g.n; ++arrived) segment_arrive(g.counter);
+      bulk_wait<0>();  // every store of this CTA performed before the CTA ends
+    }
+  } else {
+    // ----------------------------------------------------------- consumers --
+    const int j = (threadIdx.x - 64) * EPT;
+    TileCursor cur;
+    for (int it = 0;; ++it) {
+      long long e0, ed;
+      unsigned cnt;
+      if (!cursor_next<T, true>(cur, g, 0, 0, e0, ed, cnt)) break;
+      const int s = it % stages;
+      const unsigned k = (unsigned)(it / stages);
+      const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], k & 1u, a.wait_ns));
+      if (!ok) {
+        if (lane == 0) atomicOr(a.error, 2u);
+        *abort_flag = 1;
+        break;
+      }
+      if (__any_sync(0xFFFFFFFFu, *abort_flag != 0)) break;
+      unsigned char* st = smem + (size_t)s * sb;
+      if (j < (int)cnt) {  // cnt is a multiple of 8, so a lane's four elements are whole
+        float4 p = *reinterpret_cast<const float4*>(st + 2 * T + 4 * j);
+        float4 m = *reinterpret_cast<const float4*>(st + 6 * T + 4 * j);
+        float4 v = *reinterpret_cast<const float4*>(st + 10 * T + 4 * j);
+        uint2 pw;
+        if (skip) {
+          pw = make_uint2(pack2(F::rn(p.x), F::rn(p.y)), pack2(F::rn(p.z), F::rn(p.w)));
+        } else {
+          const uint2 gw = *reinterpret_cast<const uint2*>(st + 2 * j);
+          const uint16_t h0 = F::rn(adam1(F::lo(gw.x), p.x, m.x, v.x, sc));  // loss-scale and clip factors via sc.flags
+          const uint16_t h1 = F::rn(adam1(F::hi(gw.x), p.y, m.y, v.y, sc));
+          const uint16_t h2 = F::rn(adam1(F::lo(gw.y), p.z, m.z, v.z, sc));
+          const uint16_t h3 = F::rn(adam1(F::hi(gw.y), p.w, m.w, v.w, sc));
+          pw = make_uint2(pack2(h0, h1), pack2(h2, h3));
+          *reinterpret_cast<float4*>(st + 2 * T + 4 * j) = p;
+          *reinterpret_cast<float4*>(st + 6 * T + 4 * j) = m;
+          *reinterpret_cast<float4*>(st + 10 * T + 4 * j) = v;
+        }
+        *reinterpret_cast<uint2*>(st + 2 * j) = pw;  // over the gradient, which this lane alone read here
+      }
+      fence_proxy_async_smem();  // this lane's stage writes before the storer's bulk copies read them
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&computed[s]);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // drain the bulk loads already issued before the CTA's memory goes away
+    for (int s = 0; s < stages; ++s)
+      if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.error, 4u);
+  }
+}
+
 template <class K>
 cudaError_t opt_in(K kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTmaMaxSmem);
@@ -746,6 +926,8 @@ cudaError_t two_pass_configure() {
   if (e == cudaSuccess) e = opt_in(adam_bcast_tma_kernel<F16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_kernel<Bf16>);
   if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_kernel<F16>);
+  if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_layered_kernel<Bf16>);
+  if (e == cudaSuccess) e = opt_in(adam_bcast_bulk_layered_kernel<F16>);
   if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<false, Bf16>);
   if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<true, Bf16>);
   if (e == cudaSuccess) e = opt_in(reduce_bulk_kernel<false, F16>);
@@ -798,6 +980,30 @@ cudaError_t launch_adam_bcast_bulk(const AdamBcastArgs& a, int grid, bool unifor
   else
     adam_bcast_bulk_kernel<Bf16><<<grid, kBulkBcastThreads, bytes, s>>>(a, stages, uniform ? 1 : 0, store_hint);
   return cudaGetLastError();
+}
+
+cudaError_t launch_adam_bcast_bulk_layered(const AdamBcastArgs& a, const SegTable& g, int grid, bool uniform,
+                                           int stages, int store_hint, cudaStream_t s) {
+  if (g.n < 1 || g.n > kMaxSegments || !g.counter || a.lo != 0) return cudaErrorInvalidValue;
+  if (stages < 2) stages = 2;
+  if (stages > kTmaMaxStages) stages = kTmaMaxStages;
+  while (stages > 2 && bulk_bcast_smem_bytes(stages) > (size_t)kTmaMaxSmem) --stages;
+  // at least 116 KB, so that an SM holds one CTA: tiles are dealt by CTA index
+  const size_t bytes = std::max<size_t>(bulk_bcast_smem_bytes(stages), 116 * 1024);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3((unsigned)kBulkBcastThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int un = uniform ? 1 : 0;
+  if (a.fmt == kFmtF16)
+    return cudaLaunchKernelEx(&cfg, adam_bcast_bulk_layered_kernel<F16>, a, stages, un, store_hint, g);
+  return cudaLaunchKernelEx(&cfg, adam_bcast_bulk_layered_kernel<Bf16>, a, stages, un, store_hint, g);
 }
 
 cudaError_t launch_reduce_bulk(const ReduceArgs& a, int grid, int stages, int store_hint, cudaStream_t s) {

@@ -967,6 +967,71 @@ cudaError_t launch_pass2(zero_ctx* c, const zsm::AdamBcastArgs& b, bool uniform,
 
 // Clipped / overflow-checked step: reduce everything, read the norm, then
 // Adam + broadcast.
+// Pass 2 of a clipped stage-3 step without a gather callback as one
+// cooperative launch over its layers (ZERO_OPT_LAYERED, the bulk-store pass
+// 2): each layer's stores into the temporary layer buffers follow every
+// CTA's stores of the layers before it.  *refused: the device could not hold
+// every CTA at once; nothing was launched.
+zero_status pass2_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, zsm::ClipDecision* dec, cudaStream_t s,
+                          bool* refused) {
+  *refused = false;
+  const int N = c->plan.n_ranks;
+  zsm::AdamBcastArgs b;
+  std::memset(&b, 0, sizeof b);
+  b.fmt = c->fmt;
+  for (int r = 0; r < N; ++r) {
+    b.gsrc[r] = grad_shard_ptr(c);
+    b.out[r] = gather_ptr(c, r, 0);
+  }
+  b.n_out = N;
+  b.master = master_ptr(c);
+  b.m = m_ptr(c);
+  b.v = v_ptr(c);
+  b.param_shard = param_ptr(c, 0);
+  b.lo = 0;
+  b.shard = c->plan.shard;
+  b.n_vec = c->plan.psi_pad / zsm::kVec;
+  b.sc_dev = &state_ptr(c)->sc;
+  b.dec = dec;
+  b.error = norm_scratch(c).error;
+  b.wait_ns = c->wait_ns;
+  zsm::SegTable g;
+  std::memset(&g, 0, sizeof g);
+  g.counter = reinterpret_cast<unsigned*>(c->arena[ZERO_ARENA_SCRATCH] + kSegCounterOffset);
+  int64_t elems = 0, max_tiles = 1;
+  const int64_t tile = zsm::bulk_bcast_tile();
+  for (const zsm::Span& sp : iv) {
+    if (sp.hi == sp.lo) continue;
+    g.lo[g.n] = sp.lo;
+    g.len[g.n] = sp.hi - sp.lo;
+    ++g.n;
+    elems += sp.hi - sp.lo;
+    max_tiles = std::max(max_tiles, (sp.hi - sp.lo + tile - 1) / tile);
+  }
+  const NvtxRange range(c->nvtx, "update layers x %d [%lld, %lld) in one launch", g.n, (long long)g.lo[g.n - 1],
+                        (long long)(g.lo[0] + g.len[0]));
+  cudaError_t e = cudaMemsetAsync(g.counter, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(c, e, "clearing the layered launch's counter");
+  cudaEvent_t* ev = c->timing ? timing_pair(c) : nullptr;
+  if (ev) cudaEventRecord(ev[0], s);
+  e = zsm::launch_adam_bcast_bulk_layered(b, g, (int)std::min<int64_t>(max_tiles, c->sm_count), true,
+                                          c->tma_stages_opt ? c->tma_stages_opt : 4,
+                                          c->store_hint >= 0 ? c->store_hint : 1, s);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();  // a launch-configuration error: the context stays usable
+    *refused = true;
+    return ZERO_OK;
+  }
+  e = counted(c, e);
+  if (e != cudaSuccess) return cuda_fail(c, e, "layered adam-broadcast kernel launch");
+  if (ev) {
+    cudaEventRecord(ev[1], s);
+    c->timed += 1;
+    c->timed_bytes += (double)(2 + 24 + 2 * N + 2) * (double)elems;
+  }
+  return ZERO_OK;
+}
+
 zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* const* resident,
                          zero_gather_fn gfn, void* guser, StepOrder& o, zero_step_stats* stats) {
   const int N = c->plan.n_ranks;
@@ -1042,6 +1107,16 @@ zero_status run_two_pass(zero_ctx* c, zero_grad_fn fn, void* user, const void* c
   std::vector<zsm::Span> p2;
   if (c->stage == ZERO_STAGE_3) p2 = iv;
   else p2.push_back({0, c->plan.psi_pad});
+  if (c->stage == ZERO_STAGE_3 && !gfn && c->layered && use_bulk(c)) {
+    int n = 0;
+    for (const zsm::Span& sp : iv) n += sp.hi > sp.lo ? 1 : 0;
+    if (n >= 2 && n <= zsm::kMaxSegments) {
+      bool refused = false;
+      st = pass2_layered(c, iv, dec, s, &refused);
+      if (st != ZERO_OK) return st;
+      if (!refused) p2.clear();  // every layer done in the one launch
+    }
+  }
   for (size_t k = 0; k < p2.size(); ++k) {
     const int64_t lo = p2[k].lo, hi = p2[k].hi;
     const int layer_idx = c->stage == ZERO_STAGE_3 ? n_layers - 1 - (int)k : 0;
