@@ -48,7 +48,7 @@
 extern "C" {
 #endif
 
-#define ZERO_SM_VERSION 2
+#define ZERO_SM_VERSION 3
 #define ZERO_MAX_RANKS 128
 
 typedef enum zero_status {

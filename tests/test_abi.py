@@ -31,7 +31,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = ctypes.CDLL(z.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), f"{name} declared in zero_sm.h but not exported"
-    assert z.zero_version() == 2
+    assert z.zero_version() == 3
     # and the binding exposes the same names
     for name in declared:
         assert callable(getattr(z, name)), name
