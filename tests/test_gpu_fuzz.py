@@ -2,8 +2,9 @@
 sizes including zero-size tensors, layer grouping), N, stage, bucket, 16-bit
 format and loss scale, clipping with the overflow skip, the callback
 pipeline, programmatic dependent launch and the kernel family, each run for
-two steps through the C ABI and compared with the oracle's literal per-rank
-run: fp32 states, parameters and reduced gradients bit for bit, statistics
+two steps through the C ABI -- through the gradient callback and from
+resident replicas -- and compared with the oracle's literal per-rank run:
+fp32 states, parameters and reduced gradients bit for bit, statistics
 exactly (the norm within its summation bound)."""
 import gc
 import math
@@ -121,4 +122,79 @@ def test_random_configuration_against_the_oracle(k):
     else:
         for r in range(w.n_ranks):
             assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GRAD_BUF, r)), ranks[r].grads, f"{what} all-reduced {r}")
+    opt.close()
+
+
+@pytest.mark.parametrize("k", range(N_CASES))
+def test_random_configuration_resident_against_the_oracle(k):
+    """The same seeded configurations stepped from resident replicas
+    (zero_step_resident): a stage-3 step on the bulk-store kernel runs as
+    one layered launch, a clipped step's first pass as one launch over the
+    flat space.  States, parameters and reduced gradients bit for bit, and
+    at stage 3 every rank's layer buffers: each byte the parameter of the
+    last layer in the schedule long enough to write it."""
+    import zero_sharded_optimizer_sm_b200 as z
+
+    c = _case(k)
+    dist = synth.Dist(synth.NORMAL, 1e-2 * c["scale"], zero_mod=9)
+    w = W.Workload("fuzz", c["numel"], c["layer"], c["n_ranks"], (c["stage"],), c["bucket"], dist, W.MASTER_DIST, 2,
+                   W.Hyper(lr=1e-2, weight_decay=0.05), c["seed"])
+    p = oracle.plan(w.numel, w.layer_id, w.n_ranks, c["bucket"])
+    m0 = W.host_padded(p.offset, p.numel, p.psi_pad, W.master_base(w), W.MASTER_DIST, as_f32=True)
+
+    def g(t, r):
+        return W.host_padded(p.offset, p.numel, p.psi_pad, W.grad_base(w, t, r), dist, f16=c["f16"])
+
+    fmt = oracle.F16 if c["f16"] else oracle.BF16
+    ranks, reps = oracle.run(p, STAGE_OF[c["stage"]], m0, g, 2, oracle.AdamHP(**w.hyper.__dict__),
+                             clip_norm=c["clip"], skip_nonfinite=c["clip"] > 0, fmt=fmt, loss_scale=c["scale"])
+    ref = oracle.full_view(p, STAGE_OF[c["stage"]], ranks)
+
+    opt = z.ZeroOptimizer(w.numel, w.layer_id, w.n_ranks, c["stage"], bucket_elems=c["bucket"],
+                          hparams=z.AdamHParams(**w.hyper.__dict__), kernel=c["kernel"], pipeline=c["pipeline"],
+                          tma_tile=c["tile"], tma_warps=c["warps"],
+                          dtype=z.ZERO_DTYPE_F16 if c["f16"] else z.ZERO_DTYPE_BF16)
+    opt.set_pdl(c["pdl"])
+    if c["scale"] != 1.0:
+        opt.set_loss_scale(c["scale"])
+    if c["clip"] > 0:
+        opt.set_clip(c["clip"], True)
+    fill = DeviceFill(w, opt.offsets(), opt.psi_pad, f16=c["f16"])
+    s = torch.cuda.current_stream().cuda_stream
+    mv = opt.view(z.ZERO_VIEW_MASTER)
+    fill.master_into(mv.data_ptr(), mv, s)
+    opt.load_master(None)
+    for t in (1, 2):
+        rp = torch.empty((w.n_ranks, opt.psi_pad), dtype=torch.int16, device="cuda")
+        for r in range(w.n_ranks):
+            fill.grads_into(t, r, 0, opt.psi_pad, rp[r].data_ptr(), rp[r], s)
+        st = opt.step_resident(list(rp), stats=True)
+        rep = reps[t - 1]
+        assert st["nonfinite"] == rep.nonfinite and st["skipped"] == rep.skipped, c
+        if c["clip"] > 0 and not rep.skipped:
+            assert st["clip_coef"] == rep.coef, c
+        assert st["grad_norm"] == rep.grad_norm or math.isclose(
+            st["grad_norm"], rep.grad_norm, rel_tol=2 * p.psi_pad * 2.0**-53 + 1e-15), c
+    torch.cuda.synchronize()
+    what = f"resident case {k} {c}"
+    for name, v in (("master", z.ZERO_VIEW_MASTER), ("m", z.ZERO_VIEW_EXP_AVG), ("v", z.ZERO_VIEW_EXP_AVG_SQ)):
+        assert_bits_equal(to_np(opt.view(v)), ref[name], f"{what} {name}")
+    for r in (range(w.n_ranks) if c["stage"] != 3 else [0]):
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_PARAM, r)), ref["params"], f"{what} params {r}")
+    if c["stage"] != 1:
+        assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GRAD_SHARD)), ref["grad"], f"{what} grad shards")
+    else:  # the all-reduce written back into the resident replicas
+        for r in range(w.n_ranks):
+            assert_bits_equal(to_np(rp[r]), ranks[r].grads, f"{what} all-reduced {r}")
+    if c["stage"] == 3:
+        layers = [(lo, hi) for _, lo, hi in opt.layers() if hi > lo]
+        width = max(hi - lo for lo, hi in layers)
+        want = np.zeros(width, dtype=ref["params"].dtype)
+        done = np.zeros(width, dtype=bool)
+        for lo, hi in layers:  # flat order = the schedule's last launch first
+            fresh = ~done[: hi - lo]
+            want[: hi - lo][fresh] = ref["params"][lo:hi][fresh]
+            done[: hi - lo] = True
+        for r in range(w.n_ranks):
+            assert_bits_equal(to_np(opt.view(z.ZERO_VIEW_GATHER, r))[:width], want, f"{what} layer buffer {r}")
     opt.close()
