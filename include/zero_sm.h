@@ -239,10 +239,13 @@ enum {
                                     with no gather_fn) launches its fused kernels with
                                     programmatic dependent launch, so that each launch's CTAs
                                     start on the SMs the previous launch leaves and, at stage
-                                    1/2, stream their own interval while it finishes (a staged
-                                    launch then reserves at least 116 KB of shared memory, so
-                                    that an SM never holds two CTAs of one grid); 0: plain
-                                    launches.  Values are unchanged either way.  Off while
+                                    1/2, stream their own interval while it finishes; at stage 3
+                                    a launch loads and computes at once and stores after the
+                                    launch before has completed (a staged launch then reserves
+                                    at least 116 KB of shared memory, so that an SM never holds
+                                    two CTAs of one grid).  A stage-3 step that runs as one
+                                    layered launch (ZERO_OPT_LAYERED) has no launch to chain.
+                                    0: plain launches.  Values are unchanged either way.  Off while
                                     ZERO_OPT_TIMING is on, and with ZERO_OPT_TMA_CTAS_PER_SM
                                     above 1.  May be set at any time */
 };
