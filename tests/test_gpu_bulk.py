@@ -387,3 +387,45 @@ def test_zero3_chained_layers_order_their_shared_buffer_stores(n_ranks):
                           f"chained ZeRO-3 last gathered layer, rank {r}")
     a.close()
     b.close()
+
+
+@pytest.mark.parametrize("clipped", [False, True])
+def test_layered_buffers_equal_per_layer_launches_step_after_step(clipped):
+    """Ordering stress for the layered stage-3 launches: layer lengths that
+    fall along the schedule, so every layer leaves a part of the layer
+    buffers and a store landing out of layer order would change bytes that
+    survive the step.  Twelve steps, every rank's layer buffers, the states
+    and the parameter shards compared bit for bit after each step between the
+    layered launch and one launch per layer (the fused step, and the clipped
+    step's update pass)."""
+    z = _z()
+    numel, layer = [300_008, 700_000, 1_500_000, 2_500_000], [0, 1, 2, 3]
+    n_ranks = 8
+    w = _workload(numel, layer, n_ranks, 3, 1 << 30, steps=12)
+    s = torch.cuda.current_stream().cuda_stream
+    opts = []
+    for layered in (True, False):
+        opt = z.ZeroOptimizer(w.numel, w.layer_id, n_ranks, 3, bucket_elems=1 << 30,
+                              hparams=z.AdamHParams(**w.hyper.__dict__), kernel=BULK)
+        fill = DeviceFill(w, opt.offsets(), opt.psi_pad)
+        mv = opt.view(z.ZERO_VIEW_MASTER)
+        fill.master_into(mv.data_ptr(), mv, s)
+        opt.load_master(None)
+        opt.set_layered(layered)
+        if clipped:
+            opt.set_clip(0.05, True)
+        opts.append((opt, fill))
+    (a, fa), (b, _) = opts
+    rp = torch.empty((n_ranks, a.psi_pad), dtype=torch.int16, device="cuda")
+    for t in range(1, w.steps + 1):
+        for r in range(n_ranks):
+            fa.grads_into(t, r, 0, a.psi_pad, rp[r].data_ptr(), rp[r], s)
+        sa = a.step_resident(list(rp), stats=True)
+        sb = b.step_resident(list(rp), stats=True)
+        assert sa["step"] == sb["step"] == t and sa["clip_coef"] == sb["clip_coef"]
+        for r in range(n_ranks):
+            assert torch.equal(a.view(z.ZERO_VIEW_GATHER, r), b.view(z.ZERO_VIEW_GATHER, r)), (t, r)
+        for view in (z.ZERO_VIEW_MASTER, z.ZERO_VIEW_EXP_AVG, z.ZERO_VIEW_EXP_AVG_SQ, z.ZERO_VIEW_PARAM):
+            assert torch.equal(a.view(view), b.view(view)), (t, view)
+    a.close()
+    b.close()
