@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
   if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
-  unsigned long long nf = 0;
+  unsigned nf32 = 0;  // non-finite count of this lane (well below 2^32 elements a lane)
   const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp == 0) {
@@ -313,8 +313,10 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
             g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
             const float g = F::f32(g16[q]);
             const double d = (double)g;
-            sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
-            nf += isfinite(g) ? 0ull : 1ull;
+            // the square is exact (at most 11-bit significands, in range), so the
+            // fused multiply-add rounds once, as the add after an exact product
+            sq = __fma_rn(d, d, sq);
+            nf32 += isfinite(g) ? 0u : 1u;
             p16[q] = F::rn(adam1(g, p.f[q], m.f[q], v.f[q], sc));
           }
 #pragma unroll
@@ -341,7 +343,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
   if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
-  norm_epilogue<NT>(a.ns, sq, nf, a.accumulate);
+  norm_epilogue<NT>(a.ns, sq, (unsigned long long)nf32, a.accumulate);
 }
 
 // The layered stage-3 launch: the kernel above with the tile walk through
@@ -386,7 +388,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
   if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
-  unsigned long long nf = 0;
+  unsigned nf32 = 0;  // non-finite count of this lane (well below 2^32 elements a lane)
   const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp == 0) {
@@ -540,8 +542,10 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
             g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
             const float g = F::f32(g16[q]);
             const double d = (double)g;
-            sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
-            nf += isfinite(g) ? 0ull : 1ull;
+            // the square is exact (at most 11-bit significands, in range), so the
+            // fused multiply-add rounds once, as the add after an exact product
+            sq = __fma_rn(d, d, sq);
+            nf32 += isfinite(g) ? 0u : 1u;
             p16[q] = F::rn(adam1(g, p.f[q], m.f[q], v.f[q], sc));
           }
 #pragma unroll
@@ -568,7 +572,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
       if (last_k[s] >= 0 && !mbar_wait(&full[s], (unsigned)last_k[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
   if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
-  norm_epilogue<NT>(a.ns, sq, nf, a.accumulate);
+  norm_epilogue<NT>(a.ns, sq, (unsigned long long)nf32, a.accumulate);
 }
 
 // --------------------------------------- rank-chunked bulk-store variant --
@@ -640,7 +644,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
   if (a.pdl == kPdlWaitFirst) pdl_wait();
 
   double sq = 0.0;
-  unsigned long long nf = 0;
+  unsigned nf32 = 0;  // non-finite count of this lane (well below 2^32 elements a lane)
   const AdamScalars sc = a.sc_dev ? *a.sc_dev : a.sc;
 
   if (warp == 0) {
@@ -814,8 +818,10 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
             g16[q] = F::rn(__fmul_rn(acc[q], a.inv_n));
             const float g = F::f32(g16[q]);
             const double d = (double)g;
-            sq = __dadd_rn(sq, __dmul_rn(d, d));  // each square exact (at most 11-bit significands)
-            nf += isfinite(g) ? 0ull : 1ull;
+            // the square is exact (at most 11-bit significands, in range), so the
+            // fused multiply-add rounds once, as the add after an exact product
+            sq = __fma_rn(d, d, sq);
+            nf32 += isfinite(g) ? 0u : 1u;
             p16[q] = F::rn(adam1(g, p.f[q], m.f[q], v.f[q], sc));
           }
 #pragma unroll
@@ -844,7 +850,7 @@ __global__ void __launch_bounds__(32 * (W + 2), 1)
       if (last_sk[s] >= 0 && !mbar_wait(&sfull[s], (unsigned)last_sk[s] & 1u)) atomicOr(a.ns.error, 4u);
   }
   if (a.pdl == kPdlEarly || a.pdl == kPdlEarlyLoads) pdl_wait();  // the norm scratch is shared with the grid before
-  norm_epilogue<NT>(a.ns, sq, nf, a.accumulate);
+  norm_epilogue<NT>(a.ns, sq, (unsigned long long)nf32, a.accumulate);
 }
 
 // A programmatic dependent launch may place its CTAs while the grid before it
