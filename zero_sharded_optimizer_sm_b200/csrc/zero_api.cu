@@ -589,11 +589,32 @@ std::vector<zsm::Span> step_intervals(const zero_ctx* c) {
   return out;
 }
 
+// A launch range against the planner's buffers: inside the flat space, on
+// the 8-element granule, and no longer than the buffer it passes through
+// (the stage-3 layer buffers; the stage-2 gradient bucket when the
+// gradients come through it).  A failure is a planner error, reported
+// before anything is launched.
+zero_status check_launch_range(zero_ctx* c, int64_t lo, int64_t hi, bool through_bucket) {
+  const zsm::Plan& p = c->plan;
+  const bool ok = 0 <= lo && lo <= hi && hi <= p.psi_pad && lo % zsm::kVec == 0 && hi % zsm::kVec == 0 &&
+                  (c->stage != ZERO_STAGE_3 || hi - lo <= p.max_layer) &&
+                  (!through_bucket || c->stage != ZERO_STAGE_2 || hi - lo <= p.max_bucket);
+  if (ok) return ZERO_OK;
+  return fail(c, ZERO_EINVAL, "launch range [%lld, %lld) does not fit the plan (psi_pad %lld, largest layer %lld, "
+              "bucket %lld)", (long long)lo, (long long)hi, (long long)p.psi_pad, (long long)p.max_layer,
+              (long long)p.max_bucket);
+}
+
 // One fused launch over [lo, hi).  grad[r] are at flat element lo.
 zero_status fused_interval(zero_ctx* c, int64_t lo, int64_t hi, uint16_t* const* grad, int layer_idx,
                            bool accumulate, const zsm::AdamScalars& sc, cudaStream_t s, int slot = 0,
-                           int pdl = zsm::kPdlNone, const zsm::AdamScalars* sc_dev = nullptr, bool twin = false) {
+                           int pdl = zsm::kPdlNone, const zsm::AdamScalars* sc_dev = nullptr, bool twin = false,
+                           bool through_bucket = false) {
   if (hi == lo) return ZERO_OK;
+  {
+    const zero_status st = check_launch_range(c, lo, hi, through_bucket);
+    if (st != ZERO_OK) return st;
+  }
   const int N = c->plan.n_ranks;
   zsm::FusedArgs a;
   std::memset(&a, 0, sizeof a);
@@ -701,6 +722,8 @@ zero_status fused_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, uint16_
   const int64_t tile = bulk_tile(c);
   for (const zsm::Span& sp : iv) {
     if (sp.hi == sp.lo) continue;
+    const zero_status st = check_launch_range(c, sp.lo, sp.hi, false);
+    if (st != ZERO_OK) return st;
     g.lo[g.n] = sp.lo;
     g.len[g.n] = sp.hi - sp.lo;
     ++g.n;
@@ -1002,6 +1025,8 @@ zero_status pass2_layered(zero_ctx* c, const std::vector<zsm::Span>& iv, zsm::Cl
   const int64_t tile = zsm::bulk_bcast_tile();
   for (const zsm::Span& sp : iv) {
     if (sp.hi == sp.lo) continue;
+    const zero_status st = check_launch_range(c, sp.lo, sp.hi, false);
+    if (st != ZERO_OK) return st;
     g.lo[g.n] = sp.lo;
     g.len[g.n] = sp.hi - sp.lo;
     ++g.n;
@@ -1265,7 +1290,8 @@ zero_status run_step(zero_ctx* c, zero_grad_fn fn, void* user, const void* const
     const NvtxRange range(c->nvtx, "%s %d [%lld, %lld)", c->stage == ZERO_STAGE_3 ? "layer" : "bucket",
                           c->stage == ZERO_STAGE_3 ? c->plan.layers[layer_idx].id : (int)k, (long long)lo,
                           (long long)hi);
-    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl, &state_ptr(c)->sc);
+    st = fused_interval(c, lo, hi, grad.data(), layer_idx, launched, sc, s, o.slot(k), pdl, &state_ptr(c)->sc,
+                        false, !resident);
     if (st != ZERO_OK) break;
     launched = launched || hi > lo;
     o.after_kernel(k);
