@@ -99,3 +99,20 @@ def test_clock_sampler_matches_the_gpu_by_pci_bus_id(monkeypatch):
 
     monkeypatch.setattr(bench.subprocess, "run", no_smi)
     assert bench.nvsmi_index(3) == 3
+
+
+def test_fused_kernel_name_follows_the_context_configuration():
+    """The roofline's kernel name (the one the ncu launch list shows) from a
+    context's fused configuration: the bulk-store kernel, its rank-chunked
+    form above 16 ranks, its layered stage-3 launch, and the older kernels."""
+    import bench
+
+    bulk = {"kernel": "bulk", "groups": 8, "stages": 4, "tile": 1024}
+    assert bench.fused_kernel_name(bulk, 8) == "fused_bulk_kernel"
+    assert bench.fused_kernel_name(bulk, 8, layered=True) == "fused_bulk_layered_kernel"
+    assert bench.fused_kernel_name(bulk, 64) == "fused_bulk_chunked_kernel"
+    assert bench.fused_kernel_name(bulk, 64, layered=True) == "fused_bulk_chunked_kernel"
+    assert bench.fused_kernel_name({"kernel": "register", "groups": 0}, 8) == "fused_step_kernel"
+    assert bench.fused_kernel_name({"kernel": "tma", "groups": 1}, 8) == "fused_step_tma_kernel"
+    assert bench.fused_kernel_name({"kernel": "tma", "groups": 3}, 8) == "fused_step_tma_wide_kernel"
+    assert bench.fused_kernel_name({"kernel": "tma", "groups": 1}, 17) == "fused_step_chunked_kernel"
