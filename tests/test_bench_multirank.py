@@ -1,7 +1,9 @@
 """bench.py's multi-process plumbing on CPU: two ranks over gloo, as
 torch.distributed.run would launch them.  The timing taken is the maximum
 over ranks, every rank makes the same collective calls, and only rank 0
-prints the JSON line (the reference arm runs on rank 0 alone)."""
+prints the JSON line (the reference arm runs on rank 0 alone).  Also its
+host helpers: the clock sampler's GPU match and the kernel name the
+roofline reports."""
 import json
 import os
 import socket
